@@ -1,0 +1,352 @@
+// PagedAttention oracle: plain, slow, fp64 CPU restatement of what the paged
+// KV-cache hot path computes.
+//
+// TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU-baseline
+// leg of the benchmark may load this library. The CUDA library never includes,
+// links or calls it, and it shares no header, helper or constant with the CUDA
+// sources.
+//
+// Sources (web pages; cited by title and section):
+//   [DS] "vLLM 深度实战：从 PagedAttention 到 Speculative Decoding"
+//        (chenxutan.com/d/2880), §3.2 KV Cache Block, §3.3 PagedAttention 的实现细节
+//   [VS] vLLM study notes (zihan-zhang.net/vLLM-study), §1.1.1 (attention with a
+//        causal mask), §1.2.1-1.2.2 (KV cache, size formula), §3.2 (block table,
+//        page-wise read of K/V), §4.3.1 (online softmax)
+//   [DP] "vLLM 深度解析：连续批处理与内存高效推理" (plumephp.com/ai-vllm-system),
+//        §1.2 (KV size formula), §2.1 (block table), §4.1 (block count example)
+//
+// Readings taken where the pages are silent or disagree (all stated here so the
+// code can be checked against them by eye):
+//   * Pool layout is [num_blocks][block_size][num_kv_heads][head_dim], token-major
+//     with head_dim innermost ([VS] §3.2 gives K_pool[phys] as
+//     [16, kv_heads, head_dim]; [DS] §3.3 prints a different, garbled order).
+//   * slot = physical_block * block_size + offset ([DS] §3.3 address mapping);
+//     a negative slot means "skip this token".
+//   * A sequence with context length ctx owns ceil(ctx / block_size) blocks.
+//   * GQA: query head h reads kv head h / (num_q_heads / num_kv_heads).
+//   * The q_per_seq query tokens of a sequence sit at the last q_per_seq
+//     positions: query token i is at position ctx - q_per_seq + i and sees keys
+//     at positions 0..ctx - q_per_seq + i ([VS] §1.1.1 causal mask).
+//   * A query row with no visible key has output 0.
+//   * bf16 is widened to fp64 exactly (bit pattern << 16 is the fp32 value).
+//
+// Parity pins for every function here live in the CPU test-suite (brute force
+// contiguous attention, a library attention routine, closed forms, invariants,
+// and the pages' worked numbers).
+//
+// ORACLE_MUTANT (compile-time, default 0) plants one plausible mistake; it
+// exists only so the test-suite can show that its pins catch such mistakes.
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+namespace {
+
+// Exact bf16 -> fp64 widening: a bf16 value is the upper 16 bits of an fp32.
+double bf16_to_f64(uint16_t bits) {
+#if ORACLE_MUTANT == 11
+  uint32_t w = static_cast<uint32_t>(bits) << 15;  // planted: wrong shift
+#else
+  uint32_t w = static_cast<uint32_t>(bits) << 16;
+#endif
+  float f;
+  std::memcpy(&f, &w, sizeof f);
+  return static_cast<double>(f);
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Index of element (block, offset, kv_head, d) in the pool.
+int64_t pool_index(int64_t block, int64_t offset, int64_t kv_head, int64_t d,
+                   int64_t block_size, int64_t num_kv_heads, int64_t head_dim) {
+#if ORACLE_MUTANT == 12
+  // planted: head-major inside a block
+  return ((block * num_kv_heads + kv_head) * block_size + offset) * head_dim + d;
+#else
+  return ((block * block_size + offset) * num_kv_heads + kv_head) * head_dim + d;
+#endif
+}
+
+struct Shape {
+  int num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size;
+  int max_blocks_per_seq;
+  int64_t num_blocks;
+};
+
+// Gather the keys and values of one (sequence, kv head) into contiguous fp64
+// arrays [ctx][head_dim], walking the block table as [DS] §3.3 and [VS] §3.2 do:
+// token i lives in physical block block_table[i / block_size] at offset
+// i % block_size. Returns false if the table points outside the pool.
+bool gather_kv(const uint16_t* key_cache, const uint16_t* value_cache,
+               const int32_t* table_row, int ctx, int kv_head, const Shape& s,
+               std::vector<double>& k_out, std::vector<double>& v_out) {
+  k_out.assign(static_cast<size_t>(ctx) * s.head_dim, 0.0);
+  v_out.assign(static_cast<size_t>(ctx) * s.head_dim, 0.0);
+  for (int i = 0; i < ctx; ++i) {
+    int64_t logical_block = i / s.block_size;
+#if ORACLE_MUTANT == 1
+    int64_t offset = (i / s.block_size) % s.block_size;  // planted: wrong offset
+#else
+    int64_t offset = i % s.block_size;
+#endif
+    int64_t phys = table_row[logical_block];
+    if (phys < 0 || phys >= s.num_blocks) return false;
+    for (int d = 0; d < s.head_dim; ++d) {
+      int64_t idx = pool_index(phys, offset, kv_head, d, s.block_size,
+                               s.num_kv_heads, s.head_dim);
+      k_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(key_cache[idx]);
+      v_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(value_cache[idx]);
+    }
+  }
+  return true;
+}
+
+// Attention of one query row against contiguous K/V, by the definition
+// softmax(q K^T * scale) V over the visible keys 0..last_visible ([VS] §1.1.1).
+// Two passes: first the maximum score, then the weights; no online rescaling.
+void attend_row(const double* q, const std::vector<double>& k,
+                const std::vector<double>& v, int last_visible, int head_dim,
+                double scale, double* out) {
+  for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
+  if (last_visible < 0) return;  // no visible key: output defined as 0
+  const int n = last_visible + 1;
+  std::vector<double> score(n);
+  for (int t = 0; t < n; ++t) {
+    double dot = 0.0;
+    for (int d = 0; d < head_dim; ++d) {
+#if ORACLE_MUTANT == 8
+      dot += q[d] * v[static_cast<size_t>(t) * head_dim + d];  // planted: V for K
+#else
+      dot += q[d] * k[static_cast<size_t>(t) * head_dim + d];
+#endif
+    }
+#if ORACLE_MUTANT == 5
+    score[t] = dot;  // planted: scale dropped
+#else
+    score[t] = dot * scale;
+#endif
+  }
+  double m = score[0];
+  for (int t = 1; t < n; ++t) m = std::max(m, score[t]);
+  double denom = 0.0;
+  for (int t = 0; t < n; ++t) {
+    double w = std::exp(score[t] - m);
+    denom += w;
+    for (int d = 0; d < head_dim; ++d) out[d] += w * v[static_cast<size_t>(t) * head_dim + d];
+  }
+#if ORACLE_MUTANT == 6
+  (void)denom;  // planted: missing normalisation
+#else
+  for (int d = 0; d < head_dim; ++d) out[d] /= denom;
+#endif
+}
+
+// Last key position visible to query token i of a sequence with ctx tokens.
+int last_visible_position(int ctx, int q_per_seq, int i) {
+#if ORACLE_MUTANT == 3
+  return ctx - q_per_seq + i - 1;  // planted: strict causal inequality
+#elif ORACLE_MUTANT == 7
+  (void)q_per_seq; (void)i;
+  return ctx - 1;  // planted: no causal window for speculative rows
+#else
+  return ctx - q_per_seq + i;
+#endif
+}
+
+int kv_head_of(int q_head, int num_q_heads, int num_kv_heads) {
+#if ORACLE_MUTANT == 2
+  (void)num_q_heads;
+  return q_head % num_kv_heads;  // planted: interleaved grouping
+#else
+  return q_head / (num_q_heads / num_kv_heads);
+#endif
+}
+
+const int32_t* table_row_of(const int32_t* block_tables, int b, const Shape& s,
+                            const int32_t* context_lens) {
+#if ORACLE_MUTANT == 9
+  // planted: rows packed by used length instead of max_blocks_per_seq
+  int64_t off = 0;
+  for (int j = 0; j < b; ++j) off += ceil_div(context_lens[j], s.block_size);
+  return block_tables + off;
+#else
+  (void)context_lens;
+  return block_tables + static_cast<int64_t>(b) * s.max_blocks_per_seq;
+#endif
+}
+
+int g_threads_used = 0;
+
+int resolve_threads(int requested) {
+  if (requested > 0) return requested;
+  unsigned hc = std::thread::hardware_concurrency();
+  return hc == 0 ? 1 : static_cast<int>(hc);
+}
+
+// Computes the rows listed in `rows` ((b, i, h) triples) into out[r][head_dim].
+// Work is split over (sequence, kv head) pairs so each gather is done once.
+int decode_rows_impl(double* out, const uint16_t* query, const uint16_t* key_cache,
+                     const uint16_t* value_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, const Shape& s, double scale,
+                     const int32_t* rows, int64_t n_rows, int num_threads) {
+  if (s.num_q_heads % s.num_kv_heads != 0) return 1;
+  // Bucket requested rows by (b, kv_head).
+  const int64_t units = static_cast<int64_t>(s.num_seqs) * s.num_kv_heads;
+  std::vector<std::vector<int64_t>> by_unit(units);
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+    if (b < 0 || b >= s.num_seqs || i < 0 || i >= s.q_per_seq || h < 0 ||
+        h >= s.num_q_heads)
+      return 2;
+    int kvh = kv_head_of(h, s.num_q_heads, s.num_kv_heads);
+    by_unit[static_cast<int64_t>(b) * s.num_kv_heads + kvh].push_back(r);
+  }
+  for (int b = 0; b < s.num_seqs; ++b) {
+    int ctx = context_lens[b];
+    if (ctx < 0 || ceil_div(ctx, s.block_size) > s.max_blocks_per_seq) return 3;
+  }
+  std::atomic<int64_t> next{0};
+  std::atomic<int> err{0};
+  auto worker = [&]() {
+    std::vector<double> k, v, qrow(s.head_dim);
+    for (;;) {
+      int64_t u = next.fetch_add(1);
+      if (u >= units) break;
+      if (by_unit[u].empty()) continue;
+      int b = static_cast<int>(u / s.num_kv_heads);
+      int kvh = static_cast<int>(u % s.num_kv_heads);
+      int ctx = context_lens[b];
+      if (!gather_kv(key_cache, value_cache, table_row_of(block_tables, b, s, context_lens),
+                     ctx, kvh, s, k, v)) {
+        err.store(4);
+        continue;
+      }
+      for (int64_t r : by_unit[u]) {
+        int i = rows[3 * r + 1], h = rows[3 * r + 2];
+        const uint16_t* qsrc =
+            query + ((static_cast<int64_t>(b) * s.q_per_seq + i) * s.num_q_heads + h) * s.head_dim;
+        for (int d = 0; d < s.head_dim; ++d) qrow[d] = bf16_to_f64(qsrc[d]);
+        attend_row(qrow.data(), k, v, last_visible_position(ctx, s.q_per_seq, i),
+                   s.head_dim, scale, out + r * s.head_dim);
+      }
+    }
+  };
+  int nt = static_cast<int>(std::min<int64_t>(resolve_threads(num_threads), std::max<int64_t>(units, 1)));
+  g_threads_used = nt;
+  std::vector<std::thread> pool;
+  for (int t = 1; t < nt; ++t) pool.emplace_back(worker);
+  worker();
+  for (auto& th : pool) th.join();
+  return err.load();
+}
+
+}  // namespace
+
+extern "C" {
+
+// bf16 bit pattern -> fp64 (exact).
+double oracle_bf16_to_f64(uint16_t bits) { return bf16_to_f64(bits); }
+
+// Number of blocks a sequence of n tokens occupies ([DS] §3.2, [DP] §4.1).
+int64_t oracle_blocks_for_tokens(int64_t n_tokens, int64_t block_size) {
+  return ceil_div(n_tokens, block_size);
+}
+
+// KV-cache bytes per token of a whole model: 2 (K and V) x layers x kv heads x
+// head_dim x bytes per value ([VS] §1.2.2, [DP] §1.2).
+int64_t oracle_kv_bytes_per_token(int64_t layers, int64_t kv_heads, int64_t head_dim,
+                                  int64_t bytes_per_value) {
+  return 2 * layers * kv_heads * head_dim * bytes_per_value;
+}
+
+// Cache write: for every token t with slot_mapping[t] >= 0, copy the bf16 bit
+// patterns of key[t] and value[t] ([num_kv_heads][head_dim], rows `key_stride` /
+// `value_stride` elements apart) into pool row slot = block * block_size + offset.
+// Every other pool element is left untouched. Returns 0, or 1 for an
+// out-of-range slot (nothing is written for that token).
+int oracle_reshape_and_cache(const uint16_t* key, const uint16_t* value,
+                             int64_t key_stride, int64_t value_stride,
+                             uint16_t* key_cache, uint16_t* value_cache,
+                             const int64_t* slot_mapping, int64_t num_tokens,
+                             int num_kv_heads, int head_dim, int64_t num_blocks,
+                             int block_size) {
+  int status = 0;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    int64_t block = slot / block_size;
+    int64_t offset = slot % block_size;
+#if ORACLE_MUTANT == 10
+    offset = (offset + 1) % block_size;  // planted: off-by-one slot
+#endif
+    if (block >= num_blocks) {
+      status = 1;
+      continue;
+    }
+    for (int h = 0; h < num_kv_heads; ++h) {
+      for (int d = 0; d < head_dim; ++d) {
+        int64_t dst = pool_index(block, offset, h, d, block_size, num_kv_heads, head_dim);
+        key_cache[dst] = key[t * key_stride + static_cast<int64_t>(h) * head_dim + d];
+        value_cache[dst] = value[t * value_stride + static_cast<int64_t>(h) * head_dim + d];
+      }
+    }
+  }
+  return status;
+}
+
+// Paged decode attention, every row: out[b][i][h][d] (fp64) for b < num_seqs,
+// i < q_per_seq, h < num_q_heads. block_tables is [num_seqs][max_blocks_per_seq],
+// context_lens[b] counts all tokens of sequence b including its q_per_seq new
+// ones. num_threads <= 0 uses every hardware thread. Returns 0 on success.
+int oracle_decode(double* out, const uint16_t* query, const uint16_t* key_cache,
+                  const uint16_t* value_cache, const int32_t* block_tables,
+                  const int32_t* context_lens, int num_seqs, int q_per_seq,
+                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int64_t num_blocks, double scale,
+                  int num_threads) {
+  Shape s{num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size,
+          max_blocks_per_seq, num_blocks};
+  const int64_t n_rows = static_cast<int64_t>(num_seqs) * q_per_seq * num_q_heads;
+  std::vector<int32_t> rows(3 * n_rows);
+  int64_t r = 0;
+  for (int b = 0; b < num_seqs; ++b)
+    for (int i = 0; i < q_per_seq; ++i)
+      for (int h = 0; h < num_q_heads; ++h, ++r) {
+        rows[3 * r] = b;
+        rows[3 * r + 1] = i;
+        rows[3 * r + 2] = h;
+      }
+  return decode_rows_impl(out, query, key_cache, value_cache, block_tables, context_lens,
+                          s, scale, rows.data(), n_rows, num_threads);
+}
+
+// Same as oracle_decode for a chosen list of rows: rows holds n_rows (b, i, h)
+// triples and out receives n_rows x head_dim values in that order. Used to
+// check sampled outputs of full-size problems.
+int oracle_decode_rows(double* out, const uint16_t* query, const uint16_t* key_cache,
+                       const uint16_t* value_cache, const int32_t* block_tables,
+                       const int32_t* context_lens, int num_seqs, int q_per_seq,
+                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, double scale,
+                       const int32_t* rows, int64_t n_rows, int num_threads) {
+  Shape s{num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size,
+          max_blocks_per_seq, num_blocks};
+  return decode_rows_impl(out, query, key_cache, value_cache, block_tables, context_lens,
+                          s, scale, rows, n_rows, num_threads);
+}
+
+// Threads the last decode call ran on.
+int oracle_threads_used() { return g_threads_used; }
+
+int oracle_mutant_id() { return ORACLE_MUTANT; }
+
+}  // extern "C"

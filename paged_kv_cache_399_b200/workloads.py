@@ -1,0 +1,205 @@
+"""Seeded synthetic inputs for the paged KV-cache hot path.
+
+This module holds no attention arithmetic: it only draws context lengths,
+block tables, slot mappings and bf16 ~N(0, 1) tensors, the way a serving
+engine's block manager would hand them to the kernels. Both the CUDA tests and
+the fp64 oracle read the same objects built here.
+
+Workloads (sizes follow the decode shapes that the vLLM pages discuss: the
+16-token block of "vLLM 深度实战" §3.2 and the Llama shapes of the vLLM study
+notes §1.2.2):
+
+* ``tiny``            4 seqs x 1 query token, 4 q heads / 2 kv heads, head_dim 64,
+                      context U[1, 80], a 64-block pool drawn without replacement,
+                      scale 1/8; the slot mapping writes each sequence's newest token.
+* ``llama8b``         64 x 1, 32/8 heads, head_dim 128, context U[512, 4096], pool
+                      1.25x the blocks needed, shuffled.
+* ``llama70b_long``   4 x 1, 64/8 heads, head_dim 128, contexts 32k/64k/96k/128k,
+                      pool 1.25x the blocks needed, shuffled.
+* ``prefix_sharing``  16 prompts x 8 samples, 32/8 heads: the 8 samples of a prompt
+                      map their first 2048 tokens to the same 128 physical blocks,
+                      then private tails of U[1, 256] tokens.
+* ``spec_verify``     32 seqs x 6 query tokens (causal inside the window), 32/8 heads,
+                      context lognormal(ln 2048, 0.8) clipped to [16, 16384]; the slot
+                      mapping writes all 6 new tokens.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+BLOCK_SIZE = 16
+
+
+@dataclass
+class Workload:
+    name: str
+    seed: int
+    num_seqs: int
+    q_per_seq: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    scale: float
+    context_lens: np.ndarray          # int32 [B]
+    block_tables: np.ndarray          # int32 [B, max_blocks_per_seq]
+    num_blocks: int
+    query: torch.Tensor               # bf16 [B, q, H_q, D]
+    key: torch.Tensor                 # bf16 [T, H_kv, D], T = B * q
+    value: torch.Tensor               # bf16 [T, H_kv, D]
+    slot_mapping: np.ndarray          # int64 [T]
+    key_cache: torch.Tensor           # bf16 [NB, bs, H_kv, D], pool before the write
+    value_cache: torch.Tensor         # bf16 [NB, bs, H_kv, D]
+    blocks_used: np.ndarray = field(default=None)   # int32 [B] blocks owned per sequence
+    shared_groups: list = field(default_factory=list)  # [(members, prefix_tokens)]
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.slot_mapping.shape[0])
+
+    def describe(self) -> str:
+        return (f"{self.name}: B={self.num_seqs} q={self.q_per_seq} H_q={self.num_q_heads} "
+                f"H_kv={self.num_kv_heads} D={self.head_dim} bs={self.block_size} "
+                f"ctx[min/mean/max]={int(self.context_lens.min())}/"
+                f"{float(self.context_lens.mean()):.0f}/{int(self.context_lens.max())} "
+                f"NB={self.num_blocks} seed={self.seed}")
+
+
+def _blocks(n_tokens: int, block_size: int) -> int:
+    return -(-int(n_tokens) // block_size)
+
+
+def _randn_bf16(shape, gen: torch.Generator, chunk: int = 1 << 24) -> torch.Tensor:
+    """bf16 ~N(0,1): fp32 normal draws rounded to nearest even, in chunks."""
+    out = torch.empty(shape, dtype=torch.bfloat16)
+    flat = out.view(-1)
+    n = flat.numel()
+    for start in range(0, n, chunk):
+        stop = min(n, start + chunk)
+        flat[start:stop] = torch.randn(stop - start, generator=gen, dtype=torch.float32).to(
+            torch.bfloat16)
+    return out
+
+
+def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_heads: int,
+                   num_kv_heads: int, head_dim: int, scale: float | None = None,
+                   block_size: int = BLOCK_SIZE, pool_factor: float = 1.25,
+                   num_blocks: int | None = None, share_groups=None,
+                   max_blocks_per_seq: int | None = None) -> Workload:
+    """General builder.
+
+    share_groups: optional list of (member_sequence_ids, prefix_tokens); the
+    members map their first prefix_tokens (a multiple of block_size) to the same
+    physical blocks. All other blocks are private. Physical ids come from one
+    seeded permutation of the pool, so no two sequences alias a private block.
+    """
+    rng = np.random.default_rng(seed)
+    gen = torch.Generator().manual_seed(seed)
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    B = int(ctx.shape[0])
+    if np.any(ctx < q_per_seq):
+        raise ValueError("every context must hold its q_per_seq new tokens")
+    need = np.array([_blocks(c, block_size) for c in ctx], dtype=np.int64)
+    share_groups = list(share_groups or [])
+    shared_prefix_blocks = np.zeros(B, dtype=np.int64)
+    leader = np.arange(B)
+    for members, prefix_tokens in share_groups:
+        if prefix_tokens % block_size:
+            raise ValueError("shared prefixes cover whole blocks")
+        for m in members:
+            shared_prefix_blocks[m] = prefix_tokens // block_size
+            leader[m] = members[0]
+    distinct = int(need.sum() - sum(shared_prefix_blocks[m] for members, _ in share_groups
+                                     for m in members[1:]))
+    if num_blocks is None:
+        num_blocks = int(math.ceil(pool_factor * distinct))
+    if num_blocks < distinct:
+        raise ValueError("pool too small")
+    perm = rng.permutation(num_blocks).astype(np.int64)
+    width = int(max_blocks_per_seq or need.max())
+    tables = np.zeros((B, width), dtype=np.int32)  # padding entries point at block 0
+    cursor = 0
+    for b in range(B):
+        start = 0
+        if shared_prefix_blocks[b] and leader[b] != b:
+            start = int(shared_prefix_blocks[b])
+            tables[b, :start] = tables[leader[b], :start]
+        n = int(need[b]) - start
+        tables[b, start:start + n] = perm[cursor:cursor + n]
+        cursor += n
+    # new tokens of this step: the last q_per_seq positions of every sequence
+    slots = np.empty(B * q_per_seq, dtype=np.int64)
+    for b in range(B):
+        for i in range(q_per_seq):
+            p = int(ctx[b]) - q_per_seq + i
+            slots[b * q_per_seq + i] = int(tables[b, p // block_size]) * block_size + p % block_size
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    query = _randn_bf16((B, q_per_seq, num_q_heads, head_dim), gen)
+    key = _randn_bf16((B * q_per_seq, num_kv_heads, head_dim), gen)
+    value = _randn_bf16((B * q_per_seq, num_kv_heads, head_dim), gen)
+    key_cache = _randn_bf16((num_blocks, block_size, num_kv_heads, head_dim), gen)
+    value_cache = _randn_bf16((num_blocks, block_size, num_kv_heads, head_dim), gen)
+    return Workload(name=name, seed=seed, num_seqs=B, q_per_seq=q_per_seq,
+                    num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+                    block_size=block_size, scale=float(scale),
+                    context_lens=ctx.astype(np.int32), block_tables=tables,
+                    num_blocks=int(num_blocks), query=query, key=key, value=value,
+                    slot_mapping=slots, key_cache=key_cache, value_cache=value_cache,
+                    blocks_used=need.astype(np.int32), shared_groups=share_groups)
+
+
+def tiny(seed: int = 1000) -> Workload:
+    rng = np.random.default_rng(seed + 7919)
+    ctx = rng.integers(1, 80, size=4, endpoint=True)
+    return build_workload("tiny", seed, ctx, 1, 4, 2, 64, scale=1.0 / 8.0, num_blocks=64)
+
+
+def llama8b(seed: int = 1001, num_seqs: int = 64) -> Workload:
+    rng = np.random.default_rng(seed + 7919)
+    ctx = rng.integers(512, 4096, size=num_seqs, endpoint=True)
+    return build_workload("llama8b", seed, ctx, 1, 32, 8, 128)
+
+
+def llama70b_long(seed: int = 1002, context_lens=(32768, 65536, 98304, 131072)) -> Workload:
+    return build_workload("llama70b_long", seed, list(context_lens), 1, 64, 8, 128)
+
+
+def prefix_sharing(seed: int = 1003, prompts: int = 16, samples: int = 8,
+                   prefix_tokens: int = 2048, max_tail: int = 256) -> Workload:
+    rng = np.random.default_rng(seed + 7919)
+    tails = rng.integers(1, max_tail, size=prompts * samples, endpoint=True)
+    ctx = prefix_tokens + tails
+    groups = [(list(range(p * samples, (p + 1) * samples)), prefix_tokens)
+              for p in range(prompts)]
+    return build_workload("prefix_sharing", seed, ctx, 1, 32, 8, 128, share_groups=groups)
+
+
+def spec_verify(seed: int = 1004, num_seqs: int = 32, q_per_seq: int = 6) -> Workload:
+    rng = np.random.default_rng(seed + 7919)
+    ctx = np.rint(rng.lognormal(mean=math.log(2048.0), sigma=0.8, size=num_seqs))
+    ctx = np.clip(ctx, 16, 16384).astype(np.int64)
+    return build_workload("spec_verify", seed, ctx, q_per_seq, 32, 8, 128)
+
+
+WORKLOADS = {
+    "tiny": tiny,
+    "llama8b": llama8b,
+    "llama70b_long": llama70b_long,
+    "prefix_sharing": prefix_sharing,
+    "spec_verify": spec_verify,
+}
+
+
+def make(name: str, seed: int | None = None) -> Workload:
+    fn = WORKLOADS[name]
+    return fn() if seed is None else fn(seed)
