@@ -1,0 +1,475 @@
+"""Benchmark of the paged KV-cache hot path on B200: one step = pa_reshape_and_cache
+(the step's new K/V into the pool) + pa_decode (paged attention over the pool),
+through the C ABI of libpa_b200.so, on seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+    python bench.py --impl reference ...        # the fp64 CPU oracle, timed on host cores
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one independent replica per GPU)
+
+Prints ONE JSON line (rank 0). value = algorithmic bytes of all ranks' steps /
+max-over-ranks device time, in GB/s.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "llama8b"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+# DRAM traffic per pa_decode launch measured by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum summed over the launch's kernels), keyed by workload, with
+# the hash of the kernel sources it was measured on. A different hash -> null.
+NCU_TRAFFIC = {}
+
+
+# ------------------------------------------------------------------ accounting
+
+def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, bytes_per_value: int = 2) -> int:
+    """KV-cache bytes per token of a model: K and V, every layer and kv head."""
+    return 2 * layers * kv_heads * head_dim * bytes_per_value
+
+
+def decode_bytes(w, unique: bool = True) -> int:
+    """Algorithmic bytes of one pa_decode call: the K/V of every visible token (shared
+    physical slots counted once when `unique`), q, out, the used block-table
+    entries and context_lens."""
+    bs = w.block_size
+    if unique:
+        slots = set()
+        for b in range(w.num_seqs):
+            ctx = int(w.context_lens[b])
+            tbl = w.block_tables[b]
+            nfull, tail = divmod(ctx, bs)
+            for j in range(nfull):
+                slots.add((int(tbl[j]), bs))
+            if tail:
+                key = (int(tbl[nfull]), tail)
+                slots.add(key)
+        # a block read to `fill` tokens by one sequence and fully by another counts once, fully
+        per_block = {}
+        for blk, fill in slots:
+            per_block[blk] = max(per_block.get(blk, 0), fill)
+        tokens = sum(per_block.values())
+    else:
+        tokens = int(np.sum(w.context_lens.astype(np.int64)))
+    kv = tokens * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_seqs * w.q_per_seq * w.num_q_heads * w.head_dim * 2
+    tables = int(sum(-(-int(c) // bs) for c in w.context_lens)) * 4
+    return kv + qo + tables + w.num_seqs * 4
+
+
+def cache_write_bytes(w) -> int:
+    """K and V rows read and written, plus the slot mapping."""
+    row = w.num_kv_heads * w.head_dim * 2
+    return w.num_tokens * (2 * row * 2 + 8)
+
+
+def decode_flops(w) -> int:
+    """QK^T and PV multiply-adds over the visible keys of every query row."""
+    vis = 0
+    for b in range(w.num_seqs):
+        ctx = int(w.context_lens[b])
+        vis += sum(ctx - w.q_per_seq + i + 1 for i in range(w.q_per_seq))
+    return 4 * w.head_dim * (w.num_q_heads // w.num_kv_heads) * w.num_kv_heads * vis
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_399_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return dict(PEAKS_FALLBACK, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while timing."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        import torch
+        self.uuid = None
+        try:
+            u = torch.cuda.get_device_properties(device_index).uuid
+            self.uuid = "GPU-" + str(u)
+        except Exception:
+            pass
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    from paged_kv_cache_399_b200 import build as pa_build
+    pa_build.build()
+    from paged_kv_cache_399_b200 import pa, workloads
+
+    # weak scaling: every rank decodes its own replica of the workload (own seed)
+    base_seed = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
+                 "spec_verify": 1004}[args.workload]
+    w = workloads.make(args.workload, seed=base_seed + 100 * rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+
+    query = w.query.to(dev)
+    key = w.key.to(dev)
+    value = w.value.to(dev)
+    slots = torch.from_numpy(w.slot_mapping).to(dev)
+    tables = torch.from_numpy(w.block_tables).to(dev)
+    ctx = torch.from_numpy(w.context_lens).to(dev)
+    key_cache = w.key_cache.to(dev)
+    value_cache = w.value_cache.to(dev)
+    out = torch.empty_like(query)
+    plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                             w.max_blocks_per_seq)
+    ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads,
+                                           w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
+
+    def step():
+        pa.pa_reshape_and_cache(key, value, key_cache, value_cache, slots, stream=stream)
+        pa.pa_decode(out, query, key_cache, value_cache, tables, ctx, w.q_per_seq, w.scale, plan=plan,
+                     workspace=ws, stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    launches_per_step = 2 + (1 if plan.num_splits > 1 else 0)
+    step_bytes = decode_bytes(w) + cache_write_bytes(w)
+    dec_bytes = decode_bytes(w)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        # (1) headline: K whole steps, events only around the region
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+        ms_total = max_over_ranks(e0.elapsed_time(e1))
+
+        # (2) per-kernel: events around each pa_decode launch of another K steps
+        barrier()
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for a, b in pairs:
+            pa.pa_reshape_and_cache(key, value, key_cache, value_cache, slots, stream=stream)
+            a.record(stream)
+            pa.pa_decode(out, query, key_cache, value_cache, tables, ctx, w.q_per_seq, w.scale,
+                         plan=plan, workspace=ws, stream=stream)
+            b.record(stream)
+        barrier()
+        decode_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        decode_ms = max_over_ranks(decode_ms)
+
+        # (3) end to end: host (pinned) inputs in, output back to the host, every step
+        h_query = query.cpu().pin_memory()
+        h_key = key.cpu().pin_memory()
+        h_value = value.cpu().pin_memory()
+        h_slots = slots.cpu().pin_memory()
+        h_tables = tables.cpu().pin_memory()
+        h_ctx = ctx.cpu().pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (h_query, h_key, h_value, h_slots, h_tables, h_ctx))
+        d2h = h_out.numel() * h_out.element_size()
+        e2e_steps = max(1, args.steps // 4)
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            query.copy_(h_query, non_blocking=True)
+            key.copy_(h_key, non_blocking=True)
+            value.copy_(h_value, non_blocking=True)
+            slots.copy_(h_slots, non_blocking=True)
+            tables.copy_(h_tables, non_blocking=True)
+            ctx.copy_(h_ctx, non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
+        f1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+
+    ms_per_step = ms_total / args.steps
+    value_gbs = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    e2e_gbs = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
+    traffic = None
+    rec = NCU_TRAFFIC.get(args.workload)
+    if rec and rec.get("source_hash") == source_hash():
+        traffic = rec["bytes_per_launch"]
+    clocks = sampler.summary()
+
+    if rank == 0:
+        cpu = cpu_baseline(w, args) if (world == 1 and not args.no_cpu_baseline) else None
+        line = {
+            "metric": "pa_decode achieved HBM GB/s & % of B200 peak; us/call per config",
+            "value": round(value_gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": w.describe(),
+                "step": "pa_reshape_and_cache + pa_decode",
+                "alg_bytes_per_step": step_bytes,
+                "decode_alg_bytes": dec_bytes,
+                "decode_logical_bytes": decode_bytes(w, unique=False),
+                "decode_us_per_call": round(decode_ms * 1e3, 3),
+                "decode_gbs": round(achieved, 2),
+                "decode_frac_of_measured_hbm": round(achieved / peaks["hbm_gbs"], 4),
+                "decode_frac_of_spec_8tbs": round(achieved / 8000.0, 4),
+                "step_frac_of_measured_hbm": round(value_gbs / world / peaks["hbm_gbs"], 4),
+                "plan": {"path": {1: "single", 2: "tile"}[plan.path], "split_blocks": plan.split_blocks,
+                         "num_splits": plan.num_splits, "rows_per_cta": plan.rows_per_cta},
+                "l2": "no flush: each step reads more bytes than the 126 MB L2 holds"
+                      if dec_bytes > 2 * 126e6 else "no flush: working set near L2 size (see DESIGN)",
+                "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
+            },
+            "roofline": {
+                "bound": "hbm",
+                "achieved": round(achieved, 2),
+                "peak": peaks["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic,
+                "peak_source": peaks["source"],
+                "kernel": "pa_decode (decode kernel + merge when split)",
+            },
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+def _oracle_step(orc, w, seqs):
+    """One oracle step over the sequences `seqs` of w: cache write, then decode."""
+    sub_slots = np.concatenate([w.slot_mapping[b * w.q_per_seq:(b + 1) * w.q_per_seq] for b in seqs])
+    sub_key = w.key.view(w.num_seqs, w.q_per_seq, w.num_kv_heads, w.head_dim)[seqs].reshape(
+        -1, w.num_kv_heads, w.head_dim)
+    sub_val = w.value.view(w.num_seqs, w.q_per_seq, w.num_kv_heads, w.head_dim)[seqs].reshape(
+        -1, w.num_kv_heads, w.head_dim)
+    kc, vc = orc.reshape_and_cache(sub_key, sub_val, w.key_cache, w.value_cache, sub_slots)
+    return orc.decode(w.query[seqs], kc, vc, w.block_tables[seqs], w.context_lens[seqs], w.q_per_seq,
+                      w.scale)
+
+
+def _sample_workload(w, seqs):
+    import copy
+    s = copy.copy(w)
+    s.num_seqs = len(seqs)
+    s.context_lens = w.context_lens[seqs]
+    s.block_tables = w.block_tables[seqs]
+    s.slot_mapping = np.concatenate([w.slot_mapping[b * w.q_per_seq:(b + 1) * w.q_per_seq] for b in seqs])
+    return s
+
+
+def cpu_baseline(w, args, target_s: float = 8.0):
+    """The oracle, as it stands, on host cores over a bounded sample of the workload."""
+    from oracle import Oracle
+    orc = Oracle()
+    seqs = list(range(min(w.num_seqs, args.cpu_sample_seqs)))
+    sub = _sample_workload(w, seqs)
+    sample_bytes = decode_bytes(sub) + cache_write_bytes(sub)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        _oracle_step(orc, w, seqs)
+        reps += 1
+        if time.perf_counter() - t0 >= target_s or reps >= 50:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(sample_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": orc.threads_used(),
+            "kind": "oracle",
+            "sample": f"{len(seqs)} of {w.num_seqs} sequences of {w.name} (cache write + decode, fp64), "
+                      f"{reps} repetitions, {dt:.3f} s each"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import Oracle
+    from paged_kv_cache_399_b200 import workloads
+    base_seed = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
+                 "spec_verify": 1004}[args.workload]
+    w = workloads.make(args.workload, seed=base_seed)
+    orc = Oracle()
+    seqs = list(range(min(w.num_seqs, args.ref_sample_seqs)))
+    sub = _sample_workload(w, seqs)
+    sample_bytes = decode_bytes(sub) + cache_write_bytes(sub)
+    for _ in range(args.warmup):
+        _oracle_step(orc, w, seqs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(orc, w, seqs)
+    dt = time.perf_counter() - t0
+    value = sample_bytes * args.steps / dt / 1e9
+    sample = f"{len(seqs)} of {w.num_seqs} sequences of {w.name} per step (cache write + decode, fp64)"
+    line = {
+        "impl": "reference",
+        "metric": "pa_decode achieved HBM GB/s & % of B200 peak; us/call per config",
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.describe(), "step": "oracle cache write + oracle decode"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": orc.threads_used(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seqs", type=int, default=16)
+    ap.add_argument("--ref-sample-seqs", type=int, default=4)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

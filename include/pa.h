@@ -1,0 +1,173 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged KV-cache hot path.
+ *
+ * Two operations, as the vLLM pages describe them:
+ *   pa_reshape_and_cache  writes this step's new K/V rows into the paged pool at
+ *                         the slots named by slot_mapping
+ *                         ("vLLM 深度实战：从 PagedAttention 到 Speculative Decoding",
+ *                          §3.3: block_table and slot_mapping address the blocks);
+ *   pa_decode             attention softmax(q K^T * scale) V computed straight over
+ *                         the scattered blocks through each sequence's block table
+ *                         (same page §3.3; vLLM study notes, zihan-zhang.net, §3.2
+ *                          page-table walk and §4.3.1 online softmax), with GQA
+ *                         head groups and causal masking of multi-token
+ *                         (speculative-verify) queries (vLLM study notes §1.1.1).
+ *
+ * Conventions shared by every call
+ *   - All data pointers are DEVICE pointers on the current CUDA device; the library
+ *     never allocates, frees or synchronises (except pa_validate and
+ *     pa_get_device_error, which are synchronous debug calls). All work is enqueued
+ *     on `stream` (a cudaStream_t; NULL = legacy default stream). The caller owns
+ *     every buffer and must keep it alive until the stream has executed the work.
+ *   - bf16 tensors are passed as raw 16-bit storage.
+ *   - Shapes (row-major, innermost last):
+ *       key, value     [num_tokens][num_kv_heads][head_dim]; token rows may be
+ *                      `*_token_stride` elements apart (>= num_kv_heads*head_dim)
+ *       key_cache,
+ *       value_cache    [num_blocks][block_size][num_kv_heads][head_dim]
+ *                      (token-major block, head_dim innermost)
+ *       slot_mapping   int64 [num_tokens]; slot = physical_block * block_size +
+ *                      offset; a negative slot skips the token
+ *       query, out     [num_seqs][q_per_seq][num_q_heads][head_dim]
+ *       block_tables   int32 [num_seqs][max_blocks_per_seq]; entry j is the
+ *                      physical block holding tokens j*block_size ..
+ *                      j*block_size + block_size - 1 of the sequence
+ *       context_lens   int32 [num_seqs]; tokens of the sequence INCLUDING its
+ *                      q_per_seq new ones (already written by pa_reshape_and_cache)
+ *   - Query token i of a sequence sits at position context_len - q_per_seq + i and
+ *     attends to positions 0 .. context_len - q_per_seq + i. Query head h reads kv
+ *     head h / (num_q_heads / num_kv_heads).
+ *   - Supported: block_size 16, head_dim 64 or 128, num_q_heads % num_kv_heads == 0,
+ *     1 <= q_per_seq <= 16. Anything else returns PA_ERR_UNSUPPORTED before any
+ *     launch. There is no CPU fallback.
+ *   - Errors: host-side argument checks run before any launch and return a status
+ *     with nothing enqueued. Device-resident values (slots, block ids, context
+ *     lengths) are preconditions: 0 <= slot < num_blocks*block_size or slot < 0,
+ *     0 <= block id < num_blocks for the first ceil(context_len/block_size)
+ *     entries of each table row, q_per_seq <= context_len <=
+ *     max_blocks_per_seq*block_size. pa_validate checks them on request. A launch
+ *     failure returns PA_ERR_CUDA. Kernels never trap: a bounded wait that times
+ *     out records a code that pa_get_device_error returns.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+typedef struct CUstream_st* pa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or stride */
+  PA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported set above */
+  PA_ERR_WORKSPACE = 3,     /* split plan without a large enough workspace */
+  PA_ERR_OUT_OF_RANGE = 4,  /* pa_validate found a bad slot / block id / length */
+  PA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  PA_ERR_DEVICE = 6         /* pa_get_device_error: a kernel reported a timeout */
+} pa_status_t;
+
+/* Decode kernels. */
+typedef enum {
+  PA_PATH_AUTO = 0,   /* heuristic (pa_decode_plan) */
+  PA_PATH_SINGLE = 1, /* CUDA-core kernel: warp-shuffle reductions, fp32 FMA */
+  PA_PATH_TILE = 2    /* tensor-core kernel: mma.sync m16n8k16 bf16 -> fp32 */
+} pa_path_t;
+
+/* How pa_decode splits the work. num_splits > 1 means each sequence's context is
+ * cut into chunks of split_blocks blocks (flash-decoding); the chunks write fp32
+ * partial (o, m, l) records to the workspace and a log-sum-exp merge kernel
+ * combines them. */
+typedef struct {
+  int32_t path;          /* PA_PATH_SINGLE or PA_PATH_TILE */
+  int32_t split_blocks;  /* blocks per split, >= 1 */
+  int32_t num_splits;    /* ceil(max_blocks_per_seq / split_blocks) */
+  int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds */
+} pa_plan_t;
+
+/* Write the step's new K/V into the pool: for each token t with slot s =
+ * slot_mapping[t] >= 0, key_cache[s / block_size][s % block_size][:][:] = key[t]
+ * and likewise value -> value_cache. Bit-exact copy; every other pool byte is left
+ * untouched. Requirements: 16-byte aligned key, value, key_cache, value_cache;
+ * token strides in elements with stride*2 a multiple of 16; num_kv_heads*head_dim*2
+ * a multiple of 16. Duplicate slots in one call are a precondition violation (the
+ * surviving row is unspecified). num_tokens == 0 is a no-op. */
+PA_API pa_status_t pa_reshape_and_cache(const void* key, const void* value,
+                                 int64_t key_token_stride, int64_t value_token_stride,
+                                 void* key_cache, void* value_cache,
+                                 const int64_t* slot_mapping, int64_t num_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim,
+                                 int64_t num_blocks, int32_t block_size,
+                                 pa_stream_t stream);
+
+/* Choose a plan from host-known shape values only (no device read). path_hint
+ * PA_PATH_AUTO lets the heuristic pick the kernel; split_blocks_hint 0 lets it
+ * pick the split length. The heuristic reads the SM count of the current device. */
+PA_API pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t head_dim,
+                           int32_t max_blocks_per_seq, int32_t path_hint,
+                           int32_t split_blocks_hint, pa_plan_t* plan);
+
+/* Workspace bytes pa_decode needs for `plan` (NULL = the heuristic plan for these
+ * shapes): num_seqs * num_splits * q_per_seq * num_q_heads * (head_dim + 2) * 4
+ * when num_splits > 1, else 0. */
+PA_API size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs,
+                                int32_t q_per_seq, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_blocks_per_seq);
+
+/* Paged decode attention. out[b][i][h][:] = sum_t softmax_t(scale * q.k_t) v_t over
+ * the visible positions t of sequence b, rounded to bf16 (nearest even) from fp32
+ * accumulation. A row with no visible key (context_len < q_per_seq, a precondition
+ * violation) yields 0. plan NULL = heuristic. workspace: 16-byte aligned device
+ * buffer of at least pa_decode_workspace_size(plan, ...) bytes, may be NULL when
+ * that size is 0; its contents need no initialisation and are scratch afterwards.
+ * Reads query/block_tables/context_lens/caches only after the preceding work on
+ * the stream has completed (programmatic dependent launch is used to hide the
+ * launch latency). num_seqs == 0 is a no-op. */
+PA_API pa_status_t pa_decode(void* out, const void* query, const void* key_cache,
+                      const void* value_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int32_t num_seqs, int32_t q_per_seq,
+                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                      float scale, const pa_plan_t* plan, void* workspace,
+                      size_t workspace_bytes, pa_stream_t stream);
+
+/* Debug check of the device-resident preconditions (synchronous: waits for
+ * `stream`). Counts context lengths outside [q_per_seq, max_blocks_per_seq *
+ * block_size], used block-table entries outside [0, num_blocks) and slots >=
+ * num_blocks*block_size. slot_mapping may be NULL (num_tokens ignored). On return
+ * *num_bad (may be NULL) holds the count; the status is PA_ERR_OUT_OF_RANGE when
+ * it is non-zero. */
+PA_API pa_status_t pa_validate(const int32_t* block_tables, const int32_t* context_lens,
+                        const int64_t* slot_mapping, int32_t num_seqs,
+                        int32_t max_blocks_per_seq, int32_t q_per_seq,
+                        int64_t num_tokens, int64_t num_blocks, int32_t block_size,
+                        int64_t* num_bad, pa_stream_t stream);
+
+/* Reads (and with reset != 0 clears) the device error word that kernels set when a
+ * bounded wait times out (synchronous: waits for `stream`). *code = 0 means no
+ * error; the status is PA_ERR_DEVICE when *code != 0. */
+PA_API pa_status_t pa_get_device_error(uint32_t* code, int32_t reset, pa_stream_t stream);
+
+/* Static description of a status code. */
+PA_API const char* pa_status_string(pa_status_t status);
+
+/* ABI version (major * 10000 + minor * 100 + patch). */
+PA_API int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

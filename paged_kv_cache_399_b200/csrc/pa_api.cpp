@@ -1,0 +1,321 @@
+// Host side of the C ABI declared in include/pa.h: argument checks, the plan
+// heuristic, TMA descriptors for the paged pool, and the kernel launches.
+// Nothing here touches device data; all work is enqueued on the caller's stream.
+
+#include "pa.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa_internal.h"
+
+namespace {
+
+using pa::DecodeParams;
+
+constexpr int32_t kVersion = 10000;  // 1.0.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ----------------------------------------------------------------- device facts
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+DeviceInfo device_info() {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{148};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev].sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    cache[dev].sms = sms;
+  }
+  return cache[dev];
+}
+
+// ----------------------------------------------------------------- TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The pool [num_blocks][16][H_kv][D] as a 3-D tensor {D, H_kv, num_blocks*16}; one
+// box is {64, 1, 16}: half of head_dim for one kv head over the 16 tokens of a block,
+// 128-byte swizzled in shared memory.
+bool encode_pool_map(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
+                     int32_t head_dim) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
+                        static_cast<cuuint64_t>(num_blocks) * pa::kBlockSize};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(head_dim) * num_kv_heads * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(pa::kBlockSize)};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                  elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- plan
+
+int rows_per_cta_for(int path, int rows) {
+  if (path == pa::kPathTile) {
+    const int r8 = static_cast<int>(ceil_div(rows, 8)) * 8;
+    return r8 < pa::kTileMaxRows ? r8 : pa::kTileMaxRows;
+  }
+  int r = 1;
+  while (r < rows && r < pa::kSingleMaxRows) r <<= 1;
+  return r;
+}
+
+pa_status_t check_shapes(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq) {
+  if (num_seqs < 0 || q_per_seq <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq <= 0 || head_dim <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (q_per_seq > 16) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;  // grid y
+  if (static_cast<int64_t>(max_blocks_per_seq) * pa::kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t max_blocks_per_seq, int32_t path_hint,
+                      int32_t split_blocks_hint, pa_plan_t* plan) {
+  pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                max_blocks_per_seq);
+  if (st != PA_OK) return st;
+  if (path_hint != PA_PATH_AUTO && path_hint != PA_PATH_SINGLE && path_hint != PA_PATH_TILE)
+    return PA_ERR_INVALID_ARG;
+  if (split_blocks_hint < 0) return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / num_kv_heads;
+  const int rows = group * q_per_seq;
+  int path = path_hint;
+  if (path == PA_PATH_AUTO) path = rows <= 2 ? PA_PATH_SINGLE : PA_PATH_TILE;
+  const int rpc = rows_per_cta_for(path, rows);
+  const int64_t row_chunks = ceil_div(rows, rpc);
+  if (num_kv_heads * row_chunks > 65535) return PA_ERR_UNSUPPORTED;  // grid x
+  int split_blocks = split_blocks_hint;
+  if (split_blocks == 0) {
+    // Host-known values only: units of (sequence, kv head, row chunk) against the
+    // number of resident CTAs. Enough units: one split. Otherwise cut the longest
+    // possible context into pieces so that about four waves of CTAs exist.
+    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * row_chunks;
+    const int64_t slots = static_cast<int64_t>(device_info().sms) *
+                          pa::decode_ctas_per_sm(path, head_dim, rpc);
+    if (units >= 2 * slots || units == 0) {
+      split_blocks = max_blocks_per_seq;
+    } else {
+      const int64_t splits = ceil_div(4 * slots, units);
+      int64_t sb = ceil_div(max_blocks_per_seq, splits);
+      sb = ceil_div(sb, pa::kWarpsPerCta) * pa::kWarpsPerCta;
+      if (sb < 8 * pa::kWarpsPerCta) sb = 8 * pa::kWarpsPerCta;
+      split_blocks = static_cast<int32_t>(sb < max_blocks_per_seq ? sb : max_blocks_per_seq);
+    }
+  }
+  const int64_t num_splits = ceil_div(max_blocks_per_seq, split_blocks);
+  if (num_splits > 65535) return PA_ERR_UNSUPPORTED;  // grid z
+  plan->path = path;
+  plan->split_blocks = split_blocks;
+  plan->num_splits = static_cast<int32_t>(num_splits);
+  plan->rows_per_cta = rpc;
+  return PA_OK;
+}
+
+size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
+                           int32_t num_q_heads, int32_t head_dim) {
+  if (plan.num_splits <= 1) return 0;
+  return static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads *
+         (static_cast<size_t>(head_dim) + 2) * 4;
+}
+
+pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t max_blocks_per_seq) {
+  if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE) return PA_ERR_INVALID_ARG;
+  if (plan.split_blocks <= 0) return PA_ERR_INVALID_ARG;
+  if (plan.num_splits != ceil_div(max_blocks_per_seq, plan.split_blocks)) return PA_ERR_INVALID_ARG;
+  const int rows = num_q_heads / num_kv_heads * q_per_seq;
+  if (plan.rows_per_cta != rows_per_cta_for(plan.path, rows)) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_version(void) { return kVersion; }
+
+const char* pa_status_string(pa_status_t status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: null/misaligned pointer or bad size";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: outside the supported shapes";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace missing or too small";
+    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE: bad slot, block id or context length";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime error";
+    case PA_ERR_DEVICE: return "PA_ERR_DEVICE: a kernel reported a bounded-wait timeout";
+  }
+  return "unknown pa_status_t";
+}
+
+pa_status_t pa_reshape_and_cache(const void* key, const void* value, int64_t key_token_stride,
+                                 int64_t value_token_stride, void* key_cache, void* value_cache,
+                                 const int64_t* slot_mapping, int64_t num_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim, int64_t num_blocks,
+                                 int32_t block_size, pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  const int64_t row_elems = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if ((row_elems * 2) % 16 != 0 || row_elems > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (key_token_stride < row_elems || value_token_stride < row_elems) return PA_ERR_INVALID_ARG;
+  if ((key_token_stride * 2) % 16 != 0 || (value_token_stride * 2) % 16 != 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens > (int64_t{1} << 30)) return PA_ERR_UNSUPPORTED;
+  cudaError_t e = pa::launch_cache_write(
+      static_cast<const uint16_t*>(key), static_cast<const uint16_t*>(value), key_token_stride,
+      value_token_stride, static_cast<uint16_t*>(key_cache), static_cast<uint16_t*>(value_cache),
+      slot_mapping, num_tokens, static_cast<int32_t>(row_elems), num_blocks * pa::kBlockSize,
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+                           int32_t path_hint, int32_t split_blocks_hint, pa_plan_t* plan) {
+  if (!plan) return PA_ERR_INVALID_ARG;
+  return make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                   path_hint, split_blocks_hint, plan);
+}
+
+size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq,
+                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_blocks_per_seq) {
+  pa_plan_t local;
+  if (!plan) {
+    if (make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                  PA_PATH_AUTO, 0, &local) != PA_OK)
+      return 0;
+    plan = &local;
+  }
+  return workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, head_dim);
+}
+
+pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+                      int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                      int64_t num_blocks, float scale, const pa_plan_t* plan, void* workspace,
+                      size_t workspace_bytes, pa_stream_t stream) {
+  pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                max_blocks_per_seq);
+  if (st != PA_OK) return st;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (num_blocks <= 0 || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (num_blocks * pa::kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;  // TMA coordinate range
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_INVALID_ARG;
+  pa_plan_t local;
+  if (plan) {
+    st = check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
+  } else {
+    st = make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                   PA_PATH_AUTO, 0, &local);
+    plan = &local;
+  }
+  if (st != PA_OK) return st;
+  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, head_dim);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
+
+  CUtensorMap tk, tv;
+  if (!encode_pool_map(&tk, key_cache, num_blocks, num_kv_heads, head_dim) ||
+      !encode_pool_map(&tv, value_cache, num_blocks, num_kv_heads, head_dim))
+    return PA_ERR_CUDA;
+
+  DecodeParams p = {};
+  p.out = static_cast<uint16_t*>(out);
+  p.query = static_cast<const uint16_t*>(query);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
+  if (need > 0) {
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_ml = reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                        static_cast<size_t>(num_seqs) * plan->num_splits * rq * head_dim);
+  }
+  p.num_seqs = num_seqs;
+  p.q_per_seq = q_per_seq;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.rows = p.group * q_per_seq;
+  p.max_blocks = max_blocks_per_seq;
+  p.split_blocks = plan->split_blocks;
+  p.num_splits = plan->num_splits;
+  p.rows_per_cta = plan->rows_per_cta;
+  p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = pa::launch_decode(p, plan->path, head_dim, tk, tv, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status_t pa_validate(const int32_t* block_tables, const int32_t* context_lens,
+                        const int64_t* slot_mapping, int32_t num_seqs, int32_t max_blocks_per_seq,
+                        int32_t q_per_seq, int64_t num_tokens, int64_t num_blocks,
+                        int32_t block_size, int64_t* num_bad, pa_stream_t stream) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || q_per_seq <= 0 || num_blocks <= 0 ||
+      (slot_mapping && num_tokens < 0))
+    return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 0 && (!block_tables || !context_lens)) return PA_ERR_INVALID_ARG;
+  int64_t bad = 0;
+  cudaError_t e = pa::run_validate(block_tables, context_lens, slot_mapping, num_seqs,
+                                   max_blocks_per_seq, q_per_seq, num_tokens, num_blocks, &bad,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (num_bad) *num_bad = bad;
+  return bad ? PA_ERR_OUT_OF_RANGE : PA_OK;
+}
+
+pa_status_t pa_get_device_error(uint32_t* code, int32_t reset, pa_stream_t stream) {
+  if (!code) return PA_ERR_INVALID_ARG;
+  cudaError_t e = pa::read_device_error(code, reset != 0, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  return *code ? PA_ERR_DEVICE : PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+"""ctypes binding of the C ABI in include/pa.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls. Tensors are
+torch CUDA tensors (PyTorch only provides device memory and streams); all
+computation happens in the sm_100a kernels of libpa_b200.so. Importing this
+module fails loudly when the library is missing -- there is no CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa_b200.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"CUDA library {_LIB_PATH} is not built: run "
+                      "`python -m paged_kv_cache_399_b200.build` (there is no CPU fallback)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_WORKSPACE = 3
+PA_ERR_OUT_OF_RANGE = 4
+PA_ERR_CUDA = 5
+PA_ERR_DEVICE = 6
+
+PA_PATH_AUTO = 0
+PA_PATH_SINGLE = 1
+PA_PATH_TILE = 2
+
+EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
+            "pa_validate", "pa_get_device_error", "pa_status_string", "pa_version"]
+
+
+class pa_plan_t(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("split_blocks", ctypes.c_int32),
+                ("num_splits", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32)]
+
+    def __repr__(self):
+        return (f"pa_plan_t(path={self.path}, split_blocks={self.split_blocks}, "
+                f"num_splits={self.num_splits}, rows_per_cta={self.rows_per_cta})")
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+
+_lib.pa_reshape_and_cache.restype = _I32
+_lib.pa_reshape_and_cache.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _I32, _I64, _I32, _P]
+_lib.pa_decode_plan.restype = _I32
+_lib.pa_decode_plan.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(pa_plan_t)]
+_lib.pa_decode_workspace_size.restype = ctypes.c_size_t
+_lib.pa_decode_workspace_size.argtypes = [ctypes.POINTER(pa_plan_t), _I32, _I32, _I32, _I32, _I32, _I32]
+_lib.pa_decode.restype = _I32
+_lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
+                           ctypes.c_float, ctypes.POINTER(pa_plan_t), _P, ctypes.c_size_t, _P]
+_lib.pa_validate.restype = _I32
+_lib.pa_validate.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I64, _I64, _I32, ctypes.POINTER(_I64), _P]
+_lib.pa_get_device_error.restype = _I32
+_lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), _I32, _P]
+_lib.pa_status_string.restype = ctypes.c_char_p
+_lib.pa_status_string.argtypes = [_I32]
+_lib.pa_version.restype = _I32
+_lib.pa_version.argtypes = []
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {pa_status_string(status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def pa_status_string(status: int) -> str:
+    return _lib.pa_status_string(status).decode()
+
+
+def pa_version() -> int:
+    return _lib.pa_version()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _check(status: int, where: str) -> None:
+    if status != PA_OK:
+        raise PAError(status, where)
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                         value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                         stream=None) -> None:
+    """key/value [T, H_kv, D] bf16 (token stride may exceed H_kv*D); caches
+    [NB, 16, H_kv, D] bf16; slot_mapping [T] int64."""
+    assert key.dtype == value.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.is_contiguous()
+    T, H, D = key.shape
+    assert key.stride(2) == 1 and key.stride(1) == D and value.stride(2) == 1 and value.stride(1) == D
+    assert key_cache.is_contiguous() and value_cache.is_contiguous()
+    NB, BS = key_cache.shape[0], key_cache.shape[1]
+    st = _lib.pa_reshape_and_cache(_ptr(key), _ptr(value), key.stride(0), value.stride(0),
+                                   _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping), T, H, D,
+                                   NB, BS, _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,
+                   head_dim: int, max_blocks_per_seq: int, path_hint: int = PA_PATH_AUTO,
+                   split_blocks_hint: int = 0) -> pa_plan_t:
+    plan = pa_plan_t()
+    st = _lib.pa_decode_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                             max_blocks_per_seq, path_hint, split_blocks_hint, ctypes.byref(plan))
+    _check(st, "pa_decode_plan")
+    return plan
+
+
+def pa_decode_workspace_size(plan: pa_plan_t | None, num_seqs: int, q_per_seq: int,
+                             num_q_heads: int, num_kv_heads: int, head_dim: int,
+                             max_blocks_per_seq: int) -> int:
+    return int(_lib.pa_decode_workspace_size(None if plan is None else ctypes.byref(plan), num_seqs,
+                                             q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                             max_blocks_per_seq))
+
+
+def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+              value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+              q_per_seq: int, scale: float, plan: pa_plan_t | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> None:
+    """out/query [B, q, H_q, D] bf16; caches [NB, 16, H_kv, D] bf16; block_tables
+    [B, max_blocks] int32; context_lens [B] int32. workspace: any contiguous CUDA
+    tensor of at least pa_decode_workspace_size(plan, ...) bytes (None when 0)."""
+    assert out.dtype == query.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    for t in (out, query, key_cache, value_cache, block_tables, context_lens):
+        assert t.is_contiguous()
+    B, QS, HQ, D = query.shape
+    assert QS == q_per_seq and tuple(out.shape) == tuple(query.shape)
+    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                        _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
+                        block_tables.shape[1], NB, float(scale),
+                        None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
+                        _stream(stream))
+    _check(st, "pa_decode")
+
+
+def pa_validate(block_tables: torch.Tensor, context_lens: torch.Tensor,
+                slot_mapping: torch.Tensor | None, q_per_seq: int, num_blocks: int,
+                block_size: int = 16, stream=None) -> int:
+    """Returns the number of out-of-range entries (0 = all preconditions hold)."""
+    bad = _I64(0)
+    T = 0 if slot_mapping is None else slot_mapping.numel()
+    st = _lib.pa_validate(_ptr(block_tables), _ptr(context_lens), _ptr(slot_mapping),
+                          block_tables.shape[0], block_tables.shape[1], q_per_seq, T, num_blocks,
+                          block_size, ctypes.byref(bad), _stream(stream))
+    if st not in (PA_OK, PA_ERR_OUT_OF_RANGE):
+        _check(st, "pa_validate")
+    return int(bad.value)
+
+
+def pa_get_device_error(reset: bool = True, stream=None) -> int:
+    code = ctypes.c_uint32(0)
+    st = _lib.pa_get_device_error(ctypes.byref(code), int(reset), _stream(stream))
+    if st not in (PA_OK, PA_ERR_DEVICE):
+        _check(st, "pa_get_device_error")
+    return int(code.value)
+
+
+def raw_library() -> ctypes.CDLL:
+    """The loaded ctypes handle (tests call entry points with raw pointers through it)."""
+    return _lib

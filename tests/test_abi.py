@@ -1,0 +1,117 @@
+"""The C-ABI library: loads, exports every declared symbol, and rejects bad
+arguments on the host before any launch (none of these calls touch a GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_399_b200 import build
+    build.build()
+    from paged_kv_cache_399_b200 import pa as mod
+    return mod
+
+
+def test_header_declares_the_north_star_calls():
+    syms = declared_symbols()
+    for name in ["pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size", "pa_decode_plan",
+                 "pa_validate", "pa_get_device_error", "pa_status_string", "pa_version"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(pa):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(pa.raw_library(), name)
+    assert set(pa.EXPORTED) == set(declared_symbols())
+    # only the C ABI is visible
+    assert all(s.startswith("pa_") or not s[0].isalpha() or s.startswith("_") for s in exported
+               if not s.startswith(("_init", "_fini"))), sorted(exported)[:20]
+
+
+def test_status_strings_and_version(pa):
+    for code in range(7):
+        assert pa.pa_status_string(code).startswith("PA_")
+    assert pa.pa_version() == 10000
+
+
+def _decode_raw(lib, **kw):
+    args = dict(out=8 * 1024, query=16 * 1024, kc=32 * 1024, vc=48 * 1024, bt=64 * 1024, cl=80 * 1024,
+                B=2, q=1, hq=4, hkv=2, d=64, bs=16, mb=4, nb=8, scale=0.125, plan=None, ws=None,
+                ws_bytes=0)
+    args.update(kw)
+    return lib.pa_decode(args["out"], args["query"], args["kc"], args["vc"], args["bt"], args["cl"],
+                         args["B"], args["q"], args["hq"], args["hkv"], args["d"], args["bs"],
+                         args["mb"], args["nb"], args["scale"], args["plan"], args["ws"],
+                         args["ws_bytes"], None)
+
+
+def test_decode_rejects_bad_arguments_before_launch(pa):
+    lib = pa.raw_library()
+    assert _decode_raw(lib, out=None) == pa.PA_ERR_INVALID_ARG
+    assert _decode_raw(lib, query=16 * 1024 + 2) == pa.PA_ERR_INVALID_ARG      # misaligned
+    assert _decode_raw(lib, hq=3) == pa.PA_ERR_INVALID_ARG                     # H_q % H_kv
+    assert _decode_raw(lib, d=96) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_raw(lib, bs=32) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_raw(lib, q=17) == pa.PA_ERR_UNSUPPORTED
+    assert _decode_raw(lib, q=0) == pa.PA_ERR_INVALID_ARG
+    assert _decode_raw(lib, scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert _decode_raw(lib, B=0) == pa.PA_OK                                    # no-op
+    # a split plan needs a workspace
+    plan = pa.pa_decode_plan(2, 1, 4, 2, 64, 4, pa.PA_PATH_TILE, 1)
+    assert plan.num_splits == 4
+    assert _decode_raw(lib, plan=ctypes.byref(plan)) == pa.PA_ERR_WORKSPACE
+    need = pa.pa_decode_workspace_size(plan, 2, 1, 4, 2, 64, 4)
+    assert need == 2 * 4 * 1 * 4 * (64 + 2) * 4
+    assert _decode_raw(lib, plan=ctypes.byref(plan), ws=96 * 1024, ws_bytes=need - 1) == pa.PA_ERR_WORKSPACE
+    bad = pa.pa_plan_t(plan.path, plan.split_blocks, plan.num_splits + 1, plan.rows_per_cta)
+    assert _decode_raw(lib, plan=ctypes.byref(bad), ws=96 * 1024, ws_bytes=need) == pa.PA_ERR_INVALID_ARG
+
+
+def test_cache_write_rejects_bad_arguments_before_launch(pa):
+    lib = pa.raw_library()
+
+    def call(**kw):
+        a = dict(k=1024, v=2048, ks=128, vs=128, kc=4096, vc=8192, slots=16384, T=4, hkv=2, d=64,
+                 nb=8, bs=16)
+        a.update(kw)
+        return lib.pa_reshape_and_cache(a["k"], a["v"], a["ks"], a["vs"], a["kc"], a["vc"], a["slots"],
+                                        a["T"], a["hkv"], a["d"], a["nb"], a["bs"], None)
+    assert call(k=None) == pa.PA_ERR_INVALID_ARG
+    assert call(kc=4096 + 8) == pa.PA_ERR_INVALID_ARG
+    assert call(ks=100) == pa.PA_ERR_INVALID_ARG          # stride below a row
+    assert call(ks=132) == pa.PA_ERR_INVALID_ARG          # stride*2 not a multiple of 16
+    assert call(slots=16384 + 4) == pa.PA_ERR_INVALID_ARG
+    assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
+    assert call(T=0, k=None) == pa.PA_OK                  # no-op
+
+
+def test_plan_heuristic_host_logic(pa):
+    # rows = G*q <= 2 -> CUDA-core kernel; more rows -> tensor-core tiles
+    assert pa.pa_decode_plan(4, 1, 4, 2, 64, 5).path == pa.PA_PATH_SINGLE
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024)
+    assert p.path == pa.PA_PATH_TILE and p.rows_per_cta == 24
+    p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192)
+    assert p.num_splits > 1 and p.split_blocks * p.num_splits >= 8192
+    forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)
+    assert (forced.path, forced.split_blocks, forced.num_splits, forced.rows_per_cta) == (1, 64, 128, 8)
+    # rows beyond one CTA are split into row chunks
+    assert pa.pa_decode_plan(2, 16, 16, 1, 128, 8).rows_per_cta == 32
+    with pytest.raises(pa.PAError):
+        pa.pa_decode_plan(2, 1, 4, 2, 80, 8)

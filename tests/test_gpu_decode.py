@@ -1,0 +1,139 @@
+"""pa_decode against the fp64 oracle on small shapes that span several blocks,
+ragged tails, every kernel and forced context splits, plus the degenerate cases."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import DeviceWorkload, assert_close, oracle_pools, run_step
+from paged_kv_cache_399_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+# (name, context lengths, q_per_seq, H_q, H_kv, head_dim, scale)
+CASES = [
+    ("ctx1", [1, 1, 1], 1, 4, 2, 64, None),
+    ("mult16", [16, 32, 64, 128], 1, 8, 2, 128, None),
+    ("ragged", [17, 49, 33, 200, 255], 1, 8, 2, 128, None),
+    ("mha", [40, 97, 300], 1, 4, 4, 128, None),
+    ("mqa", [40, 97, 300], 1, 8, 1, 128, None),
+    ("d64_gqa4", [5, 77, 160, 333], 1, 8, 2, 64, None),
+    ("spec2", [9, 40, 129], 2, 8, 2, 128, None),
+    ("spec6", [6, 16, 22, 300, 517], 6, 32, 8, 128, None),
+    ("spec6_d64", [7, 100, 64], 6, 4, 1, 64, None),
+    ("rows64", [33, 70], 16, 16, 4, 128, None),        # G*q = 64: two 32-row chunks
+    ("single_rows16", [50, 81], 2, 8, 1, 128, None),  # 16 rows on the CUDA-core path: two chunks
+    ("zero_scale", [25, 66], 3, 4, 2, 128, 0.0),
+    ("long_ragged", [1000, 2049, 3001], 1, 8, 1, 128, None),
+]
+
+PLANS = [
+    ("auto", None, None),
+    ("single", 1, None),
+    ("tile", 2, None),
+    ("single_split1", 1, 1),
+    ("tile_split1", 2, 1),
+    ("tile_split3", 2, 3),
+    ("tile_split8", 2, 8),
+]
+
+
+def _workload(case, seed):
+    name, ctxs, q, hq, hkv, d, scale = case
+    return workloads.build_workload(name, seed, ctxs, q, hq, hkv, d,
+                                    scale=(1.0 / math.sqrt(d)) if scale is None else scale,
+                                    pool_factor=1.5)
+
+
+@pytest.fixture(scope="module")
+def prepared(oracle_lib):
+    out = {}
+    for k, case in enumerate(CASES):
+        w = _workload(case, 2000 + k)
+        kc, vc = oracle_pools(oracle_lib, w)
+        ref = oracle_lib.decode(w.query, kc, vc, w.block_tables, w.context_lens, w.q_per_seq, w.scale)
+        out[case[0]] = (w, ref)
+    return out
+
+
+@pytest.mark.parametrize("plan_spec", PLANS, ids=[p[0] for p in PLANS])
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_decode_matches_oracle(case, plan_spec, prepared):
+    from paged_kv_cache_399_b200 import pa
+    w, ref = prepared[case[0]]
+    _, path, split = plan_spec
+    plan = None
+    if path is not None:
+        plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                 w.max_blocks_per_seq, path, split or 0)
+    dw = DeviceWorkload(w)
+    out = run_step(dw, plan)
+    assert_close(out, ref, f"{case[0]}/{plan_spec[0]}")
+
+
+def test_tiny_workload_every_path(oracle_lib):
+    from paged_kv_cache_399_b200 import pa
+    w = workloads.tiny()
+    kc, vc = oracle_pools(oracle_lib, w)
+    ref = oracle_lib.decode(w.query, kc, vc, w.block_tables, w.context_lens, 1, w.scale)
+    outs = []
+    for path in (pa.PA_PATH_SINGLE, pa.PA_PATH_TILE):
+        for split in (0, 1, 2):
+            plan = pa.pa_decode_plan(w.num_seqs, 1, 4, 2, 64, w.max_blocks_per_seq, path, split)
+            out = run_step(DeviceWorkload(w), plan)
+            assert_close(out, ref, f"tiny path={path} split={split}")
+            outs.append(out.float().cpu())
+    # cross-path agreement: every kernel / split within rounding of each other
+    for o in outs[1:]:
+        assert float((o - outs[0]).abs().max()) <= 2e-2
+
+
+def test_ctx1_returns_v0_exactly(oracle_lib):
+    """Closed form: one visible key gives out == v_0 (bf16 round trip is exact)."""
+    w = _workload(CASES[0], 2000)
+    dw = DeviceWorkload(w)
+    out = run_step(dw)
+    kc, vc = oracle_pools(oracle_lib, w)
+    g = w.num_q_heads // w.num_kv_heads
+    for b in range(w.num_seqs):
+        blk = int(w.block_tables[b, 0])
+        v0 = torch.from_numpy(vc[blk, 0].view(np.int16)).view(torch.bfloat16)
+        for h in range(w.num_q_heads):
+            assert torch.equal(out[b, 0, h].cpu(), v0[h // g])
+
+
+def test_block_permutation_invariance():
+    """Moving physical blocks (with a matching table) leaves the output unchanged."""
+    from paged_kv_cache_399_b200 import pa
+    w = _workload(CASES[2], 2002)
+    base = run_step(DeviceWorkload(w)).clone()
+    dw = DeviceWorkload(w)
+    pa.pa_reshape_and_cache(dw.key, dw.value, dw.key_cache, dw.value_cache, dw.slots)
+    sigma = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(5))
+    inv = torch.empty_like(sigma)
+    inv[sigma] = torch.arange(w.num_blocks)
+    kc = torch.empty_like(dw.key_cache)
+    vc = torch.empty_like(dw.value_cache)
+    kc[sigma.cuda()] = dw.key_cache
+    vc[sigma.cuda()] = dw.value_cache
+    dw.key_cache, dw.value_cache = kc, vc
+    dw.tables = sigma.cuda()[dw.tables.long()].to(torch.int32)
+    out = run_step(dw, write=False)
+    assert torch.equal(out, base)
+
+
+def test_validate_reports_bad_entries():
+    from paged_kv_cache_399_b200 import pa
+    w = _workload(CASES[2], 2002)
+    dw = DeviceWorkload(w)
+    assert pa.pa_validate(dw.tables, dw.ctx, dw.slots, w.q_per_seq, w.num_blocks) == 0
+    bad_tables = dw.tables.clone()
+    bad_tables[1, 0] = w.num_blocks + 3
+    bad_tables[2, 1] = -1
+    bad_ctx = dw.ctx.clone()
+    bad_ctx[0] = w.max_blocks_per_seq * 16 + 1
+    bad_slots = dw.slots.clone()
+    bad_slots[0] = w.num_blocks * 16
+    assert pa.pa_validate(bad_tables, bad_ctx, bad_slots, w.q_per_seq, w.num_blocks) == 4
