@@ -756,10 +756,10 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
 template <int D, int NT>
 constexpr int tile_stages() { return 2; }
 
-// Opt a kernel into its dynamic shared memory size once per device.
+// Opt a kernel into its dynamic shared memory size once per device. `done_mask`
+// (bit d: done on device d) must be owned by the kernel instance itself.
 template <typename Kernel>
-cudaError_t configure_smem(Kernel kernel, int smem) {
-  static unsigned long long done_mask = 0;  // bit d: done on device d
+cudaError_t configure_smem(Kernel kernel, int smem, unsigned long long& done_mask) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -776,7 +776,8 @@ cudaError_t launch_tile(const DecodeParams& p, const CUtensorMap& tk, const CUte
   constexpr int ST = tile_stages<D, NT>();
   constexpr int smem = DecodeSmem<D, NT * 8, kWarpsPerCta, ST>::kBytes;
   auto kernel = decode_tile_kernel<D, NT, kWarpsPerCta, ST>;
-  cudaError_t e = configure_smem(kernel, smem);
+  static unsigned long long done_mask = 0;  // one per template instance
+  cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, kWarpsPerCta * 32, smem);
   dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
@@ -789,7 +790,8 @@ cudaError_t launch_single(const DecodeParams& p, const CUtensorMap& tk, const CU
   constexpr int ST = 2;
   constexpr int smem = DecodeSmem<D, ROWS, kWarpsPerCta, ST>::kBytes;
   auto kernel = decode_single_kernel<D, ROWS, kWarpsPerCta, ST>;
-  cudaError_t e = configure_smem(kernel, smem);
+  static unsigned long long done_mask = 0;  // one per template instance
+  cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, kWarpsPerCta * 32, smem);
   dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
