@@ -143,6 +143,36 @@ PA_API pa_status_t pa_decode(void* out, const void* query, const void* key_cache
                       float scale, const pa_plan_t* plan, void* workspace,
                       size_t workspace_bytes, pa_stream_t stream);
 
+/* Size of the fixed scratch array pa_decode_static_scratch uses (16 MiB, held on
+ * every GPU that loads the library until the process exits). */
+#define PA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* pa_decode for callers that cannot allocate device memory where they decode: code
+ * inside another framework's memory pool that has already claimed the GPU's memory,
+ * loops that must avoid the implicit synchronisation of cudaMalloc/cudaFree, or
+ * plug-in hosts that forbid allocation in their execute step. The source pages have
+ * no counterpart to this call; it exists for such callers only.
+ * Same arguments and result as pa_decode without the workspace: the split path's
+ * partial records go to a PA_STATIC_SCRATCH_BYTES array compiled into the library.
+ * The caller still provides every input and output buffer. It calls no allocator.
+ * - A plan whose pa_decode_workspace_size exceeds PA_STATIC_SCRATCH_BYTES is
+ *   rejected with PA_ERR_WORKSPACE before anything is launched (pass an explicit
+ *   plan with longer splits, or use pa_decode).
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that first
+ *   call before any stream capture.
+ * - All calls share the one array per device and it keeps the last call's contents;
+ *   nothing in it needs to start at zero. Calls whose GPU work overlaps (unordered
+ *   streams) race on it: keep them ordered on one stream. */
+PA_API pa_status_t pa_decode_static_scratch(void* out, const void* query, const void* key_cache,
+                                     const void* value_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t q_per_seq, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq,
+                                     int64_t num_blocks, float scale, const pa_plan_t* plan,
+                                     pa_stream_t stream);
+
 /* Debug check of the device-resident preconditions (synchronous: waits for
  * `stream`). Counts context lengths outside [q_per_seq, max_blocks_per_seq *
  * block_size], used block-table entries outside [0, num_blocks) and slots >=

@@ -32,7 +32,10 @@ PA_PATH_SINGLE = 1
 PA_PATH_TILE = 2
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
-            "pa_validate", "pa_get_device_error", "pa_status_string", "pa_version"]
+            "pa_decode_static_scratch", "pa_validate", "pa_get_device_error", "pa_status_string",
+            "pa_version"]
+
+PA_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class pa_plan_t(ctypes.Structure):
@@ -57,6 +60,9 @@ _lib.pa_decode_workspace_size.argtypes = [ctypes.POINTER(pa_plan_t), _I32, _I32,
 _lib.pa_decode.restype = _I32
 _lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
                            ctypes.c_float, ctypes.POINTER(pa_plan_t), _P, ctypes.c_size_t, _P]
+_lib.pa_decode_static_scratch.restype = _I32
+_lib.pa_decode_static_scratch.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32,
+                                          _I32, _I64, ctypes.c_float, ctypes.POINTER(pa_plan_t), _P]
 _lib.pa_validate.restype = _I32
 _lib.pa_validate.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I64, _I64, _I32, ctypes.POINTER(_I64), _P]
 _lib.pa_get_device_error.restype = _I32
@@ -158,6 +164,27 @@ def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
                         None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
                         _stream(stream))
     _check(st, "pa_decode")
+
+
+def pa_decode_static_scratch(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, block_tables: torch.Tensor,
+                             context_lens: torch.Tensor, q_per_seq: int, scale: float,
+                             plan: pa_plan_t | None = None, stream=None) -> None:
+    """pa_decode without a caller workspace: for callers that cannot allocate device
+    memory where they decode. Split partials go to the library's fixed
+    PA_STATIC_SCRATCH_BYTES array; calls must not overlap on the GPU."""
+    assert out.dtype == query.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    for t in (out, query, key_cache, value_cache, block_tables, context_lens):
+        assert t.is_contiguous()
+    B, QS, HQ, D = query.shape
+    assert QS == q_per_seq and tuple(out.shape) == tuple(query.shape)
+    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    st = _lib.pa_decode_static_scratch(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                       _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
+                                       block_tables.shape[1], NB, float(scale),
+                                       None if plan is None else ctypes.byref(plan), _stream(stream))
+    _check(st, "pa_decode_static_scratch")
 
 
 def pa_validate(block_tables: torch.Tensor, context_lens: torch.Tensor,
