@@ -207,8 +207,11 @@ def run_gpu(args):
     key_cache = w.key_cache.to(dev)
     value_cache = w.value_cache.to(dev)
     out = torch.empty_like(query)
+    # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
+    share = bool(w.shared_groups) and not args.no_share_prefix
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                             w.max_blocks_per_seq)
+                             w.max_blocks_per_seq, share_prefix=share,
+                             schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
     ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads,
                                            w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
@@ -231,7 +234,7 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    launches_per_step = 2 + (1 if plan.num_splits > 1 else 0)
+    launches_per_step = 1 + (2 if (plan.schedule == pa.PA_SCHEDULE_PERSISTENT or plan.num_splits > 1) else 1)
     step_bytes = decode_bytes(w) + cache_write_bytes(w)
     dec_bytes = decode_bytes(w)
 
@@ -333,8 +336,7 @@ def run_gpu(args):
                 "decode_frac_of_measured_hbm": round(achieved / peaks["hbm_gbs"], 4),
                 "decode_frac_of_spec_8tbs": round(achieved / 8000.0, 4),
                 "step_frac_of_measured_hbm": round(value_gbs / world / peaks["hbm_gbs"], 4),
-                "plan": {"path": {1: "single", 2: "tile"}[plan.path], "split_blocks": plan.split_blocks,
-                         "num_splits": plan.num_splits, "rows_per_cta": plan.rows_per_cta},
+                "plan": plan.as_dict(),
                 "l2": "no flush: each step reads more bytes than the 126 MB L2 holds"
                       if dec_bytes > 2 * 126e6 else "no flush: working set near L2 size (see DESIGN)",
                 "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
@@ -347,7 +349,7 @@ def run_gpu(args):
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic,
                 "peak_source": peaks["source"],
-                "kernel": "pa_decode (decode kernel + merge when split)",
+                "kernel": "pa_decode (schedule pre-pass + decode kernel, or grid decode + merge)",
             },
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -460,6 +462,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", choices=["auto", "grid", "persistent"], default="auto")
+    ap.add_argument("--no-share-prefix", action="store_true",
+                    help="do not ask pa_decode to read shared prefix blocks once per group")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     args = ap.parse_args(argv)

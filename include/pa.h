@@ -84,15 +84,39 @@ typedef enum {
   PA_PATH_TILE = 2    /* tensor-core kernel: mma.sync m16n8k16 bf16 -> fp32 */
 } pa_path_t;
 
-/* How pa_decode splits the work. num_splits > 1 means each sequence's context is
- * cut into chunks of split_blocks blocks (flash-decoding); the chunks write fp32
- * partial (o, m, l) records to the workspace and a log-sum-exp merge kernel
- * combines them. */
+/* How the work is spread over CTAs. */
+typedef enum {
+  PA_SCHEDULE_AUTO = 0,
+  PA_SCHEDULE_GRID = 1,       /* one CTA per (kv head, sequence, context split of
+                                 split_blocks blocks) + a log-sum-exp merge kernel */
+  PA_SCHEDULE_PERSISTENT = 2  /* a one-CTA pre-pass reads context_lens and cuts all
+                                 (sequence, kv head, block) work into num_ctas equal
+                                 shares; one resident CTA per share; pieces of an
+                                 output are merged by the CTA that finishes it */
+} pa_schedule_t;
+
+/* Optional hints for pa_decode_plan; zero-initialised = all automatic. */
+typedef struct {
+  int32_t path;          /* pa_path_t */
+  int32_t schedule;      /* pa_schedule_t */
+  int32_t split_blocks;  /* grid schedule: blocks per split (0 = heuristic) */
+  int32_t share_prefix;  /* persistent schedule: 1 = adjacent sequences whose block
+                            tables start with the same physical blocks (parallel
+                            sampling, beam search, a common system prompt) are
+                            detected on the device and their common prefix blocks
+                            are read once for all of them; 0 = off */
+} pa_plan_hints_t;
+
+/* A decode plan; fill it with pa_decode_plan and treat it as opaque. */
 typedef struct {
   int32_t path;          /* PA_PATH_SINGLE or PA_PATH_TILE */
-  int32_t split_blocks;  /* blocks per split, >= 1 */
-  int32_t num_splits;    /* ceil(max_blocks_per_seq / split_blocks) */
+  int32_t schedule;      /* PA_SCHEDULE_GRID or PA_SCHEDULE_PERSISTENT */
+  int32_t split_blocks;  /* grid: blocks per split */
+  int32_t num_splits;    /* grid: ceil(max_blocks_per_seq / split_blocks) */
   int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds */
+  int32_t num_ctas;      /* persistent: CTAs launched (resident slots of the device) */
+  int32_t share_cap;     /* persistent: sequences per shared-prefix unit, 0 = off */
+  int32_t reserved;
 } pa_plan_t;
 
 /* Write the step's new K/V into the pool: for each token t with slot s =
@@ -110,17 +134,18 @@ PA_API pa_status_t pa_reshape_and_cache(const void* key, const void* value,
                                  int64_t num_blocks, int32_t block_size,
                                  pa_stream_t stream);
 
-/* Choose a plan from host-known shape values only (no device read). path_hint
- * PA_PATH_AUTO lets the heuristic pick the kernel; split_blocks_hint 0 lets it
- * pick the split length. The heuristic reads the SM count of the current device. */
+/* Choose a plan from host-known shape values only (no device read). hints may be
+ * NULL. The heuristic reads the SM count of the current device and the occupancy of
+ * the chosen kernel. */
 PA_API pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
                            int32_t num_kv_heads, int32_t head_dim,
-                           int32_t max_blocks_per_seq, int32_t path_hint,
-                           int32_t split_blocks_hint, pa_plan_t* plan);
+                           int32_t max_blocks_per_seq, const pa_plan_hints_t* hints,
+                           pa_plan_t* plan);
 
 /* Workspace bytes pa_decode needs for `plan` (NULL = the heuristic plan for these
- * shapes): num_seqs * num_splits * q_per_seq * num_q_heads * (head_dim + 2) * 4
- * when num_splits > 1, else 0. */
+ * shapes). Grid schedule: split partials, 0 when there is one split. Persistent
+ * schedule: the pre-pass tables, per-output counters and record lists, and a pool of
+ * fp32 partial records (a few MB for the shapes above). */
 PA_API size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs,
                                 int32_t q_per_seq, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim,
@@ -131,7 +156,8 @@ PA_API size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs,
  * accumulation. A row with no visible key (context_len < q_per_seq, a precondition
  * violation) yields 0. plan NULL = heuristic. workspace: 16-byte aligned device
  * buffer of at least pa_decode_workspace_size(plan, ...) bytes, may be NULL when
- * that size is 0; its contents need no initialisation and are scratch afterwards.
+ * that size is 0; its contents need no initialisation and are scratch afterwards
+ * (the persistent schedule's pre-pass resets its counters on every call).
  * Reads query/block_tables/context_lens/caches only after the preceding work on
  * the stream has completed (programmatic dependent launch is used to hide the
  * launch latency). num_seqs == 0 is a no-op. */

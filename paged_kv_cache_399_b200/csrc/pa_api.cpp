@@ -105,34 +105,60 @@ pa_status_t check_shapes(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_head
   return PA_OK;
 }
 
+// Members of one shared-prefix unit: as many sequences as fit the tile kernel's rows.
+int share_cap_for(int rows) { return rows <= pa::kTileMaxRows / 2 ? pa::kTileMaxRows / rows : 0; }
+
 pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
-                      int32_t head_dim, int32_t max_blocks_per_seq, int32_t path_hint,
-                      int32_t split_blocks_hint, pa_plan_t* plan) {
+                      int32_t head_dim, int32_t max_blocks_per_seq, const pa_plan_hints_t* hints,
+                      pa_plan_t* plan) {
   pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
                                 max_blocks_per_seq);
   if (st != PA_OK) return st;
-  if (path_hint != PA_PATH_AUTO && path_hint != PA_PATH_SINGLE && path_hint != PA_PATH_TILE)
+  pa_plan_hints_t h = {};
+  if (hints) h = *hints;
+  if (h.path != PA_PATH_AUTO && h.path != PA_PATH_SINGLE && h.path != PA_PATH_TILE)
     return PA_ERR_INVALID_ARG;
-  if (split_blocks_hint < 0) return PA_ERR_INVALID_ARG;
+  if (h.schedule != PA_SCHEDULE_AUTO && h.schedule != PA_SCHEDULE_GRID &&
+      h.schedule != PA_SCHEDULE_PERSISTENT)
+    return PA_ERR_INVALID_ARG;
+  if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1) return PA_ERR_INVALID_ARG;
   const int group = num_q_heads / num_kv_heads;
   const int rows = group * q_per_seq;
-  int path = path_hint;
-  if (path == PA_PATH_AUTO) path = rows <= 2 ? PA_PATH_SINGLE : PA_PATH_TILE;
-  const int rpc = rows_per_cta_for(path, rows);
+  int schedule = h.schedule == PA_SCHEDULE_AUTO ? PA_SCHEDULE_PERSISTENT : h.schedule;
+  int share_cap = 0;
+  if (h.share_prefix) {
+    if (schedule != PA_SCHEDULE_PERSISTENT) return PA_ERR_INVALID_ARG;
+    share_cap = share_cap_for(rows);
+    if (share_cap < 2 || h.path == PA_PATH_SINGLE) return PA_ERR_UNSUPPORTED;
+  }
+  int path = h.path;
+  if (path == PA_PATH_AUTO) path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
+  // a shared-prefix unit holds share_cap sequences' rows in one CTA
+  const int rpc = share_cap ? pa::kTileMaxRows : rows_per_cta_for(path, rows);
   const int64_t row_chunks = ceil_div(rows, rpc);
   if (num_kv_heads * row_chunks > 65535) return PA_ERR_UNSUPPORTED;  // grid x
-  int split_blocks = split_blocks_hint;
+  const int slots = device_info().sms * pa::decode_ctas_per_sm(path, schedule, head_dim, rpc);
+  plan->path = path;
+  plan->schedule = schedule;
+  plan->rows_per_cta = rpc;
+  plan->share_cap = share_cap;
+  plan->reserved = 0;
+  if (schedule == PA_SCHEDULE_PERSISTENT) {
+    plan->num_ctas = slots;
+    plan->split_blocks = max_blocks_per_seq;
+    plan->num_splits = 1;
+    return PA_OK;
+  }
+  int split_blocks = h.split_blocks;
   if (split_blocks == 0) {
     // Host-known values only: units of (sequence, kv head, row chunk) against the
     // number of resident CTAs. Enough units: one split. Otherwise cut the longest
     // possible context into pieces so that about four waves of CTAs exist.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * row_chunks;
-    const int64_t slots = static_cast<int64_t>(device_info().sms) *
-                          pa::decode_ctas_per_sm(path, head_dim, rpc);
-    if (units >= 2 * slots || units == 0) {
+    if (units >= 2 * static_cast<int64_t>(slots) || units == 0) {
       split_blocks = max_blocks_per_seq;
     } else {
-      const int64_t splits = ceil_div(4 * slots, units);
+      const int64_t splits = ceil_div(4 * static_cast<int64_t>(slots), units);
       int64_t sb = ceil_div(max_blocks_per_seq, splits);
       sb = ceil_div(sb, pa::kWarpsPerCta) * pa::kWarpsPerCta;
       if (sb < 8 * pa::kWarpsPerCta) sb = 8 * pa::kWarpsPerCta;
@@ -141,15 +167,55 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   }
   const int64_t num_splits = ceil_div(max_blocks_per_seq, split_blocks);
   if (num_splits > 65535) return PA_ERR_UNSUPPORTED;  // grid z
-  plan->path = path;
   plan->split_blocks = split_blocks;
   plan->num_splits = static_cast<int32_t>(num_splits);
-  plan->rows_per_cta = rpc;
+  plan->num_ctas = 0;
   return PA_OK;
 }
 
+// Byte layout of the persistent schedule's workspace.
+struct PersistentLayout {
+  size_t hdr, seq_start, seq_info, cta_seq, arrive, list_len, list, records, total;
+  int32_t target_rows, list_cap, pool_cap, rec_stride;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
+
+PersistentLayout persistent_layout(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
+  PersistentLayout L = {};
+  const int64_t rows = static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq;
+  const int64_t rc = ceil_div(rows, plan.rows_per_cta);
+  const int64_t targets = static_cast<int64_t>(num_seqs) * num_kv_heads * rc;
+  const int64_t P = plan.num_ctas;
+  L.target_rows = static_cast<int32_t>(rows < plan.rows_per_cta ? rows : plan.rows_per_cta);
+  L.list_cap = static_cast<int32_t>(2 * P + 4);
+  // records: one per non-direct private piece (<= targets + P) plus, with prefix
+  // sharing, up to share_cap per shared piece (<= H_kv * B/2 shared sub-units + P)
+  int64_t pool = targets + P;
+  if (plan.share_cap >= 2) pool += plan.share_cap * (num_kv_heads * ceil_div(num_seqs, 2) + P);
+  L.pool_cap = static_cast<int32_t>(pool);
+  // o rows then (m, l) pairs, rounded to 4 floats so every record is 16-byte aligned
+  L.rec_stride = (L.target_rows * head_dim + 2 * L.target_rows + 3) & ~3;
+  size_t off = 0;
+  L.hdr = off; off = align256(off + sizeof(pa::SchedHeader));
+  L.seq_start = off; off = align256(off + sizeof(long long) * num_seqs);
+  L.seq_info = off; off = align256(off + 16 * static_cast<size_t>(num_seqs));
+  L.cta_seq = off; off = align256(off + 4 * static_cast<size_t>(P));
+  L.arrive = off; off = align256(off + 4 * static_cast<size_t>(targets));
+  L.list_len = off; off = align256(off + 4 * static_cast<size_t>(targets));
+  L.list = off; off = align256(off + 4 * static_cast<size_t>(targets) * L.list_cap);
+  L.records = off; off = align256(off + 4 * static_cast<size_t>(pool) * L.rec_stride);
+  L.total = off;
+  return L;
+}
+
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
-                           int32_t num_q_heads, int32_t head_dim) {
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
+  if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
+    if (num_seqs == 0) return 0;
+    return persistent_layout(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim).total;
+  }
   if (plan.num_splits <= 1) return 0;
   return static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads *
          (static_cast<size_t>(head_dim) + 2) * 4;
@@ -158,9 +224,21 @@ size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_pe
 pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_heads,
                        int32_t num_kv_heads, int32_t max_blocks_per_seq) {
   if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE) return PA_ERR_INVALID_ARG;
-  if (plan.split_blocks <= 0) return PA_ERR_INVALID_ARG;
-  if (plan.num_splits != ceil_div(max_blocks_per_seq, plan.split_blocks)) return PA_ERR_INVALID_ARG;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
+  if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
+    if (plan.num_ctas <= 0 || plan.num_ctas > (1 << 20)) return PA_ERR_INVALID_ARG;
+    if (plan.share_cap != 0) {
+      if (plan.path != PA_PATH_TILE || plan.share_cap != share_cap_for(rows) ||
+          plan.rows_per_cta != pa::kTileMaxRows)
+        return PA_ERR_INVALID_ARG;
+      return PA_OK;
+    }
+  } else if (plan.schedule == PA_SCHEDULE_GRID) {
+    if (plan.split_blocks <= 0 || plan.share_cap != 0) return PA_ERR_INVALID_ARG;
+    if (plan.num_splits != ceil_div(max_blocks_per_seq, plan.split_blocks)) return PA_ERR_INVALID_ARG;
+  } else {
+    return PA_ERR_INVALID_ARG;
+  }
   if (plan.rows_per_cta != rows_per_cta_for(plan.path, rows)) return PA_ERR_INVALID_ARG;
   return PA_OK;
 }
@@ -212,10 +290,10 @@ pa_status_t pa_reshape_and_cache(const void* key, const void* value, int64_t key
 
 pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
                            int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
-                           int32_t path_hint, int32_t split_blocks_hint, pa_plan_t* plan) {
+                           const pa_plan_hints_t* hints, pa_plan_t* plan) {
   if (!plan) return PA_ERR_INVALID_ARG;
   return make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                   path_hint, split_blocks_hint, plan);
+                   hints, plan);
 }
 
 size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq,
@@ -224,11 +302,11 @@ size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs, int32_t
   pa_plan_t local;
   if (!plan) {
     if (make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                  PA_PATH_AUTO, 0, &local) != PA_OK)
+                  nullptr, &local) != PA_OK)
       return 0;
     plan = &local;
   }
-  return workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, head_dim);
+  return workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
 }
 
 pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -254,11 +332,11 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
     st = check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
   } else {
     st = make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                   PA_PATH_AUTO, 0, &local);
+                   nullptr, &local);
     plan = &local;
   }
   if (st != PA_OK) return st;
-  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, head_dim);
+  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
 
   CUtensorMap tk, tv;
@@ -271,12 +349,6 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   p.query = static_cast<const uint16_t*>(query);
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
-  if (need > 0) {
-    p.ws_o = static_cast<float*>(workspace);
-    p.ws_ml = reinterpret_cast<float2*>(static_cast<float*>(workspace) +
-                                        static_cast<size_t>(num_seqs) * plan->num_splits * rq * head_dim);
-  }
   p.num_seqs = num_seqs;
   p.q_per_seq = q_per_seq;
   p.num_q_heads = num_q_heads;
@@ -284,12 +356,36 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   p.group = num_q_heads / num_kv_heads;
   p.rows = p.group * q_per_seq;
   p.max_blocks = max_blocks_per_seq;
-  p.split_blocks = plan->split_blocks;
-  p.num_splits = plan->num_splits;
   p.rows_per_cta = plan->rows_per_cta;
   p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
   p.scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = pa::launch_decode(p, plan->path, head_dim, tk, tv, reinterpret_cast<cudaStream_t>(stream));
+  p.split_blocks = plan->split_blocks;
+  p.num_splits = plan->num_splits;
+  const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
+  char* ws = static_cast<char*>(workspace);
+  if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
+    const PersistentLayout L = persistent_layout(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
+    p.num_ctas = plan->num_ctas;
+    p.share_cap = plan->share_cap;
+    p.target_rows = L.target_rows;
+    p.list_cap = L.list_cap;
+    p.pool_cap = L.pool_cap;
+    p.rec_stride = L.rec_stride;
+    p.hdr = reinterpret_cast<pa::SchedHeader*>(ws + L.hdr);
+    p.seq_start = reinterpret_cast<long long*>(ws + L.seq_start);
+    p.seq_info = reinterpret_cast<int4*>(ws + L.seq_info);
+    p.cta_seq = reinterpret_cast<int32_t*>(ws + L.cta_seq);
+    p.arrive = reinterpret_cast<int32_t*>(ws + L.arrive);
+    p.list_len = reinterpret_cast<int32_t*>(ws + L.list_len);
+    p.list = reinterpret_cast<int32_t*>(ws + L.list);
+    p.records = reinterpret_cast<float*>(ws + L.records);
+  } else if (need > 0) {
+    p.ws_o = reinterpret_cast<float*>(ws);
+    p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) +
+                                        static_cast<size_t>(num_seqs) * plan->num_splits * rq * head_dim);
+  }
+  cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, tk, tv,
+                                    reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -11,34 +11,64 @@ namespace pa {
 constexpr int kBlockSize = 16;   // tokens per KV block
 constexpr int kWarpsPerCta = 4;  // decode CTA = 4 warps, each with its own TMA pipeline
 
+// Kernel families (pa_path_t values) and schedules (pa_schedule_t values).
+constexpr int kPathSingle = 1;
+constexpr int kPathTile = 2;
+constexpr int kScheduleGrid = 1;
+constexpr int kSchedulePersistent = 2;
+
+// Largest rows one CTA holds for each family.
+constexpr int kTileMaxRows = 32;   // 4 n-tiles of 8 rows
+constexpr int kSingleMaxRows = 8;
+
+// Persistent schedule: header written by the pre-pass, read by the decode CTAs.
+struct SchedHeader {
+  long long work;   // total work units (blocks x kv-head sub-units), W
+  int pool;         // partial records handed out so far
+  int pad[13];
+};
+
 struct DecodeParams {
   uint16_t* out;                 // bf16 [B][q][H_q][D]
   const uint16_t* query;         // bf16 [B][q][H_q][D]
   const int32_t* block_tables;   // [B][max_blocks]
   const int32_t* context_lens;   // [B]
-  float* ws_o;                   // fp32 [B][num_splits][q*H_q][D]   (split plans only)
-  float2* ws_ml;                 // fp32 [B][num_splits][q*H_q] (m in log2 units, l)
   int32_t num_seqs, q_per_seq, num_q_heads, num_kv_heads, group;  // group = H_q / H_kv
-  int32_t rows;                  // group * q_per_seq query rows per kv head
-  int32_t max_blocks, split_blocks, num_splits, row_chunks, rows_per_cta;
+  int32_t rows;                  // group * q_per_seq query rows per (sequence, kv head)
+  int32_t max_blocks;
+  int32_t rows_per_cta;          // rows the kernel instance holds (ROWS)
+  int32_t row_chunks;            // ceil(rows / rows_per_cta)
   float scale_log2;              // scale * log2(e)
+
+  // grid schedule: split partials for the merge kernel
+  int32_t split_blocks, num_splits;
+  float* ws_o;                   // fp32 [B][num_splits][q*H_q][D]
+  float2* ws_ml;                 // fp32 [B][num_splits][q*H_q] (m in log2 units, l)
+
+  // persistent schedule
+  int32_t num_ctas;              // persistent grid size
+  int32_t share_cap;             // >= 2: members per shared-prefix unit; 0: no prefix sharing
+  int32_t target_rows;           // rows of one output target (<= rows_per_cta)
+  int32_t list_cap;              // record list capacity per target
+  int32_t pool_cap;              // record pool capacity
+  int32_t rec_stride;            // floats per record: target_rows * D + 2 * target_rows
+  SchedHeader* hdr;
+  long long* seq_start;          // [B] first work unit of the sequence's bands
+  int4* seq_info;                // [B] {P_b shared prefix blocks, members if leader else 0, nblk, 0}
+  int32_t* cta_seq;              // [num_ctas] sequence holding the CTA's first unit
+  int32_t* arrive;               // [targets] blocks merged so far
+  int32_t* list_len;             // [targets]
+  int32_t* list;                 // [targets][list_cap] record slots
+  float* records;                // [pool_cap][rec_stride]
 };
 
-// Kernel families (pa_path_t values).
-constexpr int kPathSingle = 1;
-constexpr int kPathTile = 2;
-
-// Largest rows_per_cta each family is instantiated for.
-constexpr int kTileMaxRows = 32;   // 4 n-tiles of 8 rows
-constexpr int kSingleMaxRows = 8;
-
-// Launch the decode kernel of `path` (and the merge kernel when num_splits > 1).
-cudaError_t launch_decode(const DecodeParams& p, int path, int head_dim,
+// Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).
+cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim,
                           const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
                           cudaStream_t stream);
 
-// Resident CTAs per SM of the decode kernel that launch_decode would use.
-int decode_ctas_per_sm(int path, int head_dim, int rows_per_cta);
+// Resident CTAs per SM of the decode kernel launch_decode would use.
+int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta);
 
 cudaError_t launch_cache_write(const uint16_t* key, const uint16_t* value, int64_t key_stride,
                                int64_t value_stride, uint16_t* key_cache, uint16_t* value_cache,

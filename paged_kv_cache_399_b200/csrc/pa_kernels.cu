@@ -1,29 +1,39 @@
 // sm_100a kernels of the paged KV-cache hot path.
 //
-//   cache_write_kernel   slot_mapping scatter of the step's new K/V rows
-//                        ("vLLM 深度实战：从 PagedAttention 到 Speculative Decoding" §3.3)
-//   decode_tile_kernel   paged decode on tensor cores (mma.sync m16n8k16, bf16 -> fp32)
-//   decode_single_kernel paged decode on CUDA cores (fp32 FMA, warp-shuffle reductions)
-//   merge_kernel         log-sum-exp merge of split-context partials
-//   validate_kernel      debug bounds check of slots / block ids / context lengths
+//   cache_write_kernel       slot_mapping scatter of the step's new K/V rows
+//                            ("vLLM 深度实战：从 PagedAttention 到 Speculative Decoding" §3.3)
+//   sched_prepass_kernel     persistent schedule: equal-work partition of all
+//                            (sequence, kv head, block) units, optional detection of
+//                            adjacent sequences sharing prefix blocks
+//   decode_persistent_kernel paged decode, one CTA per resident slot, each over an
+//                            equal share of the work; partial results are merged by
+//                            the CTA that completes an output
+//   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split)
+//   merge_kernel             log-sum-exp merge of the grid schedule's split partials
+//   validate_kernel          debug bounds check of slots / block ids / context lengths
 //
-// Both decode kernels walk each sequence's block table ("vLLM study notes"
-// zihan-zhang.net §3.2: logical block -> physical block, then a contiguous read of
-// the block) and keep a running max / running sum / rescaled output per query row
-// (same notes §4.3.1, online softmax). Work unit = one CTA per (kv head, sequence,
-// context split, row chunk); the CTA's 4 warps take the split's blocks round-robin,
-// each warp with its own TMA pipeline, and are merged through shared memory.
+// Two compute cores run inside the decode kernels:
+//   TileCore   tensor cores: mma.sync m16n8k16 bf16 -> fp32 on S^T = K Q^T and
+//              O^T += V^T P^T, online softmax on the accumulator fragments;
+//   SimtCore   CUDA cores: fp32 FMA dot products, warp-shuffle max / sum.
+// Both walk a sequence's block table ("vLLM study notes", zihan-zhang.net §3.2: logical
+// block -> physical block, contiguous read inside a block) and keep a running max,
+// running sum and rescaled output per query row (same notes §4.3.1). Partial states
+// (m, l, o) of disjoint key ranges combine by the same rescaling: out =
+// sum_k o_k 2^(m_k - M) / sum_k l_k 2^(m_k - M), M = max_k m_k (log2 units).
 //
-// Pool layout [num_blocks][16][H_kv][D] bf16: the 16 rows of one (block, kv head)
-// are D*2 bytes each, H_kv*D*2 bytes apart. One TMA box {64 elems, 1 head, 16
-// tokens} moves one 2 KB half-tile with the 128-byte swizzle, so ldmatrix reads are
-// bank-conflict free: 16-byte chunk c of tile row r sits at chunk c ^ (r & 7).
+// Pool layout [num_blocks][16][H_kv][D] bf16: the 16 rows of one (block, kv head) are
+// D*2 bytes each, H_kv*D*2 bytes apart. One TMA box {64 elems, 1 head, 16 tokens}
+// moves one 2 KB half-tile with the 128-byte swizzle, so ldmatrix reads are bank-
+// conflict free: 16-byte chunk c of tile row r sits at chunk c ^ (r & 7). Every CTA
+// warp owns a private STAGES-deep TMA pipeline (one mbarrier per stage).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cfloat>
+#include <climits>
 #include <cstdint>
 
 #include "pa_device.cuh"
@@ -34,6 +44,10 @@ namespace pa {
 __device__ unsigned int g_device_error = 0;
 
 __device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_device_error, 0u, code); }
+
+constexpr unsigned kErrRecordPool = 0x300u;
+constexpr unsigned kErrRecordList = 0x400u;
+constexpr unsigned kErrSchedule = 0x500u;
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kHalfTileBytes = 16 * 64 * 2;  // 16 tokens x 64 bf16
@@ -50,10 +64,43 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// Byte offset of 16-byte chunk `c` (0..D/8-1) of token row `t` inside a K or V
-// tile made of 128-byte-swizzled 2 KB halves.
+// Byte offset of 16-byte chunk `c` (0..D/8-1) of token row `t` inside a K or V tile
+// made of 128-byte-swizzled 2 KB halves.
 __device__ __forceinline__ uint32_t tile_chunk_offset(int t, int c) {
   return static_cast<uint32_t>((c >> 3) * kHalfTileBytes + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+__device__ __forceinline__ int num_blocks_of(const DecodeParams& p, int ctx) {
+  return min(max(ctx, 0) + kBlockSize - 1, p.max_blocks * kBlockSize) / kBlockSize;
+}
+
+// ---------------------------------------------------------------------------
+// A segment: consecutive blocks [blk0, blk1) of one kv head, for a set of query rows.
+// Private: rows row0 .. row0+nrows-1 of sequence b0. Shared: `members` sequences
+// b0 .. b0+members-1 that map these blocks to the same physical blocks; local row r
+// is row r % rows of member r / rows.
+// ---------------------------------------------------------------------------
+struct Seg {
+  int b0, members, kvh, row0, nrows, blk0, blk1;
+  bool shared;
+};
+
+__device__ __forceinline__ bool seg_row(const DecodeParams& p, const Seg& s, int r, int& b, int& i,
+                                        int& h) {
+  if (r >= s.nrows) return false;
+  int m = 0, rr = s.row0 + r;
+  if (s.shared) {
+    m = r / p.rows;
+    rr = r - m * p.rows;
+  }
+  b = s.b0 + m;
+  i = rr / p.group;
+  h = s.kvh * p.group + (rr - i * p.group);
+  return true;
+}
+
+__device__ __forceinline__ size_t out_offset(const DecodeParams& p, int b, int i, int h, int D) {
+  return ((static_cast<size_t>(b) * p.q_per_seq + i) * p.num_q_heads + h) * D;
 }
 
 // ---------------------------------------------------------------------------
@@ -67,20 +114,28 @@ struct WarpPipe {
   int blk0, warp, lane, n_my, kvh;
   int tchunk, tbase;     // 32 table entries cached in registers, lane k -> entry tbase+k
   int issued;
+  uint32_t phase_base;   // loads issued on this warp's barriers before this run
 
   __device__ __forceinline__ int table_entry(int k) const {
     return k < n_my ? __ldg(trow + blk0 + warp + NW * k) : 0;
   }
-  __device__ __forceinline__ void init(uint8_t* smem, uint64_t* all_bars, const int32_t* row,
-                                       int blk0_, int blk1, int warp_, int lane_, int kvh_) {
+  __device__ __forceinline__ void init(uint8_t* smem, uint64_t* all_bars, int warp_, int lane_) {
     warp = warp_;
     lane = lane_;
+    stage_base = smem + warp * STAGES * TileGeom<D>::kStageBytes;
+    bars = all_bars + warp * STAGES;
+    phase_base = 0;
+    issued = 0;
+    n_my = 0;
+  }
+  // Start a new run of blocks [blk0_, blk1_) of kv head kvh_. The barrier phases
+  // continue from the previous run.
+  __device__ __forceinline__ void start(const int32_t* row, int blk0_, int blk1_, int kvh_) {
+    phase_base += issued;
     blk0 = blk0_;
     kvh = kvh_;
     trow = row;
-    stage_base = smem + warp * STAGES * TileGeom<D>::kStageBytes;
-    bars = all_bars + warp * STAGES;
-    const int span = blk1 - blk0;
+    const int span = blk1_ - blk0_;
     n_my = span > warp ? (span - warp + NW - 1) / NW : 0;
     tbase = 0;
     tchunk = table_entry(lane);
@@ -89,9 +144,9 @@ struct WarpPipe {
   __device__ __forceinline__ uint8_t* kbuf(int s) const {
     return stage_base + s * TileGeom<D>::kStageBytes;
   }
-  __device__ __forceinline__ uint8_t* vbuf(int s) const {
-    return kbuf(s) + TileGeom<D>::kTileBytes;
-  }
+  __device__ __forceinline__ uint8_t* vbuf(int s) const { return kbuf(s) + TileGeom<D>::kTileBytes; }
+  __device__ __forceinline__ int stage_of(int k) const { return (phase_base + k) % STAGES; }
+  __device__ __forceinline__ uint32_t parity_of(int k) const { return ((phase_base + k) / STAGES) & 1; }
   // Called by all lanes, in increasing k.
   __device__ __forceinline__ void issue(int k, const CUtensorMap* tk, const CUtensorMap* tv) {
     if ((k & ~31) != tbase) {
@@ -99,7 +154,7 @@ struct WarpPipe {
       tchunk = table_entry(tbase + lane);
     }
     const int phys = __shfl_sync(kFull, tchunk, k & 31);
-    const int s = k % STAGES;
+    const int s = stage_of(k);
     if (lane == 0) {
       fence_proxy_async_smem();
       uint64_t* bar = &bars[s];
@@ -113,206 +168,73 @@ struct WarpPipe {
     }
     issued = k + 1;
   }
-  // Uniform across the warp: true when stage of block k holds its data.
+  // Uniform across the warp: true when the stage of block k holds its data.
   __device__ __forceinline__ bool wait(int k) {
-    const bool ok = mbar_wait_bounded(&bars[k % STAGES], (k / STAGES) & 1);
+    const bool ok = mbar_wait_bounded(&bars[stage_of(k)], parity_of(k));
     return __all_sync(kFull, ok);
   }
-  // After a timeout: wait (bounded) for every load still in flight.
+  // After a timeout: wait (bounded) for every load still in flight, then stop.
   __device__ __forceinline__ void drain(int from) {
     for (int k = from; k < issued; ++k)
-      if (!mbar_wait_bounded(&bars[k % STAGES], (k / STAGES) & 1)) record_error(kErrTimeoutDrain);
+      if (!mbar_wait_bounded(&bars[stage_of(k)], parity_of(k))) record_error(kErrTimeoutDrain);
     __syncwarp();
   }
 };
 
 // ---------------------------------------------------------------------------
-// Cross-warp combine of (m, l, O) and the final store.
-//   ow:  NW regions of ROWS x OS fp32 (unnormalised O, row r, column d)
-//   ml:  NW x ROWS (m in log2 units, l)
-// One split: out = (sum_w O_w 2^(m_w - M)) / (sum_w l_w 2^(m_w - M)) as bf16.
-// Several splits: the unnormalised sum and (M, L) go to the workspace.
-// ---------------------------------------------------------------------------
-template <int D, int ROWS, int NW>
-__device__ __forceinline__ void cta_combine_store(const DecodeParams& p, const float* ow,
-                                                  const float2* ml, int b, int kvh, int rc,
-                                                  int split, bool single_split) {
-  constexpr int OS = D + 4;
-  constexpr int DC = D / 8;
-  for (int task = threadIdx.x; task < ROWS * DC; task += NW * 32) {
-    const int r = task / DC;
-    const int dc = task % DC;
-    const int rg = rc * p.rows_per_cta + r;
-    if (rg >= p.rows) continue;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[w * ROWS + r].x);
-    float L = 0.f;
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float2 mlw = ml[w * ROWS + r];
-      const float wt = (mlw.x == -INFINITY) ? 0.f : fast_exp2(mlw.x - M);
-      L += wt * mlw.y;
-      const float4* src = reinterpret_cast<const float4*>(ow + (w * ROWS + r) * OS + dc * 8);
-      const float4 x0 = src[0], x1 = src[1];
-      acc[0] += wt * x0.x; acc[1] += wt * x0.y; acc[2] += wt * x0.z; acc[3] += wt * x0.w;
-      acc[4] += wt * x1.x; acc[5] += wt * x1.y; acc[6] += wt * x1.z; acc[7] += wt * x1.w;
-    }
-    const int i = rg / p.group;
-    const int h = kvh * p.group + rg % p.group;
-    const int rq = i * p.num_q_heads + h;
-    if (single_split) {
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      uint4 v;
-      v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-      v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-      const size_t off = ((static_cast<size_t>(b) * p.q_per_seq + i) * p.num_q_heads + h) * D + dc * 8;
-      *reinterpret_cast<uint4*>(p.out + off) = v;
-    } else {
-      const size_t rec = (static_cast<size_t>(b) * p.num_splits + split) * (p.q_per_seq * p.num_q_heads) + rq;
-      float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + dc * 8);
-      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      if (dc == 0) p.ws_ml[rec] = make_float2(M, L);
-    }
-  }
-}
-
-// Rows of a sequence with no visible key at all (context_len 0) get zeros.
-template <int D, int NW>
-__device__ void store_zero_rows(const DecodeParams& p, int b, int kvh, int rc) {
-  constexpr int DC = D / 8;
-  for (int task = threadIdx.x; task < p.rows_per_cta * DC; task += NW * 32) {
-    const int rg = rc * p.rows_per_cta + task / DC;
-    if (rg >= p.rows) continue;
-    const int i = rg / p.group;
-    const int h = kvh * p.group + rg % p.group;
-    const size_t off = ((static_cast<size_t>(b) * p.q_per_seq + i) * p.num_q_heads + h) * D + (task % DC) * 8;
-    *reinterpret_cast<uint4*>(p.out + off) = make_uint4(0, 0, 0, 0);
-  }
-}
-
-template <int D, int ROWS, int NW, int STAGES>
-struct DecodeSmem {
-  static constexpr int kStages = NW * STAGES * TileGeom<D>::kStageBytes;
-  static constexpr int kMerge = NW * ROWS * (D + 4) * 4;
-  static constexpr int kBytes = (kStages > kMerge ? kStages : kMerge) + 1024;  // + alignment slack
-};
-
-// ---------------------------------------------------------------------------
-// Tensor-core decode. Per warp and per 16-token block:
+// Tensor-core core. Per warp and per 16-token block:
 //   S^T[16 tok][8 rows] = K[16 tok][D] . Q^T[D][8 rows]   (A = K via ldmatrix, B = Q regs)
 //   online softmax on S^T in registers (a row's 16 scores sit in 8 lanes)
 //   O^T[D][8 rows] += V^T[D][16 tok] . P^T[16 tok][8 rows] (A = V via ldmatrix.trans,
 //                                                            B = P^T via movmatrix)
-// NT n-tiles of 8 rows: rows = GQA group x query tokens, row r = i * group + g.
+// NT n-tiles of 8 rows; only the first nt_active carry real rows in a segment.
 // ---------------------------------------------------------------------------
-template <int D, int NT, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32)
-decode_tile_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
-                   const __grid_constant__ CUtensorMap tmap_v) {
-  constexpr int ROWS = NT * 8;
-  constexpr int KSTEPS = D / 16;
-  constexpr int OS = D + 4;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bars[NW * STAGES];
-  __shared__ float2 ml_s[NW * ROWS];
-
-  uint8_t* smem = align1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x / p.row_chunks;
-  const int rc = blockIdx.x % p.row_chunks;
-  const int b = blockIdx.y;
-  const int split = blockIdx.z;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NW * STAGES; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_v);
-  }
-  __syncthreads();
-  grid_dependency_wait();  // inputs may be produced by the previous kernel on the stream
-
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = min(max(ctx, 0) + kBlockSize - 1, p.max_blocks * kBlockSize) / kBlockSize;
-  const int blk0 = split * p.split_blocks;
-  if (blk0 >= nblk) {
-    if (split == 0) store_zero_rows<D, NW>(p, b, kvh, rc);
-    grid_launch_dependents();
-    return;
-  }
-  const int blk1 = min(nblk, blk0 + p.split_blocks);
-  const bool single_split = (nblk + p.split_blocks - 1) / p.split_blocks == 1;
-
-  WarpPipe<D, NW, STAGES> pipe;
-  pipe.init(smem, bars, p.block_tables + static_cast<size_t>(b) * p.max_blocks, blk0, blk1, warp,
-            lane, kvh);
-#pragma unroll
-  for (int s = 0; s < STAGES; ++s)
-    if (s < pipe.n_my) pipe.issue(s, &tmap_k, &tmap_v);
-
-  // Q^T fragments (B operand): row n = lane/4, k pairs 2*(lane%4) and +8.
+template <int D, int NT>
+struct TileCore {
+  static constexpr int ROWS = NT * 8;
+  static constexpr int KSTEPS = D / 16;
+  static constexpr bool kNeedsQSmem = false;
   uint32_t qf[NT][KSTEPS][2];
-  int lim[NT][2];  // last visible key position of the thread's two rows per n-tile
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int rg = rc * ROWS + nt * 8 + (lane >> 2);
-    const bool valid = rg < p.rows;
-    const int i = valid ? rg / p.group : 0;
-    const int h = kvh * p.group + (valid ? rg % p.group : 0);
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-        p.query + ((static_cast<size_t>(b) * p.q_per_seq + i) * p.num_q_heads + h) * D);
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      qf[nt][kk][0] = valid ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
-      qf[nt][kk][1] = valid ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = rc * ROWS + nt * 8 + 2 * (lane & 3) + e;
-      lim[nt][e] = r < p.rows ? ctx - p.q_per_seq + r / p.group : ctx - 1;
-    }
-  }
-
-  const float c = p.scale_log2;
+  int lim[NT][2];
   float m_run[NT][2], l_run[NT][2];
   float o[KSTEPS][NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-  }
-#pragma unroll
-  for (int mt = 0; mt < KSTEPS; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+  int nt_active;
 
-  // ldmatrix lane roles
-  const int lm = lane >> 3;         // which 8x8 matrix this lane addresses
-  const int lr = lane & 7;          // row inside it
-  const int k_tok = lr + (lm & 1) * 8, k_chk = lm >> 1;   // K (non-transposed A)
-  const int v_tok = lr + (lm >> 1) * 8, v_chk = lm & 1;   // V (transposed A)
-
-  for (int k = 0; k < pipe.n_my; ++k) {
-    if (!pipe.wait(k)) {
-      if (lane == 0) record_error(kErrTimeoutDecode);
-      pipe.drain(k);
-      break;
+  __device__ __forceinline__ void begin(const DecodeParams& p, const Seg& s, int ctx, int lane) {
+    nt_active = (s.nrows + 7) >> 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      int b = 0, i = 0, h = 0;
+      const bool valid = seg_row(p, s, nt * 8 + (lane >> 2), b, i, h);
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.query + out_offset(p, b, i, h, D));
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        qf[nt][kk][0] = valid ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
+        qf[nt][kk][1] = valid ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool v = seg_row(p, s, nt * 8 + 2 * (lane & 3) + e, b, i, h);
+        lim[nt][e] = v ? ctx - p.q_per_seq + i : ctx - 1;
+      }
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.f;
     }
-    const int s = k % STAGES;
-    const uint32_t kb = smem_u32(pipe.kbuf(s));
-    const uint32_t vb = smem_u32(pipe.vbuf(s));
-    const int tb = (blk0 + warp + NW * k) * kBlockSize;
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+  }
 
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, int tb, bool need_mask,
+                                        float c, int lane, float*) {
+    const uint32_t kb = smem_u32(kt);
+    const uint32_t vb = smem_u32(vt);
+    const int lm = lane >> 3, lr = lane & 7;
+    const int k_tok = lr + (lm & 1) * 8, k_chk = lm >> 1;  // K (non-transposed A)
+    const int v_tok = lr + (lm >> 1) * 8, v_chk = lm & 1;  // V (transposed A)
     float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
@@ -321,16 +243,15 @@ decode_tile_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4(kb + tile_chunk_offset(k_tok, 2 * kk + k_chk), a0, a1, a2, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      for (int nt = 0; nt < NT; ++nt)
+        if (nt < nt_active) mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
     }
-
-    // scores in log2 units, then the causal / end-of-context mask (only blocks
-    // reaching past the first query position need it)
+    // scores in log2 units, then the causal / end-of-context mask
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[nt][e] *= c;
-    if (tb + kBlockSize - 1 > ctx - p.q_per_seq) {
+    if (need_mask) {
       const int t0 = tb + (lane >> 2);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -340,12 +261,14 @@ decode_tile_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
         if (t0 + 8 > lim[nt][1]) sc[nt][3] = -INFINITY;
       }
     }
-
     uint32_t pb[NT][2];
     float alpha[NT][2];
     bool rescale = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+      alpha[nt][0] = alpha[nt][1] = 1.f;
+      pb[nt][0] = pb[nt][1] = 0u;
+      if (nt >= nt_active) continue;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         float mx = fmaxf(sc[nt][e], sc[nt][e + 2]);
@@ -382,167 +305,115 @@ decode_tile_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4_trans(vb + tile_chunk_offset(v_tok, 2 * mt + v_chk), a0, a1, a2, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      for (int nt = 0; nt < NT; ++nt)
+        if (nt < nt_active) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
     }
-    __syncwarp();
-    if (k + STAGES < pipe.n_my) pipe.issue(k + STAGES, &tmap_k, &tmap_v);
   }
 
-  // row sums: a row's partial sums live in the 8 lanes sharing lane % 4
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float l = l_run[nt][e];
-      l += __shfl_xor_sync(kFull, l, 4);
-      l += __shfl_xor_sync(kFull, l, 8);
-      l += __shfl_xor_sync(kFull, l, 16);
-      l_run[nt][e] = l;
-    }
-
-  grid_launch_dependents();
-  __syncthreads();  // every warp is done with its stage buffers
-  float* ow = reinterpret_cast<float*>(smem) + warp * ROWS * OS;
-#pragma unroll
-  for (int mt = 0; mt < KSTEPS; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int r = nt * 8 + 2 * (lane & 3);
-      const int d = mt * 16 + (lane >> 2);
-      ow[r * OS + d] = o[mt][nt][0];
-      ow[(r + 1) * OS + d] = o[mt][nt][1];
-      ow[r * OS + d + 8] = o[mt][nt][2];
-      ow[(r + 1) * OS + d + 8] = o[mt][nt][3];
-    }
-  if (lane < 4) {
+  // Row sums across the 8 lanes of a row, then O and (m, l) of this warp to smem.
+  __device__ __forceinline__ void finish(float* ow, float2* ml, int lane) {
+    constexpr int OS = D + 4;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        ml_s[warp * ROWS + nt * 8 + 2 * lane + e] = make_float2(m_run[nt][e], l_run[nt][e]);
+        float l = l_run[nt][e];
+        l += __shfl_xor_sync(kFull, l, 4);
+        l += __shfl_xor_sync(kFull, l, 8);
+        l += __shfl_xor_sync(kFull, l, 16);
+        l_run[nt][e] = l;
       }
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (nt >= nt_active) continue;
+        const int r = nt * 8 + 2 * (lane & 3);
+        const int d = mt * 16 + (lane >> 2);
+        ow[r * OS + d] = o[mt][nt][0];
+        ow[(r + 1) * OS + d] = o[mt][nt][1];
+        ow[r * OS + d + 8] = o[mt][nt][2];
+        ow[(r + 1) * OS + d + 8] = o[mt][nt][3];
+      }
+    if (lane < 4) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          ml[nt * 8 + 2 * lane + e] = make_float2(m_run[nt][e], l_run[nt][e]);
+    }
   }
-  __syncthreads();
-  cta_combine_store<D, ROWS, NW>(p, reinterpret_cast<const float*>(smem), ml_s, b, kvh, rc, split,
-                                 single_split);
-}
+};
 
 // ---------------------------------------------------------------------------
-// CUDA-core decode. Per warp and per 16-token block:
-//   QK^T: lane (t = lane/2, half = lane%2) dots token t with every row over its
-//         half of head_dim (fp32 FMA), the two halves are joined by one shuffle;
+// CUDA-core core. Per warp and per 16-token block:
+//   QK^T: lane (t = lane/2, half = lane%2) dots token t with every row over its half
+//         of head_dim (fp32 FMA); the two halves are joined by one shuffle;
 //   online softmax: row max over the 16 tokens by 4 xor-shuffles;
-//   PV:   lane owns D/32 output columns; p broadcast through shared memory.
-// ROWS query rows (GQA group x query tokens) per CTA, Q held in shared memory.
+//   PV:   lane owns D/32 output columns; p is broadcast through shared memory.
+// Q of the segment's rows is staged in shared memory as fp32 by the whole CTA.
 // ---------------------------------------------------------------------------
-template <int D, int ROWS, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32)
-decode_single_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v) {
-  constexpr int OS = D + 4;
-  constexpr int CPL = D / 16;  // 16-byte chunks of a row each lane of a pair covers
-  constexpr int DPL = D / 32;  // output columns per lane
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bars[NW * STAGES];
-  __shared__ float2 ml_s[NW * ROWS];
-  __shared__ __align__(16) float q_s[ROWS][D];
-  __shared__ __align__(16) float p_s[NW][16][ROWS];
-
-  uint8_t* smem = align1024(smem_raw);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x / p.row_chunks;
-  const int rc = blockIdx.x % p.row_chunks;
-  const int b = blockIdx.y;
-  const int split = blockIdx.z;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NW * STAGES; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_v);
-  }
-  __syncthreads();
-  grid_dependency_wait();
-
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = min(max(ctx, 0) + kBlockSize - 1, p.max_blocks * kBlockSize) / kBlockSize;
-  const int blk0 = split * p.split_blocks;
-  if (blk0 >= nblk) {
-    if (split == 0) store_zero_rows<D, NW>(p, b, kvh, rc);
-    grid_launch_dependents();
-    return;
-  }
-  const int blk1 = min(nblk, blk0 + p.split_blocks);
-  const bool single_split = (nblk + p.split_blocks - 1) / p.split_blocks == 1;
-
-  WarpPipe<D, NW, STAGES> pipe;
-  pipe.init(smem, bars, p.block_tables + static_cast<size_t>(b) * p.max_blocks, blk0, blk1, warp,
-            lane, kvh);
-#pragma unroll
-  for (int s = 0; s < STAGES; ++s)
-    if (s < pipe.n_my) pipe.issue(s, &tmap_k, &tmap_v);
-
-  for (int idx = threadIdx.x; idx < ROWS * D / 2; idx += NW * 32) {
-    const int r = idx / (D / 2);
-    const int d2 = idx % (D / 2);
-    const int rg = rc * ROWS + r;
-    float lo = 0.f, hi = 0.f;
-    if (rg < p.rows) {
-      const int h = kvh * p.group + rg % p.group;
-      const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(
-          p.query + ((static_cast<size_t>(b) * p.q_per_seq + rg / p.group) * p.num_q_heads + h) * D) + d2);
-      lo = bf16_lo(v);
-      hi = bf16_hi(v);
-    }
-    q_s[r][2 * d2] = lo;
-    q_s[r][2 * d2 + 1] = hi;
-  }
-  int lim[ROWS];
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    const int rg = rc * ROWS + r;
-    lim[r] = rg < p.rows ? ctx - p.q_per_seq + rg / p.group : ctx - 1;
-  }
-  __syncthreads();
-
-  const float c = p.scale_log2;
+template <int D, int ROWS_>
+struct SimtCore {
+  static constexpr int ROWS = ROWS_;
+  static constexpr int CPL = D / 16;  // 16-byte chunks of a row each lane of a pair covers
+  static constexpr int DPL = D / 32;  // output columns per lane
+  static constexpr bool kNeedsQSmem = true;
   float m_run[ROWS], l_run[ROWS], o[ROWS][DPL];
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    m_run[r] = -INFINITY;
-    l_run[r] = 0.f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) o[r][e] = 0.f;
-  }
-  const int t_me = lane >> 1;   // token of this lane for QK^T
-  const int half = lane & 1;
-  // PV: columns [lane*DPL, lane*DPL + DPL) -> chunk and byte offset inside it
-  const int pv_chunk = (lane * DPL) / 8;
-  const int pv_byte = ((lane * DPL) % 8) * 2;
+  int lim[ROWS];
+  const float (*q_s)[D];
+  float* p_w;  // this warp's [16][ROWS] probabilities
 
-  for (int k = 0; k < pipe.n_my; ++k) {
-    if (!pipe.wait(k)) {
-      if (lane == 0) record_error(kErrTimeoutDecode);
-      pipe.drain(k);
-      break;
+  // All threads of the CTA; a __syncthreads() must follow.
+  static __device__ __forceinline__ void stage_q(const DecodeParams& p, const Seg& s, float (*qs)[D],
+                                                 int nthreads) {
+    for (int idx = threadIdx.x; idx < ROWS * D / 2; idx += nthreads) {
+      const int r = idx / (D / 2);
+      const int d2 = idx % (D / 2);
+      int b, i, h;
+      float lo = 0.f, hi = 0.f;
+      if (seg_row(p, s, r, b, i, h)) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p.query + out_offset(p, b, i, h, D)) + d2);
+        lo = bf16_lo(v);
+        hi = bf16_hi(v);
+      }
+      qs[r][2 * d2] = lo;
+      qs[r][2 * d2 + 1] = hi;
     }
-    const int s = k % STAGES;
-    const uint8_t* kt = pipe.kbuf(s);
-    const uint8_t* vt = pipe.vbuf(s);
-    const int tb = (blk0 + warp + NW * k) * kBlockSize;
+  }
 
+  __device__ __forceinline__ void bind(const float (*qs)[D], float* pw) {
+    q_s = qs;
+    p_w = pw;
+  }
+
+  __device__ __forceinline__ void begin(const DecodeParams& p, const Seg& s, int ctx, int) {
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      int b, i, h;
+      lim[r] = seg_row(p, s, r, b, i, h) ? ctx - p.q_per_seq + i : ctx - 1;
+      m_run[r] = -INFINITY;
+      l_run[r] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[r][e] = 0.f;
+    }
+  }
+
+  __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, int tb, bool need_mask,
+                                        float c, int lane, float*) {
+    const int t_me = lane >> 1;
+    const int half = lane & 1;
     float sc[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) sc[r] = 0.f;
 #pragma unroll
     for (int ci = 0; ci < CPL; ++ci) {
-      // the two lanes of a pair start half a row apart and walk the 8 chunk
-      // positions in a rotated order so that they never share a bank group
+      // the two lanes of a pair start half a row apart and walk the chunk positions in
+      // a rotated order so that they never share a bank group
       const int cc = half * CPL + (ci ^ (half * (CPL / 2)));
       const uint4 kv = *reinterpret_cast<const uint4*>(kt + tile_chunk_offset(t_me, cc));
-      float kf[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
-                     bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
+      const float kf[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
+                           bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
         const float4 q0 = *reinterpret_cast<const float4*>(&q_s[r][cc * 8]);
@@ -555,13 +426,12 @@ decode_single_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap t
       }
     }
     const int t_glob = tb + t_me;
-    const bool masked_blk = tb + kBlockSize - 1 > ctx - p.q_per_seq;
     bool rescale = false;
     float alpha[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       float sv = (sc[r] + __shfl_xor_sync(kFull, sc[r], 1)) * c;  // log2 units
-      if (masked_blk && t_glob > lim[r]) sv = -INFINITY;
+      if (need_mask && t_glob > lim[r]) sv = -INFINITY;
       float mx = sv;
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
@@ -574,7 +444,7 @@ decode_single_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap t
       const float pr = fast_exp2(sv - m_use);
       l_run[r] = fmaf(l_run[r], alpha[r], half == 0 ? pr : 0.f);
       m_run[r] = m_new;
-      if (half == 0) p_s[warp][t_me][r] = pr;
+      if (half == 0) p_w[t_me * ROWS + r] = pr;
     }
     if (rescale) {  // m_run is warp-uniform, so is alpha
 #pragma unroll
@@ -583,6 +453,8 @@ decode_single_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap t
         for (int e = 0; e < DPL; ++e) o[r][e] *= alpha[r];
     }
     __syncwarp();
+    const int pv_chunk = (lane * DPL) / 8;
+    const int pv_byte = ((lane * DPL) % 8) * 2;
 #pragma unroll 4
     for (int t = 0; t < kBlockSize; ++t) {
       const uint8_t* vrow = vt + tile_chunk_offset(t, pv_chunk) + pv_byte;
@@ -596,43 +468,579 @@ decode_single_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap t
       }
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
-        const float pr = p_s[warp][t][r];
+        const float pr = p_w[t * ROWS + r];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[r][e] = fmaf(pr, vf[e], o[r][e]);
       }
     }
     __syncwarp();
-    if (k + STAGES < pipe.n_my) pipe.issue(k + STAGES, &tmap_k, &tmap_v);
   }
 
+  __device__ __forceinline__ void finish(float* ow, float2* ml, int lane) {
+    constexpr int OS = D + 4;
 #pragma unroll
-  for (int r = 0; r < ROWS; ++r) {
-    float l = l_run[r];
+    for (int r = 0; r < ROWS; ++r) {
+      float l = l_run[r];
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(kFull, l, off);
-    l_run[r] = l;
-  }
-  grid_launch_dependents();
-  __syncthreads();
-  float* ow = reinterpret_cast<float*>(smem) + warp * ROWS * OS;
-#pragma unroll
-  for (int r = 0; r < ROWS; ++r)
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) ow[r * OS + lane * DPL + e] = o[r][e];
-  if (lane == 0) {
+      for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(kFull, l, off);
+      l_run[r] = l;
+    }
 #pragma unroll
     for (int r = 0; r < ROWS; ++r)
-      ml_s[warp * ROWS + r] = make_float2(m_run[r], l_run[r]);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) ow[r * OS + lane * DPL + e] = o[r][e];
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) ml[r] = make_float2(m_run[r], l_run[r]);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Shared memory of a decode CTA and the per-segment driver.
+// ---------------------------------------------------------------------------
+template <int D, int ROWS, int NW, int STAGES>
+struct DecodeSmem {
+  static constexpr int kStages = NW * STAGES * TileGeom<D>::kStageBytes;
+  static constexpr int kMerge = NW * ROWS * (D + 4) * 4;
+  static constexpr int kBytes = (kStages > kMerge ? kStages : kMerge) + 1024;  // + alignment slack
+};
+
+// Static shared state; the q / p staging areas exist for the CUDA-core core only.
+template <int D, int ROWS, int NW, int STAGES, bool kQ>
+struct CtaState {
+  uint64_t bars[NW * STAGES];
+  float2 ml[NW * ROWS];
+  int slot[kTileMaxRows];
+  int last[kTileMaxRows];
+  __align__(16) float q_s[kQ ? ROWS : 1][D];
+  __align__(16) float p_s[NW][kQ ? 16 * ROWS : 1];
+};
+
+// Run one segment through the warps' pipelines; on return every warp's (m, l, O)
+// sits in shared memory (ow: NW x ROWS x (D+4) fp32 over the stage buffers; st.ml).
+template <class Core, int D, int NW, int STAGES, class State>
+__device__ __forceinline__ void run_segment(const DecodeParams& p, const Seg& sg, int ctx,
+                                            WarpPipe<D, NW, STAGES>& pipe, Core& core, State& st,
+                                            uint8_t* smem, const CUtensorMap* tk,
+                                            const CUtensorMap* tv, int warp, int lane) {
+  constexpr int OS = D + 4;
+  const int32_t* trow = p.block_tables + static_cast<size_t>(sg.b0) * p.max_blocks;
+  pipe.start(trow, sg.blk0, sg.blk1, sg.kvh);
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s)
+    if (s < pipe.n_my) pipe.issue(s, tk, tv);
+  if constexpr (Core::kNeedsQSmem) {
+    Core::stage_q(p, sg, st.q_s, NW * 32);
+    core.bind(st.q_s, st.p_s[warp]);
+    __syncthreads();
+  }
+  core.begin(p, sg, ctx, lane);
+  const float c = p.scale_log2;
+  const int first_masked = ctx - p.q_per_seq;  // blocks ending past this position need the mask
+  for (int k = 0; k < pipe.n_my; ++k) {
+    if (!pipe.wait(k)) {
+      if (lane == 0) record_error(kErrTimeoutDecode);
+      pipe.drain(k);
+      break;
+    }
+    const int s = pipe.stage_of(k);
+    const int tb = (sg.blk0 + warp + NW * k) * kBlockSize;
+    const bool need_mask = !sg.shared && tb + kBlockSize - 1 > first_masked;
+    core.block(pipe.kbuf(s), pipe.vbuf(s), tb, need_mask, c, lane, nullptr);
+    __syncwarp();
+    if (k + STAGES < pipe.n_my) pipe.issue(k + STAGES, tk, tv);
+  }
+  __syncthreads();  // every warp is done with its stage buffers
+  core.finish(reinterpret_cast<float*>(smem) + warp * Core::ROWS * OS, st.ml + warp * Core::ROWS, lane);
+  __syncthreads();
+}
+
+// Cross-warp combine of local row r, 8 output columns starting at dc*8:
+// M = max_w m_w, L = sum_w l_w 2^(m_w - M), acc = sum_w O_w 2^(m_w - M).
+template <int D, int ROWS, int NW>
+__device__ __forceinline__ void combine_row(const float* ow, const float2* ml, int r, int dc, float& M,
+                                            float& L, float (&acc)[8]) {
+  constexpr int OS = D + 4;
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) M = fmaxf(M, ml[w * ROWS + r].x);
+  L = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const float2 mlw = ml[w * ROWS + r];
+    const float wt = (mlw.x == -INFINITY) ? 0.f : fast_exp2(mlw.x - M);
+    L += wt * mlw.y;
+    const float4* src = reinterpret_cast<const float4*>(ow + (w * ROWS + r) * OS + dc * 8);
+    const float4 x0 = src[0], x1 = src[1];
+    acc[0] += wt * x0.x; acc[1] += wt * x0.y; acc[2] += wt * x0.z; acc[3] += wt * x0.w;
+    acc[4] += wt * x1.x; acc[5] += wt * x1.y; acc[6] += wt * x1.z; acc[7] += wt * x1.w;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x8(uint16_t* dst, const float (&acc)[8], float inv) {
+  uint4 v;
+  v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(dst) = v;
+}
+
+template <int NW, int STAGES>
+__device__ __forceinline__ void init_cta(uint64_t* bars, const CUtensorMap* tk, const CUtensorMap* tv) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NW * STAGES; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(tk);
+    tma_prefetch_desc(tv);
   }
   __syncthreads();
-  cta_combine_store<D, ROWS, NW>(p, reinterpret_cast<const float*>(smem), ml_s, b, kvh, rc, split,
-                                 single_split);
 }
 
 // ---------------------------------------------------------------------------
-// Log-sum-exp merge of split partials: one warp per (sequence, query token, head).
-// M = max_s m_s, L = sum_s l_s 2^(m_s - M), out = sum_s o_s 2^(m_s - M) / L.
+// Persistent decode. CTA c covers work units [c*W/P, (c+1)*W/P) of the flattened
+// list the pre-pass built: per sequence b, its shared-prefix band (leaders only:
+// H_kv sub-units of P_b blocks, rows = members x rows) then its private band
+// (H_kv x row_chunks sub-units of nblk_b - P_b blocks). A sub-unit cut by the CTA
+// range, or a target that also has a shared part, is completed through partial
+// records: each piece adds its block count to the target's arrival counter and the
+// piece that brings it to nblk merges all of the target's records.
 // ---------------------------------------------------------------------------
+template <class Core, int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32)
+decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v) {
+  constexpr int ROWS = Core::ROWS;
+  constexpr int DC = D / 8;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ CtaState<D, ROWS, NW, STAGES, Core::kNeedsQSmem> st;
+  uint8_t* smem = align1024(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  init_cta<NW, STAGES>(st.bars, &tmap_k, &tmap_v);
+  grid_dependency_wait();  // the pre-pass (and anything before it) has completed
+
+  const long long W = __ldcg(&p.hdr->work);
+  const long long pos_end = W * (blockIdx.x + 1) / gridDim.x;
+  long long pos = W * blockIdx.x / gridDim.x;
+  if (pos >= pos_end) {
+    grid_launch_dependents();
+    return;
+  }
+  WarpPipe<D, NW, STAGES> pipe;
+  pipe.init(smem, st.bars, warp, lane);
+  Core core;
+  const int H = p.num_kv_heads;
+  const int RC = p.row_chunks;
+  int b = __ldcg(p.cta_seq + blockIdx.x);
+  if (b < 0 || b >= p.num_seqs) {  // inconsistent schedule tables
+    record_error(kErrSchedule);
+    grid_launch_dependents();
+    return;
+  }
+  while (pos < pos_end && b < p.num_seqs) {
+    const long long base = __ldcg(p.seq_start + b);
+    const int4 info = __ldcg(p.seq_info + b);
+    const int P_b = info.x, members = info.y, nblk = info.z;
+    const long long sh_work = members > 0 ? static_cast<long long>(H) * P_b : 0;
+    const int pv_len = nblk - P_b;
+    const long long pv_work = static_cast<long long>(H) * RC * pv_len;
+    if (pos >= base + sh_work + pv_work) {
+      ++b;
+      continue;
+    }
+    Seg sg;
+    int rc = 0;
+    long long len;
+    if (pos < base + sh_work) {
+      const long long off = pos - base;
+      const int kvh = static_cast<int>(off / P_b);
+      const int j = static_cast<int>(off - static_cast<long long>(kvh) * P_b);
+      len = min(pos_end - pos, static_cast<long long>(P_b - j));
+      sg = Seg{b, members, kvh, 0, members * p.rows, j, j + static_cast<int>(len), true};
+    } else {
+      const long long off = pos - base - sh_work;
+      const int sub = static_cast<int>(off / pv_len);
+      const int jo = static_cast<int>(off - static_cast<long long>(sub) * pv_len);
+      rc = sub % RC;
+      const int kvh = sub / RC;
+      len = min(pos_end - pos, static_cast<long long>(pv_len - jo));
+      sg = Seg{b, 1, kvh, rc * ROWS, min(ROWS, p.rows - rc * ROWS), P_b + jo,
+               P_b + jo + static_cast<int>(len), false};
+    }
+    if (len <= 0) {  // cannot happen with consistent tables; never loop forever
+      if (threadIdx.x == 0) record_error(kErrSchedule);
+      break;
+    }
+    const int ctx = __ldg(p.context_lens + b);
+    run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
+    const float* ow = reinterpret_cast<const float*>(smem);
+
+    const bool direct = !sg.shared && P_b == 0 && sg.blk0 == 0 && sg.blk1 == nblk;
+    if (direct) {
+      for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+        const int r = task / DC, dc = task % DC;
+        float M, L, acc[8];
+        combine_row<D, ROWS, NW>(ow, st.ml, r, dc, M, L, acc);
+        int bb, i, h;
+        seg_row(p, sg, r, bb, i, h);
+        store_bf16x8(p.out + out_offset(p, bb, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
+      }
+    } else {
+      // one partial record per output target (sequence, kv head, row chunk) touched
+      const int tr = p.target_rows;
+      if (threadIdx.x < sg.members) {
+        int slot = atomicAdd(&p.hdr->pool, 1);
+        if (slot >= p.pool_cap) {
+          record_error(kErrRecordPool);
+          slot = -1;
+        }
+        st.slot[threadIdx.x] = slot;
+      }
+      __syncthreads();
+      for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+        const int r = task / DC, dc = task % DC;
+        const int m = sg.shared ? r / p.rows : 0;
+        const int rr = sg.shared ? r - m * p.rows : r;  // row inside the target
+        const int slot = st.slot[m];
+        if (slot < 0) continue;
+        float M, L, acc[8];
+        combine_row<D, ROWS, NW>(ow, st.ml, r, dc, M, L, acc);
+        float* rec = p.records + static_cast<size_t>(slot) * p.rec_stride;
+        float4* dst = reinterpret_cast<float4*>(rec + rr * D + dc * 8);
+        __stcg(dst, make_float4(acc[0], acc[1], acc[2], acc[3]));
+        __stcg(dst + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
+        if (dc == 0) __stcg(reinterpret_cast<float2*>(rec + tr * D) + rr, make_float2(M, L));
+      }
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x < sg.members) {
+        const int bm = sg.b0 + threadIdx.x;
+        const int t = (bm * H + sg.kvh) * RC + rc;
+        const int slot = st.slot[threadIdx.x];
+        if (slot >= 0) {
+          const int idx = atomicAdd(p.list_len + t, 1);
+          if (idx < p.list_cap) {
+            p.list[static_cast<size_t>(t) * p.list_cap + idx] = slot;
+          } else {
+            record_error(kErrRecordList);
+          }
+        }
+        __threadfence();
+        const int nb_m = num_blocks_of(p, __ldg(p.context_lens + bm));
+        const int prev = atomicAdd(p.arrive + t, static_cast<int>(len));
+        st.last[threadIdx.x] = (prev + static_cast<int>(len) == nb_m) ? 1 : 0;
+      }
+      __syncthreads();
+      for (int m = 0; m < sg.members; ++m) {
+        if (!st.last[m]) continue;  // uniform: shared memory flag
+        __threadfence();
+        const int bm = sg.b0 + m;
+        const int t = (bm * H + sg.kvh) * RC + rc;
+        const int n = min(__ldcg(p.list_len + t), p.list_cap);
+        const int* lst = p.list + static_cast<size_t>(t) * p.list_cap;
+        const int rows_t = min(tr, p.rows - rc * ROWS);
+        for (int task = threadIdx.x; task < rows_t * DC; task += NW * 32) {
+          const int rr = task / DC, dc = task % DC;
+          float M = -INFINITY;
+          for (int k = 0; k < n; ++k) {
+            const float* rec = p.records + static_cast<size_t>(__ldcg(lst + k)) * p.rec_stride;
+            M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(rec + tr * D) + rr).x);
+          }
+          float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int k = 0; k < n; ++k) {
+            const float* rec = p.records + static_cast<size_t>(__ldcg(lst + k)) * p.rec_stride;
+            const float2 mlk = __ldcg(reinterpret_cast<const float2*>(rec + tr * D) + rr);
+            const float wt = (mlk.x == -INFINITY) ? 0.f : fast_exp2(mlk.x - M);
+            L += wt * mlk.y;
+            const float4* src = reinterpret_cast<const float4*>(rec + rr * D + dc * 8);
+            const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+            acc[0] += wt * x0.x; acc[1] += wt * x0.y; acc[2] += wt * x0.z; acc[3] += wt * x0.w;
+            acc[4] += wt * x1.x; acc[5] += wt * x1.y; acc[6] += wt * x1.z; acc[7] += wt * x1.w;
+          }
+          const int rg = rc * ROWS + rr;
+          const int i = rg / p.group;
+          const int h = sg.kvh * p.group + (rg - i * p.group);
+          store_bf16x8(p.out + out_offset(p, bm, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
+        }
+      }
+    }
+    __syncthreads();  // shared memory is reused by the next segment
+    pos += len;
+  }
+  grid_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
+// Pre-pass of the persistent schedule (one CTA of kPrepassThreads threads).
+//   1. per sequence: nblk; with prefix sharing on, groups = maximal runs of adjacent
+//      sequences whose first block is the same physical block, cut into chunks of
+//      share_cap members; a chunk's shared prefix P = the leading blocks identical in
+//      all members' tables, limited to blocks every member's query rows fully see.
+//   2. work(b) = [leader: H_kv * P] + H_kv * row_chunks * (nblk - P_b); exclusive scan
+//      -> seq_start; W = total; CTA c starts in the sequence holding unit c*W/P.
+//   3. zero the arrival counters and record lists; zero outputs of empty sequences.
+// ---------------------------------------------------------------------------
+constexpr int kPrepassThreads = 1024;
+
+__device__ __forceinline__ long long block_exclusive_scan(long long v, long long* warp_tot,
+                                                          long long& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long y = __shfl_up_sync(kFull, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < kPrepassThreads / 32 ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(kFull, w, off);
+      if (lane >= off) w += y;
+    }
+    warp_tot[lane] = w;  // inclusive prefix over warps
+  }
+  __syncthreads();
+  const long long before = (warp > 0 ? warp_tot[warp - 1] : 0) + x - v;
+  total = warp_tot[kPrepassThreads / 32 - 1];
+  __syncthreads();
+  return before;
+}
+
+// True when sequence b does not continue the shared group of b - 1.
+__device__ __forceinline__ bool group_start(const DecodeParams& p, int b) {
+  if (b == 0) return true;
+  if (num_blocks_of(p, __ldg(p.context_lens + b)) == 0 ||
+      num_blocks_of(p, __ldg(p.context_lens + b - 1)) == 0)
+    return true;
+  return __ldg(p.block_tables + static_cast<size_t>(b) * p.max_blocks) !=
+         __ldg(p.block_tables + static_cast<size_t>(b - 1) * p.max_blocks);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const DecodeParams p) {
+  __shared__ long long warp_tot[kPrepassThreads / 32];
+  __shared__ int wmax[kPrepassThreads / 32];
+  __shared__ int s_g0carry;
+  __shared__ int s_lead[kPrepassThreads];  // leaders of this chunk with a possible shared prefix
+  __shared__ int s_pmax[kPrepassThreads];
+  __shared__ int s_mem[kPrepassThreads];
+  __shared__ int s_bad[kPrepassThreads];
+  __shared__ int s_nlead;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int B = p.num_seqs;
+  const int H = p.num_kv_heads;
+  const int RC = p.row_chunks;
+  const int cap = p.share_cap;
+  constexpr int T = kPrepassThreads;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // ---- pass 1: sharing, P_b, work(b) (kept in seq_start for now), W
+  if (threadIdx.x == 0) s_g0carry = 0;
+  __syncthreads();
+  long long W = 0;
+  for (int c0 = 0; c0 < B; c0 += T) {
+    const int b = c0 + threadIdx.x;
+    const bool in = b < B;
+    const int ctx = in ? __ldg(p.context_lens + b) : 0;
+    const int nblk = in ? num_blocks_of(p, ctx) : 0;
+    int g0 = 0;
+    if (cap >= 2) {
+      // first sequence of b's group: inclusive max-scan of group start positions
+      int v = (in && group_start(p, b)) ? b : -1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(kFull, v, off);
+        if (lane >= off) v = max(v, y);
+      }
+      if (lane == 31) wmax[warp] = v;
+      if (threadIdx.x == 0) s_nlead = 0;
+      __syncthreads();
+      int before = s_g0carry;
+      for (int w = 0; w < warp; ++w) before = max(before, wmax[w]);
+      g0 = max(v, before);
+      __syncthreads();
+      if (threadIdx.x == T - 1) s_g0carry = g0;
+      // chunk leaders: members, and the blocks every member's rows fully see
+      if (in && (b - g0) % cap == 0) {
+        int mem = 1;
+        int pmax = (ctx - p.q_per_seq + 1) / kBlockSize;
+        while (mem < cap && b + mem < B && !group_start(p, b + mem)) {
+          pmax = min(pmax, (__ldg(p.context_lens + b + mem) - p.q_per_seq + 1) / kBlockSize);
+          ++mem;
+        }
+        pmax = max(0, min(pmax, nblk));
+        if (mem > 1 && pmax > 0) {
+          const int k = atomicAdd(&s_nlead, 1);
+          s_lead[k] = b;
+          s_pmax[k] = pmax;
+          s_mem[k] = mem;
+          s_bad[k] = pmax;
+        } else {
+          p.seq_info[b] = make_int4(0, 0, nblk, 0);
+        }
+      }
+      __syncthreads();
+      // longest common table prefix: warps take (leader, 32-block window) pairs
+      const int nlead = s_nlead;
+      int npairs = 0;
+      for (int k = 0; k < nlead; ++k) npairs += (s_pmax[k] + 31) / 32;
+      for (int pr = warp; pr < npairs; pr += T / 32) {
+        int k = 0, rem = pr;
+        while (rem >= (s_pmax[k] + 31) / 32) {
+          rem -= (s_pmax[k] + 31) / 32;
+          ++k;
+        }
+        const int j = rem * 32 + lane;
+        bool ok = true;
+        if (j < s_pmax[k]) {
+          const int32_t* t0 = p.block_tables + static_cast<size_t>(s_lead[k]) * p.max_blocks;
+          const int ref = __ldg(t0 + j);
+          for (int m = 1; m < s_mem[k]; ++m) ok &= __ldg(t0 + static_cast<size_t>(m) * p.max_blocks + j) == ref;
+        }
+        const unsigned badmask = __ballot_sync(kFull, !ok);
+        if (badmask && lane == 0) atomicMin(&s_bad[k], rem * 32 + __ffs(badmask) - 1);
+      }
+      __syncthreads();
+      for (int k = threadIdx.x; k < nlead; k += T) {
+        const int P = s_bad[k];
+        p.seq_info[s_lead[k]] = make_int4(P, P > 0 ? s_mem[k] : 0,
+                                          num_blocks_of(p, __ldg(p.context_lens + s_lead[k])), 0);
+      }
+    }
+    __syncthreads();
+    int P_b = 0, lead_members = 0;
+    if (in && cap >= 2) {
+      const int leader = g0 + ((b - g0) / cap) * cap;
+      const int4 li = p.seq_info[leader];
+      if (li.y > 0) P_b = li.x;  // the chunk has a shared unit
+      if (leader == b) lead_members = li.y;
+    }
+    __syncthreads();  // every leader entry is read before any is rewritten
+    long long work = 0;
+    if (in) {
+      p.seq_info[b] = make_int4(P_b, lead_members, nblk, 0);
+      work = (lead_members > 0 ? static_cast<long long>(H) * P_b : 0) +
+             static_cast<long long>(H) * RC * (nblk - P_b);
+      p.seq_start[b] = work;
+    }
+    long long tot;
+    block_exclusive_scan(work, warp_tot, tot);
+    W += tot;
+  }
+  __syncthreads();
+
+  // ---- pass 2: starts, CTA assignment, counters
+  const long long P = p.num_ctas;
+  long long carry = 0;
+  for (int c0 = 0; c0 < B; c0 += T) {
+    const int b = c0 + threadIdx.x;
+    const long long work = b < B ? p.seq_start[b] : 0;
+    long long tot;
+    const long long start = carry + block_exclusive_scan(work, warp_tot, tot);
+    if (b < B) {
+      p.seq_start[b] = start;
+      if (W > 0 && work > 0) {
+        const long long c_lo = (start * P + W - 1) / W;
+        const long long c_hi = min(P, ((start + work) * P + W - 1) / W);
+        for (long long c = c_lo; c < c_hi; ++c) p.cta_seq[c] = b;
+      }
+    }
+    carry += tot;
+  }
+  const int targets = B * H * RC;
+  for (int t = threadIdx.x; t < targets; t += T) {
+    p.arrive[t] = 0;
+    p.list_len[t] = 0;
+  }
+  // sequences without any block: outputs are zero
+  for (int b = warp; b < B; b += T / 32) {
+    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;
+    uint16_t* dst = p.out + static_cast<size_t>(b) * p.q_per_seq * p.num_q_heads * D;
+    for (int e = lane; e < p.q_per_seq * p.num_q_heads * D / 8; e += 32)
+      reinterpret_cast<uint4*>(dst)[e] = make_uint4(0, 0, 0, 0);
+  }
+  if (threadIdx.x == 0) {
+    p.hdr->work = W;
+    p.hdr->pool = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Grid decode: one CTA per (kv head x row chunk, sequence, split of split_blocks
+// blocks). A sequence with one split writes bf16 directly; otherwise each split
+// writes fp32 partials (o, m, l) for merge_kernel.
+// ---------------------------------------------------------------------------
+template <class Core, int D, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32)
+decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v) {
+  constexpr int ROWS = Core::ROWS;
+  constexpr int DC = D / 8;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ CtaState<D, ROWS, NW, STAGES, Core::kNeedsQSmem> st;
+  uint8_t* smem = align1024(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kvh = blockIdx.x / p.row_chunks;
+  const int rc = blockIdx.x % p.row_chunks;
+  const int b = blockIdx.y;
+  const int split = blockIdx.z;
+  init_cta<NW, STAGES>(st.bars, &tmap_k, &tmap_v);
+  grid_dependency_wait();  // inputs may be produced by the previous kernel on the stream
+
+  const int ctx = __ldg(p.context_lens + b);
+  const int nblk = num_blocks_of(p, ctx);
+  const int blk0 = split * p.split_blocks;
+  Seg sg{b, 1, kvh, rc * ROWS, min(ROWS, p.rows - rc * ROWS), 0, 0, false};
+  if (blk0 >= nblk) {
+    if (split == 0) {  // no block at all: zero output
+      for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+        int bb, i, h;
+        seg_row(p, sg, task / DC, bb, i, h);
+        *reinterpret_cast<uint4*>(p.out + out_offset(p, bb, i, h, D) + (task % DC) * 8) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    grid_launch_dependents();
+    return;
+  }
+  sg.blk0 = blk0;
+  sg.blk1 = min(nblk, blk0 + p.split_blocks);
+  const bool single_split = (nblk + p.split_blocks - 1) / p.split_blocks == 1;
+  WarpPipe<D, NW, STAGES> pipe;
+  pipe.init(smem, st.bars, warp, lane);
+  Core core;
+  run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
+  grid_launch_dependents();
+  const float* ow = reinterpret_cast<const float*>(smem);
+  for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+    const int r = task / DC, dc = task % DC;
+    float M, L, acc[8];
+    combine_row<D, ROWS, NW>(ow, st.ml, r, dc, M, L, acc);
+    int bb, i, h;
+    seg_row(p, sg, r, bb, i, h);
+    if (single_split) {
+      store_bf16x8(p.out + out_offset(p, bb, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
+    } else {
+      const int rq = i * p.num_q_heads + h;
+      const size_t rec = (static_cast<size_t>(b) * p.num_splits + split) * (p.q_per_seq * p.num_q_heads) + rq;
+      float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + dc * 8);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      if (dc == 0) p.ws_ml[rec] = make_float2(M, L);
+    }
+  }
+}
+
+// Log-sum-exp merge of the grid schedule's split partials: one warp per (sequence,
+// query token, head).
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
   constexpr int DPL = D / 32;
@@ -643,16 +1051,19 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
   if (row >= p.num_seqs * RQ) return;
   const int b = row / RQ;
   const int rq = row % RQ;
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = min(max(ctx, 0) + kBlockSize - 1, p.max_blocks * kBlockSize) / kBlockSize;
+  const int nblk = num_blocks_of(p, __ldg(p.context_lens + b));
   const int ns = (nblk + p.split_blocks - 1) / p.split_blocks;
   if (ns <= 1) return;  // written directly by the decode kernel
   const size_t base = static_cast<size_t>(b) * p.num_splits * RQ + rq;
+  // (m, l) of split s in lane s % 32: independent loads, then a warp reduction
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, p.ws_ml[base + static_cast<size_t>(s) * RQ].x);
+  for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.ws_ml[base + static_cast<size_t>(s) * RQ].x);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
   float L = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
   for (int s = 0; s < ns; ++s) {
     const size_t rec = base + static_cast<size_t>(s) * RQ;
     const float2 ml = p.ws_ml[rec];
@@ -670,7 +1081,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const int i = rq / p.num_q_heads;
   const int h = rq % p.num_q_heads;
-  uint16_t* dst = p.out + ((static_cast<size_t>(b) * p.q_per_seq + i) * p.num_q_heads + h) * D + lane * DPL;
+  uint16_t* dst = p.out + out_offset(p, b, i, h, D) + lane * DPL;
   if constexpr (DPL == 4) {
     *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
                                                 pack_bf16x2(acc[2] * inv, acc[3] * inv));
@@ -737,9 +1148,9 @@ __device__ unsigned long long g_validate_count = 0;
 // ---------------------------------------------------------------------------
 namespace {
 
-template <typename Kernel>
+template <typename Kernel, typename... Args>
 cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv) {
+                       Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -750,11 +1161,8 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p, tk, tv);
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
-
-template <int D, int NT>
-constexpr int tile_stages() { return 2; }
 
 // Opt a kernel into its dynamic shared memory size once per device. `done_mask`
 // (bit d: done on device d) must be owned by the kernel instance itself.
@@ -770,86 +1178,70 @@ cudaError_t configure_smem(Kernel kernel, int smem, unsigned long long& done_mas
   return e;
 }
 
-template <int D, int NT>
-cudaError_t launch_tile(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                        cudaStream_t stream, int* occupancy) {
-  constexpr int ST = tile_stages<D, NT>();
-  constexpr int smem = DecodeSmem<D, NT * 8, kWarpsPerCta, ST>::kBytes;
-  auto kernel = decode_tile_kernel<D, NT, kWarpsPerCta, ST>;
-  static unsigned long long done_mask = 0;  // one per template instance
-  cudaError_t e = configure_smem(kernel, smem, done_mask);
-  if (e != cudaSuccess) return e;
-  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, kWarpsPerCta * 32, smem);
-  dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
-  return launch_pdl(kernel, grid, dim3(kWarpsPerCta * 32), smem, stream, p, tk, tv);
-}
+constexpr int kStages = 2;
 
-template <int D, int ROWS>
-cudaError_t launch_single(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                          cudaStream_t stream, int* occupancy) {
-  constexpr int ST = 2;
-  constexpr int smem = DecodeSmem<D, ROWS, kWarpsPerCta, ST>::kBytes;
-  auto kernel = decode_single_kernel<D, ROWS, kWarpsPerCta, ST>;
-  static unsigned long long done_mask = 0;  // one per template instance
+template <class Core, int D>
+cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& tk,
+                        const CUtensorMap& tv, cudaStream_t stream, int* occupancy) {
+  constexpr int smem = DecodeSmem<D, Core::ROWS, kWarpsPerCta, kStages>::kBytes;
+  const dim3 block(kWarpsPerCta * 32);
+  if (schedule == kSchedulePersistent) {
+    auto kernel = decode_persistent_kernel<Core, D, kWarpsPerCta, kStages>;
+    static unsigned long long done_mask = 0;  // one per template instance
+    cudaError_t e = configure_smem(kernel, smem, done_mask);
+    if (e != cudaSuccess) return e;
+    if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, block.x, smem);
+    e = launch_pdl(sched_prepass_kernel<D>, dim3(1), dim3(kPrepassThreads), 0, stream, p);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, dim3(p.num_ctas), block, smem, stream, p, tk, tv);
+  }
+  auto kernel = decode_grid_kernel<Core, D, kWarpsPerCta, kStages>;
+  static unsigned long long done_mask = 0;
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
-  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, kWarpsPerCta * 32, smem);
-  dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
-  return launch_pdl(kernel, grid, dim3(kWarpsPerCta * 32), smem, stream, p, tk, tv);
+  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, block.x, smem);
+  const dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
+  e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
+  if (e != cudaSuccess || p.num_splits <= 1) return e;
+  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
+  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, stream, p);
 }
 
 template <int D>
-cudaError_t dispatch_rows(int path, int rows_per_cta, const DecodeParams& p, const CUtensorMap& tk,
-                          const CUtensorMap& tv, cudaStream_t stream, int* occ) {
+cudaError_t dispatch(int path, int schedule, int rows_per_cta, const DecodeParams& p,
+                     const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, int* occ) {
   if (path == kPathTile) {
     switch (rows_per_cta) {
-      case 8: return launch_tile<D, 1>(p, tk, tv, stream, occ);
-      case 16: return launch_tile<D, 2>(p, tk, tv, stream, occ);
-      case 24: return launch_tile<D, 3>(p, tk, tv, stream, occ);
-      case 32: return launch_tile<D, 4>(p, tk, tv, stream, occ);
+      case 8: return launch_core<TileCore<D, 1>, D>(p, schedule, tk, tv, stream, occ);
+      case 16: return launch_core<TileCore<D, 2>, D>(p, schedule, tk, tv, stream, occ);
+      case 24: return launch_core<TileCore<D, 3>, D>(p, schedule, tk, tv, stream, occ);
+      case 32: return launch_core<TileCore<D, 4>, D>(p, schedule, tk, tv, stream, occ);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (rows_per_cta) {
-    case 1: return launch_single<D, 1>(p, tk, tv, stream, occ);
-    case 2: return launch_single<D, 2>(p, tk, tv, stream, occ);
-    case 4: return launch_single<D, 4>(p, tk, tv, stream, occ);
-    case 8: return launch_single<D, 8>(p, tk, tv, stream, occ);
+    case 1: return launch_core<SimtCore<D, 1>, D>(p, schedule, tk, tv, stream, occ);
+    case 2: return launch_core<SimtCore<D, 2>, D>(p, schedule, tk, tv, stream, occ);
+    case 4: return launch_core<SimtCore<D, 4>, D>(p, schedule, tk, tv, stream, occ);
+    case 8: return launch_core<SimtCore<D, 8>, D>(p, schedule, tk, tv, stream, occ);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D>
-cudaError_t launch_merge(const DecodeParams& p, cudaStream_t stream) {
-  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
-  cfg.blockDim = dim3(128);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, merge_kernel<D>, p);
-}
-
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, int path, int head_dim, const CUtensorMap& tk,
-                          const CUtensorMap& tv, cudaStream_t stream) {
-  cudaError_t e = head_dim == 128 ? dispatch_rows<128>(path, p.rows_per_cta, p, tk, tv, stream, nullptr)
-                                  : dispatch_rows<64>(path, p.rows_per_cta, p, tk, tv, stream, nullptr);
-  if (e != cudaSuccess || p.num_splits <= 1) return e;
-  return head_dim == 128 ? launch_merge<128>(p, stream) : launch_merge<64>(p, stream);
+cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim,
+                          const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+  return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, p, tk, tv, stream, nullptr)
+                         : dispatch<64>(path, schedule, p.rows_per_cta, p, tk, tv, stream, nullptr);
 }
 
-int decode_ctas_per_sm(int path, int head_dim, int rows_per_cta) {
+int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta) {
   DecodeParams dummy = {};
   CUtensorMap tm = {};
   int occ = 0;
-  cudaError_t e = head_dim == 128 ? dispatch_rows<128>(path, rows_per_cta, dummy, tm, tm, nullptr, &occ)
-                                  : dispatch_rows<64>(path, rows_per_cta, dummy, tm, tm, nullptr, &occ);
+  cudaError_t e = head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ)
+                                  : dispatch<64>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ);
   return e == cudaSuccess && occ > 0 ? occ : 1;
 }
 
@@ -858,17 +1250,9 @@ cudaError_t launch_cache_write(const uint16_t* key, const uint16_t* value, int64
                                const int64_t* slots, int64_t num_tokens, int32_t row_elems,
                                int64_t num_slots, cudaStream_t stream) {
   const int64_t threads = 2 * num_tokens * 32;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((threads + 255) / 256));
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, cache_write_kernel, key, value, key_stride, value_stride, key_cache,
-                            value_cache, slots, num_tokens, row_elems, num_slots);
+  return launch_pdl(cache_write_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0,
+                    stream, key, value, key_stride, value_stride, key_cache, value_cache, slots,
+                    num_tokens, row_elems, num_slots);
 }
 
 cudaError_t run_validate(const int32_t* block_tables, const int32_t* context_lens,

@@ -59,7 +59,7 @@ extern "C" PA_API pa_status_t pa_decode_static_scratch(
   pa_plan_t local;
   if (plan == nullptr) {
     const pa_status_t st = pa_decode_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
-                                          max_blocks_per_seq, PA_PATH_AUTO, 0, &local);
+                                          max_blocks_per_seq, nullptr, &local);
     if (st != PA_OK) return st;
     plan = &local;
   }

@@ -38,13 +38,31 @@ EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size"
 PA_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
+PA_SCHEDULE_AUTO = 0
+PA_SCHEDULE_GRID = 1
+PA_SCHEDULE_PERSISTENT = 2
+
+
+class pa_plan_hints_t(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
+                ("split_blocks", ctypes.c_int32), ("share_prefix", ctypes.c_int32)]
+
+
 class pa_plan_t(ctypes.Structure):
-    _fields_ = [("path", ctypes.c_int32), ("split_blocks", ctypes.c_int32),
-                ("num_splits", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32)]
+    _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
+                ("split_blocks", ctypes.c_int32), ("num_splits", ctypes.c_int32),
+                ("rows_per_cta", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
+                ("share_cap", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {"path": {1: "single", 2: "tile"}.get(self.path, self.path),
+                "schedule": {1: "grid", 2: "persistent"}.get(self.schedule, self.schedule),
+                "split_blocks": self.split_blocks, "num_splits": self.num_splits,
+                "rows_per_cta": self.rows_per_cta, "num_ctas": self.num_ctas,
+                "share_cap": self.share_cap}
 
     def __repr__(self):
-        return (f"pa_plan_t(path={self.path}, split_blocks={self.split_blocks}, "
-                f"num_splits={self.num_splits}, rows_per_cta={self.rows_per_cta})")
+        return f"pa_plan_t({self.as_dict()})"
 
 
 _P = ctypes.c_void_p
@@ -54,7 +72,8 @@ _I64 = ctypes.c_int64
 _lib.pa_reshape_and_cache.restype = _I32
 _lib.pa_reshape_and_cache.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _I32, _I64, _I32, _P]
 _lib.pa_decode_plan.restype = _I32
-_lib.pa_decode_plan.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(pa_plan_t)]
+_lib.pa_decode_plan.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, ctypes.POINTER(pa_plan_hints_t),
+                                ctypes.POINTER(pa_plan_t)]
 _lib.pa_decode_workspace_size.restype = ctypes.c_size_t
 _lib.pa_decode_workspace_size.argtypes = [ctypes.POINTER(pa_plan_t), _I32, _I32, _I32, _I32, _I32, _I32]
 _lib.pa_decode.restype = _I32
@@ -126,11 +145,16 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
 
 
 def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,
-                   head_dim: int, max_blocks_per_seq: int, path_hint: int = PA_PATH_AUTO,
-                   split_blocks_hint: int = 0) -> pa_plan_t:
+                   head_dim: int, max_blocks_per_seq: int, path: int = PA_PATH_AUTO,
+                   split_blocks: int = 0, schedule: int = PA_SCHEDULE_AUTO,
+                   share_prefix: bool = False) -> pa_plan_t:
+    """A forced split length implies the grid schedule."""
+    if split_blocks and schedule == PA_SCHEDULE_AUTO:
+        schedule = PA_SCHEDULE_GRID
+    hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)))
     plan = pa_plan_t()
     st = _lib.pa_decode_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
-                             max_blocks_per_seq, path_hint, split_blocks_hint, ctypes.byref(plan))
+                             max_blocks_per_seq, ctypes.byref(hints), ctypes.byref(plan))
     _check(st, "pa_decode_plan")
     return plan
 

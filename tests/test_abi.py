@@ -80,8 +80,14 @@ def test_decode_rejects_bad_arguments_before_launch(pa):
     need = pa.pa_decode_workspace_size(plan, 2, 1, 4, 2, 64, 4)
     assert need == 2 * 4 * 1 * 4 * (64 + 2) * 4
     assert _decode_raw(lib, plan=ctypes.byref(plan), ws=96 * 1024, ws_bytes=need - 1) == pa.PA_ERR_WORKSPACE
-    bad = pa.pa_plan_t(plan.path, plan.split_blocks, plan.num_splits + 1, plan.rows_per_cta)
+    bad = pa.pa_plan_t.from_buffer_copy(plan)
+    bad.num_splits += 1
     assert _decode_raw(lib, plan=ctypes.byref(bad), ws=96 * 1024, ws_bytes=need) == pa.PA_ERR_INVALID_ARG
+    # the persistent schedule always needs its pre-pass tables
+    pplan = pa.pa_decode_plan(2, 1, 4, 2, 64, 4, pa.PA_PATH_TILE, schedule=pa.PA_SCHEDULE_PERSISTENT)
+    pneed = pa.pa_decode_workspace_size(pplan, 2, 1, 4, 2, 64, 4)
+    assert pneed > 0
+    assert _decode_raw(lib, plan=ctypes.byref(pplan)) == pa.PA_ERR_WORKSPACE
 
 
 def test_cache_write_rejects_bad_arguments_before_launch(pa):
@@ -108,7 +114,17 @@ def test_plan_heuristic_host_logic(pa):
     p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024)
     assert p.path == pa.PA_PATH_TILE and p.rows_per_cta == 24
     p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192)
+    assert p.schedule == pa.PA_SCHEDULE_PERSISTENT and p.num_ctas >= 1 and p.share_cap == 0
+    p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, schedule=pa.PA_SCHEDULE_GRID)
     assert p.num_splits > 1 and p.split_blocks * p.num_splits >= 8192
+    # prefix sharing: a shared unit holds 32 rows = 8 sequences of 4 rows
+    p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, share_prefix=True)
+    assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (2, 2, 32, 8)
+    with pytest.raises(pa.PAError) as exc:   # 24 rows per sequence: two do not fit 32 rows
+        pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, share_prefix=True)
+    assert exc.value.status == pa.PA_ERR_UNSUPPORTED
+    with pytest.raises(pa.PAError):          # sharing needs the persistent schedule
+        pa.pa_decode_plan(8, 1, 32, 8, 128, 64, schedule=pa.PA_SCHEDULE_GRID, share_prefix=True)
     forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)
     assert (forced.path, forced.split_blocks, forced.num_splits, forced.rows_per_cta) == (1, 64, 128, 8)
     # rows beyond one CTA are split into row chunks

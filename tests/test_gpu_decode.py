@@ -12,39 +12,49 @@ from paged_kv_cache_399_b200 import workloads
 
 pytestmark = pytest.mark.gpu
 
-# (name, context lengths, q_per_seq, H_q, H_kv, head_dim, scale)
+# name, context lengths, q_per_seq, H_q, H_kv, head_dim, scale, shared-prefix groups
+# [(first sequence, members, prefix tokens)]
 CASES = [
-    ("ctx1", [1, 1, 1], 1, 4, 2, 64, None),
-    ("mult16", [16, 32, 64, 128], 1, 8, 2, 128, None),
-    ("ragged", [17, 49, 33, 200, 255], 1, 8, 2, 128, None),
-    ("mha", [40, 97, 300], 1, 4, 4, 128, None),
-    ("mqa", [40, 97, 300], 1, 8, 1, 128, None),
-    ("d64_gqa4", [5, 77, 160, 333], 1, 8, 2, 64, None),
-    ("spec2", [9, 40, 129], 2, 8, 2, 128, None),
-    ("spec6", [6, 16, 22, 300, 517], 6, 32, 8, 128, None),
-    ("spec6_d64", [7, 100, 64], 6, 4, 1, 64, None),
-    ("rows64", [33, 70], 16, 16, 4, 128, None),        # G*q = 64: two 32-row chunks
-    ("single_rows16", [50, 81], 2, 8, 1, 128, None),  # 16 rows on the CUDA-core path: two chunks
-    ("zero_scale", [25, 66], 3, 4, 2, 128, 0.0),
-    ("long_ragged", [1000, 2049, 3001], 1, 8, 1, 128, None),
+    ("ctx1", [1, 1, 1], 1, 4, 2, 64, None, []),
+    ("mult16", [16, 32, 64, 128], 1, 8, 2, 128, None, []),
+    ("ragged", [17, 49, 33, 200, 255], 1, 8, 2, 128, None, []),
+    ("mha", [40, 97, 300], 1, 4, 4, 128, None, []),
+    ("mqa", [40, 97, 300], 1, 8, 1, 128, None, []),
+    ("d64_gqa4", [5, 77, 160, 333], 1, 8, 2, 64, None, []),
+    ("spec2", [9, 40, 129], 2, 8, 2, 128, None, []),
+    ("spec6", [6, 16, 22, 300, 517], 6, 32, 8, 128, None, []),
+    ("spec6_d64", [7, 100, 64], 6, 4, 1, 64, None, []),
+    ("rows64", [33, 70], 16, 16, 4, 128, None, []),        # G*q = 64: two 32-row chunks
+    ("single_rows16", [50, 81], 2, 8, 1, 128, None, []),  # 16 rows on the CUDA-core path
+    ("zero_scale", [25, 66], 3, 4, 2, 128, 0.0, []),
+    ("long_ragged", [1000, 2049, 3001], 1, 8, 1, 128, None, []),
+    # prefix sharing: groups of adjacent sequences over the same physical prefix blocks
+    ("shared3", [70, 49, 95, 33, 300], 1, 8, 2, 128, None, [(0, 3, 48)]),
+    ("shared9", [260 + 7 * k for k in range(9)] + [40], 1, 8, 2, 128, None, [(0, 9, 256)]),
+    ("shared_spec2", [64, 70, 81, 66], 2, 4, 2, 128, None, [(0, 4, 64)]),
+    ("shared_short", [20, 16, 300, 310], 1, 4, 1, 64, None, [(0, 2, 16), (2, 2, 288)]),
+    ("many_seqs", [1 + (37 * k) % 40 for k in range(1500)], 1, 4, 2, 64, None, []),
 ]
 
 PLANS = [
-    ("auto", None, None),
-    ("single", 1, None),
-    ("tile", 2, None),
-    ("single_split1", 1, 1),
-    ("tile_split1", 2, 1),
-    ("tile_split3", 2, 3),
-    ("tile_split8", 2, 8),
+    ("auto", {}),
+    ("single_grid", dict(path=1, schedule=1)),
+    ("tile_grid", dict(path=2, schedule=1)),
+    ("single_persist", dict(path=1, schedule=2)),
+    ("tile_persist", dict(path=2, schedule=2)),
+    ("share", dict(path=2, schedule=2, share_prefix=True)),
+    ("single_split1", dict(path=1, split_blocks=1)),
+    ("tile_split1", dict(path=2, split_blocks=1)),
+    ("tile_split3", dict(path=2, split_blocks=3)),
 ]
 
 
 def _workload(case, seed):
-    name, ctxs, q, hq, hkv, d, scale = case
+    name, ctxs, q, hq, hkv, d, scale, groups = case
+    share = [(list(range(first, first + n)), tokens) for first, n, tokens in groups]
     return workloads.build_workload(name, seed, ctxs, q, hq, hkv, d,
                                     scale=(1.0 / math.sqrt(d)) if scale is None else scale,
-                                    pool_factor=1.5)
+                                    pool_factor=1.5, share_groups=share)
 
 
 @pytest.fixture(scope="module")
@@ -63,11 +73,14 @@ def prepared(oracle_lib):
 def test_decode_matches_oracle(case, plan_spec, prepared):
     from paged_kv_cache_399_b200 import pa
     w, ref = prepared[case[0]]
-    _, path, split = plan_spec
     plan = None
-    if path is not None:
-        plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                 w.max_blocks_per_seq, path, split or 0)
+    if plan_spec[1]:
+        try:
+            plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads,
+                                     w.head_dim, w.max_blocks_per_seq, **plan_spec[1])
+        except pa.PAError as exc:
+            assert exc.status == pa.PA_ERR_UNSUPPORTED and plan_spec[1].get("share_prefix")
+            pytest.skip("prefix sharing needs G*q <= 16 rows")
     dw = DeviceWorkload(w)
     out = run_step(dw, plan)
     assert_close(out, ref, f"{case[0]}/{plan_spec[0]}")
@@ -80,7 +93,7 @@ def test_tiny_workload_every_path(oracle_lib):
     ref = oracle_lib.decode(w.query, kc, vc, w.block_tables, w.context_lens, 1, w.scale)
     outs = []
     for path in (pa.PA_PATH_SINGLE, pa.PA_PATH_TILE):
-        for split in (0, 1, 2):
+        for split in (0, 1, 2):  # 0: persistent schedule, else grid with that split
             plan = pa.pa_decode_plan(w.num_seqs, 1, 4, 2, 64, w.max_blocks_per_seq, path, split)
             out = run_step(DeviceWorkload(w), plan)
             assert_close(out, ref, f"tiny path={path} split={split}")
