@@ -107,6 +107,32 @@ def measured_peaks():
     return dict(PEAKS_FALLBACK, source="fallback")
 
 
+# ------------------------------------------------------------------ ranks
+
+BASE_SEEDS = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
+              "spec_verify": 1004}
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Weak scaling: every rank decodes its own replica of the workload, own seed."""
+    return BASE_SEEDS[workload] + 100 * rank
+
+
+def reduce_over_ranks(value: float, op: str, dist=None, device=None) -> float:
+    """max / sum of a per-rank float over the default process group (no-op alone)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate_throughput(bytes_per_step_per_rank: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job GB/s: all ranks' bytes over the slowest rank's device time."""
+    return world * bytes_per_step_per_rank * steps / (max_ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -191,24 +217,35 @@ def run_gpu(args):
     pa_build.build()
     from paged_kv_cache_399_b200 import pa, workloads
 
-    # weak scaling: every rank decodes its own replica of the workload (own seed)
-    base_seed = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
-                 "spec_verify": 1004}[args.workload]
-    w = workloads.make(args.workload, seed=base_seed + 100 * rank)
+    w = workloads.make(args.workload, seed=rank_seed(args.workload, rank))
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream(dev)
 
-    query = w.query.to(dev)
-    key = w.key.to(dev)
-    value = w.value.to(dev)
-    slots = torch.from_numpy(w.slot_mapping).to(dev)
-    tables = torch.from_numpy(w.block_tables).to(dev)
-    ctx = torch.from_numpy(w.context_lens).to(dev)
+    # the step's per-call inputs live in one device buffer (and one pinned host buffer for
+    # the end-to-end leg), so a step's host->device traffic is a single copy
+    parts = [("query", w.query), ("key", w.key), ("value", w.value),
+             ("slots", torch.from_numpy(w.slot_mapping)), ("tables", torch.from_numpy(w.block_tables)),
+             ("ctx", torch.from_numpy(w.context_lens))]
+    offsets, total = {}, 0
+    for name, t in parts:
+        offsets[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+    views = {}
+    for name, t in parts:
+        n = t.numel() * t.element_size()
+        h_in[offsets[name]:offsets[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        views[name] = d_in[offsets[name]:offsets[name] + n].view(t.dtype).view(t.shape)
+    d_in.copy_(h_in)
+    query, key, value = views["query"], views["key"], views["value"]
+    slots, tables, ctx = views["slots"], views["tables"], views["ctx"]
     key_cache = w.key_cache.to(dev)
     value_cache = w.value_cache.to(dev)
     out = torch.empty_like(query)
-    # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
-    share = bool(w.shared_groups) and not args.no_share_prefix
+    # prefix sharing is opt-in: the persistent shared-prefix path is slower than the
+    # grid schedule on these shapes, so it is not the default
+    share = bool(w.shared_groups) and args.share_prefix
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
                              w.max_blocks_per_seq, share_prefix=share,
                              schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
@@ -228,11 +265,7 @@ def run_gpu(args):
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_over_ranks(x, "max", dist if world > 1 else None, dev)
 
     launches_per_step = 1 + (2 if (plan.schedule == pa.PA_SCHEDULE_PERSISTENT or plan.num_splits > 1) else 1)
     step_bytes = decode_bytes(w) + cache_write_bytes(w)
@@ -271,14 +304,8 @@ def run_gpu(args):
         decode_ms = max_over_ranks(decode_ms)
 
         # (3) end to end: host (pinned) inputs in, output back to the host, every step
-        h_query = query.cpu().pin_memory()
-        h_key = key.cpu().pin_memory()
-        h_value = value.cpu().pin_memory()
-        h_slots = slots.cpu().pin_memory()
-        h_tables = tables.cpu().pin_memory()
-        h_ctx = ctx.cpu().pin_memory()
         h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in (h_query, h_key, h_value, h_slots, h_tables, h_ctx))
+        h2d = total
         d2h = h_out.numel() * h_out.element_size()
         e2e_steps = max(1, args.steps // 4)
         barrier()
@@ -286,12 +313,7 @@ def run_gpu(args):
         f1 = torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for _ in range(e2e_steps):
-            query.copy_(h_query, non_blocking=True)
-            key.copy_(h_key, non_blocking=True)
-            value.copy_(h_value, non_blocking=True)
-            slots.copy_(h_slots, non_blocking=True)
-            tables.copy_(h_tables, non_blocking=True)
-            ctx.copy_(h_ctx, non_blocking=True)
+            d_in.copy_(h_in, non_blocking=True)
             step()
             h_out.copy_(out, non_blocking=True)
         f1.record(stream)
@@ -300,8 +322,8 @@ def run_gpu(args):
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
 
     ms_per_step = ms_total / args.steps
-    value_gbs = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
-    e2e_gbs = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    value_gbs = aggregate_throughput(step_bytes, args.steps, ms_total, world)
+    e2e_gbs = aggregate_throughput(step_bytes, e2e_steps, e2e_ms, world)
     peaks = measured_peaks()
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
     traffic = None
@@ -415,9 +437,7 @@ def run_reference(args):
         return
     from oracle import Oracle
     from paged_kv_cache_399_b200 import workloads
-    base_seed = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
-                 "spec_verify": 1004}[args.workload]
-    w = workloads.make(args.workload, seed=base_seed)
+    w = workloads.make(args.workload, seed=rank_seed(args.workload, 0))
     orc = Oracle()
     seqs = list(range(min(w.num_seqs, args.ref_sample_seqs)))
     sub = _sample_workload(w, seqs)
@@ -463,8 +483,8 @@ def main(argv=None):
                     choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=["auto", "grid", "persistent"], default="auto")
-    ap.add_argument("--no-share-prefix", action="store_true",
-                    help="do not ask pa_decode to read shared prefix blocks once per group")
+    ap.add_argument("--share-prefix", action="store_true",
+                    help="ask pa_decode to read shared prefix blocks once per group (persistent)")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     args = ap.parse_args(argv)

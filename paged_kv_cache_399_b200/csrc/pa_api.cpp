@@ -124,7 +124,9 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1) return PA_ERR_INVALID_ARG;
   const int group = num_q_heads / num_kv_heads;
   const int rows = group * q_per_seq;
-  int schedule = h.schedule == PA_SCHEDULE_AUTO ? PA_SCHEDULE_PERSISTENT : h.schedule;
+  // automatic: the grid schedule, unless prefix sharing (persistent only) is asked for
+  int schedule = h.schedule;
+  if (schedule == PA_SCHEDULE_AUTO) schedule = h.share_prefix ? PA_SCHEDULE_PERSISTENT : PA_SCHEDULE_GRID;
   int share_cap = 0;
   if (h.share_prefix) {
     if (schedule != PA_SCHEDULE_PERSISTENT) return PA_ERR_INVALID_ARG;
@@ -204,7 +206,7 @@ PersistentLayout persistent_layout(const pa_plan_t& plan, int32_t num_seqs, int3
   L.cta_seq = off; off = align256(off + 4 * static_cast<size_t>(P));
   L.arrive = off; off = align256(off + 4 * static_cast<size_t>(targets));
   L.list_len = off; off = align256(off + 4 * static_cast<size_t>(targets));
-  L.list = off; off = align256(off + 4 * static_cast<size_t>(targets) * L.list_cap);
+  L.list = off; off = align256(off + 8 * static_cast<size_t>(targets) * L.list_cap);
   L.records = off; off = align256(off + 4 * static_cast<size_t>(pool) * L.rec_stride);
   L.total = off;
   return L;
@@ -377,7 +379,7 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
     p.cta_seq = reinterpret_cast<int32_t*>(ws + L.cta_seq);
     p.arrive = reinterpret_cast<int32_t*>(ws + L.arrive);
     p.list_len = reinterpret_cast<int32_t*>(ws + L.list_len);
-    p.list = reinterpret_cast<int32_t*>(ws + L.list);
+    p.list = reinterpret_cast<int2*>(ws + L.list);
     p.records = reinterpret_cast<float*>(ws + L.records);
   } else if (need > 0) {
     p.ws_o = reinterpret_cast<float*>(ws);

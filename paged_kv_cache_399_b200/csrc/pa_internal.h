@@ -54,11 +54,11 @@ struct DecodeParams {
   int32_t rec_stride;            // floats per record: target_rows * D + 2 * target_rows
   SchedHeader* hdr;
   long long* seq_start;          // [B] first work unit of the sequence's bands
-  int4* seq_info;                // [B] {P_b shared prefix blocks, members if leader else 0, nblk, 0}
+  int4* seq_info;                // [B] {P_b shared prefix blocks, members if leader else 0, nblk, ctx}
   int32_t* cta_seq;              // [num_ctas] sequence holding the CTA's first unit
   int32_t* arrive;               // [targets] blocks merged so far
   int32_t* list_len;             // [targets]
-  int32_t* list;                 // [targets][list_cap] record slots
+  int2* list;                    // [targets][list_cap] {piece start block, record slot}
   float* records;                // [pool_cap][rec_stride]
 };
 

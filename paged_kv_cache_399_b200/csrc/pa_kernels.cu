@@ -116,8 +116,10 @@ struct WarpPipe {
   int issued;
   uint32_t phase_base;   // loads issued on this warp's barriers before this run
 
+  // Block index (within the sequence) of this warp's k-th block of the run.
+  __device__ __forceinline__ int block_of(int k) const { return blk0 + warp + NW * k; }
   __device__ __forceinline__ int table_entry(int k) const {
-    return k < n_my ? __ldg(trow + blk0 + warp + NW * k) : 0;
+    return k < n_my ? __ldg(trow + block_of(k)) : 0;
   }
   __device__ __forceinline__ void init(uint8_t* smem, uint64_t* all_bars, int warp_, int lane_) {
     warp = warp_;
@@ -545,7 +547,7 @@ __device__ __forceinline__ void run_segment(const DecodeParams& p, const Seg& sg
       break;
     }
     const int s = pipe.stage_of(k);
-    const int tb = (sg.blk0 + warp + NW * k) * kBlockSize;
+    const int tb = pipe.block_of(k) * kBlockSize;
     const bool need_mask = !sg.shared && tb + kBlockSize - 1 > first_masked;
     core.block(pipe.kbuf(s), pipe.vbuf(s), tb, need_mask, c, lane, nullptr);
     __syncwarp();
@@ -675,7 +677,7 @@ decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorM
       if (threadIdx.x == 0) record_error(kErrSchedule);
       break;
     }
-    const int ctx = __ldg(p.context_lens + b);
+    const int ctx = info.w;
     run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
     const float* ow = reinterpret_cast<const float*>(smem);
 
@@ -724,7 +726,7 @@ decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorM
         if (slot >= 0) {
           const int idx = atomicAdd(p.list_len + t, 1);
           if (idx < p.list_cap) {
-            p.list[static_cast<size_t>(t) * p.list_cap + idx] = slot;
+            p.list[static_cast<size_t>(t) * p.list_cap + idx] = make_int2(sg.blk0, slot);
           } else {
             record_error(kErrRecordList);
           }
@@ -737,22 +739,34 @@ decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorM
       __syncthreads();
       for (int m = 0; m < sg.members; ++m) {
         if (!st.last[m]) continue;  // uniform: shared memory flag
+        // This piece completed target t: merge its records in order of their first
+        // block (unique per target), so the result does not depend on arrival order.
         __threadfence();
         const int bm = sg.b0 + m;
         const int t = (bm * H + sg.kvh) * RC + rc;
         const int n = min(__ldcg(p.list_len + t), p.list_cap);
-        const int* lst = p.list + static_cast<size_t>(t) * p.list_cap;
+        const int2* lst = p.list + static_cast<size_t>(t) * p.list_cap;
+        int2* raw = reinterpret_cast<int2*>(smem);  // stage buffers are free here
+        int* sorted = reinterpret_cast<int*>(raw + n);
+        for (int k = threadIdx.x; k < n; k += NW * 32) raw[k] = __ldcg(lst + k);
+        __syncthreads();
+        for (int k = threadIdx.x; k < n; k += NW * 32) {
+          int rank = 0;
+          for (int k2 = 0; k2 < n; ++k2) rank += raw[k2].x < raw[k].x;
+          sorted[rank] = raw[k].y;
+        }
+        __syncthreads();
         const int rows_t = min(tr, p.rows - rc * ROWS);
         for (int task = threadIdx.x; task < rows_t * DC; task += NW * 32) {
           const int rr = task / DC, dc = task % DC;
           float M = -INFINITY;
           for (int k = 0; k < n; ++k) {
-            const float* rec = p.records + static_cast<size_t>(__ldcg(lst + k)) * p.rec_stride;
+            const float* rec = p.records + static_cast<size_t>(sorted[k]) * p.rec_stride;
             M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(rec + tr * D) + rr).x);
           }
           float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           for (int k = 0; k < n; ++k) {
-            const float* rec = p.records + static_cast<size_t>(__ldcg(lst + k)) * p.rec_stride;
+            const float* rec = p.records + static_cast<size_t>(sorted[k]) * p.rec_stride;
             const float2 mlk = __ldcg(reinterpret_cast<const float2*>(rec + tr * D) + rr);
             const float wt = (mlk.x == -INFINITY) ? 0.f : fast_exp2(mlk.x - M);
             L += wt * mlk.y;
@@ -766,6 +780,7 @@ decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorM
           const int h = sg.kvh * p.group + (rg - i * p.group);
           store_bf16x8(p.out + out_offset(p, bm, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
         }
+        __syncthreads();  // the sort buffer is reused by the next member
       }
     }
     __syncthreads();  // shared memory is reused by the next segment
@@ -813,25 +828,19 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v, long long
   return before;
 }
 
-// True when sequence b does not continue the shared group of b - 1.
-__device__ __forceinline__ bool group_start(const DecodeParams& p, int b) {
-  if (b == 0) return true;
-  if (num_blocks_of(p, __ldg(p.context_lens + b)) == 0 ||
-      num_blocks_of(p, __ldg(p.context_lens + b - 1)) == 0)
-    return true;
-  return __ldg(p.block_tables + static_cast<size_t>(b) * p.max_blocks) !=
-         __ldg(p.block_tables + static_cast<size_t>(b - 1) * p.max_blocks);
-}
-
 template <int D>
 __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const DecodeParams p) {
-  __shared__ long long warp_tot[kPrepassThreads / 32];
-  __shared__ int wmax[kPrepassThreads / 32];
+  constexpr int T = kPrepassThreads;
+  constexpr int kLook = 16;                 // >= share_cap - 1: lookahead past the chunk
+  __shared__ long long warp_tot[T / 32];
+  __shared__ int wmax[T / 32];
   __shared__ int s_g0carry;
-  __shared__ int s_lead[kPrepassThreads];  // leaders of this chunk with a possible shared prefix
-  __shared__ int s_pmax[kPrepassThreads];
-  __shared__ int s_mem[kPrepassThreads];
-  __shared__ int s_bad[kPrepassThreads];
+  __shared__ int s_ctx[T + kLook];          // context lengths of the chunk (+ lookahead)
+  __shared__ int s_gstart[T + kLook];       // 1: the sequence starts a new shared group
+  __shared__ int s_lead[T];                 // leaders of this chunk with a possible shared prefix
+  __shared__ int s_pmax[T];
+  __shared__ int s_mem[T];
+  __shared__ int s_bad[T];
   __shared__ int s_nlead;
   grid_dependency_wait();
   grid_launch_dependents();
@@ -839,7 +848,6 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
   const int H = p.num_kv_heads;
   const int RC = p.row_chunks;
   const int cap = p.share_cap;
-  constexpr int T = kPrepassThreads;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   // ---- pass 1: sharing, P_b, work(b) (kept in seq_start for now), W
@@ -849,19 +857,36 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
   for (int c0 = 0; c0 < B; c0 += T) {
     const int b = c0 + threadIdx.x;
     const bool in = b < B;
-    const int ctx = in ? __ldg(p.context_lens + b) : 0;
+    // one round of independent loads: context lengths and group-start flags
+    for (int idx = threadIdx.x; idx < T + kLook; idx += T) {
+      const int bb = c0 + idx;
+      int c = 0, g = 1;
+      if (bb < B) {
+        c = __ldg(p.context_lens + bb);
+        if (cap >= 2 && bb > 0) {
+          const int cprev = __ldg(p.context_lens + bb - 1);
+          const int t0 = __ldg(p.block_tables + static_cast<size_t>(bb) * p.max_blocks);
+          const int t1 = __ldg(p.block_tables + static_cast<size_t>(bb - 1) * p.max_blocks);
+          g = (num_blocks_of(p, c) == 0 || num_blocks_of(p, cprev) == 0 || t0 != t1) ? 1 : 0;
+        }
+      }
+      s_ctx[idx] = c;
+      s_gstart[idx] = g;
+    }
+    if (threadIdx.x == 0) s_nlead = 0;
+    __syncthreads();
+    const int ctx = s_ctx[threadIdx.x];
     const int nblk = in ? num_blocks_of(p, ctx) : 0;
     int g0 = 0;
     if (cap >= 2) {
       // first sequence of b's group: inclusive max-scan of group start positions
-      int v = (in && group_start(p, b)) ? b : -1;
+      int v = (in && s_gstart[threadIdx.x]) ? b : -1;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int y = __shfl_up_sync(kFull, v, off);
         if (lane >= off) v = max(v, y);
       }
       if (lane == 31) wmax[warp] = v;
-      if (threadIdx.x == 0) s_nlead = 0;
       __syncthreads();
       int before = s_g0carry;
       for (int w = 0; w < warp; ++w) before = max(before, wmax[w]);
@@ -872,8 +897,8 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
       if (in && (b - g0) % cap == 0) {
         int mem = 1;
         int pmax = (ctx - p.q_per_seq + 1) / kBlockSize;
-        while (mem < cap && b + mem < B && !group_start(p, b + mem)) {
-          pmax = min(pmax, (__ldg(p.context_lens + b + mem) - p.q_per_seq + 1) / kBlockSize);
+        while (mem < cap && b + mem < B && !s_gstart[threadIdx.x + mem]) {
+          pmax = min(pmax, (s_ctx[threadIdx.x + mem] - p.q_per_seq + 1) / kBlockSize);
           ++mem;
         }
         pmax = max(0, min(pmax, nblk));
@@ -884,11 +909,12 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
           s_mem[k] = mem;
           s_bad[k] = pmax;
         } else {
-          p.seq_info[b] = make_int4(0, 0, nblk, 0);
+          p.seq_info[b] = make_int4(0, 0, nblk, ctx);
         }
       }
       __syncthreads();
-      // longest common table prefix: warps take (leader, 32-block window) pairs
+      // longest common table prefix: warps take (leader, 32-block window) pairs; the
+      // members' entries of a window are loaded together
       const int nlead = s_nlead;
       int npairs = 0;
       for (int k = 0; k < nlead; ++k) npairs += (s_pmax[k] + 31) / 32;
@@ -899,11 +925,17 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
           ++k;
         }
         const int j = rem * 32 + lane;
+        const int mem = s_mem[k];
         bool ok = true;
         if (j < s_pmax[k]) {
-          const int32_t* t0 = p.block_tables + static_cast<size_t>(s_lead[k]) * p.max_blocks;
-          const int ref = __ldg(t0 + j);
-          for (int m = 1; m < s_mem[k]; ++m) ok &= __ldg(t0 + static_cast<size_t>(m) * p.max_blocks + j) == ref;
+          const int32_t* t0 = p.block_tables + static_cast<size_t>(s_lead[k]) * p.max_blocks + j;
+          const int ref = __ldg(t0);
+          int vals[kLook];
+#pragma unroll
+          for (int m = 1; m < kLook; ++m)
+            vals[m] = m < mem ? __ldg(t0 + static_cast<size_t>(m) * p.max_blocks) : ref;
+#pragma unroll
+          for (int m = 1; m < kLook; ++m) ok &= vals[m] == ref;
         }
         const unsigned badmask = __ballot_sync(kFull, !ok);
         if (badmask && lane == 0) atomicMin(&s_bad[k], rem * 32 + __ffs(badmask) - 1);
@@ -911,8 +943,8 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
       __syncthreads();
       for (int k = threadIdx.x; k < nlead; k += T) {
         const int P = s_bad[k];
-        p.seq_info[s_lead[k]] = make_int4(P, P > 0 ? s_mem[k] : 0,
-                                          num_blocks_of(p, __ldg(p.context_lens + s_lead[k])), 0);
+        const int lb = s_lead[k] - c0;
+        p.seq_info[s_lead[k]] = make_int4(P, P > 0 ? s_mem[k] : 0, num_blocks_of(p, s_ctx[lb]), s_ctx[lb]);
       }
     }
     __syncthreads();
@@ -926,7 +958,7 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
     __syncthreads();  // every leader entry is read before any is rewritten
     long long work = 0;
     if (in) {
-      p.seq_info[b] = make_int4(P_b, lead_members, nblk, 0);
+      p.seq_info[b] = make_int4(P_b, lead_members, nblk, ctx);
       work = (lead_members > 0 ? static_cast<long long>(H) * P_b : 0) +
              static_cast<long long>(H) * RC * (nblk - P_b);
       p.seq_start[b] = work;
@@ -1039,36 +1071,41 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   }
 }
 
-// Log-sum-exp merge of the grid schedule's split partials: one warp per (sequence,
-// query token, head).
+// Log-sum-exp merge of the grid schedule's split partials. One CTA per output row
+// (sequence, query token, head) with MW warps: warp w folds splits w, w+MW, ... into
+// (M_w, L_w, acc_w) with lanes over head_dim, and the CTA combines the MW states.
+constexpr int kMergeMaxWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const DecodeParams p) {
   constexpr int DPL = D / 32;
+  __shared__ float2 s_ml[kMergeMaxWarps];
+  __shared__ __align__(16) float s_acc[kMergeMaxWarps][D];
   grid_dependency_wait();
   const int RQ = p.q_per_seq * p.num_q_heads;
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= p.num_seqs * RQ) return;
+  const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int MW = blockDim.x >> 5;
   const int b = row / RQ;
   const int rq = row % RQ;
   const int nblk = num_blocks_of(p, __ldg(p.context_lens + b));
   const int ns = (nblk + p.split_blocks - 1) / p.split_blocks;
-  if (ns <= 1) return;  // written directly by the decode kernel
+  if (ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
   const size_t base = static_cast<size_t>(b) * p.num_splits * RQ + rq;
-  // (m, l) of split s in lane s % 32: independent loads, then a warp reduction
-  float M = -INFINITY;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.ws_ml[base + static_cast<size_t>(s) * RQ].x);
+  // this warp's maximum: its splits' (m, l) are spread over the lanes
+  float Mw = -INFINITY;
+  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[base + static_cast<size_t>(s) * RQ].x);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-  float L = 0.f, acc[DPL];
+  for (int off = 16; off > 0; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(kFull, Mw, off));
+  float Lw = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
 #pragma unroll 4
-  for (int s = 0; s < ns; ++s) {
+  for (int s = warp; s < ns; s += MW) {
     const size_t rec = base + static_cast<size_t>(s) * RQ;
     const float2 ml = p.ws_ml[rec];
-    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-    L += w * ml.y;
+    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mw);
+    Lw += w * ml.y;
     const float* src = p.ws_o + rec * D + lane * DPL;
     if constexpr (DPL == 4) {
       const float4 x = *reinterpret_cast<const float4*>(src);
@@ -1078,15 +1115,26 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
       acc[0] += w * x.x; acc[1] += w * x.y;
     }
   }
+  if (lane == 0) s_ml[warp] = make_float2(Mw, Lw);
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) s_acc[warp][lane * DPL + e] = acc[e];
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < MW; ++w) M = fmaxf(M, s_ml[w].x);
+  float L = 0.f;
+  for (int w = 0; w < MW; ++w) L += s_ml[w].x == -INFINITY ? 0.f : s_ml[w].y * fast_exp2(s_ml[w].x - M);
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const int i = rq / p.num_q_heads;
   const int h = rq % p.num_q_heads;
-  uint16_t* dst = p.out + out_offset(p, b, i, h, D) + lane * DPL;
-  if constexpr (DPL == 4) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                                                pack_bf16x2(acc[2] * inv, acc[3] * inv));
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  uint16_t* dst = p.out + out_offset(p, b, i, h, D);
+  for (int d = threadIdx.x; d < D / 2; d += blockDim.x) {
+    float v0 = 0.f, v1 = 0.f;
+    for (int w = 0; w < MW; ++w) {
+      const float wt = s_ml[w].x == -INFINITY ? 0.f : fast_exp2(s_ml[w].x - M);
+      v0 += wt * s_acc[w][2 * d];
+      v1 += wt * s_acc[w][2 * d + 1];
+    }
+    reinterpret_cast<uint32_t*>(dst)[d] = pack_bf16x2(v0 * inv, v1 * inv);
   }
 }
 
@@ -1204,7 +1252,9 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
   e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
   if (e != cudaSuccess || p.num_splits <= 1) return e;
   const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
-  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>((rows + 3) / 4)), dim3(128), 0, stream, p);
+  // about four splits per warp, at most kMergeMaxWarps warps per row
+  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + 3) / 4));
+  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
 }
 
 template <int D>

@@ -113,7 +113,7 @@ def test_plan_heuristic_host_logic(pa):
     assert pa.pa_decode_plan(4, 1, 4, 2, 64, 5).path == pa.PA_PATH_SINGLE
     p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024)
     assert p.path == pa.PA_PATH_TILE and p.rows_per_cta == 24
-    p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192)
+    p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, schedule=pa.PA_SCHEDULE_PERSISTENT)
     assert p.schedule == pa.PA_SCHEDULE_PERSISTENT and p.num_ctas >= 1 and p.share_cap == 0
     p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, schedule=pa.PA_SCHEDULE_GRID)
     assert p.num_splits > 1 and p.split_blocks * p.num_splits >= 8192

@@ -1,0 +1,39 @@
+"""bench.py's byte accounting, checked against the pages' numbers and by hand."""
+
+import json
+import os
+
+import numpy as np
+
+import bench
+from paged_kv_cache_399_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_numbers.json")
+
+
+def test_kv_bytes_per_token_matches_the_pages():
+    data = json.load(open(GOLDEN))
+    for row in data["kv_bytes"]:
+        per_tok = bench.kv_bytes_per_token(row["layers"], row["kv_heads"], row["head_dim"],
+                                           row["bytes_per_value"])
+        if "bytes_per_token" in row:
+            assert per_tok == row["bytes_per_token"], row["cite"]
+        if "gib_per_request" in row:
+            assert per_tok * row["context"] / 2 ** 30 == row["gib_per_request"], row["cite"]
+
+
+def test_decode_bytes_by_hand_and_shared_prefix_counted_once():
+    w = workloads.build_workload("t", 5, [16, 20], 1, 4, 2, 64)
+    kv = (16 + 20) * 2 * 64 * 2 * 2
+    qo = 2 * 2 * 1 * 4 * 64 * 2
+    assert bench.decode_bytes(w) == kv + qo + (1 + 2) * 4 + 2 * 4
+    g = workloads.build_workload("g", 6, [40, 45], 1, 4, 2, 64, share_groups=[([0, 1], 32)])
+    logical = bench.decode_bytes(g, unique=False)
+    unique = bench.decode_bytes(g)
+    assert logical - unique == 32 * 2 * 64 * 2 * 2   # the 32 shared tokens once, not twice
+
+
+def test_prefix_sharing_workload_unique_bytes():
+    w = workloads.prefix_sharing()
+    assert np.all(w.block_tables[0:8, :128] == w.block_tables[0, :128])
+    assert bench.decode_bytes(w) < bench.decode_bytes(w, unique=False) / 4
