@@ -248,6 +248,8 @@ def run_gpu(args):
     share = bool(w.shared_groups) and args.share_prefix
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
                              w.max_blocks_per_seq, share_prefix=share,
+                             path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
+                             split_blocks=args.split_blocks,
                              schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
     ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads,
                                            w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
@@ -483,6 +485,8 @@ def main(argv=None):
                     choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=["auto", "grid", "persistent"], default="auto")
+    ap.add_argument("--path", choices=["auto", "single", "tile", "tcgen05"], default="auto")
+    ap.add_argument("--split-blocks", type=int, default=0, help="grid schedule split length (0 = heuristic)")
     ap.add_argument("--share-prefix", action="store_true",
                     help="ask pa_decode to read shared prefix blocks once per group (persistent)")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)

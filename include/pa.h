@@ -81,7 +81,10 @@ typedef enum {
 typedef enum {
   PA_PATH_AUTO = 0,   /* heuristic (pa_decode_plan) */
   PA_PATH_SINGLE = 1, /* CUDA-core kernel: warp-shuffle reductions, fp32 FMA */
-  PA_PATH_TILE = 2    /* tensor-core kernel: mma.sync m16n8k16 bf16 -> fp32 */
+  PA_PATH_TILE = 2,   /* tensor-core kernel: mma.sync m16n8k16 bf16 -> fp32 */
+  PA_PATH_TCGEN05 = 3 /* 5th-generation tensor cores: tcgen05.mma with accumulators in
+                         tensor memory, one TMA warp, one MMA-issuing thread, one
+                         softmax warp (32 query rows per CTA); grid schedule only */
 } pa_path_t;
 
 /* How the work is spread over CTAs. */

@@ -83,6 +83,7 @@ bool encode_pool_map(CUtensorMap* map, const void* base, int64_t num_blocks, int
 // ----------------------------------------------------------------- plan
 
 int rows_per_cta_for(int path, int rows) {
+  if (path == pa::kPathTcgen05) return pa::kTc5Rows;
   if (path == pa::kPathTile) {
     const int r8 = static_cast<int>(ceil_div(rows, 8)) * 8;
     return r8 < pa::kTileMaxRows ? r8 : pa::kTileMaxRows;
@@ -116,7 +117,8 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (st != PA_OK) return st;
   pa_plan_hints_t h = {};
   if (hints) h = *hints;
-  if (h.path != PA_PATH_AUTO && h.path != PA_PATH_SINGLE && h.path != PA_PATH_TILE)
+  if (h.path != PA_PATH_AUTO && h.path != PA_PATH_SINGLE && h.path != PA_PATH_TILE &&
+      h.path != PA_PATH_TCGEN05)
     return PA_ERR_INVALID_ARG;
   if (h.schedule != PA_SCHEDULE_AUTO && h.schedule != PA_SCHEDULE_GRID &&
       h.schedule != PA_SCHEDULE_PERSISTENT)
@@ -131,8 +133,9 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (h.share_prefix) {
     if (schedule != PA_SCHEDULE_PERSISTENT) return PA_ERR_INVALID_ARG;
     share_cap = share_cap_for(rows);
-    if (share_cap < 2 || h.path == PA_PATH_SINGLE) return PA_ERR_UNSUPPORTED;
+    if (share_cap < 2 || h.path == PA_PATH_SINGLE || h.path == PA_PATH_TCGEN05) return PA_ERR_UNSUPPORTED;
   }
+  if (h.path == PA_PATH_TCGEN05 && schedule != PA_SCHEDULE_GRID) return PA_ERR_UNSUPPORTED;
   int path = h.path;
   if (path == PA_PATH_AUTO) path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
   // a shared-prefix unit holds share_cap sequences' rows in one CTA
@@ -225,7 +228,9 @@ size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_pe
 
 pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_heads,
                        int32_t num_kv_heads, int32_t max_blocks_per_seq) {
-  if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE) return PA_ERR_INVALID_ARG;
+  if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE && plan.path != PA_PATH_TCGEN05)
+    return PA_ERR_INVALID_ARG;
+  if (plan.path == PA_PATH_TCGEN05 && plan.schedule != PA_SCHEDULE_GRID) return PA_ERR_INVALID_ARG;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (plan.num_ctas <= 0 || plan.num_ctas > (1 << 20)) return PA_ERR_INVALID_ARG;
@@ -358,6 +363,7 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   p.group = num_q_heads / num_kv_heads;
   p.rows = p.group * q_per_seq;
   p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
   p.rows_per_cta = plan->rows_per_cta;
   p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
   p.scale_log2 = scale * 1.4426950408889634f;

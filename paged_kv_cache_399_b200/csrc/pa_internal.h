@@ -14,12 +14,14 @@ constexpr int kWarpsPerCta = 4;  // decode CTA = 4 warps, each with its own TMA 
 // Kernel families (pa_path_t values) and schedules (pa_schedule_t values).
 constexpr int kPathSingle = 1;
 constexpr int kPathTile = 2;
+constexpr int kPathTcgen05 = 3;
 constexpr int kScheduleGrid = 1;
 constexpr int kSchedulePersistent = 2;
 
 // Largest rows one CTA holds for each family.
 constexpr int kTileMaxRows = 32;   // 4 n-tiles of 8 rows
 constexpr int kSingleMaxRows = 8;
+constexpr int kTc5Rows = 32;      // tcgen05 kernel: one softmax warp, 32 TMEM lanes
 
 // Persistent schedule: header written by the pre-pass, read by the decode CTAs.
 struct SchedHeader {
@@ -36,6 +38,7 @@ struct DecodeParams {
   int32_t num_seqs, q_per_seq, num_q_heads, num_kv_heads, group;  // group = H_q / H_kv
   int32_t rows;                  // group * q_per_seq query rows per (sequence, kv head)
   int32_t max_blocks;
+  int64_t num_blocks;             // pool size (blocks)
   int32_t rows_per_cta;          // rows the kernel instance holds (ROWS)
   int32_t row_chunks;            // ceil(rows / rows_per_cta)
   float scale_log2;              // scale * log2(e)

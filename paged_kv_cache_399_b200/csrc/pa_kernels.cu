@@ -1010,8 +1010,14 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
 // blocks). A sequence with one split writes bf16 directly; otherwise each split
 // writes fp32 partials (o, m, l) for merge_kernel.
 // ---------------------------------------------------------------------------
+// Resident CTAs per SM the compiler must allow for (a register cap of 168): 3 for the
+// cores that fit without spilling; the 24- and 32-row tensor-core cores keep their
+// registers (they spill under the cap, which measured slower) and run 2 per SM.
+template <class Core>
+constexpr int min_ctas_per_sm() { return Core::ROWS > 16 && !Core::kNeedsQSmem ? 2 : 3; }
+
 template <class Core, int D, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, min_ctas_per_sm<Core>())
 decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v) {
   constexpr int ROWS = Core::ROWS;
@@ -1191,6 +1197,12 @@ __global__ void validate_kernel(const int32_t* block_tables, const int32_t* cont
 
 __device__ unsigned long long g_validate_count = 0;
 
+}  // namespace pa
+
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+
 // ---------------------------------------------------------------------------
 // Host-side launchers
 // ---------------------------------------------------------------------------
@@ -1222,6 +1234,9 @@ cudaError_t configure_smem(Kernel kernel, int smem, unsigned long long& done_mas
   const unsigned long long bit = 1ull << (dev & 63);
   if (done_mask & bit) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // ask for the largest shared-memory carveout, so that as many CTAs as the shared
+  // memory allows are resident (the driver may otherwise pick a smaller one)
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess) done_mask |= bit;
   return e;
 }
@@ -1258,8 +1273,29 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
 }
 
 template <int D>
+cudaError_t launch_tc5(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                       cudaStream_t stream, int* occupancy) {
+  constexpr int smem = tc5::Smem<D>::kBytes;
+  auto kernel = decode_tc5_kernel<D>;
+  static unsigned long long done_mask = 0;
+  cudaError_t e = configure_smem(kernel, smem, done_mask);
+  if (e != cudaSuccess) return e;
+  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tc5::kThreads, smem);
+  const dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
+  e = launch_pdl(kernel, grid, dim3(tc5::kThreads), smem, stream, p, tk, tv);
+  if (e != cudaSuccess || p.num_splits <= 1) return e;
+  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
+  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + 3) / 4));
+  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
+}
+
+template <int D>
 cudaError_t dispatch(int path, int schedule, int rows_per_cta, const DecodeParams& p,
                      const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, int* occ) {
+  if (path == kPathTcgen05) {
+    if (schedule != kScheduleGrid || rows_per_cta != kTc5Rows) return cudaErrorInvalidValue;
+    return launch_tc5<D>(p, tk, tv, stream, occ);
+  }
   if (path == kPathTile) {
     switch (rows_per_cta) {
       case 8: return launch_core<TileCore<D, 1>, D>(p, schedule, tk, tv, stream, occ);

@@ -30,6 +30,7 @@ PA_ERR_DEVICE = 6
 PA_PATH_AUTO = 0
 PA_PATH_SINGLE = 1
 PA_PATH_TILE = 2
+PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error", "pa_status_string",
@@ -55,7 +56,7 @@ class pa_plan_t(ctypes.Structure):
                 ("share_cap", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
-        return {"path": {1: "single", 2: "tile"}.get(self.path, self.path),
+        return {"path": {1: "single", 2: "tile", 3: "tcgen05"}.get(self.path, self.path),
                 "schedule": {1: "grid", 2: "persistent"}.get(self.schedule, self.schedule),
                 "split_blocks": self.split_blocks, "num_splits": self.num_splits,
                 "rows_per_cta": self.rows_per_cta, "num_ctas": self.num_ctas,

@@ -123,6 +123,10 @@ def test_plan_heuristic_host_logic(pa):
     with pytest.raises(pa.PAError) as exc:   # 24 rows per sequence: two do not fit 32 rows
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, share_prefix=True)
     assert exc.value.status == pa.PA_ERR_UNSUPPORTED
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05)
+    assert (p.path, p.schedule, p.rows_per_cta) == (3, 1, 32)
+    with pytest.raises(pa.PAError):          # tcgen05 runs the grid schedule only
+        pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05, schedule=pa.PA_SCHEDULE_PERSISTENT)
     with pytest.raises(pa.PAError):          # sharing needs the persistent schedule
         pa.pa_decode_plan(8, 1, 32, 8, 128, 64, schedule=pa.PA_SCHEDULE_GRID, share_prefix=True)
     forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)

@@ -46,6 +46,9 @@ PLANS = [
     ("single_split1", dict(path=1, split_blocks=1)),
     ("tile_split1", dict(path=2, split_blocks=1)),
     ("tile_split3", dict(path=2, split_blocks=3)),
+    ("tcgen05", dict(path=3)),
+    ("tcgen05_split1", dict(path=3, split_blocks=1)),
+    ("tcgen05_split5", dict(path=3, split_blocks=5)),
 ]
 
 
@@ -81,6 +84,8 @@ def test_decode_matches_oracle(case, plan_spec, prepared):
         except pa.PAError as exc:
             assert exc.status == pa.PA_ERR_UNSUPPORTED and plan_spec[1].get("share_prefix")
             pytest.skip("prefix sharing needs G*q <= 16 rows")
+        if plan.path == pa.PA_PATH_TCGEN05:
+            assert plan.schedule == pa.PA_SCHEDULE_GRID and plan.rows_per_cta == 32
     dw = DeviceWorkload(w)
     out = run_step(dw, plan)
     assert_close(out, ref, f"{case[0]}/{plan_spec[0]}")
