@@ -243,9 +243,8 @@ def run_gpu(args):
     key_cache = w.key_cache.to(dev)
     value_cache = w.value_cache.to(dev)
     out = torch.empty_like(query)
-    # prefix sharing is opt-in: the persistent shared-prefix path is slower than the
-    # grid schedule on these shapes, so it is not the default
-    share = bool(w.shared_groups) and args.share_prefix
+    # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
+    share = bool(w.shared_groups) and not args.no_share_prefix
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
                              w.max_blocks_per_seq, share_prefix=share,
                              path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
@@ -487,8 +486,8 @@ def main(argv=None):
     ap.add_argument("--schedule", choices=["auto", "grid", "persistent"], default="auto")
     ap.add_argument("--path", choices=["auto", "single", "tile", "tcgen05"], default="auto")
     ap.add_argument("--split-blocks", type=int, default=0, help="grid schedule split length (0 = heuristic)")
-    ap.add_argument("--share-prefix", action="store_true",
-                    help="ask pa_decode to read shared prefix blocks once per group (persistent)")
+    ap.add_argument("--no-share-prefix", action="store_true",
+                    help="do not ask pa_decode to read shared prefix blocks once per group")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     args = ap.parse_args(argv)

@@ -103,11 +103,12 @@ typedef struct {
   int32_t path;          /* pa_path_t */
   int32_t schedule;      /* pa_schedule_t */
   int32_t split_blocks;  /* grid schedule: blocks per split (0 = heuristic) */
-  int32_t share_prefix;  /* persistent schedule: 1 = adjacent sequences whose block
-                            tables start with the same physical blocks (parallel
-                            sampling, beam search, a common system prompt) are
-                            detected on the device and their common prefix blocks
-                            are read once for all of them; 0 = off */
+  int32_t share_prefix;  /* 1 = adjacent sequences whose block tables start with the
+                            same physical blocks (parallel sampling, beam search, a
+                            common system prompt) are detected on the device and their
+                            common prefix blocks are read once for all of them (up to
+                            32 / (GQA group x q_per_seq) sequences per read, tensor-core
+                            kernel); 0 = off */
 } pa_plan_hints_t;
 
 /* A decode plan; fill it with pa_decode_plan and treat it as opaque. */
@@ -118,8 +119,8 @@ typedef struct {
   int32_t num_splits;    /* grid: ceil(max_blocks_per_seq / split_blocks) */
   int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds */
   int32_t num_ctas;      /* persistent: CTAs launched (resident slots of the device) */
-  int32_t share_cap;     /* persistent: sequences per shared-prefix unit, 0 = off */
-  int32_t reserved;
+  int32_t share_cap;     /* sequences per shared-prefix unit, 0 = off */
+  int32_t share_split_blocks; /* grid with sharing: blocks per split of a shared prefix */
 } pa_plan_t;
 
 /* Write the step's new K/V into the pool: for each token t with slot s =

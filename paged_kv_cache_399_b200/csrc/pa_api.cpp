@@ -126,12 +126,9 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1) return PA_ERR_INVALID_ARG;
   const int group = num_q_heads / num_kv_heads;
   const int rows = group * q_per_seq;
-  // automatic: the grid schedule, unless prefix sharing (persistent only) is asked for
-  int schedule = h.schedule;
-  if (schedule == PA_SCHEDULE_AUTO) schedule = h.share_prefix ? PA_SCHEDULE_PERSISTENT : PA_SCHEDULE_GRID;
+  int schedule = h.schedule == PA_SCHEDULE_AUTO ? PA_SCHEDULE_GRID : h.schedule;
   int share_cap = 0;
   if (h.share_prefix) {
-    if (schedule != PA_SCHEDULE_PERSISTENT) return PA_ERR_INVALID_ARG;
     share_cap = share_cap_for(rows);
     if (share_cap < 2 || h.path == PA_PATH_SINGLE || h.path == PA_PATH_TCGEN05) return PA_ERR_UNSUPPORTED;
   }
@@ -147,12 +144,24 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   plan->schedule = schedule;
   plan->rows_per_cta = rpc;
   plan->share_cap = share_cap;
-  plan->reserved = 0;
+  plan->share_split_blocks = 0;
   if (schedule == PA_SCHEDULE_PERSISTENT) {
     plan->num_ctas = slots;
     plan->split_blocks = max_blocks_per_seq;
     plan->num_splits = 1;
     return PA_OK;
+  }
+  plan->share_split_blocks = 0;
+  if (share_cap) {
+    // the bulk of the work is the shared prefixes: at most ceil(B / cap) chunk windows
+    // per kv head; cut the longest possible prefix into as many splits as fill one wave
+    // of resident CTAs (long CTAs amortise their prologue and the records they write)
+    const int64_t units = ceil_div(num_seqs, share_cap) * num_kv_heads;
+    int64_t splits = static_cast<int64_t>(slots) / units;
+    if (splits < 1) splits = 1;
+    int64_t sb = ceil_div(ceil_div(max_blocks_per_seq, splits), pa::kWarpsPerCta) * pa::kWarpsPerCta;
+    if (sb < 4 * pa::kWarpsPerCta) sb = 4 * pa::kWarpsPerCta;
+    plan->share_split_blocks = static_cast<int32_t>(sb < max_blocks_per_seq ? sb : max_blocks_per_seq);
   }
   int split_blocks = h.split_blocks;
   if (split_blocks == 0) {
@@ -215,11 +224,25 @@ PersistentLayout persistent_layout(const pa_plan_t& plan, int32_t num_seqs, int3
   return L;
 }
 
+// Records of the grid schedule with prefix sharing: [B][share splits][q*H_q] for the
+// shared prefixes, then [B][num_splits][q*H_q] for the sequences' own blocks. The
+// share-split count is derived from share_split_blocks and the plan's split_blocks x
+// num_splits (= the table width rounded up).
+size_t share_records(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads) {
+  const int64_t width = static_cast<int64_t>(plan.split_blocks) * plan.num_splits;
+  const int64_t ssplits = plan.share_split_blocks > 0 ? ceil_div(width, plan.share_split_blocks) : 0;
+  return static_cast<size_t>(num_seqs) * (ssplits + plan.num_splits) * q_per_seq * num_q_heads;
+}
+
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (num_seqs == 0) return 0;
     return persistent_layout(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim).total;
+  }
+  if (plan.share_cap) {  // records of the shared-prefix splits and of the own splits + seq_info
+    const size_t recs = share_records(plan, num_seqs, q_per_seq, num_q_heads);
+    return align256(recs * (static_cast<size_t>(head_dim) + 2) * 4) + 16 * static_cast<size_t>(num_seqs);
   }
   if (plan.num_splits <= 1) return 0;
   return static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads *
@@ -234,6 +257,7 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (plan.num_ctas <= 0 || plan.num_ctas > (1 << 20)) return PA_ERR_INVALID_ARG;
+    if (plan.share_split_blocks != 0) return PA_ERR_INVALID_ARG;  // grid-only field
     if (plan.share_cap != 0) {
       if (plan.path != PA_PATH_TILE || plan.share_cap != share_cap_for(rows) ||
           plan.rows_per_cta != pa::kTileMaxRows)
@@ -241,8 +265,15 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
       return PA_OK;
     }
   } else if (plan.schedule == PA_SCHEDULE_GRID) {
-    if (plan.split_blocks <= 0 || plan.share_cap != 0) return PA_ERR_INVALID_ARG;
+    if (plan.split_blocks <= 0) return PA_ERR_INVALID_ARG;
     if (plan.num_splits != ceil_div(max_blocks_per_seq, plan.split_blocks)) return PA_ERR_INVALID_ARG;
+    if (plan.share_cap != 0) {
+      if (plan.path != PA_PATH_TILE || plan.share_cap != share_cap_for(rows) ||
+          plan.rows_per_cta != pa::kTileMaxRows || plan.share_split_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+      return PA_OK;
+    }
+    if (plan.share_split_blocks != 0) return PA_ERR_INVALID_ARG;
   } else {
     return PA_ERR_INVALID_ARG;
   }
@@ -388,9 +419,18 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
     p.list = reinterpret_cast<int2*>(ws + L.list);
     p.records = reinterpret_cast<float*>(ws + L.records);
   } else if (need > 0) {
+    const size_t recs = plan->share_cap ? share_records(*plan, num_seqs, q_per_seq, num_q_heads)
+                                        : static_cast<size_t>(num_seqs) * plan->num_splits * rq;
     p.ws_o = reinterpret_cast<float*>(ws);
-    p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) +
-                                        static_cast<size_t>(num_seqs) * plan->num_splits * rq * head_dim);
+    p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + recs * head_dim);
+    if (plan->share_cap) {
+      p.share_cap = plan->share_cap;
+      p.share_split_blocks = plan->share_split_blocks;
+      p.share_splits = static_cast<int32_t>(
+          ceil_div(static_cast<int64_t>(plan->split_blocks) * plan->num_splits, plan->share_split_blocks));
+      p.share_windows = static_cast<int32_t>(ceil_div(num_seqs, plan->share_cap));
+      p.seq_info = reinterpret_cast<int4*>(ws + align256(recs * (static_cast<size_t>(head_dim) + 2) * 4));
+    }
   }
   cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, tk, tv,
                                     reinterpret_cast<cudaStream_t>(stream));

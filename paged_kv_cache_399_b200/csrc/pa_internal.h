@@ -43,8 +43,10 @@ struct DecodeParams {
   int32_t row_chunks;            // ceil(rows / rows_per_cta)
   float scale_log2;              // scale * log2(e)
 
-  // grid schedule: split partials for the merge kernel
+  // grid schedule: split partials for the merge kernel; with prefix sharing also the
+  // shared-prefix splits (a 1-D grid: shared CTAs, then the sequences' own CTAs)
   int32_t split_blocks, num_splits;
+  int32_t share_split_blocks, share_splits, share_windows;
   float* ws_o;                   // fp32 [B][num_splits][q*H_q][D]
   float2* ws_ml;                 // fp32 [B][num_splits][q*H_q] (m in log2 units, l)
 

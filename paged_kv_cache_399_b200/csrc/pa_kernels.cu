@@ -83,10 +83,12 @@ __device__ __forceinline__ int num_blocks_of(const DecodeParams& p, int ctx) {
 struct Seg {
   int b0, members, kvh, row0, nrows, blk0, blk1;
   bool shared;
+  int roff;  // local row r of this view is row r + roff of the segment (row-split CTAs)
 };
 
 __device__ __forceinline__ bool seg_row(const DecodeParams& p, const Seg& s, int r, int& b, int& i,
                                         int& h) {
+  r += s.roff;
   if (r >= s.nrows) return false;
   int m = 0, rr = s.row0 + r;
   if (s.shared) {
@@ -1027,19 +1029,85 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   uint8_t* smem = align1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x / p.row_chunks;
-  const int rc = blockIdx.x % p.row_chunks;
-  const int b = blockIdx.y;
-  const int split = blockIdx.z;
   init_cta<NW, STAGES>(st.bars, &tmap_k, &tmap_v);
   grid_dependency_wait();  // inputs may be produced by the previous kernel on the stream
+  const int H = p.num_kv_heads;
+  const int RQ = p.q_per_seq * p.num_q_heads;
+  const float* ow = reinterpret_cast<const float*>(smem);
+  WarpPipe<D, NW, STAGES> pipe;
+  pipe.init(smem, st.bars, warp, lane);
+  Core core;
+
+  // Grid layout. Without prefix sharing: x = kv head x row chunk, y = sequence,
+  // z = split of split_blocks blocks. With prefix sharing, a 1-D grid: first the
+  // shared CTAs (kv head, window of share_cap sequences, split of a shared prefix),
+  // then the sequences' own CTAs (kv head, sequence, split of the blocks after the
+  // shared prefix).
+  int kvh, rc = 0, b = 0, z;
+  bool shared_role = false;
+  if (p.share_cap) {
+    const long long idx = blockIdx.x;
+    const long long n_sh = static_cast<long long>(H) * p.share_windows * p.share_splits;
+    if (idx < n_sh) {
+      shared_role = true;
+      kvh = static_cast<int>(idx % H);
+      b = static_cast<int>((idx / H) % p.share_windows) * p.share_cap;  // first sequence of the window
+      z = static_cast<int>(idx / (static_cast<long long>(H) * p.share_windows));
+    } else {
+      const long long j = idx - n_sh;
+      kvh = static_cast<int>(j % H);
+      b = static_cast<int>((j / H) % p.num_seqs);
+      z = static_cast<int>(j / (static_cast<long long>(H) * p.num_seqs));
+    }
+  } else {
+    kvh = blockIdx.x / p.row_chunks;
+    rc = blockIdx.x % p.row_chunks;
+    b = blockIdx.y;
+    z = blockIdx.z;
+  }
+
+  if (shared_role) {
+    // every chunk leader of the window whose shared prefix reaches split z
+    const int ssb = p.share_split_blocks;
+    const int wend = min(p.num_seqs, b + p.share_cap);
+    if (threadIdx.x < wend - b) {
+      const int4 info = __ldcg(p.seq_info + b + threadIdx.x);
+      st.slot[threadIdx.x] = info.x;  // shared prefix blocks
+      st.last[threadIdx.x] = info.y;  // members if this sequence leads a chunk
+    }
+    __syncthreads();
+    for (int L = b; L < wend; ++L) {
+      const int P_L = st.slot[L - b], members = st.last[L - b];
+      if (members == 0 || z * ssb >= P_L) continue;  // uniform
+      const Seg sg{L, members, kvh, 0, members * p.rows, z * ssb, min(P_L, z * ssb + ssb), true};
+      run_segment<Core, D, NW, STAGES>(p, sg, 0, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
+      for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+        const int r = task / DC, dc = task % DC;
+        float M, L2, acc[8];
+        combine_row<D, ROWS, NW>(ow, st.ml, r, dc, M, L2, acc);
+        int bb, i, h;
+        seg_row(p, sg, r, bb, i, h);
+        const size_t rec = (static_cast<size_t>(bb) * p.share_splits + z) * RQ + i * p.num_q_heads + h;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + dc * 8);
+        dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if (dc == 0) p.ws_ml[rec] = make_float2(M, L2);
+      }
+      __syncthreads();  // shared memory is reused by the next segment
+    }
+    grid_launch_dependents();
+    return;
+  }
 
   const int ctx = __ldg(p.context_lens + b);
   const int nblk = num_blocks_of(p, ctx);
-  const int blk0 = split * p.split_blocks;
+  const int S = p.num_splits;
+  const int sb = p.split_blocks;
+  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : 0;  // own blocks start after the shared prefix
   Seg sg{b, 1, kvh, rc * ROWS, min(ROWS, p.rows - rc * ROWS), 0, 0, false};
+  const int blk0 = P_b + z * sb;
   if (blk0 >= nblk) {
-    if (split == 0) {  // no block at all: zero output
+    if (z == 0 && nblk == 0) {  // no block at all: zero output
       for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
         int bb, i, h;
         seg_row(p, sg, task / DC, bb, i, h);
@@ -1050,31 +1118,105 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
     return;
   }
   sg.blk0 = blk0;
-  sg.blk1 = min(nblk, blk0 + p.split_blocks);
-  const bool single_split = (nblk + p.split_blocks - 1) / p.split_blocks == 1;
-  WarpPipe<D, NW, STAGES> pipe;
-  pipe.init(smem, st.bars, warp, lane);
-  Core core;
+  sg.blk1 = min(nblk, blk0 + sb);
+  // the only piece of its outputs: write bf16 directly
+  const bool direct = P_b == 0 && nblk <= sb;
   run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
   grid_launch_dependents();
-  const float* ow = reinterpret_cast<const float*>(smem);
+  // own-block records follow the shared-prefix records when sharing is on
+  const size_t region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
   for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
     const int r = task / DC, dc = task % DC;
     float M, L, acc[8];
     combine_row<D, ROWS, NW>(ow, st.ml, r, dc, M, L, acc);
     int bb, i, h;
     seg_row(p, sg, r, bb, i, h);
-    if (single_split) {
+    if (direct) {
       store_bf16x8(p.out + out_offset(p, bb, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
     } else {
-      const int rq = i * p.num_q_heads + h;
-      const size_t rec = (static_cast<size_t>(b) * p.num_splits + split) * (p.q_per_seq * p.num_q_heads) + rq;
+      const size_t rec = (region + static_cast<size_t>(b) * S + z) * RQ + i * p.num_q_heads + h;
       float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + dc * 8);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
       if (dc == 0) p.ws_ml[rec] = make_float2(M, L);
     }
   }
+}
+
+// Prefix sharing for the grid schedule, one warp per sequence b. Sequences are cut
+// into windows of share_cap aligned at multiples of share_cap; inside a window, a
+// chunk is a maximal run of sequences whose block tables start with the same
+// physical block. The chunk's shared prefix P = the leading table entries identical
+// for all its members, limited to blocks every member's query rows fully see and to
+// kShareScanBlocks. Every member computes the same chunk and P from the same data.
+// seq_info[b] = {P (0: no shared part), members if b leads a chunk with P > 0, nblk, ctx}.
+constexpr int kShareScanBlocks = 8192;
+
+__global__ void __launch_bounds__(128) share_prepass_kernel(const DecodeParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (b >= p.num_seqs) return;
+  const int cap = p.share_cap;  // 2..16
+  const int W0 = (b / cap) * cap;
+  const int span = min(cap, p.num_seqs - W0);
+  int ctx_l = 0, nb_l = 0;
+  bool gs = true;
+  if (lane < span) {
+    const int bb = W0 + lane;
+    ctx_l = __ldg(p.context_lens + bb);
+    nb_l = num_blocks_of(p, ctx_l);
+    if (lane > 0) {
+      const int nprev = num_blocks_of(p, __ldg(p.context_lens + bb - 1));
+      gs = nb_l == 0 || nprev == 0 ||
+           __ldg(p.block_tables + static_cast<size_t>(bb) * p.max_blocks) !=
+               __ldg(p.block_tables + static_cast<size_t>(bb - 1) * p.max_blocks);
+    }
+  }
+  const unsigned starts = __ballot_sync(kFull, lane < span && gs);  // bit 0 is always set
+  const int m = b - W0;
+  const unsigned upto = (m >= 31) ? kFull : ((2u << m) - 1u);
+  const int Li = 31 - __clz(starts & upto);
+  const unsigned above = starts & ~upto;
+  const int Ni = above ? __ffs(above) - 1 : span;
+  const int members = Ni - Li;
+  const int leader = W0 + Li;
+  int pm = (lane >= Li && lane < Ni) ? min((ctx_l - p.q_per_seq + 1) / kBlockSize, nb_l) : INT_MAX;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) pm = min(pm, __shfl_xor_sync(kFull, pm, off));
+  const int pmax = max(0, min(pm, kShareScanBlocks));
+  int P = 0;
+  if (members > 1 && pmax > 0) {
+    const int32_t* t0 = p.block_tables + static_cast<size_t>(leader) * p.max_blocks;
+    P = pmax;
+    // 128 table positions per round: the loads of a round are all issued before any
+    // comparison, so a 2048-token prefix costs one round trip
+    for (int j0 = 0; j0 < pmax && P == pmax; j0 += 128) {
+      unsigned bad[4];
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        const int j = j0 + part * 32 + lane;
+        bool ok = true;
+        if (j < pmax) {
+          const int ref = __ldg(t0 + j);
+          int vals[16];
+#pragma unroll
+          for (int mm = 1; mm < 16; ++mm)
+            vals[mm] = mm < members ? __ldg(t0 + static_cast<size_t>(mm) * p.max_blocks + j) : ref;
+#pragma unroll
+          for (int mm = 1; mm < 16; ++mm) ok &= vals[mm] == ref;
+        }
+        bad[part] = __ballot_sync(kFull, !ok);
+      }
+#pragma unroll
+      for (int part = 3; part >= 0; --part)
+        if (bad[part]) P = j0 + part * 32 + __ffs(bad[part]) - 1;
+    }
+  }
+  const int my_ctx = __shfl_sync(kFull, ctx_l, m);
+  if (lane == 0)
+    p.seq_info[b] = make_int4(P, (b == leader && P > 0) ? members : 0, num_blocks_of(p, my_ctx), my_ctx);
 }
 
 // Log-sum-exp merge of the grid schedule's split partials. One CTA per output row
@@ -1095,12 +1237,21 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
   const int b = row / RQ;
   const int rq = row % RQ;
   const int nblk = num_blocks_of(p, __ldg(p.context_lens + b));
-  const int ns = (nblk + p.split_blocks - 1) / p.split_blocks;
-  if (ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
-  const size_t base = static_cast<size_t>(b) * p.num_splits * RQ + rq;
+  const int sb = p.split_blocks;
+  // records: the shared-prefix splits (region 0, with prefix sharing) then the
+  // sequence's own splits (region 1 with prefix sharing, else region 0)
+  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : 0;
+  const int nsh = P_b > 0 ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
+  const int ns = nsh + (nblk - P_b + sb - 1) / sb;
+  if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
+  const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
+  auto rec_of = [&](int k) -> size_t {
+    return (k < nsh ? static_cast<size_t>(b) * p.share_splits + k
+                    : own_region + static_cast<size_t>(b) * p.num_splits + (k - nsh)) * RQ + rq;
+  };
   // this warp's maximum: its splits' (m, l) are spread over the lanes
   float Mw = -INFINITY;
-  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[base + static_cast<size_t>(s) * RQ].x);
+  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[rec_of(s)].x);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(kFull, Mw, off));
   float Lw = 0.f, acc[DPL];
@@ -1108,7 +1259,7 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
 #pragma unroll 4
   for (int s = warp; s < ns; s += MW) {
-    const size_t rec = base + static_cast<size_t>(s) * RQ;
+    const size_t rec = rec_of(s);
     const float2 ml = p.ws_ml[rec];
     const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mw);
     Lw += w * ml.y;
@@ -1263,12 +1414,23 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, block.x, smem);
-  const dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
+  if (p.share_cap) {
+    e = launch_pdl(share_prepass_kernel, dim3(static_cast<unsigned>((p.num_seqs + 3) / 4)), dim3(128), 0,
+                   stream, p);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
+  if (p.share_cap) {
+    const long long ctas = static_cast<long long>(p.num_kv_heads) *
+                           (static_cast<long long>(p.share_windows) * p.share_splits +
+                            static_cast<long long>(p.num_seqs) * p.num_splits);
+    grid = dim3(static_cast<unsigned>(ctas));
+  }
   e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
-  if (e != cudaSuccess || p.num_splits <= 1) return e;
+  if (e != cudaSuccess || (p.num_splits <= 1 && !p.share_cap)) return e;
   const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
-  // about four splits per warp, at most kMergeMaxWarps warps per row
-  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + 3) / 4));
+  // about four records per warp, at most kMergeMaxWarps warps per row
+  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + p.share_splits + 3) / 4));
   return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
 }
 

@@ -53,14 +53,14 @@ class pa_plan_t(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
                 ("split_blocks", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("rows_per_cta", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
-                ("share_cap", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("share_cap", ctypes.c_int32), ("share_split_blocks", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {"path": {1: "single", 2: "tile", 3: "tcgen05"}.get(self.path, self.path),
                 "schedule": {1: "grid", 2: "persistent"}.get(self.schedule, self.schedule),
                 "split_blocks": self.split_blocks, "num_splits": self.num_splits,
                 "rows_per_cta": self.rows_per_cta, "num_ctas": self.num_ctas,
-                "share_cap": self.share_cap}
+                "share_cap": self.share_cap, "share_split_blocks": self.share_split_blocks}
 
     def __repr__(self):
         return f"pa_plan_t({self.as_dict()})"

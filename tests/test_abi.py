@@ -119,6 +119,9 @@ def test_plan_heuristic_host_logic(pa):
     assert p.num_splits > 1 and p.split_blocks * p.num_splits >= 8192
     # prefix sharing: a shared unit holds 32 rows = 8 sequences of 4 rows
     p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, share_prefix=True)
+    assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (2, 1, 32, 8)
+    assert pa.pa_decode_workspace_size(p, 128, 1, 32, 8, 128, 144) > 0
+    p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, share_prefix=True, schedule=pa.PA_SCHEDULE_PERSISTENT)
     assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (2, 2, 32, 8)
     with pytest.raises(pa.PAError) as exc:   # 24 rows per sequence: two do not fit 32 rows
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, share_prefix=True)
@@ -127,11 +130,28 @@ def test_plan_heuristic_host_logic(pa):
     assert (p.path, p.schedule, p.rows_per_cta) == (3, 1, 32)
     with pytest.raises(pa.PAError):          # tcgen05 runs the grid schedule only
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05, schedule=pa.PA_SCHEDULE_PERSISTENT)
-    with pytest.raises(pa.PAError):          # sharing needs the persistent schedule
-        pa.pa_decode_plan(8, 1, 32, 8, 128, 64, schedule=pa.PA_SCHEDULE_GRID, share_prefix=True)
+    with pytest.raises(pa.PAError):          # sharing runs on the mma.sync tensor-core kernel
+        pa.pa_decode_plan(8, 1, 32, 8, 128, 64, pa.PA_PATH_TCGEN05, share_prefix=True)
     forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)
     assert (forced.path, forced.split_blocks, forced.num_splits, forced.rows_per_cta) == (1, 64, 128, 8)
     # rows beyond one CTA are split into row chunks
     assert pa.pa_decode_plan(2, 16, 16, 1, 128, 8).rows_per_cta == 32
     with pytest.raises(pa.PAError):
         pa.pa_decode_plan(2, 1, 4, 2, 80, 8)
+
+
+@pytest.mark.parametrize("hints", [
+    {}, {"path": 1}, {"path": 2}, {"path": 3}, {"schedule": 2}, {"path": 1, "schedule": 2},
+    {"share_prefix": True}, {"share_prefix": True, "schedule": 2}, {"split_blocks": 3},
+    {"path": 3, "split_blocks": 2}, {"share_prefix": True, "split_blocks": 5},
+])
+def test_every_plan_passes_decode_validation(pa, hints):
+    """A plan from pa_decode_plan is accepted by pa_decode's own checks (on a machine
+    without a GPU the call then stops at the first CUDA call, never at validation)."""
+    lib = pa.raw_library()
+    B, q, hq, hkv, d, mb = 8, 1, 8, 2, 128, 40
+    plan = pa.pa_decode_plan(B, q, hq, hkv, d, mb, **hints)
+    need = pa.pa_decode_workspace_size(plan, B, q, hq, hkv, d, mb)
+    st = _decode_raw(lib, B=B, q=q, hq=hq, hkv=hkv, d=d, mb=mb, nb=400, plan=ctypes.byref(plan),
+                     ws=1 << 20, ws_bytes=need)
+    assert st not in (pa.PA_ERR_INVALID_ARG, pa.PA_ERR_UNSUPPORTED, pa.PA_ERR_WORKSPACE), (plan, st)

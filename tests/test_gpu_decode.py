@@ -42,7 +42,9 @@ PLANS = [
     ("tile_grid", dict(path=2, schedule=1)),
     ("single_persist", dict(path=1, schedule=2)),
     ("tile_persist", dict(path=2, schedule=2)),
-    ("share", dict(path=2, schedule=2, share_prefix=True)),
+    ("share", dict(path=2, share_prefix=True)),
+    ("share_persist", dict(path=2, schedule=2, share_prefix=True)),
+    ("share_split2", dict(path=2, split_blocks=2, share_prefix=True)),
     ("single_split1", dict(path=1, split_blocks=1)),
     ("tile_split1", dict(path=2, split_blocks=1)),
     ("tile_split3", dict(path=2, split_blocks=3)),
