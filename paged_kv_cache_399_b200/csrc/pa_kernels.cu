@@ -203,6 +203,7 @@ struct TileCore {
   float m_run[NT][2], l_run[NT][2];
   float o[KSTEPS][NT][4];
   int nt_active;
+  int vlim;  // largest row limit of the segment: no row sees a token past it
 
   __device__ __forceinline__ void begin(const DecodeParams& p, const Seg& s, int ctx, int lane) {
     nt_active = (s.nrows + 7) >> 3;
@@ -224,6 +225,11 @@ struct TileCore {
       m_run[nt][0] = m_run[nt][1] = -INFINITY;
       l_run[nt][0] = l_run[nt][1] = 0.f;
     }
+    int vl = lim[0][0];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) vl = max(vl, max(lim[nt][0], lim[nt][1]));
+    vl = max(vl, __shfl_xor_sync(kFull, vl, 1));
+    vlim = max(vl, __shfl_xor_sync(kFull, vl, 2));
 #pragma unroll
     for (int mt = 0; mt < KSTEPS; ++mt)
 #pragma unroll
@@ -293,6 +299,16 @@ struct TileCore {
       pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[nt][0], sc[nt][1]));
       pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[nt][2], sc[nt][3]));
     }
+    // Slots of the last block past the context may hold any bits (NaN too): their p is 0,
+    // but 0 * NaN is NaN, so their V elements are cleared in the operand fragments
+    // (a0/a1 hold tokens 2c, 2c+1 and a2/a3 tokens 2c+8, 2c+9 of the block, c = lane & 3).
+    const bool vmask = need_mask && tb + kBlockSize - 1 > vlim;
+    uint32_t vm_lo = ~0u, vm_hi = ~0u;
+    if (vmask) {
+      const int t = tb + 2 * (lane & 3);
+      vm_lo = (t <= vlim ? 0x0000FFFFu : 0u) | (t + 1 <= vlim ? 0xFFFF0000u : 0u);
+      vm_hi = (t + 8 <= vlim ? 0x0000FFFFu : 0u) | (t + 9 <= vlim ? 0xFFFF0000u : 0u);
+    }
     if (__any_sync(kFull, rescale)) {
 #pragma unroll
       for (int mt = 0; mt < KSTEPS; ++mt)
@@ -308,6 +324,12 @@ struct TileCore {
     for (int mt = 0; mt < KSTEPS; ++mt) {
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4_trans(vb + tile_chunk_offset(v_tok, 2 * mt + v_chk), a0, a1, a2, a3);
+      if (vmask) {
+        a0 &= vm_lo;
+        a1 &= vm_lo;
+        a2 &= vm_hi;
+        a3 &= vm_hi;
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         if (nt < nt_active) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
@@ -365,6 +387,7 @@ struct SimtCore {
   static constexpr bool kNeedsQSmem = true;
   float m_run[ROWS], l_run[ROWS], o[ROWS][DPL];
   int lim[ROWS];
+  int vlim;  // largest row limit of the segment: no row sees a token past it
   const float (*q_s)[D];
   float* p_w;  // this warp's [16][ROWS] probabilities
 
@@ -401,6 +424,9 @@ struct SimtCore {
 #pragma unroll
       for (int e = 0; e < DPL; ++e) o[r][e] = 0.f;
     }
+    vlim = lim[0];
+#pragma unroll
+    for (int r = 1; r < ROWS; ++r) vlim = max(vlim, lim[r]);
   }
 
   __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, int tb, bool need_mask,
@@ -469,6 +495,10 @@ struct SimtCore {
       } else {
         const uint32_t vv = *reinterpret_cast<const uint32_t*>(vrow);
         vf[0] = bf16_lo(vv); vf[1] = bf16_hi(vv);
+      }
+      if (need_mask && tb + t > vlim) {  // a slot past the context: p = 0, V may be NaN
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) vf[e] = 0.f;
       }
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {

@@ -245,6 +245,10 @@ decode_tc5_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     }
     const int lim = valid ? ctx - p.q_per_seq + qi : ctx - 1;
     const int end_tok = min(ctx, blk1 * kBlockSize);
+    // The sequence's last block, when partly filled, is in this split's tile zero_tile:
+    // its slots past the context may hold any bits (NaN too), and although their p is 0,
+    // 0 * NaN is NaN, so those V rows are cleared in shared memory before the PV reads them.
+    const int zero_tile = (blk1 == nblk && (ctx & (kBlockSize - 1))) ? (nblk - 1 - blk0) / tc5::kTileBlocks : -1;
     const float c = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
@@ -297,6 +301,21 @@ decode_tc5_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       if (t >= 1) {  // the PV of tile t-1 reads the P buffer: wait until it has completed
         ok = __all_sync(kFull, mbar_wait_bounded(&bars.p_free, (t - 1) & 1));
         if (!ok) break;
+      }
+      if (t == zero_tile) {
+        const int su = t % tc5::kStages;
+        ok = __all_sync(kFull, mbar_wait_bounded(&bars.v_full[su], (t / tc5::kStages) & 1));
+        if (!ok) break;
+        const int jj = (nblk - 1 - blk0) % tc5::kTileBlocks;
+        const int r0 = ctx & (kBlockSize - 1);  // first unwritten row of the block
+        const int nrow = kBlockSize - r0;
+        uint8_t* vblk = smem + L::offV + su * L::kKV + jj * kHalfTileBytes;
+        for (int idx = lane; idx < HALVES * nrow * 8; idx += 32) {
+          const int hf = idx / (nrow * 8);
+          const int rem = idx - hf * (nrow * 8);
+          *reinterpret_cast<uint4*>(vblk + hf * (tc5::kTileBlocks * kHalfTileBytes) +
+                                    (r0 + (rem >> 3)) * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
       }
       const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       float ps4[4] = {0.f, 0.f, 0.f, 0.f};

@@ -252,6 +252,24 @@ def check_block_permutation(oracle):
         "physical block placement changed the output"
 
 
+def check_unwritten_slots_ignored(oracle):
+    """Pool slots that no sequence sees (past a context, or in blocks no table names) may
+    hold any bits: NaN or Inf there leaves every output bit unchanged."""
+    p = Problem(seed=36, ctxs=[17, 40, 5, 33], q=2, hq=4, hkv=2, d=16, extra_blocks=4)
+    base = p.run(oracle)
+    live = np.zeros((p.nb, p.bs), dtype=bool)
+    for b, c in enumerate(p.ctxs):
+        for t in range(c):
+            live[p.tables[b, t // p.bs], t % p.bs] = True
+    assert (~live).sum() > 0
+    pk, pv = p.pool_k.copy(), p.pool_v.copy()
+    pk[~live] = np.nan
+    pv[~live] = np.inf
+    pv[~live & (np.arange(p.bs)[None, :] % 2 == 0)] = np.nan
+    assert np.array_equal(p.run(oracle, pool_k=pk, pool_v=pv), base), \
+        "a slot outside every context reached the output"
+
+
 def check_shared_prefix(oracle):
     """Two sequences sharing prefix blocks equal their unshared copies."""
     rng = np.random.default_rng(41)
@@ -370,6 +388,7 @@ ALL_CHECKS = [
     check_library_attention,
     check_closed_forms,
     check_block_permutation,
+    check_unwritten_slots_ignored,
     check_shared_prefix,
     check_gqa_equals_repeated_mha,
     check_spec_rows_equal_short_calls,

@@ -73,24 +73,71 @@ def prepared(oracle_lib):
     return out
 
 
+def _plan(w, plan_spec):
+    from paged_kv_cache_399_b200 import pa
+    if not plan_spec[1]:
+        return None
+    try:
+        plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads,
+                                 w.head_dim, w.max_blocks_per_seq, **plan_spec[1])
+    except pa.PAError as exc:
+        assert exc.status == pa.PA_ERR_UNSUPPORTED and plan_spec[1].get("share_prefix")
+        pytest.skip("prefix sharing needs G*q <= 16 rows")
+    if plan.path == pa.PA_PATH_TCGEN05:
+        assert plan.schedule == pa.PA_SCHEDULE_GRID and plan.rows_per_cta == 32
+    return plan
+
+
 @pytest.mark.parametrize("plan_spec", PLANS, ids=[p[0] for p in PLANS])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_decode_matches_oracle(case, plan_spec, prepared):
-    from paged_kv_cache_399_b200 import pa
     w, ref = prepared[case[0]]
-    plan = None
-    if plan_spec[1]:
-        try:
-            plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads,
-                                     w.head_dim, w.max_blocks_per_seq, **plan_spec[1])
-        except pa.PAError as exc:
-            assert exc.status == pa.PA_ERR_UNSUPPORTED and plan_spec[1].get("share_prefix")
-            pytest.skip("prefix sharing needs G*q <= 16 rows")
-        if plan.path == pa.PA_PATH_TCGEN05:
-            assert plan.schedule == pa.PA_SCHEDULE_GRID and plan.rows_per_cta == 32
+    plan = _plan(w, plan_spec)
     dw = DeviceWorkload(w)
     out = run_step(dw, plan)
     assert_close(out, ref, f"{case[0]}/{plan_spec[0]}")
+
+
+def _poison_unwritten(dw, w):
+    """Fill the slots of each sequence's last block that lie past its context (and that no
+    other sequence sees) with NaN in K and NaN / +Inf in V; returns how many slots."""
+    bs = 16
+    live = set()
+    for b in range(w.num_seqs):
+        for t in range(int(w.context_lens[b])):
+            live.add((int(w.block_tables[b, t // bs]), t % bs))
+    dead = set()
+    for b in range(w.num_seqs):
+        ctx = int(w.context_lens[b])
+        if ctx % bs:
+            phys = int(w.block_tables[b, (ctx - 1) // bs])
+            dead.update((phys, off) for off in range(ctx % bs, bs) if (phys, off) not in live)
+    dead = sorted(dead)
+    if not dead:
+        return 0
+    blk = torch.tensor([d[0] for d in dead], device=dw.key_cache.device)
+    off = torch.tensor([d[1] for d in dead], device=dw.key_cache.device)
+    dw.key_cache[blk, off] = float("nan")
+    dw.value_cache[blk, off] = float("nan")
+    dw.value_cache[blk[::2], off[::2]] = float("inf")
+    return len(dead)
+
+
+POISON_CASES = ["ragged", "spec6", "spec6_d64", "rows64", "long_ragged", "shared9", "shared_spec2"]
+
+
+@pytest.mark.parametrize("plan_spec", PLANS, ids=[p[0] for p in PLANS])
+@pytest.mark.parametrize("name", POISON_CASES)
+def test_unwritten_slots_do_not_leak(name, plan_spec, prepared):
+    """Slots past a sequence's context hold whatever the pool memory held. Their softmax
+    weight is exactly zero, so NaN or Inf there must leave the output unchanged (the oracle
+    reads only visible tokens, so its reference is the un-poisoned one)."""
+    w, ref = prepared[name]
+    plan = _plan(w, plan_spec)
+    dw = DeviceWorkload(w)
+    assert _poison_unwritten(dw, w) > 0
+    out = run_step(dw, plan)
+    assert_close(out, ref, f"{name}/{plan_spec[0]} poisoned")
 
 
 def test_tiny_workload_every_path(oracle_lib):
