@@ -83,7 +83,7 @@ bool encode_pool_map(CUtensorMap* map, const void* base, int64_t num_blocks, int
 // ----------------------------------------------------------------- plan
 
 int rows_per_cta_for(int path, int rows) {
-  if (path == pa::kPathTcgen05) return pa::kTc5Rows;
+  if (path == pa::kPathTcgen05) return rows <= 16 ? 16 : pa::kTcmMaxRows;
   if (path == pa::kPathTile) {
     const int r8 = static_cast<int>(ceil_div(rows, 8)) * 8;
     return r8 < pa::kTileMaxRows ? r8 : pa::kTileMaxRows;
@@ -132,7 +132,11 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     share_cap = share_cap_for(rows);
     if (share_cap < 2 || h.path == PA_PATH_SINGLE || h.path == PA_PATH_TCGEN05) return PA_ERR_UNSUPPORTED;
   }
-  if (h.path == PA_PATH_TCGEN05 && schedule != PA_SCHEDULE_GRID) return PA_ERR_UNSUPPORTED;
+  if (h.path == PA_PATH_TCGEN05) {
+    // tokens-on-M tensor-core kernel: head_dim 128, its own persistent equal-tile schedule
+    if (head_dim != 128 || h.schedule == PA_SCHEDULE_GRID) return PA_ERR_UNSUPPORTED;
+    schedule = PA_SCHEDULE_PERSISTENT;
+  }
   int path = h.path;
   if (path == PA_PATH_AUTO) path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
   // a shared-prefix unit holds share_cap sequences' rows in one CTA
@@ -151,7 +155,6 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     plan->num_splits = 1;
     return PA_OK;
   }
-  plan->share_split_blocks = 0;
   if (share_cap) {
     // the bulk of the work is the shared prefixes: at most ceil(B / cap) chunk windows
     // per kv head; cut the longest possible prefix into as many splits as fill one wave
@@ -234,8 +237,21 @@ size_t share_records(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
   return static_cast<size_t>(num_seqs) * (ssplits + plan.num_splits) * q_per_seq * num_q_heads;
 }
 
+// Workspace of the tcgen05 path: two partial records per CTA, then one piece descriptor
+// per CTA. A record holds rows_per_cta rows of O (fp32) and their (m, l) pairs.
+int32_t tcm_rec_stride(const pa_plan_t& plan, int32_t head_dim) {
+  return plan.rows_per_cta * head_dim + 2 * plan.rows_per_cta;
+}
+size_t tcm_desc_offset(const pa_plan_t& plan, int32_t head_dim) {
+  return align256(static_cast<size_t>(2) * plan.num_ctas * tcm_rec_stride(plan, head_dim) * 4);
+}
+
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
+  if (plan.path == PA_PATH_TCGEN05) {
+    if (num_seqs == 0) return 0;
+    return tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas);
+  }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (num_seqs == 0) return 0;
     return persistent_layout(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim).total;
@@ -253,8 +269,13 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
                        int32_t num_kv_heads, int32_t max_blocks_per_seq) {
   if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE && plan.path != PA_PATH_TCGEN05)
     return PA_ERR_INVALID_ARG;
-  if (plan.path == PA_PATH_TCGEN05 && plan.schedule != PA_SCHEDULE_GRID) return PA_ERR_INVALID_ARG;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
+  if (plan.path == PA_PATH_TCGEN05) {
+    if (plan.schedule != PA_SCHEDULE_PERSISTENT || plan.share_cap != 0 || plan.share_split_blocks != 0 ||
+        plan.num_ctas <= 0 || plan.num_ctas > (1 << 20) || plan.rows_per_cta != rows_per_cta_for(plan.path, rows))
+      return PA_ERR_INVALID_ARG;
+    return PA_OK;
+  }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (plan.num_ctas <= 0 || plan.num_ctas > (1 << 20)) return PA_ERR_INVALID_ARG;
     if (plan.share_split_blocks != 0) return PA_ERR_INVALID_ARG;  // grid-only field
@@ -402,7 +423,13 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   p.num_splits = plan->num_splits;
   const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
   char* ws = static_cast<char*>(workspace);
-  if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
+  if (plan->path == PA_PATH_TCGEN05) {
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+    p.num_ctas = plan->num_ctas;
+    p.rec_stride = tcm_rec_stride(*plan, head_dim);
+    p.records = reinterpret_cast<float*>(ws);
+    p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
+  } else if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
     const PersistentLayout L = persistent_layout(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
     p.num_ctas = plan->num_ctas;
     p.share_cap = plan->share_cap;

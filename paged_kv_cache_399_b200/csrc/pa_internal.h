@@ -21,7 +21,7 @@ constexpr int kSchedulePersistent = 2;
 // Largest rows one CTA holds for each family.
 constexpr int kTileMaxRows = 32;   // 4 n-tiles of 8 rows
 constexpr int kSingleMaxRows = 8;
-constexpr int kTc5Rows = 32;      // tcgen05 kernel: one softmax warp, 32 TMEM lanes
+constexpr int kTcmMaxRows = 32;   // tcgen05 kernel: query rows of a unit (the MMA's N)
 
 // Persistent schedule: header written by the pre-pass, read by the decode CTAs.
 struct SchedHeader {
@@ -64,7 +64,11 @@ struct DecodeParams {
   int32_t* arrive;               // [targets] blocks merged so far
   int32_t* list_len;             // [targets]
   int2* list;                    // [targets][list_cap] {piece start block, record slot}
-  float* records;                // [pool_cap][rec_stride]
+  float* records;                // [pool_cap][rec_stride]; tcgen05 path: [2 * num_ctas][rec_stride]
+
+  // tcgen05 path: per CTA, the unit whose first piece it holds when that unit continues
+  // in later CTAs: {record slot, last CTA with a piece, sequence, unit}, or {-1, ...}
+  int4* tc_desc;
 };
 
 // Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).

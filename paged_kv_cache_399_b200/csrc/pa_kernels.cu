@@ -1464,29 +1464,32 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
   return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
 }
 
-template <int D>
-cudaError_t launch_tc5(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+template <int N>
+cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                        cudaStream_t stream, int* occupancy) {
-  constexpr int smem = tc5::Smem<D>::kBytes;
-  auto kernel = decode_tc5_kernel<D>;
+  constexpr int smem = tcm::Smem<N>::kBytes;
+  auto kernel = decode_tcm_kernel<N>;
   static unsigned long long done_mask = 0;
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
-  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tc5::kThreads, smem);
-  const dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
-  e = launch_pdl(kernel, grid, dim3(tc5::kThreads), smem, stream, p, tk, tv);
-  if (e != cudaSuccess || p.num_splits <= 1) return e;
-  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
-  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + 3) / 4));
-  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
+  if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
+  e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kD), 0, stream, p);
 }
 
 template <int D>
 cudaError_t dispatch(int path, int schedule, int rows_per_cta, const DecodeParams& p,
                      const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, int* occ) {
   if (path == kPathTcgen05) {
-    if (schedule != kScheduleGrid || rows_per_cta != kTc5Rows) return cudaErrorInvalidValue;
-    return launch_tc5<D>(p, tk, tv, stream, occ);
+    if constexpr (D != tcm::kD) {
+      return cudaErrorInvalidValue;
+    } else {
+      if (schedule != kSchedulePersistent) return cudaErrorInvalidValue;
+      if (rows_per_cta == 16) return launch_tcm<16>(p, tk, tv, stream, occ);
+      if (rows_per_cta == 32) return launch_tcm<32>(p, tk, tv, stream, occ);
+      return cudaErrorInvalidValue;
+    }
   }
   if (path == kPathTile) {
     switch (rows_per_cta) {

@@ -1,122 +1,216 @@
-// Paged decode on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
-// Included by pa_kernels.cu (shares its helpers and device error word).
+// Paged decode on the 5th-generation tensor cores (tcgen05, accumulators in TMEM), with
+// the tokens of a tile on the MMA's M dimension. Included by pa_kernels.cu (shares its
+// helpers and device error word).
 //
-// One CTA per (kv head x row chunk, sequence, context split) of up to 32 query rows,
-// three warps with fixed roles:
-//   warp 1  TMA producer: tiles of 4 blocks (64 tokens) of K and of V, 3 stages;
-//   warp 2  MMA issuer (one thread) and TMEM owner:
-//             S_t = Q . K_t^T     M=128 (query rows, 32 used), N=64 tokens, K=head_dim
-//             O  += P_t . V_t     M=128, N=head_dim, K=64 tokens (V is an MN-major operand
-//                                 read straight from the TMA tile)
-//           completions are signalled with tcgen05.commit on mbarriers;
-//   warp 0  softmax, one thread per query row = TMEM lane: reads its row of S_t,
-//           masks, keeps a reference maximum, writes P_t (bf16) to shared memory in the
-//           128-byte-swizzled K-major layout, and rescales its row of O in TMEM only
-//           when the row maximum grows by more than 2^8 over the reference (the result
-//           is exact either way: numerator and denominator share the reference).
-// TMEM: S double buffer in columns [0,64) and [64,128), O in [128, 128+head_dim).
-// Shared memory: Q (32 rows), one P buffer, 3 stages of K and of V: 108 KB at head_dim
-// 128, so two CTAs share an SM.
-// Rows 32..127 of the A operands (Q, P) alias neighbouring shared memory: their
-// products land in TMEM lanes 32..127, which nobody reads.
+// Work. A unit is (sequence, kv head, row chunk of N query rows); its blocks are cut into
+// tiles of 8 blocks = 128 tokens. All units' tiles, in (sequence, kv head, row chunk)
+// order, are split into equal contiguous ranges, one per CTA of a persistent grid; each
+// CTA finds its range from context_lens itself (no pre-pass). A unit cut by a range
+// boundary leaves partial records, combined afterwards by tcm_merge_kernel.
+//
+// Per tile, with Q of the unit's N (16 or 32) rows:
+//   S^T[128 tok][N]  = K[128 tok][D] . Q^T[D][N]           tcgen05.mma M=128, K-major A and B
+//   softmax over the tile's 128 tokens: thread t of the softmax warpgroup owns token t
+//   (TMEM lane t) and all N columns; the column maxima are reduced across the 128
+//   threads, and the running reference maximum of a column moves only when the tile
+//   maximum exceeds it by more than 2^8 (the output is exact either way, since
+//   numerator and denominator share the reference);
+//   O^T[D][N] += V^T[D][128 tok] . P^T[128 tok][N]         tcgen05.mma M=D=128, MN-major A
+//                                                          (the TMA tile) and B (P^T)
+// Roles: warps 0-3 softmax and epilogue (TMEM lanes 0..127), warp 4 TMA producer and Q
+// loads, warp 5 MMA issuer (one thread) and TMEM owner. The issuer polls both of its
+// inputs and issues whichever MMA is ready: the S of the next tile once its K has
+// landed, the PV of the oldest tile once its P^T is written; a K stage is released
+// when its S completes, a V stage when its PV completes.
+// TMEM columns: S double buffer [0, 2N), O double buffer (by unit parity) [2N, 4N).
+// Shared memory: 2 Q buffers, 2 P^T buffers, 3 stages of K and of V (32 KB each).
 
 namespace pa {
-namespace tc5 {
+namespace tcm {
 
-constexpr int kTileBlocks = 4;
-constexpr int kTileTokens = kTileBlocks * kBlockSize;  // 64
+constexpr int kD = 128;
+constexpr int kTileBlocks = 8;
+constexpr int kTileTokens = kTileBlocks * kBlockSize;   // 128
 constexpr int kStages = 3;
-constexpr int kRows = 32;          // query rows per CTA: the softmax warp's 32 TMEM lanes
-constexpr int kThreads = 96;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
+constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
+constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
 
-template <int D>
+template <int N>
 struct Smem {
-  static constexpr int kHalves = D / 64;
-  static constexpr int kQ = kHalves * 4096;              // rows 0..31 of each 64-column half
-  static constexpr int kP = 4096;                        // rows 0..31 x 64 tokens
-  static constexpr int kKV = kTileBlocks * kHalves * kHalfTileBytes;  // one K or V stage
+  static constexpr int kQ = 2 * N * 128;             // 2 halves x N rows x 128 B, 128-B swizzle
+  static constexpr int kP = (N / 8) * kPGroupBytes;  // 128 tokens x N bf16, core matrices
   static constexpr int offQ = 0;
-  static constexpr int offP = kQ;
-  static constexpr int offK = offP + kP;
-  static constexpr int offV = offK + kStages * kKV;
-  static constexpr int kUsed = offV + kStages * kKV;
-  static constexpr int offBars = kUsed;                  // barriers, TMEM address, flags
-  // no static shared memory: the dynamic buffer starts at the (1024-aligned) base of the
-  // CTA's window, so two 113 KB CTAs fit an SM; at least 77 KB so that no more than two
-  // CTAs (2 x 256 TMEM columns) share an SM and a TMEM allocation never waits
-  static constexpr int kBytes = (kUsed + 256) > 77 * 1024 ? (kUsed + 256) : 77 * 1024;
-  // descriptors of Q and P span 128 rows = 16 KB from their start: stay inside
-  static_assert(offQ + (kHalves - 1) * 4096 + 16384 <= kUsed, "Q rows 32..127 must alias allocated smem");
-  static_assert(offP + kP + 16384 <= kUsed, "P rows 32..127 must alias allocated smem");
+  static constexpr int offP = offQ + 2 * kQ;
+  static constexpr int offK = offP + 2 * kP;
+  static constexpr int offV = offK + kStages * kStageBytes;
+  static constexpr int offRed = offV + kStages * kStageBytes;  // [3][4 warps][32] floats
+  static constexpr int offScan = offRed + 3 * 4 * 32 * 4;      // [8] int64, then the start
+  static constexpr int offBars = offScan + 128;
+  static constexpr int kBytes = offBars + 256;
+  static_assert(offK % 1024 == 0 && kQ % 1024 == 0, "swizzled operands need 1024-B alignment");
 };
 
 struct Bars {
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full, p_free;
-  uint64_t q_full, o_final, drain;
+  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t drain;
 };
 
-}  // namespace tc5
-
-template <int D>
-__global__ void __launch_bounds__(tc5::kThreads)
-decode_tc5_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v) {
-  using L = tc5::Smem<D>;
-  constexpr int HALVES = D / 64;
-  constexpr int KSTEPS = D / 16;
-  constexpr int DC = D / 32;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  static_assert(sizeof(tc5::Bars) + 8 <= 256, "barrier area");
-  tc5::Bars& bars = *reinterpret_cast<tc5::Bars*>(smem + L::offBars);
-  uint32_t& tmem_base_s = *reinterpret_cast<uint32_t*>(smem + L::offBars + sizeof(tc5::Bars));
-  int& abort_s = *reinterpret_cast<int*>(smem + L::offBars + sizeof(tc5::Bars) + 4);
-  if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1024-aligned base
-    if (threadIdx.x == 0) record_error(kErrSchedule);
-    return;
+// Position in the CTA's tile range: sequence b, unit k (kv head x row chunk) of it,
+// tile x of the unit.
+struct Walk {
+  int b, k, x, ctx, nblk, tiles;
+  __device__ __forceinline__ void seq(const DecodeParams& p) {
+    ctx = b < p.num_seqs ? __ldg(p.context_lens + b) : 0;
+    nblk = num_blocks_of(p, ctx);
+    ctx = min(ctx, nblk * kBlockSize);
+    tiles = (nblk + kTileBlocks - 1) / kTileBlocks;
   }
+  __device__ __forceinline__ void next(const DecodeParams& p, int upb) {
+    if (++x < tiles) return;
+    x = 0;
+    if (++k < upb) return;
+    k = 0;
+    do {
+      ++b;
+      seq(p);
+    } while (tiles == 0 && b < p.num_seqs);
+  }
+};
+
+__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Column reduction of a warp: lane l holds V values (columns 0..V-1); on return every
+// lane holds the reduction over all 32 lanes of column (l % V). Halving exchange: at
+// each step a lane keeps the half of its columns selected by one lane bit and sends
+// the other half to the partner lane (31 shuffles for V = 32).
+template <int V, bool kMax>
+__device__ __forceinline__ float column_reduce(float (&v)[V], int lane) {
+#pragma unroll
+  for (int h = V / 2; h >= 1; h >>= 1) {
+    const bool upper = (lane & h) != 0;
+#pragma unroll
+    for (int k = 0; k < h; ++k) {
+      const float send = upper ? v[k] : v[k + h];
+      const float keep = upper ? v[k + h] : v[k];
+      const float got = __shfl_xor_sync(kFull, send, h);
+      v[k] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int o = V; o < 32; o <<= 1) {
+    const float got = __shfl_xor_sync(kFull, r, o);
+    r = kMax ? fmaxf(r, got) : r + got;
+  }
+  return r;
+}
+
+}  // namespace tcm
+
+template <int N>
+__global__ void __launch_bounds__(tcm::kThreads, 1)
+decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v) {
+  using L = tcm::Smem<N>;
+  using tcm::kStages;
+  using tcm::kTileBlocks;
+  using tcm::kTileTokens;
+  constexpr int D = tcm::kD;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  static_assert(sizeof(tcm::Bars) + 16 <= 256, "barrier area");
+  tcm::Bars& bars = *reinterpret_cast<tcm::Bars*>(smem + L::offBars);
+  uint32_t& tmem_base_s = *reinterpret_cast<uint32_t*>(smem + L::offBars + sizeof(tcm::Bars));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x / p.row_chunks;
-  const int rc = blockIdx.x % p.row_chunks;
-  const int b = blockIdx.y;
-  const int split = blockIdx.z;
-
+  const int c = blockIdx.x;
+  if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1024-aligned base
+    if (threadIdx.x == 0) {
+      record_error(kErrSchedule);
+      p.tc_desc[c] = make_int4(-1, 0, 0, 0);
+    }
+    return;
+  }
   if (threadIdx.x == 0) {
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
-    for (int i = 0; i < static_cast<int>(sizeof(tc5::Bars) / 8); ++i) mbar_init(all + i, 1);
+    for (int i = 0; i < static_cast<int>(sizeof(tcm::Bars) / 8); ++i) mbar_init(all + i, 1);
+    for (int i = 0; i < 2; ++i) {  // one arrival per softmax warp
+      mbar_init(&bars.s_free[i], 4);
+      mbar_init(&bars.p_full[i], 4);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
-    abort_s = 0;
   }
-  __syncthreads();
   grid_dependency_wait();
 
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = num_blocks_of(p, ctx);
-  const int blk0 = split * p.split_blocks;
-  const Seg sg{b, 1, kvh, rc * tc5::kRows, min(tc5::kRows, p.rows - rc * tc5::kRows), blk0,
-               min(nblk, blk0 + p.split_blocks), false};
-  if (blk0 >= nblk) {  // uniform: nothing to read
-    if (split == 0 && warp == 0) {
-      int bb, i, h;
-      if (seg_row(p, sg, lane, bb, i, h)) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + out_offset(p, bb, i, h, D));
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+  // ---- this CTA's tile range [t0, t1) of W tiles: prefix sums over the sequences
+  const int upb = p.num_kv_heads * p.row_chunks;  // units per sequence
+  long long* wsum = reinterpret_cast<long long*>(smem + L::offScan);
+  int* start = reinterpret_cast<int*>(smem + L::offScan + 64);
+  long long W, t0, t1;
+  int G;  // CTAs that take part: at most one per tile, so that every range is non-empty
+  {
+    const int B = p.num_seqs;
+    const int chunk = (B + tcm::kThreads - 1) / tcm::kThreads;
+    const int s0 = min(B, static_cast<int>(threadIdx.x) * chunk), s1 = min(B, s0 + chunk);
+    long long local = 0;
+    for (int b = s0; b < s1; ++b) {
+      const int nb = num_blocks_of(p, __ldg(p.context_lens + b));
+      local += static_cast<long long>((nb + kTileBlocks - 1) / kTileBlocks) * upb;
+    }
+    long long v = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long nv = __shfl_up_sync(kFull, v, o);
+      if (lane >= o) v += nv;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    long long base = 0;
+    W = 0;
+    for (int w2 = 0; w2 < tcm::kThreads / 32; ++w2) {
+      if (w2 < warp) base += wsum[w2];
+      W += wsum[w2];
+    }
+    G = static_cast<int>(min(static_cast<long long>(gridDim.x), W));
+    t0 = c < G ? static_cast<long long>(c) * W / G : 0;
+    t1 = c < G ? static_cast<long long>(c + 1) * W / G : 0;
+    const long long excl = base + v - local;
+    if (local > 0 && t0 < t1 && t0 >= excl && t0 < excl + local) {
+      long long acc = excl;
+      for (int b = s0; b < s1; ++b) {
+        const int nb = num_blocks_of(p, __ldg(p.context_lens + b));
+        const long long tb = static_cast<long long>((nb + kTileBlocks - 1) / kTileBlocks) * upb;
+        if (t0 < acc + tb) {
+          start[0] = b;
+          start[1] = static_cast<int>(t0 - acc);
+          break;
+        }
+        acc += tb;
       }
     }
+    __syncthreads();
+  }
+  const int n = static_cast<int>(t1 - t0);
+  if (n <= 0) {  // uniform: no tiles for this CTA
+    if (threadIdx.x == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     grid_launch_dependents();
     return;
   }
-  const int blk1 = sg.blk1;
-  const int ntiles = (blk1 - blk0 + tc5::kTileBlocks - 1) / tc5::kTileBlocks;
-  const bool single_split = (nblk + p.split_blocks - 1) / p.split_blocks == 1;
+  tcm::Walk w0;
+  w0.b = start[0];
+  w0.seq(p);
+  w0.k = start[1] / w0.tiles;
+  w0.x = start[1] - w0.k * w0.tiles;
 
-  if (warp == 2) {
-    tmem_alloc(&tmem_base_s, tc5::kTmemCols);
+  if (warp == tcm::kMmaWarp) {
+    tmem_alloc(&tmem_base_s, 4 * N < 32 ? 32 : 4 * N);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -124,261 +218,418 @@ decode_tc5_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   tc_fence_after_sync();
   const uint32_t tmem = tmem_base_s;
   const uint32_t sm = smem_u32(smem);
-  const uint32_t q_s = sm + L::offQ;
-  const uint32_t p_s = sm + L::offP;
-  const uint32_t k_s = sm + L::offK;
-  const uint32_t v_s = sm + L::offV;
 
-  if (warp == 1) {
-    // ------------------------------------------------------------ TMA producer
-    const int32_t* trow = p.block_tables + static_cast<size_t>(b) * p.max_blocks;
+  if (warp == tcm::kProducerWarp) {
+    // ------------------------------------------------------------ TMA producer + Q
+    // Lanes 0..15 issue the tile's 16 boxes of K (half = lane / 8, block = lane % 8),
+    // then of V; lanes 0..7 load the next tile's block ids while this one is issued.
+    tcm::Walk w = w0;
     const int oob = static_cast<int>(p.num_blocks);  // block id past the pool: TMA fills zeros
-    int t = 0;
-    for (; t < ntiles; ++t) {
-      const int s = t % tc5::kStages;
-      if (t >= tc5::kStages) {
-        const bool ok = mbar_wait_bounded(&bars.kv_empty[s], ((t / tc5::kStages) - 1) & 1);
-        if (!__all_sync(kFull, ok)) {
-          if (lane == 0) record_error(kErrTimeoutDecode);
-          abort_s = 1;
-          break;
-        }
-      }
-      // lanes 0..3 read the tile's 4 block ids; blocks past the split use an id past the
-      // pool, which the TMA fills with zeros
-      const int blk = blk0 + t * tc5::kTileBlocks + lane;
-      const int phys_l = (lane < tc5::kTileBlocks && blk < blk1) ? __ldg(trow + blk) : oob;
-      int ph[tc5::kTileBlocks];
-#pragma unroll
-      for (int jj = 0; jj < tc5::kTileBlocks; ++jj) ph[jj] = __shfl_sync(kFull, phys_l, jj);
-      if (lane == 0) {
-        uint8_t* kdst = smem + L::offK + s * L::kKV;
-        uint8_t* vdst = smem + L::offV + s * L::kKV;
-        mbar_arrive_expect_tx(&bars.k_full[s], L::kKV);
-        mbar_arrive_expect_tx(&bars.v_full[s], L::kKV);
-#pragma unroll
-        for (int jj = 0; jj < tc5::kTileBlocks; ++jj)
-#pragma unroll
-          for (int hf = 0; hf < HALVES; ++hf) {
-            const int off = hf * (tc5::kTileBlocks * kHalfTileBytes) + jj * kHalfTileBytes;
-            tma_load_3d(kdst + off, &tmap_k, &bars.k_full[s], hf * 64, kvh, ph[jj] * kBlockSize);
-            tma_load_3d(vdst + off, &tmap_v, &bars.v_full[s], hf * 64, kvh, ph[jj] * kBlockSize);
-          }
-      }
-      __syncwarp();
-    }
-    if (abort_s) {  // wait (bounded) for the loads still in flight before leaving
-      for (int u = max(0, t - tc5::kStages); u < t; ++u) {
-        const int s = u % tc5::kStages;
-        if (!mbar_wait_bounded(&bars.k_full[s], (u / tc5::kStages) & 1) ||
-            !mbar_wait_bounded(&bars.v_full[s], (u / tc5::kStages) & 1))
-          record_error(kErrTimeoutDrain);
-      }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, tc5::kTileTokens, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
-      bool ok = mbar_wait_bounded(&bars.q_full, 0);
-      for (int t = 0; ok && t <= ntiles; ++t) {
-        if (t < ntiles) {
-          const int s = t % tc5::kStages;
-          ok = mbar_wait_bounded(&bars.k_full[s], (t / tc5::kStages) & 1);
-          if (ok && t >= 2) ok = mbar_wait_bounded(&bars.s_free[t & 1], ((t >> 1) - 1) & 1);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t kst = k_s + s * L::kKV;
-#pragma unroll
-          for (int k = 0; k < KSTEPS; ++k) {
-            const uint64_t ad = smem_desc_sw128(q_s + (k >> 2) * 4096 + (k & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kst + (k >> 2) * (tc5::kTileBlocks * kHalfTileBytes) +
-                                                    (k & 3) * 32, 16, 1024);
-            tc_mma_bf16(tmem + (t & 1) * tc5::kTileTokens, ad, bd, idesc_s, k > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars.s_full[t & 1]);
-        }
-        if (t >= 1) {
-          const int u = t - 1;
-          const int su = u % tc5::kStages;
-          ok = mbar_wait_bounded(&bars.p_full, u & 1);
-          if (ok) ok = mbar_wait_bounded(&bars.v_full[su], (u / tc5::kStages) & 1);
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t vst = v_s + su * L::kKV;
-#pragma unroll
-          for (int kk = 0; kk < tc5::kTileTokens / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(p_s + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(vst + kk * 2048, tc5::kTileBlocks * kHalfTileBytes, 1024);
-            tc_mma_bf16(tmem + 128, ad, bd, idesc_o, (u > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&bars.p_free);
-          tc_commit(&bars.kv_empty[su]);
-        }
-      }
-      if (!ok) {
-        record_error(kErrTimeoutDecode);
-        abort_s = 1;
-      }
-      tc_commit(&bars.o_final);
-      // every MMA issued so far has completed once o_final flips
-      if (!mbar_wait_bounded(&bars.o_final, 0)) record_error(kErrTimeoutDrain);
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax (warp 0)
-    const int r = lane;
-    int bb = 0, qi = 0, qh = 0;
-    const bool valid = seg_row(p, sg, r, bb, qi, qh);
-    {  // Q row r -> shared memory (128-byte swizzle, K-major), zeros for padded rows
-      const uint4* qsrc = reinterpret_cast<const uint4*>(p.query + out_offset(p, bb, qi, qh, D));
-#pragma unroll
-      for (int hf = 0; hf < HALVES; ++hf)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = valid ? __ldg(qsrc + hf * 8 + c) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(smem + L::offQ + hf * 4096 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
-        }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.q_full);
-    }
-    const int lim = valid ? ctx - p.q_per_seq + qi : ctx - 1;
-    const int end_tok = min(ctx, blk1 * kBlockSize);
-    // The sequence's last block, when partly filled, is in this split's tile zero_tile:
-    // its slots past the context may hold any bits (NaN too), and although their p is 0,
-    // 0 * NaN is NaN, so those V rows are cleared in shared memory before the PV reads them.
-    const int zero_tile = (blk1 == nblk && (ctx & (kBlockSize - 1))) ? (nblk - 1 - blk0) / tc5::kTileBlocks : -1;
-    const float c = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
+    auto block_id = [&](const tcm::Walk& at) {
+      const int blk = at.x * kTileBlocks + lane;
+      return (lane < kTileBlocks && blk < at.nblk)
+                 ? __ldg(p.block_tables + static_cast<size_t>(at.b) * p.max_blocks + blk)
+                 : oob;
+    };
+    int phys_next = block_id(w);
+    int j = -1, g = 0;
     bool ok = true;
-    for (int t = 0; t < ntiles && ok; ++t) {
-      ok = __all_sync(kFull, mbar_wait_bounded(&bars.s_full[t & 1], (t >> 1) & 1));
-      if (!ok) break;
-      tc_fence_after_sync();
-      uint32_t sv[tc5::kTileTokens];
-      tmem_ld32(tmem + (t & 1) * tc5::kTileTokens, *reinterpret_cast<uint32_t(*)[32]>(sv));
-      tmem_ld32(tmem + (t & 1) * tc5::kTileTokens + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-      tc_wait_ld();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[t & 1]);
-
-      const int tok0 = (blk0 + t * tc5::kTileBlocks) * kBlockSize;
-      const bool edge = tok0 + tc5::kTileTokens > min(end_tok, ctx - p.q_per_seq + 1);
-      float x[tc5::kTileTokens];
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 independent chains
+    for (; g < n; ++g) {
+      if (g == 0 || w.x == 0) {
+        ++j;
+        if (j >= 2) ok = __all_sync(kFull, mbar_wait_bounded(&bars.q_empty[j & 1], ((j >> 1) - 1) & 1));
+        if (!ok) break;
+        // Q rows of the unit -> Q[j & 1], 128-byte swizzled K-major; zeros for padded rows
+        const int kvh = w.k / p.row_chunks;
+        const int rc = w.k - kvh * p.row_chunks;
+        const int nrows = min(N, p.rows - rc * N);
+        uint8_t* qb = smem + L::offQ + (j & 1) * L::kQ;
+        if (lane < N) {
+          const int r = lane;
+          const bool valid = r < nrows;
+          const int rr = rc * N + r;
+          const int i = valid ? rr / p.group : 0;
+          const int gg = valid ? rr - i * p.group : 0;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.query + (static_cast<size_t>(w.b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D);
 #pragma unroll
-      for (int j = 0; j < tc5::kTileTokens; ++j) {
-        float v = __uint_as_float(sv[j]) * c;
-        if (edge && (tok0 + j >= end_tok || tok0 + j > lim)) v = -INFINITY;
-        x[j] = v;
-        mx4[j & 3] = fmaxf(mx4[j & 3], v);
-      }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const bool need = mx > m_ref + tc5::kRescaleLog2 || (m_ref == -INFINITY && mx != -INFINITY);
-      if (__any_sync(kFull, need)) {
-        const float new_ref = need ? mx : m_ref;
-        const float alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - new_ref);
-        l *= alpha;
-        if (t > 0) {  // O holds tiles 0..t-1 once the PV of tile t-1 has completed
-          ok = __all_sync(kFull, mbar_wait_bounded(&bars.p_free, (t - 1) & 1));
-          if (!ok) break;
-          tc_fence_after_sync();
-#pragma unroll
-          for (int ch = 0; ch < DC; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tmem + 128 + ch * 32, o);
-            tc_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tmem + 128 + ch * 32, o);
+          for (int ch = 0; ch < D / 8; ++ch) {
+            const uint4 v = valid ? __ldg(src + ch) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(qb + (ch >> 3) * (N * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v;
           }
-          tc_wait_st();
         }
-        m_ref = new_ref;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_full[j & 1]);
       }
-      if (t >= 1) {  // the PV of tile t-1 reads the P buffer: wait until it has completed
-        ok = __all_sync(kFull, mbar_wait_bounded(&bars.p_free, (t - 1) & 1));
-        if (!ok) break;
-      }
-      if (t == zero_tile) {
-        const int su = t % tc5::kStages;
-        ok = __all_sync(kFull, mbar_wait_bounded(&bars.v_full[su], (t / tc5::kStages) & 1));
-        if (!ok) break;
-        const int jj = (nblk - 1 - blk0) % tc5::kTileBlocks;
-        const int r0 = ctx & (kBlockSize - 1);  // first unwritten row of the block
-        const int nrow = kBlockSize - r0;
-        uint8_t* vblk = smem + L::offV + su * L::kKV + jj * kHalfTileBytes;
-        for (int idx = lane; idx < HALVES * nrow * 8; idx += 32) {
-          const int hf = idx / (nrow * 8);
-          const int rem = idx - hf * (nrow * 8);
-          *reinterpret_cast<uint4*>(vblk + hf * (tc5::kTileBlocks * kHalfTileBytes) +
-                                    (r0 + (rem >> 3)) * 128 + (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float ps4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[tc5::kTileTokens / 2];
-#pragma unroll
-      for (int j = 0; j < tc5::kTileTokens; j += 2) {
-        const float p0 = fast_exp2(x[j] - mref_use);
-        const float p1 = fast_exp2(x[j + 1] - mref_use);
-        ps4[(j >> 1) & 3] += p0 + p1;
-        pk[j / 2] = pack_bf16x2(p0, p1);
-      }
-      l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-      uint8_t* prow = smem + L::offP + r * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before_sync();
+      const int s = g % kStages;
+      const int kvh = w.k / p.row_chunks;
+      const int ph = __shfl_sync(kFull, phys_next, lane & (kTileBlocks - 1));
+      tcm::Walk wn = w;
+      wn.next(p, upb);
+      if (g + 1 < n) phys_next = block_id(wn);
+      const int hf = lane >> 3, jj = lane & (kTileBlocks - 1);
+      const uint32_t box = hf * tcm::kHalfBytes + jj * kHalfTileBytes;
+      if (g >= kStages) ok = __all_sync(kFull, mbar_wait_bounded(&bars.k_empty[s], ((g / kStages) - 1) & 1));
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&bars.k_full[s], tcm::kStageBytes);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
+      if (lane < 2 * kTileBlocks)
+        tma_load_3d(smem + L::offK + s * tcm::kStageBytes + box, &tmap_k, &bars.k_full[s], hf * 64, kvh,
+                    ph * kBlockSize);
+      if (g >= kStages) ok = __all_sync(kFull, mbar_wait_bounded(&bars.v_empty[s], ((g / kStages) - 1) & 1));
+      if (!ok) {
+        ++g;  // this tile's K load is in flight: drain it below
+        break;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&bars.v_full[s], tcm::kStageBytes);
+      __syncwarp();
+      if (lane < 2 * kTileBlocks)
+        tma_load_3d(smem + L::offV + s * tcm::kStageBytes + box, &tmap_v, &bars.v_full[s], hf * 64, kvh,
+                    ph * kBlockSize);
+      __syncwarp();
+      w = wn;
     }
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
-      abort_s = 1;
-    }
-    // epilogue: wait for the last PV, then O row r -> output or partial record
-    const bool done = __all_sync(kFull, mbar_wait_bounded(&bars.o_final, 0));
-    tc_fence_after_sync();
-    if (!done) record_error(kErrTimeoutDecode);
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const int rq = qi * p.num_q_heads + qh;
-    const size_t rec = (static_cast<size_t>(b) * p.num_splits + split) * (p.q_per_seq * p.num_q_heads) + rq;
-#pragma unroll
-    for (int ch = 0; ch < DC; ++ch) {
-      uint32_t o[32];
-      tmem_ld32(tmem + 128 + ch * 32, o);
-      tc_wait_ld();
-      if (!valid || !done) continue;
-      if (single_split) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + out_offset(p, bb, qi, qh, D) + ch * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float a[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(o[q4 * 8 + e]);
-          store_bf16x8(reinterpret_cast<uint16_t*>(dst + q4), a, inv);
+      // wait (bounded) for the loads still in flight before leaving (a tile whose V was
+      // not issued has only its K pending: waiting on its V times out harmlessly)
+      for (int u = max(0, g - kStages); u < g; ++u) {
+        const int s = u % kStages;
+        if (!mbar_wait_bounded(&bars.k_full[s], (u / kStages) & 1)) {
+          if (lane == 0) record_error(kErrTimeoutDrain);
         }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + ch * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
-                                __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+        mbar_wait_bounded(&bars.v_full[s], (u / kStages) & 1);
       }
     }
-    if (valid && done && !single_split) p.ws_ml[rec] = make_float2(m_ref, l);
+  } else if (warp == tcm::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, N, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, N, 1, 1);
+      tcm::Walk w = w0;      // position of the next S
+      int js = -1;           // unit counter of the S issued last
+      int gs = 0, gp = 0;    // next tile to issue S for / PV for (gp <= gs <= gp + 3)
+      int ring = 0;          // per tile in flight: bit 2(g&3) O buffer, bit 2(g&3)+1 first of unit
+      bool ok = true;
+      unsigned long long idle_since = 0;
+      while (gp < n) {
+        bool progressed = false;
+        if (gs < n && gs - gp < 3) {
+          const bool first = gs == 0 || w.x == 0;
+          const int jn = first ? js + 1 : js;
+          const int s = gs % kStages;
+          if ((!first || mbar_test_wait(&bars.q_full[jn & 1], (jn >> 1) & 1)) &&
+              mbar_test_wait(&bars.k_full[s], (gs / kStages) & 1) &&
+              (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1))) {
+            js = jn;
+            const int obuf = js & 1;
+            const bool last = gs == n - 1 || w.x == w.tiles - 1;
+            tc_fence_after_sync();
+            const uint32_t kst = sm + L::offK + s * tcm::kStageBytes;
+            const uint32_t qst = sm + L::offQ + obuf * L::kQ;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(kst + (k >> 2) * tcm::kHalfBytes + (k & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(qst + (k >> 2) * (N * 128) + (k & 3) * 32, 16, 1024);
+              tc_mma_bf16(tmem + (gs & 1) * N, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars.s_full[gs & 1]);
+            tc_commit(&bars.k_empty[s]);
+            if (last) tc_commit(&bars.q_empty[obuf]);
+            const int sh = 2 * (gs & 3);
+            ring = (ring & ~(3 << sh)) | (obuf << sh) | ((first ? 1 : 0) << (sh + 1));
+            w.next(p, upb);
+            ++gs;
+            progressed = true;
+          }
+        }
+        if (gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
+            mbar_test_wait(&bars.v_full[gp % kStages], (gp / kStages) & 1)) {
+          const int sh = 2 * (gp & 3);
+          const int obuf = (ring >> sh) & 1;
+          const bool first = (ring >> (sh + 1)) & 1;
+          tc_fence_after_sync();
+          const uint32_t vst = sm + L::offV + (gp % kStages) * tcm::kStageBytes;
+          const uint32_t pst = sm + L::offP + (gp & 1) * L::kP;
+#pragma unroll
+          for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(vst + kk * 2048, tcm::kHalfBytes, 1024);
+            const uint64_t bd = smem_desc_noswizzle(pst + kk * 256, 128, tcm::kPGroupBytes);
+            tc_mma_bf16(tmem + 2 * N + obuf * N, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&bars.pv_done[gp & 1]);
+          tc_commit(&bars.v_empty[gp % kStages]);
+          ++gp;
+          progressed = true;
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const unsigned long long now = global_timer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!ok) record_error(kErrTimeoutDecode);
+      tc_commit(&bars.drain);  // every MMA issued so far has completed once drain flips
+      if (!mbar_wait_bounded(&bars.drain, 0)) record_error(kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = threadIdx.x;  // token of the tile = TMEM lane = head-dim index in O^T
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + L::offRed);
+    const float cs = p.scale_log2;
+    tcm::Walk w = w0;
+    int j = -1, first_x = 0, kvh = 0, rc = 0, nrows = 0, minlim = 0;
+    float mref_c = -INFINITY;  // reference maximum of column (lane % N)
+    float mref[N], lpart[N];
+    int lim[N];
+    // A bounded wait that gives up makes `ok` false for good: the later waits are skipped
+    // and nothing more is written to global memory, but every warp still passes every
+    // named barrier, so none of the four is left waiting for the others.
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFull, mbar_wait_bounded(bar, parity));
+    };
+    for (int g = 0; g < n; ++g) {
+      const bool first = g == 0 || w.x == 0;
+      const bool last = g == n - 1 || w.x == w.tiles - 1;
+      if (first) {
+        ++j;
+        first_x = w.x;
+        kvh = w.k / p.row_chunks;
+        rc = w.k - kvh * p.row_chunks;
+        nrows = min(N, p.rows - rc * N);
+        int i = (rc * N) / p.group, gg = rc * N - i * p.group;
+        minlim = w.ctx - p.q_per_seq + i;
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+          lim[r] = r < nrows ? w.ctx - p.q_per_seq + i : w.ctx - 1;
+          if (++gg == p.group) {
+            gg = 0;
+            ++i;
+          }
+          mref[r] = -INFINITY;
+          lpart[r] = 0.f;
+        }
+        mref_c = -INFINITY;
+      }
+      // ---- S^T of this tile: the N scores of token t
+      wait(&bars.s_full[g & 1], (g >> 1) & 1);
+      tc_fence_after_sync();
+      uint32_t sv[N];
+      tmem_ld<N>(tmem + lane_off + (g & 1) * N, sv);
+      tc_wait_ld();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.s_free[g & 1]);
+      const int tok = w.x * kTileTokens + t;
+      const bool edge = w.x * kTileTokens + kTileTokens - 1 > minlim;
+      float x[N], tmp[N];
+#pragma unroll
+      for (int r = 0; r < N; ++r) {
+        float v = __uint_as_float(sv[r]) * cs;
+        if (edge && tok > lim[r]) v = -INFINITY;
+        x[r] = v;
+        tmp[r] = v;
+      }
+      // ---- column maxima over the 128 tokens
+      const float wmax = tcm::column_reduce<N, true>(tmp, lane);
+      float* rb = red + (g & 1) * 128;
+      if (lane < N) rb[warp * 32 + lane] = wmax;
+      tcm::named_sync_softmax();
+      const int jc = lane % N;
+      const float M = fmaxf(fmaxf(rb[jc], rb[32 + jc]), fmaxf(rb[64 + jc], rb[96 + jc]));
+      const bool need = M > mref_c + tcm::kRescaleLog2 || (mref_c == -INFINITY && M != -INFINITY);
+      if (__any_sync(kFull, need)) {  // the same decision in all four warps
+        const float nm = need ? M : mref_c;
+        const float alpha_c = need ? (mref_c == -INFINITY ? 0.f : fast_exp2(mref_c - nm)) : 1.f;
+        mref_c = nm;
+        float alpha[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+          mref[r] = __shfl_sync(kFull, mref_c, r);
+          alpha[r] = __shfl_sync(kFull, alpha_c, r);
+          lpart[r] *= alpha[r];
+        }
+        if (!first) {  // O holds this unit's earlier tiles once the PV of tile g-1 is done
+          wait(&bars.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1);
+          tc_fence_after_sync();
+          uint32_t ov[N];
+          const uint32_t oaddr = tmem + lane_off + 2 * N + (j & 1) * N;
+          tmem_ld<N>(oaddr, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int r = 0; r < N; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
+          tmem_st<N>(oaddr, ov);
+          tc_wait_st();
+        }
+      }
+      // ---- probabilities, bf16 pairs (column 2q in the low half)
+      uint32_t pk[N / 2];
+#pragma unroll
+      for (int r = 0; r < N; r += 2) {
+        const float p0 = fast_exp2(x[r] - (mref[r] == -INFINITY ? 0.f : mref[r]));
+        const float p1 = fast_exp2(x[r + 1] - (mref[r + 1] == -INFINITY ? 0.f : mref[r + 1]));
+        lpart[r] += p0;
+        lpart[r + 1] += p1;
+        pk[r / 2] = pack_bf16x2(p0, p1);
+      }
+      // the P^T buffer of this tile was read by the PV of tile g-2
+      if (g >= 2) wait(&bars.pv_done[g & 1], ((g >> 1) - 1) & 1);
+      if (w.x == w.tiles - 1 && (w.ctx & (kBlockSize - 1))) {
+        // The sequence's last block is partly filled: its slots past the context may hold
+        // any bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows
+        // are cleared before the PV reads them.
+        const int s = g % kStages;
+        wait(&bars.v_full[s], (g / kStages) & 1);
+        const int jj = (w.nblk - 1) - w.x * kTileBlocks;
+        const int r0 = w.ctx & (kBlockSize - 1);
+        const int nrow = kBlockSize - r0;
+        uint8_t* vblk = smem + L::offV + s * tcm::kStageBytes + jj * kHalfTileBytes;
+        for (int idx = t; idx < 2 * nrow * 8; idx += 128) {
+          const int hf = idx / (nrow * 8);
+          const int rem = idx - hf * (nrow * 8);
+          *reinterpret_cast<uint4*>(vblk + hf * tcm::kHalfBytes + (r0 + (rem >> 3)) * 128 + (rem & 7) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+      uint8_t* pb = smem + L::offP + (g & 1) * L::kP;
+#pragma unroll
+      for (int q8 = 0; q8 < N / 8; ++q8)
+        *reinterpret_cast<uint4*>(pb + q8 * tcm::kPGroupBytes + t * 16) =
+            make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full[g & 1]);
+
+      if (last) {
+        // ---- epilogue of the unit's piece: wait for its last PV, then O^T / l
+        wait(&bars.pv_done[g & 1], (g >> 1) & 1);
+        tc_fence_after_sync();
+        float ls[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) ls[r] = lpart[r];
+        const float wl = tcm::column_reduce<N, false>(ls, lane);
+        float* rl = red + 256;
+        if (lane < N) rl[warp * 32 + lane] = wl;
+        tcm::named_sync_softmax();
+        const float L_c = (rl[jc] + rl[32 + jc]) + (rl[64 + jc] + rl[96 + jc]);
+        float lall[N];
+#pragma unroll
+        for (int r = 0; r < N; ++r) lall[r] = __shfl_sync(kFull, L_c, r);
+        uint32_t ov[N];
+        tmem_ld<N>(tmem + lane_off + 2 * N + (j & 1) * N, ov);
+        tc_wait_ld();
+        tc_fence_before_sync();
+        const bool complete = first_x == 0 && w.x == w.tiles - 1;
+        if (!ok) {
+          // nothing is written after a timeout
+        } else if (complete) {
+          int i = (rc * N) / p.group, gg = rc * N - i * p.group;
+#pragma unroll
+          for (int r = 0; r < N; ++r) {
+            if (r < nrows) {
+              const float inv = lall[r] > 0.f ? 1.f / lall[r] : 0.f;
+              p.out[(static_cast<size_t>(w.b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D + t] =
+                  static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
+            }
+            if (++gg == p.group) {
+              gg = 0;
+              ++i;
+            }
+          }
+        } else {
+          float* rec = p.records + static_cast<size_t>(j == 0 ? 2 * c : 2 * c + 1) * p.rec_stride;
+#pragma unroll
+          for (int r = 0; r < N; ++r)
+            if (r < nrows) rec[r * D + t] = __uint_as_float(ov[r]);
+          if (t < nrows) reinterpret_cast<float2*>(rec + N * D)[t] = make_float2(mref_c, L_c);
+        }
+        if (g == n - 1 && t == 0) {
+          // the merge descriptor: this CTA's last unit continues in the next CTAs and
+          // started here, so this CTA holds its first piece
+          int4 dsc = make_int4(-1, 0, 0, 0);
+          if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
+            const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
+            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * G - 1) / W), w.b, w.k);
+          }
+          p.tc_desc[c] = dsc;
+        }
+      }
+      w.next(p, upb);
+    }
+    if (!ok) {
+      if (lane == 0) record_error(kErrTimeoutDecode);
+      if (t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
+    }
   }
   grid_launch_dependents();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 2) tmem_dealloc(tmem, tc5::kTmemCols);
+  if (warp == tcm::kMmaWarp) tmem_dealloc(tmem, 4 * N < 32 ? 32 : 4 * N);
+}
+
+// Combines the partial records of every unit cut by a range boundary (one CTA per
+// decode CTA; the descriptor of CTA c names the unit whose first piece c holds and the
+// last CTA c1 with a piece of it: pieces in record slots desc.x, then 2c' for
+// c' = c+1..c1, in that order), then writes zeros for sequences with no keys.
+template <int N>
+__global__ void __launch_bounds__(128) tcm_merge_kernel(const DecodeParams p) {
+  constexpr int D = tcm::kD;
+  grid_dependency_wait();
+  const int c = blockIdx.x;
+  const int d = threadIdx.x;
+  const int4 dsc = p.tc_desc[c];
+  if (dsc.x >= 0) {
+    const int b = dsc.z;
+    const int kvh = dsc.w / p.row_chunks;
+    const int rc = dsc.w - kvh * p.row_chunks;
+    const int nrows = min(N, p.rows - rc * N);
+    const int pieces = 1 + (dsc.y - c);
+    int i = (rc * N) / p.group, gg = rc * N - i * p.group;
+    for (int r = 0; r < nrows; ++r) {
+      float M = -INFINITY;
+      for (int k = 0; k < pieces; ++k) {
+        const int slot = k == 0 ? dsc.x : 2 * (c + k);
+        M = fmaxf(M, reinterpret_cast<const float2*>(p.records + static_cast<size_t>(slot) * p.rec_stride + N * D)[r].x);
+      }
+      float acc = 0.f, l = 0.f;
+      if (M != -INFINITY) {
+        for (int k = 0; k < pieces; ++k) {
+          const int slot = k == 0 ? dsc.x : 2 * (c + k);
+          const float* rec = p.records + static_cast<size_t>(slot) * p.rec_stride;
+          const float2 ml = reinterpret_cast<const float2*>(rec + N * D)[r];
+          const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+          l = fmaf(ml.y, wk, l);
+          acc = fmaf(rec[r * D + d], wk, acc);
+        }
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      p.out[(static_cast<size_t>(b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D + d] =
+          static_cast<uint16_t>(pack_bf16x2(acc * inv, 0.f) & 0xFFFFu);
+      if (++gg == p.group) {
+        gg = 0;
+        ++i;
+      }
+    }
+  }
+  // sequences without a visible key (context length 0) get zero rows
+  const int rq = p.q_per_seq * p.num_q_heads;
+  for (int b = c; b < p.num_seqs; b += gridDim.x) {
+    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;
+    uint16_t* o = p.out + static_cast<size_t>(b) * rq * D;
+    for (int e = d; e < rq * D; e += blockDim.x) o[e] = 0;
+  }
 }
 
 }  // namespace pa

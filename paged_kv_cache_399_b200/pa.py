@@ -149,8 +149,9 @@ def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads
                    head_dim: int, max_blocks_per_seq: int, path: int = PA_PATH_AUTO,
                    split_blocks: int = 0, schedule: int = PA_SCHEDULE_AUTO,
                    share_prefix: bool = False) -> pa_plan_t:
-    """A forced split length implies the grid schedule."""
-    if split_blocks and schedule == PA_SCHEDULE_AUTO:
+    """A forced split length implies the grid schedule (the tcgen05 path has no split
+    length: its schedule cuts the work into equal tile ranges, and ignores it)."""
+    if split_blocks and schedule == PA_SCHEDULE_AUTO and path != PA_PATH_TCGEN05:
         schedule = PA_SCHEDULE_GRID
     hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)))
     plan = pa_plan_t()

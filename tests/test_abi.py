@@ -126,10 +126,16 @@ def test_plan_heuristic_host_logic(pa):
     with pytest.raises(pa.PAError) as exc:   # 24 rows per sequence: two do not fit 32 rows
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, share_prefix=True)
     assert exc.value.status == pa.PA_ERR_UNSUPPORTED
+    # tcgen05: N = 16 or 32 rows per unit, its own persistent equal-tile schedule
     p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05)
-    assert (p.path, p.schedule, p.rows_per_cta) == (3, 1, 32)
-    with pytest.raises(pa.PAError):          # tcgen05 runs the grid schedule only
-        pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05, schedule=pa.PA_SCHEDULE_PERSISTENT)
+    assert (p.path, p.schedule, p.rows_per_cta, p.num_splits) == (3, 2, 32, 1) and p.num_ctas >= 1
+    p = pa.pa_decode_plan(64, 1, 32, 8, 128, 256, pa.PA_PATH_TCGEN05)
+    assert (p.path, p.schedule, p.rows_per_cta) == (3, 2, 16)
+    assert pa.pa_decode_workspace_size(p, 64, 1, 32, 8, 128, 256) >= 2 * p.num_ctas * (16 * 128 + 32) * 4
+    with pytest.raises(pa.PAError):          # no grid schedule on the tcgen05 path
+        pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05, schedule=pa.PA_SCHEDULE_GRID)
+    with pytest.raises(pa.PAError):          # head_dim 128 only
+        pa.pa_decode_plan(32, 6, 32, 8, 64, 1024, pa.PA_PATH_TCGEN05)
     with pytest.raises(pa.PAError):          # sharing runs on the mma.sync tensor-core kernel
         pa.pa_decode_plan(8, 1, 32, 8, 128, 64, pa.PA_PATH_TCGEN05, share_prefix=True)
     forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)

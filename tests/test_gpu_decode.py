@@ -49,8 +49,9 @@ PLANS = [
     ("tile_split1", dict(path=2, split_blocks=1)),
     ("tile_split3", dict(path=2, split_blocks=3)),
     ("tcgen05", dict(path=3)),
-    ("tcgen05_split1", dict(path=3, split_blocks=1)),
-    ("tcgen05_split5", dict(path=3, split_blocks=5)),
+    # fewer / more CTAs than usual: units cut into many pieces, CTAs without work
+    ("tcgen05_ctas3", dict(path=3, num_ctas=3)),
+    ("tcgen05_ctas1000", dict(path=3, num_ctas=1000)),
 ]
 
 
@@ -77,14 +78,21 @@ def _plan(w, plan_spec):
     from paged_kv_cache_399_b200 import pa
     if not plan_spec[1]:
         return None
+    hints = dict(plan_spec[1])
+    num_ctas = hints.pop("num_ctas", None)
     try:
         plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads,
-                                 w.head_dim, w.max_blocks_per_seq, **plan_spec[1])
+                                 w.head_dim, w.max_blocks_per_seq, **hints)
     except pa.PAError as exc:
-        assert exc.status == pa.PA_ERR_UNSUPPORTED and plan_spec[1].get("share_prefix")
-        pytest.skip("prefix sharing needs G*q <= 16 rows")
+        assert exc.status == pa.PA_ERR_UNSUPPORTED
+        if hints.get("share_prefix"):
+            pytest.skip("prefix sharing needs G*q <= 16 rows")
+        assert hints.get("path") == pa.PA_PATH_TCGEN05 and w.head_dim != 128
+        pytest.skip("the tcgen05 path runs head_dim 128")
     if plan.path == pa.PA_PATH_TCGEN05:
-        assert plan.schedule == pa.PA_SCHEDULE_GRID and plan.rows_per_cta == 32
+        assert plan.schedule == pa.PA_SCHEDULE_PERSISTENT and plan.rows_per_cta in (16, 32)
+    if num_ctas is not None:
+        plan.num_ctas = num_ctas
     return plan
 
 
