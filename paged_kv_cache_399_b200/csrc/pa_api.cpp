@@ -429,6 +429,13 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
     p.rec_stride = tcm_rec_stride(*plan, head_dim);
     p.records = reinterpret_cast<float*>(ws);
     p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
+    // CTAs per group: the largest divisor of H_kv that the grid holds
+    p.tc_group = 1;
+    for (int sz = num_kv_heads; sz >= 1; --sz)
+      if (num_kv_heads % sz == 0 && sz <= plan->num_ctas) {
+        p.tc_group = sz;
+        break;
+      }
   } else if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
     const PersistentLayout L = persistent_layout(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
     p.num_ctas = plan->num_ctas;

@@ -251,14 +251,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-// N (16 or 32) consecutive columns of this thread's TMEM lane.
+// 8 consecutive fp32 columns of this thread's TMEM lane (warp-wide, 32 lanes x 8 columns).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// N (8, 16 or 32) consecutive columns of this thread's TMEM lane.
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
-  if constexpr (N == 16) tmem_ld16(taddr, r); else tmem_ld32(taddr, r);
+  if constexpr (N == 8) tmem_ld8(taddr, r); else if constexpr (N == 16) tmem_ld16(taddr, r); else tmem_ld32(taddr, r);
 }
 template <int N>
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
-  if constexpr (N == 16) tmem_st16(taddr, r); else tmem_st32(taddr, r);
+  if constexpr (N == 8) tmem_st8(taddr, r); else if constexpr (N == 16) tmem_st16(taddr, r); else tmem_st32(taddr, r);
 }
 
 // Shared-memory matrix descriptor without swizzle (layout type 0): 8 x 16-byte core

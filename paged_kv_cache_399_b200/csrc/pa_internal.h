@@ -69,6 +69,7 @@ struct DecodeParams {
   // tcgen05 path: per CTA, the unit whose first piece it holds when that unit continues
   // in later CTAs: {record slot, last CTA with a piece, sequence, unit}, or {-1, ...}
   int4* tc_desc;
+  int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
 };
 
 // Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).

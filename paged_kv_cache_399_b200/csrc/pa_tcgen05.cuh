@@ -3,10 +3,13 @@
 // helpers and device error word).
 //
 // Work. A unit is (sequence, kv head, row chunk of N query rows); its blocks are cut into
-// tiles of 8 blocks = 128 tokens. All units' tiles, in (sequence, kv head, row chunk)
-// order, are split into equal contiguous ranges, one per CTA of a persistent grid; each
-// CTA finds its range from context_lens itself (no pre-pass). A unit cut by a range
-// boundary leaves partial records, combined afterwards by tcm_merge_kernel.
+// tiles of 8 blocks = 128 tokens. The CTAs of the persistent grid form groups of S
+// (a divisor of H_kv); CTA li of a group takes the kv heads li, li + S, ... . All groups
+// walk the same enumeration of (sequence, kv-head index, row chunk, tile) and split it
+// into equal contiguous ranges, one per group, computed in the kernel from context_lens
+// (no pre-pass); the S CTAs of a group therefore read the kv-head slices of the same
+// blocks at about the same time. A unit cut by a range boundary leaves partial records,
+// combined afterwards by tcm_merge_kernel.
 //
 // Per tile, with Q of the unit's N (16 or 32) rows:
 //   S^T[128 tok][N]  = K[128 tok][D] . Q^T[D][N]           tcgen05.mma M=128, K-major A and B
@@ -17,13 +20,16 @@
 //   numerator and denominator share the reference);
 //   O^T[D][N] += V^T[D][128 tok] . P^T[128 tok][N]         tcgen05.mma M=D=128, MN-major A
 //                                                          (the TMA tile) and B (P^T)
-// Roles: warps 0-3 softmax and epilogue (TMEM lanes 0..127), warp 4 TMA producer and Q
-// loads, warp 5 MMA issuer (one thread) and TMEM owner. The issuer polls both of its
+// Roles: warps 0-7 softmax and epilogue in two warpgroups, each over TMEM lanes 0..127 and
+// owning half of the N columns (its own maxima, references, P^T half and O^T half);
+// warp 8 TMA producer of K and Q loads, warp 10 TMA producer of V (one warp issues about
+// 16 2-KB boxes per us, so K and V get a warp each), warp 9 MMA issuer (one thread) and
+// TMEM owner. The issuer polls both of its
 // inputs and issues whichever MMA is ready: the S of the next tile once its K has
 // landed, the PV of the oldest tile once its P^T is written; a K stage is released
 // when its S completes, a V stage when its PV completes.
 // TMEM columns: S double buffer [0, 2N), O double buffer (by unit parity) [2N, 4N).
-// Shared memory: 2 Q buffers, 2 P^T buffers, 3 stages of K and of V (32 KB each).
+// Shared memory: 2 Q buffers, 2 P^T buffers, 3 stages of K and 3 of V (32 KB each).
 
 namespace pa {
 namespace tcm {
@@ -31,10 +37,13 @@ namespace tcm {
 constexpr int kD = 128;
 constexpr int kTileBlocks = 8;
 constexpr int kTileTokens = kTileBlocks * kBlockSize;   // 128
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kKStages = 3;  // a K stage is released as soon as its S has completed
+constexpr int kVStages = 3;  // a V stage is held until the PV, after the tile's softmax
+constexpr int kSoftmaxWarps = 8;   // two warpgroups, each owning half of the N columns
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8;   // K boxes and Q rows
+constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10; // V boxes
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
@@ -47,16 +56,16 @@ struct Smem {
   static constexpr int offQ = 0;
   static constexpr int offP = offQ + 2 * kQ;
   static constexpr int offK = offP + 2 * kP;
-  static constexpr int offV = offK + kStages * kStageBytes;
-  static constexpr int offRed = offV + kStages * kStageBytes;  // [3][4 warps][32] floats
-  static constexpr int offScan = offRed + 3 * 4 * 32 * 4;      // [8] int64, then the start
+  static constexpr int offV = offK + kKStages * kStageBytes;
+  static constexpr int offRed = offV + kVStages * kStageBytes;  // [2 wg][3][4 warps][N/2] floats
+  static constexpr int offScan = offRed + 2 * 3 * 4 * (N / 2) * 4;  // [11] int64, then the start
   static constexpr int offBars = offScan + 128;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && kQ % 1024 == 0, "swizzled operands need 1024-B alignment");
 };
 
 struct Bars {
-  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], pv_done[2];
   uint64_t drain;
 };
@@ -83,7 +92,10 @@ struct Walk {
   }
 };
 
-__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of one softmax warpgroup (ids 1 and 2).
+__device__ __forceinline__ void named_sync_softmax(int wg) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
+}
 
 // Column reduction of a warp: lane l holds V values (columns 0..V-1); on return every
 // lane holds the reduction over all 32 lanes of column (l % V). Halving exchange: at
@@ -118,12 +130,14 @@ __global__ void __launch_bounds__(tcm::kThreads, 1)
 decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
   using L = tcm::Smem<N>;
-  using tcm::kStages;
+  using tcm::kKStages;
+  using tcm::kVStages;
   using tcm::kTileBlocks;
   using tcm::kTileTokens;
   constexpr int D = tcm::kD;
   extern __shared__ __align__(1024) uint8_t smem[];
   static_assert(sizeof(tcm::Bars) + 16 <= 256, "barrier area");
+  static_assert(tcm::kThreads / 32 * 8 <= 96, "scan area");
   tcm::Bars& bars = *reinterpret_cast<tcm::Bars*>(smem + L::offBars);
   uint32_t& tmem_base_s = *reinterpret_cast<uint32_t*>(smem + L::offBars + sizeof(tcm::Bars));
   const int warp = threadIdx.x >> 5;
@@ -140,8 +154,8 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
     for (int i = 0; i < static_cast<int>(sizeof(tcm::Bars) / 8); ++i) mbar_init(all + i, 1);
     for (int i = 0; i < 2; ++i) {  // one arrival per softmax warp
-      mbar_init(&bars.s_free[i], 4);
-      mbar_init(&bars.p_full[i], 4);
+      mbar_init(&bars.s_free[i], tcm::kSoftmaxWarps);
+      mbar_init(&bars.p_full[i], tcm::kSoftmaxWarps);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
@@ -149,12 +163,16 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   }
   grid_dependency_wait();
 
-  // ---- this CTA's tile range [t0, t1) of W tiles: prefix sums over the sequences
-  const int upb = p.num_kv_heads * p.row_chunks;  // units per sequence
+  // ---- this CTA's group, kv-head set and tile range [t0, t1) of the W tiles every group
+  // walks: prefix sums over the sequences
+  const int S = p.tc_group;
+  const int li = c % S;
+  const int NG = static_cast<int>(gridDim.x) / S;
+  const int upb = (p.num_kv_heads / S) * p.row_chunks;  // units per sequence of one CTA
   long long* wsum = reinterpret_cast<long long*>(smem + L::offScan);
-  int* start = reinterpret_cast<int*>(smem + L::offScan + 64);
+  int* start = reinterpret_cast<int*>(smem + L::offScan + 96);
   long long W, t0, t1;
-  int G;  // CTAs that take part: at most one per tile, so that every range is non-empty
+  int NGe;  // groups that take part: at most one per tile, so that every range is non-empty
   {
     const int B = p.num_seqs;
     const int chunk = (B + tcm::kThreads - 1) / tcm::kThreads;
@@ -178,9 +196,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       if (w2 < warp) base += wsum[w2];
       W += wsum[w2];
     }
-    G = static_cast<int>(min(static_cast<long long>(gridDim.x), W));
-    t0 = c < G ? static_cast<long long>(c) * W / G : 0;
-    t1 = c < G ? static_cast<long long>(c + 1) * W / G : 0;
+    NGe = static_cast<int>(min(static_cast<long long>(NG), W));
+    const int gi = c / S;
+    t0 = gi < NGe ? static_cast<long long>(gi) * W / NGe : 0;
+    t1 = gi < NGe ? static_cast<long long>(gi + 1) * W / NGe : 0;
     const long long excl = base + v - local;
     if (local > 0 && t0 < t1 && t0 >= excl && t0 < excl + local) {
       long long acc = excl;
@@ -203,6 +222,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     grid_launch_dependents();
     return;
   }
+  // unit k of a sequence -> kv head and row chunk of this CTA
+  auto unit_kvh = [&](int k) { return li + S * (k / p.row_chunks); };
+  auto unit_rc = [&](int k) { return k % p.row_chunks; };
   tcm::Walk w0;
   w0.b = start[0];
   w0.seq(p);
@@ -219,10 +241,15 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   const uint32_t tmem = tmem_base_s;
   const uint32_t sm = smem_u32(smem);
 
-  if (warp == tcm::kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer + Q
-    // Lanes 0..15 issue the tile's 16 boxes of K (half = lane / 8, block = lane % 8),
-    // then of V; lanes 0..7 load the next tile's block ids while this one is issued.
+  if (warp == tcm::kProducerWarp || warp == tcm::kVProducerWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // Lanes 0..15 issue a tile's 16 boxes (half = lane / 8, block = lane % 8) of K (warp 4)
+    // or V (warp 6); lanes 0..7 load the next tile's block ids while this one is issued.
+    const bool is_k = warp == tcm::kProducerWarp;
+    const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+    uint64_t* full = is_k ? bars.k_full : bars.v_full;
+    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+    const int stage_off = is_k ? L::offK : L::offV;
     tcm::Walk w = w0;
     const int oob = static_cast<int>(p.num_blocks);  // block id past the pool: TMA fills zeros
     auto block_id = [&](const tcm::Walk& at) {
@@ -235,13 +262,13 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     int j = -1, g = 0;
     bool ok = true;
     for (; g < n; ++g) {
-      if (g == 0 || w.x == 0) {
+      if (is_k && (g == 0 || w.x == 0)) {
         ++j;
         if (j >= 2) ok = __all_sync(kFull, mbar_wait_bounded(&bars.q_empty[j & 1], ((j >> 1) - 1) & 1));
         if (!ok) break;
         // Q rows of the unit -> Q[j & 1], 128-byte swizzled K-major; zeros for padded rows
-        const int kvh = w.k / p.row_chunks;
-        const int rc = w.k - kvh * p.row_chunks;
+        const int kvh = unit_kvh(w.k);
+        const int rc = unit_rc(w.k);
         const int nrows = min(N, p.rows - rc * N);
         uint8_t* qb = smem + L::offQ + (j & 1) * L::kQ;
         if (lane < N) {
@@ -262,45 +289,30 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.q_full[j & 1]);
       }
-      const int s = g % kStages;
-      const int kvh = w.k / p.row_chunks;
+      const int stages = is_k ? kKStages : kVStages;
+      const int s = g % stages;
+      const int kvh = unit_kvh(w.k);
       const int ph = __shfl_sync(kFull, phys_next, lane & (kTileBlocks - 1));
       tcm::Walk wn = w;
       wn.next(p, upb);
       if (g + 1 < n) phys_next = block_id(wn);
-      const int hf = lane >> 3, jj = lane & (kTileBlocks - 1);
-      const uint32_t box = hf * tcm::kHalfBytes + jj * kHalfTileBytes;
-      if (g >= kStages) ok = __all_sync(kFull, mbar_wait_bounded(&bars.k_empty[s], ((g / kStages) - 1) & 1));
+      if (g >= stages) ok = __all_sync(kFull, mbar_wait_bounded(&empty[s], ((g / stages) - 1) & 1));
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&bars.k_full[s], tcm::kStageBytes);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], tcm::kStageBytes);
       __syncwarp();
+      const int hf = lane >> 3, jj = lane & (kTileBlocks - 1);
       if (lane < 2 * kTileBlocks)
-        tma_load_3d(smem + L::offK + s * tcm::kStageBytes + box, &tmap_k, &bars.k_full[s], hf * 64, kvh,
-                    ph * kBlockSize);
-      if (g >= kStages) ok = __all_sync(kFull, mbar_wait_bounded(&bars.v_empty[s], ((g / kStages) - 1) & 1));
-      if (!ok) {
-        ++g;  // this tile's K load is in flight: drain it below
-        break;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&bars.v_full[s], tcm::kStageBytes);
-      __syncwarp();
-      if (lane < 2 * kTileBlocks)
-        tma_load_3d(smem + L::offV + s * tcm::kStageBytes + box, &tmap_v, &bars.v_full[s], hf * 64, kvh,
-                    ph * kBlockSize);
+        tma_load_3d(smem + stage_off + s * tcm::kStageBytes + hf * tcm::kHalfBytes + jj * kHalfTileBytes, tmap,
+                    &full[s], hf * 64, kvh, ph * kBlockSize);
       __syncwarp();
       w = wn;
     }
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
-      // wait (bounded) for the loads still in flight before leaving (a tile whose V was
-      // not issued has only its K pending: waiting on its V times out harmlessly)
-      for (int u = max(0, g - kStages); u < g; ++u) {
-        const int s = u % kStages;
-        if (!mbar_wait_bounded(&bars.k_full[s], (u / kStages) & 1)) {
-          if (lane == 0) record_error(kErrTimeoutDrain);
-        }
-        mbar_wait_bounded(&bars.v_full[s], (u / kStages) & 1);
-      }
+      // wait (bounded) for the loads still in flight before leaving
+      const int stages = is_k ? kKStages : kVStages;
+      for (int u = max(0, g - stages); u < g; ++u)
+        if (!mbar_wait_bounded(&full[u % stages], (u / stages) & 1) && lane == 0) record_error(kErrTimeoutDrain);
     }
   } else if (warp == tcm::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -313,14 +325,34 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       int ring = 0;          // per tile in flight: bit 2(g&3) O buffer, bit 2(g&3)+1 first of unit
       bool ok = true;
       unsigned long long idle_since = 0;
+      unsigned idle_polls = 0;
       while (gp < n) {
         bool progressed = false;
+        if (gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
+            mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1)) {
+          const int sh = 2 * (gp & 3);
+          const int obuf = (ring >> sh) & 1;
+          const bool first = (ring >> (sh + 1)) & 1;
+          tc_fence_after_sync();
+          const uint32_t vst = sm + L::offV + (gp % kVStages) * tcm::kStageBytes;
+          const uint32_t pst = sm + L::offP + (gp & 1) * L::kP;
+#pragma unroll
+          for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(vst + kk * 2048, tcm::kHalfBytes, 1024);
+            const uint64_t bd = smem_desc_noswizzle(pst + kk * 256, 128, tcm::kPGroupBytes);
+            tc_mma_bf16(tmem + 2 * N + obuf * N, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&bars.pv_done[gp & 1]);
+          tc_commit(&bars.v_empty[gp % kVStages]);
+          ++gp;
+          progressed = true;
+        }
         if (gs < n && gs - gp < 3) {
           const bool first = gs == 0 || w.x == 0;
           const int jn = first ? js + 1 : js;
-          const int s = gs % kStages;
+          const int s = gs % kKStages;
           if ((!first || mbar_test_wait(&bars.q_full[jn & 1], (jn >> 1) & 1)) &&
-              mbar_test_wait(&bars.k_full[s], (gs / kStages) & 1) &&
+              mbar_test_wait(&bars.k_full[s], (gs / kKStages) & 1) &&
               (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1))) {
             js = jn;
             const int obuf = js & 1;
@@ -344,28 +376,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
             progressed = true;
           }
         }
-        if (gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
-            mbar_test_wait(&bars.v_full[gp % kStages], (gp / kStages) & 1)) {
-          const int sh = 2 * (gp & 3);
-          const int obuf = (ring >> sh) & 1;
-          const bool first = (ring >> (sh + 1)) & 1;
-          tc_fence_after_sync();
-          const uint32_t vst = sm + L::offV + (gp % kStages) * tcm::kStageBytes;
-          const uint32_t pst = sm + L::offP + (gp & 1) * L::kP;
-#pragma unroll
-          for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(vst + kk * 2048, tcm::kHalfBytes, 1024);
-            const uint64_t bd = smem_desc_noswizzle(pst + kk * 256, 128, tcm::kPGroupBytes);
-            tc_mma_bf16(tmem + 2 * N + obuf * N, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
-          }
-          tc_commit(&bars.pv_done[gp & 1]);
-          tc_commit(&bars.v_empty[gp % kStages]);
-          ++gp;
-          progressed = true;
-        }
         if (progressed) {
           idle_since = 0;
-        } else {
+          idle_polls = 0;
+        } else if ((++idle_polls & 63) == 0) {  // the clock is read once every 64 idle polls
           const unsigned long long now = global_timer_ns();
           if (idle_since == 0) {
             idle_since = now;
@@ -382,21 +396,63 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int t = threadIdx.x;  // token of the tile = TMEM lane = head-dim index in O^T
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + L::offRed);
+    constexpr int NC = N / 2;  // columns of this warpgroup
+    const int wg = warp >> 2;
+    const int cb = wg * NC;    // first column of this warpgroup
+    const int t = (warp & 3) * 32 + lane;  // token of the tile = TMEM lane = head-dim index in O^T
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + L::offRed) + wg * 3 * 4 * NC;
     const float cs = p.scale_log2;
     tcm::Walk w = w0;
     int j = -1, first_x = 0, kvh = 0, rc = 0, nrows = 0, minlim = 0;
-    float mref_c = -INFINITY;  // reference maximum of column (lane % N)
-    float mref[N], lpart[N];
-    int lim[N];
+    float mref_c = -INFINITY;  // reference maximum of column cb + (lane % NC)
+    float mref[NC], lpart[NC];
+    int lim[NC];
     // A bounded wait that gives up makes `ok` false for good: the later waits are skipped
     // and nothing more is written to global memory, but every warp still passes every
-    // named barrier, so none of the four is left waiting for the others.
+    // named barrier, so none of a warpgroup's four warps is left waiting for the others.
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(kFull, mbar_wait_bounded(bar, parity));
+    };
+    // A unit piece whose output is written one tile later: by then its last PV is done.
+    struct Pending {
+      bool on, complete;
+      int g, obuf, b, kvh, rc, nrows, slot;
+      float L_c, m_c;  // l and the reference maximum of column cb + (lane % NC)
+    } pend;
+    pend.on = false;
+    auto flush = [&](Pending& e) {
+      e.on = false;
+      wait(&bars.pv_done[e.g & 1], (e.g >> 1) & 1);
+      tc_fence_after_sync();
+      uint32_t ov[NC];
+      tmem_ld<NC>(tmem + lane_off + 2 * N + e.obuf * N + cb, ov);
+      tc_wait_ld();
+      tc_fence_before_sync();
+      if (!ok) return;  // nothing is written after a timeout
+      if (e.complete) {
+        int i = (e.rc * N + cb) / p.group, gg = e.rc * N + cb - i * p.group;
+#pragma unroll
+        for (int r = 0; r < NC; ++r) {
+          const float lr = __shfl_sync(kFull, e.L_c, r);
+          if (cb + r < e.nrows) {
+            const float inv = lr > 0.f ? 1.f / lr : 0.f;
+            p.out[(static_cast<size_t>(e.b * p.q_per_seq + i) * p.num_q_heads + e.kvh * p.group + gg) * D + t] =
+                static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
+          }
+          if (++gg == p.group) {
+            gg = 0;
+            ++i;
+          }
+        }
+      } else {
+        float* rec = p.records + static_cast<size_t>(e.slot) * p.rec_stride;
+#pragma unroll
+        for (int r = 0; r < NC; ++r)
+          if (cb + r < e.nrows) rec[(cb + r) * D + t] = __uint_as_float(ov[r]);
+        if (t < NC && cb + t < e.nrows) reinterpret_cast<float2*>(rec + N * D)[cb + t] = make_float2(e.m_c, e.L_c);
+      }
     };
     for (int g = 0; g < n; ++g) {
       const bool first = g == 0 || w.x == 0;
@@ -404,14 +460,14 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       if (first) {
         ++j;
         first_x = w.x;
-        kvh = w.k / p.row_chunks;
-        rc = w.k - kvh * p.row_chunks;
+        kvh = unit_kvh(w.k);
+        rc = unit_rc(w.k);
         nrows = min(N, p.rows - rc * N);
-        int i = (rc * N) / p.group, gg = rc * N - i * p.group;
-        minlim = w.ctx - p.q_per_seq + i;
+        int i = (rc * N + cb) / p.group, gg = rc * N + cb - i * p.group;
+        minlim = w.ctx - p.q_per_seq + (rc * N) / p.group;
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
-          lim[r] = r < nrows ? w.ctx - p.q_per_seq + i : w.ctx - 1;
+        for (int r = 0; r < NC; ++r) {
+          lim[r] = cb + r < nrows ? w.ctx - p.q_per_seq + i : w.ctx - 1;
           if (++gg == p.group) {
             gg = 0;
             ++i;
@@ -421,40 +477,40 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         }
         mref_c = -INFINITY;
       }
-      // ---- S^T of this tile: the N scores of token t
+      // ---- S^T of this tile: this warpgroup's NC scores of token t
       wait(&bars.s_full[g & 1], (g >> 1) & 1);
       tc_fence_after_sync();
-      uint32_t sv[N];
-      tmem_ld<N>(tmem + lane_off + (g & 1) * N, sv);
+      uint32_t sv[NC];
+      tmem_ld<NC>(tmem + lane_off + (g & 1) * N + cb, sv);
       tc_wait_ld();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[g & 1]);
       const int tok = w.x * kTileTokens + t;
       const bool edge = w.x * kTileTokens + kTileTokens - 1 > minlim;
-      float x[N], tmp[N];
+      float x[NC], tmp[NC];
 #pragma unroll
-      for (int r = 0; r < N; ++r) {
+      for (int r = 0; r < NC; ++r) {
         float v = __uint_as_float(sv[r]) * cs;
         if (edge && tok > lim[r]) v = -INFINITY;
         x[r] = v;
         tmp[r] = v;
       }
       // ---- column maxima over the 128 tokens
-      const float wmax = tcm::column_reduce<N, true>(tmp, lane);
-      float* rb = red + (g & 1) * 128;
-      if (lane < N) rb[warp * 32 + lane] = wmax;
-      tcm::named_sync_softmax();
-      const int jc = lane % N;
-      const float M = fmaxf(fmaxf(rb[jc], rb[32 + jc]), fmaxf(rb[64 + jc], rb[96 + jc]));
+      const float wmax = tcm::column_reduce<NC, true>(tmp, lane);
+      float* rb = red + (g & 1) * 4 * NC;
+      if (lane < NC) rb[(warp & 3) * NC + lane] = wmax;
+      tcm::named_sync_softmax(wg);
+      const int jc = lane % NC;
+      const float M = fmaxf(fmaxf(rb[jc], rb[NC + jc]), fmaxf(rb[2 * NC + jc], rb[3 * NC + jc]));
       const bool need = M > mref_c + tcm::kRescaleLog2 || (mref_c == -INFINITY && M != -INFINITY);
-      if (__any_sync(kFull, need)) {  // the same decision in all four warps
+      if (__any_sync(kFull, need)) {  // the same decision in the warpgroup's four warps
         const float nm = need ? M : mref_c;
         const float alpha_c = need ? (mref_c == -INFINITY ? 0.f : fast_exp2(mref_c - nm)) : 1.f;
         mref_c = nm;
-        float alpha[N];
+        float alpha[NC];
 #pragma unroll
-        for (int r = 0; r < N; ++r) {
+        for (int r = 0; r < NC; ++r) {
           mref[r] = __shfl_sync(kFull, mref_c, r);
           alpha[r] = __shfl_sync(kFull, alpha_c, r);
           lpart[r] *= alpha[r];
@@ -462,20 +518,20 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         if (!first) {  // O holds this unit's earlier tiles once the PV of tile g-1 is done
           wait(&bars.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1);
           tc_fence_after_sync();
-          uint32_t ov[N];
-          const uint32_t oaddr = tmem + lane_off + 2 * N + (j & 1) * N;
-          tmem_ld<N>(oaddr, ov);
+          uint32_t ov[NC];
+          const uint32_t oaddr = tmem + lane_off + 2 * N + (j & 1) * N + cb;
+          tmem_ld<NC>(oaddr, ov);
           tc_wait_ld();
 #pragma unroll
-          for (int r = 0; r < N; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
-          tmem_st<N>(oaddr, ov);
+          for (int r = 0; r < NC; ++r) ov[r] = __float_as_uint(__uint_as_float(ov[r]) * alpha[r]);
+          tmem_st<NC>(oaddr, ov);
           tc_wait_st();
         }
       }
       // ---- probabilities, bf16 pairs (column 2q in the low half)
-      uint32_t pk[N / 2];
+      uint32_t pk[NC / 2];
 #pragma unroll
-      for (int r = 0; r < N; r += 2) {
+      for (int r = 0; r < NC; r += 2) {
         const float p0 = fast_exp2(x[r] - (mref[r] == -INFINITY ? 0.f : mref[r]));
         const float p1 = fast_exp2(x[r + 1] - (mref[r + 1] == -INFINITY ? 0.f : mref[r + 1]));
         lpart[r] += p0;
@@ -484,12 +540,12 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       }
       // the P^T buffer of this tile was read by the PV of tile g-2
       if (g >= 2) wait(&bars.pv_done[g & 1], ((g >> 1) - 1) & 1);
-      if (w.x == w.tiles - 1 && (w.ctx & (kBlockSize - 1))) {
+      if (wg == 0 && w.x == w.tiles - 1 && (w.ctx & (kBlockSize - 1))) {
         // The sequence's last block is partly filled: its slots past the context may hold
         // any bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows
         // are cleared before the PV reads them.
-        const int s = g % kStages;
-        wait(&bars.v_full[s], (g / kStages) & 1);
+        const int s = g % kVStages;
+        wait(&bars.v_full[s], (g / kVStages) & 1);
         const int jj = (w.nblk - 1) - w.x * kTileBlocks;
         const int r0 = w.ctx & (kBlockSize - 1);
         const int nrow = kBlockSize - r0;
@@ -501,9 +557,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
               make_uint4(0, 0, 0, 0);
         }
       }
-      uint8_t* pb = smem + L::offP + (g & 1) * L::kP;
+      uint8_t* pb = smem + L::offP + (g & 1) * L::kP + (cb / 8) * tcm::kPGroupBytes;
 #pragma unroll
-      for (int q8 = 0; q8 < N / 8; ++q8)
+      for (int q8 = 0; q8 < NC / 8; ++q8)
         *reinterpret_cast<uint4*>(pb + q8 * tcm::kPGroupBytes + t * 16) =
             make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
       fence_proxy_async_smem();
@@ -511,65 +567,45 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[g & 1]);
 
+      // ---- the previous unit's output, now that its last PV has had a tile's time
+      if (pend.on) flush(pend);
       if (last) {
-        // ---- epilogue of the unit's piece: wait for its last PV, then O^T / l
-        wait(&bars.pv_done[g & 1], (g >> 1) & 1);
-        tc_fence_after_sync();
-        float ls[N];
+        // ---- end of the unit's piece: l now; O^T / l after the next tile (deferred)
+        float ls[NC];
 #pragma unroll
-        for (int r = 0; r < N; ++r) ls[r] = lpart[r];
-        const float wl = tcm::column_reduce<N, false>(ls, lane);
-        float* rl = red + 256;
-        if (lane < N) rl[warp * 32 + lane] = wl;
-        tcm::named_sync_softmax();
-        const float L_c = (rl[jc] + rl[32 + jc]) + (rl[64 + jc] + rl[96 + jc]);
-        float lall[N];
-#pragma unroll
-        for (int r = 0; r < N; ++r) lall[r] = __shfl_sync(kFull, L_c, r);
-        uint32_t ov[N];
-        tmem_ld<N>(tmem + lane_off + 2 * N + (j & 1) * N, ov);
-        tc_wait_ld();
-        tc_fence_before_sync();
-        const bool complete = first_x == 0 && w.x == w.tiles - 1;
-        if (!ok) {
-          // nothing is written after a timeout
-        } else if (complete) {
-          int i = (rc * N) / p.group, gg = rc * N - i * p.group;
-#pragma unroll
-          for (int r = 0; r < N; ++r) {
-            if (r < nrows) {
-              const float inv = lall[r] > 0.f ? 1.f / lall[r] : 0.f;
-              p.out[(static_cast<size_t>(w.b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D + t] =
-                  static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
-            }
-            if (++gg == p.group) {
-              gg = 0;
-              ++i;
-            }
-          }
-        } else {
-          float* rec = p.records + static_cast<size_t>(j == 0 ? 2 * c : 2 * c + 1) * p.rec_stride;
-#pragma unroll
-          for (int r = 0; r < N; ++r)
-            if (r < nrows) rec[r * D + t] = __uint_as_float(ov[r]);
-          if (t < nrows) reinterpret_cast<float2*>(rec + N * D)[t] = make_float2(mref_c, L_c);
-        }
-        if (g == n - 1 && t == 0) {
+        for (int r = 0; r < NC; ++r) ls[r] = lpart[r];
+        const float wl = tcm::column_reduce<NC, false>(ls, lane);
+        float* rl = red + 2 * 4 * NC;
+        if (lane < NC) rl[(warp & 3) * NC + lane] = wl;
+        tcm::named_sync_softmax(wg);
+        pend.on = true;
+        pend.g = g;
+        pend.obuf = j & 1;
+        pend.b = w.b;
+        pend.kvh = kvh;
+        pend.rc = rc;
+        pend.nrows = nrows;
+        pend.complete = first_x == 0 && w.x == w.tiles - 1;
+        pend.slot = j == 0 ? 2 * c : 2 * c + 1;
+        pend.L_c = (rl[jc] + rl[NC + jc]) + (rl[2 * NC + jc] + rl[3 * NC + jc]);
+        pend.m_c = mref_c;
+        if (g == n - 1 && wg == 0 && t == 0) {
           // the merge descriptor: this CTA's last unit continues in the next CTAs and
           // started here, so this CTA holds its first piece
           int4 dsc = make_int4(-1, 0, 0, 0);
           if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
             const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
-            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * G - 1) / W), w.b, w.k);
+            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.b, w.k);
           }
           p.tc_desc[c] = dsc;
         }
       }
       w.next(p, upb);
     }
+    if (pend.on) flush(pend);
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
-      if (t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
+      if (wg == 0 && t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     }
   }
   grid_launch_dependents();
@@ -581,8 +617,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
 
 // Combines the partial records of every unit cut by a range boundary (one CTA per
 // decode CTA; the descriptor of CTA c names the unit whose first piece c holds and the
-// last CTA c1 with a piece of it: pieces in record slots desc.x, then 2c' for
-// c' = c+1..c1, in that order), then writes zeros for sequences with no keys.
+// last CTA c1 with a piece of it: the pieces are in record slots desc.x, then 2c' for
+// c' = c+S, c+2S, ..., c1 (the same CTA of the following groups), in that order), then
+// writes zeros for sequences with no keys.
 template <int N>
 __global__ void __launch_bounds__(128) tcm_merge_kernel(const DecodeParams p) {
   constexpr int D = tcm::kD;
@@ -592,21 +629,22 @@ __global__ void __launch_bounds__(128) tcm_merge_kernel(const DecodeParams p) {
   const int4 dsc = p.tc_desc[c];
   if (dsc.x >= 0) {
     const int b = dsc.z;
-    const int kvh = dsc.w / p.row_chunks;
-    const int rc = dsc.w - kvh * p.row_chunks;
+    const int S = p.tc_group;
+    const int kvh = c % S + S * (dsc.w / p.row_chunks);
+    const int rc = dsc.w % p.row_chunks;
     const int nrows = min(N, p.rows - rc * N);
-    const int pieces = 1 + (dsc.y - c);
+    const int pieces = 1 + (dsc.y - c) / S;
     int i = (rc * N) / p.group, gg = rc * N - i * p.group;
     for (int r = 0; r < nrows; ++r) {
       float M = -INFINITY;
       for (int k = 0; k < pieces; ++k) {
-        const int slot = k == 0 ? dsc.x : 2 * (c + k);
+        const int slot = k == 0 ? dsc.x : 2 * (c + k * S);
         M = fmaxf(M, reinterpret_cast<const float2*>(p.records + static_cast<size_t>(slot) * p.rec_stride + N * D)[r].x);
       }
       float acc = 0.f, l = 0.f;
       if (M != -INFINITY) {
         for (int k = 0; k < pieces; ++k) {
-          const int slot = k == 0 ? dsc.x : 2 * (c + k);
+          const int slot = k == 0 ? dsc.x : 2 * (c + k * S);
           const float* rec = p.records + static_cast<size_t>(slot) * p.rec_stride;
           const float2 ml = reinterpret_cast<const float2*>(rec + N * D)[r];
           const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
