@@ -130,7 +130,7 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   int share_cap = 0;
   if (h.share_prefix) {
     share_cap = share_cap_for(rows);
-    if (share_cap < 2 || h.path == PA_PATH_SINGLE || h.path == PA_PATH_TCGEN05) return PA_ERR_UNSUPPORTED;
+    if (share_cap < 2 || h.path == PA_PATH_SINGLE) return PA_ERR_UNSUPPORTED;
   }
   if (h.path == PA_PATH_TCGEN05) {
     // tokens-on-M tensor-core kernel: head_dim 128, its own persistent equal-tile schedule
@@ -139,7 +139,7 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   }
   int path = h.path;
   if (path == PA_PATH_AUTO) path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
-  // a shared-prefix unit holds share_cap sequences' rows in one CTA
+  // a shared-prefix unit holds share_cap sequences' rows in one CTA (32 rows)
   const int rpc = share_cap ? pa::kTileMaxRows : rows_per_cta_for(path, rows);
   const int64_t row_chunks = ceil_div(rows, rpc);
   if (num_kv_heads * row_chunks > 65535) return PA_ERR_UNSUPPORTED;  // grid x
@@ -246,10 +246,18 @@ size_t tcm_desc_offset(const pa_plan_t& plan, int32_t head_dim) {
   return align256(static_cast<size_t>(2) * plan.num_ctas * tcm_rec_stride(plan, head_dim) * 4);
 }
 
+// With prefix sharing the shared-prefix length of every window of share_cap sequences
+// follows the descriptors.
+size_t tcm_prefix_offset(const pa_plan_t& plan, int32_t head_dim) {
+  return align256(tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas));
+}
+
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
   if (plan.path == PA_PATH_TCGEN05) {
     if (num_seqs == 0) return 0;
+    if (plan.share_cap > 1)
+      return tcm_prefix_offset(plan, head_dim) + 4 * static_cast<size_t>(ceil_div(num_seqs, plan.share_cap));
     return tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas);
   }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
@@ -271,10 +279,13 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
     return PA_ERR_INVALID_ARG;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
   if (plan.path == PA_PATH_TCGEN05) {
-    if (plan.schedule != PA_SCHEDULE_PERSISTENT || plan.share_cap != 0 || plan.share_split_blocks != 0 ||
-        plan.num_ctas <= 0 || plan.num_ctas > (1 << 20) || plan.rows_per_cta != rows_per_cta_for(plan.path, rows))
+    if (plan.schedule != PA_SCHEDULE_PERSISTENT || plan.share_split_blocks != 0 || plan.num_ctas <= 0 ||
+        plan.num_ctas > (1 << 20))
       return PA_ERR_INVALID_ARG;
-    return PA_OK;
+    if (plan.share_cap != 0)
+      return plan.share_cap == share_cap_for(rows) && plan.rows_per_cta == pa::kTcmMaxRows ? PA_OK
+                                                                                            : PA_ERR_INVALID_ARG;
+    return plan.rows_per_cta == rows_per_cta_for(plan.path, rows) ? PA_OK : PA_ERR_INVALID_ARG;
   }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (plan.num_ctas <= 0 || plan.num_ctas > (1 << 20)) return PA_ERR_INVALID_ARG;
@@ -426,8 +437,10 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   if (plan->path == PA_PATH_TCGEN05) {
     if (head_dim != 128) return PA_ERR_UNSUPPORTED;
     p.num_ctas = plan->num_ctas;
+    p.share_cap = plan->share_cap;
     p.rec_stride = tcm_rec_stride(*plan, head_dim);
     p.records = reinterpret_cast<float*>(ws);
+    if (plan->share_cap > 1) p.win_prefix = reinterpret_cast<int32_t*>(ws + tcm_prefix_offset(*plan, head_dim));
     p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
     // CTAs per group: the largest divisor of H_kv that the grid holds
     p.tc_group = 1;

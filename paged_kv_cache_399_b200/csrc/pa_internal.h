@@ -70,6 +70,7 @@ struct DecodeParams {
   // in later CTAs: {record slot, last CTA with a piece, sequence, unit}, or {-1, ...}
   int4* tc_desc;
   int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
+  int32_t* win_prefix;           // tcgen05 path with prefix sharing: shared blocks per window
 };
 
 // Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).

@@ -1473,9 +1473,14 @@ cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUten
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
+  if (p.share_cap > 1) {
+    const int windows = (p.num_seqs + p.share_cap - 1) / p.share_cap;
+    e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(128), 0, stream, p);
+    if (e != cudaSuccess) return e;
+  }
   e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kD), 0, stream, p);
+  return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kMergeThreads), 0, stream, p);
 }
 
 template <int D>

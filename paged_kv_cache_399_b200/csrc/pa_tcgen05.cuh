@@ -48,6 +48,7 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
 constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
+constexpr int kMergeThreads = 256;
 
 template <int N>
 struct Smem {
@@ -70,26 +71,118 @@ struct Bars {
   uint64_t drain;
 };
 
-// Position in the CTA's tile range: sequence b, unit k (kv head x row chunk) of it,
-// tile x of the unit.
+// Tiles of every unit of window w (one thread, for the partition scan).
+__device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
+  const int cap = p.share_cap > 1 ? p.share_cap : 1;
+  const int b0 = w * cap;
+  const int m = min(cap, p.num_seqs - b0);
+  if (m <= 0) return 0;
+  const int P = cap > 1 ? __ldg(p.win_prefix + w) : 0;
+  int tiles = (P + kTileBlocks - 1) / kTileBlocks;
+  for (int jj = 0; jj < m; ++jj)
+    tiles += (num_blocks_of(p, __ldg(p.context_lens + b0 + jj)) - P + kTileBlocks - 1) / kTileBlocks;
+  return tiles;
+}
+
+// Position in the CTA's tile range, kept by a whole warp. A window is `cap` consecutive
+// sequences (cap = 1 without prefix sharing) whose tables may start with the same P
+// physical blocks; its units are (kv-head index, row chunk) of this CTA, and every unit
+// walks the window's tiles: the shared prefix (P blocks, read once for all members) then
+// each member's own blocks. Lane jj holds member jj's context length and blocks, so moving
+// between members takes shuffles, not loads.
 struct Walk {
-  int b, k, x, ctx, nblk, tiles;
-  __device__ __forceinline__ void seq(const DecodeParams& p) {
-    ctx = b < p.num_seqs ? __ldg(p.context_lens + b) : 0;
-    nblk = num_blocks_of(p, ctx);
-    ctx = min(ctx, nblk * kBlockSize);
-    tiles = (nblk + kTileBlocks - 1) / kTileBlocks;
+  int w, k, x;          // window, unit of the window, tile of the unit
+  int b0, m, P, tiles;  // window: first sequence, members, shared blocks, tiles of a unit
+  int j, y, seg;        // segment: member j (-1: the shared prefix), its tile y, its tiles
+  int ctx, nblk;        // member j: context length (clamped to its blocks) and blocks
+  int lctx, lnblk;      // this lane's member
+
+  __device__ __forceinline__ int own_tiles_lane() const {
+    return (lnblk - P + kTileBlocks - 1) / kTileBlocks;
   }
-  __device__ __forceinline__ void next(const DecodeParams& p, int upb) {
-    if (++x < tiles) return;
+  __device__ __forceinline__ void member(int jj) {
+    ctx = __shfl_sync(kFull, lctx, jj);
+    nblk = __shfl_sync(kFull, lnblk, jj);
+  }
+  __device__ __forceinline__ void window(const DecodeParams& p) {
+    const int lane = threadIdx.x & 31;
+    const int cap = p.share_cap > 1 ? p.share_cap : 1;
+    b0 = w * cap;
+    m = min(cap, p.num_seqs - b0);
+    tiles = 0;
+    lctx = 0;
+    lnblk = 0;
+    if (m <= 0) return;
+    P = cap > 1 ? __ldg(p.win_prefix + w) : 0;
+    if (lane < m) {
+      lctx = __ldg(p.context_lens + b0 + lane);
+      lnblk = num_blocks_of(p, lctx);
+      lctx = min(lctx, lnblk * kBlockSize);
+    }
+    int t = lane < m ? own_tiles_lane() : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+    tiles = t + (P + kTileBlocks - 1) / kTileBlocks;
+  }
+  __device__ __forceinline__ void seek(int xx) {
+    const int lane = threadIdx.x & 31;
+    x = xx;
+    int r = xx;
+    const int sh = (P + kTileBlocks - 1) / kTileBlocks;
+    if (r < sh) {
+      j = -1;
+      y = r;
+      seg = sh;
+      ctx = 0;
+      nblk = P;
+      return;
+    }
+    r -= sh;
+    // member holding own tile r: inclusive prefix sum of the members' own tiles
+    int ot = lane < m ? own_tiles_lane() : 0;
+    int incl = ot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const unsigned past = __ballot_sync(kFull, lane < m && incl <= r);  // members wholly before r
+    const int jj = __popc(past);
+    const int before = jj > 0 ? __shfl_sync(kFull, incl, jj - 1) : 0;
+    j = jj;
+    y = r - before;
+    seg = __shfl_sync(kFull, ot, jj);
+    member(jj);
+  }
+  __device__ __forceinline__ void next(const DecodeParams& p, int upb, int nwin) {
+    const int lane = threadIdx.x & 31;
+    ++x;
+    if (++y < seg) return;
+    if (x < tiles) {  // the next member with own tiles
+      const unsigned more = __ballot_sync(kFull, lane > j && lane < m && own_tiles_lane() > 0);
+      const int jj = __ffs(more) - 1;
+      j = jj;
+      y = 0;
+      seg = __shfl_sync(kFull, own_tiles_lane(), jj & 31);
+      member(jj & 31);
+      return;
+    }
     x = 0;
-    if (++k < upb) return;
+    if (++k < upb) {
+      seek(0);
+      return;
+    }
     k = 0;
     do {
-      ++b;
-      seq(p);
-    } while (tiles == 0 && b < p.num_seqs);
+      ++w;
+      window(p);
+    } while (tiles == 0 && w < nwin);
+    if (w < nwin) seek(0);
   }
+  // the tile's blocks: [bstart, bend) of table row `row`
+  __device__ __forceinline__ int row() const { return b0 + (j < 0 ? 0 : j); }
+  __device__ __forceinline__ int bstart() const { return (j < 0 ? 0 : P) + kTileBlocks * y; }
+  __device__ __forceinline__ int bend() const { return j < 0 ? P : nblk; }
 };
 
 // Named barrier of one softmax warpgroup (ids 1 and 2).
@@ -164,24 +257,23 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   grid_dependency_wait();
 
   // ---- this CTA's group, kv-head set and tile range [t0, t1) of the W tiles every group
-  // walks: prefix sums over the sequences
+  // walks: prefix sums over the windows
   const int S = p.tc_group;
   const int li = c % S;
   const int NG = static_cast<int>(gridDim.x) / S;
-  const int upb = (p.num_kv_heads / S) * p.row_chunks;  // units per sequence of one CTA
+  const int upb = (p.num_kv_heads / S) * p.row_chunks;  // units per window of one CTA
+  const int cap = p.share_cap > 1 ? p.share_cap : 1;
+  const int nwin = (p.num_seqs + cap - 1) / cap;
+  const int rpm = p.rows;  // query rows of one member (sequence)
   long long* wsum = reinterpret_cast<long long*>(smem + L::offScan);
   int* start = reinterpret_cast<int*>(smem + L::offScan + 96);
   long long W, t0, t1;
   int NGe;  // groups that take part: at most one per tile, so that every range is non-empty
   {
-    const int B = p.num_seqs;
-    const int chunk = (B + tcm::kThreads - 1) / tcm::kThreads;
-    const int s0 = min(B, static_cast<int>(threadIdx.x) * chunk), s1 = min(B, s0 + chunk);
+    const int chunk = (nwin + tcm::kThreads - 1) / tcm::kThreads;
+    const int s0 = min(nwin, static_cast<int>(threadIdx.x) * chunk), s1 = min(nwin, s0 + chunk);
     long long local = 0;
-    for (int b = s0; b < s1; ++b) {
-      const int nb = num_blocks_of(p, __ldg(p.context_lens + b));
-      local += static_cast<long long>((nb + kTileBlocks - 1) / kTileBlocks) * upb;
-    }
+    for (int ww = s0; ww < s1; ++ww) local += static_cast<long long>(tcm::window_tiles(p, ww)) * upb;
     long long v = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -203,11 +295,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     const long long excl = base + v - local;
     if (local > 0 && t0 < t1 && t0 >= excl && t0 < excl + local) {
       long long acc = excl;
-      for (int b = s0; b < s1; ++b) {
-        const int nb = num_blocks_of(p, __ldg(p.context_lens + b));
-        const long long tb = static_cast<long long>((nb + kTileBlocks - 1) / kTileBlocks) * upb;
+      for (int ww = s0; ww < s1; ++ww) {
+        const long long tb = static_cast<long long>(tcm::window_tiles(p, ww)) * upb;
         if (t0 < acc + tb) {
-          start[0] = b;
+          start[0] = ww;
           start[1] = static_cast<int>(t0 - acc);
           break;
         }
@@ -226,10 +317,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   auto unit_kvh = [&](int k) { return li + S * (k / p.row_chunks); };
   auto unit_rc = [&](int k) { return k % p.row_chunks; };
   tcm::Walk w0;
-  w0.b = start[0];
-  w0.seq(p);
+  w0.w = start[0];
+  w0.window(p);  // every warp: its lanes hold the window's members
   w0.k = start[1] / w0.tiles;
-  w0.x = start[1] - w0.k * w0.tiles;
+  w0.seek(start[1] - w0.k * w0.tiles);
 
   if (warp == tcm::kMmaWarp) {
     tmem_alloc(&tmem_base_s, 4 * N < 32 ? 32 : 4 * N);
@@ -253,9 +344,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     tcm::Walk w = w0;
     const int oob = static_cast<int>(p.num_blocks);  // block id past the pool: TMA fills zeros
     auto block_id = [&](const tcm::Walk& at) {
-      const int blk = at.x * kTileBlocks + lane;
-      return (lane < kTileBlocks && blk < at.nblk)
-                 ? __ldg(p.block_tables + static_cast<size_t>(at.b) * p.max_blocks + blk)
+      const int blk = at.bstart() + lane;
+      return (lane < kTileBlocks && blk < at.bend())
+                 ? __ldg(p.block_tables + static_cast<size_t>(at.row()) * p.max_blocks + blk)
                  : oob;
     };
     int phys_next = block_id(w);
@@ -269,16 +360,18 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         // Q rows of the unit -> Q[j & 1], 128-byte swizzled K-major; zeros for padded rows
         const int kvh = unit_kvh(w.k);
         const int rc = unit_rc(w.k);
-        const int nrows = min(N, p.rows - rc * N);
         uint8_t* qb = smem + L::offQ + (j & 1) * L::kQ;
         if (lane < N) {
           const int r = lane;
-          const bool valid = r < nrows;
-          const int rr = rc * N + r;
+          const int cg = rc * N + r;  // row of the window: member cg / rpm, row cg % rpm of it
+          const bool valid = cg < w.m * rpm;
+          const int mem = valid ? cg / rpm : 0;
+          const int rr = cg - mem * rpm;
           const int i = valid ? rr / p.group : 0;
           const int gg = valid ? rr - i * p.group : 0;
           const uint4* src = reinterpret_cast<const uint4*>(
-              p.query + (static_cast<size_t>(w.b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D);
+              p.query +
+              (static_cast<size_t>((w.b0 + mem) * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D);
 #pragma unroll
           for (int ch = 0; ch < D / 8; ++ch) {
             const uint4 v = valid ? __ldg(src + ch) : make_uint4(0, 0, 0, 0);
@@ -294,7 +387,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       const int kvh = unit_kvh(w.k);
       const int ph = __shfl_sync(kFull, phys_next, lane & (kTileBlocks - 1));
       tcm::Walk wn = w;
-      wn.next(p, upb);
+      wn.next(p, upb, nwin);
       if (g + 1 < n) phys_next = block_id(wn);
       if (g >= stages) ok = __all_sync(kFull, mbar_wait_bounded(&empty[s], ((g / stages) - 1) & 1));
       if (!ok) break;
@@ -316,7 +409,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     }
   } else if (warp == tcm::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks (its lanes hold the window's members); lane 0 tests the barriers
+    // and issues, and its decisions are broadcast so that the warp stays converged.
+    {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, N, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, N, 1, 1);
       tcm::Walk w = w0;      // position of the next S
@@ -328,22 +423,28 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       unsigned idle_polls = 0;
       while (gp < n) {
         bool progressed = false;
-        if (gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
-            mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1)) {
-          const int sh = 2 * (gp & 3);
-          const int obuf = (ring >> sh) & 1;
-          const bool first = (ring >> (sh + 1)) & 1;
-          tc_fence_after_sync();
-          const uint32_t vst = sm + L::offV + (gp % kVStages) * tcm::kStageBytes;
-          const uint32_t pst = sm + L::offP + (gp & 1) * L::kP;
+        bool pv_ready = false;
+        if (lane == 0)
+          pv_ready = gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
+                     mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1);
+        if (__shfl_sync(kFull, pv_ready, 0)) {
+          if (lane == 0) {
+            const int sh = 2 * (gp & 3);
+            const int obuf = (ring >> sh) & 1;
+            const bool first = (ring >> (sh + 1)) & 1;
+            tc_fence_after_sync();
+            const uint32_t vst = sm + L::offV + (gp % kVStages) * tcm::kStageBytes;
+            const uint32_t pst = sm + L::offP + (gp & 1) * L::kP;
 #pragma unroll
-          for (int kk = 0; kk < kTileTokens / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(vst + kk * 2048, tcm::kHalfBytes, 1024);
-            const uint64_t bd = smem_desc_noswizzle(pst + kk * 256, 128, tcm::kPGroupBytes);
-            tc_mma_bf16(tmem + 2 * N + obuf * N, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < kTileTokens / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(vst + kk * 2048, tcm::kHalfBytes, 1024);
+              const uint64_t bd = smem_desc_noswizzle(pst + kk * 256, 128, tcm::kPGroupBytes);
+              tc_mma_bf16(tmem + 2 * N + obuf * N, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+            }
+            tc_commit(&bars.pv_done[gp & 1]);
+            tc_commit(&bars.v_empty[gp % kVStages]);
           }
-          tc_commit(&bars.pv_done[gp & 1]);
-          tc_commit(&bars.v_empty[gp % kVStages]);
+          __syncwarp();
           ++gp;
           progressed = true;
         }
@@ -351,27 +452,33 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           const bool first = gs == 0 || w.x == 0;
           const int jn = first ? js + 1 : js;
           const int s = gs % kKStages;
-          if ((!first || mbar_test_wait(&bars.q_full[jn & 1], (jn >> 1) & 1)) &&
-              mbar_test_wait(&bars.k_full[s], (gs / kKStages) & 1) &&
-              (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1))) {
+          bool s_ready = false;
+          if (lane == 0)
+            s_ready = (!first || mbar_test_wait(&bars.q_full[jn & 1], (jn >> 1) & 1)) &&
+                      mbar_test_wait(&bars.k_full[s], (gs / kKStages) & 1) &&
+                      (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1));
+          if (__shfl_sync(kFull, s_ready, 0)) {
             js = jn;
             const int obuf = js & 1;
             const bool last = gs == n - 1 || w.x == w.tiles - 1;
-            tc_fence_after_sync();
-            const uint32_t kst = sm + L::offK + s * tcm::kStageBytes;
-            const uint32_t qst = sm + L::offQ + obuf * L::kQ;
+            if (lane == 0) {
+              tc_fence_after_sync();
+              const uint32_t kst = sm + L::offK + s * tcm::kStageBytes;
+              const uint32_t qst = sm + L::offQ + obuf * L::kQ;
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t ad = smem_desc_sw128(kst + (k >> 2) * tcm::kHalfBytes + (k & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(qst + (k >> 2) * (N * 128) + (k & 3) * 32, 16, 1024);
-              tc_mma_bf16(tmem + (gs & 1) * N, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+              for (int k = 0; k < D / 16; ++k) {
+                const uint64_t ad = smem_desc_sw128(kst + (k >> 2) * tcm::kHalfBytes + (k & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(qst + (k >> 2) * (N * 128) + (k & 3) * 32, 16, 1024);
+                tc_mma_bf16(tmem + (gs & 1) * N, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+              }
+              tc_commit(&bars.s_full[gs & 1]);
+              tc_commit(&bars.k_empty[s]);
+              if (last) tc_commit(&bars.q_empty[obuf]);
             }
-            tc_commit(&bars.s_full[gs & 1]);
-            tc_commit(&bars.k_empty[s]);
-            if (last) tc_commit(&bars.q_empty[obuf]);
+            __syncwarp();
             const int sh = 2 * (gs & 3);
             ring = (ring & ~(3 << sh)) | (obuf << sh) | ((first ? 1 : 0) << (sh + 1));
-            w.next(p, upb);
+            w.next(p, upb, nwin);
             ++gs;
             progressed = true;
           }
@@ -380,7 +487,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           idle_since = 0;
           idle_polls = 0;
         } else if ((++idle_polls & 63) == 0) {  // the clock is read once every 64 idle polls
-          const unsigned long long now = global_timer_ns();
+          const unsigned long long now = __shfl_sync(kFull, global_timer_ns(), 0);
           if (idle_since == 0) {
             idle_since = now;
           } else if (now - idle_since > kWaitLimitNs) {
@@ -389,9 +496,11 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           }
         }
       }
-      if (!ok) record_error(kErrTimeoutDecode);
-      tc_commit(&bars.drain);  // every MMA issued so far has completed once drain flips
-      if (!mbar_wait_bounded(&bars.drain, 0)) record_error(kErrTimeoutDrain);
+      if (lane == 0) {
+        if (!ok) record_error(kErrTimeoutDecode);
+        tc_commit(&bars.drain);  // every MMA issued so far has completed once drain flips
+        if (!mbar_wait_bounded(&bars.drain, 0)) record_error(kErrTimeoutDrain);
+      }
     }
     __syncwarp();
   } else {
@@ -418,7 +527,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     // A unit piece whose output is written one tile later: by then its last PV is done.
     struct Pending {
       bool on, complete;
-      int g, obuf, b, kvh, rc, nrows, slot;
+      int g, obuf, b0, kvh, rc, nrows, slot;
       float L_c, m_c;  // l and the reference maximum of column cb + (lane % NC)
     } pend;
     pend.on = false;
@@ -432,18 +541,24 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       tc_fence_before_sync();
       if (!ok) return;  // nothing is written after a timeout
       if (e.complete) {
-        int i = (e.rc * N + cb) / p.group, gg = e.rc * N + cb - i * p.group;
+        // column cb + r = row cg of the window: member cg / rpm, (i, g) of its row cg % rpm
+        int cg = e.rc * N + cb;
+        int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+        int gg = cg - mem * rpm - i * p.group;
 #pragma unroll
         for (int r = 0; r < NC; ++r) {
           const float lr = __shfl_sync(kFull, e.L_c, r);
           if (cb + r < e.nrows) {
             const float inv = lr > 0.f ? 1.f / lr : 0.f;
-            p.out[(static_cast<size_t>(e.b * p.q_per_seq + i) * p.num_q_heads + e.kvh * p.group + gg) * D + t] =
-                static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
+            p.out[(static_cast<size_t>((e.b0 + mem) * p.q_per_seq + i) * p.num_q_heads + e.kvh * p.group + gg) * D +
+                  t] = static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
           }
           if (++gg == p.group) {
             gg = 0;
-            ++i;
+            if (++i == p.q_per_seq) {
+              i = 0;
+              ++mem;
+            }
           }
         }
       } else {
@@ -462,15 +577,25 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         first_x = w.x;
         kvh = unit_kvh(w.k);
         rc = unit_rc(w.k);
-        nrows = min(N, p.rows - rc * N);
-        int i = (rc * N + cb) / p.group, gg = rc * N + cb - i * p.group;
-        minlim = w.ctx - p.q_per_seq + (rc * N) / p.group;
+        nrows = min(N, w.m * rpm - rc * N);
+        // the last visible token of each column's row (member mem of the window, query i);
+        // padded columns see everything (their Q is zero and their output unused)
+        int cg = rc * N + cb;
+        int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+        int gg = cg - mem * rpm - i * p.group;
+        auto ctx_of = [&](int mm) { return __shfl_sync(kFull, w.lctx, mm & 31); };  // lane mm: member mm
+        int cm = ctx_of(mem);
+        minlim = (cap == 1) ? cm - p.q_per_seq + (rc * N) / p.group : 0;
 #pragma unroll
         for (int r = 0; r < NC; ++r) {
-          lim[r] = cb + r < nrows ? w.ctx - p.q_per_seq + i : w.ctx - 1;
+          lim[r] = cb + r < nrows ? cm - p.q_per_seq + i : INT_MAX;
           if (++gg == p.group) {
             gg = 0;
-            ++i;
+            if (++i == p.q_per_seq) {
+              i = 0;
+              ++mem;
+              cm = ctx_of(mem);
+            }
           }
           mref[r] = -INFINITY;
           lpart[r] = 0.f;
@@ -486,13 +611,29 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[g & 1]);
-      const int tok = w.x * kTileTokens + t;
-      const bool edge = w.x * kTileTokens + kTileTokens - 1 > minlim;
+      // visible: the shared prefix for every column below P*16; a member's own tile for
+      // that member's columns up to their causal limit
+      const int tok0 = w.bstart() * kBlockSize;
+      const int tok = tok0 + t;
+      bool edge;
+      int lo = 0, hi = NC, tok_hi = INT_MAX;
+      bool use_lim = true;
+      if (w.j < 0) {
+        tok_hi = w.P * kBlockSize;
+        edge = tok0 + kTileTokens > tok_hi;
+        use_lim = false;
+      } else if (cap > 1) {
+        edge = true;
+        lo = max(0, w.j * rpm - rc * N - cb);
+        hi = min(NC, (w.j + 1) * rpm - rc * N - cb);
+      } else {
+        edge = tok0 + kTileTokens - 1 > minlim;
+      }
       float x[NC], tmp[NC];
 #pragma unroll
       for (int r = 0; r < NC; ++r) {
         float v = __uint_as_float(sv[r]) * cs;
-        if (edge && tok > lim[r]) v = -INFINITY;
+        if (edge && (r < lo || r >= hi || tok >= tok_hi || (use_lim && tok > lim[r]))) v = -INFINITY;
         x[r] = v;
         tmp[r] = v;
       }
@@ -540,13 +681,13 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       }
       // the P^T buffer of this tile was read by the PV of tile g-2
       if (g >= 2) wait(&bars.pv_done[g & 1], ((g >> 1) - 1) & 1);
-      if (wg == 0 && w.x == w.tiles - 1 && (w.ctx & (kBlockSize - 1))) {
+      if (wg == 0 && w.j >= 0 && w.y == w.seg - 1 && (w.ctx & (kBlockSize - 1))) {
         // The sequence's last block is partly filled: its slots past the context may hold
         // any bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows
         // are cleared before the PV reads them.
         const int s = g % kVStages;
         wait(&bars.v_full[s], (g / kVStages) & 1);
-        const int jj = (w.nblk - 1) - w.x * kTileBlocks;
+        const int jj = (w.nblk - 1) - w.bstart();
         const int r0 = w.ctx & (kBlockSize - 1);
         const int nrow = kBlockSize - r0;
         uint8_t* vblk = smem + L::offV + s * tcm::kStageBytes + jj * kHalfTileBytes;
@@ -581,7 +722,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         pend.on = true;
         pend.g = g;
         pend.obuf = j & 1;
-        pend.b = w.b;
+        pend.b0 = w.b0;
         pend.kvh = kvh;
         pend.rc = rc;
         pend.nrows = nrows;
@@ -595,12 +736,12 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           int4 dsc = make_int4(-1, 0, 0, 0);
           if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
             const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
-            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.b, w.k);
+            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.w, w.k);
           }
           p.tc_desc[c] = dsc;
         }
       }
-      w.next(p, upb);
+      w.next(p, upb, nwin);
     }
     if (pend.on) flush(pend);
     if (!ok) {
@@ -615,50 +756,74 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   if (warp == tcm::kMmaWarp) tmem_dealloc(tmem, 4 * N < 32 ? 32 : 4 * N);
 }
 
-// Combines the partial records of every unit cut by a range boundary (one CTA per
+// Combines the partial records of every unit (window, kv head, row chunk) cut by a range
+// boundary (one CTA per
 // decode CTA; the descriptor of CTA c names the unit whose first piece c holds and the
 // last CTA c1 with a piece of it: the pieces are in record slots desc.x, then 2c' for
 // c' = c+S, c+2S, ..., c1 (the same CTA of the following groups), in that order), then
 // writes zeros for sequences with no keys.
 template <int N>
-__global__ void __launch_bounds__(128) tcm_merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const DecodeParams p) {
   constexpr int D = tcm::kD;
   grid_dependency_wait();
   const int c = blockIdx.x;
-  const int d = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int4 dsc = p.tc_desc[c];
   if (dsc.x >= 0) {
-    const int b = dsc.z;
+    const int cap = p.share_cap > 1 ? p.share_cap : 1;
+    const int rpm = p.rows;
+    const int b0 = dsc.z * cap;  // the window's first sequence
+    const int m = min(cap, p.num_seqs - b0);
     const int S = p.tc_group;
     const int kvh = c % S + S * (dsc.w / p.row_chunks);
     const int rc = dsc.w % p.row_chunks;
-    const int nrows = min(N, p.rows - rc * N);
+    const int nrows = min(N, m * rpm - rc * N);
     const int pieces = 1 + (dsc.y - c) / S;
-    int i = (rc * N) / p.group, gg = rc * N - i * p.group;
-    for (int r = 0; r < nrows; ++r) {
+    const float* recs = p.records;
+    const int rs = p.rec_stride, slot0 = dsc.x;
+    auto rec_of = [=](int k) {
+      return recs + static_cast<size_t>(k == 0 ? slot0 : 2 * (c + k * S)) * rs;
+    };
+    // one row per warp: lanes take the pieces for the maximum and the weights, then each
+    // lane accumulates 4 of the D columns over the pieces in order
+    for (int r = warp; r < nrows; r += tcm::kMergeThreads / 32) {
       float M = -INFINITY;
-      for (int k = 0; k < pieces; ++k) {
-        const int slot = k == 0 ? dsc.x : 2 * (c + k * S);
-        M = fmaxf(M, reinterpret_cast<const float2*>(p.records + static_cast<size_t>(slot) * p.rec_stride + N * D)[r].x);
-      }
-      float acc = 0.f, l = 0.f;
+      for (int k = lane; k < pieces; k += 32) M = fmaxf(M, reinterpret_cast<const float2*>(rec_of(k) + N * D)[r].x);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float l = 0.f;
       if (M != -INFINITY) {
-        for (int k = 0; k < pieces; ++k) {
-          const int slot = k == 0 ? dsc.x : 2 * (c + k * S);
-          const float* rec = p.records + static_cast<size_t>(slot) * p.rec_stride;
-          const float2 ml = reinterpret_cast<const float2*>(rec + N * D)[r];
-          const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
-          l = fmaf(ml.y, wk, l);
-          acc = fmaf(rec[r * D + d], wk, acc);
+        for (int k0 = 0; k0 < pieces; k0 += 32) {
+          float wk = 0.f, lk = 0.f;
+          if (k0 + lane < pieces) {
+            const float2 ml = reinterpret_cast<const float2*>(rec_of(k0 + lane) + N * D)[r];
+            wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+            lk = ml.y * wk;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
+          l += lk;
+          const int kn = min(32, pieces - k0);
+          for (int kk = 0; kk < kn; ++kk) {
+            const float wb = __shfl_sync(kFull, wk, kk);
+            const float4 o4 = reinterpret_cast<const float4*>(rec_of(k0 + kk) + r * D)[lane];
+            acc.x = fmaf(o4.x, wb, acc.x);
+            acc.y = fmaf(o4.y, wb, acc.y);
+            acc.z = fmaf(o4.z, wb, acc.z);
+            acc.w = fmaf(o4.w, wb, acc.w);
+          }
         }
       }
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      p.out[(static_cast<size_t>(b * p.q_per_seq + i) * p.num_q_heads + kvh * p.group + gg) * D + d] =
-          static_cast<uint16_t>(pack_bf16x2(acc * inv, 0.f) & 0xFFFFu);
-      if (++gg == p.group) {
-        gg = 0;
-        ++i;
-      }
+      const int cg = rc * N + r;
+      const int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+      const int gg = cg - mem * rpm - i * p.group;
+      uint2 packed;
+      packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      reinterpret_cast<uint2*>(p.out + (static_cast<size_t>((b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
+                                        kvh * p.group + gg) * D)[lane] = packed;
     }
   }
   // sequences without a visible key (context length 0) get zero rows
@@ -666,8 +831,40 @@ __global__ void __launch_bounds__(128) tcm_merge_kernel(const DecodeParams p) {
   for (int b = c; b < p.num_seqs; b += gridDim.x) {
     if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;
     uint16_t* o = p.out + static_cast<size_t>(b) * rq * D;
-    for (int e = d; e < rq * D; e += blockDim.x) o[e] = 0;
+    for (int e = threadIdx.x; e < rq * D; e += blockDim.x) o[e] = 0;
   }
+}
+
+// Prefix sharing: the shared prefix of each window of `cap` consecutive sequences, in
+// blocks: the longest run of table entries from position 0 on that all members share,
+// at most the blocks every member sees whole from every query row
+// (floor((ctx - q + 1) / 16)); 0 for a window of one sequence. One CTA per window.
+__global__ void __launch_bounds__(128) tcm_share_prepass(const DecodeParams p) {
+  grid_dependency_wait();
+  __shared__ int first_diff;
+  const int cap = p.share_cap;
+  const int w = blockIdx.x;
+  const int b0 = w * cap;
+  const int m = min(cap, p.num_seqs - b0);
+  if (threadIdx.x == 0) first_diff = INT_MAX;
+  int pcap = m >= 2 ? INT_MAX : 0;
+  for (int jj = 0; jj < m && pcap > 0; ++jj) {
+    const int cx = __ldg(p.context_lens + b0 + jj);
+    pcap = min(pcap, min(max(cx - p.q_per_seq + 1, 0) / kBlockSize, num_blocks_of(p, cx)));
+  }
+  __syncthreads();
+  const int32_t* lead = p.block_tables + static_cast<size_t>(b0) * p.max_blocks;
+  for (int x = threadIdx.x; x < pcap; x += blockDim.x) {
+    const int id = __ldg(lead + x);
+    for (int jj = 1; jj < m; ++jj)
+      if (__ldg(lead + static_cast<size_t>(jj) * p.max_blocks + x) != id) {
+        atomicMin(&first_diff, x);
+        break;
+      }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) p.win_prefix[w] = min(pcap, first_diff);
+  grid_launch_dependents();
 }
 
 }  // namespace pa

@@ -136,8 +136,9 @@ def test_plan_heuristic_host_logic(pa):
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, pa.PA_PATH_TCGEN05, schedule=pa.PA_SCHEDULE_GRID)
     with pytest.raises(pa.PAError):          # head_dim 128 only
         pa.pa_decode_plan(32, 6, 32, 8, 64, 1024, pa.PA_PATH_TCGEN05)
-    with pytest.raises(pa.PAError):          # sharing runs on the mma.sync tensor-core kernel
-        pa.pa_decode_plan(8, 1, 32, 8, 128, 64, pa.PA_PATH_TCGEN05, share_prefix=True)
+    # prefix sharing on the tcgen05 path: windows of 8 sequences x 4 rows = N 32
+    p = pa.pa_decode_plan(8, 1, 32, 8, 128, 64, pa.PA_PATH_TCGEN05, share_prefix=True)
+    assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (3, 2, 32, 8)
     forced = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, pa.PA_PATH_SINGLE, 64)
     assert (forced.path, forced.split_blocks, forced.num_splits, forced.rows_per_cta) == (1, 64, 128, 8)
     # rows beyond one CTA are split into row chunks
@@ -150,6 +151,7 @@ def test_plan_heuristic_host_logic(pa):
     {}, {"path": 1}, {"path": 2}, {"path": 3}, {"schedule": 2}, {"path": 1, "schedule": 2},
     {"share_prefix": True}, {"share_prefix": True, "schedule": 2}, {"split_blocks": 3},
     {"path": 3, "split_blocks": 2}, {"share_prefix": True, "split_blocks": 5},
+    {"path": 3, "share_prefix": True},
 ])
 def test_every_plan_passes_decode_validation(pa, hints):
     """A plan from pa_decode_plan is accepted by pa_decode's own checks (on a machine

@@ -52,6 +52,8 @@ PLANS = [
     # fewer / more CTAs than usual: units cut into many pieces, CTAs without work
     ("tcgen05_ctas3", dict(path=3, num_ctas=3)),
     ("tcgen05_ctas1000", dict(path=3, num_ctas=1000)),
+    ("tcgen05_share", dict(path=3, share_prefix=True)),
+    ("tcgen05_share_ctas5", dict(path=3, share_prefix=True, num_ctas=5)),
 ]
 
 
@@ -85,12 +87,14 @@ def _plan(w, plan_spec):
                                  w.head_dim, w.max_blocks_per_seq, **hints)
     except pa.PAError as exc:
         assert exc.status == pa.PA_ERR_UNSUPPORTED
-        if hints.get("share_prefix"):
-            pytest.skip("prefix sharing needs G*q <= 16 rows")
-        assert hints.get("path") == pa.PA_PATH_TCGEN05 and w.head_dim != 128
-        pytest.skip("the tcgen05 path runs head_dim 128")
+        if hints.get("path") == pa.PA_PATH_TCGEN05 and w.head_dim != 128:
+            pytest.skip("the tcgen05 path runs head_dim 128")
+        assert hints.get("share_prefix")
+        pytest.skip("prefix sharing needs G*q <= 16 rows")
     if plan.path == pa.PA_PATH_TCGEN05:
         assert plan.schedule == pa.PA_SCHEDULE_PERSISTENT and plan.rows_per_cta in (16, 32)
+        assert plan.share_cap == (32 // (w.num_q_heads // w.num_kv_heads * w.q_per_seq)
+                                  if hints.get("share_prefix") else 0)
     if num_ctas is not None:
         plan.num_ctas = num_ctas
     return plan
