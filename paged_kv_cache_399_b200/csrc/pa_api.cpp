@@ -138,7 +138,17 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     schedule = PA_SCHEDULE_PERSISTENT;
   }
   int path = h.path;
-  if (path == PA_PATH_AUTO) path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
+  if (path == PA_PATH_AUTO) {
+    // measured on B200: the tcgen05 kernel wins for head_dim 128 with more than 16 rows per
+    // kv head or with prefix sharing; mma.sync tiles win below that; CUDA cores for <= 2 rows
+    if (head_dim == 128 && (rows > 16 || share_cap > 0) && h.schedule != PA_SCHEDULE_GRID &&
+        h.split_blocks == 0) {
+      path = PA_PATH_TCGEN05;
+      schedule = PA_SCHEDULE_PERSISTENT;
+    } else {
+      path = (rows <= 2 && share_cap == 0) ? PA_PATH_SINGLE : PA_PATH_TILE;
+    }
+  }
   // a shared-prefix unit holds share_cap sequences' rows in one CTA (32 rows)
   const int rpc = share_cap ? pa::kTileMaxRows : rows_per_cta_for(path, rows);
   const int64_t row_chunks = ceil_div(rows, rpc);

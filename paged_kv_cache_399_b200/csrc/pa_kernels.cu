@@ -1475,7 +1475,7 @@ cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUten
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
   if (p.share_cap > 1) {
     const int windows = (p.num_seqs + p.share_cap - 1) / p.share_cap;
-    e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(128), 0, stream, p);
+    e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(256), 0, stream, p);
     if (e != cudaSuccess) return e;
   }
   e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);

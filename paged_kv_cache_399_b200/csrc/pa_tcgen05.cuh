@@ -48,7 +48,7 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
 constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
-constexpr int kMergeThreads = 256;
+constexpr int kMergeThreads = 1024;  // one warp per row of a unit (N <= 32)
 
 template <int N>
 struct Smem {
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const Dec
       return recs + static_cast<size_t>(k == 0 ? slot0 : 2 * (c + k * S)) * rs;
     };
     // one row per warp: lanes take the pieces for the maximum and the weights, then each
-    // lane accumulates 4 of the D columns over the pieces in order
+    // lane accumulates 4 of the D columns over the pieces in order, 4 pieces' loads at a time
     for (int r = warp; r < nrows; r += tcm::kMergeThreads / 32) {
       float M = -INFINITY;
       for (int k = lane; k < pieces; k += 32) M = fmaxf(M, reinterpret_cast<const float2*>(rec_of(k) + N * D)[r].x);
@@ -805,13 +805,22 @@ __global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const Dec
           for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
           l += lk;
           const int kn = min(32, pieces - k0);
-          for (int kk = 0; kk < kn; ++kk) {
-            const float wb = __shfl_sync(kFull, wk, kk);
-            const float4 o4 = reinterpret_cast<const float4*>(rec_of(k0 + kk) + r * D)[lane];
-            acc.x = fmaf(o4.x, wb, acc.x);
-            acc.y = fmaf(o4.y, wb, acc.y);
-            acc.z = fmaf(o4.z, wb, acc.z);
-            acc.w = fmaf(o4.w, wb, acc.w);
+          for (int kk = 0; kk < kn; kk += 4) {
+            float4 o4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              o4[u] = kk + u < kn ? reinterpret_cast<const float4*>(rec_of(k0 + kk + u) + r * D)[lane]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float wb = __shfl_sync(kFull, wk, (kk + u) & 31);
+              if (kk + u < kn) {
+                acc.x = fmaf(o4[u].x, wb, acc.x);
+                acc.y = fmaf(o4[u].y, wb, acc.y);
+                acc.z = fmaf(o4[u].z, wb, acc.z);
+                acc.w = fmaf(o4[u].w, wb, acc.w);
+              }
+            }
           }
         }
       }
@@ -839,29 +848,36 @@ __global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const Dec
 // blocks: the longest run of table entries from position 0 on that all members share,
 // at most the blocks every member sees whole from every query row
 // (floor((ctx - q + 1) / 16)); 0 for a window of one sequence. One CTA per window.
-__global__ void __launch_bounds__(128) tcm_share_prepass(const DecodeParams p) {
+__global__ void __launch_bounds__(256) tcm_share_prepass(const DecodeParams p) {
   grid_dependency_wait();
   __shared__ int first_diff;
   const int cap = p.share_cap;
   const int w = blockIdx.x;
   const int b0 = w * cap;
   const int m = min(cap, p.num_seqs - b0);
-  if (threadIdx.x == 0) first_diff = INT_MAX;
-  int pcap = m >= 2 ? INT_MAX : 0;
-  for (int jj = 0; jj < m && pcap > 0; ++jj) {
-    const int cx = __ldg(p.context_lens + b0 + jj);
-    pcap = min(pcap, min(max(cx - p.q_per_seq + 1, 0) / kBlockSize, num_blocks_of(p, cx)));
+  __shared__ int pcap_s;
+  if (threadIdx.x == 0) {
+    first_diff = INT_MAX;
+    pcap_s = m >= 2 ? INT_MAX : 0;
   }
   __syncthreads();
-  const int32_t* lead = p.block_tables + static_cast<size_t>(b0) * p.max_blocks;
-  for (int x = threadIdx.x; x < pcap; x += blockDim.x) {
-    const int id = __ldg(lead + x);
-    for (int jj = 1; jj < m; ++jj)
-      if (__ldg(lead + static_cast<size_t>(jj) * p.max_blocks + x) != id) {
-        atomicMin(&first_diff, x);
-        break;
-      }
+  if (m >= 2 && static_cast<int>(threadIdx.x) < m) {  // thread jj: member jj (cap <= 32)
+    const int cx = __ldg(p.context_lens + b0 + threadIdx.x);
+    atomicMin(&pcap_s, min(max(cx - p.q_per_seq + 1, 0) / kBlockSize, num_blocks_of(p, cx)));
   }
+  __syncthreads();
+  const int pcap = pcap_s;
+  // every (position, member) pair is one independent comparison with the first member
+  const int32_t* lead = p.block_tables + static_cast<size_t>(b0) * p.max_blocks;
+  const int pairs = m >= 2 ? pcap * (m - 1) : 0;
+  int mine = INT_MAX;
+#pragma unroll 4
+  for (int idx = threadIdx.x; idx < pairs; idx += blockDim.x) {
+    const int x = idx / (m - 1);
+    const int jj = 1 + (idx - x * (m - 1));
+    if (__ldg(lead + static_cast<size_t>(jj) * p.max_blocks + x) != __ldg(lead + x)) mine = min(mine, x);
+  }
+  if (mine != INT_MAX) atomicMin(&first_diff, mine);
   __syncthreads();
   if (threadIdx.x == 0) p.win_prefix[w] = min(pcap, first_diff);
   grid_launch_dependents();

@@ -111,17 +111,28 @@ def test_cache_write_rejects_bad_arguments_before_launch(pa):
 def test_plan_heuristic_host_logic(pa):
     # rows = G*q <= 2 -> CUDA-core kernel; more rows -> tensor-core tiles
     assert pa.pa_decode_plan(4, 1, 4, 2, 64, 5).path == pa.PA_PATH_SINGLE
-    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024)
+    p = pa.pa_decode_plan(32, 6, 32, 8, 64, 1024)      # 24 rows, head_dim 64: mma.sync tiles
     assert p.path == pa.PA_PATH_TILE and p.rows_per_cta == 24
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024)     # 24 rows, head_dim 128: tcgen05
+    assert (p.path, p.schedule, p.rows_per_cta) == (pa.PA_PATH_TCGEN05, pa.PA_SCHEDULE_PERSISTENT, 32)
+    p = pa.pa_decode_plan(64, 1, 32, 8, 128, 256)      # 4 rows: mma.sync tiles, grid schedule
+    assert (p.path, p.schedule, p.rows_per_cta) == (pa.PA_PATH_TILE, pa.PA_SCHEDULE_GRID, 8)
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, split_blocks=16)   # a forced split: grid tiles
+    assert (p.path, p.schedule) == (pa.PA_PATH_TILE, pa.PA_SCHEDULE_GRID)
     p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, schedule=pa.PA_SCHEDULE_PERSISTENT)
     assert p.schedule == pa.PA_SCHEDULE_PERSISTENT and p.num_ctas >= 1 and p.share_cap == 0
     p = pa.pa_decode_plan(4, 1, 64, 8, 128, 8192, schedule=pa.PA_SCHEDULE_GRID)
     assert p.num_splits > 1 and p.split_blocks * p.num_splits >= 8192
-    # prefix sharing: a shared unit holds 32 rows = 8 sequences of 4 rows
+    # prefix sharing: a shared unit holds 32 rows = 8 sequences of 4 rows; automatic choice:
+    # tcgen05 windows; mma.sync grid or persistent sharing on request
     p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, share_prefix=True)
+    assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (3, 2, 32, 8)
+    assert pa.pa_decode_workspace_size(p, 128, 1, 32, 8, 128, 144) > 0
+    p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, pa.PA_PATH_TILE, share_prefix=True)
     assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (2, 1, 32, 8)
     assert pa.pa_decode_workspace_size(p, 128, 1, 32, 8, 128, 144) > 0
-    p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, share_prefix=True, schedule=pa.PA_SCHEDULE_PERSISTENT)
+    p = pa.pa_decode_plan(128, 1, 32, 8, 128, 144, pa.PA_PATH_TILE, share_prefix=True,
+                          schedule=pa.PA_SCHEDULE_PERSISTENT)
     assert (p.path, p.schedule, p.rows_per_cta, p.share_cap) == (2, 2, 32, 8)
     with pytest.raises(pa.PAError) as exc:   # 24 rows per sequence: two do not fit 32 rows
         pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, share_prefix=True)
