@@ -58,8 +58,10 @@ struct Smem {
   static constexpr int offP = offQ + 2 * kQ;
   static constexpr int offK = offP + 2 * kP;
   static constexpr int offV = offK + kKStages * kStageBytes;
-  static constexpr int offRed = offV + kVStages * kStageBytes;  // [2 wg][3][4 warps][N/2] floats
-  static constexpr int offScan = offRed + 2 * 3 * 4 * (N / 2) * 4;  // [11] int64, then the start
+  // per softmax warpgroup: [3][4 warps][N/2] floats (2 maxima buffers, 1 sum), [2][4] votes
+  static constexpr int kRedWg = 3 * 4 * (N / 2) + 8;
+  static constexpr int offRed = offV + kVStages * kStageBytes;
+  static constexpr int offScan = offRed + 2 * kRedWg * 4;     // [11] int64, then the start
   static constexpr int offBars = offScan + 128;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && kQ % 1024 == 0, "swizzled operands need 1024-B alignment");
@@ -510,7 +512,8 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     const int cb = wg * NC;    // first column of this warpgroup
     const int t = (warp & 3) * 32 + lane;  // token of the tile = TMEM lane = head-dim index in O^T
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + L::offRed) + wg * 3 * 4 * NC;
+    float* red = reinterpret_cast<float*>(smem + L::offRed) + wg * L::kRedWg;
+    int* votes = reinterpret_cast<int*>(red + 3 * 4 * NC);  // [2][4 warps]
     const float cs = p.scale_log2;
     tcm::Walk w = w0;
     int j = -1, first_x = 0, kvh = 0, rc = 0, nrows = 0, minlim = 0;
@@ -637,12 +640,22 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         x[r] = v;
         tmp[r] = v;
       }
+      // ---- do the references still hold (every score within 2^8 of its column's reference)?
+      // Only then can the column maxima be skipped; a vote of the four warps decides.
+      bool over = false;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) over |= x[r] > mref[r] + tcm::kRescaleLog2;
+      const int* vb = votes + (g & 1) * 4;
+      const bool wover = __any_sync(kFull, over);
+      if (lane == 0) votes[(g & 1) * 4 + (warp & 3)] = wover ? 1 : 0;
+      tcm::named_sync_softmax(wg);
+      const int jc = lane % NC;
+      if ((vb[0] | vb[1] | vb[2] | vb[3]) != 0) {
       // ---- column maxima over the 128 tokens
       const float wmax = tcm::column_reduce<NC, true>(tmp, lane);
       float* rb = red + (g & 1) * 4 * NC;
       if (lane < NC) rb[(warp & 3) * NC + lane] = wmax;
       tcm::named_sync_softmax(wg);
-      const int jc = lane % NC;
       const float M = fmaxf(fmaxf(rb[jc], rb[NC + jc]), fmaxf(rb[2 * NC + jc], rb[3 * NC + jc]));
       const bool need = M > mref_c + tcm::kRescaleLog2 || (mref_c == -INFINITY && M != -INFINITY);
       if (__any_sync(kFull, need)) {  // the same decision in the warpgroup's four warps
@@ -668,6 +681,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           tmem_st<NC>(oaddr, ov);
           tc_wait_st();
         }
+      }
       }
       // ---- probabilities, bf16 pairs (column 2q in the low half)
       uint32_t pk[NC / 2];
