@@ -33,7 +33,15 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # DRAM traffic per pa_decode launch measured by ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum summed over the launch's kernels), keyed by workload, with
 # the hash of the kernel sources it was measured on. A different hash -> null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call, from
+    # one ncu capture per workload (summaries with the commands in profiles/); valid only for
+    # the kernel sources they were taken on
+    "llama8b": {"source_hash": "80bd461eae1d3fb0", "bytes_per_launch": 658_270_000},
+    "llama70b_long": {"source_hash": "80bd461eae1d3fb0", "bytes_per_launch": 1_354_850_000},
+    "spec_verify": {"source_hash": "80bd461eae1d3fb0", "bytes_per_launch": 416_750_000},
+    "prefix_sharing": {"source_hash": "80bd461eae1d3fb0", "bytes_per_launch": 214_020_000},
+}
 
 
 # ------------------------------------------------------------------ accounting
