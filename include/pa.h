@@ -79,12 +79,17 @@ typedef enum {
 
 /* Decode kernels. */
 typedef enum {
-  PA_PATH_AUTO = 0,   /* heuristic (pa_decode_plan) */
+  PA_PATH_AUTO = 0,   /* heuristic (pa_decode_plan): tcgen05 for head_dim 128 with more
+                         than 16 rows (GQA group x q_per_seq) per kv head or with prefix
+                         sharing, else the mma.sync tiles (the CUDA-core kernel for <= 2
+                         rows) */
   PA_PATH_SINGLE = 1, /* CUDA-core kernel: warp-shuffle reductions, fp32 FMA */
   PA_PATH_TILE = 2,   /* tensor-core kernel: mma.sync m16n8k16 bf16 -> fp32 */
-  PA_PATH_TCGEN05 = 3 /* 5th-generation tensor cores: tcgen05.mma with accumulators in
-                         tensor memory, one TMA warp, one MMA-issuing thread, one
-                         softmax warp (32 query rows per CTA); grid schedule only */
+  PA_PATH_TCGEN05 = 3 /* 5th-generation tensor cores, head_dim 128 only: tcgen05.mma with
+                         the 128 tokens of a tile on M and 16 or 32 query rows on N,
+                         accumulators in tensor memory, TMA producer warps, one issuing
+                         thread, two softmax warpgroups; always its own persistent
+                         schedule (PA_SCHEDULE_PERSISTENT, no pre-pass, no split length) */
 } pa_path_t;
 
 /* How the work is spread over CTAs. */
@@ -92,33 +97,39 @@ typedef enum {
   PA_SCHEDULE_AUTO = 0,
   PA_SCHEDULE_GRID = 1,       /* one CTA per (kv head, sequence, context split of
                                  split_blocks blocks) + a log-sum-exp merge kernel */
-  PA_SCHEDULE_PERSISTENT = 2  /* a one-CTA pre-pass reads context_lens and cuts all
-                                 (sequence, kv head, block) work into num_ctas equal
-                                 shares; one resident CTA per share; pieces of an
-                                 output are merged by the CTA that finishes it */
+  PA_SCHEDULE_PERSISTENT = 2  /* mma.sync / CUDA-core paths: a one-CTA pre-pass reads
+                                 context_lens and cuts all (sequence, kv head, block)
+                                 work into num_ctas equal shares; one resident CTA per
+                                 share; pieces of an output are merged by the CTA that
+                                 finishes it. tcgen05 path: num_ctas CTAs cut the
+                                 8-block tiles into equal ranges themselves; range-cut
+                                 units are merged by a second kernel */
 } pa_schedule_t;
 
 /* Optional hints for pa_decode_plan; zero-initialised = all automatic. */
 typedef struct {
   int32_t path;          /* pa_path_t */
   int32_t schedule;      /* pa_schedule_t */
-  int32_t split_blocks;  /* grid schedule: blocks per split (0 = heuristic) */
+  int32_t split_blocks;  /* grid schedule: blocks per split (0 = heuristic); a nonzero
+                            value makes the automatic path a grid one */
   int32_t share_prefix;  /* 1 = adjacent sequences whose block tables start with the
                             same physical blocks (parallel sampling, beam search, a
                             common system prompt) are detected on the device and their
                             common prefix blocks are read once for all of them (up to
-                            32 / (GQA group x q_per_seq) sequences per read, tensor-core
-                            kernel); 0 = off */
+                            32 / (GQA group x q_per_seq) sequences per read; tensor-core
+                            kernels only); 0 = off */
 } pa_plan_hints_t;
 
 /* A decode plan; fill it with pa_decode_plan and treat it as opaque. */
 typedef struct {
-  int32_t path;          /* PA_PATH_SINGLE or PA_PATH_TILE */
+  int32_t path;          /* PA_PATH_SINGLE, PA_PATH_TILE or PA_PATH_TCGEN05 */
   int32_t schedule;      /* PA_SCHEDULE_GRID or PA_SCHEDULE_PERSISTENT */
   int32_t split_blocks;  /* grid: blocks per split */
   int32_t num_splits;    /* grid: ceil(max_blocks_per_seq / split_blocks) */
-  int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds */
-  int32_t num_ctas;      /* persistent: CTAs launched (resident slots of the device) */
+  int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds; tcgen05:
+                            the MMA's N (16 or 32) */
+  int32_t num_ctas;      /* persistent: CTAs launched (resident slots of the device); a
+                            caller may lower or raise it (the workspace size follows) */
   int32_t share_cap;     /* sequences per shared-prefix unit, 0 = off */
   int32_t share_split_blocks; /* grid with sharing: blocks per split of a shared prefix */
 } pa_plan_t;
@@ -149,7 +160,9 @@ PA_API pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t n
 /* Workspace bytes pa_decode needs for `plan` (NULL = the heuristic plan for these
  * shapes). Grid schedule: split partials, 0 when there is one split. Persistent
  * schedule: the pre-pass tables, per-output counters and record lists, and a pool of
- * fp32 partial records (a few MB for the shapes above). */
+ * fp32 partial records (a few MB for the shapes above). tcgen05: two fp32 records of
+ * rows_per_cta rows per CTA, a descriptor per CTA and, with sharing, one prefix
+ * length per window (about 5 MB for 148 CTAs). */
 PA_API size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs,
                                 int32_t q_per_seq, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim,
@@ -161,7 +174,9 @@ PA_API size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs,
  * violation) yields 0. plan NULL = heuristic. workspace: 16-byte aligned device
  * buffer of at least pa_decode_workspace_size(plan, ...) bytes, may be NULL when
  * that size is 0; its contents need no initialisation and are scratch afterwards
- * (the persistent schedule's pre-pass resets its counters on every call).
+ * (the persistent schedule's pre-pass resets its counters on every call; every
+ * tcgen05 CTA rewrites its descriptor on every call). Pool slots outside every
+ * sequence's context may hold any bits, NaN included: they never reach the output.
  * Reads query/block_tables/context_lens/caches only after the preceding work on
  * the stream has completed (programmatic dependent launch is used to hide the
  * launch latency). num_seqs == 0 is a no-op. */
