@@ -64,8 +64,35 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // The pool [num_blocks][16][H_kv][D] as a 3-D tensor {D, H_kv, num_blocks*16}; one
 // box is {64, 1, 16}: half of head_dim for one kv head over the 16 tokens of a block,
 // 128-byte swizzled in shared memory.
+bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
+                              int32_t head_dim);
+
+// The maps of the last few pools this thread used: encoding costs microseconds of host
+// time on every call otherwise, and a decode loop passes the same two pools each step.
 bool encode_pool_map(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
                      int32_t head_dim) {
+  struct Entry {
+    const void* base;
+    int64_t num_blocks;
+    int32_t num_kv_heads, head_dim;
+    CUtensorMap map;
+  };
+  thread_local Entry cache[4] = {};
+  thread_local int next = 0;
+  for (const Entry& e : cache)
+    if (e.base == base && e.base != nullptr && e.num_blocks == num_blocks && e.num_kv_heads == num_kv_heads &&
+        e.head_dim == head_dim) {
+      *map = e.map;
+      return true;
+    }
+  if (!encode_pool_map_uncached(map, base, num_blocks, num_kv_heads, head_dim)) return false;
+  cache[next] = Entry{base, num_blocks, num_kv_heads, head_dim, *map};
+  next = (next + 1) & 3;
+  return true;
+}
+
+bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
+                              int32_t head_dim) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),

@@ -34,6 +34,7 @@
 
 #include <cfloat>
 #include <climits>
+#include <mutex>
 #include <cstdint>
 
 #include "pa_device.cuh"
@@ -1523,12 +1524,33 @@ cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int hea
 }
 
 int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta) {
+  // the occupancy query costs microseconds of host time: remember it per device and kernel
+  struct Entry {
+    int dev, path, schedule, head_dim, rows, occ;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (cache[i].dev == dev && cache[i].path == path && cache[i].schedule == schedule &&
+          cache[i].head_dim == head_dim && cache[i].rows == rows_per_cta)
+        return cache[i].occ;
+  }
   DecodeParams dummy = {};
   CUtensorMap tm = {};
   int occ = 0;
   cudaError_t e = head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ)
                                   : dispatch<64>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ);
-  return e == cudaSuccess && occ > 0 ? occ : 1;
+  const int result = e == cudaSuccess && occ > 0 ? occ : 1;
+  if (e == cudaSuccess && occ > 0 && dev >= 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64) cache[used++] = Entry{dev, path, schedule, head_dim, rows_per_cta, occ};
+  }
+  return result;
 }
 
 cudaError_t launch_cache_write(const uint16_t* key, const uint16_t* value, int64_t key_stride,

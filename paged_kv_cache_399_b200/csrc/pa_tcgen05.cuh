@@ -420,6 +420,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       int js = -1;           // unit counter of the S issued last
       int gs = 0, gp = 0;    // next tile to issue S for / PV for (gp <= gs <= gp + 3)
       int ring = 0;          // per tile in flight: bit 2(g&3) O buffer, bit 2(g&3)+1 first of unit
+      int zring = 0;         // per tile in flight, byte g&3: V rows to clear (bit 0 on, block, row)
       bool ok = true;
       unsigned long long idle_since = 0;
       unsigned idle_polls = 0;
@@ -430,6 +431,23 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           pv_ready = gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
                      mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1);
         if (__shfl_sync(kFull, pv_ready, 0)) {
+          const int z = (zring >> (8 * (gp & 3))) & 0xFF;
+          if (z & 1) {
+            // A member's last block is partly filled: its slots past the context may hold any
+            // bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows are
+            // cleared before the PV reads them.
+            mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1);  // every lane sees the data
+            const int jj = (z >> 1) & 7, r0 = z >> 4, nrow = kBlockSize - r0;
+            uint8_t* vblk = smem + L::offV + (gp % kVStages) * tcm::kStageBytes + jj * kHalfTileBytes;
+            for (int idx = lane; idx < 2 * nrow * 8; idx += 32) {
+              const int hf = idx / (nrow * 8);
+              const int rem = idx - hf * (nrow * 8);
+              *reinterpret_cast<uint4*>(vblk + hf * tcm::kHalfBytes + (r0 + (rem >> 3)) * 128 + (rem & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
           if (lane == 0) {
             const int sh = 2 * (gp & 3);
             const int obuf = (ring >> sh) & 1;
@@ -480,6 +498,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
             __syncwarp();
             const int sh = 2 * (gs & 3);
             ring = (ring & ~(3 << sh)) | (obuf << sh) | ((first ? 1 : 0) << (sh + 1));
+            int z = 0;
+            if (w.j >= 0 && w.y == w.seg - 1 && (w.ctx & (kBlockSize - 1)))
+              z = 1 | (((w.nblk - 1) - w.bstart()) << 1) | ((w.ctx & (kBlockSize - 1)) << 4);
+            zring = (zring & ~(0xFF << (8 * (gs & 3)))) | (z << (8 * (gs & 3)));
             w.next(p, upb, nwin);
             ++gs;
             progressed = true;
@@ -695,23 +717,6 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       }
       // the P^T buffer of this tile was read by the PV of tile g-2
       if (g >= 2) wait(&bars.pv_done[g & 1], ((g >> 1) - 1) & 1);
-      if (wg == 0 && w.j >= 0 && w.y == w.seg - 1 && (w.ctx & (kBlockSize - 1))) {
-        // The sequence's last block is partly filled: its slots past the context may hold
-        // any bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows
-        // are cleared before the PV reads them.
-        const int s = g % kVStages;
-        wait(&bars.v_full[s], (g / kVStages) & 1);
-        const int jj = (w.nblk - 1) - w.bstart();
-        const int r0 = w.ctx & (kBlockSize - 1);
-        const int nrow = kBlockSize - r0;
-        uint8_t* vblk = smem + L::offV + s * tcm::kStageBytes + jj * kHalfTileBytes;
-        for (int idx = t; idx < 2 * nrow * 8; idx += 128) {
-          const int hf = idx / (nrow * 8);
-          const int rem = idx - hf * (nrow * 8);
-          *reinterpret_cast<uint4*>(vblk + hf * tcm::kHalfBytes + (r0 + (rem >> 3)) * 128 + (rem & 7) * 16) =
-              make_uint4(0, 0, 0, 0);
-        }
-      }
       uint8_t* pb = smem + L::offP + (g & 1) * L::kP + (cb / 8) * tcm::kPGroupBytes;
 #pragma unroll
       for (int q8 = 0; q8 < NC / 8; ++q8)
