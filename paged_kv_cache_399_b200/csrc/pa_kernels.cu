@@ -84,12 +84,10 @@ __device__ __forceinline__ int num_blocks_of(const DecodeParams& p, int ctx) {
 struct Seg {
   int b0, members, kvh, row0, nrows, blk0, blk1;
   bool shared;
-  int roff;  // local row r of this view is row r + roff of the segment (row-split CTAs)
 };
 
 __device__ __forceinline__ bool seg_row(const DecodeParams& p, const Seg& s, int r, int& b, int& i,
                                         int& h) {
-  r += s.roff;
   if (r >= s.nrows) return false;
   int m = 0, rr = s.row0 + r;
   if (s.shared) {
