@@ -232,8 +232,18 @@ PA_API pa_status_t pa_validate(const int32_t* block_tables, const int32_t* conte
 
 /* Reads (and with reset != 0 clears) the device error word that kernels set when a
  * bounded wait times out (synchronous: waits for `stream`). *code = 0 means no
- * error; the status is PA_ERR_DEVICE when *code != 0. */
+ * error; the status is PA_ERR_DEVICE when *code != 0. The first code set since the
+ * last reset is kept:
+ *   0x100 a decode wait timed out, 0x200 draining in-flight copies timed out,
+ *   0x300 / 0x400 the persistent schedule's record pool / list is full,
+ *   0x500 an inconsistent schedule or shared-memory layout, 0x600 the self-test. */
 PA_API pa_status_t pa_get_device_error(uint32_t* code, int32_t reset, pa_stream_t stream);
+
+/* Self-test of the failure path (no counterpart on the pages): enqueues one CTA that
+ * waits on an mbarrier nothing completes; after the bounded-wait limit (about 1 s)
+ * it records 0x600 in the device error word and returns, leaving the context usable.
+ * Asynchronous; read the result with pa_get_device_error. */
+PA_API pa_status_t pa_selftest_bounded_wait(pa_stream_t stream);
 
 /* Static description of a status code. */
 PA_API const char* pa_status_string(pa_status_t status);

@@ -539,6 +539,10 @@ pa_status_t pa_validate(const int32_t* block_tables, const int32_t* context_lens
   return bad ? PA_ERR_OUT_OF_RANGE : PA_OK;
 }
 
+pa_status_t pa_selftest_bounded_wait(pa_stream_t stream) {
+  return pa::run_selftest_wait(reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 pa_status_t pa_get_device_error(uint32_t* code, int32_t reset, pa_stream_t stream) {
   if (!code) return PA_ERR_INVALID_ARG;
   cudaError_t e = pa::read_device_error(code, reset != 0, reinterpret_cast<cudaStream_t>(stream));

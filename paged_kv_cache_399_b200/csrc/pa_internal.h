@@ -94,4 +94,7 @@ cudaError_t run_validate(const int32_t* block_tables, const int32_t* context_len
 
 cudaError_t read_device_error(uint32_t* code, bool reset, cudaStream_t stream);
 
+// Launch the bounded-wait self-test kernel (about one wait limit long).
+cudaError_t run_selftest_wait(cudaStream_t stream);
+
 }  // namespace pa

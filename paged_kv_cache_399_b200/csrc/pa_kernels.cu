@@ -49,6 +49,7 @@ __device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_devic
 constexpr unsigned kErrRecordPool = 0x300u;
 constexpr unsigned kErrRecordList = 0x400u;
 constexpr unsigned kErrSchedule = 0x500u;
+constexpr unsigned kErrSelftest = 0x600u;
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kHalfTileBytes = 16 * 64 * 2;  // 16 tokens x 64 bf16
@@ -1587,6 +1588,22 @@ cudaError_t run_validate(const int32_t* block_tables, const int32_t* context_len
   if (e != cudaSuccess) return e;
   *bad = static_cast<int64_t>(count);
   return cudaSuccess;
+}
+
+// Self-test of the failure path: one thread waits on an mbarrier that nothing
+// completes; the bounded wait gives up after its limit and the kernel records
+// kErrSelftest and returns.
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (!mbar_wait_bounded(&bar, 0)) record_error(kErrSelftest);
+}
+
+cudaError_t run_selftest_wait(cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>();
+  return cudaGetLastError();
 }
 
 cudaError_t read_device_error(uint32_t* code, bool reset, cudaStream_t stream) {

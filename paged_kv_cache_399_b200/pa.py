@@ -33,8 +33,8 @@ PA_PATH_TILE = 2
 PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
-            "pa_decode_static_scratch", "pa_validate", "pa_get_device_error", "pa_status_string",
-            "pa_version"]
+            "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
+            "pa_selftest_bounded_wait", "pa_status_string", "pa_version"]
 
 PA_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -87,6 +87,8 @@ _lib.pa_validate.restype = _I32
 _lib.pa_validate.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I64, _I64, _I32, ctypes.POINTER(_I64), _P]
 _lib.pa_get_device_error.restype = _I32
 _lib.pa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), _I32, _P]
+_lib.pa_selftest_bounded_wait.argtypes = [_P]
+_lib.pa_selftest_bounded_wait.restype = _I32
 _lib.pa_status_string.restype = ctypes.c_char_p
 _lib.pa_status_string.argtypes = [_I32]
 _lib.pa_version.restype = _I32
@@ -225,6 +227,12 @@ def pa_validate(block_tables: torch.Tensor, context_lens: torch.Tensor,
     if st not in (PA_OK, PA_ERR_OUT_OF_RANGE):
         _check(st, "pa_validate")
     return int(bad.value)
+
+
+def pa_selftest_bounded_wait(stream=None) -> None:
+    """Enqueue the failure-path self-test: about one wait limit later the device error
+    word holds 0x600 (read it with pa_get_device_error)."""
+    _check(_lib.pa_selftest_bounded_wait(_stream(stream)), "pa_selftest_bounded_wait")
 
 
 def pa_get_device_error(reset: bool = True, stream=None) -> int:

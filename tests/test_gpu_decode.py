@@ -216,3 +216,24 @@ def test_validate_reports_bad_entries():
     bad_slots = dw.slots.clone()
     bad_slots[0] = w.num_blocks * 16
     assert pa.pa_validate(bad_tables, bad_ctx, bad_slots, w.q_per_seq, w.num_blocks) == 4
+
+
+@pytest.mark.parametrize("plan_spec", PLANS, ids=[p[0] for p in PLANS])
+def test_empty_sequences_give_zero_rows(plan_spec, oracle_lib):
+    """Sequences with context length 0 (nothing to attend to, no slot written) between
+    ordinary ones: their rows are 0, the others match the oracle."""
+    w = _workload(("with_empty", [5, 37, 9, 300, 12], 1, 8, 2, 128, None, []), 2990)
+    empty = [0, 2, 4]
+    w.context_lens = w.context_lens.copy()
+    w.slot_mapping = w.slot_mapping.copy()
+    for b in empty:
+        w.context_lens[b] = 0
+        w.slot_mapping[b * w.q_per_seq:(b + 1) * w.q_per_seq] = -1
+    kc, vc = oracle_pools(oracle_lib, w)
+    ref = oracle_lib.decode(w.query, kc, vc, w.block_tables, w.context_lens, w.q_per_seq, w.scale)
+    assert all(float(np.abs(ref[b]).max()) == 0.0 for b in empty)
+    plan = _plan(w, plan_spec)
+    out = run_step(DeviceWorkload(w), plan)
+    assert_close(out, ref, f"with_empty/{plan_spec[0]}")
+    for b in empty:
+        assert float(out[b].float().abs().max()) == 0.0
