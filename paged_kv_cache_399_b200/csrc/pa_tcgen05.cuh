@@ -336,8 +336,8 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
 
   if (warp == tcm::kProducerWarp || warp == tcm::kVProducerWarp) {
     // ------------------------------------------------------------ TMA producers
-    // Lanes 0..15 issue a tile's 16 boxes (half = lane / 8, block = lane % 8) of K (warp 4)
-    // or V (warp 6); lanes 0..7 load the next tile's block ids while this one is issued.
+    // Lanes 0..15 issue a tile's 16 boxes (half = lane / 8, block = lane % 8) of K (warp 8)
+    // or V (warp 10); lanes 0..7 load the next tile's block ids while this one is issued.
     const bool is_k = warp == tcm::kProducerWarp;
     const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
     uint64_t* full = is_k ? bars.k_full : bars.v_full;
