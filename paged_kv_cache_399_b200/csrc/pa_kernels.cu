@@ -11,8 +11,14 @@
 //   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split)
 //   merge_kernel             log-sum-exp merge of the grid schedule's split partials
 //   validate_kernel          debug bounds check of slots / block ids / context lengths
+//   selftest_wait_kernel     the bounded-wait failure path, taken without a fault
+// and, from pa_tcgen05.cuh, the 5th-generation tensor-core path:
+//   decode_tcm_kernel        tokens on M, tcgen05.mma with TMEM accumulators, persistent
+//                            equal-tile schedule over windows of sequences
+//   tcm_merge_kernel         merge of the units a tile range boundary cuts
+//   tcm_share_prepass        common table prefix of each window (prefix sharing)
 //
-// Two compute cores run inside the decode kernels:
+// Two compute cores run inside the mma.sync / CUDA-core decode kernels:
 //   TileCore   tensor cores: mma.sync m16n8k16 bf16 -> fp32 on S^T = K Q^T and
 //              O^T += V^T P^T, online softmax on the accumulator fragments;
 //   SimtCore   CUDA cores: fp32 FMA dot products, warp-shuffle max / sum.
