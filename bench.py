@@ -37,10 +37,10 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call, from
     # one ncu capture per workload (summaries with the commands in profiles/); valid only for
     # the kernel sources they were taken on
-    "llama8b": {"source_hash": "7cfd10f25d69a7af", "bytes_per_launch": 656_910_000},
-    "llama70b_long": {"source_hash": "7cfd10f25d69a7af", "bytes_per_launch": 1_354_790_000},
-    "spec_verify": {"source_hash": "7cfd10f25d69a7af", "bytes_per_launch": 417_110_000},
-    "prefix_sharing": {"source_hash": "7cfd10f25d69a7af", "bytes_per_launch": 215_310_000},
+    "llama8b": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 658_770_000},
+    "llama70b_long": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 1_354_610_000},
+    "spec_verify": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 416_740_000},
+    "prefix_sharing": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 213_430_000},
 }
 
 
