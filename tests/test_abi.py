@@ -25,7 +25,7 @@ def pa():
     return mod
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_hot_path_calls():
     syms = declared_symbols()
     for name in ["pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size", "pa_decode_plan",
                  "pa_validate", "pa_get_device_error", "pa_status_string", "pa_version"]:
