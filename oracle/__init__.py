@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the paged KV-cache hot path (cache write + paged decode).
+"""fp64 CPU oracle for the paged KV-cache hot path (cache write + paged decode) and the
+copy-on-write block copy.
 
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it. The
@@ -62,6 +63,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode_rows.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                        _I32, _I32, _I32, _I64, ctypes.c_double, _P, _I64,
                                        _I32]
+    lib.oracle_copy_blocks.restype = _I32
+    lib.oracle_copy_blocks.argtypes = [_P, _P, _I64, _I64, _P, _I64]
     lib.oracle_threads_used.restype = _I32
     lib.oracle_mutant_id.restype = _I32
     return lib
@@ -163,6 +166,19 @@ class Oracle:
         if st != 0:
             raise ValueError(f"oracle_decode_rows status {st}")
         return out
+
+    def copy_blocks(self, key_cache, value_cache, block_mapping):
+        """Copy-on-write block copy. block_mapping is [n][2] {source, destination}.
+        Returns new (key_cache, value_cache) uint16 arrays; inputs untouched."""
+        kc = _u16(key_cache).copy()
+        vc = _u16(value_cache).copy()
+        m = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
+        NB = kc.shape[0]
+        block_elems = int(np.prod(kc.shape[1:]))
+        st = self.lib.oracle_copy_blocks(_ptr(kc), _ptr(vc), NB, block_elems, _ptr(m), m.shape[0])
+        if st != 0:
+            raise ValueError(f"oracle_copy_blocks status {st}")
+        return kc, vc
 
     def threads_used(self) -> int:
         return self.lib.oracle_threads_used()

@@ -1,5 +1,6 @@
 // PagedAttention oracle: plain, slow, fp64 CPU restatement of what the paged
-// KV-cache hot path computes.
+// KV-cache hot path computes (cache write, paged decode), and of the copy-on-write
+// block copy.
 //
 // TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU-baseline
 // leg of the benchmark may load this library. The CUDA library never includes,
@@ -11,9 +12,11 @@
 //        (chenxutan.com/d/2880), §3.2 KV Cache Block, §3.3 PagedAttention 的实现细节
 //   [VS] vLLM study notes (zihan-zhang.net/vLLM-study), §1.1.1 (attention with a
 //        causal mask), §1.2.1-1.2.2 (KV cache, size formula), §3.2 (block table,
-//        page-wise read of K/V), §4.3.1 (online softmax)
+//        page-wise read of K/V), §3.2.2 (sharing and copy-on-write), §4.3.1 (online
+//        softmax)
 //   [DP] "vLLM 深度解析：连续批处理与内存高效推理" (plumephp.com/ai-vllm-system),
-//        §1.2 (KV size formula), §2.1 (block table), §4.1 (block count example)
+//        §1.2 (KV size formula), §2.1 (block table, copy on write), §4.1 (block count
+//        example), §4.2 (reference counts and sharing)
 //
 // Readings taken where the pages are silent or disagree (all stated here so the
 // code can be checked against them by eye):
@@ -342,6 +345,50 @@ int oracle_decode_rows(double* out, const uint16_t* query, const uint16_t* key_c
           max_blocks_per_seq, num_blocks};
   return decode_rows_impl(out, query, key_cache, value_cache, block_tables, context_lens,
                           s, scale, rows, n_rows, num_threads);
+}
+
+// Copy-on-write block copy ([VS] §3.2.2 写时复制: a sequence about to write into a block
+// that other sequences still reference first gets a private copy of it; [DP] §2.1 and
+// §4.2: the same at the forks of parallel sampling and beam search). Each pair p of
+// `mapping` ([num_pairs][2] = {source block, destination block}) copies every element of
+// the source block (block_elems = block_size x num_kv_heads x head_dim values, in the key
+// pool and in the value pool) onto the destination block; every other block is left as it
+// was. A pair with a negative entry is padding and is skipped. Returns 0; 1 if an id is
+// past the pool, 2 if a destination repeats or is also a source (the result would then
+// depend on the order of the copies); nothing is copied in either error case.
+int oracle_copy_blocks(uint16_t* key_cache, uint16_t* value_cache, int64_t num_blocks,
+                       int64_t block_elems, const int64_t* mapping, int64_t num_pairs) {
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    const int64_t src = mapping[2 * p], dst = mapping[2 * p + 1];
+    if (src < 0 || dst < 0) continue;
+    if (src >= num_blocks || dst >= num_blocks) return 1;
+    for (int64_t o = 0; o < num_pairs; ++o) {
+      const int64_t os = mapping[2 * o], od = mapping[2 * o + 1];
+      if (os < 0 || od < 0) continue;
+      if (od == dst && o != p) return 2;
+      if (os == dst) return 2;
+    }
+  }
+  for (int64_t p = 0; p < num_pairs; ++p) {
+#if ORACLE_MUTANT == 33
+    const int64_t src = mapping[2 * p + 1], dst = mapping[2 * p];  // planted: pair reversed
+#else
+    const int64_t src = mapping[2 * p], dst = mapping[2 * p + 1];
+#endif
+    if (src < 0 || dst < 0) continue;
+#if ORACLE_MUTANT == 32
+    const int64_t n = block_elems - block_elems / 16;  // planted: the last token left behind
+#else
+    const int64_t n = block_elems;
+#endif
+    for (int64_t e = 0; e < n; ++e) {
+      key_cache[dst * block_elems + e] = key_cache[src * block_elems + e];
+#if ORACLE_MUTANT != 31  // planted (31): the value pool is not copied
+      value_cache[dst * block_elems + e] = value_cache[src * block_elems + e];
+#endif
+    }
+  }
+  return 0;
 }
 
 // Threads the last decode call ran on.

@@ -7,7 +7,9 @@ when the oracle disagrees with:
   * a library routine (torch scaled_dot_product_attention, fp64, CPU),
   * closed forms (one-token context, identical keys, zero scale),
   * invariants (block permutation, shared prefixes, GQA vs MHA, speculative
-    rows vs shorter single-token calls, tiled online softmax and split/merge).
+    rows vs shorter single-token calls, tiled online softmax and split/merge),
+  * the copy-on-write rule of parallel sampling (a fork's writer copies the shared
+    last block and writes there; the other candidates still read the original).
 The same checks run against deliberately broken builds of the oracle
 (tests/test_oracle_mutants.py) to show that each planted mistake is caught.
 """
@@ -379,6 +381,83 @@ def check_cache_write(oracle):
         raise AssertionError("out-of-range slot not reported")
 
 
+def _attend_rows(q, K, V, scale):
+    """Textbook attention of one query token's heads over contiguous K/V [t][hkv][d]."""
+    hq, hkv = q.shape[0], K.shape[1]
+    out = np.zeros((hq, q.shape[1]))
+    for h in range(hq):
+        kv = h // (hq // hkv)
+        s = scale * (K[:, kv] @ q[h])
+        w = np.exp(s - s.max())
+        out[h] = (w[:, None] * V[:, kv]).sum(0) / w.sum()
+    return out
+
+
+def check_copy_on_write(oracle):
+    """The parallel-sampling fork of the copy-on-write rule (golden/copy_on_write.json):
+    the candidates share every prompt block; a candidate about to write into the shared
+    last block gets a copy first, writes there, and the others still read the original."""
+    g = json.load(open(os.path.join(GOLDEN, "copy_on_write.json")))
+    bs, n, L, writers = g["block_size"], g["parallel_samples"], g["prompt_tokens"], g["writers"]
+    rng = np.random.default_rng(91)
+    hq, hkv, d, nb = 4, 2, 8, 12
+    pk = _bf16_round(rng.standard_normal((nb, bs, hkv, d)))
+    pv = _bf16_round(rng.standard_normal((nb, bs, hkv, d)))
+    prompt = [5, 2, 9]                                      # physical blocks of the prompt
+    K = _bf16_round(rng.standard_normal((L, hkv, d)))
+    V = _bf16_round(rng.standard_normal((L, hkv, d)))
+    for t in range(L):
+        pk[prompt[t // bs], t % bs] = K[t]
+        pv[prompt[t // bs], t % bs] = V[t]
+    tables = np.array([prompt] * n, dtype=np.int32)
+    free = [b for b in range(nb) if b not in prompt]
+    # the rule: a write into a block referenced by more than one table copies it first
+    mapping = []
+    for w in writers:
+        blk = tables[w, L // bs]
+        refs = int((tables[:, L // bs] == blk).sum())
+        assert refs > g["copy_when_ref_count_above"]
+        dst = free.pop(0)
+        mapping.append([blk, dst])
+        tables[w, L // bs] = dst
+    for w in writers:   # after the copies every block a writer writes has one reference
+        assert int((tables == tables[w, L // bs]).sum()) == 1
+    kc, vc = oracle.copy_blocks(_bits(pk), _bits(pv), mapping + [[-1, 0]])
+    newk = _bf16_round(rng.standard_normal((len(writers), hkv, d)))
+    newv = _bf16_round(rng.standard_normal((len(writers), hkv, d)))
+    slots = np.array([tables[w, L // bs] * bs + L % bs for w in writers], dtype=np.int64)
+    kc, vc = oracle.reshape_and_cache(_bits(newk), _bits(newv), kc, vc, slots)
+    # every candidate attends over its own logical sequence, built here without the pool
+    Q = _bf16_round(rng.standard_normal((n, 1, hq, d)))
+    ctxs = np.array([L + 1 if b in writers else L for b in range(n)], dtype=np.int32)
+    out = oracle.decode(_bits(Q), kc, vc, tables, ctxs, 1, 1.0 / math.sqrt(d))
+    for b in range(n):
+        Kb, Vb = K, V
+        if b in writers:
+            Kb = np.concatenate([K, newk[writers.index(b)][None]])
+            Vb = np.concatenate([V, newv[writers.index(b)][None]])
+        _close(out[b, 0], _attend_rows(Q[b, 0], Kb, Vb, 1.0 / math.sqrt(d)), what=f"candidate {b}")
+    # bit level: the source block is untouched, each copy equals it except the written
+    # token, and no other block changed
+    k0, v0 = _bits(pk), _bits(pv)
+    for j, (src, dst) in enumerate(mapping):
+        for pool, pool0, new in ((kc, k0, newk), (vc, v0, newv)):
+            assert np.array_equal(pool[src], pool0[src]), "source block changed"
+            exp = pool0[src].copy()
+            exp[L % bs] = _bits(new[j])
+            assert np.array_equal(pool[dst], exp), f"copy {j} differs from its source"
+    others = [b for b in range(nb) if b not in [m[1] for m in mapping]]
+    assert np.array_equal(kc[others], k0[others]) and np.array_equal(vc[others], v0[others]), "stray write"
+    kc2, vc2 = oracle.copy_blocks(k0, v0, np.zeros((0, 2), dtype=np.int64))
+    assert np.array_equal(kc2, k0) and np.array_equal(vc2, v0), "empty mapping changed the pools"
+    for bad in ([[1, 3], [2, 3]], [[1, 3], [3, 4]], [[0, nb]]):
+        try:
+            oracle.copy_blocks(k0, v0, bad)
+        except ValueError:
+            continue
+        raise AssertionError(f"mapping {bad} not rejected")
+
+
 ALL_CHECKS = [
     check_bf16_widening,
     check_block_counts_golden,
@@ -394,4 +473,5 @@ ALL_CHECKS = [
     check_spec_rows_equal_short_calls,
     check_online_and_split_merge,
     check_cache_write,
+    check_copy_on_write,
 ]
