@@ -42,6 +42,12 @@ NCU_TRAFFIC = {
     "spec_verify": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 416_740_000},
     "prefix_sharing": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 213_430_000},
 }
+# the same for one pa_copy_blocks launch of a copy workload (keyed by COPY_SOURCES' hash;
+# mean of three 2048-pair launches: the writes still in L2 when a launch ends are not
+# counted, so the traffic sits below the algorithmic bytes)
+NCU_COPY_TRAFFIC = {
+    "cow_bulk": {"source_hash": "d46ea268e31f8d30", "bytes_per_launch": 211_644_000},
+}
 
 
 # ------------------------------------------------------------------ accounting
@@ -95,10 +101,17 @@ def decode_flops(w) -> int:
     return 4 * w.head_dim * (w.num_q_heads // w.num_kv_heads) * w.num_kv_heads * vis
 
 
-def source_hash() -> str:
+# the sources each kernel family is compiled from (the decode kernels share nothing with
+# the block copy, so a change to one leaves the other's measured traffic valid)
+DECODE_SOURCES = ("pa_api.cpp", "pa_device.cuh", "pa_internal.h", "pa_kernels.cu",
+                  "pa_static_scratch.cu", "pa_tcgen05.cuh")
+COPY_SOURCES = ("pa_copy.cu",)
+
+
+def source_hash(names=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_399_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -118,7 +131,7 @@ def measured_peaks():
 # ------------------------------------------------------------------ ranks
 
 BASE_SEEDS = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
-              "spec_verify": 1004}
+              "spec_verify": 1004, "cow_fork": 1005, "cow_bulk": 1006}
 
 
 def rank_seed(workload: str, rank: int) -> int:
@@ -507,6 +520,228 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ block copy
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def copy_bytes(w) -> int:
+    """Algorithmic bytes of one pa_copy_blocks call: each copied block is read once and
+    written once, in the key pool and in the value pool."""
+    return 2 * 2 * w.block_bytes * w.num_pairs
+
+
+def run_copy_gpu(args):
+    """One step = one pa_copy_blocks call over the workload's pairs (the copies a fork
+    needs before the step's cache write)."""
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from paged_kv_cache_399_b200 import build as pa_build
+    pa_build.build()
+    from paged_kv_cache_399_b200 import pa, workloads
+
+    w = workloads.make_copy(args.workload, seed=rank_seed(args.workload, rank))
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    kc = w.key_cache.to(dev)
+    vc = w.value_cache.to(dev)
+    mapping = np.ascontiguousarray(w.mapping)
+    nbytes = copy_bytes(w)
+    launches = -(-w.num_pairs // 2048)
+    # a step that moves less than twice L2 would find its blocks in L2 on the next step:
+    # write a buffer larger than L2 between steps, outside the timed events
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if nbytes < 2 * L2_BYTES else None
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        return reduce_over_ranks(x, "max", dist if world > 1 else None, dev)
+
+    def step():
+        pa.pa_copy_blocks(kc, vc, mapping, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        barrier()
+        if flush is None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
+            barrier()
+            ms_total = e0.elapsed_time(e1)
+        else:
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)]
+            for a, b in pairs:
+                flush.zero_()
+                a.record(stream)
+                step()
+                b.record(stream)
+            barrier()
+            ms_total = sum(a.elapsed_time(b) for a, b in pairs)
+        ms_total = max_over_ranks(ms_total)
+        # end to end through the C ABI: the host mapping enters with the launches (its
+        # checks and marshalling inside the timed region); the copies stay in the pools
+        e2e_steps = max(1, args.steps // 4)
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            step()
+        f1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    clocks = sampler.summary()
+    ms_per_step = ms_total / args.steps
+    value_gbs = aggregate_throughput(nbytes, args.steps, ms_total, world)
+    e2e_gbs = aggregate_throughput(nbytes, e2e_steps, e2e_ms, world)
+    peaks = measured_peaks()
+    # bytes of one launch over one launch's time (the launches of a step split the pairs
+    # evenly, so this is the step's bytes over the step's time)
+    achieved = nbytes / (ms_per_step * 1e-3) / 1e9
+    traffic = None
+    rec = NCU_COPY_TRAFFIC.get(args.workload)
+    if rec and rec.get("source_hash") == source_hash(COPY_SOURCES):
+        traffic = rec["bytes_per_launch"]
+    if rank == 0:
+        cpu = copy_cpu_baseline(w, args) if (world == 1 and not args.no_cpu_baseline) else None
+        line = {
+            "metric": "pa_copy_blocks GB/s (bytes read + written per copy-on-write step)",
+            "value": round(value_gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16 bits (u16 copy)",
+            "data": "synthetic",
+            "config": {
+                "workload": w.describe(),
+                "step": "pa_copy_blocks",
+                "alg_bytes_per_step": nbytes,
+                "launches_per_step": launches,
+                "us_per_call": round(ms_per_step * 1e3, 3),
+                "l2": "flushed between steps (a 252 MB write outside the timed events)" if flush is not None
+                      else "no flush: each step moves more bytes than twice the 126 MB L2",
+                "parallelism": f"replicas x{world} (independent pools per GPU, no collective)",
+            },
+            "roofline": {
+                "bound": "hbm",
+                "achieved": round(achieved, 2),
+                "peak": peaks["hbm_gbs"],
+                "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic,
+                "peak_source": peaks["source"],
+                "kernel": "copy_blocks_kernel (the measured peak is itself a copy: read + write bytes)",
+            },
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(mapping.nbytes), "d2h_bytes_per_step": 0,
+                    "steps": e2e_steps,
+                    "note": "the mapping is a host array carried by the launches; the result stays in the "
+                            "device pools, where the next decode reads it"},
+            "gpu_launches": launches * args.steps,
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_copy_arrays(w, pairs):
+    from oracle import _u16
+    kc = _u16(w.key_cache).copy()
+    vc = _u16(w.value_cache).copy()
+    m = np.ascontiguousarray(w.mapping[:pairs])
+    return kc, vc, m
+
+
+def _time_oracle_copy(orc, kc, vc, m, block_elems, min_s, max_reps=1000, fixed_reps=None):
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        st = orc.lib.oracle_copy_blocks(kc.ctypes.data, vc.ctypes.data, kc.shape[0], block_elems,
+                                        m.ctypes.data, m.shape[0])
+        assert st == 0
+        reps += 1
+        if fixed_reps is not None:
+            if reps >= fixed_reps:
+                break
+        elif time.perf_counter() - t0 >= min_s or reps >= max_reps:
+            break
+    return (time.perf_counter() - t0) / reps, reps
+
+
+def copy_cpu_baseline(w, args, target_s: float = 8.0):
+    """The oracle's copy, as it stands, on one host core over a bounded sample of pairs."""
+    from oracle import Oracle
+    orc = Oracle()
+    pairs = min(w.num_pairs, 1024)
+    kc, vc, m = _oracle_copy_arrays(w, pairs)
+    block_elems = int(np.prod(kc.shape[1:]))
+    dt, reps = _time_oracle_copy(orc, kc, vc, m, block_elems, target_s)
+    sample_bytes = 2 * 2 * w.block_bytes * pairs
+    return {"value": round(sample_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{pairs} of {w.num_pairs} pairs of {w.name} (element-wise copy), {reps} repetitions, "
+                      f"{dt * 1e3:.2f} ms each"}
+
+
+def run_copy_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import Oracle
+    from paged_kv_cache_399_b200 import workloads
+    w = workloads.make_copy(args.workload, seed=rank_seed(args.workload, 0))
+    orc = Oracle()
+    pairs = min(w.num_pairs, 256)
+    kc, vc, m = _oracle_copy_arrays(w, pairs)
+    block_elems = int(np.prod(kc.shape[1:]))
+    _time_oracle_copy(orc, kc, vc, m, block_elems, 0.0, fixed_reps=args.warmup)
+    dt, _ = _time_oracle_copy(orc, kc, vc, m, block_elems, 0.0, fixed_reps=args.steps)
+    sample_bytes = 2 * 2 * w.block_bytes * pairs
+    value = sample_bytes / dt / 1e9
+    sample = f"{pairs} of {w.num_pairs} pairs of {w.name} per step (element-wise copy)"
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "pa_copy_blocks GB/s (bytes read + written per copy-on-write step)",
+        "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u16", "data": "synthetic",
+        "config": {"workload": w.describe(), "step": "oracle block copy"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -514,7 +749,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify"])
+                    choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify",
+                             "cow_fork", "cow_bulk"],
+                    help="decode workloads time cache write + decode; cow_fork / cow_bulk time the "
+                         "copy-on-write block copy")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=["auto", "grid", "persistent"], default="auto")
     ap.add_argument("--path", choices=["auto", "single", "tile", "tcgen05"], default="auto")
@@ -525,10 +763,11 @@ def main(argv=None):
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    copy = args.workload in ("cow_fork", "cow_bulk")
     if args.impl == "reference":
-        run_reference(args)
+        (run_copy_reference if copy else run_reference)(args)
     else:
-        run_gpu(args)
+        (run_copy_gpu if copy else run_gpu)(args)
     return 0
 
 

@@ -1,7 +1,7 @@
 /*
  * pa.h -- C ABI of the B200 (sm_100a) paged KV-cache hot path.
  *
- * Two operations, as the vLLM pages describe them:
+ * The operations, as the vLLM pages describe them:
  *   pa_reshape_and_cache  writes this step's new K/V rows into the paged pool at
  *                         the slots named by slot_mapping
  *                         ("vLLM 深度实战：从 PagedAttention 到 Speculative Decoding",
@@ -11,10 +11,13 @@
  *                         (same page §3.3; vLLM study notes, zihan-zhang.net, §3.2
  *                          page-table walk and §4.3.1 online softmax), with GQA
  *                         head groups and causal masking of multi-token
- *                         (speculative-verify) queries (vLLM study notes §1.1.1).
+ *                         (speculative-verify) queries (vLLM study notes §1.1.1);
+ *   pa_copy_blocks        the copy-on-write block copy behind shared blocks
+ *                         (vLLM study notes §3.2.2).
  *
  * Conventions shared by every call
- *   - All data pointers are DEVICE pointers on the current CUDA device; the library
+ *   - All data pointers are DEVICE pointers on the current CUDA device (the one
+ *     exception: pa_copy_blocks' block_mapping is a host array); the library
  *     never allocates, frees or synchronises (except pa_validate and
  *     pa_get_device_error, which are synchronous debug calls). All work is enqueued
  *     on `stream` (a cudaStream_t; NULL = legacy default stream). The caller owns
@@ -72,7 +75,8 @@ typedef enum {
   PA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or stride */
   PA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported set above */
   PA_ERR_WORKSPACE = 3,     /* split plan without a large enough workspace */
-  PA_ERR_OUT_OF_RANGE = 4,  /* pa_validate found a bad slot / block id / length */
+  PA_ERR_OUT_OF_RANGE = 4,  /* pa_validate found a bad slot / block id / length;
+                               pa_copy_blocks was given a block id past the pool */
   PA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
   PA_ERR_DEVICE = 6         /* pa_get_device_error: a kernel reported a timeout */
 } pa_status_t;
@@ -244,6 +248,27 @@ PA_API pa_status_t pa_get_device_error(uint32_t* code, int32_t reset, pa_stream_
  * it records 0x600 in the device error word and returns, leaving the context usable.
  * Asynchronous; read the result with pa_get_device_error. */
 PA_API pa_status_t pa_selftest_bounded_wait(pa_stream_t stream);
+
+/* Copy-on-write block copy (vLLM study notes, zihan-zhang.net, §3.2.2 写时复制: a
+ * sequence about to write into a block other sequences still reference first gets a copy
+ * of it; "vLLM 深度解析：连续批处理与内存高效推理" §2.1 Copy on Write and §4.2, the forks of
+ * parallel sampling and beam search). For each pair p of block_mapping ([num_pairs][2] =
+ * {source, destination} physical block ids), every element of the source block -- its
+ * block_size tokens x num_kv_heads x head_dim values -- is copied onto the destination
+ * block, in key_cache and in value_cache. Bit-exact; every other block is left untouched.
+ * A pair with a negative entry is padding and is skipped.
+ *   block_mapping is a HOST array (the block manager decides the copies on the host). It
+ *   is read during the call, its entries travel inside the launches (up to 2048 pairs a
+ *   launch), and it may be reused as soon as the call returns.
+ *   Host checks, before anything is enqueued: block_size 16, head_dim 64 or 128
+ *   (else PA_ERR_UNSUPPORTED); num_kv_heads >= 1, num_pairs >= 0 (0 is a no-op), non-null
+ *   16-byte aligned pools (else PA_ERR_INVALID_ARG); every id < num_blocks (else
+ *   PA_ERR_OUT_OF_RANGE); destinations distinct and none of them also a source (else
+ *   PA_ERR_INVALID_ARG: the result would depend on the order of the copies). */
+PA_API pa_status_t pa_copy_blocks(void* key_cache, void* value_cache, int64_t num_blocks,
+                                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  const int64_t* block_mapping, int64_t num_pairs,
+                                  pa_stream_t stream);
 
 /* Static description of a status code. */
 PA_API const char* pa_status_string(pa_status_t status);

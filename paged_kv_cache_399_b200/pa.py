@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa_b200.so")
@@ -34,7 +35,7 @@ PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
-            "pa_selftest_bounded_wait", "pa_status_string", "pa_version"]
+            "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_status_string", "pa_version"]
 
 PA_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -70,6 +71,8 @@ _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
 _I64 = ctypes.c_int64
 
+_lib.pa_copy_blocks.restype = _I32
+_lib.pa_copy_blocks.argtypes = [_P, _P, _I64, _I32, _I32, _I32, _P, _I64, _P]
 _lib.pa_reshape_and_cache.restype = _I32
 _lib.pa_reshape_and_cache.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _I32, _I64, _I32, _P]
 _lib.pa_decode_plan.restype = _I32
@@ -145,6 +148,24 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
                                    _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping), T, H, D,
                                    NB, BS, _stream(stream))
     _check(st, "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, block_mapping,
+                   stream=None) -> None:
+    """Copy-on-write block copy. Caches [NB, 16, H_kv, D] bf16 on the device;
+    block_mapping [n, 2] int64 {source, destination} block ids, a HOST array (CPU tensor
+    or numpy), read during the call."""
+    assert key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert key_cache.is_contiguous() and value_cache.is_contiguous()
+    assert key_cache.shape == value_cache.shape
+    if isinstance(block_mapping, torch.Tensor):
+        assert block_mapping.device.type == "cpu", "block_mapping is a host array"
+        block_mapping = block_mapping.numpy()
+    m = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
+    NB, BS, H, D = key_cache.shape
+    st = _lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), NB, H, D, BS,
+                             m.ctypes.data if m.shape[0] else None, m.shape[0], _stream(stream))
+    _check(st, "pa_copy_blocks")
 
 
 def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,

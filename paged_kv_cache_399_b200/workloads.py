@@ -22,6 +22,15 @@ notes §1.2.2):
 * ``spec_verify``     32 seqs x 6 query tokens (causal inside the window), 32/8 heads,
                       context lognormal(ln 2048, 0.8) clipped to [16, 16384]; the slot
                       mapping writes all 6 new tokens.
+
+Copy-on-write block copies (``make_copy``; the copy rule of the vLLM study notes
+§3.2.2):
+
+* ``cow_fork``        the fork of 16 prompts (U[1, 2048] tokens) into 8 samples each:
+                      7 copies of every partly filled last prompt block, 8 kv heads,
+                      head_dim 128 (32 KB per block and pool).
+* ``cow_bulk``        8192 copies in a 20480-block pool (same block shape), sources
+                      with repeats, distinct destinations.
 """
 
 from __future__ import annotations
@@ -189,6 +198,102 @@ def spec_verify(seed: int = 1004, num_seqs: int = 32, q_per_seq: int = 6) -> Wor
     ctx = np.rint(rng.lognormal(mean=math.log(2048.0), sigma=0.8, size=num_seqs))
     ctx = np.clip(ctx, 16, 16384).astype(np.int64)
     return build_workload("spec_verify", seed, ctx, q_per_seq, 32, 8, 128)
+
+
+@dataclass
+class CopyWorkload:
+    """The copy-on-write block copies of one step: the pools and the {source,
+    destination} pairs the block manager hands to pa_copy_blocks."""
+    name: str
+    seed: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    mapping: np.ndarray               # int64 [n, 2] {source, destination}
+    key_cache: torch.Tensor           # bf16 [NB, bs, H_kv, D]
+    value_cache: torch.Tensor
+
+    @property
+    def block_bytes(self) -> int:
+        return self.block_size * self.num_kv_heads * self.head_dim * 2
+
+    @property
+    def num_pairs(self) -> int:
+        return int((self.mapping >= 0).all(axis=1).sum())
+
+    def describe(self) -> str:
+        return (f"{self.name}: {self.num_pairs} block copies of {self.block_bytes} B per pool "
+                f"(H_kv={self.num_kv_heads} D={self.head_dim} bs={self.block_size}), "
+                f"NB={self.num_blocks} seed={self.seed}")
+
+
+def _bits_bf16(shape, gen: torch.Generator) -> torch.Tensor:
+    """Uniformly random 16-bit patterns as bf16 (NaN and infinity patterns included):
+    a copy must move every pattern unchanged."""
+    return torch.randint(-32768, 32768, shape, generator=gen, dtype=torch.int32).to(
+        torch.int16).view(torch.bfloat16)
+
+
+def cow_fork(seed: int = 1005, prompts: int = 16, samples: int = 8, max_prompt: int = 2048,
+             num_kv_heads: int = 8, head_dim: int = 128) -> CopyWorkload:
+    """The copy-on-write step of a parallel-sampling fork (the prefix-sharing shape: 16
+    prompts x 8 samples, 8 kv heads, head_dim 128): the samples of a prompt share all of
+    its blocks; every sample but the first writes its next token into the prompt's last
+    block, so when that block is partly filled it is copied once per such sample. Prompt
+    lengths U[1, max_prompt]; pool 1.25x the blocks needed, shuffled."""
+    rng = np.random.default_rng(seed + 7919)
+    gen = torch.Generator().manual_seed(seed)
+    lens = rng.integers(1, max_prompt, size=prompts, endpoint=True)
+    prompt_blocks = [_blocks(n, BLOCK_SIZE) for n in lens]
+    copies = sum(samples - 1 for n in lens if n % BLOCK_SIZE)
+    num_blocks = int(math.ceil(1.25 * (sum(prompt_blocks) + copies)))
+    perm = rng.permutation(num_blocks).astype(np.int64)
+    cursor = sum(prompt_blocks)
+    pairs = []
+    start = 0
+    for n, nb in zip(lens, prompt_blocks):
+        last = int(perm[start + nb - 1])
+        start += nb
+        if n % BLOCK_SIZE == 0:
+            continue  # the next token opens a new block: nothing shared is written
+        for _ in range(samples - 1):
+            pairs.append([last, int(perm[cursor])])
+            cursor += 1
+    shape = (num_blocks, BLOCK_SIZE, num_kv_heads, head_dim)
+    return CopyWorkload("cow_fork", seed, num_kv_heads, head_dim, BLOCK_SIZE, num_blocks,
+                        np.asarray(pairs, dtype=np.int64).reshape(-1, 2),
+                        _bits_bf16(shape, gen), _bits_bf16(shape, gen))
+
+
+def cow_bulk(seed: int = 1006, pairs: int = 8192, num_blocks: int = 20480, num_kv_heads: int = 8,
+             head_dim: int = 128) -> CopyWorkload:
+    """A burst of copies large enough to time the copy against HBM bandwidth (many forks
+    at once, e.g. beam search over a large batch): sources drawn with repeats from one half
+    of a shuffled pool, destinations distinct blocks of the other half."""
+    rng = np.random.default_rng(seed + 7919)
+    gen = torch.Generator().manual_seed(seed)
+    perm = rng.permutation(num_blocks).astype(np.int64)
+    half = num_blocks // 2
+    if pairs > num_blocks - half:
+        raise ValueError("pool too small for the destinations")
+    src = rng.choice(perm[:half], size=pairs, replace=True)
+    dst = perm[half:half + pairs]
+    shape = (num_blocks, BLOCK_SIZE, num_kv_heads, head_dim)
+    return CopyWorkload("cow_bulk", seed, num_kv_heads, head_dim, BLOCK_SIZE, num_blocks,
+                        np.stack([src, dst], axis=1).astype(np.int64),
+                        _bits_bf16(shape, gen), _bits_bf16(shape, gen))
+
+
+COPY_WORKLOADS = {
+    "cow_fork": cow_fork,
+    "cow_bulk": cow_bulk,
+}
+
+
+def make_copy(name: str, seed: int | None = None) -> CopyWorkload:
+    fn = COPY_WORKLOADS[name]
+    return fn() if seed is None else fn(seed)
 
 
 WORKLOADS = {

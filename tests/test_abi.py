@@ -28,7 +28,8 @@ def pa():
 def test_header_declares_the_hot_path_calls():
     syms = declared_symbols()
     for name in ["pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size", "pa_decode_plan",
-                 "pa_validate", "pa_get_device_error", "pa_status_string", "pa_version"]:
+                 "pa_validate", "pa_get_device_error", "pa_copy_blocks", "pa_status_string",
+                 "pa_version"]:
         assert name in syms
 
 
@@ -106,6 +107,30 @@ def test_cache_write_rejects_bad_arguments_before_launch(pa):
     assert call(slots=16384 + 4) == pa.PA_ERR_INVALID_ARG
     assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
     assert call(T=0, k=None) == pa.PA_OK                  # no-op
+
+
+def test_copy_blocks_rejects_bad_mappings_before_launch(pa):
+    """Every check of pa_copy_blocks runs on the host before any CUDA call (the pools
+    are never touched here, so fake aligned addresses stand in for them)."""
+    import numpy as np
+    lib = pa.raw_library()
+
+    def call(pairs, **kw):
+        a = dict(kc=4096, vc=8192, nb=10, hkv=2, d=64, bs=16)
+        a.update(kw)
+        m = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+        return lib.pa_copy_blocks(a["kc"], a["vc"], a["nb"], a["hkv"], a["d"], a["bs"],
+                                  m.ctypes.data if m.shape[0] else None, m.shape[0], None)
+    assert call([]) == pa.PA_OK                                   # no-op
+    assert call([[1, 2]], kc=None) == pa.PA_ERR_INVALID_ARG
+    assert call([[1, 2]], vc=8192 + 4) == pa.PA_ERR_INVALID_ARG
+    assert call([[1, 2]], bs=32) == pa.PA_ERR_UNSUPPORTED
+    assert call([[1, 2]], d=96) == pa.PA_ERR_UNSUPPORTED
+    assert call([[1, 10]]) == pa.PA_ERR_OUT_OF_RANGE              # past the pool
+    assert call([[10, 1]]) == pa.PA_ERR_OUT_OF_RANGE
+    assert call([[1, 3], [2, 3]]) == pa.PA_ERR_INVALID_ARG        # a destination twice
+    assert call([[1, 3], [3, 4]]) == pa.PA_ERR_INVALID_ARG        # a destination also a source
+    assert lib.pa_copy_blocks(4096, 8192, 10, 2, 64, 16, None, -1, None) == pa.PA_ERR_INVALID_ARG
 
 
 def test_plan_heuristic_host_logic(pa):

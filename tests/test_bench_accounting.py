@@ -37,3 +37,26 @@ def test_prefix_sharing_workload_unique_bytes():
     w = workloads.prefix_sharing()
     assert np.all(w.block_tables[0:8, :128] == w.block_tables[0, :128])
     assert bench.decode_bytes(w) < bench.decode_bytes(w, unique=False) / 4
+
+
+def test_copy_bytes_by_hand_and_fork_workload():
+    w = workloads.cow_fork()
+    # every pair moves one 16-token block of 8 kv heads x 128 dims (32 KB) in each pool,
+    # read once and written once
+    assert w.block_bytes == 16 * 8 * 128 * 2
+    assert bench.copy_bytes(w) == w.num_pairs * 2 * 2 * 32768
+    # the fork copies only partly filled last blocks, once per sample but the first
+    src, counts = np.unique(w.mapping[:, 0], return_counts=True)
+    assert np.all(counts == 7)
+    assert len(set(w.mapping[:, 1].tolist())) == len(w.mapping)
+    assert not set(w.mapping[:, 0].tolist()) & set(w.mapping[:, 1].tolist())
+    padded = workloads.CopyWorkload("p", 0, 8, 128, 16, 4, np.array([[0, 1], [-1, 2]], dtype=np.int64),
+                                    w.key_cache[:4], w.value_cache[:4])
+    assert bench.copy_bytes(padded) == 2 * 2 * 32768   # the padding pair moves nothing
+
+
+def test_copy_traffic_keyed_by_the_copy_sources_only():
+    assert bench.source_hash() != bench.source_hash(bench.COPY_SOURCES)
+    assert set(bench.DECODE_SOURCES).isdisjoint(bench.COPY_SOURCES)
+    csrc = os.path.join(os.path.dirname(bench.__file__), "paged_kv_cache_399_b200", "csrc")
+    assert set(bench.DECODE_SOURCES) | set(bench.COPY_SOURCES) == set(os.listdir(csrc))
