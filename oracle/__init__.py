@@ -63,6 +63,13 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode_rows.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                        _I32, _I32, _I32, _I64, ctypes.c_double, _P, _I64,
                                        _I32]
+    lib.oracle_decode_window.restype = _I32
+    lib.oracle_decode_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                         _I32, _I32, _I64, ctypes.c_double, _I32, _I32]
+    lib.oracle_decode_rows_window.restype = _I32
+    lib.oracle_decode_rows_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
+                                              _I32, _I32, _I32, _I64, ctypes.c_double, _P, _I64,
+                                              _I32, _I32]
     lib.oracle_copy_blocks.restype = _I32
     lib.oracle_copy_blocks.argtypes = [_P, _P, _I64, _I64, _P, _I64]
     lib.oracle_threads_used.restype = _I32
@@ -130,8 +137,10 @@ class Oracle:
         return kc, vc
 
     def decode(self, query, key_cache, value_cache, block_tables, context_lens,
-               q_per_seq: int, scale: float, num_threads: int = 0) -> np.ndarray:
-        """fp64 output [B, q_per_seq, H_q, D]. query is [B, q_per_seq, H_q, D] bf16."""
+               q_per_seq: int, scale: float, num_threads: int = 0, window: int = 0) -> np.ndarray:
+        """fp64 output [B, q_per_seq, H_q, D]. query is [B, q_per_seq, H_q, D] bf16.
+        window > 0: sliding window of that many tokens (table entries before every
+        row's window are not read)."""
         q = _u16(query)
         kc = _u16(key_cache)
         vc = _u16(value_cache)
@@ -141,15 +150,20 @@ class Oracle:
         assert QS == q_per_seq
         NB, BS, HKV = kc.shape[0], kc.shape[1], kc.shape[2]
         out = np.zeros((B, QS, HQ, D), dtype=np.float64)
-        st = self.lib.oracle_decode(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
-                                    _ptr(cl), B, QS, HQ, HKV, D, BS, bt.shape[1], NB,
-                                    float(scale), num_threads)
+        if window > 0:
+            st = self.lib.oracle_decode_window(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
+                                               _ptr(cl), B, QS, HQ, HKV, D, BS, bt.shape[1], NB,
+                                               float(scale), int(window), num_threads)
+        else:
+            st = self.lib.oracle_decode(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
+                                        _ptr(cl), B, QS, HQ, HKV, D, BS, bt.shape[1], NB,
+                                        float(scale), num_threads)
         if st != 0:
             raise ValueError(f"oracle_decode status {st}")
         return out
 
     def decode_rows(self, rows, query, key_cache, value_cache, block_tables, context_lens,
-                    q_per_seq: int, scale: float, num_threads: int = 0) -> np.ndarray:
+                    q_per_seq: int, scale: float, num_threads: int = 0, window: int = 0) -> np.ndarray:
         """fp64 outputs [len(rows), D] for the (b, i, h) triples in rows."""
         q = _u16(query)
         kc = _u16(key_cache)
@@ -160,9 +174,10 @@ class Oracle:
         B, QS, HQ, D = q.shape
         NB, BS, HKV = kc.shape[0], kc.shape[1], kc.shape[2]
         out = np.zeros((r.shape[0], D), dtype=np.float64)
-        st = self.lib.oracle_decode_rows(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
-                                         _ptr(cl), B, QS, HQ, HKV, D, BS, bt.shape[1], NB,
-                                         float(scale), _ptr(r), r.shape[0], num_threads)
+        st = self.lib.oracle_decode_rows_window(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt),
+                                                _ptr(cl), B, QS, HQ, HKV, D, BS, bt.shape[1], NB,
+                                                float(scale), _ptr(r), r.shape[0], int(window),
+                                                num_threads)
         if st != 0:
             raise ValueError(f"oracle_decode_rows status {st}")
         return out

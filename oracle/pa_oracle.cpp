@@ -31,6 +31,10 @@
 //     positions: query token i is at position ctx - q_per_seq + i and sees keys
 //     at positions 0..ctx - q_per_seq + i ([VS] §1.1.1 causal mask).
 //   * A query row with no visible key has output 0.
+//   * Sliding window W ([VS] §3.6.3: only the most recent W tokens are attended):
+//     query token i sees keys max(0, pos - W + 1) .. pos, pos = ctx - q_per_seq + i.
+//     Table entries wholly before every row's window are never read ([VS] §5.5 points
+//     them at the null block 0).
 //   * bf16 is widened to fp64 exactly (bit pattern << 16 is the fp32 value).
 //
 // Parity pins for every function here live in the CPU test-suite (brute force
@@ -83,18 +87,21 @@ struct Shape {
   int num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size;
   int max_blocks_per_seq;
   int64_t num_blocks;
+  int window;  // sliding window in tokens; 0 = none
 };
 
 // Gather the keys and values of one (sequence, kv head) into contiguous fp64
 // arrays [ctx][head_dim], walking the block table as [DS] §3.3 and [VS] §3.2 do:
 // token i lives in physical block block_table[i / block_size] at offset
-// i % block_size. Returns false if the table points outside the pool.
+// i % block_size. Positions before `from` are not read (they stay 0): no query row
+// sees them, and their table entries may name the null block. Returns false if the
+// table points outside the pool.
 bool gather_kv(const uint16_t* key_cache, const uint16_t* value_cache,
                const int32_t* table_row, int ctx, int kv_head, const Shape& s,
-               std::vector<double>& k_out, std::vector<double>& v_out) {
+               std::vector<double>& k_out, std::vector<double>& v_out, int from = 0) {
   k_out.assign(static_cast<size_t>(ctx) * s.head_dim, 0.0);
   v_out.assign(static_cast<size_t>(ctx) * s.head_dim, 0.0);
-  for (int i = 0; i < ctx; ++i) {
+  for (int i = from; i < ctx; ++i) {
     int64_t logical_block = i / s.block_size;
 #if ORACLE_MUTANT == 1
     int64_t offset = (i / s.block_size) % s.block_size;  // planted: wrong offset
@@ -114,37 +121,40 @@ bool gather_kv(const uint16_t* key_cache, const uint16_t* value_cache,
 }
 
 // Attention of one query row against contiguous K/V, by the definition
-// softmax(q K^T * scale) V over the visible keys 0..last_visible ([VS] §1.1.1).
-// Two passes: first the maximum score, then the weights; no online rescaling.
+// softmax(q K^T * scale) V over the visible keys first_visible..last_visible
+// ([VS] §1.1.1; first_visible > 0 only under a sliding window). Two passes: first
+// the maximum score, then the weights; no online rescaling.
 void attend_row(const double* q, const std::vector<double>& k,
-                const std::vector<double>& v, int last_visible, int head_dim,
-                double scale, double* out) {
+                const std::vector<double>& v, int first_visible, int last_visible,
+                int head_dim, double scale, double* out) {
   for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
-  if (last_visible < 0) return;  // no visible key: output defined as 0
-  const int n = last_visible + 1;
+  if (last_visible < first_visible) return;  // no visible key: output defined as 0
+  const int n = last_visible - first_visible + 1;
   std::vector<double> score(n);
-  for (int t = 0; t < n; ++t) {
+  for (int j = 0; j < n; ++j) {
+    const size_t t = static_cast<size_t>(first_visible + j);
     double dot = 0.0;
     for (int d = 0; d < head_dim; ++d) {
 #if ORACLE_MUTANT == 8
-      dot += q[d] * v[static_cast<size_t>(t) * head_dim + d];  // planted: V for K
+      dot += q[d] * v[t * head_dim + d];  // planted: V for K
 #else
-      dot += q[d] * k[static_cast<size_t>(t) * head_dim + d];
+      dot += q[d] * k[t * head_dim + d];
 #endif
     }
 #if ORACLE_MUTANT == 5
-    score[t] = dot;  // planted: scale dropped
+    score[j] = dot;  // planted: scale dropped
 #else
-    score[t] = dot * scale;
+    score[j] = dot * scale;
 #endif
   }
   double m = score[0];
-  for (int t = 1; t < n; ++t) m = std::max(m, score[t]);
+  for (int j = 1; j < n; ++j) m = std::max(m, score[j]);
   double denom = 0.0;
-  for (int t = 0; t < n; ++t) {
-    double w = std::exp(score[t] - m);
+  for (int j = 0; j < n; ++j) {
+    const size_t t = static_cast<size_t>(first_visible + j);
+    double w = std::exp(score[j] - m);
     denom += w;
-    for (int d = 0; d < head_dim; ++d) out[d] += w * v[static_cast<size_t>(t) * head_dim + d];
+    for (int d = 0; d < head_dim; ++d) out[d] += w * v[t * head_dim + d];
   }
 #if ORACLE_MUTANT == 6
   (void)denom;  // planted: missing normalisation
@@ -162,6 +172,18 @@ int last_visible_position(int ctx, int q_per_seq, int i) {
   return ctx - 1;  // planted: no causal window for speculative rows
 #else
   return ctx - q_per_seq + i;
+#endif
+}
+
+// First key position visible to a query whose last visible key is `last`. A sliding
+// window of W tokens ([VS] §3.6.3: a Mistral-style window attends to the most recent W
+// tokens only) starts at last - W + 1 (at least 0); without a window (W <= 0), at 0.
+int first_visible_position(int last, int window) {
+  if (window <= 0) return 0;
+#if ORACLE_MUTANT == 13
+  return std::max(0, last - window);  // planted: one key too many
+#else
+  return std::max(0, last - window + 1);
 #endif
 }
 
@@ -228,8 +250,10 @@ int decode_rows_impl(double* out, const uint16_t* query, const uint16_t* key_cac
       int b = static_cast<int>(u / s.num_kv_heads);
       int kvh = static_cast<int>(u % s.num_kv_heads);
       int ctx = context_lens[b];
+      // the lowest first-visible position of the sequence's query rows (row 0's)
+      const int from = std::max(0, first_visible_position(last_visible_position(ctx, s.q_per_seq, 0), s.window));
       if (!gather_kv(key_cache, value_cache, table_row_of(block_tables, b, s, context_lens),
-                     ctx, kvh, s, k, v)) {
+                     ctx, kvh, s, k, v, std::min(from, ctx))) {
         err.store(4);
         continue;
       }
@@ -238,7 +262,8 @@ int decode_rows_impl(double* out, const uint16_t* query, const uint16_t* key_cac
         const uint16_t* qsrc =
             query + ((static_cast<int64_t>(b) * s.q_per_seq + i) * s.num_q_heads + h) * s.head_dim;
         for (int d = 0; d < s.head_dim; ++d) qrow[d] = bf16_to_f64(qsrc[d]);
-        attend_row(qrow.data(), k, v, last_visible_position(ctx, s.q_per_seq, i),
+        const int last = last_visible_position(ctx, s.q_per_seq, i);
+        attend_row(qrow.data(), k, v, first_visible_position(last, s.window), last,
                    s.head_dim, scale, out + r * s.head_dim);
       }
     }
@@ -309,15 +334,18 @@ int oracle_reshape_and_cache(const uint16_t* key, const uint16_t* value,
 // Paged decode attention, every row: out[b][i][h][d] (fp64) for b < num_seqs,
 // i < q_per_seq, h < num_q_heads. block_tables is [num_seqs][max_blocks_per_seq],
 // context_lens[b] counts all tokens of sequence b including its q_per_seq new
-// ones. num_threads <= 0 uses every hardware thread. Returns 0 on success.
-int oracle_decode(double* out, const uint16_t* query, const uint16_t* key_cache,
-                  const uint16_t* value_cache, const int32_t* block_tables,
-                  const int32_t* context_lens, int num_seqs, int q_per_seq,
-                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                  int max_blocks_per_seq, int64_t num_blocks, double scale,
-                  int num_threads) {
+// ones. window > 0: a sliding window of that many tokens ending at each query's
+// position (table entries wholly before the window are not read; the pages point them
+// at the null block 0, [VS] §5.5); window <= 0: none. num_threads <= 0 uses every
+// hardware thread. Returns 0 on success.
+int oracle_decode_window(double* out, const uint16_t* query, const uint16_t* key_cache,
+                         const uint16_t* value_cache, const int32_t* block_tables,
+                         const int32_t* context_lens, int num_seqs, int q_per_seq,
+                         int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                         int max_blocks_per_seq, int64_t num_blocks, double scale,
+                         int window, int num_threads) {
   Shape s{num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size,
-          max_blocks_per_seq, num_blocks};
+          max_blocks_per_seq, num_blocks, window};
   const int64_t n_rows = static_cast<int64_t>(num_seqs) * q_per_seq * num_q_heads;
   std::vector<int32_t> rows(3 * n_rows);
   int64_t r = 0;
@@ -332,17 +360,17 @@ int oracle_decode(double* out, const uint16_t* query, const uint16_t* key_cache,
                           s, scale, rows.data(), n_rows, num_threads);
 }
 
-// Same as oracle_decode for a chosen list of rows: rows holds n_rows (b, i, h)
+// Same as oracle_decode_window for a chosen list of rows: rows holds n_rows (b, i, h)
 // triples and out receives n_rows x head_dim values in that order. Used to
 // check sampled outputs of full-size problems.
-int oracle_decode_rows(double* out, const uint16_t* query, const uint16_t* key_cache,
-                       const uint16_t* value_cache, const int32_t* block_tables,
-                       const int32_t* context_lens, int num_seqs, int q_per_seq,
-                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                       int max_blocks_per_seq, int64_t num_blocks, double scale,
-                       const int32_t* rows, int64_t n_rows, int num_threads) {
+int oracle_decode_rows_window(double* out, const uint16_t* query, const uint16_t* key_cache,
+                              const uint16_t* value_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, int num_seqs, int q_per_seq,
+                              int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                              int max_blocks_per_seq, int64_t num_blocks, double scale,
+                              const int32_t* rows, int64_t n_rows, int window, int num_threads) {
   Shape s{num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size,
-          max_blocks_per_seq, num_blocks};
+          max_blocks_per_seq, num_blocks, window};
   return decode_rows_impl(out, query, key_cache, value_cache, block_tables, context_lens,
                           s, scale, rows, n_rows, num_threads);
 }
@@ -389,6 +417,30 @@ int oracle_copy_blocks(uint16_t* key_cache, uint16_t* value_cache, int64_t num_b
     }
   }
   return 0;
+}
+
+// Without a sliding window: every key up to the query's position is visible.
+int oracle_decode(double* out, const uint16_t* query, const uint16_t* key_cache,
+                  const uint16_t* value_cache, const int32_t* block_tables,
+                  const int32_t* context_lens, int num_seqs, int q_per_seq,
+                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int64_t num_blocks, double scale,
+                  int num_threads) {
+  return oracle_decode_window(out, query, key_cache, value_cache, block_tables, context_lens,
+                              num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                              block_size, max_blocks_per_seq, num_blocks, scale, 0, num_threads);
+}
+
+int oracle_decode_rows(double* out, const uint16_t* query, const uint16_t* key_cache,
+                       const uint16_t* value_cache, const int32_t* block_tables,
+                       const int32_t* context_lens, int num_seqs, int q_per_seq,
+                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, double scale,
+                       const int32_t* rows, int64_t n_rows, int num_threads) {
+  return oracle_decode_rows_window(out, query, key_cache, value_cache, block_tables,
+                                   context_lens, num_seqs, q_per_seq, num_q_heads,
+                                   num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                   num_blocks, scale, rows, n_rows, 0, num_threads);
 }
 
 // Threads the last decode call ran on.

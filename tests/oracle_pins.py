@@ -9,7 +9,9 @@ when the oracle disagrees with:
   * invariants (block permutation, shared prefixes, GQA vs MHA, speculative
     rows vs shorter single-token calls, tiled online softmax and split/merge),
   * the copy-on-write rule of parallel sampling (a fork's writer copies the shared
-    last block and writes there; the other candidates still read the original).
+    last block and writes there; the other candidates still read the original),
+  * the sliding window (the most recent W tokens; entries before it may name the null
+    block 0 and are never read).
 The same checks run against deliberately broken builds of the oracle
 (tests/test_oracle_mutants.py) to show that each planted mistake is caught.
 """
@@ -79,7 +81,7 @@ class Problem:
         self.pool_k, self.pool_v = pool_k, pool_v
 
     def run(self, oracle, pool_k=None, pool_v=None, tables=None, ctxs=None, Q=None, q=None,
-            scale=None):
+            scale=None, window=0):
         pk = self.pool_k if pool_k is None else pool_k
         pv = self.pool_v if pool_v is None else pool_v
         qq = self.Q if Q is None else Q
@@ -87,7 +89,7 @@ class Problem:
                              self.tables if tables is None else tables,
                              np.asarray(self.ctxs if ctxs is None else ctxs, dtype=np.int32),
                              self.q if q is None else q,
-                             self.scale if scale is None else scale)
+                             self.scale if scale is None else scale, window=window)
 
 
 def brute_force(p: Problem) -> np.ndarray:
@@ -458,6 +460,67 @@ def check_copy_on_write(oracle):
         raise AssertionError(f"mapping {bad} not rejected")
 
 
+def _brute_force_window(p, window):
+    """Textbook attention over the keys max(0, pos - W + 1) .. pos of the contiguous K/V."""
+    g = p.hq // p.hkv
+    out = np.zeros((p.B, p.q, p.hq, p.d))
+    for b in range(p.B):
+        for i in range(p.q):
+            last = p.ctxs[b] - p.q + i
+            first = max(0, last - window + 1)
+            for h in range(p.hq):
+                kv = h // g
+                keys = range(first, last + 1)
+                s = np.array([p.scale * float(np.dot(p.Q[b, i, h], p.K[b][t, kv])) for t in keys])
+                w = np.exp(s - s.max())
+                out[b, i, h] = (w[:, None] * p.V[b][first:last + 1, kv]).sum(0) / w.sum()
+    return out
+
+
+def check_sliding_window(oracle):
+    """golden/sliding_window.json: the most recent W tokens only; positions before the window
+    may point at the null block 0, whose contents are never read."""
+    g = json.load(open(os.path.join(GOLDEN, "sliding_window.json")))
+    p = Problem(seed=101, ctxs=[37, 50, 5, 16], q=3, hq=4, hkv=2, d=16, extra_blocks=4)
+    for W in (1, 2, 7, 16, 17, 33, 64):
+        _close(p.run(oracle, window=W), _brute_force_window(p, W), tol=1e-10, what=f"window {W}")
+    # a one-token window is the query's own value row exactly
+    out1 = p.run(oracle, window=1)
+    for b in range(p.B):
+        for i in range(p.q):
+            last = p.ctxs[b] - p.q + i
+            for h in range(p.hq):
+                assert np.array_equal(out1[b, i, h], p.V[b][last, h // (p.hq // p.hkv)]), "W=1 closed form"
+    # a window at least as long as every context is no window
+    assert np.array_equal(p.run(oracle, window=max(p.ctxs)), p.run(oracle)), "W >= ctx"
+    # the null block: relabel so that block 0 is unused, fill it with NaN, point every entry
+    # wholly before a sequence's window at it
+    null = g["null_block"]
+    used = set(int(x) for b in range(p.B) for x in p.tables[b, :-(-p.ctxs[b] // p.bs)])
+    spare = next(x for x in range(p.nb) if x not in used)
+    tables = p.tables.copy()
+    pk, pv = p.pool_k.copy(), p.pool_v.copy()
+    if null in used:   # swap the contents and names of block `null` and the spare block
+        pk[[null, spare]] = pk[[spare, null]]
+        pv[[null, spare]] = pv[[spare, null]]
+        tables = np.where(p.tables == null, spare, p.tables).astype(np.int32)
+    W = 7
+    ref = p.run(oracle, pool_k=pk, pool_v=pv, tables=tables, window=W)
+    pk[null] = np.nan
+    pv[null] = np.nan
+    for b in range(p.B):
+        first = max(0, p.ctxs[b] - p.q - W + 1)   # row 0's first visible key
+        tables[b, :first // p.bs] = null
+    got = p.run(oracle, pool_k=pk, pool_v=pv, tables=tables, window=W)
+    assert np.array_equal(got, ref), "an entry before the window was read"
+    # visible key counts: min(W, pos + 1), through weights on a one-hot value pattern
+    q1 = Problem(seed=103, ctxs=[30], q=1, hq=1, hkv=1, d=16, same_keys=True)
+    for W in (1, 5, 30, 40):
+        o = q1.run(oracle, window=W)[0, 0, 0]
+        n = min(W, 30)
+        assert np.allclose(o, q1.V[0][30 - n:30, 0].mean(0), atol=1e-12), f"visible keys for W={W}"
+
+
 ALL_CHECKS = [
     check_bf16_widening,
     check_block_counts_golden,
@@ -474,4 +537,5 @@ ALL_CHECKS = [
     check_online_and_split_merge,
     check_cache_write,
     check_copy_on_write,
+    check_sliding_window,
 ]

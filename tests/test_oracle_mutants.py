@@ -21,6 +21,7 @@ MUTANTS = {
     10: "cache write one slot off",
     11: "bf16 widened with the wrong shift",
     12: "pool laid out head-major inside a block",
+    13: "sliding window one key too long",
     31: "block copy leaves the value pool out",
     32: "block copy leaves the block's last token behind",
     33: "block copy with source and destination swapped",
