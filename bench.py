@@ -34,14 +34,16 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram__bytes_write.sum summed over the launch's kernels), keyed by workload, with
 # the hash of the kernel sources it was measured on. A different hash -> null.
 NCU_TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call, from
-    # one ncu capture per workload (summaries with the commands in profiles/); valid only for
+    # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call (mean
+    # of three calls), from one ncu capture per workload (commands in profiles/); valid only for
     # the kernel sources they were taken on
-    "llama8b": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 658_770_000},
-    "llama70b_long": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 1_354_610_000},
-    "spec_verify": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 416_740_000},
-    "prefix_sharing": {"source_hash": "1f9ec32cbf2fc15e", "bytes_per_launch": 213_430_000},
+    "llama8b": {"source_hash": "8e875f10c7ef699b", "bytes_per_launch": 654_500_000},
+    "llama70b_long": {"source_hash": "8e875f10c7ef699b", "bytes_per_launch": 1_352_200_000},
+    "spec_verify": {"source_hash": "8e875f10c7ef699b", "bytes_per_launch": 414_700_000},
+    "prefix_sharing": {"source_hash": "8e875f10c7ef699b", "bytes_per_launch": 210_050_000},
+    "sliding_window": {"source_hash": "8e875f10c7ef699b", "bytes_per_launch": 274_200_000},
 }
+
 # the same for one pa_copy_blocks launch of a copy workload (keyed by COPY_SOURCES' hash;
 # mean of three 2048-pair launches: the writes still in L2 when a launch ends are not
 # counted, so the traffic sits below the algorithmic bytes)
@@ -62,27 +64,30 @@ def decode_bytes(w, unique: bool = True) -> int:
     physical slots counted once when `unique`), q, out, the used block-table
     entries and context_lens."""
     bs = w.block_size
+    win = getattr(w, "window", 0)
+    # the first position any query row of a sequence sees (its first row's window start)
+    lo = [max(0, int(c) - w.q_per_seq - win + 1) if win > 0 else 0 for c in w.context_lens]
     if unique:
-        slots = set()
+        ranges = {}   # physical block -> offset ranges [s, e) some sequence sees
         for b in range(w.num_seqs):
             ctx = int(w.context_lens[b])
             tbl = w.block_tables[b]
-            nfull, tail = divmod(ctx, bs)
-            for j in range(nfull):
-                slots.add((int(tbl[j]), bs))
-            if tail:
-                key = (int(tbl[nfull]), tail)
-                slots.add(key)
-        # a block read to `fill` tokens by one sequence and fully by another counts once, fully
-        per_block = {}
-        for blk, fill in slots:
-            per_block[blk] = max(per_block.get(blk, 0), fill)
-        tokens = sum(per_block.values())
+            for j in range(lo[b] // bs, -(-ctx // bs)):
+                s, e = max(lo[b], j * bs) - j * bs, min(ctx, (j + 1) * bs) - j * bs
+                ranges.setdefault(int(tbl[j]), []).append((s, e))
+        tokens = 0
+        for rs in ranges.values():   # a slot seen by several sequences counts once
+            end = 0
+            for s, e in sorted(rs):
+                s = max(s, end)
+                if e > s:
+                    tokens += e - s
+                    end = e
     else:
-        tokens = int(np.sum(w.context_lens.astype(np.int64)))
+        tokens = int(sum(int(c) - l for c, l in zip(w.context_lens, lo)))
     kv = tokens * w.num_kv_heads * w.head_dim * 2 * 2
     qo = 2 * w.num_seqs * w.q_per_seq * w.num_q_heads * w.head_dim * 2
-    tables = int(sum(-(-int(c) // bs) for c in w.context_lens)) * 4
+    tables = int(sum(-(-int(c) // bs) - l // bs for c, l in zip(w.context_lens, lo))) * 4
     return kv + qo + tables + w.num_seqs * 4
 
 
@@ -131,7 +136,7 @@ def measured_peaks():
 # ------------------------------------------------------------------ ranks
 
 BASE_SEEDS = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
-              "spec_verify": 1004, "cow_fork": 1005, "cow_bulk": 1006}
+              "spec_verify": 1004, "cow_fork": 1005, "cow_bulk": 1006, "sliding_window": 1007}
 
 
 def rank_seed(workload: str, rank: int) -> int:
@@ -267,7 +272,7 @@ def run_gpu(args):
     # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
     share = bool(w.shared_groups) and not args.no_share_prefix
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                             w.max_blocks_per_seq, share_prefix=share,
+                             w.max_blocks_per_seq, share_prefix=share, sliding_window=w.window,
                              path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
                              split_blocks=args.split_blocks,
                              schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
@@ -444,7 +449,7 @@ def _oracle_step(orc, w, seqs):
         -1, w.num_kv_heads, w.head_dim)
     kc, vc = orc.reshape_and_cache(sub_key, sub_val, w.key_cache, w.value_cache, sub_slots)
     return orc.decode(w.query[seqs], kc, vc, w.block_tables[seqs], w.context_lens[seqs], w.q_per_seq,
-                      w.scale)
+                      w.scale, window=w.window)
 
 
 def _sample_workload(w, seqs):
@@ -750,7 +755,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify",
-                             "cow_fork", "cow_bulk"],
+                             "sliding_window", "cow_fork", "cow_bulk"],
                     help="decode workloads time cache write + decode; cow_fork / cow_bulk time the "
                          "copy-on-write block copy")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -122,6 +122,13 @@ typedef struct {
                             common prefix blocks are read once for all of them (up to
                             32 / (GQA group x q_per_seq) sequences per read; tensor-core
                             kernels only); 0 = off */
+  int32_t sliding_window; /* > 0: each query token attends to the most recent
+                            sliding_window tokens only, keys pos - W + 1 .. pos (vLLM
+                            study notes §3.6.3); table entries wholly before every row's
+                            window are never read (the pages point them at the null
+                            block 0, §5.5). Grid schedule, mma.sync or CUDA-core path;
+                            with the tcgen05 path, the persistent schedule or
+                            share_prefix: PA_ERR_UNSUPPORTED. 0 = no window */
 } pa_plan_hints_t;
 
 /* A decode plan; fill it with pa_decode_plan and treat it as opaque. */
@@ -129,13 +136,18 @@ typedef struct {
   int32_t path;          /* PA_PATH_SINGLE, PA_PATH_TILE or PA_PATH_TCGEN05 */
   int32_t schedule;      /* PA_SCHEDULE_GRID or PA_SCHEDULE_PERSISTENT */
   int32_t split_blocks;  /* grid: blocks per split */
-  int32_t num_splits;    /* grid: ceil(max_blocks_per_seq / split_blocks) */
+  int32_t num_splits;    /* grid: ceil(max_blocks_per_seq / split_blocks) (see
+                            sliding_window) */
   int32_t rows_per_cta;  /* query rows (GQA group x q_per_seq) one CTA holds; tcgen05:
                             the MMA's N (16 or 32) */
   int32_t num_ctas;      /* persistent: CTAs launched (resident slots of the device); a
                             caller may lower or raise it (the workspace size follows) */
   int32_t share_cap;     /* sequences per shared-prefix unit, 0 = off */
   int32_t share_split_blocks; /* grid with sharing: blocks per split of a shared prefix */
+  int32_t sliding_window; /* tokens of the sliding window, 0 = none; with a window,
+                            num_splits covers the window's blocks,
+                            ceil(min(max_blocks_per_seq, ceil((W + q_per_seq - 1) / 16) + 1)
+                            / split_blocks) */
 } pa_plan_t;
 
 /* Write the step's new K/V into the pool: for each token t with slot s =

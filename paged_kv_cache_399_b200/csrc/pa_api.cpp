@@ -109,6 +109,14 @@ bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_bl
 
 // ----------------------------------------------------------------- plan
 
+// Blocks of one sequence's table that a decode reads: every block without a window; with
+// a window of W tokens at most the blocks spanning the last W + q - 1 positions.
+int32_t window_span_blocks(int32_t window, int32_t q_per_seq, int32_t max_blocks_per_seq) {
+  if (window <= 0) return max_blocks_per_seq;
+  const int64_t span = ceil_div(static_cast<int64_t>(window) + q_per_seq - 1, pa::kBlockSize) + 1;
+  return static_cast<int32_t>(span < max_blocks_per_seq ? span : max_blocks_per_seq);
+}
+
 int rows_per_cta_for(int path, int rows) {
   if (path == pa::kPathTcgen05) return rows <= 16 ? 16 : pa::kTcmMaxRows;
   if (path == pa::kPathTile) {
@@ -150,7 +158,12 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (h.schedule != PA_SCHEDULE_AUTO && h.schedule != PA_SCHEDULE_GRID &&
       h.schedule != PA_SCHEDULE_PERSISTENT)
     return PA_ERR_INVALID_ARG;
-  if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1) return PA_ERR_INVALID_ARG;
+  if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1 || h.sliding_window < 0)
+    return PA_ERR_INVALID_ARG;
+  // a sliding window runs on the grid schedule of the mma.sync and CUDA-core kernels
+  if (h.sliding_window > 0 && (h.path == PA_PATH_TCGEN05 || h.schedule == PA_SCHEDULE_PERSISTENT ||
+                               h.share_prefix))
+    return PA_ERR_UNSUPPORTED;
   const int group = num_q_heads / num_kv_heads;
   const int rows = group * q_per_seq;
   int schedule = h.schedule == PA_SCHEDULE_AUTO ? PA_SCHEDULE_GRID : h.schedule;
@@ -169,7 +182,7 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     // measured on B200: the tcgen05 kernel wins for head_dim 128 with more than 16 rows per
     // kv head or with prefix sharing; mma.sync tiles win below that; CUDA cores for <= 2 rows
     if (head_dim == 128 && (rows > 16 || share_cap > 0) && h.schedule != PA_SCHEDULE_GRID &&
-        h.split_blocks == 0) {
+        h.split_blocks == 0 && h.sliding_window == 0) {
       path = PA_PATH_TCGEN05;
       schedule = PA_SCHEDULE_PERSISTENT;
     } else {
@@ -186,6 +199,9 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   plan->rows_per_cta = rpc;
   plan->share_cap = share_cap;
   plan->share_split_blocks = 0;
+  plan->sliding_window = h.sliding_window;
+  // blocks one sequence reads: all of its table, or the span of the window
+  const int32_t span = window_span_blocks(h.sliding_window, q_per_seq, max_blocks_per_seq);
   if (schedule == PA_SCHEDULE_PERSISTENT) {
     plan->num_ctas = slots;
     plan->split_blocks = max_blocks_per_seq;
@@ -210,16 +226,16 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     // possible context into pieces so that about four waves of CTAs exist.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * row_chunks;
     if (units >= 2 * static_cast<int64_t>(slots) || units == 0) {
-      split_blocks = max_blocks_per_seq;
+      split_blocks = span;
     } else {
       const int64_t splits = ceil_div(4 * static_cast<int64_t>(slots), units);
-      int64_t sb = ceil_div(max_blocks_per_seq, splits);
+      int64_t sb = ceil_div(span, splits);
       sb = ceil_div(sb, pa::kWarpsPerCta) * pa::kWarpsPerCta;
       if (sb < 8 * pa::kWarpsPerCta) sb = 8 * pa::kWarpsPerCta;
-      split_blocks = static_cast<int32_t>(sb < max_blocks_per_seq ? sb : max_blocks_per_seq);
+      split_blocks = static_cast<int32_t>(sb < span ? sb : span);
     }
   }
-  const int64_t num_splits = ceil_div(max_blocks_per_seq, split_blocks);
+  const int64_t num_splits = ceil_div(span, split_blocks);
   if (num_splits > 65535) return PA_ERR_UNSUPPORTED;  // grid z
   plan->split_blocks = split_blocks;
   plan->num_splits = static_cast<int32_t>(num_splits);
@@ -314,6 +330,10 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
                        int32_t num_kv_heads, int32_t max_blocks_per_seq) {
   if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE && plan.path != PA_PATH_TCGEN05)
     return PA_ERR_INVALID_ARG;
+  if (plan.sliding_window < 0) return PA_ERR_INVALID_ARG;
+  if (plan.sliding_window > 0 &&
+      (plan.path == PA_PATH_TCGEN05 || plan.schedule != PA_SCHEDULE_GRID || plan.share_cap != 0))
+    return PA_ERR_UNSUPPORTED;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
   if (plan.path == PA_PATH_TCGEN05) {
     if (plan.schedule != PA_SCHEDULE_PERSISTENT || plan.share_split_blocks != 0 || plan.num_ctas <= 0 ||
@@ -335,7 +355,9 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
     }
   } else if (plan.schedule == PA_SCHEDULE_GRID) {
     if (plan.split_blocks <= 0) return PA_ERR_INVALID_ARG;
-    if (plan.num_splits != ceil_div(max_blocks_per_seq, plan.split_blocks)) return PA_ERR_INVALID_ARG;
+    if (plan.num_splits !=
+        ceil_div(window_span_blocks(plan.sliding_window, q_per_seq, max_blocks_per_seq), plan.split_blocks))
+      return PA_ERR_INVALID_ARG;
     if (plan.share_cap != 0) {
       if (plan.path != PA_PATH_TILE || plan.share_cap != share_cap_for(rows) ||
           plan.rows_per_cta != pa::kTileMaxRows || plan.share_split_blocks <= 0)
@@ -468,6 +490,7 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
   p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
   p.scale_log2 = scale * 1.4426950408889634f;
   p.split_blocks = plan->split_blocks;
+  p.window = plan->sliding_window;
   p.num_splits = plan->num_splits;
   const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
   char* ws = static_cast<char*>(workspace);

@@ -42,6 +42,7 @@ struct DecodeParams {
   int32_t rows_per_cta;          // rows the kernel instance holds (ROWS)
   int32_t row_chunks;            // ceil(rows / rows_per_cta)
   float scale_log2;              // scale * log2(e)
+  int32_t window;                // sliding window in tokens (grid schedule only); 0 = none
 
   // grid schedule: split partials for the merge kernel; with prefix sharing also the
   // shared-prefix splits (a 1-D grid: shared CTAs, then the sequences' own CTAs)

@@ -82,6 +82,12 @@ __device__ __forceinline__ int num_blocks_of(const DecodeParams& p, int ctx) {
   return min(max(ctx, 0) + kBlockSize - 1, p.max_blocks * kBlockSize) / kBlockSize;
 }
 
+// Sliding window: the first block holding a key that some query row of a sequence with
+// ctx tokens sees (its first query token's window start); 0 without a window.
+__device__ __forceinline__ int window_first_block(const DecodeParams& p, int ctx) {
+  return p.window > 0 ? max(0, ctx - p.q_per_seq - p.window + 1) / kBlockSize : 0;
+}
+
 // ---------------------------------------------------------------------------
 // A segment: consecutive blocks [blk0, blk1) of one kv head, for a set of query rows.
 // Private: rows row0 .. row0+nrows-1 of sequence b0. Shared: `members` sequences
@@ -244,8 +250,10 @@ struct TileCore {
         for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
   }
 
+  // win > 0: sliding window (a row with last visible key lim sees keys lim - win + 1 ..
+  // lim); vlo: no row of the segment sees a key before it (INT_MIN without a window)
   __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, int tb, bool need_mask,
-                                        float c, int lane, float*) {
+                                        float c, int lane, float*, int win, int vlo) {
     const uint32_t kb = smem_u32(kt);
     const uint32_t vb = smem_u32(vt);
     const int lm = lane >> 3, lr = lane & 7;
@@ -276,6 +284,15 @@ struct TileCore {
         if (t0 + 8 > lim[nt][0]) sc[nt][2] = -INFINITY;
         if (t0 + 8 > lim[nt][1]) sc[nt][3] = -INFINITY;
       }
+      if (win > 0) {  // keys before a row's window: t <= lim - win
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (t0 + win <= lim[nt][0]) sc[nt][0] = -INFINITY;
+          if (t0 + win <= lim[nt][1]) sc[nt][1] = -INFINITY;
+          if (t0 + 8 + win <= lim[nt][0]) sc[nt][2] = -INFINITY;
+          if (t0 + 8 + win <= lim[nt][1]) sc[nt][3] = -INFINITY;
+        }
+      }
     }
     uint32_t pb[NT][2];
     float alpha[NT][2];
@@ -305,15 +322,17 @@ struct TileCore {
       pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[nt][0], sc[nt][1]));
       pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[nt][2], sc[nt][3]));
     }
-    // Slots of the last block past the context may hold any bits (NaN too): their p is 0,
-    // but 0 * NaN is NaN, so their V elements are cleared in the operand fragments
-    // (a0/a1 hold tokens 2c, 2c+1 and a2/a3 tokens 2c+8, 2c+9 of the block, c = lane & 3).
-    const bool vmask = need_mask && tb + kBlockSize - 1 > vlim;
+    // Slots of the last block past the context, and slots before every row's window, may
+    // hold any bits (NaN too): their p is 0, but 0 * NaN is NaN, so their V elements are
+    // cleared in the operand fragments (a0/a1 hold tokens 2c, 2c+1 and a2/a3 tokens
+    // 2c+8, 2c+9 of the block, c = lane & 3).
+    const bool vmask = need_mask && (tb + kBlockSize - 1 > vlim || tb < vlo);
     uint32_t vm_lo = ~0u, vm_hi = ~0u;
     if (vmask) {
       const int t = tb + 2 * (lane & 3);
-      vm_lo = (t <= vlim ? 0x0000FFFFu : 0u) | (t + 1 <= vlim ? 0xFFFF0000u : 0u);
-      vm_hi = (t + 8 <= vlim ? 0x0000FFFFu : 0u) | (t + 9 <= vlim ? 0xFFFF0000u : 0u);
+      auto keep = [&](int tt) { return tt <= vlim && tt >= vlo; };
+      vm_lo = (keep(t) ? 0x0000FFFFu : 0u) | (keep(t + 1) ? 0xFFFF0000u : 0u);
+      vm_hi = (keep(t + 8) ? 0x0000FFFFu : 0u) | (keep(t + 9) ? 0xFFFF0000u : 0u);
     }
     if (__any_sync(kFull, rescale)) {
 #pragma unroll
@@ -436,7 +455,7 @@ struct SimtCore {
   }
 
   __device__ __forceinline__ void block(const uint8_t* kt, const uint8_t* vt, int tb, bool need_mask,
-                                        float c, int lane, float*) {
+                                        float c, int lane, float*, int win, int vlo) {
     const int t_me = lane >> 1;
     const int half = lane & 1;
     float sc[ROWS];
@@ -467,7 +486,7 @@ struct SimtCore {
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       float sv = (sc[r] + __shfl_xor_sync(kFull, sc[r], 1)) * c;  // log2 units
-      if (need_mask && t_glob > lim[r]) sv = -INFINITY;
+      if (need_mask && (t_glob > lim[r] || (win > 0 && t_glob + win <= lim[r]))) sv = -INFINITY;
       float mx = sv;
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
@@ -502,7 +521,7 @@ struct SimtCore {
         const uint32_t vv = *reinterpret_cast<const uint32_t*>(vrow);
         vf[0] = bf16_lo(vv); vf[1] = bf16_hi(vv);
       }
-      if (need_mask && tb + t > vlim) {  // a slot past the context: p = 0, V may be NaN
+      if (need_mask && (tb + t > vlim || tb + t < vlo)) {  // outside every row's keys: p = 0, V may be NaN
 #pragma unroll
         for (int e = 0; e < DPL; ++e) vf[e] = 0.f;
       }
@@ -578,6 +597,10 @@ __device__ __forceinline__ void run_segment(const DecodeParams& p, const Seg& sg
   core.begin(p, sg, ctx, lane);
   const float c = p.scale_log2;
   const int first_masked = ctx - p.q_per_seq;  // blocks ending past this position need the mask
+  // sliding window: the segment's first row (query token row0 / G) has the lowest window
+  // start; blocks starting before ctx - win (the last query's window start) need the mask
+  const int win = p.window;
+  const int vlo = win > 0 ? ctx - p.q_per_seq + sg.row0 / p.group - win + 1 : INT_MIN;
   for (int k = 0; k < pipe.n_my; ++k) {
     if (!pipe.wait(k)) {
       if (lane == 0) record_error(kErrTimeoutDecode);
@@ -586,8 +609,8 @@ __device__ __forceinline__ void run_segment(const DecodeParams& p, const Seg& sg
     }
     const int s = pipe.stage_of(k);
     const int tb = pipe.block_of(k) * kBlockSize;
-    const bool need_mask = !sg.shared && tb + kBlockSize - 1 > first_masked;
-    core.block(pipe.kbuf(s), pipe.vbuf(s), tb, need_mask, c, lane, nullptr);
+    const bool need_mask = !sg.shared && (tb + kBlockSize - 1 > first_masked || (win > 0 && tb < ctx - win));
+    core.block(pipe.kbuf(s), pipe.vbuf(s), tb, need_mask, c, lane, nullptr, win, vlo);
     __syncwarp();
     if (k + STAGES < pipe.n_my) pipe.issue(k + STAGES, tk, tv);
   }
@@ -1139,7 +1162,8 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   const int nblk = num_blocks_of(p, ctx);
   const int S = p.num_splits;
   const int sb = p.split_blocks;
-  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : 0;  // own blocks start after the shared prefix
+  // own blocks start after the shared prefix, or at the first block of the window
+  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
   Seg sg{b, 1, kvh, rc * ROWS, min(ROWS, p.rows - rc * ROWS), 0, 0, false};
   const int blk0 = P_b + z * sb;
   if (blk0 >= nblk) {
@@ -1156,7 +1180,7 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   sg.blk0 = blk0;
   sg.blk1 = min(nblk, blk0 + sb);
   // the only piece of its outputs: write bf16 directly
-  const bool direct = P_b == 0 && nblk <= sb;
+  const bool direct = (p.share_cap == 0 || P_b == 0) && nblk - P_b <= sb;
   run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
   grid_launch_dependents();
   // own-block records follow the shared-prefix records when sharing is on
@@ -1272,12 +1296,14 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
   const int MW = blockDim.x >> 5;
   const int b = row / RQ;
   const int rq = row % RQ;
-  const int nblk = num_blocks_of(p, __ldg(p.context_lens + b));
+  const int ctx = __ldg(p.context_lens + b);
+  const int nblk = num_blocks_of(p, ctx);
   const int sb = p.split_blocks;
   // records: the shared-prefix splits (region 0, with prefix sharing) then the
-  // sequence's own splits (region 1 with prefix sharing, else region 0)
-  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : 0;
-  const int nsh = P_b > 0 ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
+  // sequence's own splits (region 1 with prefix sharing, else region 0); with a sliding
+  // window the own blocks start at the window's first block
+  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
+  const int nsh = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
   const int ns = nsh + (nblk - P_b + sb - 1) / sb;
   if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
   const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;

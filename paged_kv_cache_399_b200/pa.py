@@ -47,21 +47,24 @@ PA_SCHEDULE_PERSISTENT = 2
 
 class pa_plan_hints_t(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
-                ("split_blocks", ctypes.c_int32), ("share_prefix", ctypes.c_int32)]
+                ("split_blocks", ctypes.c_int32), ("share_prefix", ctypes.c_int32),
+                ("sliding_window", ctypes.c_int32)]
 
 
 class pa_plan_t(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
                 ("split_blocks", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("rows_per_cta", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
-                ("share_cap", ctypes.c_int32), ("share_split_blocks", ctypes.c_int32)]
+                ("share_cap", ctypes.c_int32), ("share_split_blocks", ctypes.c_int32),
+                ("sliding_window", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {"path": {1: "single", 2: "tile", 3: "tcgen05"}.get(self.path, self.path),
                 "schedule": {1: "grid", 2: "persistent"}.get(self.schedule, self.schedule),
                 "split_blocks": self.split_blocks, "num_splits": self.num_splits,
                 "rows_per_cta": self.rows_per_cta, "num_ctas": self.num_ctas,
-                "share_cap": self.share_cap, "share_split_blocks": self.share_split_blocks}
+                "share_cap": self.share_cap, "share_split_blocks": self.share_split_blocks,
+                "sliding_window": self.sliding_window}
 
     def __repr__(self):
         return f"pa_plan_t({self.as_dict()})"
@@ -171,12 +174,12 @@ def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, block_map
 def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,
                    head_dim: int, max_blocks_per_seq: int, path: int = PA_PATH_AUTO,
                    split_blocks: int = 0, schedule: int = PA_SCHEDULE_AUTO,
-                   share_prefix: bool = False) -> pa_plan_t:
+                   share_prefix: bool = False, sliding_window: int = 0) -> pa_plan_t:
     """A forced split length implies the grid schedule (the tcgen05 path has no split
     length: its schedule cuts the work into equal tile ranges, and ignores it)."""
     if split_blocks and schedule == PA_SCHEDULE_AUTO and path != PA_PATH_TCGEN05:
         schedule = PA_SCHEDULE_GRID
-    hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)))
+    hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)), int(sliding_window))
     plan = pa_plan_t()
     st = _lib.pa_decode_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
                              max_blocks_per_seq, ctypes.byref(hints), ctypes.byref(plan))

@@ -22,6 +22,9 @@ notes §1.2.2):
 * ``spec_verify``     32 seqs x 6 query tokens (causal inside the window), 32/8 heads,
                       context lognormal(ln 2048, 0.8) clipped to [16, 16384]; the slot
                       mapping writes all 6 new tokens.
+* ``sliding_window``  16 x 1, 32/8 heads, head_dim 128, a 4096-token sliding window over
+                      contexts U[8192, 32768]; entries before the window name the null
+                      block 0.
 
 Copy-on-write block copies (``make_copy``; the copy rule of the vLLM study notes
 §3.2.2):
@@ -66,6 +69,7 @@ class Workload:
     value_cache: torch.Tensor         # bf16 [NB, bs, H_kv, D]
     blocks_used: np.ndarray = field(default=None)   # int32 [B] blocks owned per sequence
     shared_groups: list = field(default_factory=list)  # [(members, prefix_tokens)]
+    window: int = 0                   # sliding window in tokens, 0 = none
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -80,7 +84,7 @@ class Workload:
                 f"H_kv={self.num_kv_heads} D={self.head_dim} bs={self.block_size} "
                 f"ctx[min/mean/max]={int(self.context_lens.min())}/"
                 f"{float(self.context_lens.mean()):.0f}/{int(self.context_lens.max())} "
-                f"NB={self.num_blocks} seed={self.seed}")
+                f"NB={self.num_blocks} seed={self.seed}" + (f" window={self.window}" if self.window else ""))
 
 
 def _blocks(n_tokens: int, block_size: int) -> int:
@@ -103,13 +107,17 @@ def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_hea
                    num_kv_heads: int, head_dim: int, scale: float | None = None,
                    block_size: int = BLOCK_SIZE, pool_factor: float = 1.25,
                    num_blocks: int | None = None, share_groups=None,
-                   max_blocks_per_seq: int | None = None) -> Workload:
+                   max_blocks_per_seq: int | None = None, window: int = 0) -> Workload:
     """General builder.
 
     share_groups: optional list of (member_sequence_ids, prefix_tokens); the
     members map their first prefix_tokens (a multiple of block_size) to the same
     physical blocks. All other blocks are private. Physical ids come from one
     seeded permutation of the pool, so no two sequences alias a private block.
+
+    window > 0: a sliding window of that many tokens. Only the blocks a sequence's rows
+    can see are allocated; the table entries wholly before the first row's window point
+    at the null block 0, which is reserved (the vLLM study notes, §5.5).
     """
     rng = np.random.default_rng(seed)
     gen = torch.Generator().manual_seed(seed)
@@ -118,7 +126,12 @@ def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_hea
     if np.any(ctx < q_per_seq):
         raise ValueError("every context must hold its q_per_seq new tokens")
     need = np.array([_blocks(c, block_size) for c in ctx], dtype=np.int64)
+    # first block a row of the sequence sees (0 without a window)
+    lo_blk = np.array([max(0, int(c) - q_per_seq - window + 1) // block_size if window > 0 else 0
+                       for c in ctx], dtype=np.int64)
     share_groups = list(share_groups or [])
+    if window > 0 and share_groups:
+        raise ValueError("a sliding window with shared prefixes is not generated")
     shared_prefix_blocks = np.zeros(B, dtype=np.int64)
     leader = np.arange(B)
     for members, prefix_tokens in share_groups:
@@ -127,18 +140,19 @@ def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_hea
         for m in members:
             shared_prefix_blocks[m] = prefix_tokens // block_size
             leader[m] = members[0]
-    distinct = int(need.sum() - sum(shared_prefix_blocks[m] for members, _ in share_groups
-                                     for m in members[1:]))
+    distinct = int((need - lo_blk).sum() - sum(shared_prefix_blocks[m] for members, _ in share_groups
+                                                for m in members[1:]))
+    reserved = 1 if window > 0 else 0   # the null block
     if num_blocks is None:
-        num_blocks = int(math.ceil(pool_factor * distinct))
-    if num_blocks < distinct:
+        num_blocks = int(math.ceil(pool_factor * distinct)) + reserved
+    if num_blocks < distinct + reserved:
         raise ValueError("pool too small")
-    perm = rng.permutation(num_blocks).astype(np.int64)
+    perm = (reserved + rng.permutation(num_blocks - reserved)).astype(np.int64)
     width = int(max_blocks_per_seq or need.max())
     tables = np.zeros((B, width), dtype=np.int32)  # padding entries point at block 0
     cursor = 0
     for b in range(B):
-        start = 0
+        start = int(lo_blk[b])   # entries before it stay 0: the null block
         if shared_prefix_blocks[b] and leader[b] != b:
             start = int(shared_prefix_blocks[b])
             tables[b, :start] = tables[leader[b], :start]
@@ -164,7 +178,7 @@ def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_hea
                     context_lens=ctx.astype(np.int32), block_tables=tables,
                     num_blocks=int(num_blocks), query=query, key=key, value=value,
                     slot_mapping=slots, key_cache=key_cache, value_cache=value_cache,
-                    blocks_used=need.astype(np.int32), shared_groups=share_groups)
+                    blocks_used=need.astype(np.int32), shared_groups=share_groups, window=int(window))
 
 
 def tiny(seed: int = 1000) -> Workload:
@@ -296,12 +310,22 @@ def make_copy(name: str, seed: int | None = None) -> CopyWorkload:
     return fn() if seed is None else fn(seed)
 
 
+def sliding_window(seed: int = 1007, num_seqs: int = 16, window: int = 4096) -> Workload:
+    """A Mistral-7B-shaped decode layer with a sliding window (32 q heads, 8 kv heads,
+    head_dim 128, window 4096): contexts U[8192, 32768], so every sequence reads the last
+    4096 tokens of a longer context; the blocks before the window are the null block."""
+    rng = np.random.default_rng(seed + 7919)
+    ctx = rng.integers(8192, 32768, size=num_seqs, endpoint=True)
+    return build_workload("sliding_window", seed, ctx, 1, 32, 8, 128, window=window)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "llama8b": llama8b,
     "llama70b_long": llama70b_long,
     "prefix_sharing": prefix_sharing,
     "spec_verify": spec_verify,
+    "sliding_window": sliding_window,
 }
 
 

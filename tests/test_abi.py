@@ -188,6 +188,8 @@ def test_plan_heuristic_host_logic(pa):
     {"share_prefix": True}, {"share_prefix": True, "schedule": 2}, {"split_blocks": 3},
     {"path": 3, "split_blocks": 2}, {"share_prefix": True, "split_blocks": 5},
     {"path": 3, "share_prefix": True},
+    {"sliding_window": 64}, {"sliding_window": 64, "path": 1}, {"sliding_window": 17, "split_blocks": 2},
+    {"sliding_window": 5000},
 ])
 def test_every_plan_passes_decode_validation(pa, hints):
     """A plan from pa_decode_plan is accepted by pa_decode's own checks (on a machine
@@ -199,3 +201,23 @@ def test_every_plan_passes_decode_validation(pa, hints):
     st = _decode_raw(lib, B=B, q=q, hq=hq, hkv=hkv, d=d, mb=mb, nb=400, plan=ctypes.byref(plan),
                      ws=1 << 20, ws_bytes=need)
     assert st not in (pa.PA_ERR_INVALID_ARG, pa.PA_ERR_UNSUPPORTED, pa.PA_ERR_WORKSPACE), (plan, st)
+
+
+def test_window_plans_on_the_host(pa):
+    """Sliding-window plans: grid schedule only, splits over the window's span of blocks;
+    the other kernels and prefix sharing are refused before any device query."""
+    lib = pa.raw_library()
+    plan = pa.pa_plan_t()
+    for hints in ((3, 0, 0, 0, 64), (0, 2, 0, 0, 64), (2, 0, 0, 1, 64)):
+        h = pa.pa_plan_hints_t(*hints)
+        assert lib.pa_decode_plan(4, 1, 32, 8, 128, 64, ctypes.byref(h), ctypes.byref(plan)) == \
+            pa.PA_ERR_UNSUPPORTED, hints
+    h = pa.pa_plan_hints_t(0, 0, 0, 0, -1)
+    assert lib.pa_decode_plan(4, 1, 32, 8, 128, 64, ctypes.byref(h), ctypes.byref(plan)) == pa.PA_ERR_INVALID_ARG
+    # 24 rows at head_dim 128 would take tcgen05; with a window the tiles take it, on the grid
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, sliding_window=4096)
+    assert (p.path, p.schedule, p.sliding_window) == (pa.PA_PATH_TILE, pa.PA_SCHEDULE_GRID, 4096)
+    span = -(-(4096 + 6 - 1) // 16) + 1
+    assert p.split_blocks <= span and p.num_splits == -(-span // p.split_blocks)
+    p = pa.pa_decode_plan(4, 1, 32, 8, 128, 64, sliding_window=100000)   # wider than the table
+    assert p.num_splits == -(-64 // p.split_blocks)
