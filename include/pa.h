@@ -37,9 +37,9 @@
  *                      j*block_size + block_size - 1 of the sequence
  *       context_lens   int32 [num_seqs]; tokens of the sequence INCLUDING its
  *                      q_per_seq new ones (already written by pa_reshape_and_cache)
- *   - Query token i of a sequence sits at position context_len - q_per_seq + i and
- *     attends to positions 0 .. context_len - q_per_seq + i. Query head h reads kv
- *     head h / (num_q_heads / num_kv_heads).
+ *   - Query token i of a sequence sits at position pos = context_len - q_per_seq + i and
+ *     attends to positions 0 .. pos (pos - W + 1 .. pos under a plan's sliding window W).
+ *     Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported: block_size 16, head_dim 64 or 128, num_q_heads % num_kv_heads == 0,
  *     1 <= q_per_seq <= 16. Anything else returns PA_ERR_UNSUPPORTED before any
  *     launch. There is no CPU fallback.
@@ -47,7 +47,8 @@
  *     with nothing enqueued. Device-resident values (slots, block ids, context
  *     lengths) are preconditions: 0 <= slot < num_blocks*block_size or slot < 0,
  *     0 <= block id < num_blocks for the first ceil(context_len/block_size)
- *     entries of each table row, q_per_seq <= context_len <=
+ *     entries of each table row (with a sliding window, for the entries from the
+ *     window's first block on: the ones before it are never read), q_per_seq <= context_len <=
  *     max_blocks_per_seq*block_size. pa_validate checks them on request. A launch
  *     failure returns PA_ERR_CUDA. Kernels never trap: a bounded wait that times
  *     out records a code that pa_get_device_error returns.
