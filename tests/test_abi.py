@@ -6,6 +6,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -221,3 +222,17 @@ def test_window_plans_on_the_host(pa):
     assert p.split_blocks <= span and p.num_splits == -(-span // p.split_blocks)
     p = pa.pa_decode_plan(4, 1, 32, 8, 128, 64, sliding_window=100000)   # wider than the table
     assert p.num_splits == -(-64 // p.split_blocks)
+
+
+def test_window_plan_covers_every_visible_block(pa):
+    """The grid kernel walks a sequence's blocks from the window's first block,
+    floor(max(0, ctx - q - W + 1) / 16), in num_splits pieces of split_blocks: the plan must
+    leave room for every block up to ceil(ctx / 16) at every context the table allows."""
+    for W in (1, 5, 15, 16, 17, 31, 100, 1000, 4096):
+        for q in (1, 2, 6, 16):
+            for mb in (1, 3, 64, 257, 2048):
+                for forced in (0, 1, 3):
+                    p = pa.pa_decode_plan(4, q, 8, 2, 128, mb, split_blocks=forced, sliding_window=W)
+                    ctx = np.arange(q, mb * 16 + 1)
+                    need = -(-ctx // 16) - np.maximum(0, ctx - q - W + 1) // 16
+                    assert int(need.max()) <= p.num_splits * p.split_blocks, (W, q, mb, forced, p)
