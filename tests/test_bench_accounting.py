@@ -60,3 +60,18 @@ def test_copy_traffic_keyed_by_the_copy_sources_only():
     assert set(bench.DECODE_SOURCES).isdisjoint(bench.COPY_SOURCES)
     csrc = os.path.join(os.path.dirname(bench.__file__), "paged_kv_cache_399_b200", "csrc")
     assert set(bench.DECODE_SOURCES) | set(bench.COPY_SOURCES) == set(os.listdir(csrc))
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    """bench.py --impl reference (the fp64 oracle on host cores) prints one JSON line with
+    the contract's keys, for a decode workload and for a copy workload."""
+    for wl, steps in (("tiny", 2), ("cow_fork", 1)):
+        assert bench.main(["--impl", "reference", "--workload", wl, "--steps", str(steps), "--warmup", "3"]) == 0
+        lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+        assert len(lines) == 1
+        d = json.loads(lines[0])
+        for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                    "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "impl"):
+            assert key in d, (wl, key)
+        assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+        assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
