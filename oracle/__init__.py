@@ -70,6 +70,16 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode_rows_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                               _I32, _I32, _I32, _I64, ctypes.c_double, _P, _I64,
                                               _I32, _I32]
+    lib.oracle_fp8_encode.restype = None
+    lib.oracle_fp8_encode.argtypes = [_P, _P, _I64]
+    lib.oracle_fp8_decode.restype = None
+    lib.oracle_fp8_decode.argtypes = [_P, _P, _I64]
+    lib.oracle_reshape_and_cache_fp8.restype = _I32
+    lib.oracle_reshape_and_cache_fp8.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _I32, _I64, _I32,
+                                                 ctypes.c_float, ctypes.c_float]
+    lib.oracle_decode_fp8.restype = _I32
+    lib.oracle_decode_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
+                                      ctypes.c_double, ctypes.c_double, ctypes.c_double, _I32, _I32]
     lib.oracle_copy_blocks.restype = _I32
     lib.oracle_copy_blocks.argtypes = [_P, _P, _I64, _I64, _P, _I64]
     lib.oracle_threads_used.restype = _I32
@@ -180,6 +190,56 @@ class Oracle:
                                                 num_threads)
         if st != 0:
             raise ValueError(f"oracle_decode_rows status {st}")
+        return out
+
+    def fp8_encode(self, x) -> np.ndarray:
+        """E4M3 codes (uint8) of fp32 values (ties to even, saturating at +-448)."""
+        xf = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+        out = np.empty(xf.shape, dtype=np.uint8)
+        self.lib.oracle_fp8_encode(_ptr(xf), _ptr(out), xf.size)
+        return out
+
+    def fp8_decode(self, codes) -> np.ndarray:
+        """fp64 values of E4M3 codes (NaN for S.1111.111)."""
+        c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+        out = np.empty(c.shape, dtype=np.float64)
+        self.lib.oracle_fp8_decode(_ptr(c), _ptr(out), c.size)
+        return out
+
+    def reshape_and_cache_fp8(self, key, value, key_cache, value_cache, slot_mapping,
+                              k_scale: float, v_scale: float):
+        """FP8 cache write. key/value bf16 [T, H_kv, D]; caches uint8 [NB, bs, H_kv, D].
+        Returns new (key_cache, value_cache) uint8 arrays; inputs untouched."""
+        k = _u16(key)
+        v = _u16(value)
+        kc = np.ascontiguousarray(np.asarray(key_cache, dtype=np.uint8)).copy()
+        vc = np.ascontiguousarray(np.asarray(value_cache, dtype=np.uint8)).copy()
+        slots = np.ascontiguousarray(np.asarray(slot_mapping, dtype=np.int64))
+        T, H, D = k.shape
+        NB, BS = kc.shape[0], kc.shape[1]
+        st = self.lib.oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), H * D, H * D, _ptr(kc), _ptr(vc),
+                                                   _ptr(slots), T, H, D, NB, BS, float(k_scale), float(v_scale))
+        if st != 0:
+            raise ValueError(f"oracle_reshape_and_cache_fp8 status {st}")
+        return kc, vc
+
+    def decode_fp8(self, query, key_cache, value_cache, block_tables, context_lens, q_per_seq: int,
+                   scale: float, k_scale: float, v_scale: float, window: int = 0,
+                   num_threads: int = 0) -> np.ndarray:
+        """fp64 output [B, q, H_q, D] over FP8 pools (uint8 [NB, bs, H_kv, D]) and their scales."""
+        q = _u16(query)
+        kc = np.ascontiguousarray(np.asarray(key_cache, dtype=np.uint8))
+        vc = np.ascontiguousarray(np.asarray(value_cache, dtype=np.uint8))
+        bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+        cl = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+        B, QS, HQ, D = q.shape
+        NB, BS, HKV = kc.shape[0], kc.shape[1], kc.shape[2]
+        out = np.zeros((B, QS, HQ, D), dtype=np.float64)
+        st = self.lib.oracle_decode_fp8(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(bt), _ptr(cl), B, QS, HQ,
+                                        HKV, D, BS, bt.shape[1], NB, float(scale), float(k_scale), float(v_scale),
+                                        int(window), num_threads)
+        if st != 0:
+            raise ValueError(f"oracle_decode_fp8 status {st}")
         return out
 
     def copy_blocks(self, key_cache, value_cache, block_mapping):

@@ -36,6 +36,9 @@
 //     Table entries wholly before every row's window are never read ([VS] §5.5 points
 //     them at the null block 0).
 //   * bf16 is widened to fp64 exactly (bit pattern << 16 is the fp32 value).
+//   * FP8 KV cache ([VS] §4.2 names --kv-cache-dtype fp8 only): the E4M3 format, one fp32
+//     scale per pool passed by the caller; stored code = nearest E4M3 (ties to even,
+//     saturating at +-448) of the fp32 quotient x / scale; read value = code's value * scale.
 //
 // Parity pins for every function here live in the CPU test-suite (brute force
 // contiguous attention, a library attention routine, closed forms, invariants,
@@ -88,7 +91,72 @@ struct Shape {
   int max_blocks_per_seq;
   int64_t num_blocks;
   int window;  // sliding window in tokens; 0 = none
+  // FP8 pools (E4M3 codes) and their per-pool scales; null: the bf16 pools
+  const uint8_t* k8 = nullptr;
+  const uint8_t* v8 = nullptr;
+  double k_scale = 1.0, v_scale = 1.0;
 };
+
+// ---- FP8 E4M3 ([VS] §4.2: an FP8 KV cache, --kv-cache-dtype fp8) ----
+// The 8-bit floating-point format E4M3: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+// bits; exponent field 0 holds the subnormals m * 2^-9; no infinities; S.1111.111 is NaN; the
+// largest finite value is 1.75 * 2^8 = 448.
+double fp8_e4m3_decode(uint8_t c) {
+  const int e = (c >> 3) & 0xF, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) {
+    v = std::nan("");
+  } else if (e == 0) {
+    v = std::ldexp(static_cast<double>(m), -9);
+  } else {
+#if ORACLE_MUTANT == 42
+    v = std::ldexp(1.0 + m / 8.0, e - 8);  // planted: exponent bias 8
+#else
+    v = std::ldexp(1.0 + m / 8.0, e - 7);
+#endif
+  }
+  return (c & 0x80) ? -v : v;
+}
+
+// Nearest E4M3 code of x, ties to the even code; finite values above 448 in magnitude and
+// infinities saturate to +-448; NaN gives 0x7F.
+uint8_t fp8_e4m3_encode(float x) {
+  if (std::isnan(x)) return 0x7F;
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(x));
+#if ORACLE_MUTANT == 43
+  if (a >= 448.0) return sign | 0x7F;  // planted: out-of-range values become NaN
+#else
+  if (a >= 448.0) return sign | 0x7E;
+#endif
+  // the grid spacing of a's binade: 2^-9 below the smallest normal 2^-6, else 2^(e-3)
+  int e2 = 0;
+  std::frexp(a, &e2);                   // a = f * 2^e2, f in [0.5, 1)
+  const int e = a < std::ldexp(1.0, -6) ? -6 : e2 - 1;   // a in [2^e, 2^(e+1))
+  const double spacing = std::ldexp(1.0, e - 3);
+  const double units = a / spacing;     // exact: a power-of-two scaling
+  double q = std::floor(units);
+#if ORACLE_MUTANT == 41
+  (void)0;  // planted: truncation instead of rounding to nearest
+#else
+  const double frac = units - q;
+  if (frac > 0.5 || (frac == 0.5 && std::fmod(q, 2.0) != 0.0)) q += 1.0;
+#endif
+  // q * 2^(e-3): subnormal (e = -6, q < 8), or 1.mmm * 2^e with q in [8, 16]
+  int code;
+  if (e == -6 && q < 8.0) {
+    code = static_cast<int>(q);
+  } else {
+    int ee = e, mq = static_cast<int>(q);
+    if (mq == 16) {
+      mq = 8;
+      ++ee;
+    }
+    code = ((ee + 7) << 3) | (mq - 8);
+  }
+  if (code >= 0x7F) code = 0x7E;  // not reached for a < 448; kept as a guard
+  return static_cast<uint8_t>(sign | code);
+}
 
 // Gather the keys and values of one (sequence, kv head) into contiguous fp64
 // arrays [ctx][head_dim], walking the block table as [DS] §3.3 and [VS] §3.2 do:
@@ -113,8 +181,13 @@ bool gather_kv(const uint16_t* key_cache, const uint16_t* value_cache,
     for (int d = 0; d < s.head_dim; ++d) {
       int64_t idx = pool_index(phys, offset, kv_head, d, s.block_size,
                                s.num_kv_heads, s.head_dim);
-      k_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(key_cache[idx]);
-      v_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(value_cache[idx]);
+      if (s.k8) {  // FP8 pools: the code's value times the pool's scale (exact in fp64)
+        k_out[static_cast<size_t>(i) * s.head_dim + d] = fp8_e4m3_decode(s.k8[idx]) * s.k_scale;
+        v_out[static_cast<size_t>(i) * s.head_dim + d] = fp8_e4m3_decode(s.v8[idx]) * s.v_scale;
+      } else {
+        k_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(key_cache[idx]);
+        v_out[static_cast<size_t>(i) * s.head_dim + d] = bf16_to_f64(value_cache[idx]);
+      }
     }
   }
   return true;
@@ -441,6 +514,74 @@ int oracle_decode_rows(double* out, const uint16_t* query, const uint16_t* key_c
                                    context_lens, num_seqs, q_per_seq, num_q_heads,
                                    num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                                    num_blocks, scale, rows, n_rows, 0, num_threads);
+}
+
+// FP8 E4M3 codes of n fp32 values, and the values of n codes (for the format's pins).
+void oracle_fp8_encode(const float* x, uint8_t* codes, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = fp8_e4m3_encode(x[i]);
+}
+void oracle_fp8_decode(const uint8_t* codes, double* x, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) x[i] = fp8_e4m3_decode(codes[i]);
+}
+
+// Cache write into FP8 pools ([VS] §4.2). Each bf16 element x of key[t] is stored as the
+// E4M3 code of the fp32 quotient x / k_scale (value: / v_scale), at the same pool position as
+// oracle_reshape_and_cache; every other pool byte is left untouched. Returns 0, or 1 for an
+// out-of-range slot.
+int oracle_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value, int64_t key_stride,
+                                 int64_t value_stride, uint8_t* key_cache, uint8_t* value_cache,
+                                 const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                                 int head_dim, int64_t num_blocks, int block_size, float k_scale,
+                                 float v_scale) {
+  int status = 0;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    const int64_t block = slot / block_size, offset = slot % block_size;
+    if (block >= num_blocks) {
+      status = 1;
+      continue;
+    }
+    for (int h = 0; h < num_kv_heads; ++h) {
+      for (int d = 0; d < head_dim; ++d) {
+        const int64_t dst = pool_index(block, offset, h, d, block_size, num_kv_heads, head_dim);
+        const float k = static_cast<float>(bf16_to_f64(key[t * key_stride + static_cast<int64_t>(h) * head_dim + d]));
+        const float v =
+            static_cast<float>(bf16_to_f64(value[t * value_stride + static_cast<int64_t>(h) * head_dim + d]));
+        key_cache[dst] = fp8_e4m3_encode(k / k_scale);
+        value_cache[dst] = fp8_e4m3_encode(v / v_scale);
+      }
+    }
+  }
+  return status;
+}
+
+// Paged decode over FP8 pools: oracle_decode_window's definition with every key and value
+// element read as its E4M3 code's value times the pool's scale.
+int oracle_decode_fp8(double* out, const uint16_t* query, const uint8_t* key_cache,
+                      const uint8_t* value_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int num_seqs, int q_per_seq, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                      int64_t num_blocks, double scale, double k_scale, double v_scale, int window,
+                      int num_threads) {
+  Shape s{num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, block_size,
+          max_blocks_per_seq, num_blocks, window};
+  s.k8 = key_cache;
+  s.v8 = value_cache;
+  s.k_scale = k_scale;
+  s.v_scale = v_scale;
+  const int64_t n_rows = static_cast<int64_t>(num_seqs) * q_per_seq * num_q_heads;
+  std::vector<int32_t> rows(3 * n_rows);
+  int64_t r = 0;
+  for (int b = 0; b < num_seqs; ++b)
+    for (int i = 0; i < q_per_seq; ++i)
+      for (int h = 0; h < num_q_heads; ++h, ++r) {
+        rows[3 * r] = b;
+        rows[3 * r + 1] = i;
+        rows[3 * r + 2] = h;
+      }
+  return decode_rows_impl(out, query, nullptr, nullptr, block_tables, context_lens, s, scale, rows.data(),
+                          n_rows, num_threads);
 }
 
 // Threads the last decode call ran on.

@@ -11,7 +11,9 @@ when the oracle disagrees with:
   * the copy-on-write rule of parallel sampling (a fork's writer copies the shared
     last block and writes there; the other candidates still read the original),
   * the sliding window (the most recent W tokens; entries before it may name the null
-    block 0 and are never read).
+    block 0 and are never read),
+  * the FP8 (E4M3) KV cache: the format's fixed values, torch's float8_e4m3fn conversion,
+    the cache write's codes and attention over the dequantized pools.
 The same checks run against deliberately broken builds of the oracle
 (tests/test_oracle_mutants.py) to show that each planted mistake is caught.
 """
@@ -521,6 +523,86 @@ def check_sliding_window(oracle):
         assert np.allclose(o, q1.V[0][30 - n:30, 0].mean(0), atol=1e-12), f"visible keys for W={W}"
 
 
+def _torch_fp8_codes(x32: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(torch.float8_e4m3fn).view(
+        torch.uint8).numpy()
+
+
+def _torch_fp8_values(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def check_fp8_format(oracle):
+    """golden/fp8_e4m3.json (values fixed by the format's definition), torch.float8_e4m3fn (a
+    library conversion) on every code and on a dense sweep of [-448, 448] with every tie, and
+    the round trip of every code."""
+    g = json.load(open(os.path.join(GOLDEN, "fp8_e4m3.json")))
+    for table in ("codes", "saturate"):
+        xs = np.array([float(k) for k in g[table]], dtype=np.float32)
+        want = np.array(list(g[table].values()), dtype=np.uint8)
+        got = oracle.fp8_encode(xs)
+        assert np.array_equal(got, want), (table, xs[got != want], got[got != want])
+    for k, c in g["codes"].items():
+        assert oracle.fp8_decode([c])[0] == float(k) and math.copysign(1, oracle.fp8_decode([c])[0]) == \
+            math.copysign(1, float(k)), k
+    codes = np.arange(256, dtype=np.uint8)
+    mine, ref = oracle.fp8_decode(codes), _torch_fp8_values(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan) and np.array_equal(mine[~nan], ref[~nan]), "decode vs torch"
+    vals = np.unique(ref[~nan])
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([np.arange(-448 * 1024, 448 * 1024 + 1) / 1024.0, mids, -mids,
+                        np.random.default_rng(7).uniform(-448, 448, 100000)]).astype(np.float32)
+    bad = oracle.fp8_encode(x) != _torch_fp8_codes(x)
+    assert not bad.any(), ("encode vs torch", x[bad][:5])
+    finite = codes[~nan]
+    assert np.array_equal(oracle.fp8_encode(oracle.fp8_decode(finite).astype(np.float32)), finite), "round trip"
+
+
+def check_fp8_cache_and_attention(oracle):
+    """The FP8 cache write stores the codes torch gives for the fp32 quotients x / scale, and
+    FP8 attention equals brute force over the contiguous K/V dequantized with torch."""
+    rng = np.random.default_rng(111)
+    bs, hkv, hq, d, q = 16, 2, 4, 16, 2
+    ctxs = [20, 37, 5]
+    ks, vs = 0.05, 0.02
+    nb = sum(-(-c // bs) for c in ctxs) + 3
+    perm = rng.permutation(nb)
+    tables = np.zeros((len(ctxs), max(-(-c // bs) for c in ctxs)), dtype=np.int32)
+    cur = 0
+    for b, c in enumerate(ctxs):
+        n = -(-c // bs)
+        tables[b, :n] = perm[cur:cur + n]
+        cur += n
+    finite = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    kc0 = rng.choice(finite, size=(nb, bs, hkv, d)).astype(np.uint8)
+    vc0 = rng.choice(finite, size=(nb, bs, hkv, d)).astype(np.uint8)
+    # the step's new tokens: the last q positions of each sequence
+    slots = np.array([int(tables[b, p // bs]) * bs + p % bs for b, c in enumerate(ctxs)
+                      for p in range(c - q, c)], dtype=np.int64)
+    key = _bf16_round(rng.standard_normal((len(slots), hkv, d)) * 3)
+    val = _bf16_round(rng.standard_normal((len(slots), hkv, d)) * 3)
+    kc, vc = oracle.reshape_and_cache_fp8(_bits(key), _bits(val), kc0, vc0, slots, ks, vs)
+    written = np.zeros((nb, bs), dtype=bool)
+    for t, sl in enumerate(slots):
+        blk, off = divmod(int(sl), bs)
+        assert np.array_equal(kc[blk, off], _torch_fp8_codes(key[t].astype(np.float32) / np.float32(ks))), t
+        assert np.array_equal(vc[blk, off], _torch_fp8_codes(val[t].astype(np.float32) / np.float32(vs))), t
+        written[blk, off] = True
+    assert np.array_equal(kc[~written], kc0[~written]) and np.array_equal(vc[~written], vc0[~written])
+    Q = _bf16_round(rng.standard_normal((len(ctxs), q, hq, d)))
+    scale = 1.0 / math.sqrt(d)
+    out = oracle.decode_fp8(_bits(Q), kc, vc, tables, np.array(ctxs, dtype=np.int32), q, scale, ks, vs)
+    kd, vd = _torch_fp8_values(kc) * ks, _torch_fp8_values(vc) * vs
+    for b, c in enumerate(ctxs):
+        K = np.stack([kd[tables[b, t // bs], t % bs] for t in range(c)])
+        V = np.stack([vd[tables[b, t // bs], t % bs] for t in range(c)])
+        for i in range(q):
+            last = c - q + i
+            _close(out[b, i], _attend_rows(Q[b, i], K[:last + 1], V[:last + 1], scale), what=f"fp8 seq {b} row {i}")
+
+
 ALL_CHECKS = [
     check_bf16_widening,
     check_block_counts_golden,
@@ -538,4 +620,6 @@ ALL_CHECKS = [
     check_cache_write,
     check_copy_on_write,
     check_sliding_window,
+    check_fp8_format,
+    check_fp8_cache_and_attention,
 ]

@@ -22,6 +22,9 @@ MUTANTS = {
     11: "bf16 widened with the wrong shift",
     12: "pool laid out head-major inside a block",
     13: "sliding window one key too long",
+    41: "FP8 encode truncates instead of rounding to nearest",
+    42: "FP8 exponent bias 8",
+    43: "FP8 out-of-range values become NaN instead of saturating",
     31: "block copy leaves the value pool out",
     32: "block copy leaves the block's last token behind",
     33: "block copy with source and destination swapped",
