@@ -111,6 +111,7 @@ def decode_flops(w) -> int:
 DECODE_SOURCES = ("pa_api.cpp", "pa_device.cuh", "pa_internal.h", "pa_kernels.cu",
                   "pa_static_scratch.cu", "pa_tcgen05.cuh")
 COPY_SOURCES = ("pa_copy.cu",)
+FP8_SOURCES = ("pa_fp8.cu",)   # the FP8 cache write (no timed workload yet)
 
 
 def source_hash(names=DECODE_SOURCES) -> str:

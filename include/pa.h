@@ -166,6 +166,22 @@ PA_API pa_status_t pa_reshape_and_cache(const void* key, const void* value,
                                  int64_t num_blocks, int32_t block_size,
                                  pa_stream_t stream);
 
+/* FP8 KV cache write (vLLM study notes §4.2, --kv-cache-dtype fp8). The pools hold E4M3
+ * codes (uint8 [num_blocks][block_size][num_kv_heads][head_dim]); each bf16 element x of
+ * key[t] (value[t]) is stored at the slot pa_reshape_and_cache would use as the E4M3 code of
+ * the fp32 quotient x / k_scale (x / v_scale): round to nearest, ties to even, saturating at
+ * +-448 (no infinities in E4M3). k_scale, v_scale: finite, > 0, one per pool, chosen by the
+ * caller. Same layouts, strides, alignment, slot and error rules as pa_reshape_and_cache;
+ * num_kv_heads*head_dim must be a multiple of 16. The decode over FP8 pools is not built yet:
+ * this call writes the codes that such a decode (and the oracle) read back as code * scale. */
+PA_API pa_status_t pa_reshape_and_cache_fp8(const void* key, const void* value,
+                                     int64_t key_token_stride, int64_t value_token_stride,
+                                     void* key_cache, void* value_cache,
+                                     const int64_t* slot_mapping, int64_t num_tokens,
+                                     int32_t num_kv_heads, int32_t head_dim,
+                                     int64_t num_blocks, int32_t block_size, float k_scale,
+                                     float v_scale, pa_stream_t stream);
+
 /* Choose a plan from host-known shape values only (no device read). hints may be
  * NULL. The heuristic reads the SM count of the current device and the occupancy of
  * the chosen kernel. */

@@ -35,7 +35,8 @@ PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
-            "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_status_string", "pa_version"]
+            "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_status_string",
+            "pa_version"]
 
 PA_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -74,6 +75,9 @@ _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
 _I64 = ctypes.c_int64
 
+_lib.pa_reshape_and_cache_fp8.restype = _I32
+_lib.pa_reshape_and_cache_fp8.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I64, _I32, _I32, _I64, _I32,
+                                          ctypes.c_float, ctypes.c_float, _P]
 _lib.pa_copy_blocks.restype = _I32
 _lib.pa_copy_blocks.argtypes = [_P, _P, _I64, _I32, _I32, _I32, _P, _I64, _P]
 _lib.pa_reshape_and_cache.restype = _I32
@@ -169,6 +173,24 @@ def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor, block_map
     st = _lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), NB, H, D, BS,
                              m.ctypes.data if m.shape[0] else None, m.shape[0], _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, slot_mapping: torch.Tensor, k_scale: float,
+                             v_scale: float, stream=None) -> None:
+    """FP8 cache write. key/value [T, H_kv, D] bf16 (token stride may exceed H_kv*D);
+    caches [NB, 16, H_kv, D] uint8 (E4M3 codes); slot_mapping [T] int64; one scale per pool."""
+    assert key.dtype == value.dtype == torch.bfloat16
+    assert key_cache.dtype == value_cache.dtype == torch.uint8
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.is_contiguous()
+    T, H, D = key.shape
+    assert key.stride(2) == 1 and key.stride(1) == D and value.stride(2) == 1 and value.stride(1) == D
+    assert key_cache.is_contiguous() and value_cache.is_contiguous()
+    NB, BS = key_cache.shape[0], key_cache.shape[1]
+    st = _lib.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
+                                       _ptr(value_cache), _ptr(slot_mapping), T, H, D, NB, BS, float(k_scale),
+                                       float(v_scale), _stream(stream))
+    _check(st, "pa_reshape_and_cache_fp8")
 
 
 def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,

@@ -236,3 +236,24 @@ def test_window_plan_covers_every_visible_block(pa):
                     ctx = np.arange(q, mb * 16 + 1)
                     need = -(-ctx // 16) - np.maximum(0, ctx - q - W + 1) // 16
                     assert int(need.max()) <= p.num_splits * p.split_blocks, (W, q, mb, forced, p)
+
+
+def test_fp8_cache_write_rejects_bad_arguments_before_launch(pa):
+    lib = pa.raw_library()
+
+    def call(**kw):
+        a = dict(k=1024, v=2048, ks=128, vs=128, kc=4096, vc=8192, slots=16384, T=4, hkv=2, d=64,
+                 nb=8, bs=16, kscale=0.5, vscale=0.5)
+        a.update(kw)
+        return lib.pa_reshape_and_cache_fp8(a["k"], a["v"], a["ks"], a["vs"], a["kc"], a["vc"], a["slots"],
+                                            a["T"], a["hkv"], a["d"], a["nb"], a["bs"], a["kscale"], a["vscale"],
+                                            None)
+    assert call(k=None) == pa.PA_ERR_INVALID_ARG
+    assert call(kc=4096 + 8) == pa.PA_ERR_INVALID_ARG
+    assert call(ks=100) == pa.PA_ERR_INVALID_ARG
+    assert call(kscale=0.0) == pa.PA_ERR_INVALID_ARG
+    assert call(vscale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert call(kscale=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
+    assert call(hkv=1, d=8) == pa.PA_ERR_UNSUPPORTED   # a row of 8 elements: not a multiple of 16
+    assert call(T=0, k=None) == pa.PA_OK

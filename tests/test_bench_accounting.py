@@ -59,7 +59,7 @@ def test_copy_traffic_keyed_by_the_copy_sources_only():
     assert bench.source_hash() != bench.source_hash(bench.COPY_SOURCES)
     assert set(bench.DECODE_SOURCES).isdisjoint(bench.COPY_SOURCES)
     csrc = os.path.join(os.path.dirname(bench.__file__), "paged_kv_cache_399_b200", "csrc")
-    assert set(bench.DECODE_SOURCES) | set(bench.COPY_SOURCES) == set(os.listdir(csrc))
+    assert set(bench.DECODE_SOURCES) | set(bench.COPY_SOURCES) | set(bench.FP8_SOURCES) == set(os.listdir(csrc))
 
 
 def test_reference_arm_prints_the_contract_line(capsys):
