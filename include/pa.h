@@ -13,7 +13,9 @@
  *                         head groups and causal masking of multi-token
  *                         (speculative-verify) queries (vLLM study notes §1.1.1);
  *   pa_copy_blocks        the copy-on-write block copy behind shared blocks
- *                         (vLLM study notes §3.2.2).
+ *                         (vLLM study notes §3.2.2);
+ *   pa_reshape_and_cache_fp8  the cache write into FP8 (E4M3) pools with one scale per
+ *                         pool (vLLM study notes §4.2).
  *
  * Conventions shared by every call
  *   - All data pointers are DEVICE pointers on the current CUDA device (the one
