@@ -515,6 +515,20 @@ def check_sliding_window(oracle):
         tables[b, :first // p.bs] = null
     got = p.run(oracle, pool_k=pk, pool_v=pv, tables=tables, window=W)
     assert np.array_equal(got, ref), "an entry before the window was read"
+    # a library routine: torch scaled_dot_product_attention in fp64 with the window as a mask
+    g_ = p.hq // p.hkv
+    for W in (3, 16, 40):
+        got = p.run(oracle, window=W)
+        for b in range(p.B):
+            c = p.ctxs[b]
+            qb = torch.from_numpy(p.Q[b]).permute(1, 0, 2)[None]
+            kb = torch.from_numpy(p.K[b]).permute(1, 0, 2).repeat_interleave(g_, 0)[None]
+            vb = torch.from_numpy(p.V[b]).permute(1, 0, 2).repeat_interleave(g_, 0)[None]
+            pos = torch.arange(c)[None, :]
+            qpos = (c - p.q + torch.arange(p.q))[:, None]
+            mask = (pos <= qpos) & (pos > qpos - W)
+            o = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=p.scale)
+            _close(got[b], o[0].permute(1, 0, 2).numpy(), tol=1e-10, what=f"window {W} vs SDPA, seq {b}")
     # visible key counts: min(W, pos + 1), through weights on a one-hot value pattern
     q1 = Problem(seed=103, ctxs=[30], q=1, hq=1, hkv=1, d=16, same_keys=True)
     for W in (1, 5, 30, 40):
