@@ -615,6 +615,14 @@ def check_fp8_cache_and_attention(oracle):
         for i in range(q):
             last = c - q + i
             _close(out[b, i], _attend_rows(Q[b, i], K[:last + 1], V[:last + 1], scale), what=f"fp8 seq {b} row {i}")
+        # the same against torch scaled_dot_product_attention (fp64) on the dequantized K/V
+        g_ = hq // hkv
+        qb = torch.from_numpy(Q[b]).permute(1, 0, 2)[None]
+        kb = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(g_, 0)[None]
+        vb = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(g_, 0)[None]
+        mask = torch.arange(c)[None, :] <= (c - q + torch.arange(q))[:, None]
+        o = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=scale)
+        _close(out[b], o[0].permute(1, 0, 2).numpy(), tol=1e-10, what=f"fp8 seq {b} vs SDPA")
 
 
 ALL_CHECKS = [
