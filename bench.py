@@ -227,6 +227,148 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
+# The decode configurations every default run also times on the same box, beside the
+# headline workload (µs/call per config is half of the metric).
+PER_CONFIG = ("tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify", "sliding_window")
+# the 75 % bar of the measured copy bandwidth holds on the three bandwidth-scale configs
+BAR_CONFIGS = ("llama8b", "llama70b_long", "prefix_sharing")
+
+
+def _device_inputs(w, dev):
+    """The step's per-call inputs in one device buffer (and one pinned host buffer for the
+    end-to-end leg, so a step's host->device traffic is a single copy), plus the pools."""
+    import torch
+    parts = [("query", w.query), ("key", w.key), ("value", w.value),
+             ("slots", torch.from_numpy(w.slot_mapping)), ("tables", torch.from_numpy(w.block_tables)),
+             ("ctx", torch.from_numpy(w.context_lens))]
+    offsets, total = {}, 0
+    for name, t in parts:
+        offsets[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+    views = {}
+    for name, t in parts:
+        n = t.numel() * t.element_size()
+        h_in[offsets[name]:offsets[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        views[name] = d_in[offsets[name]:offsets[name] + n].view(t.dtype).view(t.shape)
+    d_in.copy_(h_in)
+    views["h_in"], views["d_in"], views["in_bytes"] = h_in, d_in, total
+    views["key_cache"] = w.key_cache.to(dev)
+    views["value_cache"] = w.value_cache.to(dev)
+    views["out"] = torch.empty_like(views["query"])
+    return views
+
+
+def _plan_for(pa, w, args):
+    # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
+    share = bool(w.shared_groups) and not args.no_share_prefix
+    return pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                             w.max_blocks_per_seq, share_prefix=share, sliding_window=w.window,
+                             path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
+                             split_blocks=args.split_blocks,
+                             schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
+
+
+def _ncu_traffic(name):
+    rec = NCU_TRAFFIC.get(name)
+    if rec and rec.get("source_hash") == source_hash():
+        return rec["bytes_per_launch"]
+    return None
+
+
+def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
+    """Mean CUDA-event time of `calls` pa_decode calls (each after the step's cache write,
+    events on the launching stream around the decode only), in ms; and the same calls
+    without host overhead: one CUDA graph of 20 back-to-back calls, replayed (µs per call,
+    None when capture is unavailable)."""
+    import torch
+    barrier()
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(calls)]
+    for a, b in pairs:
+        pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
+                                stream=stream)
+        a.record(stream)
+        pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                     w.q_per_seq, w.scale, plan=plan, workspace=ws, stream=stream)
+        b.record(stream)
+    barrier()
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+    graph_us = None
+    try:
+        per_graph, reps = 20, max(1, calls // 20)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(per_graph):
+                pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                             w.q_per_seq, w.scale, plan=plan, workspace=ws)
+        graph.replay()
+        barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        g1.record(stream)
+        barrier()
+        graph_us = g0.elapsed_time(g1) * 1e3 / (reps * per_graph)
+        del graph
+    except Exception as exc:  # capture is a measurement aid: report why it is missing
+        print(f"graph timing unavailable: {exc}", file=sys.stderr)
+    return decode_ms, graph_us
+
+
+def measure_config(name, args, dev, stream, peaks):
+    """One decode configuration on this GPU: µs per pa_decode call (CUDA events, and
+    graph-replayed), GB/s of its algorithmic bytes, the fraction of the measured copy
+    bandwidth, its plan, the ncu traffic (when taken on these sources) and the clocks."""
+    import torch
+    from paged_kv_cache_399_b200 import pa, workloads
+    w = workloads.make(name, seed=rank_seed(name, 0))
+    v = _device_inputs(w, dev)
+    plan = _plan_for(pa, w, args)
+    ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads,
+                                           w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(3, args.warmup)):
+        pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
+                                stream=stream)
+        pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                     w.q_per_seq, w.scale, plan=plan, workspace=ws, stream=stream)
+    barrier()
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        decode_ms, graph_us = _time_calls(pa, w, v, plan, ws, stream, args.config_calls, barrier)
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    dec_bytes = decode_bytes(w)
+    gbs = dec_bytes / (decode_ms * 1e-3) / 1e9
+    rec = {
+        "workload": w.describe(),
+        "calls": args.config_calls,
+        "decode_us_per_call": round(decode_ms * 1e3, 3),
+        "decode_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
+        "decode_alg_bytes": dec_bytes,
+        "decode_logical_bytes": decode_bytes(w, unique=False),
+        "decode_gbs": round(gbs, 2),
+        "frac": round(gbs / peaks["hbm_gbs"], 4),
+        "frac_graph": None if graph_us is None else round(dec_bytes / (graph_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+        "plan": plan.as_dict(),
+        "ncu_traffic": _ncu_traffic(name),
+        "clocks": sampler.summary(),
+    }
+    if name in BAR_CONFIGS:
+        rec["bar_us_at_75pct"] = round(dec_bytes / (0.75 * peaks["hbm_gbs"] * 1e9) * 1e6, 2)
+    del v, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -247,36 +389,12 @@ def run_gpu(args):
     w = workloads.make(args.workload, seed=rank_seed(args.workload, rank))
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream(dev)
-
-    # the step's per-call inputs live in one device buffer (and one pinned host buffer for
-    # the end-to-end leg), so a step's host->device traffic is a single copy
-    parts = [("query", w.query), ("key", w.key), ("value", w.value),
-             ("slots", torch.from_numpy(w.slot_mapping)), ("tables", torch.from_numpy(w.block_tables)),
-             ("ctx", torch.from_numpy(w.context_lens))]
-    offsets, total = {}, 0
-    for name, t in parts:
-        offsets[name] = total
-        total += (t.numel() * t.element_size() + 255) // 256 * 256
-    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
-    views = {}
-    for name, t in parts:
-        n = t.numel() * t.element_size()
-        h_in[offsets[name]:offsets[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
-        views[name] = d_in[offsets[name]:offsets[name] + n].view(t.dtype).view(t.shape)
-    d_in.copy_(h_in)
-    query, key, value = views["query"], views["key"], views["value"]
-    slots, tables, ctx = views["slots"], views["tables"], views["ctx"]
-    key_cache = w.key_cache.to(dev)
-    value_cache = w.value_cache.to(dev)
-    out = torch.empty_like(query)
-    # a caller that batches parallel samples of one prompt knows it: ask for prefix sharing
-    share = bool(w.shared_groups) and not args.no_share_prefix
-    plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                             w.max_blocks_per_seq, share_prefix=share, sliding_window=w.window,
-                             path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
-                             split_blocks=args.split_blocks,
-                             schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
+    v = _device_inputs(w, dev)
+    query, key, value = v["query"], v["key"], v["value"]
+    slots, tables, ctx = v["slots"], v["tables"], v["ctx"]
+    key_cache, value_cache, out = v["key_cache"], v["value_cache"], v["out"]
+    h_in, d_in, total = v["h_in"], v["d_in"], v["in_bytes"]
+    plan = _plan_for(pa, w, args)
     ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads,
                                            w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
@@ -295,7 +413,7 @@ def run_gpu(args):
     def max_over_ranks(x: float) -> float:
         return reduce_over_ranks(x, "max", dist if world > 1 else None, dev)
 
-    launches_per_step = 1 + (2 if (plan.schedule == pa.PA_SCHEDULE_PERSISTENT or plan.num_splits > 1) else 1)
+    launches_per_step = 1 + decode_launches(plan)
     step_bytes = decode_bytes(w) + cache_write_bytes(w)
     dec_bytes = decode_bytes(w)
 
@@ -317,49 +435,19 @@ def run_gpu(args):
         barrier()
         ms_total = max_over_ranks(e0.elapsed_time(e1))
 
-        # (2) per-kernel: events around each pa_decode launch of another K steps
-        barrier()
-        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                 for _ in range(args.steps)]
-        for a, b in pairs:
-            pa.pa_reshape_and_cache(key, value, key_cache, value_cache, slots, stream=stream)
-            a.record(stream)
-            pa.pa_decode(out, query, key_cache, value_cache, tables, ctx, w.q_per_seq, w.scale,
-                         plan=plan, workspace=ws, stream=stream)
-            b.record(stream)
-        barrier()
-        decode_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        # (2) per-kernel: events around each pa_decode launch of another K steps, and the
+        # same calls graph-replayed (for the small configs the events mostly time the
+        # Python call)
+        decode_ms, graph_us = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
         decode_ms = max_over_ranks(decode_ms)
-
-        # (2b) the same calls without host overhead: one CUDA graph of back-to-back pa_decode
-        # calls, replayed (for the small configs the events above mostly time the Python call)
-        graph_us = None
-        try:
-            calls, reps = 20, max(1, args.steps // 20)
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                for _ in range(calls):
-                    pa.pa_decode(out, query, key_cache, value_cache, tables, ctx, w.q_per_seq, w.scale,
-                                 plan=plan, workspace=ws)
-            graph.replay()
-            barrier()
-            g0 = torch.cuda.Event(enable_timing=True)
-            g1 = torch.cuda.Event(enable_timing=True)
-            g0.record(stream)
-            for _ in range(reps):
-                graph.replay()
-            g1.record(stream)
-            barrier()
-            graph_us = max_over_ranks(g0.elapsed_time(g1)) * 1e3 / (reps * calls)
-            del graph
-        except Exception as exc:  # capture is a measurement aid: report why it is missing
-            print(f"graph timing unavailable: {exc}", file=sys.stderr)
+        if graph_us is not None:
+            graph_us = max_over_ranks(graph_us)
 
         # (3) end to end: host (pinned) inputs in, output back to the host, every step
         h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         h2d = total
         d2h = h_out.numel() * h_out.element_size()
-        e2e_steps = max(1, args.steps // 4)
+        e2e_steps = args.steps
         barrier()
         f0 = torch.cuda.Event(enable_timing=True)
         f1 = torch.cuda.Event(enable_timing=True)
@@ -378,11 +466,16 @@ def run_gpu(args):
     e2e_gbs = aggregate_throughput(step_bytes, e2e_steps, e2e_ms, world)
     peaks = measured_peaks()
     achieved = dec_bytes / (decode_ms * 1e-3) / 1e9
-    traffic = None
-    rec = NCU_TRAFFIC.get(args.workload)
-    if rec and rec.get("source_hash") == source_hash():
-        traffic = rec["bytes_per_launch"]
+    traffic = _ncu_traffic(args.workload)
     clocks = sampler.summary()
+
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        del v, ws
+        torch.cuda.empty_cache()
+        per_config = {}
+        for name in PER_CONFIG:
+            per_config[name] = measure_config(name, args, dev, stream, peaks)
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if (world == 1 and not args.no_cpu_baseline) else None
@@ -413,8 +506,11 @@ def run_gpu(args):
                 "step_frac_of_measured_hbm": round(value_gbs / world / peaks["hbm_gbs"], 4),
                 "plan": plan.as_dict(),
                 "l2": "no flush: each step reads more bytes than the 126 MB L2 holds"
-                      if dec_bytes > 2 * 126e6 else "no flush: working set near L2 size (see DESIGN)",
+                      if dec_bytes > 2 * 126e6 else
+                      "no flush: the step's bytes are within twice the 126 MB L2, so later steps may "
+                      "find part of them in L2",
                 "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
+                "per_config": per_config,
             },
             "roofline": {
                 "bound": "hbm",
@@ -424,7 +520,7 @@ def run_gpu(args):
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic,
                 "peak_source": peaks["source"],
-                "kernel": "pa_decode (schedule pre-pass + decode kernel, or grid decode + merge)",
+                "kernel": "pa_decode (its kernels on the launching stream)",
             },
             "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -437,6 +533,16 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def decode_launches(plan) -> int:
+    """Kernel launches of one pa_decode call with this plan."""
+    from paged_kv_cache_399_b200 import pa
+    if plan.path == pa.PA_PATH_TCGEN05:
+        return 2 + (1 if plan.share_cap > 1 else 0)
+    if plan.schedule == pa.PA_SCHEDULE_PERSISTENT:
+        return 2
+    return (1 if plan.share_cap else 0) + 1 + (1 if (plan.num_splits > 1 or plan.share_cap) else 0)
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -765,6 +871,10 @@ def main(argv=None):
     ap.add_argument("--split-blocks", type=int, default=0, help="grid schedule split length (0 = heuristic)")
     ap.add_argument("--no-share-prefix", action="store_true",
                     help="do not ask pa_decode to read shared prefix blocks once per group")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the chosen workload (the default also times every decode config)")
+    ap.add_argument("--config-calls", type=int, default=200,
+                    help="pa_decode calls timed per config in config.per_config")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     args = ap.parse_args(argv)

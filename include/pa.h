@@ -239,8 +239,10 @@ PA_API pa_status_t pa_decode(void* out, const void* query, const void* key_cache
  *   rejected with PA_ERR_WORKSPACE before anything is launched (pass an explicit
  *   plan with longer splits, or use pa_decode).
  * - The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that first
- *   call before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the life of the
+ *   process; make that first call before any stream capture. Do not use this call
+ *   after cudaDeviceReset (or any teardown of the device's primary context) in the
+ *   same process: the array then lives at a new address that the cache does not see.
  * - All calls share the one array per device and it keeps the last call's contents;
  *   nothing in it needs to start at zero. Calls whose GPU work overlaps (unordered
  *   streams) race on it: keep them ordered on one stream. */

@@ -374,6 +374,18 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
 
 }  // namespace
 
+namespace pa {
+
+int check_decode_args(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq) {
+  const int st =
+      check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq);
+  if (st != PA_OK || plan == nullptr) return st;
+  return check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
+}
+
+}  // namespace pa
+
 extern "C" {
 
 int32_t pa_version(void) { return kVersion; }
@@ -434,6 +446,9 @@ size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs, int32_t
                   nullptr, &local) != PA_OK)
       return 0;
     plan = &local;
+  } else if (pa::check_decode_args(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                   max_blocks_per_seq) != PA_OK) {
+    return 0;  // the sizes below divide by plan and shape fields: never with bad ones
   }
   return workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
 }

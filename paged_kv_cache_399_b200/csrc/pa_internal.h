@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "pa.h"
+
 namespace pa {
 
 constexpr int kBlockSize = 16;   // tokens per KV block
@@ -73,6 +75,13 @@ struct DecodeParams {
   int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
   int32_t* win_prefix;           // tcgen05 path with prefix sharing: shared blocks per window
 };
+
+// Host-side checks of a decode call's shapes and (when non-null) its plan, the ones
+// pa_decode runs before anything else; returns a pa_status_t value. The workspace size
+// query and the static-scratch entry point run them first, because the sizes divide by
+// plan and shape fields.
+int check_decode_args(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq);
 
 // Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).
 cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim,

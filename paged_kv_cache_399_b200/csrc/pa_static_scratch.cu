@@ -22,6 +22,8 @@
 
 #include <mutex>
 
+#include "pa_internal.h"
+
 namespace {
 
 // File-scope scratch, PA_STATIC_SCRATCH_BYTES on every GPU that loads this library,
@@ -62,6 +64,11 @@ extern "C" PA_API pa_status_t pa_decode_static_scratch(
                                           max_blocks_per_seq, nullptr, &local);
     if (st != PA_OK) return st;
     plan = &local;
+  } else {
+    // the same shape and plan checks pa_decode runs, before the size below is computed
+    const int st = pa::check_decode_args(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                         max_blocks_per_seq);
+    if (st != PA_OK) return static_cast<pa_status_t>(st);
   }
   const size_t need = pa_decode_workspace_size(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads,
                                                head_dim, max_blocks_per_seq);

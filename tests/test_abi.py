@@ -257,3 +257,28 @@ def test_fp8_cache_write_rejects_bad_arguments_before_launch(pa):
     assert call(bs=8) == pa.PA_ERR_UNSUPPORTED
     assert call(hkv=1, d=8) == pa.PA_ERR_UNSUPPORTED   # a row of 8 elements: not a multiple of 16
     assert call(T=0, k=None) == pa.PA_OK
+
+
+def test_size_query_and_static_scratch_check_before_sizing(pa):
+    """The workspace size of a caller plan divides by plan and shape fields: both the size
+    query and pa_decode_static_scratch run pa_decode's checks first (no SIGFPE, and the same
+    status pa_decode returns)."""
+    lib = pa.raw_library()
+    size = lib.pa_decode_workspace_size
+    plan = pa.pa_decode_plan(2, 1, 4, 2, 64, 4, pa.PA_PATH_TILE, schedule=pa.PA_SCHEDULE_PERSISTENT)
+    assert size(ctypes.byref(plan), 2, 1, 4, 2, 64, 4) > 0
+    assert size(ctypes.byref(plan), 2, 1, 4, 0, 64, 4) == 0            # num_kv_heads = 0
+    assert size(ctypes.byref(plan), -3, 1, 4, 2, 64, 4) == 0           # negative num_seqs
+    zeroed = pa.pa_plan_t()
+    zeroed.path, zeroed.schedule = pa.PA_PATH_TILE, pa.PA_SCHEDULE_PERSISTENT
+    assert size(ctypes.byref(zeroed), 2, 1, 4, 2, 64, 4) == 0
+    zeroed.num_ctas = 4                                                # rows_per_cta still 0
+    assert size(ctypes.byref(zeroed), 2, 1, 4, 2, 64, 4) == 0
+
+    def static(plan_ref, B=2, hkv=2):
+        return lib.pa_decode_static_scratch(8 * 1024, 16 * 1024, 32 * 1024, 48 * 1024, 64 * 1024, 80 * 1024,
+                                            B, 1, 4, hkv, 64, 16, 4, 8, 0.125, plan_ref, None)
+    assert static(ctypes.byref(plan), hkv=0) == pa.PA_ERR_INVALID_ARG
+    assert static(ctypes.byref(plan), B=-3) == pa.PA_ERR_INVALID_ARG
+    assert static(ctypes.byref(zeroed)) == pa.PA_ERR_INVALID_ARG
+    assert _decode_raw(lib, plan=ctypes.byref(zeroed), ws=96 * 1024, ws_bytes=1 << 20) == pa.PA_ERR_INVALID_ARG
