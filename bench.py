@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "llama8b"
-PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per pa_decode launch measured by ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum summed over the launch's kernels), keyed by workload, with
@@ -85,16 +85,40 @@ def decode_bytes(w, unique: bool = True) -> int:
                     end = e
     else:
         tokens = int(sum(int(c) - l for c, l in zip(w.context_lens, lo)))
-    kv = tokens * w.num_kv_heads * w.head_dim * 2 * 2
+    kv = tokens * w.num_kv_heads * w.head_dim * kv_elem_bytes(w) * 2
     qo = 2 * w.num_seqs * w.q_per_seq * w.num_q_heads * w.head_dim * 2
     tables = int(sum(-(-int(c) // bs) - l // bs for c, l in zip(w.context_lens, lo))) * 4
     return kv + qo + tables + w.num_seqs * 4
 
 
+def kv_elem_bytes(w) -> int:
+    """Bytes of one cached K or V element: 2 (bf16) or 1 (an E4M3 code)."""
+    return 1 if getattr(w, "kv_dtype", "bf16") == "fp8_e4m3" else 2
+
+
 def cache_write_bytes(w) -> int:
-    """K and V rows read and written, plus the slot mapping."""
-    row = w.num_kv_heads * w.head_dim * 2
-    return w.num_tokens * (2 * row * 2 + 8)
+    """K and V rows read (bf16) and written (bf16 or E4M3), plus the slot mapping."""
+    elems = w.num_kv_heads * w.head_dim
+    return w.num_tokens * (2 * elems * (2 + kv_elem_bytes(w)) + 8)
+
+
+def prefill_flops(w) -> int:
+    """QK^T and PV multiply-adds of a chunked-prefill step: chunk token i of sequence b sees
+    ctx_b - qlen_b + i + 1 keys, for every query head."""
+    vis = 0
+    for c, q in zip(w.context_lens, w.query_lens):
+        c, q = int(c), int(q)
+        vis += q * (c - q) + q * (q + 1) // 2
+    return 4 * w.head_dim * w.num_q_heads * vis
+
+
+def prefill_bytes(w) -> int:
+    """Bytes a chunked-prefill step must move at least once: the K/V of every sequence's
+    context, q and out, the used table entries, context_lens and query_start."""
+    kv = int(w.context_lens.astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_tokens * w.num_q_heads * w.head_dim * 2
+    tables = int(sum(-(-int(c) // w.block_size) for c in w.context_lens)) * 4
+    return kv + qo + tables + 4 * w.num_seqs + 4 * (w.num_seqs + 1)
 
 
 def decode_flops(w) -> int:
@@ -108,10 +132,10 @@ def decode_flops(w) -> int:
 
 # the sources each kernel family is compiled from (the decode kernels share nothing with
 # the block copy, so a change to one leaves the other's measured traffic valid)
-DECODE_SOURCES = ("pa_api.cpp", "pa_device.cuh", "pa_internal.h", "pa_kernels.cu",
+DECODE_SOURCES = ("pa_api.cpp", "pa_device.cuh", "pa_internal.h", "pa_kernels.cu", "pa_prefill.cuh",
                   "pa_static_scratch.cu", "pa_tcgen05.cuh")
 COPY_SOURCES = ("pa_copy.cu",)
-FP8_SOURCES = ("pa_fp8.cu",)   # the FP8 cache write (no timed workload yet)
+FP8_SOURCES = ("pa_fp8.cu",)   # the FP8 cache write (timed inside the llama8b_fp8 step)
 
 
 def source_hash(names=DECODE_SOURCES) -> str:
@@ -130,6 +154,7 @@ def measured_peaks():
         with open(path) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
     return dict(PEAKS_FALLBACK, source="fallback")
 
@@ -137,7 +162,8 @@ def measured_peaks():
 # ------------------------------------------------------------------ ranks
 
 BASE_SEEDS = {"tiny": 1000, "llama8b": 1001, "llama70b_long": 1002, "prefix_sharing": 1003,
-              "spec_verify": 1004, "cow_fork": 1005, "cow_bulk": 1006, "sliding_window": 1007}
+              "spec_verify": 1004, "cow_fork": 1005, "cow_bulk": 1006, "sliding_window": 1007,
+              "llama8b_fp8": 1008, "chunked_prefill": 1009}
 
 
 def rank_seed(workload: str, rank: int) -> int:
@@ -229,7 +255,9 @@ class ClockSampler:
 
 # The decode configurations every default run also times on the same box, beside the
 # headline workload (µs/call per config is half of the metric).
-PER_CONFIG = ("tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify", "sliding_window")
+PER_CONFIG = ("tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify", "sliding_window",
+              "llama8b_fp8")
+PREFILL_CONFIG = ("chunked_prefill",)
 # the 75 % bar of the measured copy bandwidth holds on the three bandwidth-scale configs
 BAR_CONFIGS = ("llama8b", "llama70b_long", "prefix_sharing")
 
@@ -267,7 +295,31 @@ def _plan_for(pa, w, args):
                              w.max_blocks_per_seq, share_prefix=share, sliding_window=w.window,
                              path={"auto": 0, "single": 1, "tile": 2, "tcgen05": 3}[args.path],
                              split_blocks=args.split_blocks,
-                             schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule])
+                             schedule={"auto": 0, "grid": 1, "persistent": 2}[args.schedule],
+                             kv_cache_dtype=pa.PA_KV_FP8_E4M3 if w.kv_dtype == "fp8_e4m3" else pa.PA_KV_BF16)
+
+
+def _hot_path(pa, w, v, plan, ws, stream):
+    """The step's two calls for this workload's pools: (cache write, decode), each taking no
+    arguments. FP8 pools take the FP8 cache write and pa_decode_fp8."""
+    fp8 = w.kv_dtype == "fp8_e4m3"
+
+    def write():
+        if fp8:
+            pa.pa_reshape_and_cache_fp8(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
+                                        w.k_scale, w.v_scale, stream=stream)
+        else:
+            pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
+                                    stream=stream)
+
+    def decode(s=stream):
+        if fp8:
+            pa.pa_decode_fp8(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                             w.q_per_seq, w.scale, w.k_scale, w.v_scale, plan=plan, workspace=ws, stream=s)
+        else:
+            pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                         w.q_per_seq, w.scale, plan=plan, workspace=ws, stream=s)
+    return write, decode
 
 
 def _ncu_traffic(name):
@@ -283,15 +335,14 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
     without host overhead: one CUDA graph of 20 back-to-back calls, replayed (µs per call,
     None when capture is unavailable)."""
     import torch
+    write, decode = _hot_path(pa, w, v, plan, ws, stream)
     barrier()
     pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(calls)]
     for a, b in pairs:
-        pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
-                                stream=stream)
+        write()
         a.record(stream)
-        pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
-                     w.q_per_seq, w.scale, plan=plan, workspace=ws, stream=stream)
+        decode()
         b.record(stream)
     barrier()
     decode_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
@@ -301,8 +352,7 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             for _ in range(per_graph):
-                pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
-                             w.q_per_seq, w.scale, plan=plan, workspace=ws)
+                decode(None)   # the capture stream
         graph.replay()
         barrier()
         g0 = torch.cuda.Event(enable_timing=True)
@@ -335,11 +385,10 @@ def measure_config(name, args, dev, stream, peaks):
     def barrier():
         torch.cuda.synchronize(dev)
 
+    write, decode = _hot_path(pa, w, v, plan, ws, stream)
     for _ in range(max(3, args.warmup)):
-        pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"],
-                                stream=stream)
-        pa.pa_decode(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
-                     w.q_per_seq, w.scale, plan=plan, workspace=ws, stream=stream)
+        write()
+        decode()
     barrier()
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
     sampler = ClockSampler(dev.index)
@@ -367,6 +416,120 @@ def measure_config(name, args, dev, stream, peaks):
     del v, ws
     torch.cuda.empty_cache()
     return rec
+
+
+NCU_PREFILL_TRAFFIC = {}
+
+
+def measure_prefill(name, args, dev, stream, peaks):
+    """The chunked-prefill step (pa_reshape_and_cache of the chunks' K/V + pa_prefill): µs
+    per pa_prefill call (CUDA events, and graph-replayed), its TFLOP/s against the measured
+    sustained bf16 tensor peak, and its bytes over the copy bandwidth."""
+    import torch
+    from paged_kv_cache_399_b200 import pa, workloads
+    w = workloads.PREFILL_WORKLOADS[name](seed=rank_seed(name, 0))
+    parts = {"query": w.query, "key": w.key, "value": w.value}
+    v = {k: t.to(dev) for k, t in parts.items()}
+    v["slots"] = torch.from_numpy(w.slot_mapping).to(dev)
+    v["tables"] = torch.from_numpy(w.block_tables).to(dev)
+    v["ctx"] = torch.from_numpy(w.context_lens).to(dev)
+    v["qstart"] = torch.from_numpy(w.query_start).to(dev)
+    v["key_cache"] = w.key_cache.to(dev)
+    v["value_cache"] = w.value_cache.to(dev)
+    v["out"] = torch.empty_like(v["query"])
+
+    def write():
+        pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"], stream=stream)
+
+    def prefill(s=stream):
+        pa.pa_prefill(v["out"], v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"], v["qstart"],
+                      w.max_query_len, w.scale, stream=s)
+
+    for _ in range(max(3, args.warmup)):
+        write()
+        prefill()
+    torch.cuda.synchronize(dev)
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    calls = args.config_calls
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+        for a, b in pairs:
+            write()
+            a.record(stream)
+            prefill()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        graph_us = None
+        try:
+            per_graph, reps = 10, max(1, calls // 10)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(per_graph):
+                    prefill(None)
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            g1.record(stream)
+            torch.cuda.synchronize(dev)
+            graph_us = g0.elapsed_time(g1) * 1e3 / (reps * per_graph)
+            del graph
+        except Exception as exc:
+            print(f"graph timing unavailable: {exc}", file=sys.stderr)
+    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    flops = prefill_flops(w)
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    rec = {
+        "workload": w.describe(),
+        "calls": calls,
+        "prefill_us_per_call": round(ms * 1e3, 3),
+        "prefill_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
+        "flops": flops,
+        "tflops": round(tflops, 2),
+        "frac_of_sustained_bf16": round(tflops / peak, 4),
+        "frac_graph": None if graph_us is None else round(flops / (graph_us * 1e-6) / 1e12 / peak, 4),
+        "alg_bytes": prefill_bytes(w),
+        "bytes_frac_of_measured_hbm": round(prefill_bytes(w) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "ncu_traffic": NCU_PREFILL_TRAFFIC.get(name, {}).get("bytes_per_launch")
+        if NCU_PREFILL_TRAFFIC.get(name, {}).get("source_hash") == source_hash() else None,
+        "clocks": sampler.summary(),
+    }
+    del v
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_prefill_gpu(args):
+    """--workload chunked_prefill: one JSON line for the chunked-prefill step alone (1 GPU;
+    under torchrun every rank runs its own replica and rank 0 reports its own)."""
+    import torch
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    from paged_kv_cache_399_b200 import build as pa_build
+    pa_build.build()
+    dev = torch.device("cuda", local_rank)
+    peaks = measured_peaks()
+    args.config_calls = max(args.steps, 3)
+    rec = measure_prefill(args.workload, args, dev, torch.cuda.current_stream(dev), peaks)
+    if int(os.environ.get("RANK", "0")) == 0:
+        print(json.dumps({
+            "metric": "pa_prefill achieved TFLOP/s & fraction of the sustained bf16 tensor peak",
+            "value": rec["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(rec["prefill_us_per_call"] / 1e3, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": rec,
+            "roofline": {"bound": "tensor", "achieved": rec["tflops"], "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": rec["frac_of_sustained_bf16"], "traffic": rec["ncu_traffic"],
+                         "peak_source": peaks["source"] + " (sustained bf16)", "kernel": "prefill_tcm_kernel"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": rec["clocks"],
+        }), flush=True)
 
 
 def run_gpu(args):
@@ -399,10 +562,11 @@ def run_gpu(args):
                                            w.num_kv_heads, w.head_dim, w.max_blocks_per_seq)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
 
+    write, decode = _hot_path(pa, w, v, plan, ws, stream)
+
     def step():
-        pa.pa_reshape_and_cache(key, value, key_cache, value_cache, slots, stream=stream)
-        pa.pa_decode(out, query, key_cache, value_cache, tables, ctx, w.q_per_seq, w.scale, plan=plan,
-                     workspace=ws, stream=stream)
+        write()
+        decode()
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -476,6 +640,8 @@ def run_gpu(args):
         per_config = {}
         for name in PER_CONFIG:
             per_config[name] = measure_config(name, args, dev, stream, peaks)
+        for name in PREFILL_CONFIG:
+            per_config[name] = measure_prefill(name, args, dev, stream, peaks)
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if (world == 1 and not args.no_cpu_baseline) else None
@@ -490,11 +656,12 @@ def run_gpu(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": "bf16" if w.kv_dtype == "bf16" else "bf16 queries, e4m3 KV codes, f16 MMA, fp32 accumulate",
             "data": "synthetic",
             "config": {
                 "workload": w.describe(),
-                "step": "pa_reshape_and_cache + pa_decode",
+                "step": "pa_reshape_and_cache + pa_decode" if w.kv_dtype == "bf16"
+                        else "pa_reshape_and_cache_fp8 + pa_decode_fp8",
                 "alg_bytes_per_step": step_bytes,
                 "decode_alg_bytes": dec_bytes,
                 "decode_logical_bytes": decode_bytes(w, unique=False),
@@ -542,7 +709,8 @@ def decode_launches(plan) -> int:
         return 2 + (1 if plan.share_cap > 1 else 0)
     if plan.schedule == pa.PA_SCHEDULE_PERSISTENT:
         return 2
-    return (1 if plan.share_cap else 0) + 1 + (1 if (plan.num_splits > 1 or plan.share_cap) else 0)
+    # grid: the decode kernel, after the sharing pre-pass or the counter reset when outputs merge
+    return 1 + (1 if (plan.num_splits > 1 or plan.share_cap) else 0)
 
 
 # ------------------------------------------------------------------ CPU oracle legs
@@ -554,6 +722,11 @@ def _oracle_step(orc, w, seqs):
         -1, w.num_kv_heads, w.head_dim)
     sub_val = w.value.view(w.num_seqs, w.q_per_seq, w.num_kv_heads, w.head_dim)[seqs].reshape(
         -1, w.num_kv_heads, w.head_dim)
+    if w.kv_dtype == "fp8_e4m3":
+        kc, vc = orc.reshape_and_cache_fp8(sub_key, sub_val, w.key_cache.numpy(), w.value_cache.numpy(),
+                                           sub_slots, w.k_scale, w.v_scale)
+        return orc.decode_fp8(w.query[seqs], kc, vc, w.block_tables[seqs], w.context_lens[seqs], w.q_per_seq,
+                              w.scale, w.k_scale, w.v_scale, window=w.window)
     kc, vc = orc.reshape_and_cache(sub_key, sub_val, w.key_cache, w.value_cache, sub_slots)
     return orc.decode(w.query[seqs], kc, vc, w.block_tables[seqs], w.context_lens[seqs], w.q_per_seq,
                       w.scale, window=w.window)
@@ -630,6 +803,45 @@ def run_reference(args):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_prefill_reference(args):
+    """The oracle on the chunked-prefill workload: a bounded sample of each step (the rows of
+    a few chunk tokens of every sequence, all heads), reported as TFLOP/s of that sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import Oracle
+    from paged_kv_cache_399_b200 import workloads
+    w = workloads.PREFILL_WORKLOADS[args.workload](seed=rank_seed(args.workload, 0))
+    orc = Oracle()
+    chunk = int(w.query_lens[0])
+    toks = list(range(0, chunk, max(1, chunk // 8)))
+    rows = [(b, i, h) for b in range(w.num_seqs) for i in toks for h in range(w.num_q_heads)]
+    q = w.query.view(w.num_seqs, chunk, w.num_q_heads, w.head_dim)
+
+    def step():
+        kc, vc = orc.reshape_and_cache(w.key, w.value, w.key_cache, w.value_cache, w.slot_mapping)
+        orc.decode_rows(rows, q, kc, vc, w.block_tables, w.context_lens, chunk, w.scale)
+    flops = sum(4 * w.head_dim * (int(w.context_lens[b]) - chunk + i + 1) for b, i, _ in rows)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = f"{len(rows)} of {w.num_tokens * w.num_q_heads} query rows of {w.name} per step (fp64)"
+    print(json.dumps({
+        "impl": "reference", "metric": "pa_prefill achieved TFLOP/s & fraction of the sustained bf16 tensor peak",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.describe(), "step": "oracle cache write + oracle rows"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": orc.threads_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
 
 
 # ------------------------------------------------------------------ block copy
@@ -862,7 +1074,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["tiny", "llama8b", "llama70b_long", "prefix_sharing", "spec_verify",
-                             "sliding_window", "cow_fork", "cow_bulk"],
+                             "sliding_window", "llama8b_fp8", "chunked_prefill", "cow_fork", "cow_bulk"],
                     help="decode workloads time cache write + decode; cow_fork / cow_bulk time the "
                          "copy-on-write block copy")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -880,10 +1092,11 @@ def main(argv=None):
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     copy = args.workload in ("cow_fork", "cow_bulk")
+    prefill = args.workload in PREFILL_CONFIG
     if args.impl == "reference":
-        (run_copy_reference if copy else run_reference)(args)
+        (run_copy_reference if copy else run_prefill_reference if prefill else run_reference)(args)
     else:
-        (run_copy_gpu if copy else run_gpu)(args)
+        (run_copy_gpu if copy else run_prefill_gpu if prefill else run_gpu)(args)
     return 0
 
 

@@ -15,7 +15,11 @@
  *   pa_copy_blocks        the copy-on-write block copy behind shared blocks
  *                         (vLLM study notes §3.2.2);
  *   pa_reshape_and_cache_fp8  the cache write into FP8 (E4M3) pools with one scale per
- *                         pool (vLLM study notes §4.2).
+ *                         pool (vLLM study notes §4.2);
+ *   pa_decode_fp8         pa_decode over such FP8 pools (same notes §4.2: an FP8 KV cache
+ *                         halves attention's memory traffic);
+ *   pa_prefill            chunked-prefill attention: many query tokens per sequence over
+ *                         the paged pool, causal within the chunk (same notes §3.5).
  *
  * Conventions shared by every call
  *   - All data pointers are DEVICE pointers on the current CUDA device (the one
@@ -113,6 +117,13 @@ typedef enum {
                                  units are merged by a second kernel */
 } pa_schedule_t;
 
+/* Element type of the KV pools a plan is for. */
+typedef enum {
+  PA_KV_BF16 = 0,     /* bf16 values: pa_decode */
+  PA_KV_FP8_E4M3 = 1  /* E4M3 codes with one fp32 scale per pool: pa_decode_fp8 (mma.sync
+                         tensor-core tiles only: PA_PATH_TILE, either schedule) */
+} pa_kv_dtype_t;
+
 /* Optional hints for pa_decode_plan; zero-initialised = all automatic. */
 typedef struct {
   int32_t path;          /* pa_path_t */
@@ -132,6 +143,7 @@ typedef struct {
                             block 0, §5.5). Grid schedule, mma.sync or CUDA-core path;
                             with the tcgen05 path, the persistent schedule or
                             share_prefix: PA_ERR_UNSUPPORTED. 0 = no window */
+  int32_t kv_cache_dtype; /* pa_kv_dtype_t of the pools the plan will decode (0 = bf16) */
 } pa_plan_hints_t;
 
 /* A decode plan; fill it with pa_decode_plan and treat it as opaque. */
@@ -151,6 +163,8 @@ typedef struct {
                             num_splits covers the window's blocks,
                             ceil(min(max_blocks_per_seq, ceil((W + q_per_seq - 1) / 16) + 1)
                             / split_blocks) */
+  int32_t kv_cache_dtype; /* pa_kv_dtype_t: pa_decode takes PA_KV_BF16 plans only,
+                            pa_decode_fp8 PA_KV_FP8_E4M3 plans only */
 } pa_plan_t;
 
 /* Write the step's new K/V into the pool: for each token t with slot s =
@@ -174,8 +188,8 @@ PA_API pa_status_t pa_reshape_and_cache(const void* key, const void* value,
  * the fp32 quotient x / k_scale (x / v_scale): round to nearest, ties to even, saturating at
  * +-448 (no infinities in E4M3). k_scale, v_scale: finite, > 0, one per pool, chosen by the
  * caller. Same layouts, strides, alignment, slot and error rules as pa_reshape_and_cache;
- * num_kv_heads*head_dim must be a multiple of 16. The decode over FP8 pools is not built yet:
- * this call writes the codes that such a decode (and the oracle) read back as code * scale. */
+ * num_kv_heads*head_dim must be a multiple of 16. pa_decode_fp8 reads the codes back as
+ * code * scale. */
 PA_API pa_status_t pa_reshape_and_cache_fp8(const void* key, const void* value,
                                      int64_t key_token_stride, int64_t value_token_stride,
                                      void* key_cache, void* value_cache,
@@ -222,6 +236,56 @@ PA_API pa_status_t pa_decode(void* out, const void* query, const void* key_cache
                       int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
                       float scale, const pa_plan_t* plan, void* workspace,
                       size_t workspace_bytes, pa_stream_t stream);
+
+/* Paged decode over FP8 KV pools (vLLM study notes §4.2, --kv-cache-dtype fp8: half the
+ * cache bytes, so half the memory traffic of attention). key_cache and value_cache hold E4M3
+ * codes (uint8 [num_blocks][block_size][num_kv_heads][head_dim], as pa_reshape_and_cache_fp8
+ * writes them); element (t, h, d) of a pool has the value code's value * k_scale (v_scale).
+ * Result: pa_decode's definition over those values, i.e.
+ *   out[b][i][h][:] = sum_t softmax_t(scale * k_scale * q . code_k_t) * v_scale * code_v_t,
+ * rounded to bf16 from fp32 accumulation. The codes are widened to f16 exactly and the products
+ * run on f16 tensor cores with fp32 accumulators; each query row is scaled by a power of two
+ * before its f16 conversion (and the scores back), so any finite bf16 query is accepted.
+ * k_scale, v_scale: finite, > 0 (else PA_ERR_INVALID_ARG). plan: NULL = pa_decode_plan's
+ * heuristic for FP8 pools, else a plan made with hints.kv_cache_dtype = PA_KV_FP8_E4M3 (a bf16
+ * plan is PA_ERR_INVALID_ARG). Everything else -- shapes, layouts, alignment, workspace, the
+ * sliding window and prefix sharing of the plan, ownership, streams, errors -- is pa_decode's.
+ * Code 0x7F / 0xFF (NaN) in a slot outside every context is harmless, as in pa_decode. */
+PA_API pa_status_t pa_decode_fp8(void* out, const void* query, const void* key_cache,
+                                 const void* value_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t num_seqs, int32_t q_per_seq,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                                 float scale, float k_scale, float v_scale, const pa_plan_t* plan,
+                                 void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/* Chunked-prefill paged attention (vLLM study notes, zihan-zhang.net, §3.5 Chunked prefill;
+ * "vLLM 深度解析：连续批处理与内存高效推理" §5.4): each sequence attends a chunk of its prompt --
+ * many query tokens at once -- over the paged pool, causal within the chunk. The chunk's K/V
+ * must already be in the pool (pa_reshape_and_cache with the chunk's slots).
+ *   query, out     bf16 [num_query_tokens][num_q_heads][head_dim]: the chunks of all
+ *                  sequences, concatenated; sequence b's chunk is rows
+ *                  query_start[b] .. query_start[b+1]-1 (qlen_b = their count, may be 0)
+ *   query_start    int32 [num_seqs + 1], DEVICE array, non-decreasing, query_start[0] = 0,
+ *                  query_start[num_seqs] = num_query_tokens
+ *   context_lens   int32 [num_seqs]: tokens of the sequence including its chunk
+ *   block_tables, key_cache, value_cache: as pa_decode (bf16 pools)
+ * Chunk token i of sequence b sits at position pos = context_lens[b] - qlen_b + i and
+ * attends to keys 0 .. pos: out row = sum_t softmax_t(scale * q . k_t) v_t over them, rounded
+ * to bf16 from fp32 accumulation (tensor cores: tcgen05.mma, bf16 operands, fp32
+ * accumulators in tensor memory). max_query_len: host-known bound on every qlen_b (sizes
+ * the grid). Supported: head_dim 128, block_size 16, 128 % (num_q_heads / num_kv_heads) == 0
+ * (else PA_ERR_UNSUPPORTED). Preconditions (device data): qlen_b <= max_query_len and
+ * qlen_b <= context_lens[b] <= max_blocks_per_seq * block_size, block ids as for pa_decode;
+ * a sequence with context_lens[b] < qlen_b gets no rows written. No workspace; nothing is
+ * allocated; asynchronous on `stream`; host argument errors as pa_decode's. Zero sequences,
+ * tokens or max_query_len is a no-op. */
+PA_API pa_status_t pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              const int32_t* query_start, int32_t num_seqs, int32_t num_query_tokens,
+                              int32_t max_query_len, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                              int64_t num_blocks, float scale, pa_stream_t stream);
 
 /* Size of the fixed scratch array pa_decode_static_scratch uses (16 MiB, held on
  * every GPU that loads the library until the process exits). */
@@ -306,7 +370,8 @@ PA_API pa_status_t pa_copy_blocks(void* key_cache, void* value_cache, int64_t nu
 /* Static description of a status code. */
 PA_API const char* pa_status_string(pa_status_t status);
 
-/* ABI version (major * 10000 + minor * 100 + patch). */
+/* ABI version (major * 10000 + minor * 100 + patch). 1.1 added pa_decode_fp8, pa_prefill
+ * and the kv_cache_dtype fields at the end of pa_plan_hints_t and pa_plan_t. */
 PA_API int32_t pa_version(void);
 
 #ifdef __cplusplus

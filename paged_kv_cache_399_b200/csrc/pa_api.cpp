@@ -18,7 +18,7 @@ namespace {
 
 using pa::DecodeParams;
 
-constexpr int32_t kVersion = 10000;  // 1.0.0
+constexpr int32_t kVersion = 10100;  // 1.1.0
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -64,45 +64,52 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // The pool [num_blocks][16][H_kv][D] as a 3-D tensor {D, H_kv, num_blocks*16}; one
 // box is {64, 1, 16}: half of head_dim for one kv head over the 16 tokens of a block,
 // 128-byte swizzled in shared memory.
+// E4M3 pools ([num_blocks][16][H_kv][D] bytes): one box is {D, 1, 16}, a whole block of one
+// kv head (16 rows of D bytes), with the 128-byte swizzle at D = 128 and the 64-byte one at
+// D = 64.
 bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
-                              int32_t head_dim);
+                              int32_t head_dim, int kv_dtype);
 
 // The maps of the last few pools this thread used: encoding costs microseconds of host
 // time on every call otherwise, and a decode loop passes the same two pools each step.
 bool encode_pool_map(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
-                     int32_t head_dim) {
+                     int32_t head_dim, int kv_dtype) {
   struct Entry {
     const void* base;
     int64_t num_blocks;
-    int32_t num_kv_heads, head_dim;
+    int32_t num_kv_heads, head_dim, kv_dtype;
     CUtensorMap map;
   };
   thread_local Entry cache[4] = {};
   thread_local int next = 0;
   for (const Entry& e : cache)
     if (e.base == base && e.base != nullptr && e.num_blocks == num_blocks && e.num_kv_heads == num_kv_heads &&
-        e.head_dim == head_dim) {
+        e.head_dim == head_dim && e.kv_dtype == kv_dtype) {
       *map = e.map;
       return true;
     }
-  if (!encode_pool_map_uncached(map, base, num_blocks, num_kv_heads, head_dim)) return false;
-  cache[next] = Entry{base, num_blocks, num_kv_heads, head_dim, *map};
+  if (!encode_pool_map_uncached(map, base, num_blocks, num_kv_heads, head_dim, kv_dtype)) return false;
+  cache[next] = Entry{base, num_blocks, num_kv_heads, head_dim, kv_dtype, *map};
   next = (next + 1) & 3;
   return true;
 }
 
 bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_blocks, int32_t num_kv_heads,
-                              int32_t head_dim) {
+                              int32_t head_dim, int kv_dtype) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const bool e4m3 = kv_dtype == pa::kKvE4M3;
+  const cuuint64_t elem = e4m3 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_kv_heads),
                         static_cast<cuuint64_t>(num_blocks) * pa::kBlockSize};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
-                           static_cast<cuuint64_t>(head_dim) * num_kv_heads * 2};
-  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(pa::kBlockSize)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * elem,
+                           static_cast<cuuint64_t>(head_dim) * num_kv_heads * elem};
+  cuuint32_t box[3] = {e4m3 ? static_cast<cuuint32_t>(head_dim) : 64u, 1, static_cast<cuuint32_t>(pa::kBlockSize)};
   cuuint32_t elem_strides[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                  elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const CUtensorMapSwizzle swz =
+      (e4m3 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = fn(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -160,9 +167,15 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     return PA_ERR_INVALID_ARG;
   if (h.split_blocks < 0 || h.share_prefix < 0 || h.share_prefix > 1 || h.sliding_window < 0)
     return PA_ERR_INVALID_ARG;
-  // a sliding window runs on the grid schedule of the mma.sync and CUDA-core kernels
-  if (h.sliding_window > 0 && (h.path == PA_PATH_TCGEN05 || h.schedule == PA_SCHEDULE_PERSISTENT ||
-                               h.share_prefix))
+  if (h.kv_cache_dtype != PA_KV_BF16 && h.kv_cache_dtype != PA_KV_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  // E4M3 pools are read by the mma.sync tensor-core tiles (grid or persistent schedule)
+  const bool e4m3 = h.kv_cache_dtype == PA_KV_FP8_E4M3;
+  if (e4m3 && (h.path == PA_PATH_SINGLE || h.path == PA_PATH_TCGEN05)) return PA_ERR_UNSUPPORTED;
+  // a sliding window runs on the grid schedule of the mma.sync and CUDA-core kernels and on
+  // the tcgen05 kernel (its own schedule); not with prefix sharing or the mma.sync
+  // persistent schedule
+  if (h.sliding_window > 0 &&
+      (h.share_prefix || (h.schedule == PA_SCHEDULE_PERSISTENT && h.path != PA_PATH_TCGEN05)))
     return PA_ERR_UNSUPPORTED;
   const int group = num_q_heads / num_kv_heads;
   const int rows = group * q_per_seq;
@@ -178,11 +191,12 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     schedule = PA_SCHEDULE_PERSISTENT;
   }
   int path = h.path;
+  if (path == PA_PATH_AUTO && e4m3) path = PA_PATH_TILE;
   if (path == PA_PATH_AUTO) {
     // measured on B200: the tcgen05 kernel wins for head_dim 128 with more than 16 rows per
     // kv head or with prefix sharing; mma.sync tiles win below that; CUDA cores for <= 2 rows
     if (head_dim == 128 && (rows > 16 || share_cap > 0) && h.schedule != PA_SCHEDULE_GRID &&
-        h.split_blocks == 0 && h.sliding_window == 0) {
+        h.split_blocks == 0) {
       path = PA_PATH_TCGEN05;
       schedule = PA_SCHEDULE_PERSISTENT;
     } else {
@@ -193,7 +207,8 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   const int rpc = share_cap ? pa::kTileMaxRows : rows_per_cta_for(path, rows);
   const int64_t row_chunks = ceil_div(rows, rpc);
   if (num_kv_heads * row_chunks > 65535) return PA_ERR_UNSUPPORTED;  // grid x
-  const int slots = device_info().sms * pa::decode_ctas_per_sm(path, schedule, head_dim, rpc);
+  const int slots = device_info().sms * pa::decode_ctas_per_sm(path, schedule, head_dim, rpc, h.kv_cache_dtype);
+  plan->kv_cache_dtype = h.kv_cache_dtype;
   plan->path = path;
   plan->schedule = schedule;
   plan->rows_per_cta = rpc;
@@ -290,49 +305,67 @@ size_t share_records(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
   return static_cast<size_t>(num_seqs) * (ssplits + plan.num_splits) * q_per_seq * num_q_heads;
 }
 
-// Workspace of the tcgen05 path: two partial records per CTA, then one piece descriptor
-// per CTA. A record holds rows_per_cta rows of O (fp32) and their (m, l) pairs.
+// Workspace of the tcgen05 path: two partial records per CTA (a record holds rows_per_cta
+// rows of O (fp32) and their (m, l) pairs), with prefix sharing the shared-prefix length of
+// every window of share_cap sequences, then one arrival counter per unit (window, kv head,
+// row chunk).
 int32_t tcm_rec_stride(const pa_plan_t& plan, int32_t head_dim) {
   return plan.rows_per_cta * head_dim + 2 * plan.rows_per_cta;
 }
-size_t tcm_desc_offset(const pa_plan_t& plan, int32_t head_dim) {
+size_t tcm_prefix_offset(const pa_plan_t& plan, int32_t head_dim) {
   return align256(static_cast<size_t>(2) * plan.num_ctas * tcm_rec_stride(plan, head_dim) * 4);
 }
+int64_t tcm_windows(const pa_plan_t& plan, int32_t num_seqs) {
+  return plan.share_cap > 1 ? ceil_div(num_seqs, plan.share_cap) : num_seqs;
+}
+size_t tcm_counter_offset(const pa_plan_t& plan, int32_t num_seqs, int32_t head_dim) {
+  size_t off = tcm_prefix_offset(plan, head_dim);
+  if (plan.share_cap > 1) off = align256(off + 4 * static_cast<size_t>(tcm_windows(plan, num_seqs)));
+  return off;
+}
 
-// With prefix sharing the shared-prefix length of every window of share_cap sequences
-// follows the descriptors.
-size_t tcm_prefix_offset(const pa_plan_t& plan, int32_t head_dim) {
-  return align256(tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas));
+// Grid schedule: byte offset of the arrival counters, after the records (and, with prefix
+// sharing, the per-sequence seq_info).
+size_t grid_counter_offset(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                           int32_t head_dim) {
+  const size_t recs = plan.share_cap ? share_records(plan, num_seqs, q_per_seq, num_q_heads)
+                                     : static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads;
+  size_t off = align256(recs * (static_cast<size_t>(head_dim) + 2) * 4);
+  if (plan.share_cap) off += align256(16 * static_cast<size_t>(num_seqs));
+  return off;
 }
 
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
   if (plan.path == PA_PATH_TCGEN05) {
     if (num_seqs == 0) return 0;
-    if (plan.share_cap > 1)
-      return tcm_prefix_offset(plan, head_dim) + 4 * static_cast<size_t>(ceil_div(num_seqs, plan.share_cap));
-    return tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas);
+    const int64_t rows = static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq;
+    const int64_t units = tcm_windows(plan, num_seqs) * num_kv_heads * ceil_div(rows * (plan.share_cap > 1 ? plan.share_cap : 1), plan.rows_per_cta);
+    return tcm_counter_offset(plan, num_seqs, head_dim) + 4 * static_cast<size_t>(units);
   }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (num_seqs == 0) return 0;
     return persistent_layout(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim).total;
   }
-  if (plan.share_cap) {  // records of the shared-prefix splits and of the own splits + seq_info
-    const size_t recs = share_records(plan, num_seqs, q_per_seq, num_q_heads);
-    return align256(recs * (static_cast<size_t>(head_dim) + 2) * 4) + 16 * static_cast<size_t>(num_seqs);
-  }
+  // grid: partial records (o, then (m, l)), with sharing the per-sequence seq_info, then one
+  // arrival counter per output target (sequence, kv head, row chunk)
+  const size_t targets = static_cast<size_t>(num_seqs) * num_kv_heads *
+                         static_cast<size_t>(ceil_div(static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq,
+                                                      plan.rows_per_cta));
+  if (plan.share_cap) return grid_counter_offset(plan, num_seqs, q_per_seq, num_q_heads, head_dim) + 4 * targets;
   if (plan.num_splits <= 1) return 0;
-  return static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads *
-         (static_cast<size_t>(head_dim) + 2) * 4;
+  return grid_counter_offset(plan, num_seqs, q_per_seq, num_q_heads, head_dim) + 4 * targets;
 }
 
 pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_heads,
                        int32_t num_kv_heads, int32_t max_blocks_per_seq) {
   if (plan.path != PA_PATH_SINGLE && plan.path != PA_PATH_TILE && plan.path != PA_PATH_TCGEN05)
     return PA_ERR_INVALID_ARG;
+  if (plan.kv_cache_dtype != PA_KV_BF16 && plan.kv_cache_dtype != PA_KV_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  if (plan.kv_cache_dtype == PA_KV_FP8_E4M3 && plan.path != PA_PATH_TILE) return PA_ERR_INVALID_ARG;
   if (plan.sliding_window < 0) return PA_ERR_INVALID_ARG;
   if (plan.sliding_window > 0 &&
-      (plan.path == PA_PATH_TCGEN05 || plan.schedule != PA_SCHEDULE_GRID || plan.share_cap != 0))
+      (plan.share_cap != 0 || (plan.path != PA_PATH_TCGEN05 && plan.schedule != PA_SCHEDULE_GRID)))
     return PA_ERR_UNSUPPORTED;
   const int rows = num_q_heads / num_kv_heads * q_per_seq;
   if (plan.path == PA_PATH_TCGEN05) {
@@ -370,6 +403,120 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
   }
   if (plan.rows_per_cta != rows_per_cta_for(plan.path, rows)) return PA_ERR_INVALID_ARG;
   return PA_OK;
+}
+
+// pa_decode and pa_decode_fp8: the pools hold bf16 values, or E4M3 codes with one scale
+// per pool (k_scale, v_scale; 1 for bf16 pools).
+pa_status_t decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+                        int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, float scale,
+                        int kv_dtype, float k_scale, float v_scale, const pa_plan_t* plan, void* workspace,
+                        size_t workspace_bytes, pa_stream_t stream) {
+  pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                max_blocks_per_seq);
+  if (st != PA_OK) return st;
+  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (num_blocks <= 0 || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (!(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
+  if (num_blocks * pa::kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;  // TMA coordinate range
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_INVALID_ARG;
+  pa_plan_t local;
+  if (plan) {
+    st = check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
+    if (st == PA_OK && plan->kv_cache_dtype != kv_dtype) st = PA_ERR_INVALID_ARG;  // a plan for other pools
+  } else {
+    pa_plan_hints_t h = {};
+    h.kv_cache_dtype = kv_dtype;
+    st = make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, &h, &local);
+    plan = &local;
+  }
+  if (st != PA_OK) return st;
+  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
+
+  CUtensorMap tk, tv;
+  if (!encode_pool_map(&tk, key_cache, num_blocks, num_kv_heads, head_dim, kv_dtype) ||
+      !encode_pool_map(&tv, value_cache, num_blocks, num_kv_heads, head_dim, kv_dtype))
+    return PA_ERR_CUDA;
+
+  DecodeParams p = {};
+  p.out = static_cast<uint16_t*>(out);
+  p.query = static_cast<const uint16_t*>(query);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.num_seqs = num_seqs;
+  p.q_per_seq = q_per_seq;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.rows = p.group * q_per_seq;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.rows_per_cta = plan->rows_per_cta;
+  p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.v_scale = v_scale;
+  p.split_blocks = plan->split_blocks;
+  p.window = plan->sliding_window;
+  p.num_splits = plan->num_splits;
+  const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
+  char* ws = static_cast<char*>(workspace);
+  if (plan->path == PA_PATH_TCGEN05) {
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+    p.num_ctas = plan->num_ctas;
+    p.share_cap = plan->share_cap;
+    p.rec_stride = tcm_rec_stride(*plan, head_dim);
+    p.records = reinterpret_cast<float*>(ws);
+    if (plan->share_cap > 1) p.win_prefix = reinterpret_cast<int32_t*>(ws + tcm_prefix_offset(*plan, head_dim));
+    p.arrive = reinterpret_cast<int32_t*>(ws + tcm_counter_offset(*plan, num_seqs, head_dim));
+    // CTAs per group: the largest divisor of H_kv that the grid holds
+    p.tc_group = 1;
+    for (int sz = num_kv_heads; sz >= 1; --sz)
+      if (num_kv_heads % sz == 0 && sz <= plan->num_ctas) {
+        p.tc_group = sz;
+        break;
+      }
+  } else if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
+    const PersistentLayout L = persistent_layout(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
+    p.num_ctas = plan->num_ctas;
+    p.share_cap = plan->share_cap;
+    p.target_rows = L.target_rows;
+    p.list_cap = L.list_cap;
+    p.pool_cap = L.pool_cap;
+    p.rec_stride = L.rec_stride;
+    p.hdr = reinterpret_cast<pa::SchedHeader*>(ws + L.hdr);
+    p.seq_start = reinterpret_cast<long long*>(ws + L.seq_start);
+    p.seq_info = reinterpret_cast<int4*>(ws + L.seq_info);
+    p.cta_seq = reinterpret_cast<int32_t*>(ws + L.cta_seq);
+    p.arrive = reinterpret_cast<int32_t*>(ws + L.arrive);
+    p.list_len = reinterpret_cast<int32_t*>(ws + L.list_len);
+    p.list = reinterpret_cast<int2*>(ws + L.list);
+    p.records = reinterpret_cast<float*>(ws + L.records);
+  } else if (need > 0) {
+    const size_t recs = plan->share_cap ? share_records(*plan, num_seqs, q_per_seq, num_q_heads)
+                                        : static_cast<size_t>(num_seqs) * plan->num_splits * rq;
+    p.ws_o = reinterpret_cast<float*>(ws);
+    p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + recs * head_dim);
+    if (plan->share_cap) {
+      p.share_cap = plan->share_cap;
+      p.share_split_blocks = plan->share_split_blocks;
+      p.share_splits = static_cast<int32_t>(
+          ceil_div(static_cast<int64_t>(plan->split_blocks) * plan->num_splits, plan->share_split_blocks));
+      p.share_windows = static_cast<int32_t>(ceil_div(num_seqs, plan->share_cap));
+      p.seq_info = reinterpret_cast<int4*>(ws + align256(recs * (static_cast<size_t>(head_dim) + 2) * 4));
+    }
+    p.arrive = reinterpret_cast<int32_t*>(ws + grid_counter_offset(*plan, num_seqs, q_per_seq, num_q_heads, head_dim));
+  }
+  cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, kv_dtype, tk, tv,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace
@@ -459,103 +606,67 @@ pa_status_t pa_decode(void* out, const void* query, const void* key_cache, const
                       int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
                       int64_t num_blocks, float scale, const pa_plan_t* plan, void* workspace,
                       size_t workspace_bytes, pa_stream_t stream) {
-  pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
-                                max_blocks_per_seq);
-  if (st != PA_OK) return st;
-  if (block_size != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
-  if (num_blocks <= 0 || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  if (num_blocks * pa::kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;  // TMA coordinate range
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, num_seqs, q_per_seq,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                     PA_KV_BF16, 1.f, 1.f, plan, workspace, workspace_bytes, stream);
+}
+
+pa_status_t pa_decode_fp8(void* out, const void* query, const void* key_cache, const void* value_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+                          int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, float scale,
+                          float k_scale, float v_scale, const pa_plan_t* plan, void* workspace,
+                          size_t workspace_bytes, pa_stream_t stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, num_seqs, q_per_seq,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                     PA_KV_FP8_E4M3, k_scale, v_scale, plan, workspace, workspace_bytes, stream);
+}
+
+pa_status_t pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+                       const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+                       int32_t num_seqs, int32_t num_query_tokens, int32_t max_query_len, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                       int64_t num_blocks, float scale, pa_stream_t stream) {
+  if (num_seqs < 0 || num_query_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / num_kv_heads;
+  // 128 query rows per CTA = 128 / G chunk tokens x the G heads of a kv head
+  if (head_dim != 128 || block_size != pa::kBlockSize || 128 % group != 0) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_blocks_per_seq) * pa::kBlockSize > INT32_MAX ||
+      num_blocks * pa::kBlockSize > INT32_MAX)
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_query_tokens == 0 || max_query_len == 0) return PA_OK;
+  const int tile_tokens = 128 / group;
+  const int64_t max_tiles = ceil_div(max_query_len, tile_tokens);
+  if (num_seqs > 65535 || max_tiles > 65535) return PA_ERR_UNSUPPORTED;  // grid y, z
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens || !query_start)
     return PA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
-      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_start) & 3u))
     return PA_ERR_INVALID_ARG;
-  pa_plan_t local;
-  if (plan) {
-    st = check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
-  } else {
-    st = make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                   nullptr, &local);
-    plan = &local;
-  }
-  if (st != PA_OK) return st;
-  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
-
   CUtensorMap tk, tv;
-  if (!encode_pool_map(&tk, key_cache, num_blocks, num_kv_heads, head_dim) ||
-      !encode_pool_map(&tv, value_cache, num_blocks, num_kv_heads, head_dim))
+  if (!encode_pool_map(&tk, key_cache, num_blocks, num_kv_heads, head_dim, pa::kKvBf16) ||
+      !encode_pool_map(&tv, value_cache, num_blocks, num_kv_heads, head_dim, pa::kKvBf16))
     return PA_ERR_CUDA;
-
-  DecodeParams p = {};
+  pa::PrefillParams p = {};
   p.out = static_cast<uint16_t*>(out);
   p.query = static_cast<const uint16_t*>(query);
   p.block_tables = block_tables;
   p.context_lens = context_lens;
+  p.query_start = query_start;
   p.num_seqs = num_seqs;
-  p.q_per_seq = q_per_seq;
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
-  p.group = num_q_heads / num_kv_heads;
-  p.rows = p.group * q_per_seq;
+  p.group = group;
   p.max_blocks = max_blocks_per_seq;
+  p.tile_tokens = tile_tokens;
   p.num_blocks = num_blocks;
-  p.rows_per_cta = plan->rows_per_cta;
-  p.row_chunks = static_cast<int32_t>(ceil_div(p.rows, p.rows_per_cta));
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.split_blocks = plan->split_blocks;
-  p.window = plan->sliding_window;
-  p.num_splits = plan->num_splits;
-  const int64_t rq = static_cast<int64_t>(q_per_seq) * num_q_heads;
-  char* ws = static_cast<char*>(workspace);
-  if (plan->path == PA_PATH_TCGEN05) {
-    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
-    p.num_ctas = plan->num_ctas;
-    p.share_cap = plan->share_cap;
-    p.rec_stride = tcm_rec_stride(*plan, head_dim);
-    p.records = reinterpret_cast<float*>(ws);
-    if (plan->share_cap > 1) p.win_prefix = reinterpret_cast<int32_t*>(ws + tcm_prefix_offset(*plan, head_dim));
-    p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
-    // CTAs per group: the largest divisor of H_kv that the grid holds
-    p.tc_group = 1;
-    for (int sz = num_kv_heads; sz >= 1; --sz)
-      if (num_kv_heads % sz == 0 && sz <= plan->num_ctas) {
-        p.tc_group = sz;
-        break;
-      }
-  } else if (plan->schedule == PA_SCHEDULE_PERSISTENT) {
-    const PersistentLayout L = persistent_layout(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
-    p.num_ctas = plan->num_ctas;
-    p.share_cap = plan->share_cap;
-    p.target_rows = L.target_rows;
-    p.list_cap = L.list_cap;
-    p.pool_cap = L.pool_cap;
-    p.rec_stride = L.rec_stride;
-    p.hdr = reinterpret_cast<pa::SchedHeader*>(ws + L.hdr);
-    p.seq_start = reinterpret_cast<long long*>(ws + L.seq_start);
-    p.seq_info = reinterpret_cast<int4*>(ws + L.seq_info);
-    p.cta_seq = reinterpret_cast<int32_t*>(ws + L.cta_seq);
-    p.arrive = reinterpret_cast<int32_t*>(ws + L.arrive);
-    p.list_len = reinterpret_cast<int32_t*>(ws + L.list_len);
-    p.list = reinterpret_cast<int2*>(ws + L.list);
-    p.records = reinterpret_cast<float*>(ws + L.records);
-  } else if (need > 0) {
-    const size_t recs = plan->share_cap ? share_records(*plan, num_seqs, q_per_seq, num_q_heads)
-                                        : static_cast<size_t>(num_seqs) * plan->num_splits * rq;
-    p.ws_o = reinterpret_cast<float*>(ws);
-    p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + recs * head_dim);
-    if (plan->share_cap) {
-      p.share_cap = plan->share_cap;
-      p.share_split_blocks = plan->share_split_blocks;
-      p.share_splits = static_cast<int32_t>(
-          ceil_div(static_cast<int64_t>(plan->split_blocks) * plan->num_splits, plan->share_split_blocks));
-      p.share_windows = static_cast<int32_t>(ceil_div(num_seqs, plan->share_cap));
-      p.seq_info = reinterpret_cast<int4*>(ws + align256(recs * (static_cast<size_t>(head_dim) + 2) * 4));
-    }
-  }
-  cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, tk, tv,
-                                    reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e =
+      pa::launch_prefill(p, static_cast<int>(max_tiles), tk, tv, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -43,7 +43,8 @@ struct DecodeParams {
   int64_t num_blocks;             // pool size (blocks)
   int32_t rows_per_cta;          // rows the kernel instance holds (ROWS)
   int32_t row_chunks;            // ceil(rows / rows_per_cta)
-  float scale_log2;              // scale * log2(e)
+  float scale_log2;              // scale * log2(e) (E4M3 pools: times the key pool's scale)
+  float v_scale;                 // E4M3 pools: the value pool's scale (1 for bf16 pools)
   int32_t window;                // sliding window in tokens (grid schedule only); 0 = none
 
   // grid schedule: split partials for the merge kernel; with prefix sharing also the
@@ -64,14 +65,12 @@ struct DecodeParams {
   long long* seq_start;          // [B] first work unit of the sequence's bands
   int4* seq_info;                // [B] {P_b shared prefix blocks, members if leader else 0, nblk, ctx}
   int32_t* cta_seq;              // [num_ctas] sequence holding the CTA's first unit
-  int32_t* arrive;               // [targets] blocks merged so far
+  int32_t* arrive;               // [targets] persistent: blocks merged so far; grid and tcgen05:
+                                 // arrivals of this call (zeroed by its first kernel)
   int32_t* list_len;             // [targets]
   int2* list;                    // [targets][list_cap] {piece start block, record slot}
   float* records;                // [pool_cap][rec_stride]; tcgen05 path: [2 * num_ctas][rec_stride]
 
-  // tcgen05 path: per CTA, the unit whose first piece it holds when that unit continues
-  // in later CTAs: {record slot, last CTA with a piece, sequence, unit}, or {-1, ...}
-  int4* tc_desc;
   int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
   int32_t* win_prefix;           // tcgen05 path with prefix sharing: shared blocks per window
 };
@@ -83,13 +82,34 @@ struct DecodeParams {
 int check_decode_args(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
                       int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq);
 
-// Launch the decode (pre-pass + persistent kernel, or grid kernel + merge).
-cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim,
+// KV pool element types.
+constexpr int kKvBf16 = 0;
+constexpr int kKvE4M3 = 1;
+
+// Launch the decode (pre-pass + persistent kernel, or grid kernel + merge) over pools of
+// element type kv_dtype.
+cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim, int kv_dtype,
                           const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
                           cudaStream_t stream);
 
+// Chunked-prefill attention (pa_prefill.cuh): one CTA per (kv head, sequence, tile of
+// 128 / G chunk tokens counted from the chunk's end), max_tiles tiles per sequence.
+struct PrefillParams {
+  uint16_t* out;                 // bf16 [T][H_q][D]
+  const uint16_t* query;         // bf16 [T][H_q][D]
+  const int32_t* block_tables;   // [B][max_blocks]
+  const int32_t* context_lens;   // [B], including the chunk's tokens
+  const int32_t* query_start;    // [B + 1], first token of each sequence's chunk in query/out
+  int32_t num_seqs, num_q_heads, num_kv_heads, group, max_blocks;
+  int32_t tile_tokens;           // chunk tokens per CTA: 128 / group
+  int64_t num_blocks;            // pool size (blocks)
+  float scale_log2;              // scale * log2(e)
+};
+cudaError_t launch_prefill(const PrefillParams& p, int max_tiles, const CUtensorMap& tmap_k,
+                           const CUtensorMap& tmap_v, cudaStream_t stream);
+
 // Resident CTAs per SM of the decode kernel launch_decode would use.
-int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta);
+int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, int kv_dtype);
 
 cudaError_t launch_cache_write(const uint16_t* key, const uint16_t* value, int64_t key_stride,
                                int64_t value_stride, uint16_t* key_cache, uint16_t* value_cache,

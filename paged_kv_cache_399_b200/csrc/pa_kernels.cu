@@ -8,14 +8,14 @@
 //   decode_persistent_kernel paged decode, one CTA per resident slot, each over an
 //                            equal share of the work; partial results are merged by
 //                            the CTA that completes an output
-//   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split)
-//   merge_kernel             log-sum-exp merge of the grid schedule's split partials
+//   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split); the CTA
+//                            that completes an output's splits merges their partials
+//   grid_reset_kernel        zeroes the grid schedule's per-output arrival counters
 //   validate_kernel          debug bounds check of slots / block ids / context lengths
 //   selftest_wait_kernel     the bounded-wait failure path, taken without a fault
 // and, from pa_tcgen05.cuh, the 5th-generation tensor-core path:
 //   decode_tcm_kernel        tokens on M, tcgen05.mma with TMEM accumulators, persistent
 //                            equal-tile schedule over windows of sequences
-//   tcm_merge_kernel         merge of the units a tile range boundary cuts
 //   tcm_share_prepass        common table prefix of each window (prefix sharing)
 //
 // Two compute cores run inside the mma.sync / CUDA-core decode kernels:
@@ -60,11 +60,19 @@ constexpr unsigned kErrSelftest = 0x600u;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kHalfTileBytes = 16 * 64 * 2;  // 16 tokens x 64 bf16
 
-template <int D>
+// One block of one kv head as it sits in a pipeline stage. bf16 pools: D/64 TMA boxes of
+// 16 tokens x 64 elements (2 KB each, 128-byte swizzle). E4M3 pools: one box of 16 tokens x
+// D bytes (128-byte swizzle at D = 128, 64-byte at D = 64).
+template <int D, bool kFp8 = false>
 struct TileGeom {
-  static constexpr int kHalves = D / 64;
-  static constexpr int kTileBytes = 16 * D * 2;      // one K or V block tile of a kv head
-  static constexpr int kStageBytes = 2 * kTileBytes;  // K + V
+  static constexpr int kD = D;
+  static constexpr bool kE4M3 = kFp8;
+  static constexpr int kBoxes = kFp8 ? 1 : D / 64;                // TMA boxes per K (or V) tile
+  static constexpr int kBoxBytes = kFp8 ? 16 * D : kHalfTileBytes;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;          // one K or V block tile of a kv head
+  static constexpr int kStageBytes = 2 * kTileBytes;             // K + V
+  // element (x) coordinate of box hf: bf16 boxes cover 64 elements each
+  static __device__ __forceinline__ int box_x(int hf) { return kFp8 ? 0 : hf * 64; }
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -120,7 +128,7 @@ __device__ __forceinline__ size_t out_offset(const DecodeParams& p, int b, int i
 // ---------------------------------------------------------------------------
 // Per-warp TMA pipeline over the blocks j = blk0 + warp + NW*k, k < n_my.
 // ---------------------------------------------------------------------------
-template <int D, int NW, int STAGES>
+template <class Geom, int NW, int STAGES>
 struct WarpPipe {
   uint8_t* stage_base;   // this warp's STAGES stage buffers
   uint64_t* bars;        // this warp's STAGES mbarriers
@@ -138,7 +146,7 @@ struct WarpPipe {
   __device__ __forceinline__ void init(uint8_t* smem, uint64_t* all_bars, int warp_, int lane_) {
     warp = warp_;
     lane = lane_;
-    stage_base = smem + warp * STAGES * TileGeom<D>::kStageBytes;
+    stage_base = smem + warp * STAGES * Geom::kStageBytes;
     bars = all_bars + warp * STAGES;
     phase_base = 0;
     issued = 0;
@@ -158,9 +166,9 @@ struct WarpPipe {
     issued = 0;
   }
   __device__ __forceinline__ uint8_t* kbuf(int s) const {
-    return stage_base + s * TileGeom<D>::kStageBytes;
+    return stage_base + s * Geom::kStageBytes;
   }
-  __device__ __forceinline__ uint8_t* vbuf(int s) const { return kbuf(s) + TileGeom<D>::kTileBytes; }
+  __device__ __forceinline__ uint8_t* vbuf(int s) const { return kbuf(s) + Geom::kTileBytes; }
   __device__ __forceinline__ int stage_of(int k) const { return (phase_base + k) % STAGES; }
   __device__ __forceinline__ uint32_t parity_of(int k) const { return ((phase_base + k) / STAGES) & 1; }
   // Called by all lanes, in increasing k.
@@ -174,13 +182,13 @@ struct WarpPipe {
     if (lane == 0) {
       fence_proxy_async_smem();
       uint64_t* bar = &bars[s];
-      mbar_arrive_expect_tx(bar, TileGeom<D>::kStageBytes);
+      mbar_arrive_expect_tx(bar, Geom::kStageBytes);
 #pragma unroll
-      for (int hf = 0; hf < TileGeom<D>::kHalves; ++hf)
-        tma_load_3d(kbuf(s) + hf * kHalfTileBytes, tk, bar, hf * 64, kvh, phys * kBlockSize);
+      for (int hf = 0; hf < Geom::kBoxes; ++hf)
+        tma_load_3d(kbuf(s) + hf * Geom::kBoxBytes, tk, bar, Geom::box_x(hf), kvh, phys * kBlockSize);
 #pragma unroll
-      for (int hf = 0; hf < TileGeom<D>::kHalves; ++hf)
-        tma_load_3d(vbuf(s) + hf * kHalfTileBytes, tv, bar, hf * 64, kvh, phys * kBlockSize);
+      for (int hf = 0; hf < Geom::kBoxes; ++hf)
+        tma_load_3d(vbuf(s) + hf * Geom::kBoxBytes, tv, bar, Geom::box_x(hf), kvh, phys * kBlockSize);
     }
     issued = k + 1;
   }
@@ -204,9 +212,72 @@ struct WarpPipe {
 //   O^T[D][8 rows] += V^T[D][16 tok] . P^T[16 tok][8 rows] (A = V via ldmatrix.trans,
 //                                                            B = P^T via movmatrix)
 // NT n-tiles of 8 rows; only the first nt_active carry real rows in a segment.
+//
+// kFp8: the pools hold E4M3 codes (vLLM study notes §4.2, --kv-cache-dtype fp8) with one
+// scale per pool. The tile bytes are widened in registers, exactly, to f16
+// (cvt.rn.f16x2.e4m3x2; every E4M3 value is an f16 value) and the products run as f16
+// mma.sync with fp32 accumulators:
+//   K: ldmatrix over byte pairs gives a lane four consecutive codes of one token, so the
+//      k index of a 16-wide step is the head-dim order permuted as k 2c,2c+1 <-> d 4c,4c+1
+//      and k 2c+8,2c+9 <-> d 4c+2,4c+3 (c = lane % 4); Q's fragments use the same order,
+//      which leaves every dot product unchanged;
+//   V: ldmatrix.trans over byte pairs gives a lane two tokens x two head-dim columns; one
+//      byte permute pairs the tokens of each column, so the m index of a 16-row tile is
+//      the head-dim order permuted as m g <-> d 2g and m g+8 <-> d 2g+1 (g = lane / 4),
+//      undone when O is written out;
+//   Q: each row is scaled by a power of two 2^s (exact) that puts its largest magnitude in
+//      [2^14, 2^15) before the f16 conversion, so no bf16 query overflows f16; the scores
+//      are multiplied back by 2^-s. k_scale is folded into the softmax scale by the host and
+//      v_scale is applied to O once, before it leaves the core.
 // ---------------------------------------------------------------------------
-template <int D, int NT>
+
+// Four E4M3 codes -> two f16 pairs: lo = codes 0, 1 (code 0 in the low half), hi = codes 2, 3.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 c01, c23;\n\t"
+      "mov.b32 {c01, c23}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t sel) {
+  uint32_t y;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(y) : "r"(x), "r"(0u), "r"(sel));
+  return y;
+}
+
+// Two fp32 -> packed f16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t v;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(v) : "f"(hi), "f"(lo));
+  return v;
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `c` of token row `t` inside an E4M3 tile of D-byte rows, as TMA
+// swizzles it: 128-byte swizzle for D = 128, 64-byte swizzle for D = 64.
+template <int D>
+__device__ __forceinline__ uint32_t e4m3_chunk_offset(int t, int c) {
+  if constexpr (D == 128)
+    return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
+  else
+    return static_cast<uint32_t>(t * 64 + ((c ^ ((t >> 1) & 3)) << 4));
+}
+
+template <int D, int NT, bool kFp8 = false>
 struct TileCore {
+  using Geom = TileGeom<D, kFp8>;
+  static constexpr int kStages = kFp8 ? 4 : 2;  // stages per warp: the same bytes in flight
   static constexpr int ROWS = NT * 8;
   static constexpr int KSTEPS = D / 16;
   static constexpr bool kNeedsQSmem = false;
@@ -214,20 +285,53 @@ struct TileCore {
   int lim[NT][2];
   float m_run[NT][2], l_run[NT][2];
   float o[KSTEPS][NT][4];
+  float rs[NT][2];  // kFp8: 2^-s of the rows of this lane's score columns (1 otherwise)
+  float v_scale;
   int nt_active;
   int vlim;  // largest row limit of the segment: no row sees a token past it
 
   __device__ __forceinline__ void begin(const DecodeParams& p, const Seg& s, int ctx, int lane) {
     nt_active = (s.nrows + 7) >> 3;
+    v_scale = p.v_scale;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       int b = 0, i = 0, h = 0;
       const bool valid = seg_row(p, s, nt * 8 + (lane >> 2), b, i, h);
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.query + out_offset(p, b, i, h, D));
+      if constexpr (!kFp8) {
 #pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        qf[nt][kk][0] = valid ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
-        qf[nt][kk][1] = valid ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          qf[nt][kk][0] = valid ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
+          qf[nt][kk][1] = valid ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+        }
+        rs[nt][0] = rs[nt][1] = 1.f;
+      } else {
+        // lane (g, c) holds d = 32*kc + 4c .. 4c+3 (step 2kc) and 32*kc + 16 + 4c .. (step 2kc+1)
+        const uint2* q2 = reinterpret_cast<const uint2*>(qrow);
+        uint2 raw[KSTEPS];
+        float mx = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          raw[kk] = valid ? __ldg(q2 + kk * 4 + (lane & 3)) : make_uint2(0u, 0u);
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(bf16_lo(raw[kk].x)), fabsf(bf16_hi(raw[kk].x))),
+                               fmaxf(fabsf(bf16_lo(raw[kk].y)), fabsf(bf16_hi(raw[kk].y)))));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        // 2^s with the row's largest magnitude in [2^14, 2^15) (s clamped: a row that small is 0)
+        int sh = 0;
+        if (mx > 0.f) sh = 14 - (static_cast<int>((__float_as_uint(mx) >> 23) & 0xFFu) - 127);
+        sh = min(max(sh, -100), 100);
+        const float up = __uint_as_float(static_cast<uint32_t>(127 + sh) << 23);
+        const float down = __uint_as_float(static_cast<uint32_t>(127 - sh) << 23);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          qf[nt][kk][0] = pack_f16x2(bf16_lo(raw[kk].x) * up, bf16_hi(raw[kk].x) * up);
+          qf[nt][kk][1] = pack_f16x2(bf16_lo(raw[kk].y) * up, bf16_hi(raw[kk].y) * up);
+        }
+        // this lane's score columns are rows 2c and 2c+1, whose factors sit in lanes 4 * row
+        rs[nt][0] = __shfl_sync(kFull, down, 8 * (lane & 3));
+        rs[nt][1] = __shfl_sync(kFull, down, 8 * (lane & 3) + 4);
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -257,24 +361,49 @@ struct TileCore {
     const uint32_t kb = smem_u32(kt);
     const uint32_t vb = smem_u32(vt);
     const int lm = lane >> 3, lr = lane & 7;
-    const int k_tok = lr + (lm & 1) * 8, k_chk = lm >> 1;  // K (non-transposed A)
-    const int v_tok = lr + (lm >> 1) * 8, v_chk = lm & 1;  // V (transposed A)
     float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    if constexpr (!kFp8) {
+      const int k_tok = lr + (lm & 1) * 8, k_chk = lm >> 1;  // K (non-transposed A)
 #pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(kb + tile_chunk_offset(k_tok, 2 * kk + k_chk), a0, a1, a2, a3);
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(kb + tile_chunk_offset(k_tok, 2 * kk + k_chk), a0, a1, a2, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        if (nt < nt_active) mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+        for (int nt = 0; nt < NT; ++nt)
+          if (nt < nt_active) mma_bf16_16816(sc[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      }
+    } else {
+      // matrices: tokens 0-7 / 8-15 x the two 16-byte chunks of a 32-byte column group
+      const int k_tok = lr + (lm & 1) * 8, k_chk = lm >> 1;
+#pragma unroll
+      for (int kc = 0; kc < D / 32; ++kc) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4(kb + e4m3_chunk_offset<D>(k_tok, 2 * kc + k_chk), r0, r1, r2, r3);
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_f16x2(r0, a0, a2);  // token g: d 4c,4c+1 | 4c+2,4c+3 of the first chunk
+        e4m3x4_to_f16x2(r1, a1, a3);  // token g + 8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          if (nt < nt_active) mma_f16_16816(sc[nt], a0, a1, a2, a3, qf[nt][2 * kc][0], qf[nt][2 * kc][1]);
+        e4m3x4_to_f16x2(r2, a0, a2);  // the second chunk
+        e4m3x4_to_f16x2(r3, a1, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          if (nt < nt_active)
+            mma_f16_16816(sc[nt], a0, a1, a2, a3, qf[nt][2 * kc + 1][0], qf[nt][2 * kc + 1][1]);
+      }
     }
     // scores in log2 units, then the causal / end-of-context mask
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[nt][e] *= c;
+    for (int nt = 0; nt < NT; ++nt) {
+      const float c0 = kFp8 ? c * rs[nt][0] : c, c1 = kFp8 ? c * rs[nt][1] : c;
+      sc[nt][0] *= c0;
+      sc[nt][1] *= c1;
+      sc[nt][2] *= c0;
+      sc[nt][3] *= c1;
+    }
     if (need_mask) {
       const int t0 = tb + (lane >> 2);
 #pragma unroll
@@ -319,8 +448,13 @@ struct TileCore {
         l_run[nt][e] = fmaf(l_run[nt][e], alpha[nt][e], p0 + p1);
         m_run[nt][e] = m_new;
       }
-      pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[nt][0], sc[nt][1]));
-      pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[nt][2], sc[nt][3]));
+      if constexpr (!kFp8) {
+        pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[nt][0], sc[nt][1]));
+        pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[nt][2], sc[nt][3]));
+      } else {
+        pb[nt][0] = movmatrix_trans(pack_f16x2(sc[nt][0], sc[nt][1]));
+        pb[nt][1] = movmatrix_trans(pack_f16x2(sc[nt][2], sc[nt][3]));
+      }
     }
     // Slots of the last block past the context, and slots before every row's window, may
     // hold any bits (NaN too): their p is 0, but 0 * NaN is NaN, so their V elements are
@@ -345,19 +479,47 @@ struct TileCore {
           o[mt][nt][3] *= alpha[nt][1];
         }
     }
+    if constexpr (!kFp8) {
+      const int v_tok = lr + (lm >> 1) * 8, v_chk = lm & 1;  // V (transposed A)
 #pragma unroll
-    for (int mt = 0; mt < KSTEPS; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      ldmatrix_x4_trans(vb + tile_chunk_offset(v_tok, 2 * mt + v_chk), a0, a1, a2, a3);
-      if (vmask) {
-        a0 &= vm_lo;
-        a1 &= vm_lo;
-        a2 &= vm_hi;
-        a3 &= vm_hi;
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(vb + tile_chunk_offset(v_tok, 2 * mt + v_chk), a0, a1, a2, a3);
+        if (vmask) {
+          a0 &= vm_lo;
+          a1 &= vm_lo;
+          a2 &= vm_hi;
+          a3 &= vm_hi;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          if (nt < nt_active) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
       }
+    } else {
+      // matrices: tokens 0-7 / 8-15 x the two 16-byte chunks of a 32-byte column group; a
+      // lane receives tokens 2c, 2c+1 x codes 2g, 2g+1 of each (tokens 2c+8, 2c+9 from the
+      // second), and the byte permute 3120 pairs the two tokens of each code column
+      const int v_tok = lr + (lm & 1) * 8, v_chk = lm >> 1;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        if (nt < nt_active) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      for (int kc = 0; kc < D / 32; ++kc) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4_trans(vb + e4m3_chunk_offset<D>(v_tok, 2 * kc + v_chk), r0, r1, r2, r3);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t a0, a1, a2, a3;
+          e4m3x4_to_f16x2(byte_perm(half ? r2 : r0, 0x3120u), a0, a1);  // tokens 2c, 2c+1: d 2g | 2g+1
+          e4m3x4_to_f16x2(byte_perm(half ? r3 : r1, 0x3120u), a2, a3);  // tokens 2c+8, 2c+9
+          if (vmask) {
+            a0 &= vm_lo;
+            a1 &= vm_lo;
+            a2 &= vm_hi;
+            a3 &= vm_hi;
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            if (nt < nt_active) mma_f16_16816(o[2 * kc + half][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        }
+      }
     }
   }
 
@@ -380,11 +542,19 @@ struct TileCore {
       for (int nt = 0; nt < NT; ++nt) {
         if (nt >= nt_active) continue;
         const int r = nt * 8 + 2 * (lane & 3);
-        const int d = mt * 16 + (lane >> 2);
-        ow[r * OS + d] = o[mt][nt][0];
-        ow[(r + 1) * OS + d] = o[mt][nt][1];
-        ow[r * OS + d + 8] = o[mt][nt][2];
-        ow[(r + 1) * OS + d + 8] = o[mt][nt][3];
+        if constexpr (!kFp8) {
+          const int d = mt * 16 + (lane >> 2);
+          ow[r * OS + d] = o[mt][nt][0];
+          ow[(r + 1) * OS + d] = o[mt][nt][1];
+          ow[r * OS + d + 8] = o[mt][nt][2];
+          ow[(r + 1) * OS + d + 8] = o[mt][nt][3];
+        } else {
+          // m g <-> d 2g, m g+8 <-> d 2g+1 (see block); the pool's V scale applies here once
+          const int d = mt * 16 + 2 * (lane >> 2);
+          *reinterpret_cast<float2*>(ow + r * OS + d) = make_float2(o[mt][nt][0] * v_scale, o[mt][nt][2] * v_scale);
+          *reinterpret_cast<float2*>(ow + (r + 1) * OS + d) =
+              make_float2(o[mt][nt][1] * v_scale, o[mt][nt][3] * v_scale);
+        }
       }
     if (lane < 4) {
 #pragma unroll
@@ -406,6 +576,8 @@ struct TileCore {
 // ---------------------------------------------------------------------------
 template <int D, int ROWS_>
 struct SimtCore {
+  using Geom = TileGeom<D>;
+  static constexpr int kStages = 2;
   static constexpr int ROWS = ROWS_;
   static constexpr int CPL = D / 16;  // 16-byte chunks of a row each lane of a pair covers
   static constexpr int DPL = D / 32;  // output columns per lane
@@ -558,9 +730,10 @@ struct SimtCore {
 // ---------------------------------------------------------------------------
 // Shared memory of a decode CTA and the per-segment driver.
 // ---------------------------------------------------------------------------
-template <int D, int ROWS, int NW, int STAGES>
+template <class Geom, int ROWS, int NW, int STAGES>
 struct DecodeSmem {
-  static constexpr int kStages = NW * STAGES * TileGeom<D>::kStageBytes;
+  static constexpr int D = Geom::kD;
+  static constexpr int kStages = NW * STAGES * Geom::kStageBytes;
   static constexpr int kMerge = NW * ROWS * (D + 4) * 4;
   static constexpr int kBytes = (kStages > kMerge ? kStages : kMerge) + 1024;  // + alignment slack
 };
@@ -572,6 +745,7 @@ struct CtaState {
   float2 ml[NW * ROWS];
   int slot[kTileMaxRows];
   int last[kTileMaxRows];
+  int merge[kTileMaxRows];  // grid schedule: 1 = this CTA completed the target's splits
   __align__(16) float q_s[kQ ? ROWS : 1][D];
   __align__(16) float p_s[NW][kQ ? 16 * ROWS : 1];
 };
@@ -580,7 +754,7 @@ struct CtaState {
 // sits in shared memory (ow: NW x ROWS x (D+4) fp32 over the stage buffers; st.ml).
 template <class Core, int D, int NW, int STAGES, class State>
 __device__ __forceinline__ void run_segment(const DecodeParams& p, const Seg& sg, int ctx,
-                                            WarpPipe<D, NW, STAGES>& pipe, Core& core, State& st,
+                                            WarpPipe<typename Core::Geom, NW, STAGES>& pipe, Core& core, State& st,
                                             uint8_t* smem, const CUtensorMap* tk,
                                             const CUtensorMap* tv, int warp, int lane) {
   constexpr int OS = D + 4;
@@ -693,7 +867,7 @@ decode_persistent_kernel(const DecodeParams p, const __grid_constant__ CUtensorM
     grid_launch_dependents();
     return;
   }
-  WarpPipe<D, NW, STAGES> pipe;
+  WarpPipe<typename Core::Geom, NW, STAGES> pipe;
   pipe.init(smem, st.bars, warp, lane);
   Core core;
   const int H = p.num_kv_heads;
@@ -1069,8 +1243,71 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
 // ---------------------------------------------------------------------------
 // Grid decode: one CTA per (kv head x row chunk, sequence, split of split_blocks
 // blocks). A sequence with one split writes bf16 directly; otherwise each split
-// writes fp32 partials (o, m, l) for merge_kernel.
+// writes fp32 partials (o, m, l), adds one to its output target's arrival counter
+// (zeroed by grid_reset_kernel or the sharing pre-pass of the same call), and the CTA
+// that brings the counter to the target's split count merges the target's partials in
+// split order (so the result does not depend on which CTA finished last).
 // ---------------------------------------------------------------------------
+
+// Splits that write partials for a sequence: its shared-prefix splits (prefix sharing)
+// and the splits of its own blocks [P_b, nblk).
+struct SplitCount {
+  int shared, own;
+};
+__device__ __forceinline__ SplitCount split_count(const DecodeParams& p, int P_b, int nblk) {
+  SplitCount c;
+  c.shared = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
+  c.own = nblk > P_b ? (nblk - P_b + p.split_blocks - 1) / p.split_blocks : 0;
+  return c;
+}
+
+// Log-sum-exp merge of the partials of target rows row0 .. row0+nrows-1 of kv head kvh of
+// sequence b, in split order, to bf16: M = max_k m_k, L = sum_k l_k 2^(m_k - M),
+// out = sum_k o_k 2^(m_k - M) / L. The whole CTA; the records were written by other CTAs
+// (read through L2).
+template <int D>
+__device__ __forceinline__ void merge_target(const DecodeParams& p, int b, int kvh, int row0, int nrows,
+                                             SplitCount n) {
+  constexpr int DC = D / 8;
+  const int RQ = p.q_per_seq * p.num_q_heads;
+  const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
+  const int ns = n.shared + n.own;
+  for (int task = threadIdx.x; task < nrows * DC; task += blockDim.x) {
+    const int r = task / DC, dc = task % DC;
+    const int rr = row0 + r;
+    const int i = rr / p.group;
+    const int h = kvh * p.group + (rr - i * p.group);
+    const int rq = i * p.num_q_heads + h;
+    auto rec_of = [&](int k) -> size_t {
+      return (k < n.shared ? static_cast<size_t>(b) * p.share_splits + k
+                           : own_region + static_cast<size_t>(b) * p.num_splits + (k - n.shared)) * RQ + rq;
+    };
+    float M = -INFINITY;
+    for (int k = 0; k < ns; ++k) M = fmaxf(M, __ldcg(p.ws_ml + rec_of(k)).x);
+    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < ns; ++k) {
+      const size_t rec = rec_of(k);
+      const float2 ml = __ldcg(p.ws_ml + rec);
+      const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+      L += w * ml.y;
+      const float4* src = reinterpret_cast<const float4*>(p.ws_o + rec * D + dc * 8);
+      const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+      acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
+      acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
+    }
+    store_bf16x8(p.out + out_offset(p, b, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
+  }
+}
+
+// Zeroes the grid schedule's arrival counters of this call. It lets the decode kernel
+// launch at once (that kernel waits for this grid to complete), and zeroes only after the
+// preceding work on the stream -- possibly the previous call, still merging with these
+// counters -- has completed.
+__global__ void __launch_bounds__(256) grid_reset_kernel(int32_t* counters, int n) {
+  grid_launch_dependents();
+  grid_dependency_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) counters[i] = 0;
+}
 // Resident CTAs per SM the compiler must allow for (a register cap of 168): 3 for the
 // cores that fit without spilling; the 24- and 32-row tensor-core cores keep their
 // registers (they spill under the cap, which measured slower) and run 2 per SM.
@@ -1093,7 +1330,7 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   const int H = p.num_kv_heads;
   const int RQ = p.q_per_seq * p.num_q_heads;
   const float* ow = reinterpret_cast<const float*>(smem);
-  WarpPipe<D, NW, STAGES> pipe;
+  WarpPipe<typename Core::Geom, NW, STAGES> pipe;
   pipe.init(smem, st.bars, warp, lane);
   Core core;
 
@@ -1152,6 +1389,25 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
         dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
         if (dc == 0) p.ws_ml[rec] = make_float2(M, L2);
       }
+      // one arrival per member (target (member, kvh), one row chunk with sharing); the
+      // member whose count this completes is merged here
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x < members) {
+        const int bm = L + threadIdx.x;
+        const int4 info = __ldcg(p.seq_info + bm);
+        const SplitCount n = split_count(p, info.x, info.z);
+        const int prev = atomicAdd(p.arrive + static_cast<size_t>(bm) * H + kvh, 1);
+        st.merge[threadIdx.x] = prev == n.shared + n.own - 1 ? 1 : 0;
+      }
+      __syncthreads();
+      for (int m = 0; m < members; ++m) {
+        if (!st.merge[m]) continue;  // uniform: shared memory flag
+        __threadfence();
+        const int bm = L + m;
+        const int4 info = __ldcg(p.seq_info + bm);
+        merge_target<D>(p, bm, kvh, 0, p.rows, split_count(p, info.x, info.z));
+      }
       __syncthreads();  // shared memory is reused by the next segment
     }
     grid_launch_dependents();
@@ -1201,6 +1457,20 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
       if (dc == 0) p.ws_ml[rec] = make_float2(M, L);
     }
   }
+  if (direct) return;
+  // arrival on the target (sequence, kv head, row chunk); the CTA completing it merges
+  __threadfence();
+  __syncthreads();
+  const SplitCount n = split_count(p, P_b, nblk);  // P_b: shared prefix, or the window's first block
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(p.arrive + (static_cast<size_t>(b) * H + kvh) * p.row_chunks + rc, 1);
+    st.merge[0] = prev == n.shared + n.own - 1 ? 1 : 0;
+  }
+  __syncthreads();
+  if (st.merge[0]) {
+    __threadfence();
+    merge_target<D>(p, b, kvh, sg.row0, sg.nrows, n);
+  }
 }
 
 // Prefix sharing for the grid schedule, one warp per sequence b. Sequences are cut
@@ -1218,6 +1488,8 @@ __global__ void __launch_bounds__(128) share_prepass_kernel(const DecodeParams p
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (b >= p.num_seqs) return;
+  // this call's arrival counters of sequence b (one row chunk with sharing)
+  for (int k = lane; k < p.num_kv_heads; k += 32) p.arrive[static_cast<size_t>(b) * p.num_kv_heads + k] = 0;
   const int cap = p.share_cap;  // 2..16
   const int W0 = (b / cap) * cap;
   const int span = min(cap, p.num_seqs - W0);
@@ -1279,84 +1551,6 @@ __global__ void __launch_bounds__(128) share_prepass_kernel(const DecodeParams p
     p.seq_info[b] = make_int4(P, (b == leader && P > 0) ? members : 0, num_blocks_of(p, my_ctx), my_ctx);
 }
 
-// Log-sum-exp merge of the grid schedule's split partials. One CTA per output row
-// (sequence, query token, head) with MW warps: warp w folds splits w, w+MW, ... into
-// (M_w, L_w, acc_w) with lanes over head_dim, and the CTA combines the MW states.
-constexpr int kMergeMaxWarps = 8;
-
-template <int D>
-__global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const DecodeParams p) {
-  constexpr int DPL = D / 32;
-  __shared__ float2 s_ml[kMergeMaxWarps];
-  __shared__ __align__(16) float s_acc[kMergeMaxWarps][D];
-  grid_dependency_wait();
-  const int RQ = p.q_per_seq * p.num_q_heads;
-  const int row = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int MW = blockDim.x >> 5;
-  const int b = row / RQ;
-  const int rq = row % RQ;
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = num_blocks_of(p, ctx);
-  const int sb = p.split_blocks;
-  // records: the shared-prefix splits (region 0, with prefix sharing) then the
-  // sequence's own splits (region 1 with prefix sharing, else region 0); with a sliding
-  // window the own blocks start at the window's first block
-  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
-  const int nsh = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
-  const int ns = nsh + (nblk - P_b + sb - 1) / sb;
-  if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
-  const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
-  auto rec_of = [&](int k) -> size_t {
-    return (k < nsh ? static_cast<size_t>(b) * p.share_splits + k
-                    : own_region + static_cast<size_t>(b) * p.num_splits + (k - nsh)) * RQ + rq;
-  };
-  // this warp's maximum: its splits' (m, l) are spread over the lanes
-  float Mw = -INFINITY;
-  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[rec_of(s)].x);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(kFull, Mw, off));
-  float Lw = 0.f, acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-  for (int s = warp; s < ns; s += MW) {
-    const size_t rec = rec_of(s);
-    const float2 ml = p.ws_ml[rec];
-    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mw);
-    Lw += w * ml.y;
-    const float* src = p.ws_o + rec * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(src);
-      acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-    } else {
-      const float2 x = *reinterpret_cast<const float2*>(src);
-      acc[0] += w * x.x; acc[1] += w * x.y;
-    }
-  }
-  if (lane == 0) s_ml[warp] = make_float2(Mw, Lw);
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) s_acc[warp][lane * DPL + e] = acc[e];
-  __syncthreads();
-  float M = -INFINITY;
-  for (int w = 0; w < MW; ++w) M = fmaxf(M, s_ml[w].x);
-  float L = 0.f;
-  for (int w = 0; w < MW; ++w) L += s_ml[w].x == -INFINITY ? 0.f : s_ml[w].y * fast_exp2(s_ml[w].x - M);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  const int i = rq / p.num_q_heads;
-  const int h = rq % p.num_q_heads;
-  uint16_t* dst = p.out + out_offset(p, b, i, h, D);
-  for (int d = threadIdx.x; d < D / 2; d += blockDim.x) {
-    float v0 = 0.f, v1 = 0.f;
-    for (int w = 0; w < MW; ++w) {
-      const float wt = s_ml[w].x == -INFINITY ? 0.f : fast_exp2(s_ml[w].x - M);
-      v0 += wt * s_acc[w][2 * d];
-      v1 += wt * s_acc[w][2 * d + 1];
-    }
-    reinterpret_cast<uint32_t*>(dst)[d] = pack_bf16x2(v0 * inv, v1 * inv);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Cache write: one warp per (token, K|V) row of row_elems bf16 = row_elems*2 bytes,
 // copied in 16-byte vectors. Slots outside [0, num_slots) are skipped.
@@ -1413,6 +1607,7 @@ __device__ unsigned long long g_validate_count = 0;
 }  // namespace pa
 
 #include "pa_tcgen05.cuh"
+#include "pa_prefill.cuh"
 
 namespace pa {
 
@@ -1454,12 +1649,11 @@ cudaError_t configure_smem(Kernel kernel, int smem, unsigned long long& done_mas
   return e;
 }
 
-constexpr int kStages = 2;
-
 template <class Core, int D>
 cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& tk,
                         const CUtensorMap& tv, cudaStream_t stream, int* occupancy) {
-  constexpr int smem = DecodeSmem<D, Core::ROWS, kWarpsPerCta, kStages>::kBytes;
+  constexpr int kStages = Core::kStages;
+  constexpr int smem = DecodeSmem<typename Core::Geom, Core::ROWS, kWarpsPerCta, kStages>::kBytes;
   const dim3 block(kWarpsPerCta * 32);
   if (schedule == kSchedulePersistent) {
     auto kernel = decode_persistent_kernel<Core, D, kWarpsPerCta, kStages>;
@@ -1476,9 +1670,14 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, block.x, smem);
-  if (p.share_cap) {
+  if (p.share_cap) {  // the pre-pass also zeroes this call's arrival counters
     e = launch_pdl(share_prepass_kernel, dim3(static_cast<unsigned>((p.num_seqs + 3) / 4)), dim3(128), 0,
                    stream, p);
+    if (e != cudaSuccess) return e;
+  } else if (p.num_splits > 1) {
+    const int n = p.num_seqs * p.num_kv_heads * p.row_chunks;
+    e = launch_pdl(grid_reset_kernel, dim3(static_cast<unsigned>(min((n + 255) / 256, 32))), dim3(256), 0, stream,
+                   p.arrive, n);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
@@ -1488,12 +1687,7 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
                             static_cast<long long>(p.num_seqs) * p.num_splits);
     grid = dim3(static_cast<unsigned>(ctas));
   }
-  e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
-  if (e != cudaSuccess || (p.num_splits <= 1 && !p.share_cap)) return e;
-  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
-  // about four records per warp, at most kMergeMaxWarps warps per row
-  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + p.share_splits + 3) / 4));
-  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
+  return launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
 }
 
 template <int N>
@@ -1505,19 +1699,33 @@ cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUten
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
+  // the sharing pre-pass, or the reset kernel, zeroes this call's arrival counters first
+  const int windows = p.share_cap > 1 ? (p.num_seqs + p.share_cap - 1) / p.share_cap : p.num_seqs;
   if (p.share_cap > 1) {
-    const int windows = (p.num_seqs + p.share_cap - 1) / p.share_cap;
     e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(256), 0, stream, p);
-    if (e != cudaSuccess) return e;
+  } else {
+    const int n = windows * p.num_kv_heads * p.row_chunks;
+    e = launch_pdl(grid_reset_kernel, dim3(static_cast<unsigned>(min((n + 255) / 256, 32))), dim3(256), 0, stream,
+                   p.arrive, n);
   }
-  e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kMergeThreads), 0, stream, p);
+  return launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
 }
 
 template <int D>
-cudaError_t dispatch(int path, int schedule, int rows_per_cta, const DecodeParams& p,
+cudaError_t dispatch(int path, int schedule, int rows_per_cta, int kv_dtype, const DecodeParams& p,
                      const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, int* occ) {
+  if (kv_dtype == kKvE4M3) {  // E4M3 pools: the tensor-core tiles widen the codes to f16
+    if (path != kPathTile) return cudaErrorInvalidValue;
+    switch (rows_per_cta) {
+      case 8: return launch_core<TileCore<D, 1, true>, D>(p, schedule, tk, tv, stream, occ);
+      case 16: return launch_core<TileCore<D, 2, true>, D>(p, schedule, tk, tv, stream, occ);
+      case 24: return launch_core<TileCore<D, 3, true>, D>(p, schedule, tk, tv, stream, occ);
+      case 32: return launch_core<TileCore<D, 4, true>, D>(p, schedule, tk, tv, stream, occ);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (kv_dtype != kKvBf16) return cudaErrorInvalidValue;
   if (path == kPathTcgen05) {
     if constexpr (D != tcm::kD) {
       return cudaErrorInvalidValue;
@@ -1548,16 +1756,26 @@ cudaError_t dispatch(int path, int schedule, int rows_per_cta, const DecodeParam
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim,
-                          const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
-  return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, p, tk, tv, stream, nullptr)
-                         : dispatch<64>(path, schedule, p.rows_per_cta, p, tk, tv, stream, nullptr);
+cudaError_t launch_prefill(const PrefillParams& p, int max_tiles, const CUtensorMap& tk, const CUtensorMap& tv,
+                           cudaStream_t stream) {
+  static unsigned long long done_mask = 0;
+  cudaError_t e = configure_smem(prefill_tcm_kernel, pfl::Smem::kBytes, done_mask);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(p.num_kv_heads), static_cast<unsigned>(p.num_seqs),
+                  static_cast<unsigned>(max_tiles));
+  return launch_pdl(prefill_tcm_kernel, grid, dim3(pfl::kThreads), pfl::Smem::kBytes, stream, p, tk, tv);
 }
 
-int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta) {
+cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim, int kv_dtype,
+                          const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
+  return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, stream, nullptr)
+                         : dispatch<64>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, stream, nullptr);
+}
+
+int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, int kv_dtype) {
   // the occupancy query costs microseconds of host time: remember it per device and kernel
   struct Entry {
-    int dev, path, schedule, head_dim, rows, occ;
+    int dev, path, schedule, head_dim, rows, kv_dtype, occ;
   };
   static std::mutex mu;
   static Entry cache[64];
@@ -1568,18 +1786,19 @@ int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta) {
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
       if (cache[i].dev == dev && cache[i].path == path && cache[i].schedule == schedule &&
-          cache[i].head_dim == head_dim && cache[i].rows == rows_per_cta)
+          cache[i].head_dim == head_dim && cache[i].rows == rows_per_cta && cache[i].kv_dtype == kv_dtype)
         return cache[i].occ;
   }
   DecodeParams dummy = {};
   CUtensorMap tm = {};
   int occ = 0;
-  cudaError_t e = head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ)
-                                  : dispatch<64>(path, schedule, rows_per_cta, dummy, tm, tm, nullptr, &occ);
+  cudaError_t e =
+      head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, nullptr, &occ)
+                      : dispatch<64>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, nullptr, &occ);
   const int result = e == cudaSuccess && occ > 0 ? occ : 1;
   if (e == cudaSuccess && occ > 0 && dev >= 0) {
     std::lock_guard<std::mutex> lock(mu);
-    if (used < 64) cache[used++] = Entry{dev, path, schedule, head_dim, rows_per_cta, occ};
+    if (used < 64) cache[used++] = Entry{dev, path, schedule, head_dim, rows_per_cta, kv_dtype, occ};
   }
   return result;
 }

@@ -1,0 +1,393 @@
+// Chunked-prefill paged attention on the 5th-generation tensor cores (vLLM study notes,
+// zihan-zhang.net, §3.5 "Chunked prefill": a long prompt is attended in chunks of many
+// query tokens, batched with decode steps; "vLLM 深度解析" §5.4 Chunked Prefill). A chunk's
+// K/V are already in the paged pool (written by pa_reshape_and_cache); its query token i
+// sits at position ctx - qlen + i and sees keys 0 .. that position, i.e. the sequence's
+// earlier context plus the chunk up to itself (causal). Included by pa_kernels.cu (shares
+// its device helpers and error word).
+//
+// This is a contraction with hundreds of query rows per kv head, so the query rows go on the
+// MMA's M dimension (the decode kernels put the keys there):
+//   S[128 rows][128 keys] = Q[128 rows][D] . K^T[D][128 keys]    K-major A (Q) and B (K)
+//   softmax per row: thread r of the softmax warpgroup owns row r (TMEM lane r) and all 128
+//   keys of the tile, so the row maximum and sum need no exchange; the running reference
+//   maximum moves only when a tile's maximum exceeds it by more than 2^8 (numerator and
+//   denominator share the reference, so the result is exact either way);
+//   O[128 rows][D] += P[128 rows][128 keys] . V[128 keys][D]     K-major A (P, from shared
+//                                                                memory), MN-major B (V)
+// A CTA owns 128 rows = 128 / G consecutive chunk tokens x the G query heads of one kv head
+// (GQA: every row of a CTA reads the same K/V), and walks the key tiles of 8 blocks from
+// the sequence's first block to the block of its last row's position.
+//
+// Roles: warps 0-3 load Q, run the softmax and the epilogue; warp 4 issues the K boxes and
+// warp 5 the V boxes (16 TMA boxes of 2 KB per tile each); warp 6 holds the TMEM allocation
+// and one of its threads issues the MMAs (S of a tile as soon as its K has landed and an S
+// buffer is free; PV of a tile as soon as its P and V are in shared memory). A K stage is
+// released when its S completes, a V stage when its PV completes.
+// TMEM: S double buffer in columns [0, 256), O in [256, 384).
+// Shared memory: Q (32 KB), P (32 KB), 2 K stages and 2 V stages of 32 KB, barriers.
+
+namespace pa {
+
+namespace pfl {
+
+constexpr int kD = 128;
+constexpr int kRows = 128;                        // query rows of a CTA: the MMA's M
+constexpr int kTileBlocks = 8;
+constexpr int kKeys = kTileBlocks * kBlockSize;   // 128 keys per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 224;                     // 7 warps
+constexpr int kKWarp = 4, kVWarp = 5, kMmaWarp = 6;
+constexpr int kHalfBytes = kKeys * 128;           // one 64-column half of a K or V tile: 16 KB
+constexpr int kTileBytes = 2 * kHalfBytes;        // 32 KB
+constexpr int kRowsHalfBytes = kRows * 128;       // one 64-column half of Q or P: 16 KB
+constexpr float kRescaleLog2 = 8.f;
+constexpr uint32_t kTmemCols = 512;               // S double buffer + O, rounded to a power of 2
+constexpr uint32_t kTmemO = 2 * kKeys;            // column of O
+
+struct Smem {
+  static constexpr int offQ = 0;
+  static constexpr int offP = offQ + 2 * kRowsHalfBytes;
+  static constexpr int offK = offP + 2 * kRowsHalfBytes;
+  static constexpr int offV = offK + kStages * kTileBytes;
+  static constexpr int offBars = offV + kStages * kTileBytes;
+  static constexpr int kBytes = offBars + 256;
+  static_assert(offK % 1024 == 0 && offV % 1024 == 0 && offP % 1024 == 0, "swizzled operands");
+};
+
+struct Bars {
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], s_free[2], p_full, pv_done, q_full, drain;
+};
+
+// Byte offset of 16-byte chunk c (0..15) of row r in a 128-row operand of two 64-column
+// halves, 128-byte swizzled (the layout TMA writes for K/V and the one Q and P use).
+__device__ __forceinline__ uint32_t row_chunk_offset(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * kRowsHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+}  // namespace pfl
+
+__global__ void __launch_bounds__(pfl::kThreads, 1)
+prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v) {
+  using L = pfl::Smem;
+  using pfl::kKeys;
+  using pfl::kStages;
+  using pfl::kTileBlocks;
+  constexpr int D = pfl::kD;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  pfl::Bars& bars = *reinterpret_cast<pfl::Bars*>(smem + L::offBars);
+  uint32_t& tmem_base_s = *reinterpret_cast<uint32_t*>(smem + L::offBars + sizeof(pfl::Bars));
+  static_assert(sizeof(pfl::Bars) + 16 <= 256, "barrier area");
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1024-aligned base
+    if (threadIdx.x == 0) record_error(kErrSchedule);
+    return;
+  }
+  // grid: x = kv head, y = sequence, z = tile counted from the chunk's end (the tiles that
+  // see the most keys start first)
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y;
+  if (threadIdx.x == 0) {
+    uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
+    for (int i = 0; i < static_cast<int>(sizeof(pfl::Bars) / 8); ++i) mbar_init(all + i, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars.s_free[i], 4);  // one arrival per softmax warp
+    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.q_full, 4);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  grid_dependency_wait();
+  const int qs = __ldg(p.query_start + b);
+  const int qlen = __ldg(p.query_start + b + 1) - qs;
+  const int ctx = __ldg(p.context_lens + b);
+  const int TT = p.tile_tokens;
+  const int ntiles = qlen > 0 ? (qlen + TT - 1) / TT : 0;
+  const int rt = static_cast<int>(blockIdx.z);
+  // nothing to do: past the chunk's tiles, or a context shorter than the chunk (a
+  // precondition violation; no position would be valid)
+  if (rt >= ntiles || ctx < qlen) {
+    grid_launch_dependents();
+    return;
+  }
+  const int tile = ntiles - 1 - rt;
+  const int tok0 = tile * TT;
+  const int ntok = min(TT, qlen - tok0);
+  const int pos0 = ctx - qlen + tok0;          // position of the CTA's first token
+  const int kmax = pos0 + ntok - 1;            // position of its last token: the last key seen
+  const int nk = kmax / kKeys + 1;             // key tiles 0 .. nk-1
+  const int nblk = min((ctx + kBlockSize - 1) / kBlockSize, p.max_blocks);
+
+  if (warp == pfl::kMmaWarp) {
+    tmem_alloc(&tmem_base_s, pfl::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = tmem_base_s;
+  const uint32_t sm = smem_u32(smem);
+
+  if (warp == pfl::kKWarp || warp == pfl::kVWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // lanes 0..15 issue the tile's 16 boxes (half = lane / 8, block = lane % 8); lanes 0..7
+    // read the next tile's block ids while this one is issued
+    const bool is_k = warp == pfl::kKWarp;
+    const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+    uint64_t* full = is_k ? bars.k_full : bars.v_full;
+    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+    const int stage_off = is_k ? L::offK : L::offV;
+    const int32_t* trow = p.block_tables + static_cast<size_t>(b) * p.max_blocks;
+    const int oob = static_cast<int>(p.num_blocks);  // block id past the pool: TMA fills zeros
+    auto block_id = [&](int j) {
+      const int blk = j * kTileBlocks + lane;
+      return (lane < kTileBlocks && blk < nblk) ? __ldg(trow + blk) : oob;
+    };
+    int phys_next = block_id(0);
+    bool ok = true;
+    int j = 0;
+    for (; j < nk; ++j) {
+      const int s = j % kStages;
+      const int ph = __shfl_sync(kFull, phys_next, lane & (kTileBlocks - 1));
+      if (j + 1 < nk) phys_next = block_id(j + 1);
+      if (j >= kStages) ok = __all_sync(kFull, mbar_wait_bounded(&empty[s], ((j / kStages) - 1) & 1));
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], pfl::kTileBytes);
+      __syncwarp();
+      const int hf = lane >> 3, jj = lane & (kTileBlocks - 1);
+      if (lane < 2 * kTileBlocks)
+        tma_load_3d(smem + stage_off + s * pfl::kTileBytes + hf * pfl::kHalfBytes + jj * kHalfTileBytes, tmap,
+                    &full[s], hf * 64, kvh, ph * kBlockSize);
+      __syncwarp();
+    }
+    if (!ok) {
+      if (lane == 0) record_error(kErrTimeoutDecode);
+      for (int u = max(0, j - kStages); u < j; ++u)
+        if (!mbar_wait_bounded(&full[u % kStages], (u / kStages) & 1) && lane == 0) record_error(kErrTimeoutDrain);
+    }
+  } else if (warp == pfl::kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, 0, 0);  // Q K-major, K K-major
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
+    int gs = 0, gp = 0;  // next tile to issue S for / PV for
+    bool ok = true;
+    unsigned long long idle_since = 0;
+    unsigned idle_polls = 0;
+    // slots of the sequence's partly filled last block past the context: V rows to clear
+    // before the PV of the tile holding that block (their p is 0, but 0 * NaN is NaN)
+    const int last_blk = nblk - 1;
+    const int last_fill = ctx - last_blk * kBlockSize;  // 1..16 tokens used in the last block
+    while (gp < nk) {
+      bool progressed = false;
+      bool pv_ready = false;
+      if (lane == 0)
+        pv_ready = gp < gs && mbar_test_wait(&bars.p_full, gp & 1) &&
+                   mbar_test_wait(&bars.v_full[gp % kStages], (gp / kStages) & 1);
+      if (__shfl_sync(kFull, pv_ready, 0)) {
+        const int jj = last_blk - gp * kTileBlocks;
+        if (last_fill < kBlockSize && jj >= 0 && jj < kTileBlocks) {
+          mbar_test_wait(&bars.v_full[gp % kStages], (gp / kStages) & 1);  // every lane sees the data
+          uint8_t* vblk = smem + L::offV + (gp % kStages) * pfl::kTileBytes + jj * kHalfTileBytes;
+          const int nrow = kBlockSize - last_fill;
+          for (int idx = lane; idx < 2 * nrow * 8; idx += 32) {
+            const int hf = idx / (nrow * 8);
+            const int rem = idx - hf * (nrow * 8);
+            *reinterpret_cast<uint4*>(vblk + hf * pfl::kHalfBytes + (last_fill + (rem >> 3)) * 128 + (rem & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          tc_fence_after_sync();
+          const uint32_t vst = sm + L::offV + (gp % kStages) * pfl::kTileBytes;
+          const uint32_t pst = sm + L::offP;
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk) {
+            // A = P: keys 16kk .. 16kk+15 of each row (K-major, 128-byte swizzle, two halves)
+            const uint64_t ad = smem_desc_sw128(pst + (kk >> 2) * pfl::kRowsHalfBytes + (kk & 3) * 32, 16, 1024);
+            // B = V: keys 16kk .. 16kk+15 (rows of the tile) x all D columns (MN-major)
+            const uint64_t bd = smem_desc_sw128(vst + kk * 2048, pfl::kHalfBytes, 1024);
+            tc_mma_bf16(tmem + pfl::kTmemO, ad, bd, idesc_o, (gp == 0 && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(&bars.pv_done);
+          tc_commit(&bars.v_empty[gp % kStages]);
+        }
+        __syncwarp();
+        ++gp;
+        progressed = true;
+      }
+      if (gs < nk && gs < gp + 3) {  // S of tile j+2 may run while the softmax of tile j does
+        const int s = gs % kStages;
+        bool s_ready = false;
+        if (lane == 0)
+          s_ready = (gs > 0 || mbar_test_wait(&bars.q_full, 0)) &&
+                    mbar_test_wait(&bars.k_full[s], (gs / kStages) & 1) &&
+                    (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1));
+        if (__shfl_sync(kFull, s_ready, 0)) {
+          if (lane == 0) {
+            tc_fence_after_sync();
+            const uint32_t kst = sm + L::offK + s * pfl::kTileBytes;
+            const uint32_t qst = sm + L::offQ;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(qst + (k >> 2) * pfl::kRowsHalfBytes + (k & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(kst + (k >> 2) * pfl::kHalfBytes + (k & 3) * 32, 16, 1024);
+              tc_mma_bf16(tmem + (gs & 1) * kKeys, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars.s_full[gs & 1]);
+            tc_commit(&bars.k_empty[s]);
+          }
+          __syncwarp();
+          ++gs;
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        idle_since = 0;
+        idle_polls = 0;
+      } else if ((++idle_polls & 63) == 0) {  // the clock is read once every 64 idle polls
+        const unsigned long long now = __shfl_sync(kFull, global_timer_ns(), 0);
+        if (idle_since == 0) {
+          idle_since = now;
+        } else if (now - idle_since > kWaitLimitNs) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (!ok) record_error(kErrTimeoutDecode);
+      tc_commit(&bars.drain);  // every MMA issued so far has completed once drain flips
+      if (!mbar_wait_bounded(&bars.drain, 0)) record_error(kErrTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ Q, softmax, epilogue
+    const int r = threadIdx.x;                 // row = TMEM lane
+    const int tt = r / p.group;                // chunk token of the row (within the CTA)
+    const int h = kvh * p.group + (r - tt * p.group);
+    const bool valid = tt < ntok;
+    const int pos = valid ? pos0 + tt : -1;    // the row's position: keys 0 .. pos visible
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const size_t row_off = (static_cast<size_t>(qs + tok0 + tt) * p.num_q_heads + h) * D;
+    {  // Q row -> shared memory, 128-byte swizzled K-major; zeros for rows past the chunk
+      const uint4* src = reinterpret_cast<const uint4*>(p.query + row_off);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + L::offQ + pfl::row_chunk_offset(r, c)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.q_full);
+    }
+    const float cs = p.scale_log2;
+    float mref = -INFINITY, l = 0.f;
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok) ok = __all_sync(kFull, mbar_wait_bounded(bar, parity));
+    };
+    for (int j = 0; j < nk; ++j) {
+      wait(&bars.s_full[j & 1], (j >> 1) & 1);
+      tc_fence_after_sync();
+      uint32_t sv[kKeys];
+#pragma unroll
+      for (int q4 = 0; q4 < kKeys / 32; ++q4)
+        tmem_ld32(tmem + lane_off + (j & 1) * kKeys + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + q4 * 32));
+      tc_wait_ld();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
+      // keys past the row's position are masked (the chunk is causal; keys past every row's
+      // position are past the context or belong to later chunk tokens)
+      const int k0 = j * kKeys;
+      const bool edge = k0 + kKeys - 1 > pos;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kKeys; ++k) {
+        float x = __uint_as_float(sv[k]) * cs;
+        if (edge && k0 + k > pos) x = -INFINITY;
+        sv[k] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      // move the reference when the tile's maximum exceeds it by more than 2^8; O (TMEM) is
+      // rescaled by the whole warp whenever one of its rows moved (tcgen05.ld/st are
+      // warp-collective), the other rows by 1
+      const bool need = mx > mref + pfl::kRescaleLog2 || (mref == -INFINITY && mx != -INFINITY);
+      float alpha = 1.f;
+      if (need) {
+        alpha = mref == -INFINITY ? 0.f : fast_exp2(mref - mx);
+        l *= alpha;
+      }
+      if (__any_sync(kFull, need && j > 0 && mref != -INFINITY)) {
+        // O holds the earlier tiles once the PV of tile j-1 has completed
+        wait(&bars.pv_done, (j - 1) & 1);
+        tc_fence_after_sync();
+#pragma unroll
+        for (int q4 = 0; q4 < D / 32; ++q4) {
+          uint32_t ov[32];
+          const uint32_t oaddr = tmem + lane_off + pfl::kTmemO + q4 * 32;
+          tmem_ld32(oaddr, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(oaddr, ov);
+        }
+        tc_wait_st();
+      }
+      if (need) mref = mx;
+      const float mu = mref == -INFINITY ? 0.f : mref;
+      uint32_t pk[kKeys / 2];
+#pragma unroll
+      for (int k = 0; k < kKeys; k += 2) {
+        const float p0 = fast_exp2(__uint_as_float(sv[k]) - mu);
+        const float p1 = fast_exp2(__uint_as_float(sv[k + 1]) - mu);
+        l += p0 + p1;
+        pk[k / 2] = pack_bf16x2(p0, p1);
+      }
+      // the P buffer was read by the PV of tile j-1
+      if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
+#pragma unroll
+      for (int c = 0; c < kKeys / 8; ++c)
+        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, c)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.p_full);
+    }
+    // ---- epilogue: O / l once the last PV has completed
+    wait(&bars.pv_done, (nk - 1) & 1);
+    tc_fence_after_sync();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + row_off);
+#pragma unroll
+    for (int q4 = 0; q4 < D / 32; ++q4) {
+      uint32_t ov[32];
+      tmem_ld32(tmem + lane_off + pfl::kTmemO + q4 * 32, ov);
+      tc_wait_ld();
+      if (ok && valid) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          dst[q4 * 4 + c] = make_uint4(
+              pack_bf16x2(__uint_as_float(ov[8 * c]) * inv, __uint_as_float(ov[8 * c + 1]) * inv),
+              pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv),
+              pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv),
+              pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv));
+      }
+    }
+    tc_fence_before_sync();
+    if (!ok && lane == 0) record_error(kErrTimeoutDecode);
+  }
+  grid_launch_dependents();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == pfl::kMmaWarp) tmem_dealloc(tmem, pfl::kTmemCols);
+}
+
+}  // namespace pa

@@ -8,8 +8,9 @@
 // walk the same enumeration of (sequence, kv-head index, row chunk, tile) and split it
 // into equal contiguous ranges, one per group, computed in the kernel from context_lens
 // (no pre-pass); the S CTAs of a group therefore read the kv-head slices of the same
-// blocks at about the same time. A unit cut by a range boundary leaves partial records,
-// combined afterwards by tcm_merge_kernel.
+// blocks at about the same time. A unit cut by range boundaries leaves one partial record
+// per piece; at its end every CTA adds one to the arrival counter of each cut unit it holds
+// a piece of, and the CTA whose arrival completes the unit merges its pieces in CTA order.
 //
 // Per tile, with Q of the unit's N (16 or 32) rows:
 //   S^T[128 tok][N]  = K[128 tok][D] . Q^T[D][N]           tcgen05.mma M=128, K-major A and B
@@ -48,7 +49,6 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
 constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
-constexpr int kMergeThreads = 1024;  // one warp per row of a unit (N <= 32)
 
 template <int N>
 struct Smem {
@@ -61,7 +61,7 @@ struct Smem {
   // per softmax warpgroup: [3][4 warps][N/2] floats (2 maxima buffers, 1 sum), [2][4] votes
   static constexpr int kRedWg = 3 * 4 * (N / 2) + 8;
   static constexpr int offRed = offV + kVStages * kStageBytes;
-  static constexpr int offScan = offRed + 2 * kRedWg * 4;     // [11] int64, then the start
+  static constexpr int offScan = offRed + 2 * kRedWg * 4;     // [11] int64, the start, 2 merge flags
   static constexpr int offBars = offScan + 128;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && kQ % 1024 == 0, "swizzled operands need 1024-B alignment");
@@ -81,8 +81,12 @@ __device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
   if (m <= 0) return 0;
   const int P = cap > 1 ? __ldg(p.win_prefix + w) : 0;
   int tiles = (P + kTileBlocks - 1) / kTileBlocks;
-  for (int jj = 0; jj < m; ++jj)
-    tiles += (num_blocks_of(p, __ldg(p.context_lens + b0 + jj)) - P + kTileBlocks - 1) / kTileBlocks;
+  for (int jj = 0; jj < m; ++jj) {
+    const int cx = __ldg(p.context_lens + b0 + jj);
+    const int nb = num_blocks_of(p, cx);
+    // own blocks: after the shared prefix, from the sliding window's first block on
+    tiles += (nb - min(nb, max(P, window_first_block(p, cx))) + kTileBlocks - 1) / kTileBlocks;
+  }
   return tiles;
 }
 
@@ -90,21 +94,23 @@ __device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
 // sequences (cap = 1 without prefix sharing) whose tables may start with the same P
 // physical blocks; its units are (kv-head index, row chunk) of this CTA, and every unit
 // walks the window's tiles: the shared prefix (P blocks, read once for all members) then
-// each member's own blocks. Lane jj holds member jj's context length and blocks, so moving
-// between members takes shuffles, not loads.
+// each member's own blocks (with a sliding window, from its window's first block). Lane jj
+// holds member jj's context length and blocks, so moving between members takes shuffles,
+// not loads.
 struct Walk {
   int w, k, x;          // window, unit of the window, tile of the unit
   int b0, m, P, tiles;  // window: first sequence, members, shared blocks, tiles of a unit
   int j, y, seg;        // segment: member j (-1: the shared prefix), its tile y, its tiles
-  int ctx, nblk;        // member j: context length (clamped to its blocks) and blocks
-  int lctx, lnblk;      // this lane's member
+  int ctx, nblk, lo;    // member j: context length (clamped to its blocks), blocks, first own block
+  int lctx, lnblk, llo; // this lane's member
 
   __device__ __forceinline__ int own_tiles_lane() const {
-    return (lnblk - P + kTileBlocks - 1) / kTileBlocks;
+    return (lnblk - llo + kTileBlocks - 1) / kTileBlocks;
   }
   __device__ __forceinline__ void member(int jj) {
     ctx = __shfl_sync(kFull, lctx, jj);
     nblk = __shfl_sync(kFull, lnblk, jj);
+    lo = __shfl_sync(kFull, llo, jj);
   }
   __device__ __forceinline__ void window(const DecodeParams& p) {
     const int lane = threadIdx.x & 31;
@@ -114,11 +120,13 @@ struct Walk {
     tiles = 0;
     lctx = 0;
     lnblk = 0;
+    llo = 0;
     if (m <= 0) return;
     P = cap > 1 ? __ldg(p.win_prefix + w) : 0;
     if (lane < m) {
       lctx = __ldg(p.context_lens + b0 + lane);
       lnblk = num_blocks_of(p, lctx);
+      llo = min(lnblk, max(P, window_first_block(p, lctx)));
       lctx = min(lctx, lnblk * kBlockSize);
     }
     int t = lane < m ? own_tiles_lane() : 0;
@@ -183,7 +191,7 @@ struct Walk {
   }
   // the tile's blocks: [bstart, bend) of table row `row`
   __device__ __forceinline__ int row() const { return b0 + (j < 0 ? 0 : j); }
-  __device__ __forceinline__ int bstart() const { return (j < 0 ? 0 : P) + kTileBlocks * y; }
+  __device__ __forceinline__ int bstart() const { return (j < 0 ? 0 : lo) + kTileBlocks * y; }
   __device__ __forceinline__ int bend() const { return j < 0 ? P : nblk; }
 };
 
@@ -191,6 +199,9 @@ struct Walk {
 __device__ __forceinline__ void named_sync_softmax(int wg) {
   asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
 }
+
+// Named barrier of both softmax warpgroups (id 3, 256 threads).
+__device__ __forceinline__ void named_sync_softmax_all() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
 
 // Column reduction of a warp: lane l holds V values (columns 0..V-1); on return every
 // lane holds the reduction over all 32 lanes of column (l % V). Halving exchange: at
@@ -239,10 +250,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1024-aligned base
-    if (threadIdx.x == 0) {
-      record_error(kErrSchedule);
-      p.tc_desc[c] = make_int4(-1, 0, 0, 0);
-    }
+    if (threadIdx.x == 0) record_error(kErrSchedule);
     return;
   }
   if (threadIdx.x == 0) {
@@ -309,9 +317,15 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     }
     __syncthreads();
   }
+  // sequences without a visible key (context length 0) get zero rows
+  for (int b = c; b < p.num_seqs; b += gridDim.x) {
+    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;  // uniform
+    const int rq = p.q_per_seq * p.num_q_heads;
+    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * rq * D);
+    for (int e = threadIdx.x; e < rq * D / 8; e += blockDim.x) o[e] = make_uint4(0, 0, 0, 0);
+  }
   const int n = static_cast<int>(t1 - t0);
   if (n <= 0) {  // uniform: no tiles for this CTA
-    if (threadIdx.x == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     grid_launch_dependents();
     return;
   }
@@ -421,6 +435,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       int gs = 0, gp = 0;    // next tile to issue S for / PV for (gp <= gs <= gp + 3)
       int ring = 0;          // per tile in flight: bit 2(g&3) O buffer, bit 2(g&3)+1 first of unit
       int zring = 0;         // per tile in flight, byte g&3: V rows to clear (bit 0 on, block, row)
+      int hring = 0;         // per tile in flight, byte g&3: sliding window, rows 0 .. r-1 of the
+                             // tile's first block to clear (bit 0 on, r)
+      const int win = p.window;
       bool ok = true;
       unsigned long long idle_since = 0;
       unsigned idle_polls = 0;
@@ -432,6 +449,22 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
                      mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1);
         if (__shfl_sync(kFull, pv_ready, 0)) {
           const int z = (zring >> (8 * (gp & 3))) & 0xFF;
+          const int zh = (hring >> (8 * (gp & 3))) & 0xFF;
+          if (zh & 1) {
+            // Sliding window: the slots of a member's first block before its first row's
+            // window start are seen by no row and may hold any bits; cleared like the tail.
+            mbar_test_wait(&bars.v_full[gp % kVStages], (gp / kVStages) & 1);  // every lane sees the data
+            const int nrow = zh >> 1;
+            uint8_t* vblk = smem + L::offV + (gp % kVStages) * tcm::kStageBytes;
+            for (int idx = lane; idx < 2 * nrow * 8; idx += 32) {
+              const int hf = idx / (nrow * 8);
+              const int rem = idx - hf * (nrow * 8);
+              *reinterpret_cast<uint4*>(vblk + hf * tcm::kHalfBytes + (rem >> 3) * 128 + (rem & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
           if (z & 1) {
             // A member's last block is partly filled: its slots past the context may hold any
             // bits (NaN too), and although their p is 0, 0 * NaN is NaN, so those V rows are
@@ -502,6 +535,12 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
             if (w.j >= 0 && w.y == w.seg - 1 && (w.ctx & (kBlockSize - 1)))
               z = 1 | (((w.nblk - 1) - w.bstart()) << 1) | ((w.ctx & (kBlockSize - 1)) << 4);
             zring = (zring & ~(0xFF << (8 * (gs & 3)))) | (z << (8 * (gs & 3)));
+            int zh = 0;
+            if (win > 0 && w.j >= 0 && w.y == 0) {
+              const int r1 = max(0, w.ctx - p.q_per_seq - win + 1) - w.lo * kBlockSize;
+              if (r1 > 0) zh = 1 | (r1 << 1);
+            }
+            hring = (hring & ~(0xFF << (8 * (gs & 3)))) | (zh << (8 * (gs & 3)));
             w.next(p, upb, nwin);
             ++gs;
             progressed = true;
@@ -537,6 +576,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     float* red = reinterpret_cast<float*>(smem + L::offRed) + wg * L::kRedWg;
     int* votes = reinterpret_cast<int*>(red + 3 * 4 * NC);  // [2][4 warps]
     const float cs = p.scale_log2;
+    const int win = p.window;  // sliding window (keys lim - win + 1 .. lim of a row), 0 = none
     tcm::Walk w = w0;
     int j = -1, first_x = 0, kvh = 0, rc = 0, nrows = 0, minlim = 0;
     float mref_c = -INFINITY;  // reference maximum of column cb + (lane % NC)
@@ -556,6 +596,12 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       float L_c, m_c;  // l and the reference maximum of column cb + (lane % NC)
     } pend;
     pend.on = false;
+    // The cut units this CTA holds a piece of (its first unit and its last one, at most):
+    // counter index, the unit's first and last group, and the record slot of the first piece.
+    struct Cut {
+      int idx, gi_first, gi_last, first_slot, w, k;
+    } cut[2];
+    int ncut = 0;
     auto flush = [&](Pending& e) {
       e.on = false;
       wait(&bars.pv_done[e.g & 1], (e.g >> 1) & 1);
@@ -652,13 +698,16 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         lo = max(0, w.j * rpm - rc * N - cb);
         hi = min(NC, (w.j + 1) * rpm - rc * N - cb);
       } else {
-        edge = tok0 + kTileTokens - 1 > minlim;
+        // past the first row's last key, or (sliding window) before the last row's first key
+        edge = tok0 + kTileTokens - 1 > minlim || (win > 0 && tok0 + win <= w.ctx - 1);
       }
       float x[NC], tmp[NC];
 #pragma unroll
       for (int r = 0; r < NC; ++r) {
         float v = __uint_as_float(sv[r]) * cs;
-        if (edge && (r < lo || r >= hi || tok >= tok_hi || (use_lim && tok > lim[r]))) v = -INFINITY;
+        if (edge && (r < lo || r >= hi || tok >= tok_hi ||
+                     (use_lim && (tok > lim[r] || (win > 0 && tok + win <= lim[r])))))
+          v = -INFINITY;
         x[r] = v;
         tmp[r] = v;
       }
@@ -749,15 +798,21 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         pend.slot = j == 0 ? 2 * c : 2 * c + 1;
         pend.L_c = (rl[jc] + rl[NC + jc]) + (rl[2 * NC + jc] + rl[3 * NC + jc]);
         pend.m_c = mref_c;
-        if (g == n - 1 && wg == 0 && t == 0) {
-          // the merge descriptor: this CTA's last unit continues in the next CTAs and
-          // started here, so this CTA holds its first piece
-          int4 dsc = make_int4(-1, 0, 0, 0);
-          if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
-            const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
-            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.w, w.k);
-          }
-          p.tc_desc[c] = dsc;
+        if (!pend.complete) {
+          // a piece of a cut unit: the unit's global tiles are [Tf, E); the group holding
+          // global tile T is ((T + 1) * NGe - 1) / W; its first piece sits in the first
+          // group's slot 2c (the unit starts that CTA's range) or 2c + 1, later pieces in
+          // slot 2c of their CTA (the unit is their first)
+          const long long Tf = t0 + g - w.x;
+          const long long E = Tf + w.tiles;
+          Cut& cu = cut[ncut++];
+          cu.gi_first = static_cast<int>(((Tf + 1) * NGe - 1) / W);
+          cu.gi_last = static_cast<int>((E * NGe - 1) / W);
+          const int cf = cu.gi_first * S + li;
+          cu.first_slot = Tf == static_cast<long long>(cu.gi_first) * W / NGe ? 2 * cf : 2 * cf + 1;
+          cu.idx = (w.w * p.num_kv_heads + kvh) * p.row_chunks + rc;
+          cu.w = w.w;
+          cu.k = w.k;
         }
       }
       w.next(p, upb, nwin);
@@ -765,7 +820,62 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     if (pend.on) flush(pend);
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
-      if (wg == 0 && t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
+    } else if (ncut > 0) {
+      // ---- arrivals on the cut units; the CTA completing a unit merges its pieces in CTA
+      // order (a fixed order: the result does not depend on which CTA arrived last)
+      __threadfence();  // this CTA's records are visible device-wide before its arrival
+      tcm::named_sync_softmax_all();
+      int* flag = reinterpret_cast<int*>(smem + L::offScan + 104);  // after the range start
+      for (int q = 0; q < ncut; ++q) {
+        if (warp == 0 && lane == 0) {
+          const int prev = atomicAdd(p.arrive + cut[q].idx, 1);
+          flag[q] = prev == cut[q].gi_last - cut[q].gi_first ? 1 : 0;
+        }
+      }
+      tcm::named_sync_softmax_all();
+      for (int q = 0; q < ncut; ++q) {
+        if (!flag[q]) continue;  // uniform: shared memory flag
+        __threadfence();
+        const Cut cu = cut[q];
+        const int np = cu.gi_last - cu.gi_first + 1;
+        const int b0 = cu.w * cap;
+        const int m = min(cap, p.num_seqs - b0);
+        const int kvh_u = unit_kvh(cu.k), rc_u = unit_rc(cu.k);
+        const int nr = min(N, m * rpm - rc_u * N);
+        const float* recs = p.records;
+        const int rs = p.rec_stride;
+        auto rec_of = [&](int k) {
+          return recs + static_cast<size_t>(k == 0 ? cu.first_slot : 2 * ((cu.gi_first + k) * S + li)) * rs;
+        };
+        const int tid = threadIdx.x;  // the 256 softmax threads
+        for (int task = tid; task < nr * (D / 4); task += tcm::kSoftmaxWarps * 32) {
+          const int r = task / (D / 4), c4 = task % (D / 4);
+          float M = -INFINITY;
+          for (int k = 0; k < np; ++k) M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(rec_of(k) + N * D) + r).x);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          float l = 0.f;
+          for (int k = 0; k < np; ++k) {
+            const float* rk = rec_of(k);
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(rk + N * D) + r);
+            const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+            l += ml.y * wk;
+            const float4 o4 = __ldcg(reinterpret_cast<const float4*>(rk + r * D) + c4);
+            acc.x = fmaf(o4.x, wk, acc.x);
+            acc.y = fmaf(o4.y, wk, acc.y);
+            acc.z = fmaf(o4.z, wk, acc.z);
+            acc.w = fmaf(o4.w, wk, acc.w);
+          }
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          const int cg = rc_u * N + r;
+          const int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+          const int gg = cg - mem * rpm - i * p.group;
+          uint2 packed;
+          packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+          packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+          reinterpret_cast<uint2*>(p.out + (static_cast<size_t>((b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
+                                            kvh_u * p.group + gg) * D)[c4] = packed;
+        }
+      }
     }
   }
   grid_launch_dependents();
@@ -773,94 +883,6 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   __syncthreads();
   tc_fence_after_sync();
   if (warp == tcm::kMmaWarp) tmem_dealloc(tmem, 4 * N < 32 ? 32 : 4 * N);
-}
-
-// Combines the partial records of every unit (window, kv head, row chunk) cut by a range
-// boundary (one CTA per
-// decode CTA; the descriptor of CTA c names the unit whose first piece c holds and the
-// last CTA c1 with a piece of it: the pieces are in record slots desc.x, then 2c' for
-// c' = c+S, c+2S, ..., c1 (the same CTA of the following groups), in that order), then
-// writes zeros for sequences with no keys.
-template <int N>
-__global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const DecodeParams p) {
-  constexpr int D = tcm::kD;
-  grid_dependency_wait();
-  const int c = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int4 dsc = p.tc_desc[c];
-  if (dsc.x >= 0) {
-    const int cap = p.share_cap > 1 ? p.share_cap : 1;
-    const int rpm = p.rows;
-    const int b0 = dsc.z * cap;  // the window's first sequence
-    const int m = min(cap, p.num_seqs - b0);
-    const int S = p.tc_group;
-    const int kvh = c % S + S * (dsc.w / p.row_chunks);
-    const int rc = dsc.w % p.row_chunks;
-    const int nrows = min(N, m * rpm - rc * N);
-    const int pieces = 1 + (dsc.y - c) / S;
-    const float* recs = p.records;
-    const int rs = p.rec_stride, slot0 = dsc.x;
-    auto rec_of = [=](int k) {
-      return recs + static_cast<size_t>(k == 0 ? slot0 : 2 * (c + k * S)) * rs;
-    };
-    // one row per warp: lanes take the pieces for the maximum and the weights, then each
-    // lane accumulates 4 of the D columns over the pieces in order, 4 pieces' loads at a time
-    for (int r = warp; r < nrows; r += tcm::kMergeThreads / 32) {
-      float M = -INFINITY;
-      for (int k = lane; k < pieces; k += 32) M = fmaxf(M, reinterpret_cast<const float2*>(rec_of(k) + N * D)[r].x);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float l = 0.f;
-      if (M != -INFINITY) {
-        for (int k0 = 0; k0 < pieces; k0 += 32) {
-          float wk = 0.f, lk = 0.f;
-          if (k0 + lane < pieces) {
-            const float2 ml = reinterpret_cast<const float2*>(rec_of(k0 + lane) + N * D)[r];
-            wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
-            lk = ml.y * wk;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
-          l += lk;
-          const int kn = min(32, pieces - k0);
-          for (int kk = 0; kk < kn; kk += 4) {
-            float4 o4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              o4[u] = kk + u < kn ? reinterpret_cast<const float4*>(rec_of(k0 + kk + u) + r * D)[lane]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float wb = __shfl_sync(kFull, wk, (kk + u) & 31);
-              if (kk + u < kn) {
-                acc.x = fmaf(o4[u].x, wb, acc.x);
-                acc.y = fmaf(o4[u].y, wb, acc.y);
-                acc.z = fmaf(o4[u].z, wb, acc.z);
-                acc.w = fmaf(o4[u].w, wb, acc.w);
-              }
-            }
-          }
-        }
-      }
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int cg = rc * N + r;
-      const int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
-      const int gg = cg - mem * rpm - i * p.group;
-      uint2 packed;
-      packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-      packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-      reinterpret_cast<uint2*>(p.out + (static_cast<size_t>((b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
-                                        kvh * p.group + gg) * D)[lane] = packed;
-    }
-  }
-  // sequences without a visible key (context length 0) get zero rows
-  const int rq = p.q_per_seq * p.num_q_heads;
-  for (int b = c; b < p.num_seqs; b += gridDim.x) {
-    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;
-    uint16_t* o = p.out + static_cast<size_t>(b) * rq * D;
-    for (int e = threadIdx.x; e < rq * D; e += blockDim.x) o[e] = 0;
-  }
 }
 
 // Prefix sharing: the shared prefix of each window of `cap` consecutive sequences, in
@@ -879,6 +901,9 @@ __global__ void __launch_bounds__(256) tcm_share_prepass(const DecodeParams p) {
     first_diff = INT_MAX;
     pcap_s = m >= 2 ? INT_MAX : 0;
   }
+  // this call's arrival counters of the window's units
+  for (int k = threadIdx.x; k < p.num_kv_heads * p.row_chunks; k += blockDim.x)
+    p.arrive[static_cast<size_t>(w) * p.num_kv_heads * p.row_chunks + k] = 0;
   __syncthreads();
   if (m >= 2 && static_cast<int>(threadIdx.x) < m) {  // thread jj: member jj (cap <= 32)
     const int cx = __ldg(p.context_lens + b0 + threadIdx.x);

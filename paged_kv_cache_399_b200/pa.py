@@ -33,7 +33,8 @@ PA_PATH_SINGLE = 1
 PA_PATH_TILE = 2
 PA_PATH_TCGEN05 = 3
 
-EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode",
+EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode", "pa_decode_fp8",
+            "pa_prefill",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
             "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_status_string",
             "pa_version"]
@@ -45,11 +46,14 @@ PA_SCHEDULE_AUTO = 0
 PA_SCHEDULE_GRID = 1
 PA_SCHEDULE_PERSISTENT = 2
 
+PA_KV_BF16 = 0
+PA_KV_FP8_E4M3 = 1
+
 
 class pa_plan_hints_t(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("schedule", ctypes.c_int32),
                 ("split_blocks", ctypes.c_int32), ("share_prefix", ctypes.c_int32),
-                ("sliding_window", ctypes.c_int32)]
+                ("sliding_window", ctypes.c_int32), ("kv_cache_dtype", ctypes.c_int32)]
 
 
 class pa_plan_t(ctypes.Structure):
@@ -57,7 +61,7 @@ class pa_plan_t(ctypes.Structure):
                 ("split_blocks", ctypes.c_int32), ("num_splits", ctypes.c_int32),
                 ("rows_per_cta", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
                 ("share_cap", ctypes.c_int32), ("share_split_blocks", ctypes.c_int32),
-                ("sliding_window", ctypes.c_int32)]
+                ("sliding_window", ctypes.c_int32), ("kv_cache_dtype", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {"path": {1: "single", 2: "tile", 3: "tcgen05"}.get(self.path, self.path),
@@ -65,7 +69,8 @@ class pa_plan_t(ctypes.Structure):
                 "split_blocks": self.split_blocks, "num_splits": self.num_splits,
                 "rows_per_cta": self.rows_per_cta, "num_ctas": self.num_ctas,
                 "share_cap": self.share_cap, "share_split_blocks": self.share_split_blocks,
-                "sliding_window": self.sliding_window}
+                "sliding_window": self.sliding_window,
+                "kv_cache_dtype": {0: "bf16", 1: "fp8_e4m3"}.get(self.kv_cache_dtype, self.kv_cache_dtype)}
 
     def __repr__(self):
         return f"pa_plan_t({self.as_dict()})"
@@ -90,6 +95,13 @@ _lib.pa_decode_workspace_size.argtypes = [ctypes.POINTER(pa_plan_t), _I32, _I32,
 _lib.pa_decode.restype = _I32
 _lib.pa_decode.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
                            ctypes.c_float, ctypes.POINTER(pa_plan_t), _P, ctypes.c_size_t, _P]
+_lib.pa_decode_fp8.restype = _I32
+_lib.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
+                               ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.POINTER(pa_plan_t), _P,
+                               ctypes.c_size_t, _P]
+_lib.pa_prefill.restype = _I32
+_lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
+                            ctypes.c_float, _P]
 _lib.pa_decode_static_scratch.restype = _I32
 _lib.pa_decode_static_scratch.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32,
                                           _I32, _I64, ctypes.c_float, ctypes.POINTER(pa_plan_t), _P]
@@ -196,12 +208,14 @@ def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: 
 def pa_decode_plan(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int,
                    head_dim: int, max_blocks_per_seq: int, path: int = PA_PATH_AUTO,
                    split_blocks: int = 0, schedule: int = PA_SCHEDULE_AUTO,
-                   share_prefix: bool = False, sliding_window: int = 0) -> pa_plan_t:
+                   share_prefix: bool = False, sliding_window: int = 0,
+                   kv_cache_dtype: int = PA_KV_BF16) -> pa_plan_t:
     """A forced split length implies the grid schedule (the tcgen05 path has no split
     length: its schedule cuts the work into equal tile ranges, and ignores it)."""
     if split_blocks and schedule == PA_SCHEDULE_AUTO and path != PA_PATH_TCGEN05:
         schedule = PA_SCHEDULE_GRID
-    hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)), int(sliding_window))
+    hints = pa_plan_hints_t(path, schedule, split_blocks, int(bool(share_prefix)), int(sliding_window),
+                            int(kv_cache_dtype))
     plan = pa_plan_t()
     st = _lib.pa_decode_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
                              max_blocks_per_seq, ctypes.byref(hints), ctypes.byref(plan))
@@ -238,6 +252,51 @@ def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
                         None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
                         _stream(stream))
     _check(st, "pa_decode")
+
+
+def pa_decode_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                  value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+                  q_per_seq: int, scale: float, k_scale: float, v_scale: float,
+                  plan: pa_plan_t | None = None, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """pa_decode over FP8 pools: caches [NB, 16, H_kv, D] uint8 (E4M3 codes, values code *
+    k_scale / code * v_scale); everything else as pa_decode. plan: None or one made with
+    kv_cache_dtype=PA_KV_FP8_E4M3."""
+    assert out.dtype == query.dtype == torch.bfloat16
+    assert key_cache.dtype == value_cache.dtype == torch.uint8
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    for t in (out, query, key_cache, value_cache, block_tables, context_lens):
+        assert t.is_contiguous()
+    B, QS, HQ, D = query.shape
+    assert QS == q_per_seq and tuple(out.shape) == tuple(query.shape)
+    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_fp8(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                            _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
+                            block_tables.shape[1], NB, float(scale), float(k_scale), float(v_scale),
+                            None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
+                            _stream(stream))
+    _check(st, "pa_decode_fp8")
+
+
+def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor, value_cache: torch.Tensor,
+               block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+               max_query_len: int, scale: float, stream=None) -> None:
+    """Chunked-prefill attention. out/query [T, H_q, D] bf16 (the chunks of all sequences,
+    concatenated); query_start [B + 1] int32 on the device; caches, block_tables and
+    context_lens as pa_decode; max_query_len bounds every chunk length."""
+    assert out.dtype == query.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert block_tables.dtype == context_lens.dtype == query_start.dtype == torch.int32
+    for t in (out, query, key_cache, value_cache, block_tables, context_lens, query_start):
+        assert t.is_contiguous()
+    T, HQ, D = query.shape
+    assert tuple(out.shape) == tuple(query.shape)
+    B = block_tables.shape[0]
+    assert query_start.numel() == B + 1 and context_lens.numel() == B
+    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    st = _lib.pa_prefill(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                         _ptr(context_lens), _ptr(query_start), B, T, int(max_query_len), HQ, HKV, D, BS,
+                         block_tables.shape[1], NB, float(scale), _stream(stream))
+    _check(st, "pa_prefill")
 
 
 def pa_decode_static_scratch(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,

@@ -25,6 +25,13 @@ notes §1.2.2):
 * ``sliding_window``  16 x 1, 32/8 heads, head_dim 128, a 4096-token sliding window over
                       contexts U[8192, 32768]; entries before the window name the null
                       block 0.
+* ``llama8b_fp8``     the llama8b shapes over FP8 (E4M3) pools, one scale 0.01 per pool
+                      (the FP8 KV cache of the vLLM study notes §4.2).
+
+Chunked prefill (``PREFILL_WORKLOADS``; the vLLM study notes §3.5):
+
+* ``chunked_prefill`` 4 prompts of 4096 tokens, each attending its last 512-token chunk over
+                      the pool (3584 earlier tokens + the chunk, causal), 32/8 heads, D 128.
 
 Copy-on-write block copies (``make_copy``; the copy rule of the vLLM study notes
 §3.2.2):
@@ -70,6 +77,9 @@ class Workload:
     blocks_used: np.ndarray = field(default=None)   # int32 [B] blocks owned per sequence
     shared_groups: list = field(default_factory=list)  # [(members, prefix_tokens)]
     window: int = 0                   # sliding window in tokens, 0 = none
+    kv_dtype: str = "bf16"            # "bf16", or "fp8_e4m3": uint8 pools of E4M3 codes
+    k_scale: float = 1.0              # fp8_e4m3: value of a key code = code * k_scale
+    v_scale: float = 1.0
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -84,7 +94,9 @@ class Workload:
                 f"H_kv={self.num_kv_heads} D={self.head_dim} bs={self.block_size} "
                 f"ctx[min/mean/max]={int(self.context_lens.min())}/"
                 f"{float(self.context_lens.mean()):.0f}/{int(self.context_lens.max())} "
-                f"NB={self.num_blocks} seed={self.seed}" + (f" window={self.window}" if self.window else ""))
+                f"NB={self.num_blocks} seed={self.seed}" + (f" window={self.window}" if self.window else "")
+                + (f" kv=fp8_e4m3 k_scale={self.k_scale:g} v_scale={self.v_scale:g}"
+                   if self.kv_dtype == "fp8_e4m3" else ""))
 
 
 def _blocks(n_tokens: int, block_size: int) -> int:
@@ -179,6 +191,27 @@ def build_workload(name: str, seed: int, context_lens, q_per_seq: int, num_q_hea
                     num_blocks=int(num_blocks), query=query, key=key, value=value,
                     slot_mapping=slots, key_cache=key_cache, value_cache=value_cache,
                     blocks_used=need.astype(np.int32), shared_groups=share_groups, window=int(window))
+
+
+def with_fp8_pools(w: Workload, k_scale: float = 0.01, v_scale: float = 0.01,
+                   name: str | None = None) -> Workload:
+    """The same workload over FP8 KV pools: the pools' prior contents become E4M3 codes of
+    the bf16 values over the pool scale (torch's float8_e4m3fn conversion, magnitudes clipped
+    to the format's 448 first). The step's new K/V rows stay bf16: the FP8 cache write turns
+    them into codes. The default scale 0.01 maps the ~N(0, 1) values onto the code range
+    (|x| up to 4.48 before the codes saturate)."""
+    import copy
+    f = copy.copy(w)
+
+    def codes(pool: torch.Tensor, scale: float) -> torch.Tensor:
+        x = (pool.float() / scale).clamp_(-448.0, 448.0)
+        return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+    f.key_cache = codes(w.key_cache, k_scale)
+    f.value_cache = codes(w.value_cache, v_scale)
+    f.kv_dtype, f.k_scale, f.v_scale = "fp8_e4m3", float(k_scale), float(v_scale)
+    f.name = name or (w.name + "_fp8")
+    return f
 
 
 def tiny(seed: int = 1000) -> Workload:
@@ -319,6 +352,114 @@ def sliding_window(seed: int = 1007, num_seqs: int = 16, window: int = 4096) -> 
     return build_workload("sliding_window", seed, ctx, 1, 32, 8, 128, window=window)
 
 
+def llama8b_fp8(seed: int = 1008) -> Workload:
+    """The Llama-3.1-8B-shaped decode layer over FP8 (E4M3) KV pools, scale 0.01 per pool."""
+    return with_fp8_pools(llama8b(seed), name="llama8b_fp8")
+
+
+@dataclass
+class PrefillWorkload:
+    """One chunked-prefill step: every sequence attends a chunk of qlen_b new tokens (the
+    last qlen_b positions of its context) over the paged pool, causal within the chunk.
+    The chunk tokens' K/V are written first through the slot mapping."""
+    name: str
+    seed: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    scale: float
+    context_lens: np.ndarray          # int32 [B], including the chunk
+    query_start: np.ndarray           # int32 [B + 1]
+    block_tables: np.ndarray          # int32 [B, max_blocks_per_seq]
+    num_blocks: int
+    query: torch.Tensor               # bf16 [T, H_q, D]
+    key: torch.Tensor                 # bf16 [T, H_kv, D]: the chunk tokens' K
+    value: torch.Tensor               # bf16 [T, H_kv, D]
+    slot_mapping: np.ndarray          # int64 [T]
+    key_cache: torch.Tensor           # bf16 [NB, bs, H_kv, D], pool before the write
+    value_cache: torch.Tensor
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def query_lens(self) -> np.ndarray:
+        return np.diff(self.query_start)
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.query_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+    def describe(self) -> str:
+        ql = self.query_lens
+        return (f"{self.name}: B={self.num_seqs} chunk[min/mean/max]={int(ql.min())}/{float(ql.mean()):.0f}/"
+                f"{int(ql.max())} T={self.num_tokens} H_q={self.num_q_heads} H_kv={self.num_kv_heads} "
+                f"D={self.head_dim} bs={self.block_size} ctx[min/mean/max]={int(self.context_lens.min())}/"
+                f"{float(self.context_lens.mean()):.0f}/{int(self.context_lens.max())} NB={self.num_blocks} "
+                f"seed={self.seed}")
+
+
+def build_prefill(name: str, seed: int, context_lens, query_lens, num_q_heads: int, num_kv_heads: int,
+                  head_dim: int, scale: float | None = None, block_size: int = BLOCK_SIZE,
+                  pool_factor: float = 1.25) -> PrefillWorkload:
+    """Sequences with the given contexts, each ending in a chunk of query_lens[b] new tokens;
+    blocks from one seeded permutation of a pool pool_factor x the blocks needed; bf16
+    ~N(0, 1) values."""
+    rng = np.random.default_rng(seed)
+    gen = torch.Generator().manual_seed(seed)
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    ql = np.asarray(query_lens, dtype=np.int64)
+    if ctx.shape != ql.shape or np.any(ql < 0) or np.any(ql > ctx):
+        raise ValueError("every chunk lies inside its context")
+    B = int(ctx.shape[0])
+    need = np.array([_blocks(c, block_size) for c in ctx], dtype=np.int64)
+    num_blocks = int(math.ceil(pool_factor * int(need.sum()))) + 1
+    perm = rng.permutation(num_blocks).astype(np.int64)
+    width = int(max(1, need.max()))
+    tables = np.zeros((B, width), dtype=np.int32)
+    cursor = 0
+    for b in range(B):
+        tables[b, :need[b]] = perm[cursor:cursor + need[b]]
+        cursor += int(need[b])
+    qstart = np.zeros(B + 1, dtype=np.int32)
+    qstart[1:] = np.cumsum(ql)
+    T = int(qstart[-1])
+    slots = np.empty(T, dtype=np.int64)
+    for b in range(B):
+        for i in range(int(ql[b])):
+            pos = int(ctx[b]) - int(ql[b]) + i
+            slots[qstart[b] + i] = int(tables[b, pos // block_size]) * block_size + pos % block_size
+    return PrefillWorkload(
+        name=name, seed=seed, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+        block_size=block_size, scale=float(1.0 / math.sqrt(head_dim) if scale is None else scale),
+        context_lens=ctx.astype(np.int32), query_start=qstart, block_tables=tables, num_blocks=num_blocks,
+        query=_randn_bf16((T, num_q_heads, head_dim), gen), key=_randn_bf16((T, num_kv_heads, head_dim), gen),
+        value=_randn_bf16((T, num_kv_heads, head_dim), gen), slot_mapping=slots,
+        key_cache=_randn_bf16((num_blocks, block_size, num_kv_heads, head_dim), gen),
+        value_cache=_randn_bf16((num_blocks, block_size, num_kv_heads, head_dim), gen))
+
+
+def chunked_prefill(seed: int = 1009, num_seqs: int = 4, chunk: int = 512, context: int = 4096) -> PrefillWorkload:
+    """A chunked-prefill step of a Llama-3.1-8B-shaped layer (32 q heads, 8 kv heads,
+    head_dim 128): 4 prompts of 4096 tokens whose last 512-token chunk is attended now over
+    the 3584 tokens already in the pool plus itself (the chunk size of the vLLM study
+    notes §3.5 is 2048; 512 keeps four prompts in one step)."""
+    return build_prefill("chunked_prefill", seed, [context] * num_seqs, [chunk] * num_seqs, 32, 8, 128)
+
+
+PREFILL_WORKLOADS = {"chunked_prefill": chunked_prefill}
+
+
 WORKLOADS = {
     "tiny": tiny,
     "llama8b": llama8b,
@@ -326,6 +467,7 @@ WORKLOADS = {
     "prefix_sharing": prefix_sharing,
     "spec_verify": spec_verify,
     "sliding_window": sliding_window,
+    "llama8b_fp8": llama8b_fp8,
 }
 
 

@@ -625,6 +625,29 @@ def check_fp8_cache_and_attention(oracle):
         _close(out[b], o[0].permute(1, 0, 2).numpy(), tol=1e-10, what=f"fp8 seq {b} vs SDPA")
 
 
+def check_chunked_prefill(oracle):
+    """Chunked prefill (vLLM study notes §3.5; "vLLM 深度解析" §5.4): a prompt is attended
+    in chunks of many query tokens, each chunk causal within itself over the keys already
+    in the pool. Pinned at q = 64 and 200 against brute force and torch SDPA, and by the
+    property chunking relies on: the rows of a prompt attended as two chunks (the first
+    with context = its length, the second over the whole prompt) equal the rows of one
+    chunk over the whole prompt."""
+    for case in (dict(seed=91, ctxs=[64, 100], q=64, hq=4, hkv=2, d=16),
+                 dict(seed=92, ctxs=[200, 233], q=200, hq=4, hkv=1, d=16, bs=16)):
+        p = Problem(**case)
+        got = p.run(oracle)
+        _close(got, library_attention(p), what=f"chunked prefill sdpa q={p.q}")
+        bf = brute_force(p)
+        _close(got, bf, what=f"chunked prefill brute force q={p.q}")
+    # one chunk of 96 over a 96-token prompt == chunks of 40 and 56
+    p = Problem(seed=93, ctxs=[96, 96], q=96, hq=4, hkv=2, d=16)
+    whole = p.run(oracle)
+    first = p.run(oracle, ctxs=[40, 40], Q=p.Q[:, :40].copy(), q=40)
+    second = p.run(oracle, Q=p.Q[:, 40:].copy(), q=56)
+    assert np.array_equal(whole[:, :40], first), "first chunk differs from the whole prompt's rows"
+    assert np.array_equal(whole[:, 40:], second), "second chunk differs from the whole prompt's rows"
+
+
 ALL_CHECKS = [
     check_bf16_widening,
     check_block_counts_golden,
@@ -644,4 +667,5 @@ ALL_CHECKS = [
     check_sliding_window,
     check_fp8_format,
     check_fp8_cache_and_attention,
+    check_chunked_prefill,
 ]

@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(pa):
 def test_status_strings_and_version(pa):
     for code in range(7):
         assert pa.pa_status_string(code).startswith("PA_")
-    assert pa.pa_version() == 10000
+    assert pa.pa_version() == 10100
 
 
 def _decode_raw(lib, **kw):
@@ -80,7 +80,9 @@ def test_decode_rejects_bad_arguments_before_launch(pa):
     assert plan.num_splits == 4
     assert _decode_raw(lib, plan=ctypes.byref(plan)) == pa.PA_ERR_WORKSPACE
     need = pa.pa_decode_workspace_size(plan, 2, 1, 4, 2, 64, 4)
-    assert need == 2 * 4 * 1 * 4 * (64 + 2) * 4
+    # records (o and (m, l) of every split and query row), 256-byte aligned, then one arrival
+    # counter per output target (sequence, kv head)
+    assert need == -(-(2 * 4 * 1 * 4 * (64 + 2) * 4) // 256) * 256 + 4 * 2 * 2
     assert _decode_raw(lib, plan=ctypes.byref(plan), ws=96 * 1024, ws_bytes=need - 1) == pa.PA_ERR_WORKSPACE
     bad = pa.pa_plan_t.from_buffer_copy(plan)
     bad.num_splits += 1
@@ -205,20 +207,24 @@ def test_every_plan_passes_decode_validation(pa, hints):
 
 
 def test_window_plans_on_the_host(pa):
-    """Sliding-window plans: grid schedule only, splits over the window's span of blocks;
-    the other kernels and prefix sharing are refused before any device query."""
+    """Sliding-window plans: the grid schedule (splits over the window's span of blocks) or
+    the tcgen05 kernel; prefix sharing and the mma.sync persistent schedule are refused
+    before any device query."""
     lib = pa.raw_library()
     plan = pa.pa_plan_t()
-    for hints in ((3, 0, 0, 0, 64), (0, 2, 0, 0, 64), (2, 0, 0, 1, 64)):
+    for hints in ((2, 2, 0, 0, 64), (0, 2, 0, 0, 64), (2, 0, 0, 1, 64), (3, 0, 0, 1, 64)):
         h = pa.pa_plan_hints_t(*hints)
         assert lib.pa_decode_plan(4, 1, 32, 8, 128, 64, ctypes.byref(h), ctypes.byref(plan)) == \
             pa.PA_ERR_UNSUPPORTED, hints
     h = pa.pa_plan_hints_t(0, 0, 0, 0, -1)
     assert lib.pa_decode_plan(4, 1, 32, 8, 128, 64, ctypes.byref(h), ctypes.byref(plan)) == pa.PA_ERR_INVALID_ARG
-    # 24 rows at head_dim 128 would take tcgen05; with a window the tiles take it, on the grid
+    # 24 rows at head_dim 128: the tcgen05 kernel, window or not
     p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, sliding_window=4096)
+    assert (p.path, p.schedule, p.sliding_window) == (pa.PA_PATH_TCGEN05, pa.PA_SCHEDULE_PERSISTENT, 4096)
+    # 4 rows: the mma.sync tiles on the grid, splits over the window's span
+    p = pa.pa_decode_plan(32, 1, 32, 8, 128, 1024, sliding_window=4096)
     assert (p.path, p.schedule, p.sliding_window) == (pa.PA_PATH_TILE, pa.PA_SCHEDULE_GRID, 4096)
-    span = -(-(4096 + 6 - 1) // 16) + 1
+    span = -(-(4096 + 1 - 1) // 16) + 1
     assert p.split_blocks <= span and p.num_splits == -(-span // p.split_blocks)
     p = pa.pa_decode_plan(4, 1, 32, 8, 128, 64, sliding_window=100000)   # wider than the table
     assert p.num_splits == -(-64 // p.split_blocks)
@@ -282,3 +288,71 @@ def test_size_query_and_static_scratch_check_before_sizing(pa):
     assert static(ctypes.byref(plan), B=-3) == pa.PA_ERR_INVALID_ARG
     assert static(ctypes.byref(zeroed)) == pa.PA_ERR_INVALID_ARG
     assert _decode_raw(lib, plan=ctypes.byref(zeroed), ws=96 * 1024, ws_bytes=1 << 20) == pa.PA_ERR_INVALID_ARG
+
+
+def _decode_fp8_raw(lib, ks=0.01, vs=0.01, **kw):
+    args = dict(out=8 * 1024, query=16 * 1024, kc=32 * 1024, vc=48 * 1024, bt=64 * 1024, cl=80 * 1024,
+                B=2, q=1, hq=4, hkv=2, d=64, bs=16, mb=4, nb=8, scale=0.125, plan=None, ws=None,
+                ws_bytes=0)
+    args.update(kw)
+    return lib.pa_decode_fp8(args["out"], args["query"], args["kc"], args["vc"], args["bt"], args["cl"],
+                             args["B"], args["q"], args["hq"], args["hkv"], args["d"], args["bs"],
+                             args["mb"], args["nb"], args["scale"], ks, vs, args["plan"], args["ws"],
+                             args["ws_bytes"], None)
+
+
+def test_fp8_plans_on_the_host(pa):
+    """FP8 pools are read by the mma.sync tiles: the automatic FP8 plan takes them, the
+    CUDA-core and tcgen05 kernels are refused, and a plan only decodes the pools it was made
+    for (before any device work)."""
+    lib = pa.raw_library()
+    fp8 = pa.PA_KV_FP8_E4M3
+    p = pa.pa_decode_plan(32, 6, 32, 8, 128, 1024, kv_cache_dtype=fp8)   # 24 rows: tcgen05 for bf16
+    assert (p.path, p.kv_cache_dtype) == (pa.PA_PATH_TILE, fp8)
+    p = pa.pa_decode_plan(4, 1, 4, 2, 64, 8, kv_cache_dtype=fp8)          # 2 rows: CUDA cores for bf16
+    assert p.path == pa.PA_PATH_TILE
+    for path in (pa.PA_PATH_SINGLE, pa.PA_PATH_TCGEN05):
+        with pytest.raises(pa.PAError) as exc:
+            pa.pa_decode_plan(4, 1, 32, 8, 128, 64, path, kv_cache_dtype=fp8)
+        assert exc.value.status == pa.PA_ERR_UNSUPPORTED
+    h = pa.pa_plan_hints_t(0, 0, 0, 0, 0, 2)
+    plan = pa.pa_plan_t()
+    assert lib.pa_decode_plan(4, 1, 32, 8, 128, 64, ctypes.byref(h), ctypes.byref(plan)) == pa.PA_ERR_INVALID_ARG
+    for hints in ({}, {"schedule": pa.PA_SCHEDULE_PERSISTENT}, {"share_prefix": True}, {"split_blocks": 3},
+                  {"sliding_window": 40}):
+        p = pa.pa_decode_plan(2, 1, 4, 2, 64, 4, kv_cache_dtype=fp8, **hints)
+        need = pa.pa_decode_workspace_size(p, 2, 1, 4, 2, 64, 4)
+        # a plan for FP8 pools is refused by pa_decode, accepted by pa_decode_fp8's checks
+        assert _decode_raw(lib, plan=ctypes.byref(p), ws=96 * 1024, ws_bytes=need) == pa.PA_ERR_INVALID_ARG
+        st = _decode_fp8_raw(lib, plan=ctypes.byref(p), ws=96 * 1024, ws_bytes=need)
+        assert st not in (pa.PA_ERR_INVALID_ARG, pa.PA_ERR_UNSUPPORTED, pa.PA_ERR_WORKSPACE), (hints, st)
+    bf16_plan = pa.pa_decode_plan(2, 1, 4, 2, 64, 4, pa.PA_PATH_TILE)
+    assert _decode_fp8_raw(lib, plan=ctypes.byref(bf16_plan)) == pa.PA_ERR_INVALID_ARG
+    forged = pa.pa_plan_t.from_buffer_copy(pa.pa_decode_plan(2, 1, 4, 2, 64, 4, kv_cache_dtype=fp8))
+    forged.path = pa.PA_PATH_SINGLE
+    forged.rows_per_cta = 2
+    assert _decode_fp8_raw(lib, plan=ctypes.byref(forged)) == pa.PA_ERR_INVALID_ARG
+    for ks, vs in ((0.0, 1.0), (1.0, -2.0), (float("nan"), 1.0), (1.0, float("inf"))):
+        assert _decode_fp8_raw(lib, ks=ks, vs=vs) == pa.PA_ERR_INVALID_ARG
+
+
+def test_prefill_rejects_bad_arguments_before_launch(pa):
+    lib = pa.raw_library()
+
+    def call(**kw):
+        a = dict(out=8192, q=16384, kc=32768, vc=49152, bt=65536, cl=81920, qs=98304, B=2, T=10, mq=8, hq=32,
+                 hkv=8, d=128, bs=16, mb=8, nb=64, scale=0.088)
+        a.update(kw)
+        return lib.pa_prefill(a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["qs"], a["B"], a["T"], a["mq"],
+                              a["hq"], a["hkv"], a["d"], a["bs"], a["mb"], a["nb"], a["scale"], None)
+    assert call(d=64) == pa.PA_ERR_UNSUPPORTED             # head_dim 128 only
+    assert call(hq=24, hkv=8) == pa.PA_ERR_UNSUPPORTED     # G = 3 does not divide 128
+    assert call(bs=32) == pa.PA_ERR_UNSUPPORTED
+    assert call(hq=30, hkv=8) == pa.PA_ERR_INVALID_ARG     # H_q % H_kv
+    assert call(qs=None) == pa.PA_ERR_INVALID_ARG
+    assert call(out=8192 + 8) == pa.PA_ERR_INVALID_ARG     # misaligned
+    assert call(cl=81920 + 2) == pa.PA_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert call(B=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(B=0) == pa.PA_OK and call(T=0) == pa.PA_OK and call(mq=0) == pa.PA_OK   # no-ops
+    assert call(mq=3_000_000) == pa.PA_ERR_UNSUPPORTED     # more tiles than the grid holds

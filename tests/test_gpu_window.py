@@ -1,5 +1,6 @@
 """pa_decode with a sliding window against the fp64 oracle: the mma.sync and CUDA-core grid
-paths, windows around block and split boundaries, speculative rows, and the null block
+paths and the tcgen05 kernel, windows around block and split boundaries, speculative rows,
+and the null block
 (table entries wholly before the window point at block 0, which holds NaN, and the slots
 before the window in its first block hold NaN as well)."""
 
@@ -29,6 +30,8 @@ PLANS = [
     ("tile_grid", dict(path=2, schedule=1)),
     ("tile_split1", dict(path=2, split_blocks=1)),
     ("tile_split3", dict(path=2, split_blocks=3)),
+    ("tcgen05", dict(path=3)),
+    ("tcgen05_ctas5", dict(path=3, num_ctas=5)),   # units cut into many pieces
 ]
 
 
@@ -52,9 +55,19 @@ def prepared(oracle_lib):
 
 def _plan(w, spec, W):
     from paged_kv_cache_399_b200 import pa
+    spec = dict(spec)
+    num_ctas = spec.pop("num_ctas", None)
+    if spec.get("path") == pa.PA_PATH_TCGEN05 and w.head_dim != 128:
+        pytest.skip("the tcgen05 path runs head_dim 128")
     plan = pa.pa_decode_plan(w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads, w.head_dim,
                              w.max_blocks_per_seq, sliding_window=W, **spec)
-    assert plan.schedule == pa.PA_SCHEDULE_GRID and plan.sliding_window == W
+    assert plan.sliding_window == W
+    if plan.path == pa.PA_PATH_TCGEN05:
+        assert plan.schedule == pa.PA_SCHEDULE_PERSISTENT
+        if num_ctas is not None:
+            plan.num_ctas = num_ctas
+        return plan
+    assert plan.schedule == pa.PA_SCHEDULE_GRID
     span = min(w.max_blocks_per_seq, -(-(W + w.q_per_seq - 1) // 16) + 1)
     assert plan.num_splits == -(-span // plan.split_blocks)
     return plan
@@ -115,9 +128,10 @@ def test_window_never_reads_before_the_window(W, plan_spec, oracle_lib):
     assert_close(out, ref, f"null block W={W}/{plan_spec[0]}")
 
 
-def test_window_rejected_outside_the_grid_paths():
+def test_window_rejected_with_sharing_or_the_mma_sync_persistent_schedule():
     from paged_kv_cache_399_b200 import pa
-    for hints in (dict(path=3), dict(schedule=2), dict(path=2, share_prefix=True)):
+    for hints in (dict(path=2, schedule=2), dict(path=1, schedule=2), dict(path=2, share_prefix=True),
+                  dict(path=3, share_prefix=True)):
         with pytest.raises(pa.PAError) as err:
             pa.pa_decode_plan(4, 1, 32, 8, 128, 64, sliding_window=64, **hints)
         assert err.value.status == pa.PA_ERR_UNSUPPORTED
