@@ -706,11 +706,11 @@ def decode_launches(plan) -> int:
     """Kernel launches of one pa_decode call with this plan."""
     from paged_kv_cache_399_b200 import pa
     if plan.path == pa.PA_PATH_TCGEN05:
-        return 2 + (1 if plan.share_cap > 1 else 0)
+        return 2 + (1 if plan.share_cap > 1 else 0)      # [pre-pass], decode, merge
     if plan.schedule == pa.PA_SCHEDULE_PERSISTENT:
-        return 2
-    # grid: the decode kernel, after the sharing pre-pass or the counter reset when outputs merge
-    return 1 + (1 if (plan.num_splits > 1 or plan.share_cap) else 0)
+        return 2                                         # pre-pass, decode
+    # grid: [sharing pre-pass], decode, [merge of split partials]
+    return (1 if plan.share_cap else 0) + 1 + (1 if (plan.num_splits > 1 or plan.share_cap) else 0)
 
 
 # ------------------------------------------------------------------ CPU oracle legs

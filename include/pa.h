@@ -206,8 +206,9 @@ PA_API pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t n
                            int32_t max_blocks_per_seq, const pa_plan_hints_t* hints,
                            pa_plan_t* plan);
 
-/* Workspace bytes pa_decode needs for `plan` (NULL = the heuristic plan for these
- * shapes). Grid schedule: split partials, 0 when there is one split. Persistent
+/* Workspace bytes pa_decode (or pa_decode_fp8) needs for `plan` (NULL = enough for the
+ * heuristic plan of these shapes over bf16 pools and over FP8 pools, so that NULL works for
+ * both calls when they too are given plan NULL; 0 for invalid shapes or plans). Grid schedule: split partials, 0 when there is one split. Persistent
  * schedule: the pre-pass tables, per-output counters and record lists, and a pool of
  * fp32 partial records (a few MB for the shapes above). tcgen05: two fp32 records of
  * rows_per_cta rows per CTA, a descriptor per CTA and, with sharing, one prefix

@@ -238,15 +238,25 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
   if (split_blocks == 0) {
     // Host-known values only: units of (sequence, kv head, row chunk) against the
     // number of resident CTAs. Enough units: one split. Otherwise cut the longest
-    // possible context into pieces so that about four waves of CTAs exist.
+    // possible context into pieces so that about four waves of CTAs exist (contexts of
+    // different lengths leave many splits empty). With a sliding window every sequence
+    // reads about the same span, so about 1.5 waves of longer splits suffice (measured
+    // on B200: fewer, longer splits beat the four-wave rule there). Splits are made
+    // equal, so that no short last split is left over.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * row_chunks;
     if (units >= 2 * static_cast<int64_t>(slots) || units == 0) {
       split_blocks = span;
     } else {
-      const int64_t splits = ceil_div(4 * static_cast<int64_t>(slots), units);
+      const int64_t target = h.sliding_window > 0 ? 3 * static_cast<int64_t>(slots) / 2 : 4 * static_cast<int64_t>(slots);
+      const int64_t splits = ceil_div(target, units);
+      const int64_t floor_sb = (h.sliding_window > 0 ? 4 : 8) * pa::kWarpsPerCta;
       int64_t sb = ceil_div(span, splits);
       sb = ceil_div(sb, pa::kWarpsPerCta) * pa::kWarpsPerCta;
-      if (sb < 8 * pa::kWarpsPerCta) sb = 8 * pa::kWarpsPerCta;
+      if (sb < floor_sb) sb = floor_sb;
+      if (sb < span) {  // equal splits
+        const int64_t n = ceil_div(span, sb);
+        sb = ceil_div(ceil_div(span, n), pa::kWarpsPerCta) * pa::kWarpsPerCta;
+      }
       split_blocks = static_cast<int32_t>(sb < span ? sb : span);
     }
   }
@@ -305,56 +315,40 @@ size_t share_records(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
   return static_cast<size_t>(num_seqs) * (ssplits + plan.num_splits) * q_per_seq * num_q_heads;
 }
 
-// Workspace of the tcgen05 path: two partial records per CTA (a record holds rows_per_cta
-// rows of O (fp32) and their (m, l) pairs), with prefix sharing the shared-prefix length of
-// every window of share_cap sequences, then one arrival counter per unit (window, kv head,
-// row chunk).
+// Workspace of the tcgen05 path: two partial records per CTA, then one piece descriptor
+// per CTA. A record holds rows_per_cta rows of O (fp32) and their (m, l) pairs.
 int32_t tcm_rec_stride(const pa_plan_t& plan, int32_t head_dim) {
   return plan.rows_per_cta * head_dim + 2 * plan.rows_per_cta;
 }
-size_t tcm_prefix_offset(const pa_plan_t& plan, int32_t head_dim) {
+size_t tcm_desc_offset(const pa_plan_t& plan, int32_t head_dim) {
   return align256(static_cast<size_t>(2) * plan.num_ctas * tcm_rec_stride(plan, head_dim) * 4);
 }
-int64_t tcm_windows(const pa_plan_t& plan, int32_t num_seqs) {
-  return plan.share_cap > 1 ? ceil_div(num_seqs, plan.share_cap) : num_seqs;
-}
-size_t tcm_counter_offset(const pa_plan_t& plan, int32_t num_seqs, int32_t head_dim) {
-  size_t off = tcm_prefix_offset(plan, head_dim);
-  if (plan.share_cap > 1) off = align256(off + 4 * static_cast<size_t>(tcm_windows(plan, num_seqs)));
-  return off;
-}
 
-// Grid schedule: byte offset of the arrival counters, after the records (and, with prefix
-// sharing, the per-sequence seq_info).
-size_t grid_counter_offset(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
-                           int32_t head_dim) {
-  const size_t recs = plan.share_cap ? share_records(plan, num_seqs, q_per_seq, num_q_heads)
-                                     : static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads;
-  size_t off = align256(recs * (static_cast<size_t>(head_dim) + 2) * 4);
-  if (plan.share_cap) off += align256(16 * static_cast<size_t>(num_seqs));
-  return off;
+// With prefix sharing the shared-prefix length of every window of share_cap sequences
+// follows the descriptors.
+size_t tcm_prefix_offset(const pa_plan_t& plan, int32_t head_dim) {
+  return align256(tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas));
 }
 
 size_t workspace_bytes_for(const pa_plan_t& plan, int32_t num_seqs, int32_t q_per_seq,
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
   if (plan.path == PA_PATH_TCGEN05) {
     if (num_seqs == 0) return 0;
-    const int64_t rows = static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq;
-    const int64_t units = tcm_windows(plan, num_seqs) * num_kv_heads * ceil_div(rows * (plan.share_cap > 1 ? plan.share_cap : 1), plan.rows_per_cta);
-    return tcm_counter_offset(plan, num_seqs, head_dim) + 4 * static_cast<size_t>(units);
+    if (plan.share_cap > 1)
+      return tcm_prefix_offset(plan, head_dim) + 4 * static_cast<size_t>(ceil_div(num_seqs, plan.share_cap));
+    return tcm_desc_offset(plan, head_dim) + 16 * static_cast<size_t>(plan.num_ctas);
   }
   if (plan.schedule == PA_SCHEDULE_PERSISTENT) {
     if (num_seqs == 0) return 0;
     return persistent_layout(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim).total;
   }
-  // grid: partial records (o, then (m, l)), with sharing the per-sequence seq_info, then one
-  // arrival counter per output target (sequence, kv head, row chunk)
-  const size_t targets = static_cast<size_t>(num_seqs) * num_kv_heads *
-                         static_cast<size_t>(ceil_div(static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq,
-                                                      plan.rows_per_cta));
-  if (plan.share_cap) return grid_counter_offset(plan, num_seqs, q_per_seq, num_q_heads, head_dim) + 4 * targets;
+  if (plan.share_cap) {  // records of the shared-prefix splits and of the own splits + seq_info
+    const size_t recs = share_records(plan, num_seqs, q_per_seq, num_q_heads);
+    return align256(recs * (static_cast<size_t>(head_dim) + 2) * 4) + 16 * static_cast<size_t>(num_seqs);
+  }
   if (plan.num_splits <= 1) return 0;
-  return grid_counter_offset(plan, num_seqs, q_per_seq, num_q_heads, head_dim) + 4 * targets;
+  return static_cast<size_t>(num_seqs) * plan.num_splits * q_per_seq * num_q_heads *
+         (static_cast<size_t>(head_dim) + 2) * 4;
 }
 
 pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_heads,
@@ -475,7 +469,7 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     p.rec_stride = tcm_rec_stride(*plan, head_dim);
     p.records = reinterpret_cast<float*>(ws);
     if (plan->share_cap > 1) p.win_prefix = reinterpret_cast<int32_t*>(ws + tcm_prefix_offset(*plan, head_dim));
-    p.arrive = reinterpret_cast<int32_t*>(ws + tcm_counter_offset(*plan, num_seqs, head_dim));
+    p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
     // CTAs per group: the largest divisor of H_kv that the grid holds
     p.tc_group = 1;
     for (int sz = num_kv_heads; sz >= 1; --sz)
@@ -512,7 +506,6 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
       p.share_windows = static_cast<int32_t>(ceil_div(num_seqs, plan->share_cap));
       p.seq_info = reinterpret_cast<int4*>(ws + align256(recs * (static_cast<size_t>(head_dim) + 2) * 4));
     }
-    p.arrive = reinterpret_cast<int32_t*>(ws + grid_counter_offset(*plan, num_seqs, q_per_seq, num_q_heads, head_dim));
   }
   cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, kv_dtype, tk, tv,
                                     reinterpret_cast<cudaStream_t>(stream));
@@ -587,16 +580,25 @@ pa_status_t pa_decode_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_he
 size_t pa_decode_workspace_size(const pa_plan_t* plan, int32_t num_seqs, int32_t q_per_seq,
                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                 int32_t max_blocks_per_seq) {
-  pa_plan_t local;
   if (!plan) {
-    if (make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                  nullptr, &local) != PA_OK)
-      return 0;
-    plan = &local;
-  } else if (pa::check_decode_args(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
-                                   max_blocks_per_seq) != PA_OK) {
-    return 0;  // the sizes below divide by plan and shape fields: never with bad ones
+    // the heuristic plans for bf16 pools (pa_decode) and for E4M3 pools (pa_decode_fp8) may
+    // differ (their kernels' occupancies do): the larger of the two serves both calls
+    size_t need = 0;
+    for (int dtype : {PA_KV_BF16, PA_KV_FP8_E4M3}) {
+      pa_plan_hints_t h = {};
+      h.kv_cache_dtype = dtype;
+      pa_plan_t local;
+      if (make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, &h, &local) !=
+          PA_OK)
+        continue;
+      const size_t n = workspace_bytes_for(local, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
+      if (n > need) need = n;
+    }
+    return need;
   }
+  if (pa::check_decode_args(plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq) !=
+      PA_OK)
+    return 0;  // the sizes below divide by plan and shape fields: never with bad ones
   return workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
 }
 

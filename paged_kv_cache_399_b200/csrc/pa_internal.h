@@ -65,12 +65,14 @@ struct DecodeParams {
   long long* seq_start;          // [B] first work unit of the sequence's bands
   int4* seq_info;                // [B] {P_b shared prefix blocks, members if leader else 0, nblk, ctx}
   int32_t* cta_seq;              // [num_ctas] sequence holding the CTA's first unit
-  int32_t* arrive;               // [targets] persistent: blocks merged so far; grid and tcgen05:
-                                 // arrivals of this call (zeroed by its first kernel)
+  int32_t* arrive;               // [targets] blocks merged so far
   int32_t* list_len;             // [targets]
   int2* list;                    // [targets][list_cap] {piece start block, record slot}
   float* records;                // [pool_cap][rec_stride]; tcgen05 path: [2 * num_ctas][rec_stride]
 
+  // tcgen05 path: per CTA, the unit whose first piece it holds when that unit continues
+  // in later CTAs: {record slot, last CTA with a piece, sequence, unit}, or {-1, ...}
+  int4* tc_desc;
   int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
   int32_t* win_prefix;           // tcgen05 path with prefix sharing: shared blocks per window
 };

@@ -8,14 +8,14 @@
 //   decode_persistent_kernel paged decode, one CTA per resident slot, each over an
 //                            equal share of the work; partial results are merged by
 //                            the CTA that completes an output
-//   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split); the CTA
-//                            that completes an output's splits merges their partials
-//   grid_reset_kernel        zeroes the grid schedule's per-output arrival counters
+//   decode_grid_kernel       paged decode, one CTA per (kv head, sequence, split)
+//   merge_kernel             log-sum-exp merge of the grid schedule's split partials
 //   validate_kernel          debug bounds check of slots / block ids / context lengths
 //   selftest_wait_kernel     the bounded-wait failure path, taken without a fault
 // and, from pa_tcgen05.cuh, the 5th-generation tensor-core path:
 //   decode_tcm_kernel        tokens on M, tcgen05.mma with TMEM accumulators, persistent
 //                            equal-tile schedule over windows of sequences
+//   tcm_merge_kernel         merge of the units a tile range boundary cuts
 //   tcm_share_prepass        common table prefix of each window (prefix sharing)
 //
 // Two compute cores run inside the mma.sync / CUDA-core decode kernels:
@@ -277,7 +277,9 @@ __device__ __forceinline__ uint32_t e4m3_chunk_offset(int t, int c) {
 template <int D, int NT, bool kFp8 = false>
 struct TileCore {
   using Geom = TileGeom<D, kFp8>;
-  static constexpr int kStages = kFp8 ? 4 : 2;  // stages per warp: the same bytes in flight
+  // stages per warp: with E4M3 tiles (half the bytes) 3 stages and 4 CTAs per SM for 8 rows
+  // keep the bf16 core's bytes in flight with a third more warps to hide the conversions
+  static constexpr int kStages = kFp8 ? (NT == 1 ? 3 : 4) : 2;
   static constexpr int ROWS = NT * 8;
   static constexpr int KSTEPS = D / 16;
   static constexpr bool kNeedsQSmem = false;
@@ -745,7 +747,6 @@ struct CtaState {
   float2 ml[NW * ROWS];
   int slot[kTileMaxRows];
   int last[kTileMaxRows];
-  int merge[kTileMaxRows];  // grid schedule: 1 = this CTA completed the target's splits
   __align__(16) float q_s[kQ ? ROWS : 1][D];
   __align__(16) float p_s[NW][kQ ? 16 * ROWS : 1];
 };
@@ -1243,76 +1244,17 @@ __global__ void __launch_bounds__(kPrepassThreads) sched_prepass_kernel(const De
 // ---------------------------------------------------------------------------
 // Grid decode: one CTA per (kv head x row chunk, sequence, split of split_blocks
 // blocks). A sequence with one split writes bf16 directly; otherwise each split
-// writes fp32 partials (o, m, l), adds one to its output target's arrival counter
-// (zeroed by grid_reset_kernel or the sharing pre-pass of the same call), and the CTA
-// that brings the counter to the target's split count merges the target's partials in
-// split order (so the result does not depend on which CTA finished last).
+// writes fp32 partials (o, m, l) for merge_kernel.
 // ---------------------------------------------------------------------------
-
-// Splits that write partials for a sequence: its shared-prefix splits (prefix sharing)
-// and the splits of its own blocks [P_b, nblk).
-struct SplitCount {
-  int shared, own;
-};
-__device__ __forceinline__ SplitCount split_count(const DecodeParams& p, int P_b, int nblk) {
-  SplitCount c;
-  c.shared = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
-  c.own = nblk > P_b ? (nblk - P_b + p.split_blocks - 1) / p.split_blocks : 0;
-  return c;
-}
-
-// Log-sum-exp merge of the partials of target rows row0 .. row0+nrows-1 of kv head kvh of
-// sequence b, in split order, to bf16: M = max_k m_k, L = sum_k l_k 2^(m_k - M),
-// out = sum_k o_k 2^(m_k - M) / L. The whole CTA; the records were written by other CTAs
-// (read through L2).
-template <int D>
-__device__ __forceinline__ void merge_target(const DecodeParams& p, int b, int kvh, int row0, int nrows,
-                                             SplitCount n) {
-  constexpr int DC = D / 8;
-  const int RQ = p.q_per_seq * p.num_q_heads;
-  const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
-  const int ns = n.shared + n.own;
-  for (int task = threadIdx.x; task < nrows * DC; task += blockDim.x) {
-    const int r = task / DC, dc = task % DC;
-    const int rr = row0 + r;
-    const int i = rr / p.group;
-    const int h = kvh * p.group + (rr - i * p.group);
-    const int rq = i * p.num_q_heads + h;
-    auto rec_of = [&](int k) -> size_t {
-      return (k < n.shared ? static_cast<size_t>(b) * p.share_splits + k
-                           : own_region + static_cast<size_t>(b) * p.num_splits + (k - n.shared)) * RQ + rq;
-    };
-    float M = -INFINITY;
-    for (int k = 0; k < ns; ++k) M = fmaxf(M, __ldcg(p.ws_ml + rec_of(k)).x);
-    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < ns; ++k) {
-      const size_t rec = rec_of(k);
-      const float2 ml = __ldcg(p.ws_ml + rec);
-      const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-      L += w * ml.y;
-      const float4* src = reinterpret_cast<const float4*>(p.ws_o + rec * D + dc * 8);
-      const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
-      acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
-      acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
-    }
-    store_bf16x8(p.out + out_offset(p, b, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
-  }
-}
-
-// Zeroes the grid schedule's arrival counters of this call. It lets the decode kernel
-// launch at once (that kernel waits for this grid to complete), and zeroes only after the
-// preceding work on the stream -- possibly the previous call, still merging with these
-// counters -- has completed.
-__global__ void __launch_bounds__(256) grid_reset_kernel(int32_t* counters, int n) {
-  grid_launch_dependents();
-  grid_dependency_wait();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) counters[i] = 0;
-}
 // Resident CTAs per SM the compiler must allow for (a register cap of 168): 3 for the
 // cores that fit without spilling; the 24- and 32-row tensor-core cores keep their
-// registers (they spill under the cap, which measured slower) and run 2 per SM.
+// registers (they spill under the cap, which measured slower) and run 2 per SM; the 8-row
+// E4M3 core runs 4 (a cap of 128).
 template <class Core>
-constexpr int min_ctas_per_sm() { return Core::ROWS > 16 && !Core::kNeedsQSmem ? 2 : 3; }
+constexpr int min_ctas_per_sm() {
+  if (Core::Geom::kE4M3 && Core::ROWS <= 8) return 4;  // the 8-row E4M3 core fits 4 per SM
+  return Core::ROWS > 16 && !Core::kNeedsQSmem ? 2 : 3;
+}
 
 template <class Core, int D, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32, min_ctas_per_sm<Core>())
@@ -1389,25 +1331,6 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
         dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
         if (dc == 0) p.ws_ml[rec] = make_float2(M, L2);
       }
-      // one arrival per member (target (member, kvh), one row chunk with sharing); the
-      // member whose count this completes is merged here
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x < members) {
-        const int bm = L + threadIdx.x;
-        const int4 info = __ldcg(p.seq_info + bm);
-        const SplitCount n = split_count(p, info.x, info.z);
-        const int prev = atomicAdd(p.arrive + static_cast<size_t>(bm) * H + kvh, 1);
-        st.merge[threadIdx.x] = prev == n.shared + n.own - 1 ? 1 : 0;
-      }
-      __syncthreads();
-      for (int m = 0; m < members; ++m) {
-        if (!st.merge[m]) continue;  // uniform: shared memory flag
-        __threadfence();
-        const int bm = L + m;
-        const int4 info = __ldcg(p.seq_info + bm);
-        merge_target<D>(p, bm, kvh, 0, p.rows, split_count(p, info.x, info.z));
-      }
       __syncthreads();  // shared memory is reused by the next segment
     }
     grid_launch_dependents();
@@ -1457,20 +1380,6 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
       if (dc == 0) p.ws_ml[rec] = make_float2(M, L);
     }
   }
-  if (direct) return;
-  // arrival on the target (sequence, kv head, row chunk); the CTA completing it merges
-  __threadfence();
-  __syncthreads();
-  const SplitCount n = split_count(p, P_b, nblk);  // P_b: shared prefix, or the window's first block
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(p.arrive + (static_cast<size_t>(b) * H + kvh) * p.row_chunks + rc, 1);
-    st.merge[0] = prev == n.shared + n.own - 1 ? 1 : 0;
-  }
-  __syncthreads();
-  if (st.merge[0]) {
-    __threadfence();
-    merge_target<D>(p, b, kvh, sg.row0, sg.nrows, n);
-  }
 }
 
 // Prefix sharing for the grid schedule, one warp per sequence b. Sequences are cut
@@ -1488,8 +1397,6 @@ __global__ void __launch_bounds__(128) share_prepass_kernel(const DecodeParams p
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (b >= p.num_seqs) return;
-  // this call's arrival counters of sequence b (one row chunk with sharing)
-  for (int k = lane; k < p.num_kv_heads; k += 32) p.arrive[static_cast<size_t>(b) * p.num_kv_heads + k] = 0;
   const int cap = p.share_cap;  // 2..16
   const int W0 = (b / cap) * cap;
   const int span = min(cap, p.num_seqs - W0);
@@ -1549,6 +1456,84 @@ __global__ void __launch_bounds__(128) share_prepass_kernel(const DecodeParams p
   const int my_ctx = __shfl_sync(kFull, ctx_l, m);
   if (lane == 0)
     p.seq_info[b] = make_int4(P, (b == leader && P > 0) ? members : 0, num_blocks_of(p, my_ctx), my_ctx);
+}
+
+// Log-sum-exp merge of the grid schedule's split partials. One CTA per output row
+// (sequence, query token, head) with MW warps: warp w folds splits w, w+MW, ... into
+// (M_w, L_w, acc_w) with lanes over head_dim, and the CTA combines the MW states.
+constexpr int kMergeMaxWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const DecodeParams p) {
+  constexpr int DPL = D / 32;
+  __shared__ float2 s_ml[kMergeMaxWarps];
+  __shared__ __align__(16) float s_acc[kMergeMaxWarps][D];
+  grid_dependency_wait();
+  const int RQ = p.q_per_seq * p.num_q_heads;
+  const int row = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int MW = blockDim.x >> 5;
+  const int b = row / RQ;
+  const int rq = row % RQ;
+  const int ctx = __ldg(p.context_lens + b);
+  const int nblk = num_blocks_of(p, ctx);
+  const int sb = p.split_blocks;
+  // records: the shared-prefix splits (region 0, with prefix sharing) then the
+  // sequence's own splits (region 1 with prefix sharing, else region 0); with a sliding
+  // window the own blocks start at the window's first block
+  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
+  const int nsh = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
+  const int ns = nsh + (nblk - P_b + sb - 1) / sb;
+  if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
+  const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
+  auto rec_of = [&](int k) -> size_t {
+    return (k < nsh ? static_cast<size_t>(b) * p.share_splits + k
+                    : own_region + static_cast<size_t>(b) * p.num_splits + (k - nsh)) * RQ + rq;
+  };
+  // this warp's maximum: its splits' (m, l) are spread over the lanes
+  float Mw = -INFINITY;
+  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[rec_of(s)].x);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(kFull, Mw, off));
+  float Lw = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < ns; s += MW) {
+    const size_t rec = rec_of(s);
+    const float2 ml = p.ws_ml[rec];
+    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mw);
+    Lw += w * ml.y;
+    const float* src = p.ws_o + rec * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src);
+      acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2*>(src);
+      acc[0] += w * x.x; acc[1] += w * x.y;
+    }
+  }
+  if (lane == 0) s_ml[warp] = make_float2(Mw, Lw);
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) s_acc[warp][lane * DPL + e] = acc[e];
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < MW; ++w) M = fmaxf(M, s_ml[w].x);
+  float L = 0.f;
+  for (int w = 0; w < MW; ++w) L += s_ml[w].x == -INFINITY ? 0.f : s_ml[w].y * fast_exp2(s_ml[w].x - M);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const int i = rq / p.num_q_heads;
+  const int h = rq % p.num_q_heads;
+  uint16_t* dst = p.out + out_offset(p, b, i, h, D);
+  for (int d = threadIdx.x; d < D / 2; d += blockDim.x) {
+    float v0 = 0.f, v1 = 0.f;
+    for (int w = 0; w < MW; ++w) {
+      const float wt = s_ml[w].x == -INFINITY ? 0.f : fast_exp2(s_ml[w].x - M);
+      v0 += wt * s_acc[w][2 * d];
+      v1 += wt * s_acc[w][2 * d + 1];
+    }
+    reinterpret_cast<uint32_t*>(dst)[d] = pack_bf16x2(v0 * inv, v1 * inv);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1670,14 +1655,9 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, block.x, smem);
-  if (p.share_cap) {  // the pre-pass also zeroes this call's arrival counters
+  if (p.share_cap) {
     e = launch_pdl(share_prepass_kernel, dim3(static_cast<unsigned>((p.num_seqs + 3) / 4)), dim3(128), 0,
                    stream, p);
-    if (e != cudaSuccess) return e;
-  } else if (p.num_splits > 1) {
-    const int n = p.num_seqs * p.num_kv_heads * p.row_chunks;
-    e = launch_pdl(grid_reset_kernel, dim3(static_cast<unsigned>(min((n + 255) / 256, 32))), dim3(256), 0, stream,
-                   p.arrive, n);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(p.num_kv_heads * p.row_chunks, p.num_seqs, p.num_splits);
@@ -1687,7 +1667,12 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
                             static_cast<long long>(p.num_seqs) * p.num_splits);
     grid = dim3(static_cast<unsigned>(ctas));
   }
-  return launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
+  e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
+  if (e != cudaSuccess || (p.num_splits <= 1 && !p.share_cap)) return e;
+  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
+  // about four records per warp, at most kMergeMaxWarps warps per row
+  const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + p.share_splits + 3) / 4));
+  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
 }
 
 template <int N>
@@ -1699,17 +1684,14 @@ cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUten
   cudaError_t e = configure_smem(kernel, smem, done_mask);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
-  // the sharing pre-pass, or the reset kernel, zeroes this call's arrival counters first
-  const int windows = p.share_cap > 1 ? (p.num_seqs + p.share_cap - 1) / p.share_cap : p.num_seqs;
   if (p.share_cap > 1) {
+    const int windows = (p.num_seqs + p.share_cap - 1) / p.share_cap;
     e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(256), 0, stream, p);
-  } else {
-    const int n = windows * p.num_kv_heads * p.row_chunks;
-    e = launch_pdl(grid_reset_kernel, dim3(static_cast<unsigned>(min((n + 255) / 256, 32))), dim3(256), 0, stream,
-                   p.arrive, n);
+    if (e != cudaSuccess) return e;
   }
+  e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
+  return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kMergeThreads), 0, stream, p);
 }
 
 template <int D>

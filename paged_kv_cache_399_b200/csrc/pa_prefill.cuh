@@ -9,23 +9,28 @@
 // This is a contraction with hundreds of query rows per kv head, so the query rows go on the
 // MMA's M dimension (the decode kernels put the keys there):
 //   S[128 rows][128 keys] = Q[128 rows][D] . K^T[D][128 keys]    K-major A (Q) and B (K)
-//   softmax per row: thread r of the softmax warpgroup owns row r (TMEM lane r) and all 128
-//   keys of the tile, so the row maximum and sum need no exchange; the running reference
-//   maximum moves only when a tile's maximum exceeds it by more than 2^8 (numerator and
-//   denominator share the reference, so the result is exact either way);
+//   softmax per row over the tile's 128 keys, split between two warpgroups: thread r of
+//   warpgroup h owns row r (TMEM lane r) and keys 64h .. 64h+63, so the two threads of a row
+//   exchange only their partial maxima (shared memory, one named barrier per tile); the
+//   running reference maximum moves only when a tile's maximum exceeds it by more than 2^8
+//   (numerator and denominator share the reference, so the result is exact either way);
+//   each warpgroup keeps its own part of the row sum, joined at the end;
 //   O[128 rows][D] += P[128 rows][128 keys] . V[128 keys][D]     K-major A (P, from shared
 //                                                                memory), MN-major B (V)
+// Two warps per SM sub-partition share the softmax, so one's latencies hide behind the
+// other's work; warpgroup h also rescales and writes columns 64h .. 64h+63 of O.
 // A CTA owns 128 rows = 128 / G consecutive chunk tokens x the G query heads of one kv head
 // (GQA: every row of a CTA reads the same K/V), and walks the key tiles of 8 blocks from
 // the sequence's first block to the block of its last row's position.
 //
-// Roles: warps 0-3 load Q, run the softmax and the epilogue; warp 4 issues the K boxes and
-// warp 5 the V boxes (16 TMA boxes of 2 KB per tile each); warp 6 holds the TMEM allocation
-// and one of its threads issues the MMAs (S of a tile as soon as its K has landed and an S
-// buffer is free; PV of a tile as soon as its P and V are in shared memory). A K stage is
-// released when its S completes, a V stage when its PV completes.
+// Roles: warps 0-7 load Q, run the softmax and the epilogue (two warpgroups); warp 8 issues
+// the K boxes and warp 9 the V boxes (16 TMA boxes of 2 KB per tile each); warp 10 holds the
+// TMEM allocation and one of its threads issues the MMAs (S of a tile as soon as its K has
+// landed and an S buffer is free; PV of a tile as soon as its P and V are in shared memory).
+// A K stage is released when its S completes, a V stage when its PV completes.
 // TMEM: S double buffer in columns [0, 256), O in [256, 384).
-// Shared memory: Q (32 KB), P (32 KB), 2 K stages and 2 V stages of 32 KB, barriers.
+// Shared memory: Q (32 KB), P (32 KB), 2 K stages and 2 V stages of 32 KB, the softmax's
+// exchange area, barriers.
 
 namespace pa {
 
@@ -36,8 +41,9 @@ constexpr int kRows = 128;                        // query rows of a CTA: the MM
 constexpr int kTileBlocks = 8;
 constexpr int kKeys = kTileBlocks * kBlockSize;   // 128 keys per tile
 constexpr int kStages = 2;
-constexpr int kThreads = 224;                     // 7 warps
-constexpr int kKWarp = 4, kVWarp = 5, kMmaWarp = 6;
+constexpr int kThreads = 352;                     // 11 warps
+constexpr int kSoftmaxWarps = 8;                  // two warpgroups, each owning half of the keys
+constexpr int kKWarp = 8, kVWarp = 9, kMmaWarp = 10;
 constexpr int kHalfBytes = kKeys * 128;           // one 64-column half of a K or V tile: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;        // 32 KB
 constexpr int kRowsHalfBytes = kRows * 128;       // one 64-column half of Q or P: 16 KB
@@ -50,9 +56,12 @@ struct Smem {
   static constexpr int offP = offQ + 2 * kRowsHalfBytes;
   static constexpr int offK = offP + 2 * kRowsHalfBytes;
   static constexpr int offV = offK + kStages * kTileBytes;
-  static constexpr int offBars = offV + kStages * kTileBytes;
+  // per tile parity and warpgroup: each row's partial maximum; then the partial row sums
+  static constexpr int offX = offV + kStages * kTileBytes;
+  static constexpr int offBars = offX + (2 * 2 + 2) * kRows * 4;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && offV % 1024 == 0 && offP % 1024 == 0, "swizzled operands");
+  static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct Bars {
@@ -65,6 +74,9 @@ struct Bars {
 __device__ __forceinline__ uint32_t row_chunk_offset(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * kRowsHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
+
+// Named barrier of the two softmax warpgroups (id 1, 256 threads).
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 }  // namespace pfl
 
@@ -93,9 +105,9 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
   if (threadIdx.x == 0) {
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
     for (int i = 0; i < static_cast<int>(sizeof(pfl::Bars) / 8); ++i) mbar_init(all + i, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&bars.s_free[i], 4);  // one arrival per softmax warp
-    mbar_init(&bars.p_full, 4);
-    mbar_init(&bars.q_full, 4);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars.s_free[i], pfl::kSoftmaxWarps);  // one arrival per softmax warp
+    mbar_init(&bars.p_full, pfl::kSoftmaxWarps);
+    mbar_init(&bars.q_full, pfl::kSoftmaxWarps);
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
@@ -267,17 +279,22 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     __syncwarp();
   } else {
     // ------------------------------------------------------------ Q, softmax, epilogue
-    const int r = threadIdx.x;                 // row = TMEM lane
+    const int hk = warp >> 2;                  // warpgroup: keys 64hk .. 64hk+63 of a tile
+    const int r = threadIdx.x & 127;           // row = TMEM lane
     const int tt = r / p.group;                // chunk token of the row (within the CTA)
     const int h = kvh * p.group + (r - tt * p.group);
     const bool valid = tt < ntok;
     const int pos = valid ? pos0 + tt : -1;    // the row's position: keys 0 .. pos visible
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t o_col = tmem + lane_off + pfl::kTmemO + hk * (D / 2);
+    float* xmax = reinterpret_cast<float*>(smem + L::offX);             // [2 parities][2 groups][128]
+    float* xsum = xmax + 4 * pfl::kRows;                                 // [2 groups][128]
     const size_t row_off = (static_cast<size_t>(qs + tok0 + tt) * p.num_q_heads + h) * D;
-    {  // Q row -> shared memory, 128-byte swizzled K-major; zeros for rows past the chunk
+    {  // this warpgroup's half of the Q row -> shared memory, 128-byte swizzled K-major;
+       // zeros for rows past the chunk
       const uint4* src = reinterpret_cast<const uint4*>(p.query + row_off);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int c = hk * 8; c < hk * 8 + 8; ++c) {
         const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(smem + L::offQ + pfl::row_chunk_offset(r, c)) = v;
       }
@@ -285,7 +302,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.q_full);
     }
-    const float cs = p.scale_log2;
+    const float cs = p.scale_log2;             // > 0 or 0: the maximum commutes with it
     float mref = -INFINITY, l = 0.f;
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -294,29 +311,32 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     for (int j = 0; j < nk; ++j) {
       wait(&bars.s_full[j & 1], (j >> 1) & 1);
       tc_fence_after_sync();
-      uint32_t sv[kKeys];
-#pragma unroll
-      for (int q4 = 0; q4 < kKeys / 32; ++q4)
-        tmem_ld32(tmem + lane_off + (j & 1) * kKeys + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(sv + q4 * 32));
+      uint32_t sv[64];
+      tmem_ld32(tmem + lane_off + (j & 1) * kKeys + hk * 64, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tmem + lane_off + (j & 1) * kKeys + hk * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
       tc_wait_ld();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
       // keys past the row's position are masked (the chunk is causal; keys past every row's
-      // position are past the context or belong to later chunk tokens)
-      const int k0 = j * kKeys;
-      const bool edge = k0 + kKeys - 1 > pos;
-      float mx = -INFINITY;
+      // position are past the context or belong to later chunk tokens); scores in log2 units
+      const int k0 = j * kKeys + hk * 64;
+      const bool edge = k0 + 63 > pos;
+      float pmx = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < kKeys; ++k) {
+      for (int k = 0; k < 64; ++k) {
         float x = __uint_as_float(sv[k]) * cs;
         if (edge && k0 + k > pos) x = -INFINITY;
         sv[k] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        pmx = fmaxf(pmx, x);
       }
-      // move the reference when the tile's maximum exceeds it by more than 2^8; O (TMEM) is
-      // rescaled by the whole warp whenever one of its rows moved (tcgen05.ld/st are
-      // warp-collective), the other rows by 1
+      // the row's maximum over both halves of the tile
+      xmax[((j & 1) * 2 + hk) * pfl::kRows + r] = pmx;
+      pfl::softmax_sync();
+      const float mx = fmaxf(pmx, xmax[((j & 1) * 2 + (hk ^ 1)) * pfl::kRows + r]);
+      // move the reference when the tile's maximum exceeds it by more than 2^8; this
+      // warpgroup's half of O (TMEM) is rescaled by the whole warp whenever one of its rows
+      // moved (tcgen05.ld/st are warp-collective), the other rows by 1
       const bool need = mx > mref + pfl::kRescaleLog2 || (mref == -INFINITY && mx != -INFINITY);
       float alpha = 1.f;
       if (need) {
@@ -328,22 +348,21 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         wait(&bars.pv_done, (j - 1) & 1);
         tc_fence_after_sync();
 #pragma unroll
-        for (int q4 = 0; q4 < D / 32; ++q4) {
+        for (int q4 = 0; q4 < 2; ++q4) {
           uint32_t ov[32];
-          const uint32_t oaddr = tmem + lane_off + pfl::kTmemO + q4 * 32;
-          tmem_ld32(oaddr, ov);
+          tmem_ld32(o_col + q4 * 32, ov);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(oaddr, ov);
+          tmem_st32(o_col + q4 * 32, ov);
         }
         tc_wait_st();
       }
       if (need) mref = mx;
       const float mu = mref == -INFINITY ? 0.f : mref;
-      uint32_t pk[kKeys / 2];
+      uint32_t pk[32];
 #pragma unroll
-      for (int k = 0; k < kKeys; k += 2) {
+      for (int k = 0; k < 64; k += 2) {
         const float p0 = fast_exp2(__uint_as_float(sv[k]) - mu);
         const float p1 = fast_exp2(__uint_as_float(sv[k + 1]) - mu);
         l += p0 + p1;
@@ -352,23 +371,26 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       // the P buffer was read by the PV of tile j-1
       if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
 #pragma unroll
-      for (int c = 0; c < kKeys / 8; ++c)
-        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, c)) =
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, hk * 8 + c)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full);
     }
-    // ---- epilogue: O / l once the last PV has completed
+    // ---- epilogue: O / l once the last PV has completed; l = the two warpgroups' parts
+    xsum[hk * pfl::kRows + r] = l;
+    pfl::softmax_sync();
+    l += xsum[(hk ^ 1) * pfl::kRows + r];
     wait(&bars.pv_done, (nk - 1) & 1);
     tc_fence_after_sync();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint4* dst = reinterpret_cast<uint4*>(p.out + row_off);
+    uint4* dst = reinterpret_cast<uint4*>(p.out + row_off) + hk * 8;
 #pragma unroll
-    for (int q4 = 0; q4 < D / 32; ++q4) {
+    for (int q4 = 0; q4 < 2; ++q4) {
       uint32_t ov[32];
-      tmem_ld32(tmem + lane_off + pfl::kTmemO + q4 * 32, ov);
+      tmem_ld32(o_col + q4 * 32, ov);
       tc_wait_ld();
       if (ok && valid) {
 #pragma unroll

@@ -8,9 +8,8 @@
 // walk the same enumeration of (sequence, kv-head index, row chunk, tile) and split it
 // into equal contiguous ranges, one per group, computed in the kernel from context_lens
 // (no pre-pass); the S CTAs of a group therefore read the kv-head slices of the same
-// blocks at about the same time. A unit cut by range boundaries leaves one partial record
-// per piece; at its end every CTA adds one to the arrival counter of each cut unit it holds
-// a piece of, and the CTA whose arrival completes the unit merges its pieces in CTA order.
+// blocks at about the same time. A unit cut by a range boundary leaves partial records,
+// combined afterwards by tcm_merge_kernel.
 //
 // Per tile, with Q of the unit's N (16 or 32) rows:
 //   S^T[128 tok][N]  = K[128 tok][D] . Q^T[D][N]           tcgen05.mma M=128, K-major A and B
@@ -49,6 +48,7 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
 constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
+constexpr int kMergeThreads = 1024;  // one warp per row of a unit (N <= 32)
 
 template <int N>
 struct Smem {
@@ -61,7 +61,7 @@ struct Smem {
   // per softmax warpgroup: [3][4 warps][N/2] floats (2 maxima buffers, 1 sum), [2][4] votes
   static constexpr int kRedWg = 3 * 4 * (N / 2) + 8;
   static constexpr int offRed = offV + kVStages * kStageBytes;
-  static constexpr int offScan = offRed + 2 * kRedWg * 4;     // [11] int64, the start, 2 merge flags
+  static constexpr int offScan = offRed + 2 * kRedWg * 4;     // [11] int64, then the start
   static constexpr int offBars = offScan + 128;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && kQ % 1024 == 0, "swizzled operands need 1024-B alignment");
@@ -200,9 +200,6 @@ __device__ __forceinline__ void named_sync_softmax(int wg) {
   asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
 }
 
-// Named barrier of both softmax warpgroups (id 3, 256 threads).
-__device__ __forceinline__ void named_sync_softmax_all() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
-
 // Column reduction of a warp: lane l holds V values (columns 0..V-1); on return every
 // lane holds the reduction over all 32 lanes of column (l % V). Halving exchange: at
 // each step a lane keeps the half of its columns selected by one lane bit and sends
@@ -250,7 +247,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   if (smem_u32(smem) & 1023u) {  // the swizzled operand layouts need a 1024-aligned base
-    if (threadIdx.x == 0) record_error(kErrSchedule);
+    if (threadIdx.x == 0) {
+      record_error(kErrSchedule);
+      p.tc_desc[c] = make_int4(-1, 0, 0, 0);
+    }
     return;
   }
   if (threadIdx.x == 0) {
@@ -317,15 +317,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     }
     __syncthreads();
   }
-  // sequences without a visible key (context length 0) get zero rows
-  for (int b = c; b < p.num_seqs; b += gridDim.x) {
-    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;  // uniform
-    const int rq = p.q_per_seq * p.num_q_heads;
-    uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * rq * D);
-    for (int e = threadIdx.x; e < rq * D / 8; e += blockDim.x) o[e] = make_uint4(0, 0, 0, 0);
-  }
   const int n = static_cast<int>(t1 - t0);
   if (n <= 0) {  // uniform: no tiles for this CTA
+    if (threadIdx.x == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     grid_launch_dependents();
     return;
   }
@@ -596,12 +590,6 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       float L_c, m_c;  // l and the reference maximum of column cb + (lane % NC)
     } pend;
     pend.on = false;
-    // The cut units this CTA holds a piece of (its first unit and its last one, at most):
-    // counter index, the unit's first and last group, and the record slot of the first piece.
-    struct Cut {
-      int idx, gi_first, gi_last, first_slot, w, k;
-    } cut[2];
-    int ncut = 0;
     auto flush = [&](Pending& e) {
       e.on = false;
       wait(&bars.pv_done[e.g & 1], (e.g >> 1) & 1);
@@ -798,21 +786,15 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         pend.slot = j == 0 ? 2 * c : 2 * c + 1;
         pend.L_c = (rl[jc] + rl[NC + jc]) + (rl[2 * NC + jc] + rl[3 * NC + jc]);
         pend.m_c = mref_c;
-        if (!pend.complete) {
-          // a piece of a cut unit: the unit's global tiles are [Tf, E); the group holding
-          // global tile T is ((T + 1) * NGe - 1) / W; its first piece sits in the first
-          // group's slot 2c (the unit starts that CTA's range) or 2c + 1, later pieces in
-          // slot 2c of their CTA (the unit is their first)
-          const long long Tf = t0 + g - w.x;
-          const long long E = Tf + w.tiles;
-          Cut& cu = cut[ncut++];
-          cu.gi_first = static_cast<int>(((Tf + 1) * NGe - 1) / W);
-          cu.gi_last = static_cast<int>((E * NGe - 1) / W);
-          const int cf = cu.gi_first * S + li;
-          cu.first_slot = Tf == static_cast<long long>(cu.gi_first) * W / NGe ? 2 * cf : 2 * cf + 1;
-          cu.idx = (w.w * p.num_kv_heads + kvh) * p.row_chunks + rc;
-          cu.w = w.w;
-          cu.k = w.k;
+        if (g == n - 1 && wg == 0 && t == 0) {
+          // the merge descriptor: this CTA's last unit continues in the next CTAs and
+          // started here, so this CTA holds its first piece
+          int4 dsc = make_int4(-1, 0, 0, 0);
+          if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
+            const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
+            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.w, w.k);
+          }
+          p.tc_desc[c] = dsc;
         }
       }
       w.next(p, upb, nwin);
@@ -820,62 +802,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     if (pend.on) flush(pend);
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
-    } else if (ncut > 0) {
-      // ---- arrivals on the cut units; the CTA completing a unit merges its pieces in CTA
-      // order (a fixed order: the result does not depend on which CTA arrived last)
-      __threadfence();  // this CTA's records are visible device-wide before its arrival
-      tcm::named_sync_softmax_all();
-      int* flag = reinterpret_cast<int*>(smem + L::offScan + 104);  // after the range start
-      for (int q = 0; q < ncut; ++q) {
-        if (warp == 0 && lane == 0) {
-          const int prev = atomicAdd(p.arrive + cut[q].idx, 1);
-          flag[q] = prev == cut[q].gi_last - cut[q].gi_first ? 1 : 0;
-        }
-      }
-      tcm::named_sync_softmax_all();
-      for (int q = 0; q < ncut; ++q) {
-        if (!flag[q]) continue;  // uniform: shared memory flag
-        __threadfence();
-        const Cut cu = cut[q];
-        const int np = cu.gi_last - cu.gi_first + 1;
-        const int b0 = cu.w * cap;
-        const int m = min(cap, p.num_seqs - b0);
-        const int kvh_u = unit_kvh(cu.k), rc_u = unit_rc(cu.k);
-        const int nr = min(N, m * rpm - rc_u * N);
-        const float* recs = p.records;
-        const int rs = p.rec_stride;
-        auto rec_of = [&](int k) {
-          return recs + static_cast<size_t>(k == 0 ? cu.first_slot : 2 * ((cu.gi_first + k) * S + li)) * rs;
-        };
-        const int tid = threadIdx.x;  // the 256 softmax threads
-        for (int task = tid; task < nr * (D / 4); task += tcm::kSoftmaxWarps * 32) {
-          const int r = task / (D / 4), c4 = task % (D / 4);
-          float M = -INFINITY;
-          for (int k = 0; k < np; ++k) M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(rec_of(k) + N * D) + r).x);
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          float l = 0.f;
-          for (int k = 0; k < np; ++k) {
-            const float* rk = rec_of(k);
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(rk + N * D) + r);
-            const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
-            l += ml.y * wk;
-            const float4 o4 = __ldcg(reinterpret_cast<const float4*>(rk + r * D) + c4);
-            acc.x = fmaf(o4.x, wk, acc.x);
-            acc.y = fmaf(o4.y, wk, acc.y);
-            acc.z = fmaf(o4.z, wk, acc.z);
-            acc.w = fmaf(o4.w, wk, acc.w);
-          }
-          const float inv = l > 0.f ? 1.f / l : 0.f;
-          const int cg = rc_u * N + r;
-          const int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
-          const int gg = cg - mem * rpm - i * p.group;
-          uint2 packed;
-          packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-          packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-          reinterpret_cast<uint2*>(p.out + (static_cast<size_t>((b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
-                                            kvh_u * p.group + gg) * D)[c4] = packed;
-        }
-      }
+      if (wg == 0 && t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     }
   }
   grid_launch_dependents();
@@ -883,6 +810,94 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   __syncthreads();
   tc_fence_after_sync();
   if (warp == tcm::kMmaWarp) tmem_dealloc(tmem, 4 * N < 32 ? 32 : 4 * N);
+}
+
+// Combines the partial records of every unit (window, kv head, row chunk) cut by a range
+// boundary (one CTA per
+// decode CTA; the descriptor of CTA c names the unit whose first piece c holds and the
+// last CTA c1 with a piece of it: the pieces are in record slots desc.x, then 2c' for
+// c' = c+S, c+2S, ..., c1 (the same CTA of the following groups), in that order), then
+// writes zeros for sequences with no keys.
+template <int N>
+__global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const DecodeParams p) {
+  constexpr int D = tcm::kD;
+  grid_dependency_wait();
+  const int c = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int4 dsc = p.tc_desc[c];
+  if (dsc.x >= 0) {
+    const int cap = p.share_cap > 1 ? p.share_cap : 1;
+    const int rpm = p.rows;
+    const int b0 = dsc.z * cap;  // the window's first sequence
+    const int m = min(cap, p.num_seqs - b0);
+    const int S = p.tc_group;
+    const int kvh = c % S + S * (dsc.w / p.row_chunks);
+    const int rc = dsc.w % p.row_chunks;
+    const int nrows = min(N, m * rpm - rc * N);
+    const int pieces = 1 + (dsc.y - c) / S;
+    const float* recs = p.records;
+    const int rs = p.rec_stride, slot0 = dsc.x;
+    auto rec_of = [=](int k) {
+      return recs + static_cast<size_t>(k == 0 ? slot0 : 2 * (c + k * S)) * rs;
+    };
+    // one row per warp: lanes take the pieces for the maximum and the weights, then each
+    // lane accumulates 4 of the D columns over the pieces in order, 4 pieces' loads at a time
+    for (int r = warp; r < nrows; r += tcm::kMergeThreads / 32) {
+      float M = -INFINITY;
+      for (int k = lane; k < pieces; k += 32) M = fmaxf(M, reinterpret_cast<const float2*>(rec_of(k) + N * D)[r].x);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float l = 0.f;
+      if (M != -INFINITY) {
+        for (int k0 = 0; k0 < pieces; k0 += 32) {
+          float wk = 0.f, lk = 0.f;
+          if (k0 + lane < pieces) {
+            const float2 ml = reinterpret_cast<const float2*>(rec_of(k0 + lane) + N * D)[r];
+            wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+            lk = ml.y * wk;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
+          l += lk;
+          const int kn = min(32, pieces - k0);
+          for (int kk = 0; kk < kn; kk += 4) {
+            float4 o4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              o4[u] = kk + u < kn ? reinterpret_cast<const float4*>(rec_of(k0 + kk + u) + r * D)[lane]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float wb = __shfl_sync(kFull, wk, (kk + u) & 31);
+              if (kk + u < kn) {
+                acc.x = fmaf(o4[u].x, wb, acc.x);
+                acc.y = fmaf(o4[u].y, wb, acc.y);
+                acc.z = fmaf(o4[u].z, wb, acc.z);
+                acc.w = fmaf(o4[u].w, wb, acc.w);
+              }
+            }
+          }
+        }
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int cg = rc * N + r;
+      const int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+      const int gg = cg - mem * rpm - i * p.group;
+      uint2 packed;
+      packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      reinterpret_cast<uint2*>(p.out + (static_cast<size_t>((b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
+                                        kvh * p.group + gg) * D)[lane] = packed;
+    }
+  }
+  // sequences without a visible key (context length 0) get zero rows
+  const int rq = p.q_per_seq * p.num_q_heads;
+  for (int b = c; b < p.num_seqs; b += gridDim.x) {
+    if (num_blocks_of(p, __ldg(p.context_lens + b)) != 0) continue;
+    uint16_t* o = p.out + static_cast<size_t>(b) * rq * D;
+    for (int e = threadIdx.x; e < rq * D; e += blockDim.x) o[e] = 0;
+  }
 }
 
 // Prefix sharing: the shared prefix of each window of `cap` consecutive sequences, in
@@ -901,9 +916,6 @@ __global__ void __launch_bounds__(256) tcm_share_prepass(const DecodeParams p) {
     first_diff = INT_MAX;
     pcap_s = m >= 2 ? INT_MAX : 0;
   }
-  // this call's arrival counters of the window's units
-  for (int k = threadIdx.x; k < p.num_kv_heads * p.row_chunks; k += blockDim.x)
-    p.arrive[static_cast<size_t>(w) * p.num_kv_heads * p.row_chunks + k] = 0;
   __syncthreads();
   if (m >= 2 && static_cast<int>(threadIdx.x) < m) {  // thread jj: member jj (cap <= 32)
     const int cx = __ldg(p.context_lens + b0 + threadIdx.x);

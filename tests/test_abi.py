@@ -80,9 +80,7 @@ def test_decode_rejects_bad_arguments_before_launch(pa):
     assert plan.num_splits == 4
     assert _decode_raw(lib, plan=ctypes.byref(plan)) == pa.PA_ERR_WORKSPACE
     need = pa.pa_decode_workspace_size(plan, 2, 1, 4, 2, 64, 4)
-    # records (o and (m, l) of every split and query row), 256-byte aligned, then one arrival
-    # counter per output target (sequence, kv head)
-    assert need == -(-(2 * 4 * 1 * 4 * (64 + 2) * 4) // 256) * 256 + 4 * 2 * 2
+    assert need == 2 * 4 * 1 * 4 * (64 + 2) * 4
     assert _decode_raw(lib, plan=ctypes.byref(plan), ws=96 * 1024, ws_bytes=need - 1) == pa.PA_ERR_WORKSPACE
     bad = pa.pa_plan_t.from_buffer_copy(plan)
     bad.num_splits += 1
