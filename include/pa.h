@@ -275,8 +275,8 @@ PA_API pa_status_t pa_decode_fp8(void* out, const void* query, const void* key_c
  * attends to keys 0 .. pos: out row = sum_t softmax_t(scale * q . k_t) v_t over them, rounded
  * to bf16 from fp32 accumulation (tensor cores: tcgen05.mma, bf16 operands, fp32
  * accumulators in tensor memory). max_query_len: host-known bound on every qlen_b (sizes
- * the grid). Supported: head_dim 128, block_size 16, 128 % (num_q_heads / num_kv_heads) == 0
- * (else PA_ERR_UNSUPPORTED). Preconditions (device data): qlen_b <= max_query_len and
+ * the grid). scale: finite and >= 0 (else PA_ERR_INVALID_ARG). Supported: head_dim 128,
+ * block_size 16, 128 % (num_q_heads / num_kv_heads) == 0 (else PA_ERR_UNSUPPORTED). Preconditions (device data): qlen_b <= max_query_len and
  * qlen_b <= context_lens[b] <= max_blocks_per_seq * block_size, block ids as for pa_decode;
  * a sequence with context_lens[b] < qlen_b gets no rows written. No workspace; nothing is
  * allocated; asynchronous on `stream`; host argument errors as pa_decode's. Zero sequences,

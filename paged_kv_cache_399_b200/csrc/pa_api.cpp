@@ -629,8 +629,9 @@ pa_status_t pa_prefill(void* out, const void* query, const void* key_cache, cons
                        int32_t num_seqs, int32_t num_query_tokens, int32_t max_query_len, int32_t num_q_heads,
                        int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
                        int64_t num_blocks, float scale, pa_stream_t stream) {
+  // the kernel takes each row's maximum over the raw scores, so the scale must not be negative
   if (num_seqs < 0 || num_query_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-      head_dim <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
+      head_dim <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale) || scale < 0.f)
     return PA_ERR_INVALID_ARG;
   if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
   const int group = num_q_heads / num_kv_heads;

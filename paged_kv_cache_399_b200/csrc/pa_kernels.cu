@@ -1679,9 +1679,10 @@ template <int N>
 cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                        cudaStream_t stream, int* occupancy) {
   constexpr int smem = tcm::Smem<N>::kBytes;
-  auto kernel = decode_tcm_kernel<N>;
-  static unsigned long long done_mask = 0;
-  cudaError_t e = configure_smem(kernel, smem, done_mask);
+  // the sliding-window instance only for plans with a window
+  auto kernel = p.window > 0 ? decode_tcm_kernel<N, true> : decode_tcm_kernel<N, false>;
+  static unsigned long long done_mask[2] = {0, 0};  // one per instance
+  cudaError_t e = configure_smem(kernel, smem, done_mask[p.window > 0 ? 1 : 0]);
   if (e != cudaSuccess) return e;
   if (occupancy) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occupancy, kernel, tcm::kThreads, smem);
   if (p.share_cap > 1) {

@@ -319,21 +319,26 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
       // keys past the row's position are masked (the chunk is causal; keys past every row's
-      // position are past the context or belong to later chunk tokens); scores in log2 units
+      // position are past the context or belong to later chunk tokens): only tiles that reach
+      // past the row's position take the mask. The maximum is taken over the raw scores
+      // (the scale is >= 0) and the scale is applied once, in the exponent's FMA.
       const int k0 = j * kKeys + hk * 64;
       const bool edge = k0 + 63 > pos;
       float pmx = -INFINITY;
+      if (edge) {
+        const int nvis = min(64, max(0, pos - k0 + 1));  // keys k < nvis are visible
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        float x = __uint_as_float(sv[k]) * cs;
-        if (edge && k0 + k > pos) x = -INFINITY;
-        sv[k] = __float_as_uint(x);
-        pmx = fmaxf(pmx, x);
+        for (int k = 0; k < 64; ++k)
+          if (k < nvis) pmx = fmaxf(pmx, __uint_as_float(sv[k]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) pmx = fmaxf(pmx, __uint_as_float(sv[k]));
       }
-      // the row's maximum over both halves of the tile
+      // the row's maximum over both halves of the tile, in log2 units
       xmax[((j & 1) * 2 + hk) * pfl::kRows + r] = pmx;
       pfl::softmax_sync();
-      const float mx = fmaxf(pmx, xmax[((j & 1) * 2 + (hk ^ 1)) * pfl::kRows + r]);
+      const float rmx = fmaxf(pmx, xmax[((j & 1) * 2 + (hk ^ 1)) * pfl::kRows + r]);
+      const float mx = rmx == -INFINITY ? -INFINITY : rmx * cs;
       // move the reference when the tile's maximum exceeds it by more than 2^8; this
       // warpgroup's half of O (TMEM) is rescaled by the whole warp whenever one of its rows
       // moved (tcgen05.ld/st are warp-collective), the other rows by 1
@@ -360,14 +365,30 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       }
       if (need) mref = mx;
       const float mu = mref == -INFINITY ? 0.f : mref;
+      // p = 2^(s * scale - reference): one FMA and one exponential per key
       uint32_t pk[32];
+      float l0 = 0.f, l1 = 0.f;
+      if (edge) {
+        const int nvis = min(64, max(0, pos - k0 + 1));
 #pragma unroll
-      for (int k = 0; k < 64; k += 2) {
-        const float p0 = fast_exp2(__uint_as_float(sv[k]) - mu);
-        const float p1 = fast_exp2(__uint_as_float(sv[k + 1]) - mu);
-        l += p0 + p1;
-        pk[k / 2] = pack_bf16x2(p0, p1);
+        for (int k = 0; k < 64; k += 2) {
+          const float p0 = k < nvis ? fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu)) : 0.f;
+          const float p1 = k + 1 < nvis ? fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu)) : 0.f;
+          l0 += p0;
+          l1 += p1;
+          pk[k / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu));
+          l0 += p0;
+          l1 += p1;
+          pk[k / 2] = pack_bf16x2(p0, p1);
+        }
       }
+      l += l0 + l1;
       // the P buffer was read by the PV of tile j-1
       if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
 #pragma unroll

@@ -73,7 +73,9 @@ struct Bars {
   uint64_t drain;
 };
 
-// Tiles of every unit of window w (one thread, for the partition scan).
+// Tiles of every unit of window w (one thread, for the partition scan). kWin: the plan has a
+// sliding window (a member's own blocks start at its window's first block).
+template <bool kWin>
 __device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
   const int cap = p.share_cap > 1 ? p.share_cap : 1;
   const int b0 = w * cap;
@@ -85,7 +87,8 @@ __device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
     const int cx = __ldg(p.context_lens + b0 + jj);
     const int nb = num_blocks_of(p, cx);
     // own blocks: after the shared prefix, from the sliding window's first block on
-    tiles += (nb - min(nb, max(P, window_first_block(p, cx))) + kTileBlocks - 1) / kTileBlocks;
+    const int lo = kWin ? min(nb, max(P, window_first_block(p, cx))) : P;
+    tiles += (nb - lo + kTileBlocks - 1) / kTileBlocks;
   }
   return tiles;
 }
@@ -96,7 +99,8 @@ __device__ __forceinline__ int window_tiles(const DecodeParams& p, int w) {
 // walks the window's tiles: the shared prefix (P blocks, read once for all members) then
 // each member's own blocks (with a sliding window, from its window's first block). Lane jj
 // holds member jj's context length and blocks, so moving between members takes shuffles,
-// not loads.
+// not loads. kWin: the plan has a sliding window.
+template <bool kWin>
 struct Walk {
   int w, k, x;          // window, unit of the window, tile of the unit
   int b0, m, P, tiles;  // window: first sequence, members, shared blocks, tiles of a unit
@@ -110,7 +114,7 @@ struct Walk {
   __device__ __forceinline__ void member(int jj) {
     ctx = __shfl_sync(kFull, lctx, jj);
     nblk = __shfl_sync(kFull, lnblk, jj);
-    lo = __shfl_sync(kFull, llo, jj);
+    lo = kWin ? __shfl_sync(kFull, llo, jj) : P;
   }
   __device__ __forceinline__ void window(const DecodeParams& p) {
     const int lane = threadIdx.x & 31;
@@ -126,7 +130,7 @@ struct Walk {
     if (lane < m) {
       lctx = __ldg(p.context_lens + b0 + lane);
       lnblk = num_blocks_of(p, lctx);
-      llo = min(lnblk, max(P, window_first_block(p, lctx)));
+      llo = kWin ? min(lnblk, max(P, window_first_block(p, lctx))) : P;
       lctx = min(lctx, lnblk * kBlockSize);
     }
     int t = lane < m ? own_tiles_lane() : 0;
@@ -228,7 +232,9 @@ __device__ __forceinline__ float column_reduce(float (&v)[V], int lane) {
 
 }  // namespace tcm
 
-template <int N>
+// kWin: the plan has a sliding window (its own instance, so plans without one run none of
+// the window's per-tile work).
+template <int N, bool kWin>
 __global__ void __launch_bounds__(tcm::kThreads, 1)
 decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
@@ -283,7 +289,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     const int chunk = (nwin + tcm::kThreads - 1) / tcm::kThreads;
     const int s0 = min(nwin, static_cast<int>(threadIdx.x) * chunk), s1 = min(nwin, s0 + chunk);
     long long local = 0;
-    for (int ww = s0; ww < s1; ++ww) local += static_cast<long long>(tcm::window_tiles(p, ww)) * upb;
+    for (int ww = s0; ww < s1; ++ww) local += static_cast<long long>(tcm::window_tiles<kWin>(p, ww)) * upb;
     long long v = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -306,7 +312,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     if (local > 0 && t0 < t1 && t0 >= excl && t0 < excl + local) {
       long long acc = excl;
       for (int ww = s0; ww < s1; ++ww) {
-        const long long tb = static_cast<long long>(tcm::window_tiles(p, ww)) * upb;
+        const long long tb = static_cast<long long>(tcm::window_tiles<kWin>(p, ww)) * upb;
         if (t0 < acc + tb) {
           start[0] = ww;
           start[1] = static_cast<int>(t0 - acc);
@@ -326,7 +332,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   // unit k of a sequence -> kv head and row chunk of this CTA
   auto unit_kvh = [&](int k) { return li + S * (k / p.row_chunks); };
   auto unit_rc = [&](int k) { return k % p.row_chunks; };
-  tcm::Walk w0;
+  tcm::Walk<kWin> w0;
   w0.w = start[0];
   w0.window(p);  // every warp: its lanes hold the window's members
   w0.k = start[1] / w0.tiles;
@@ -351,9 +357,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     uint64_t* full = is_k ? bars.k_full : bars.v_full;
     uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
     const int stage_off = is_k ? L::offK : L::offV;
-    tcm::Walk w = w0;
+    tcm::Walk<kWin> w = w0;
     const int oob = static_cast<int>(p.num_blocks);  // block id past the pool: TMA fills zeros
-    auto block_id = [&](const tcm::Walk& at) {
+    auto block_id = [&](const tcm::Walk<kWin>& at) {
       const int blk = at.bstart() + lane;
       return (lane < kTileBlocks && blk < at.bend())
                  ? __ldg(p.block_tables + static_cast<size_t>(at.row()) * p.max_blocks + blk)
@@ -396,7 +402,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       const int s = g % stages;
       const int kvh = unit_kvh(w.k);
       const int ph = __shfl_sync(kFull, phys_next, lane & (kTileBlocks - 1));
-      tcm::Walk wn = w;
+      tcm::Walk<kWin> wn = w;
       wn.next(p, upb, nwin);
       if (g + 1 < n) phys_next = block_id(wn);
       if (g >= stages) ok = __all_sync(kFull, mbar_wait_bounded(&empty[s], ((g / stages) - 1) & 1));
@@ -424,14 +430,14 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, N, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, N, 1, 1);
-      tcm::Walk w = w0;      // position of the next S
+      tcm::Walk<kWin> w = w0;      // position of the next S
       int js = -1;           // unit counter of the S issued last
       int gs = 0, gp = 0;    // next tile to issue S for / PV for (gp <= gs <= gp + 3)
       int ring = 0;          // per tile in flight: bit 2(g&3) O buffer, bit 2(g&3)+1 first of unit
       int zring = 0;         // per tile in flight, byte g&3: V rows to clear (bit 0 on, block, row)
       int hring = 0;         // per tile in flight, byte g&3: sliding window, rows 0 .. r-1 of the
                              // tile's first block to clear (bit 0 on, r)
-      const int win = p.window;
+      const int win = kWin ? p.window : 0;
       bool ok = true;
       unsigned long long idle_since = 0;
       unsigned idle_polls = 0;
@@ -570,8 +576,8 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     float* red = reinterpret_cast<float*>(smem + L::offRed) + wg * L::kRedWg;
     int* votes = reinterpret_cast<int*>(red + 3 * 4 * NC);  // [2][4 warps]
     const float cs = p.scale_log2;
-    const int win = p.window;  // sliding window (keys lim - win + 1 .. lim of a row), 0 = none
-    tcm::Walk w = w0;
+    const int win = kWin ? p.window : 0;  // sliding window (keys lim - win + 1 .. lim of a row), 0 = none
+    tcm::Walk<kWin> w = w0;
     int j = -1, first_x = 0, kvh = 0, rc = 0, nrows = 0, minlim = 0;
     float mref_c = -INFINITY;  // reference maximum of column cb + (lane % NC)
     float mref[NC], lpart[NC];

@@ -351,6 +351,7 @@ def test_prefill_rejects_bad_arguments_before_launch(pa):
     assert call(out=8192 + 8) == pa.PA_ERR_INVALID_ARG     # misaligned
     assert call(cl=81920 + 2) == pa.PA_ERR_INVALID_ARG
     assert call(scale=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert call(scale=-0.5) == pa.PA_ERR_INVALID_ARG        # the row maximum is taken on raw scores
     assert call(B=-1) == pa.PA_ERR_INVALID_ARG
     assert call(B=0) == pa.PA_OK and call(T=0) == pa.PA_OK and call(mq=0) == pa.PA_OK   # no-ops
     assert call(mq=3_000_000) == pa.PA_ERR_UNSUPPORTED     # more tiles than the grid holds

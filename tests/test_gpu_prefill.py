@@ -140,3 +140,13 @@ def test_prefill_full_size_sampled_rows(oracle_lib):
     got = torch.stack([out[int(w.query_start[b]) + i, h] for b, i, h in rows])
     assert_close(got, ref, "chunked_prefill sampled rows")
     assert torch.equal(dw.step(write=False), out)   # repeatable bits
+
+
+def test_prefill_zero_scale_is_the_mean_of_visible_values(oracle_lib):
+    """scale 0: every visible key has the same weight, so each row is the mean of the values
+    it sees (the kernel takes the row maximum over raw scores; 0 must not turn masked keys
+    into NaN)."""
+    w = workloads.build_prefill("zero_scale", 5300, [300, 130, 77], [200, 5, 77], 32, 8, 128, scale=0.0)
+    _, _, ref = _oracle(oracle_lib, w)
+    out = DevicePrefill(w).step()
+    assert_close(out, ref, "zero scale")
