@@ -140,9 +140,9 @@ typedef struct {
                             sliding_window tokens only, keys pos - W + 1 .. pos (vLLM
                             study notes §3.6.3); table entries wholly before every row's
                             window are never read (the pages point them at the null
-                            block 0, §5.5). Grid schedule, mma.sync or CUDA-core path;
-                            with the tcgen05 path, the persistent schedule or
-                            share_prefix: PA_ERR_UNSUPPORTED. 0 = no window */
+                            block 0, §5.5). Grid schedule on the mma.sync or CUDA-core
+                            path, or the tcgen05 path; with share_prefix or the mma.sync
+                            persistent schedule: PA_ERR_UNSUPPORTED. 0 = no window */
   int32_t kv_cache_dtype; /* pa_kv_dtype_t of the pools the plan will decode (0 = bf16) */
 } pa_plan_hints_t;
 

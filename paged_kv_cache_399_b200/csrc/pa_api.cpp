@@ -114,6 +114,42 @@ bool encode_pool_map_uncached(CUtensorMap* map, const void* base, int64_t num_bl
   return r == CUDA_SUCCESS;
 }
 
+// Query rows of the tcgen05 decode as TMA boxes: the query [tokens][H_q][D] as a 3-D map
+// {D, H_q, tokens}, box {64 of D, group heads, box_tokens tokens} with the 128-byte swizzle
+// (the layout of the kernel's K-major Q operand). Cached like the pool maps.
+bool encode_query_map(CUtensorMap* map, const void* base, int64_t tokens, int32_t num_q_heads, int32_t head_dim,
+                      int32_t group, int32_t box_tokens) {
+  struct Entry {
+    const void* base;
+    int64_t tokens;
+    int32_t num_q_heads, head_dim, group, box_tokens;
+    CUtensorMap map;
+  };
+  thread_local Entry cache[4] = {};
+  thread_local int next = 0;
+  for (const Entry& e : cache)
+    if (e.base == base && e.base != nullptr && e.tokens == tokens && e.num_q_heads == num_q_heads &&
+        e.head_dim == head_dim && e.group == group && e.box_tokens == box_tokens) {
+      *map = e.map;
+      return true;
+    }
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(head_dim) * num_q_heads * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(box_tokens)};
+  cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                  elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cache[next] = Entry{base, tokens, num_q_heads, head_dim, group, box_tokens, *map};
+  next = (next + 1) & 3;
+  return true;
+}
+
 // ----------------------------------------------------------------- plan
 
 // Blocks of one sequence's table that a decode reads: every block without a window; with
@@ -435,7 +471,7 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
   const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
 
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tq = {};
   if (!encode_pool_map(&tk, key_cache, num_blocks, num_kv_heads, head_dim, kv_dtype) ||
       !encode_pool_map(&tv, value_cache, num_blocks, num_kv_heads, head_dim, kv_dtype))
     return PA_ERR_CUDA;
@@ -470,6 +506,16 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     p.records = reinterpret_cast<float*>(ws);
     if (plan->share_cap > 1) p.win_prefix = reinterpret_cast<int32_t*>(ws + tcm_prefix_offset(*plan, head_dim));
     p.tc_desc = reinterpret_cast<int4*>(ws + tcm_desc_offset(*plan, head_dim));
+    // Q rows by TMA: a row chunk of N rows is N / G query tokens of G heads when G divides N;
+    // a shared-prefix window is share_cap * q_per_seq tokens (share_cap * rows <= N)
+    const int group = num_q_heads / num_kv_heads;
+    if (plan->share_cap > 1)
+      p.q_box = plan->share_cap * q_per_seq;
+    else if (plan->rows_per_cta % group == 0)
+      p.q_box = plan->rows_per_cta / group;
+    if (p.q_box > 0 && !encode_query_map(&tq, query, static_cast<int64_t>(num_seqs) * q_per_seq, num_q_heads,
+                                         head_dim, group, p.q_box))
+      return PA_ERR_CUDA;
     // CTAs per group: the largest divisor of H_kv that the grid holds
     p.tc_group = 1;
     for (int sz = num_kv_heads; sz >= 1; --sz)
@@ -507,7 +553,7 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
       p.seq_info = reinterpret_cast<int4*>(ws + align256(recs * (static_cast<size_t>(head_dim) + 2) * 4));
     }
   }
-  cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, kv_dtype, tk, tv,
+  cudaError_t e = pa::launch_decode(p, plan->path, plan->schedule, head_dim, kv_dtype, tk, tv, tq,
                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -75,6 +75,10 @@ struct DecodeParams {
   int4* tc_desc;
   int32_t tc_group;              // tcgen05 path: CTAs per group (a divisor of num_kv_heads)
   int32_t* win_prefix;           // tcgen05 path with prefix sharing: shared blocks per window
+  // tcgen05 path: query tokens of one TMA box of Q rows ({64 of D, group heads, q_box
+  // tokens}: the rows of one row chunk, or of a shared-prefix window); 0 = Q rows are
+  // loaded with plain loads (a group that does not divide the MMA's N)
+  int32_t q_box;
 };
 
 // Host-side checks of a decode call's shapes and (when non-null) its plan, the ones
@@ -89,9 +93,10 @@ constexpr int kKvBf16 = 0;
 constexpr int kKvE4M3 = 1;
 
 // Launch the decode (pre-pass + persistent kernel, or grid kernel + merge) over pools of
-// element type kv_dtype.
+// element type kv_dtype. tmap_q: the query map of a tcgen05 plan with p.q_box > 0 (else
+// unused).
 cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim, int kv_dtype,
-                          const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
+                          const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, const CUtensorMap& tmap_q,
                           cudaStream_t stream);
 
 // Chunked-prefill attention (pa_prefill.cuh): one CTA per (kv head, sequence, tile of

@@ -1677,7 +1677,7 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
 
 template <int N>
 cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                       cudaStream_t stream, int* occupancy) {
+                       const CUtensorMap& tq, cudaStream_t stream, int* occupancy) {
   constexpr int smem = tcm::Smem<N>::kBytes;
   // the sliding-window instance only for plans with a window
   auto kernel = p.window > 0 ? decode_tcm_kernel<N, true> : decode_tcm_kernel<N, false>;
@@ -1690,14 +1690,15 @@ cudaError_t launch_tcm(const DecodeParams& p, const CUtensorMap& tk, const CUten
     e = launch_pdl(tcm_share_prepass, dim3(static_cast<unsigned>(windows)), dim3(256), 0, stream, p);
     if (e != cudaSuccess) return e;
   }
-  e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv);
+  e = launch_pdl(kernel, dim3(p.num_ctas), dim3(tcm::kThreads), smem, stream, p, tk, tv, tq);
   if (e != cudaSuccess) return e;
   return launch_pdl(tcm_merge_kernel<N>, dim3(p.num_ctas), dim3(tcm::kMergeThreads), 0, stream, p);
 }
 
 template <int D>
 cudaError_t dispatch(int path, int schedule, int rows_per_cta, int kv_dtype, const DecodeParams& p,
-                     const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream, int* occ) {
+                     const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
+                     int* occ) {
   if (kv_dtype == kKvE4M3) {  // E4M3 pools: the tensor-core tiles widen the codes to f16
     if (path != kPathTile) return cudaErrorInvalidValue;
     switch (rows_per_cta) {
@@ -1714,8 +1715,8 @@ cudaError_t dispatch(int path, int schedule, int rows_per_cta, int kv_dtype, con
       return cudaErrorInvalidValue;
     } else {
       if (schedule != kSchedulePersistent) return cudaErrorInvalidValue;
-      if (rows_per_cta == 16) return launch_tcm<16>(p, tk, tv, stream, occ);
-      if (rows_per_cta == 32) return launch_tcm<32>(p, tk, tv, stream, occ);
+      if (rows_per_cta == 16) return launch_tcm<16>(p, tk, tv, tq, stream, occ);
+      if (rows_per_cta == 32) return launch_tcm<32>(p, tk, tv, tq, stream, occ);
       return cudaErrorInvalidValue;
     }
   }
@@ -1750,9 +1751,10 @@ cudaError_t launch_prefill(const PrefillParams& p, int max_tiles, const CUtensor
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int head_dim, int kv_dtype,
-                          const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream) {
-  return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, stream, nullptr)
-                         : dispatch<64>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, stream, nullptr);
+                          const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                          cudaStream_t stream) {
+  return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, tq, stream, nullptr)
+                         : dispatch<64>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, tq, stream, nullptr);
 }
 
 int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, int kv_dtype) {
@@ -1776,8 +1778,8 @@ int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, i
   CUtensorMap tm = {};
   int occ = 0;
   cudaError_t e =
-      head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, nullptr, &occ)
-                      : dispatch<64>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, nullptr, &occ);
+      head_dim == 128 ? dispatch<128>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, tm, nullptr, &occ)
+                      : dispatch<64>(path, schedule, rows_per_cta, kv_dtype, dummy, tm, tm, tm, nullptr, &occ);
   const int result = e == cudaSuccess && occ > 0 ? occ : 1;
   if (e == cudaSuccess && occ > 0 && dev >= 0) {
     std::lock_guard<std::mutex> lock(mu);

@@ -237,7 +237,7 @@ __device__ __forceinline__ float column_reduce(float (&v)[V], int lane) {
 template <int N, bool kWin>
 __global__ void __launch_bounds__(tcm::kThreads, 1)
 decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v) {
+                  const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_q) {
   using L = tcm::Smem<N>;
   using tcm::kKStages;
   using tcm::kVStages;
@@ -269,6 +269,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
+    if (p.q_box > 0) tma_prefetch_desc(&tmap_q);
   }
   grid_dependency_wait();
 
@@ -345,6 +346,14 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  // Q rows past a box (a shared-prefix window of fewer than N rows) stay zero: no box
+  // writes them, and the async proxy (the MMA) reads them
+  if (p.q_box > 0 && p.q_box * p.group < N) {
+    for (int i = threadIdx.x; i < 2 * L::kQ / 16; i += tcm::kThreads)
+      reinterpret_cast<uint4*>(smem + L::offQ)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    __syncthreads();
+  }
   const uint32_t tmem = tmem_base_s;
   const uint32_t sm = smem_u32(smem);
 
@@ -377,6 +386,17 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         const int kvh = unit_kvh(w.k);
         const int rc = unit_rc(w.k);
         uint8_t* qb = smem + L::offQ + (j & 1) * L::kQ;
+        if (p.q_box > 0) {
+          // the unit's rows as two boxes (the halves of D), in flight with its first K tile:
+          // tokens of row chunk rc (rc = 0 for a shared-prefix window), heads of kv head kvh
+          if (lane == 0) {
+            const int tok0 = w.b0 * p.q_per_seq + rc * p.q_box;
+            mbar_arrive_expect_tx(&bars.q_full[j & 1], 2 * p.q_box * p.group * 128);
+            tma_load_3d(qb, &tmap_q, &bars.q_full[j & 1], 0, kvh * p.group, tok0);
+            tma_load_3d(qb + N * 128, &tmap_q, &bars.q_full[j & 1], 64, kvh * p.group, tok0);
+          }
+          __syncwarp();
+        } else {
         if (lane < N) {
           const int r = lane;
           const int cg = rc * N + r;  // row of the window: member cg / rpm, row cg % rpm of it
@@ -397,6 +417,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.q_full[j & 1]);
+        }
       }
       const int stages = is_k ? kKStages : kVStages;
       const int s = g % stages;
@@ -781,17 +802,18 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
         float* rl = red + 2 * 4 * NC;
         if (lane < NC) rl[(warp & 3) * NC + lane] = wl;
         tcm::named_sync_softmax(wg);
-        pend.on = true;
-        pend.g = g;
-        pend.obuf = j & 1;
-        pend.b0 = w.b0;
-        pend.kvh = kvh;
-        pend.rc = rc;
-        pend.nrows = nrows;
-        pend.complete = first_x == 0 && w.x == w.tiles - 1;
-        pend.slot = j == 0 ? 2 * c : 2 * c + 1;
-        pend.L_c = (rl[jc] + rl[NC + jc]) + (rl[2 * NC + jc] + rl[3 * NC + jc]);
-        pend.m_c = mref_c;
+        Pending& pe = pend;
+        pe.on = true;
+        pe.g = g;
+        pe.obuf = j & 1;
+        pe.b0 = w.b0;
+        pe.kvh = kvh;
+        pe.rc = rc;
+        pe.nrows = nrows;
+        pe.complete = first_x == 0 && w.x == w.tiles - 1;
+        pe.slot = j == 0 ? 2 * c : 2 * c + 1;
+        pe.L_c = (rl[jc] + rl[NC + jc]) + (rl[2 * NC + jc] + rl[3 * NC + jc]);
+        pe.m_c = mref_c;
         if (g == n - 1 && wg == 0 && t == 0) {
           // the merge descriptor: this CTA's last unit continues in the next CTAs and
           // started here, so this CTA holds its first piece

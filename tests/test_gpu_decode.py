@@ -34,6 +34,13 @@ CASES = [
     ("shared_spec2", [64, 70, 81, 66], 2, 4, 2, 128, None, [(0, 4, 64)]),
     ("shared_short", [20, 16, 300, 310], 1, 4, 1, 64, None, [(0, 2, 16), (2, 2, 288)]),
     ("many_seqs", [1 + (37 * k) % 40 for k in range(1500)], 1, 4, 2, 64, None, []),
+    # more sequences than the tcgen05 kernel stages in shared memory for its scan (2048 at N = 16)
+    ("many_seqs_d128", [1 + (53 * k) % 47 for k in range(2100)], 1, 8, 2, 128, None, []),
+    # GQA groups that do not divide the tcgen05 MMA's N (16 / 32): Q rows by plain loads
+    ("g3", [40, 97, 300, 17], 1, 24, 8, 128, None, []),
+    ("g6_spec3", [30, 200, 77], 3, 12, 2, 128, None, []),
+    # sharing with G = 3: windows of 10 sequences hold 30 of the 32 rows
+    ("shared_g3", [64 + 9 * k for k in range(10)] + [50, 90], 1, 24, 8, 128, None, [(0, 10, 64)]),
 ]
 
 PLANS = [
@@ -135,7 +142,8 @@ def _poison_unwritten(dw, w):
     return len(dead)
 
 
-POISON_CASES = ["ragged", "spec6", "spec6_d64", "rows64", "long_ragged", "shared9", "shared_spec2"]
+POISON_CASES = ["ragged", "spec6", "spec6_d64", "rows64", "long_ragged", "shared9", "shared_spec2", "g6_spec3",
+                "shared_g3"]
 
 
 @pytest.mark.parametrize("plan_spec", PLANS, ids=[p[0] for p in PLANS])
