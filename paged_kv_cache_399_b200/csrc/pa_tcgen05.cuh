@@ -610,6 +610,9 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok) ok = __all_sync(kFull, mbar_wait_bounded(bar, parity));
     };
+    // Complete outputs leave through shared memory and bulk copies at N = 32; at N = 16 (8 rows
+    // a warpgroup) element stores measured faster.
+    constexpr bool kStagedOut = N == 32;
     // A unit piece whose output is written one tile later: by then its last PV is done.
     struct Pending {
       bool on, complete;
@@ -617,6 +620,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       float L_c, m_c;  // l and the reference maximum of column cb + (lane % NC)
     } pend;
     pend.on = false;
+    bool bulk_pending = false;  // this thread has output copies whose shared-memory reads may be running
     auto flush = [&](Pending& e) {
       e.on = false;
       wait(&bars.pv_done[e.g & 1], (e.g >> 1) & 1);
@@ -625,20 +629,64 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       tmem_ld<NC>(tmem + lane_off + 2 * N + e.obuf * N + cb, ov);
       tc_wait_ld();
       tc_fence_before_sync();
+      if (kStagedOut && e.complete) {
+        // The rows leave through shared memory and bulk copies: element stores from these
+        // threads stall for microseconds behind the kernel's own load traffic. Staging area:
+        // this warpgroup's half of the P^T buffer of the piece's last tile (its PV is done;
+        // the next P^T written there follows this warpgroup's next vote barrier, before which
+        // the copies have finished reading), bf16 [NC rows][D].
+        uint16_t* stg =
+            reinterpret_cast<uint16_t*>(smem + L::offP + (e.g & 1) * L::kP + (cb / 8) * tcm::kPGroupBytes);
+        if (ok) {
+          const float inv_c = e.L_c > 0.f ? 1.f / e.L_c : 0.f;  // 1 / l of column cb + (lane % NC)
+#pragma unroll
+          for (int r = 0; r < NC; ++r) {
+            const float inv = __shfl_sync(kFull, inv_c, r);
+            stg[r * D + t] = static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
+          }
+          fence_proxy_async_smem();
+        }
+        tcm::named_sync_softmax(wg);  // every warp passes it, also after a timeout
+        if (ok && (warp & 3) == 0 && lane == 0) {
+          // column cb + r = row cg of the window: member cg / rpm, (i, g) of its row cg % rpm; the
+          // rows of one query token's G heads are contiguous in the output: one copy per run
+          const int cg = e.rc * N + cb;
+          int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
+          int gg = cg - mem * rpm - i * p.group;
+          const int rend = min(NC, e.nrows - cb);
+          for (int r = 0; r < rend;) {
+            const int len = min(rend - r, p.group - gg);
+            bulk_store(p.out + (static_cast<size_t>((e.b0 + mem) * p.q_per_seq + i) * p.num_q_heads +
+                                e.kvh * p.group + gg) * D,
+                       stg + r * D, static_cast<uint32_t>(len * D * 2));
+            r += len;
+            gg += len;
+            if (gg == p.group) {
+              gg = 0;
+              if (++i == p.q_per_seq) {
+                i = 0;
+                ++mem;
+              }
+            }
+          }
+          bulk_commit();
+          bulk_pending = true;
+        }
+        return;
+      }
       if (!ok) return;  // nothing is written after a timeout
       if (e.complete) {
         // column cb + r = row cg of the window: member cg / rpm, (i, g) of its row cg % rpm
         int cg = e.rc * N + cb;
         int mem = cg / rpm, i = (cg - mem * rpm) / p.group;
         int gg = cg - mem * rpm - i * p.group;
+        const float inv_c = e.L_c > 0.f ? 1.f / e.L_c : 0.f;  // 1 / l of column cb + (lane % NC)
 #pragma unroll
         for (int r = 0; r < NC; ++r) {
-          const float lr = __shfl_sync(kFull, e.L_c, r);
-          if (cb + r < e.nrows) {
-            const float inv = lr > 0.f ? 1.f / lr : 0.f;
+          const float inv = __shfl_sync(kFull, inv_c, r);
+          if (cb + r < e.nrows)
             p.out[(static_cast<size_t>((e.b0 + mem) * p.q_per_seq + i) * p.num_q_heads + e.kvh * p.group + gg) * D +
                   t] = static_cast<uint16_t>(pack_bf16x2(__uint_as_float(ov[r]) * inv, 0.f) & 0xFFFFu);
-          }
           if (++gg == p.group) {
             gg = 0;
             if (++i == p.q_per_seq) {
@@ -734,6 +782,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       const int* vb = votes + (g & 1) * 4;
       const bool wover = __any_sync(kFull, over);
       if (lane == 0) votes[(g & 1) * 4 + (warp & 3)] = wover ? 1 : 0;
+      if (bulk_pending) {  // a staged output is read out before its buffer takes a P^T again
+        bulk_wait_read();
+        bulk_pending = false;
+      }
       tcm::named_sync_softmax(wg);
       const int jc = lane % NC;
       if ((vb[0] | vb[1] | vb[2] | vb[3]) != 0) {
@@ -828,6 +880,7 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
       w.next(p, upb, nwin);
     }
     if (pend.on) flush(pend);
+    if (bulk_pending) bulk_wait_all();  // the last output copies complete before the CTA exits
     if (!ok) {
       if (lane == 0) record_error(kErrTimeoutDecode);
       if (wg == 0 && t == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
