@@ -277,13 +277,16 @@ pa_status_t make_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, 
     // possible context into pieces so that about four waves of CTAs exist (contexts of
     // different lengths leave many splits empty). With a sliding window every sequence
     // reads about the same span, so about 1.5 waves of longer splits suffice (measured
-    // on B200: fewer, longer splits beat the four-wave rule there). Splits are made
-    // equal, so that no short last split is left over.
+    // on B200: fewer, longer splits beat the four-wave rule there). Over E4M3 pools the
+    // tile core is bound by its per-block instructions, not by the loads, and three waves
+    // measured faster than four. Splits are made equal, so that no short last split is
+    // left over.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * row_chunks;
     if (units >= 2 * static_cast<int64_t>(slots) || units == 0) {
       split_blocks = span;
     } else {
-      const int64_t target = h.sliding_window > 0 ? 3 * static_cast<int64_t>(slots) / 2 : 4 * static_cast<int64_t>(slots);
+      const int64_t target = h.sliding_window > 0 ? 3 * static_cast<int64_t>(slots) / 2
+                             : (e4m3 ? 3 : 4) * static_cast<int64_t>(slots);
       const int64_t splits = ceil_div(target, units);
       const int64_t floor_sb = (h.sliding_window > 0 ? 4 : 8) * pa::kWarpsPerCta;
       int64_t sb = ceil_div(span, splits);
