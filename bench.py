@@ -215,7 +215,7 @@ class ClockSampler:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.15)
+        time.sleep(0.3)  # nvidia-smi's start-up and first sample, before the work it watches
         return self
 
     def __exit__(self, *exc):
@@ -581,13 +581,14 @@ def run_gpu(args):
     step_bytes = decode_bytes(w) + cache_write_bytes(w)
     dec_bytes = decode_bytes(w)
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
-    assert pa.pa_get_device_error(reset=True, stream=stream) == 0
-
     sampler = ClockSampler(local_rank)
     with sampler:
+        # warm-up once the clock sampler runs, right before the timed region: the GPU enters it
+        # from work at its clocks, not from the sampler's start-up idle
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        assert pa.pa_get_device_error(reset=True, stream=stream) == 0
         # (1) headline: K whole steps, events only around the region
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
