@@ -332,21 +332,24 @@ def _ncu_traffic(name):
 
 def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
     """Mean CUDA-event time of `calls` pa_decode calls (each after the step's cache write,
-    events on the launching stream around the decode only), in ms; and the same calls
-    without host overhead: one CUDA graph of 20 back-to-back calls, replayed (µs per call,
-    None when capture is unavailable)."""
+    events on the launching stream around the decode only), in ms; the same calls without
+    host overhead: one CUDA graph of 20 back-to-back calls, replayed (µs per call, None when
+    capture is unavailable); and the mean event time of the step's cache writes (ms), timed
+    apart from the decode."""
     import torch
     write, decode = _hot_path(pa, w, v, plan, ws, stream)
     barrier()
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(calls)]
-    for a, b in pairs:
+    quads = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(calls)]
+    for c, d, a, b in quads:
+        c.record(stream)
         write()
+        d.record(stream)
         a.record(stream)
         decode()
         b.record(stream)
     barrier()
-    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+    decode_ms = statistics.mean(a.elapsed_time(b) for _, _, a, b in quads)
+    write_ms = statistics.mean(c.elapsed_time(d) for c, d, _, _ in quads)
     graph_us = None
     try:
         per_graph, reps = 20, max(1, calls // 20)
@@ -367,7 +370,7 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
         del graph
     except Exception as exc:  # capture is a measurement aid: report why it is missing
         print(f"graph timing unavailable: {exc}", file=sys.stderr)
-    return decode_ms, graph_us
+    return decode_ms, graph_us, write_ms
 
 
 def measure_config(name, args, dev, stream, peaks):
@@ -394,7 +397,7 @@ def measure_config(name, args, dev, stream, peaks):
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
     sampler = ClockSampler(dev.index)
     with sampler:
-        decode_ms, graph_us = _time_calls(pa, w, v, plan, ws, stream, args.config_calls, barrier)
+        decode_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.config_calls, barrier)
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
     dec_bytes = decode_bytes(w)
     gbs = dec_bytes / (decode_ms * 1e-3) / 1e9
@@ -410,6 +413,8 @@ def measure_config(name, args, dev, stream, peaks):
         "frac_graph": None if graph_us is None else round(dec_bytes / (graph_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
         "plan": plan.as_dict(),
         "ncu_traffic": _ncu_traffic(name),
+        "cache_write_us_per_call": round(write_ms * 1e3, 3),
+        "cache_write_bytes": cache_write_bytes(w),
         "clocks": sampler.summary(),
     }
     if name in BAR_CONFIGS:
@@ -537,6 +542,119 @@ def run_prefill_gpu(args):
         }), flush=True)
 
 
+def run_context_parallel_gpu(args):
+    """--context-parallel: one decode of the workload split over the job's GPUs (strong scaling).
+    Rank r reads table entries rank_block_range(max_blocks, r, N) of every sequence
+    (pa_decode_partial), the pieces are all-gathered (NCCL) and every rank merges them
+    (pa_merge_partials). The whole decode's algorithmic bytes over the slowest rank's event
+    time per call; rank 0 also times pa_decode alone and checks the merged output against it."""
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from paged_kv_cache_399_b200 import build as pa_build
+    pa_build.build()
+    from paged_kv_cache_399_b200 import pa, workloads
+    from paged_kv_cache_399_b200.context_parallel import gather_partials, partial_pieces, rank_block_range
+
+    w = workloads.make(args.workload, seed=rank_seed(args.workload, 0))  # the same decode on every rank
+    if w.kv_dtype != "bf16" or w.shared_groups or w.window:
+        raise SystemExit("--context-parallel takes a bf16 workload without sharing or window")
+    dev = torch.device("cuda", local_rank)
+    v = _device_inputs(w, dev)
+    pa.pa_reshape_and_cache(v["key"], v["value"], v["key_cache"], v["value_cache"], v["slots"])
+    B, QS, HQ, D = w.query.shape
+    lo, hi = rank_block_range(w.max_blocks_per_seq, rank, world)
+    S = partial_pieces(v["query"], v["key_cache"], w.max_blocks_per_seq, world)
+    part_o = torch.empty((S, B, QS, HQ, D), dtype=torch.float32, device=dev)
+    part_ml = torch.empty((S, B, QS, HQ, 2), dtype=torch.float32, device=dev)
+    out = torch.empty_like(v["query"])
+
+    def call():
+        pa.pa_decode_partial(part_o, part_ml, v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
+                             w.q_per_seq, w.scale, lo, hi)
+        if world > 1:
+            all_o, all_ml = gather_partials(part_o, part_ml)
+            all_o, all_ml = all_o.flatten(0, 1), all_ml.flatten(0, 1)
+        else:
+            all_o, all_ml = part_o, part_ml
+        pa.pa_merge_partials(out, all_o, all_ml)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        for _ in range(args.warmup):
+            call()
+        barrier()
+        assert pa.pa_get_device_error(reset=True) == 0
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            call()
+        e1.record()
+        barrier()
+        ms = reduce_over_ranks(e0.elapsed_time(e1), "max", dist if world > 1 else None, dev) / args.steps
+    assert pa.pa_get_device_error(reset=True) == 0
+    ref = torch.empty_like(out)
+    plan = _plan_for(pa, w, args)
+    ws_bytes = pa.pa_decode_workspace_size(plan, w.num_seqs, w.q_per_seq, w.num_q_heads, w.num_kv_heads,
+                                           w.head_dim, w.max_blocks_per_seq)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
+    pa.pa_decode(ref, v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"], w.q_per_seq, w.scale,
+                 plan=plan, workspace=ws)
+    torch.cuda.synchronize(dev)
+    diff = float((ref.float() - out.float()).abs().max())
+    single_us = None
+    if rank == 0:
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(args.steps):
+            pa.pa_decode(ref, v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"], w.q_per_seq,
+                         w.scale, plan=plan, workspace=ws)
+        f1.record()
+        torch.cuda.synchronize(dev)
+        single_us = f0.elapsed_time(f1) * 1e3 / args.steps
+    dec_bytes = decode_bytes(w)
+    gbs = dec_bytes / (ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "pa_decode of one batch split over the job's GPUs by table ranges (context parallelism): "
+                      "achieved HBM GB/s of the whole decode",
+            "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 6), "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": w.describe(),
+                "step": "pa_decode_partial over this rank's table range + all-gather (NCCL) + pa_merge_partials",
+                "ranges": [rank_block_range(w.max_blocks_per_seq, r, world) for r in range(world)],
+                "pieces_per_rank": S,
+                "gather_bytes_per_rank": (part_o.numel() + part_ml.numel()) * 4,
+                "decode_alg_bytes": dec_bytes,
+                "frac_of_measured_hbm_per_gpu": round(gbs / world / peaks["hbm_gbs"], 4),
+                "single_gpu_pa_decode_us": None if single_us is None else round(single_us, 3),
+                "max_abs_diff_vs_pa_decode": diff,
+                "parallelism": f"context parallel x{world} (one decode's blocks split across GPUs)",
+            },
+            "gpu_launches": 2 * args.steps,
+            "clocks": sampler.summary(),
+        }), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -608,7 +726,7 @@ def run_gpu(args):
         # (2) per-kernel: events around each pa_decode launch of another K steps, and the
         # same calls graph-replayed (for the small configs the events mostly time the
         # Python call)
-        decode_ms, graph_us = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
+        decode_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
         decode_ms = max_over_ranks(decode_ms)
         if graph_us is not None:
             graph_us = max_over_ranks(graph_us)
@@ -673,6 +791,7 @@ def run_gpu(args):
                 "decode_logical_bytes": decode_bytes(w, unique=False),
                 "decode_us_per_call": round(decode_ms * 1e3, 3),
                 "decode_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
+                "cache_write_us_per_call": round(write_ms * 1e3, 3),
                 "decode_gbs": round(achieved, 2),
                 "decode_frac_of_measured_hbm": round(achieved / peaks["hbm_gbs"], 4),
                 "decode_frac_of_spec_8tbs": round(achieved / 8000.0, 4),
@@ -1095,12 +1214,17 @@ def main(argv=None):
                     help="pa_decode calls timed per config in config.per_config")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="split one decode of the workload over the job's GPUs by table ranges "
+                         "(pa_decode_partial + all-gather + pa_merge_partials; strong scaling)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     copy = args.workload in ("cow_fork", "cow_bulk")
     prefill = args.workload in PREFILL_CONFIG
     if args.impl == "reference":
         (run_copy_reference if copy else run_prefill_reference if prefill else run_reference)(args)
+    elif args.context_parallel:
+        run_context_parallel_gpu(args)
     else:
         (run_copy_gpu if copy else run_prefill_gpu if prefill else run_gpu)(args)
     return 0

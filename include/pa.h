@@ -19,7 +19,11 @@
  *   pa_decode_fp8         pa_decode over such FP8 pools (same notes §4.2: an FP8 KV cache
  *                         halves attention's memory traffic);
  *   pa_prefill            chunked-prefill attention: many query tokens per sequence over
- *                         the paged pool, causal within the chunk (same notes §3.5).
+ *                         the paged pool, causal within the chunk (same notes §3.5);
+ *   pa_decode_partial,    one sequence's blocks split over several GPUs: each computes the
+ *   pa_merge_partials     attention over its range of table entries as unnormalised pieces,
+ *                         and the pieces gathered from all of them merge by the log-sum-exp
+ *                         rule of split softmax (same notes §4.3.1).
  *
  * Conventions shared by every call
  *   - All data pointers are DEVICE pointers on the current CUDA device (the one
@@ -368,11 +372,54 @@ PA_API pa_status_t pa_copy_blocks(void* key_cache, void* value_cache, int64_t nu
                                   const int64_t* block_mapping, int64_t num_pairs,
                                   pa_stream_t stream);
 
+/* Context parallelism, step 1 (vLLM study notes §4.3.1: the softmax of a split context is
+ * recovered from per-split maxima and sums). The table entries block_begin <= j < block_end
+ * (positions 16j .. 16j+15) of every sequence are cut into num_pieces equal pieces
+ * (ceil((block_end - block_begin) / num_pieces) entries each, the last ones shorter or empty);
+ * for piece k, sequence b and query row (i, h), the attention of pa_decode restricted to the
+ * visible keys of the piece, written unnormalised and part-major:
+ *   part_o [num_pieces][num_seqs][q_per_seq][num_q_heads][head_dim] fp32: sum_t 2^(s_t - m) v_t
+ *   part_ml [num_pieces][num_seqs][q_per_seq][num_q_heads][2] fp32: {m, l = sum_t 2^(s_t - m)}
+ * with s_t the score in log2 units (q.k * scale * log2 e) and m the largest s_t of the piece
+ * (o / l and m + log2 l are what a merge needs); m = -inf, l = 0 and o = 0 when no key of the
+ * piece is visible. Positions are the sequence's own (key 16j + r, query row i at
+ * context_len - q_per_seq + i), so every GPU of a split passes the full context_lens and a block
+ * table whose entries [block_begin, block_end) name blocks of its own pool (the other entries
+ * are not read). bf16 pools only; same checks and preconditions as pa_decode, plus 0 <=
+ * block_begin <= block_end <= max_blocks_per_seq and 1 <= num_pieces <= 65535 (else
+ * PA_ERR_INVALID_ARG) and 16-byte aligned part_o / part_ml. Grid schedule, one CTA per (kv
+ * head, sequence, piece); no workspace. */
+PA_API pa_status_t pa_decode_partial(float* part_o, float* part_ml, const void* query, const void* key_cache,
+                                     const void* value_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, int32_t num_seqs, int32_t q_per_seq,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                                     float scale, int32_t block_begin, int32_t block_end, int32_t num_pieces,
+                                     pa_stream_t stream);
+
+/* Pieces for pa_decode_partial over ranges of range_blocks table entries: the split count the
+ * decode heuristic takes for tables of that length on this device (host-known values only; the
+ * same on every GPU of a group, so the gathered pieces have one shape); 0 for bad shapes. */
+PA_API int32_t pa_decode_partial_pieces(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim, int32_t range_blocks);
+
+/* Context parallelism, step 2: out[b][i][h] = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k over
+ * num_parts pieces laid out part-major (part_o [num_parts][num_seqs][q][H_q][D], part_ml
+ * [num_parts][num_seqs][q][H_q][2], as an all-gather of every GPU's pa_decode_partial pieces
+ * leaves them: num_parts = GPUs x num_pieces),
+ * M the largest m_k; a row whose pieces are all empty gets zeros. Pieces over disjoint ranges that
+ * together cover every context give pa_decode's result. bf16 out [num_seqs][q][H_q][D]; head_dim
+ * 64 or 128; 16-byte aligned buffers (else PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED). */
+PA_API pa_status_t pa_merge_partials(void* out, const float* part_o, const float* part_ml, int32_t num_parts,
+                                     int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                                     int32_t head_dim, pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char* pa_status_string(pa_status_t status);
 
 /* ABI version (major * 10000 + minor * 100 + patch). 1.1 added pa_decode_fp8, pa_prefill
- * and the kv_cache_dtype fields at the end of pa_plan_hints_t and pa_plan_t. */
+ * and the kv_cache_dtype fields at the end of pa_plan_hints_t and pa_plan_t; 1.2 added
+ * pa_decode_partial, pa_decode_partial_pieces and pa_merge_partials. */
 PA_API int32_t pa_version(void);
 
 #ifdef __cplusplus

@@ -18,7 +18,7 @@ namespace {
 
 using pa::DecodeParams;
 
-constexpr int32_t kVersion = 10100;  // 1.1.0
+constexpr int32_t kVersion = 10200;  // 1.2.0
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -440,12 +440,35 @@ pa_status_t check_plan(const pa_plan_t& plan, int32_t q_per_seq, int32_t num_q_h
 
 // pa_decode and pa_decode_fp8: the pools hold bf16 values, or E4M3 codes with one scale
 // per pool (k_scale, v_scale; 1 for bf16 pools).
+// A partial decode (context parallelism): table entries [lo, hi) of every sequence only, its
+// records written to part_o / part_ml.
+struct PartialArgs {
+  int32_t lo, hi, pieces;
+  float* part_o;
+  float* part_ml;
+};
+
+// Grid plan of a partial decode: the mma.sync tiles, or the CUDA-core kernel for up to 2 rows;
+// `pieces` splits of the range (0: as many as the split heuristic takes for a table of the
+// range's length). Returns the plan's status.
+pa_status_t partial_plan(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t lo, int32_t hi, int32_t pieces, pa_plan_t* plan) {
+  const int32_t span = hi > lo ? hi - lo : 1;
+  pa_plan_hints_t h = {};
+  h.schedule = PA_SCHEDULE_GRID;
+  h.path = q_per_seq * (num_q_heads / num_kv_heads) <= 2 ? PA_PATH_SINGLE : PA_PATH_TILE;
+  if (pieces > 0) h.split_blocks = static_cast<int32_t>(ceil_div(span, pieces));
+  const pa_status_t st = make_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, span, &h, plan);
+  if (st == PA_OK && pieces > 0) plan->num_splits = pieces;
+  return st;
+}
+
 pa_status_t decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
                         const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
                         int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                         int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, float scale,
                         int kv_dtype, float k_scale, float v_scale, const pa_plan_t* plan, void* workspace,
-                        size_t workspace_bytes, pa_stream_t stream) {
+                        size_t workspace_bytes, pa_stream_t stream, const PartialArgs* part = nullptr) {
   pa_status_t st = check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
                                 max_blocks_per_seq);
   if (st != PA_OK) return st;
@@ -455,13 +478,20 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     return PA_ERR_INVALID_ARG;
   if (num_blocks * pa::kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;  // TMA coordinate range
   if (num_seqs == 0) return PA_OK;
-  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+  if ((!out && !part) || !query || !key_cache || !value_cache || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
+  if ((out && !aligned16(out)) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
     return PA_ERR_INVALID_ARG;
   pa_plan_t local;
-  if (plan) {
+  if (part) {
+    // the range's pieces on the grid schedule; no workspace (the records go to the caller's
+    // buffers)
+    st = partial_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, part->lo, part->hi, part->pieces,
+                      &local);
+    if (st != PA_OK) return st;
+    plan = &local;
+  } else if (plan) {
     st = check_plan(*plan, q_per_seq, num_q_heads, num_kv_heads, max_blocks_per_seq);
     if (st == PA_OK && plan->kv_cache_dtype != kv_dtype) st = PA_ERR_INVALID_ARG;  // a plan for other pools
   } else {
@@ -471,7 +501,8 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     plan = &local;
   }
   if (st != PA_OK) return st;
-  const size_t need = workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
+  const size_t need =
+      part ? 0 : workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
 
   CUtensorMap tk, tv, tq = {};
@@ -542,6 +573,12 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     p.list_len = reinterpret_cast<int32_t*>(ws + L.list_len);
     p.list = reinterpret_cast<int2*>(ws + L.list);
     p.records = reinterpret_cast<float*>(ws + L.records);
+  } else if (part) {
+    p.partial_only = 1;
+    p.range_lo = part->lo;
+    p.range_hi = part->hi;
+    p.ws_o = part->part_o;
+    p.ws_ml = reinterpret_cast<float2*>(part->part_ml);
   } else if (need > 0) {
     const size_t recs = plan->share_cap ? share_records(*plan, num_seqs, q_per_seq, num_q_heads)
                                         : static_cast<size_t>(num_seqs) * plan->num_splits * rq;
@@ -671,6 +708,57 @@ pa_status_t pa_decode_fp8(void* out, const void* query, const void* key_cache, c
   return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, num_seqs, q_per_seq,
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
                      PA_KV_FP8_E4M3, k_scale, v_scale, plan, workspace, workspace_bytes, stream);
+}
+
+pa_status_t pa_decode_partial(float* part_o, float* part_ml, const void* query, const void* key_cache,
+                              const void* value_cache, const int32_t* block_tables, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                              int64_t num_blocks, float scale, int32_t block_begin, int32_t block_end,
+                              int32_t num_pieces, pa_stream_t stream) {
+  if (block_begin < 0 || block_end < block_begin || block_end > max_blocks_per_seq || num_pieces <= 0 ||
+      num_pieces > 65535)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (!part_o || !part_ml || !aligned16(part_o) || !aligned16(part_ml))) return PA_ERR_INVALID_ARG;
+  const PartialArgs part{block_begin, block_end, num_pieces, part_o, part_ml};
+  return decode_impl(nullptr, query, key_cache, value_cache, block_tables, context_lens, num_seqs, q_per_seq,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                     PA_KV_BF16, 1.f, 1.f, nullptr, nullptr, 0, stream, &part);
+}
+
+int32_t pa_decode_partial_pieces(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t range_blocks) {
+  if (range_blocks < 0 ||
+      check_shapes(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, range_blocks > 0 ? range_blocks : 1) !=
+          PA_OK)
+    return 0;
+  pa_plan_t plan;
+  if (partial_plan(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim, 0, range_blocks, 0, &plan) != PA_OK)
+    return 0;
+  return plan.num_splits;
+}
+
+pa_status_t pa_merge_partials(void* out, const float* part_o, const float* part_ml, int32_t num_parts,
+                              int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t head_dim,
+                              pa_stream_t stream) {
+  if (num_parts <= 0 || num_seqs < 0 || q_per_seq <= 0 || num_q_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  const int64_t rows = static_cast<int64_t>(num_seqs) * q_per_seq * num_q_heads;
+  if (rows > INT32_MAX || static_cast<int64_t>(num_parts) * rows > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !part_o || !part_ml || !aligned16(out) || !aligned16(part_o) || !aligned16(part_ml))
+    return PA_ERR_INVALID_ARG;
+  DecodeParams p = {};
+  p.out = static_cast<uint16_t*>(out);
+  p.num_seqs = num_seqs;
+  p.q_per_seq = q_per_seq;
+  p.num_q_heads = num_q_heads;
+  p.num_parts = num_parts;
+  p.ws_o = const_cast<float*>(part_o);
+  p.ws_ml = reinterpret_cast<float2*>(const_cast<float*>(part_ml));
+  return pa::launch_merge_partials(p, head_dim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
 }
 
 pa_status_t pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,

@@ -79,6 +79,11 @@ struct DecodeParams {
   // tokens}: the rows of one row chunk, or of a shared-prefix window); 0 = Q rows are
   // loaded with plain loads (a group that does not divide the MMA's N)
   int32_t q_box;
+  // context parallelism (grid schedule): only table entries [range_lo, range_hi) of every
+  // sequence are read, cut into num_splits pieces, and every CTA writes its (o, m, l) record
+  // part-major ([piece][sequence][row]), never the output; num_parts > 0: the merge combines
+  // num_parts such records per row, laid out [part][sequence][row] (gathered pieces)
+  int32_t range_lo, range_hi, partial_only, num_parts;
 };
 
 // Host-side checks of a decode call's shapes and (when non-null) its plan, the ones
@@ -114,6 +119,10 @@ struct PrefillParams {
 };
 cudaError_t launch_prefill(const PrefillParams& p, int max_tiles, const CUtensorMap& tmap_k,
                            const CUtensorMap& tmap_v, cudaStream_t stream);
+
+// The merge of a gathered set of p.num_parts partial decodes (p.ws_o, p.ws_ml laid out
+// [part][sequence][row]) into p.out.
+cudaError_t launch_merge_partials(const DecodeParams& p, int head_dim, cudaStream_t stream);
 
 // Resident CTAs per SM of the decode kernel launch_decode would use.
 int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, int kv_dtype);

@@ -1341,12 +1341,25 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
   const int nblk = num_blocks_of(p, ctx);
   const int S = p.num_splits;
   const int sb = p.split_blocks;
-  // own blocks start after the shared prefix, or at the first block of the window
+  // own blocks start after the shared prefix, or at the first block of the window; a partial
+  // decode (context parallelism) reads table entries [range_lo, range_hi) only
   const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
+  const int lo_b = p.partial_only ? max(P_b, p.range_lo) : P_b;
+  const int hi_b = p.partial_only ? min(nblk, p.range_hi) : nblk;
   Seg sg{b, 1, kvh, rc * ROWS, min(ROWS, p.rows - rc * ROWS), 0, 0, false};
-  const int blk0 = P_b + z * sb;
-  if (blk0 >= nblk) {
-    if (z == 0 && nblk == 0) {  // no block at all: zero output
+  const int blk0 = lo_b + z * sb;
+  if (blk0 >= hi_b) {
+    if (p.partial_only) {  // no key of this piece: an empty record (weight 0 in the merge)
+      for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
+        int bb, i, h;
+        seg_row(p, sg, task / DC, bb, i, h);
+        const size_t rec = (static_cast<size_t>(z) * p.num_seqs + b) * RQ + i * p.num_q_heads + h;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + (task % DC) * 8);
+        dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (task % DC == 0) p.ws_ml[rec] = make_float2(-INFINITY, 0.f);
+      }
+    } else if (z == 0 && nblk == 0) {  // no block at all: zero output
       for (int task = threadIdx.x; task < sg.nrows * DC; task += NW * 32) {
         int bb, i, h;
         seg_row(p, sg, task / DC, bb, i, h);
@@ -1357,9 +1370,9 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
     return;
   }
   sg.blk0 = blk0;
-  sg.blk1 = min(nblk, blk0 + sb);
-  // the only piece of its outputs: write bf16 directly
-  const bool direct = (p.share_cap == 0 || P_b == 0) && nblk - P_b <= sb;
+  sg.blk1 = min(hi_b, blk0 + sb);
+  // the only piece of its outputs: write bf16 directly (a partial decode always writes records)
+  const bool direct = !p.partial_only && (p.share_cap == 0 || P_b == 0) && nblk - P_b <= sb;
   run_segment<Core, D, NW, STAGES>(p, sg, ctx, pipe, core, st, smem, &tmap_k, &tmap_v, warp, lane);
   grid_launch_dependents();
   // own-block records follow the shared-prefix records when sharing is on
@@ -1373,7 +1386,10 @@ decode_grid_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tma
     if (direct) {
       store_bf16x8(p.out + out_offset(p, bb, i, h, D) + dc * 8, acc, L > 0.f ? 1.f / L : 0.f);
     } else {
-      const size_t rec = (region + static_cast<size_t>(b) * S + z) * RQ + i * p.num_q_heads + h;
+      // a partial decode's pieces are part-major ([piece][sequence][row]), as the merge of
+      // gathered pieces reads them
+      const size_t rec = p.partial_only ? (static_cast<size_t>(z) * p.num_seqs + b) * RQ + i * p.num_q_heads + h
+                                        : (region + static_cast<size_t>(b) * S + z) * RQ + i * p.num_q_heads + h;
       float4* dst = reinterpret_cast<float4*>(p.ws_o + rec * D + dc * 8);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -1475,18 +1491,23 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
   const int MW = blockDim.x >> 5;
   const int b = row / RQ;
   const int rq = row % RQ;
-  const int ctx = __ldg(p.context_lens + b);
-  const int nblk = num_blocks_of(p, ctx);
-  const int sb = p.split_blocks;
-  // records: the shared-prefix splits (region 0, with prefix sharing) then the
-  // sequence's own splits (region 1 with prefix sharing, else region 0); with a sliding
-  // window the own blocks start at the window's first block
-  const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
-  const int nsh = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
-  const int ns = nsh + (nblk - P_b + sb - 1) / sb;
-  if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
+  int nsh = 0, ns = p.num_parts;
+  if (p.num_parts == 0) {
+    const int ctx = __ldg(p.context_lens + b);
+    const int nblk = num_blocks_of(p, ctx);
+    const int sb = p.split_blocks;
+    // records: the shared-prefix splits (region 0, with prefix sharing) then the
+    // sequence's own splits (region 1 with prefix sharing, else region 0); with a sliding
+    // window the own blocks start at the window's first block
+    const int P_b = p.share_cap ? __ldcg(p.seq_info + b).x : window_first_block(p, ctx);
+    nsh = (p.share_cap && P_b > 0) ? (P_b + p.share_split_blocks - 1) / p.share_split_blocks : 0;
+    ns = nsh + (nblk - P_b + sb - 1) / sb;
+    if (nsh == 0 && ns <= 1) return;  // written directly by the decode kernel (uniform per CTA)
+  }
   const size_t own_region = p.share_cap ? static_cast<size_t>(p.num_seqs) * p.share_splits : 0;
   auto rec_of = [&](int k) -> size_t {
+    if (p.num_parts > 0)  // gathered partial decodes: [part][sequence][row]
+      return (static_cast<size_t>(k) * p.num_seqs + b) * RQ + rq;
     return (k < nsh ? static_cast<size_t>(b) * p.share_splits + k
                     : own_region + static_cast<size_t>(b) * p.num_splits + (k - nsh)) * RQ + rq;
   };
@@ -1668,10 +1689,18 @@ cudaError_t launch_core(const DecodeParams& p, int schedule, const CUtensorMap& 
     grid = dim3(static_cast<unsigned>(ctas));
   }
   e = launch_pdl(kernel, grid, block, smem, stream, p, tk, tv);
-  if (e != cudaSuccess || (p.num_splits <= 1 && !p.share_cap)) return e;
+  // a partial decode leaves its pieces to the merge of gathered pieces
+  if (e != cudaSuccess || (p.num_splits <= 1 && !p.share_cap) || p.partial_only) return e;
   const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
   // about four records per warp, at most kMergeMaxWarps warps per row
   const int mw = max(1, min(kMergeMaxWarps, (p.num_splits + p.share_splits + 3) / 4));
+  return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
+}
+
+template <int D>
+cudaError_t launch_merge_parts(const DecodeParams& p, cudaStream_t stream) {
+  const long rows = static_cast<long>(p.num_seqs) * p.q_per_seq * p.num_q_heads;
+  const int mw = max(1, min(kMergeMaxWarps, (p.num_parts + 3) / 4));
   return launch_pdl(merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(32 * mw), 0, stream, p);
 }
 
@@ -1755,6 +1784,10 @@ cudaError_t launch_decode(const DecodeParams& p, int path, int schedule, int hea
                           cudaStream_t stream) {
   return head_dim == 128 ? dispatch<128>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, tq, stream, nullptr)
                          : dispatch<64>(path, schedule, p.rows_per_cta, kv_dtype, p, tk, tv, tq, stream, nullptr);
+}
+
+cudaError_t launch_merge_partials(const DecodeParams& p, int head_dim, cudaStream_t stream) {
+  return head_dim == 128 ? launch_merge_parts<128>(p, stream) : launch_merge_parts<64>(p, stream);
 }
 
 int decode_ctas_per_sm(int path, int schedule, int head_dim, int rows_per_cta, int kv_dtype) {

@@ -34,7 +34,7 @@ PA_PATH_TILE = 2
 PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode", "pa_decode_fp8",
-            "pa_prefill",
+            "pa_prefill", "pa_decode_partial", "pa_decode_partial_pieces", "pa_merge_partials",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
             "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_status_string",
             "pa_version"]
@@ -102,6 +102,13 @@ _lib.pa_decode_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _
 _lib.pa_prefill.restype = _I32
 _lib.pa_prefill.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
                             ctypes.c_float, _P]
+_lib.pa_decode_partial.restype = _I32
+_lib.pa_decode_partial.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I64,
+                                   ctypes.c_float, _I32, _I32, _I32, _P]
+_lib.pa_decode_partial_pieces.restype = _I32
+_lib.pa_decode_partial_pieces.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32]
+_lib.pa_merge_partials.restype = _I32
+_lib.pa_merge_partials.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P]
 _lib.pa_decode_static_scratch.restype = _I32
 _lib.pa_decode_static_scratch.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32,
                                           _I32, _I64, ctypes.c_float, ctypes.POINTER(pa_plan_t), _P]
@@ -297,6 +304,48 @@ def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor, 
                          _ptr(context_lens), _ptr(query_start), B, T, int(max_query_len), HQ, HKV, D, BS,
                          block_tables.shape[1], NB, float(scale), _stream(stream))
     _check(st, "pa_prefill")
+
+
+def pa_decode_partial(part_o: torch.Tensor, part_ml: torch.Tensor, query: torch.Tensor,
+                      key_cache: torch.Tensor, value_cache: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, q_per_seq: int, scale: float, block_begin: int,
+                      block_end: int, stream=None) -> None:
+    """The attention over table entries [block_begin, block_end) of every sequence, cut into
+    part_o.shape[0] pieces, as unnormalised records: part_o [S, B, q, H_q, D] fp32, part_ml
+    [S, B, q, H_q, 2] fp32 {m, l} (m in log2 units). Other arguments as pa_decode."""
+    assert query.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
+    assert part_o.dtype == part_ml.dtype == torch.float32
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    for t in (part_o, part_ml, query, key_cache, value_cache, block_tables, context_lens):
+        assert t.is_contiguous()
+    B, QS, HQ, D = query.shape
+    S = part_o.shape[0]
+    assert QS == q_per_seq and tuple(part_o.shape) == (S, B, QS, HQ, D) and tuple(part_ml.shape) == (S, B, QS, HQ, 2)
+    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    st = _lib.pa_decode_partial(_ptr(part_o), _ptr(part_ml), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
+                                block_tables.shape[1], NB, float(scale), int(block_begin), int(block_end), S,
+                                _stream(stream))
+    _check(st, "pa_decode_partial")
+
+
+def pa_decode_partial_pieces(num_seqs: int, q_per_seq: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                             range_blocks: int) -> int:
+    """Pieces the decode heuristic takes for ranges of range_blocks table entries (0: bad shapes)."""
+    return int(_lib.pa_decode_partial_pieces(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
+                                             range_blocks))
+
+
+def pa_merge_partials(out: torch.Tensor, part_o: torch.Tensor, part_ml: torch.Tensor, stream=None) -> None:
+    """out [B, q, H_q, D] bf16 from the pieces part_o [P, B, q, H_q, D] and part_ml
+    [P, B, q, H_q, 2] fp32 (an all-gather of pa_decode_partial outputs)."""
+    assert out.dtype == torch.bfloat16 and part_o.dtype == part_ml.dtype == torch.float32
+    for t in (out, part_o, part_ml):
+        assert t.is_contiguous()
+    P, B, QS, HQ, D = part_o.shape
+    assert tuple(out.shape) == (B, QS, HQ, D) and tuple(part_ml.shape) == (P, B, QS, HQ, 2)
+    st = _lib.pa_merge_partials(_ptr(out), _ptr(part_o), _ptr(part_ml), P, B, QS, HQ, D, _stream(stream))
+    _check(st, "pa_merge_partials")
 
 
 def pa_decode_static_scratch(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,

@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(pa):
 def test_status_strings_and_version(pa):
     for code in range(7):
         assert pa.pa_status_string(code).startswith("PA_")
-    assert pa.pa_version() == 10100
+    assert pa.pa_version() == 10200
 
 
 def _decode_raw(lib, **kw):
@@ -355,3 +355,42 @@ def test_prefill_rejects_bad_arguments_before_launch(pa):
     assert call(B=-1) == pa.PA_ERR_INVALID_ARG
     assert call(B=0) == pa.PA_OK and call(T=0) == pa.PA_OK and call(mq=0) == pa.PA_OK   # no-ops
     assert call(mq=3_000_000) == pa.PA_ERR_UNSUPPORTED     # more tiles than the grid holds
+
+
+def test_partial_decode_and_merge_reject_bad_arguments_before_launch(pa):
+    """Context parallelism's entry points: host checks that return before any launch (fake
+    device addresses are never dereferenced)."""
+    lib = pa.raw_library()
+
+    def partial(**kw):
+        a = dict(po=8192, pml=16384, q=24576, kc=32768, vc=49152, bt=65536, cl=81920, B=2, qs=1, hq=8, hkv=2,
+                 d=128, bs=16, mb=8, nb=64, scale=0.088, lo=0, hi=8, S=2)
+        a.update(kw)
+        return lib.pa_decode_partial(a["po"], a["pml"], a["q"], a["kc"], a["vc"], a["bt"], a["cl"], a["B"], a["qs"],
+                                     a["hq"], a["hkv"], a["d"], a["bs"], a["mb"], a["nb"], a["scale"], a["lo"],
+                                     a["hi"], a["S"], None)
+    assert partial(lo=-1) == pa.PA_ERR_INVALID_ARG
+    assert partial(S=0) == pa.PA_ERR_INVALID_ARG
+    assert partial(lo=5, hi=4) == pa.PA_ERR_INVALID_ARG      # an inverted range
+    assert partial(hi=9) == pa.PA_ERR_INVALID_ARG            # past the table
+    assert partial(po=None) == pa.PA_ERR_INVALID_ARG
+    assert partial(pml=16384 + 8) == pa.PA_ERR_INVALID_ARG   # misaligned
+    assert partial(hq=7) == pa.PA_ERR_INVALID_ARG            # H_q % H_kv
+    assert partial(d=96) == pa.PA_ERR_UNSUPPORTED
+    assert partial(qs=17) == pa.PA_ERR_UNSUPPORTED
+    assert partial(B=0, po=None, pml=None) == pa.PA_OK       # nothing to do
+
+    def merge(**kw):
+        a = dict(out=8192, po=16384, pml=32768, P=3, B=2, qs=1, hq=8, d=128)
+        a.update(kw)
+        return lib.pa_merge_partials(a["out"], a["po"], a["pml"], a["P"], a["B"], a["qs"], a["hq"], a["d"], None)
+    assert merge(P=0) == pa.PA_ERR_INVALID_ARG
+    assert merge(B=-1) == pa.PA_ERR_INVALID_ARG
+    assert merge(out=None) == pa.PA_ERR_INVALID_ARG
+    assert merge(po=16384 + 4) == pa.PA_ERR_INVALID_ARG
+    assert merge(d=96) == pa.PA_ERR_UNSUPPORTED
+    assert merge(B=0, out=None) == pa.PA_OK
+    # pieces of a range: at least one for good shapes, 0 for bad ones
+    assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 128, 1024) >= 1
+    assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 96, 1024) == 0
+    assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 128, -1) == 0
