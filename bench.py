@@ -575,16 +575,18 @@ def run_context_parallel_gpu(args):
     S = partial_pieces(v["query"], v["key_cache"], w.max_blocks_per_seq, world)
     part_o = torch.empty((S, B, QS, HQ, D), dtype=torch.float32, device=dev)
     part_ml = torch.empty((S, B, QS, HQ, 2), dtype=torch.float32, device=dev)
+    rec_o = torch.empty((B, QS, HQ, D), dtype=torch.float32, device=dev)
+    rec_ml = torch.empty((B, QS, HQ, 2), dtype=torch.float32, device=dev)
     out = torch.empty_like(v["query"])
 
     def call():
         pa.pa_decode_partial(part_o, part_ml, v["query"], v["key_cache"], v["value_cache"], v["tables"], v["ctx"],
                              w.q_per_seq, w.scale, lo, hi)
+        pa.pa_combine_partials(rec_o, rec_ml, part_o, part_ml)
         if world > 1:
-            all_o, all_ml = gather_partials(part_o, part_ml)
-            all_o, all_ml = all_o.flatten(0, 1), all_ml.flatten(0, 1)
+            all_o, all_ml = gather_partials(rec_o, rec_ml)
         else:
-            all_o, all_ml = part_o, part_ml
+            all_o, all_ml = rec_o.unsqueeze(0), rec_ml.unsqueeze(0)
         pa.pa_merge_partials(out, all_o, all_ml)
 
     def barrier():
@@ -638,17 +640,18 @@ def run_context_parallel_gpu(args):
             "dtype": "bf16", "data": "synthetic",
             "config": {
                 "workload": w.describe(),
-                "step": "pa_decode_partial over this rank's table range + all-gather (NCCL) + pa_merge_partials",
+                "step": "pa_decode_partial over this rank's table range + pa_combine_partials + all-gather (NCCL) "
+                        "+ pa_merge_partials",
                 "ranges": [rank_block_range(w.max_blocks_per_seq, r, world) for r in range(world)],
                 "pieces_per_rank": S,
-                "gather_bytes_per_rank": (part_o.numel() + part_ml.numel()) * 4,
+                "gather_bytes_per_rank": (rec_o.numel() + rec_ml.numel()) * 4,
                 "decode_alg_bytes": dec_bytes,
                 "frac_of_measured_hbm_per_gpu": round(gbs / world / peaks["hbm_gbs"], 4),
                 "single_gpu_pa_decode_us": None if single_us is None else round(single_us, 3),
                 "max_abs_diff_vs_pa_decode": diff,
                 "parallelism": f"context parallel x{world} (one decode's blocks split across GPUs)",
             },
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 3 * args.steps,
             "clocks": sampler.summary(),
         }), flush=True)
     if world > 1:

@@ -403,6 +403,16 @@ PA_API pa_status_t pa_decode_partial(float* part_o, float* part_ml, const void* 
 PA_API int32_t pa_decode_partial_pieces(int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
                                         int32_t num_kv_heads, int32_t head_dim, int32_t range_blocks);
 
+/* Context parallelism, between steps 1 and 2 (on each GPU, so that the exchange carries one
+ * record per row): the num_parts pieces of each row (part_o / part_ml laid out as
+ * pa_decode_partial writes them) combined into one record of the same form, rec_o
+ * [num_seqs][q][H_q][D] = sum_k 2^(m_k - M) o_k and rec_ml [num_seqs][q][H_q][2] = {M, sum_k
+ * 2^(m_k - M) l_k}, M the largest m_k (-inf, 0 and o = 0 when every piece is empty). Checks as
+ * pa_merge_partials. */
+PA_API pa_status_t pa_combine_partials(float* rec_o, float* rec_ml, const float* part_o, const float* part_ml,
+                                       int32_t num_parts, int32_t num_seqs, int32_t q_per_seq,
+                                       int32_t num_q_heads, int32_t head_dim, pa_stream_t stream);
+
 /* Context parallelism, step 2: out[b][i][h] = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k over
  * num_parts pieces laid out part-major (part_o [num_parts][num_seqs][q][H_q][D], part_ml
  * [num_parts][num_seqs][q][H_q][2], as an all-gather of every GPU's pa_decode_partial pieces
@@ -419,7 +429,7 @@ PA_API const char* pa_status_string(pa_status_t status);
 
 /* ABI version (major * 10000 + minor * 100 + patch). 1.1 added pa_decode_fp8, pa_prefill
  * and the kv_cache_dtype fields at the end of pa_plan_hints_t and pa_plan_t; 1.2 added
- * pa_decode_partial, pa_decode_partial_pieces and pa_merge_partials. */
+ * pa_decode_partial, pa_decode_partial_pieces, pa_combine_partials and pa_merge_partials. */
 PA_API int32_t pa_version(void);
 
 #ifdef __cplusplus

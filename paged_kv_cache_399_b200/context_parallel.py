@@ -3,9 +3,10 @@
 Every rank holds the blocks of one contiguous range of table entries of every sequence
 in its own pool; it computes the attention over that range as unnormalised pieces
 (pa_decode_partial, its range cut into as many pieces as the decode heuristic would split
-it); the pieces are all-gathered (world * pieces * B * q * H_q * (D + 2) floats); every rank
-then merges them by the log-sum-exp
-rule of split softmax (pa_merge_partials; vLLM study notes, zihan-zhang.net, §4.3.1).
+it) and combines them into one record per row (pa_combine_partials); the records are
+all-gathered (world * B * q * H_q * (D + 2) floats); every rank then merges them by the
+log-sum-exp rule of split softmax (pa_merge_partials; vLLM study notes, zihan-zhang.net,
+§4.3.1).
 The exchange is the only communication: each rank reads its own pool only.
 """
 
@@ -59,8 +60,11 @@ def context_parallel_decode(out: torch.Tensor, query: torch.Tensor, key_cache: t
     part_ml = torch.empty((S, B, QS, HQ, 2), dtype=torch.float32, device=query.device)
     pa.pa_decode_partial(part_o, part_ml, query, key_cache, value_cache, block_tables, context_lens, q_per_seq,
                          scale, lo, hi)
-    all_o, all_ml = gather_partials(part_o, part_ml, group)
-    pa.pa_merge_partials(out, all_o.flatten(0, 1), all_ml.flatten(0, 1))
+    rec_o = torch.empty((B, QS, HQ, D), dtype=torch.float32, device=query.device)
+    rec_ml = torch.empty((B, QS, HQ, 2), dtype=torch.float32, device=query.device)
+    pa.pa_combine_partials(rec_o, rec_ml, part_o, part_ml)
+    all_o, all_ml = gather_partials(rec_o, rec_ml, group)
+    pa.pa_merge_partials(out, all_o, all_ml)
 
 
 def partial_pieces(query: torch.Tensor, key_cache: torch.Tensor, max_blocks_per_seq: int, world: int) -> int:

@@ -738,6 +738,32 @@ int32_t pa_decode_partial_pieces(int32_t num_seqs, int32_t q_per_seq, int32_t nu
   return plan.num_splits;
 }
 
+pa_status_t pa_combine_partials(float* rec_o, float* rec_ml, const float* part_o, const float* part_ml,
+                                int32_t num_parts, int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads,
+                                int32_t head_dim, pa_stream_t stream) {
+  if (num_parts <= 0 || num_seqs < 0 || q_per_seq <= 0 || num_q_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  const int64_t rows = static_cast<int64_t>(num_seqs) * q_per_seq * num_q_heads;
+  if (rows > INT32_MAX || static_cast<int64_t>(num_parts) * rows > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!rec_o || !rec_ml || !part_o || !part_ml || !aligned16(rec_o) || !aligned16(rec_ml) || !aligned16(part_o) ||
+      !aligned16(part_ml))
+    return PA_ERR_INVALID_ARG;
+  DecodeParams p = {};
+  p.num_seqs = num_seqs;
+  p.q_per_seq = q_per_seq;
+  p.num_q_heads = num_q_heads;
+  p.num_parts = num_parts;
+  p.partial_only = 1;
+  p.ws_o = const_cast<float*>(part_o);
+  p.ws_ml = reinterpret_cast<float2*>(const_cast<float*>(part_ml));
+  p.rec_o = rec_o;
+  p.rec_ml = reinterpret_cast<float2*>(rec_ml);
+  return pa::launch_merge_partials(p, head_dim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
 pa_status_t pa_merge_partials(void* out, const float* part_o, const float* part_ml, int32_t num_parts,
                               int32_t num_seqs, int32_t q_per_seq, int32_t num_q_heads, int32_t head_dim,
                               pa_stream_t stream) {

@@ -84,6 +84,10 @@ struct DecodeParams {
   // part-major ([piece][sequence][row]), never the output; num_parts > 0: the merge combines
   // num_parts such records per row, laid out [part][sequence][row] (gathered pieces)
   int32_t range_lo, range_hi, partial_only, num_parts;
+  // num_parts > 0 with partial_only: the merge writes one fp32 record per row instead of the
+  // output (o against the row's M [sequence][row][D], {M, L} [sequence][row])
+  float* rec_o;
+  float2* rec_ml;
 };
 
 // Host-side checks of a decode call's shapes and (when non-null) its plan, the ones

@@ -1542,6 +1542,18 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
   for (int w = 0; w < MW; ++w) M = fmaxf(M, s_ml[w].x);
   float L = 0.f;
   for (int w = 0; w < MW; ++w) L += s_ml[w].x == -INFINITY ? 0.f : s_ml[w].y * fast_exp2(s_ml[w].x - M);
+  if (p.num_parts > 0 && p.partial_only) {
+    // combine into one record of the row (o against M, then {M, L}): [sequence][row] in ws_rec_*
+    float* dst = p.rec_o + static_cast<size_t>(row) * D;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float v = 0.f;
+      for (int w = 0; w < MW; ++w)
+        v += s_ml[w].x == -INFINITY ? 0.f : fast_exp2(s_ml[w].x - M) * s_acc[w][d];
+      dst[d] = v;
+    }
+    if (threadIdx.x == 0) p.rec_ml[row] = make_float2(M, L);
+    return;
+  }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const int i = rq / p.num_q_heads;
   const int h = rq % p.num_q_heads;

@@ -34,7 +34,8 @@ PA_PATH_TILE = 2
 PA_PATH_TCGEN05 = 3
 
 EXPORTED = ["pa_reshape_and_cache", "pa_decode_plan", "pa_decode_workspace_size", "pa_decode", "pa_decode_fp8",
-            "pa_prefill", "pa_decode_partial", "pa_decode_partial_pieces", "pa_merge_partials",
+            "pa_prefill", "pa_decode_partial", "pa_decode_partial_pieces", "pa_combine_partials",
+            "pa_merge_partials",
             "pa_decode_static_scratch", "pa_validate", "pa_get_device_error",
             "pa_selftest_bounded_wait", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_status_string",
             "pa_version"]
@@ -107,6 +108,8 @@ _lib.pa_decode_partial.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
                                    ctypes.c_float, _I32, _I32, _I32, _P]
 _lib.pa_decode_partial_pieces.restype = _I32
 _lib.pa_decode_partial_pieces.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32]
+_lib.pa_combine_partials.restype = _I32
+_lib.pa_combine_partials.argtypes = [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P]
 _lib.pa_merge_partials.restype = _I32
 _lib.pa_merge_partials.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P]
 _lib.pa_decode_static_scratch.restype = _I32
@@ -334,6 +337,21 @@ def pa_decode_partial_pieces(num_seqs: int, q_per_seq: int, num_q_heads: int, nu
     """Pieces the decode heuristic takes for ranges of range_blocks table entries (0: bad shapes)."""
     return int(_lib.pa_decode_partial_pieces(num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim,
                                              range_blocks))
+
+
+def pa_combine_partials(rec_o: torch.Tensor, rec_ml: torch.Tensor, part_o: torch.Tensor, part_ml: torch.Tensor,
+                        stream=None) -> None:
+    """One record per row, rec_o [B, q, H_q, D] and rec_ml [B, q, H_q, 2] fp32, from the pieces
+    part_o [P, B, q, H_q, D] and part_ml [P, B, q, H_q, 2]."""
+    assert rec_o.dtype == rec_ml.dtype == part_o.dtype == part_ml.dtype == torch.float32
+    for t in (rec_o, rec_ml, part_o, part_ml):
+        assert t.is_contiguous()
+    P, B, QS, HQ, D = part_o.shape
+    assert tuple(rec_o.shape) == (B, QS, HQ, D) and tuple(rec_ml.shape) == (B, QS, HQ, 2)
+    assert tuple(part_ml.shape) == (P, B, QS, HQ, 2)
+    st = _lib.pa_combine_partials(_ptr(rec_o), _ptr(rec_ml), _ptr(part_o), _ptr(part_ml), P, B, QS, HQ, D,
+                                  _stream(stream))
+    _check(st, "pa_combine_partials")
 
 
 def pa_merge_partials(out: torch.Tensor, part_o: torch.Tensor, part_ml: torch.Tensor, stream=None) -> None:

@@ -390,6 +390,16 @@ def test_partial_decode_and_merge_reject_bad_arguments_before_launch(pa):
     assert merge(po=16384 + 4) == pa.PA_ERR_INVALID_ARG
     assert merge(d=96) == pa.PA_ERR_UNSUPPORTED
     assert merge(B=0, out=None) == pa.PA_OK
+    def combine(**kw):
+        a = dict(ro=8192, rml=16384, po=32768, pml=49152, P=3, B=2, qs=1, hq=8, d=128)
+        a.update(kw)
+        return lib.pa_combine_partials(a["ro"], a["rml"], a["po"], a["pml"], a["P"], a["B"], a["qs"], a["hq"],
+                                       a["d"], None)
+    assert combine(P=0) == pa.PA_ERR_INVALID_ARG
+    assert combine(ro=None) == pa.PA_ERR_INVALID_ARG
+    assert combine(rml=16384 + 8) == pa.PA_ERR_INVALID_ARG
+    assert combine(d=32) == pa.PA_ERR_UNSUPPORTED
+    assert combine(B=0, ro=None) == pa.PA_OK
     # pieces of a range: at least one for good shapes, 0 for bad ones
     assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 128, 1024) >= 1
     assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 96, 1024) == 0

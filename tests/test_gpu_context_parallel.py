@@ -1,5 +1,6 @@
 """Context parallelism on one GPU: pa_decode_partial over the table ranges that the ranks of a
-group would take, merged by pa_merge_partials, against the fp64 oracle's decode. The ranks are
+group would take, merged by pa_merge_partials (directly, or after pa_combine_partials turned each
+rank's pieces into one record per row), against the fp64 oracle's decode. The ranks are
 emulated one after another on this device (no rank waits for another): the pieces of each range
 go to their slice of one part-major buffer, as the all-gather leaves them. Table entries outside
 a range are poisoned, and in the pools of the separate-pool case every block of another range
@@ -84,6 +85,18 @@ def test_partial_pieces_merge_to_the_decode(case, world, prepared):
     pa.pa_merge_partials(out2, part_o[perm].contiguous(), part_ml[perm].contiguous())
     torch.cuda.synchronize()
     assert_close(out2, ref, f"{case[0]}/world {world}, pieces reordered")
+    # each rank combines its own pieces into one record per row; the records merge to the same
+    B, QS, HQ, D = w.query.shape
+    S = part_o.shape[0] // world
+    rec_o = torch.empty((world, B, QS, HQ, D), dtype=torch.float32, device="cuda")
+    rec_ml = torch.empty((world, B, QS, HQ, 2), dtype=torch.float32, device="cuda")
+    for r in range(world):
+        pa.pa_combine_partials(rec_o[r], rec_ml[r], part_o[r * S:(r + 1) * S].contiguous(),
+                               part_ml[r * S:(r + 1) * S].contiguous())
+    out3 = torch.empty_like(out)
+    pa.pa_merge_partials(out3, rec_o, rec_ml)
+    torch.cuda.synchronize()
+    assert_close(out3, ref, f"{case[0]}/world {world}, records combined per rank")
 
 
 @pytest.mark.parametrize("case", CASES[:2], ids=[c[0] for c in CASES[:2]])
