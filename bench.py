@@ -37,12 +37,12 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call (mean
     # of three calls), from one ncu capture per workload (commands in profiles/); valid only for
     # the kernel sources they were taken on
-    "llama8b": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 654_490_000},
-    "llama70b_long": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 1_352_650_000},
-    "spec_verify": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 414_740_000},
-    "prefix_sharing": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 210_070_000},
-    "sliding_window": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 273_410_000},
-    "llama8b_fp8": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 280_890_000},
+    "llama8b": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 654_440_000},
+    "llama70b_long": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 1_352_130_000},
+    "spec_verify": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 414_870_000},
+    "prefix_sharing": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 210_040_000},
+    "sliding_window": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 273_460_000},
+    "llama8b_fp8": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 280_740_000},
 }
 
 # the same for one pa_copy_blocks launch of a copy workload (keyed by COPY_SOURCES' hash;
@@ -427,7 +427,7 @@ def measure_config(name, args, dev, stream, peaks):
 NCU_PREFILL_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one pa_prefill launch (mean of three),
     # valid only for the kernel sources it was taken on
-    "chunked_prefill": {"source_hash": "1472c5125bdf39a6", "bytes_per_launch": 204_880_000},
+    "chunked_prefill": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 199_280_000},
 }
 
 
