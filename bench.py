@@ -330,12 +330,13 @@ def _ncu_traffic(name):
     return None
 
 
-def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
-    """Mean CUDA-event time of `calls` pa_decode calls (each after the step's cache write,
-    events on the launching stream around the decode only), in ms; the same calls without
-    host overhead: one CUDA graph of 20 back-to-back calls, replayed (µs per call, None when
-    capture is unavailable); and the mean event time of the step's cache writes (ms), timed
-    apart from the decode."""
+def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
+    """CUDA-event times of `calls` pa_decode calls (each after the step's cache write, events
+    on the launching stream around the decode only): their mean and median in ms; the median
+    of the same calls made cold, with `flush` (a buffer twice the L2 size) written before each
+    step outside the events (None without `flush`); the calls without host overhead: one CUDA graph of 20
+    back-to-back calls, replayed (µs per call, None when capture is unavailable); and the mean
+    event time of the step's cache writes (ms), timed apart from the decode."""
     import torch
     write, decode = _hot_path(pa, w, v, plan, ws, stream)
     barrier()
@@ -348,8 +349,20 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
         decode()
         b.record(stream)
     barrier()
-    decode_ms = statistics.mean(a.elapsed_time(b) for _, _, a, b in quads)
+    times = [a.elapsed_time(b) for _, _, a, b in quads]
+    decode_ms, median_ms = statistics.mean(times), statistics.median(times)
     write_ms = statistics.mean(c.elapsed_time(d) for c, d, _, _ in quads)
+    cold_ms = None
+    if flush is not None:
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+        for a, b in pairs:
+            flush.zero_()
+            write()
+            a.record(stream)
+            decode()
+            b.record(stream)
+        barrier()
+        cold_ms = statistics.median(a.elapsed_time(b) for a, b in pairs)
     graph_us = None
     try:
         per_graph, reps = 20, max(1, calls // 20)
@@ -370,7 +383,7 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier):
         del graph
     except Exception as exc:  # capture is a measurement aid: report why it is missing
         print(f"graph timing unavailable: {exc}", file=sys.stderr)
-    return decode_ms, graph_us, write_ms
+    return decode_ms, median_ms, cold_ms, graph_us, write_ms
 
 
 def measure_config(name, args, dev, stream, peaks):
@@ -395,16 +408,23 @@ def measure_config(name, args, dev, stream, peaks):
         decode()
     barrier()
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(dev.index)
     with sampler:
-        decode_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.config_calls, barrier)
+        decode_ms, median_ms, cold_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream,
+                                                                        args.config_calls, barrier, flush)
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
+    del flush
     dec_bytes = decode_bytes(w)
     gbs = dec_bytes / (decode_ms * 1e-3) / 1e9
     rec = {
         "workload": w.describe(),
         "calls": args.config_calls,
         "decode_us_per_call": round(decode_ms * 1e3, 3),
+        "decode_us_per_call_median": round(median_ms * 1e3, 3),
+        # L2 written over (a buffer twice its size) before every step, outside the events
+        "decode_us_per_call_cold": round(cold_ms * 1e3, 3),
+        "frac_cold": round(dec_bytes / (cold_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "decode_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
         "decode_alg_bytes": dec_bytes,
         "decode_logical_bytes": decode_bytes(w, unique=False),
@@ -729,7 +749,7 @@ def run_gpu(args):
         # (2) per-kernel: events around each pa_decode launch of another K steps, and the
         # same calls graph-replayed (for the small configs the events mostly time the
         # Python call)
-        decode_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
+        decode_ms, _, _, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
         decode_ms = max_over_ranks(decode_ms)
         if graph_us is not None:
             graph_us = max_over_ranks(graph_us)

@@ -6,8 +6,10 @@
 // tiles of 8 blocks = 128 tokens. The CTAs of the persistent grid form groups of S
 // (a divisor of H_kv); CTA li of a group takes the kv heads li, li + S, ... . All groups
 // walk the same enumeration of (sequence, kv-head index, row chunk, tile) and split it
-// into equal contiguous ranges, one per group, computed in the kernel from context_lens
-// (no pre-pass); the S CTAs of a group therefore read the kv-head slices of the same
+// into contiguous ranges of equal cost, one per group, computed in the kernel from
+// context_lens (no pre-pass): a tile costs kCostTile, and the start of a unit costs
+// kCostUnit more (its first tile, the previous unit's epilogue; measured at about one
+// tile period). The S CTAs of a group therefore read the kv-head slices of the same
 // blocks at about the same time. A unit cut by a range boundary leaves partial records,
 // combined afterwards by tcm_merge_kernel.
 //
@@ -45,6 +47,11 @@ constexpr int kProducerWarp = 8;   // K boxes and Q rows
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10; // V boxes
 constexpr float kRescaleLog2 = 8.f;
+// Range cost: tile kCostTile, start of a unit kCostUnit extra. Windows are summed as
+// (tiles << kPackShift) + units with tiles, one 64-bit add per window.
+constexpr int kCostTile = 4;
+constexpr int kCostUnit = 4;
+constexpr int kPackShift = 28;
 constexpr int kHalfBytes = kTileBlocks * kHalfTileBytes;  // one 64-column half of a tile
 constexpr int kStageBytes = 2 * kHalfBytes;               // K or V of one tile
 constexpr int kPGroupBytes = kTileTokens * 16;            // P^T: 8 columns x 128 tokens
@@ -273,8 +280,11 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   }
   grid_dependency_wait();
 
-  // ---- this CTA's group, kv-head set and tile range [t0, t1) of the W tiles every group
-  // walks: prefix sums over the windows
+  // ---- this CTA's group, kv-head set and range [t0, t1) of the Wc cost units every group
+  // walks: prefix sums over the windows. In cost units, unit u of a window spans kCostUnit +
+  // kCostTile * tiles positions: its tile 0 the first kCostUnit + kCostTile, every later tile
+  // kCostTile. A group takes the tiles from the one whose span holds t0 to the one before
+  // the one whose span holds t1 (all tiles past the last position when t1 = Wc).
   const int S = p.tc_group;
   const int li = c % S;
   const int NG = static_cast<int>(gridDim.x) / S;
@@ -284,13 +294,22 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
   const int rpm = p.rows;  // query rows of one member (sequence)
   long long* wsum = reinterpret_cast<long long*>(smem + L::offScan);
   int* start = reinterpret_cast<int*>(smem + L::offScan + 96);
-  long long W, t0, t1;
-  int NGe;  // groups that take part: at most one per tile, so that every range is non-empty
+  long long* tpos = reinterpret_cast<long long*>(smem + L::offScan + 104);  // T0, T1, UE
+  constexpr long long kUnitsMask = (1ll << tcm::kPackShift) - 1;
+  auto cost_of = [](long long pk) {  // cost units of a packed (tiles, units) sum
+    return tcm::kCostTile * (pk >> tcm::kPackShift) + tcm::kCostUnit * (pk & kUnitsMask);
+  };
+  long long Wc, t0, t1;
+  int NGe;  // groups that take part: each range spans at least one tile's cost, so none is empty
+  int n;    // tiles of this CTA
   {
     const int chunk = (nwin + tcm::kThreads - 1) / tcm::kThreads;
     const int s0 = min(nwin, static_cast<int>(threadIdx.x) * chunk), s1 = min(nwin, s0 + chunk);
     long long local = 0;
-    for (int ww = s0; ww < s1; ++ww) local += static_cast<long long>(tcm::window_tiles<kWin>(p, ww)) * upb;
+    for (int ww = s0; ww < s1; ++ww) {
+      const long long tw = tcm::window_tiles<kWin>(p, ww);
+      if (tw > 0) local += ((tw * upb) << tcm::kPackShift) + upb;
+    }
     long long v = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -299,32 +318,51 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
     }
     if (lane == 31) wsum[warp] = v;
     __syncthreads();
-    long long base = 0;
-    W = 0;
+    long long base = 0, Wpk = 0;
     for (int w2 = 0; w2 < tcm::kThreads / 32; ++w2) {
       if (w2 < warp) base += wsum[w2];
-      W += wsum[w2];
+      Wpk += wsum[w2];
     }
-    NGe = static_cast<int>(min(static_cast<long long>(NG), W));
+    Wc = cost_of(Wpk);
+    NGe = static_cast<int>(min(static_cast<long long>(NG), Wc / (tcm::kCostTile + tcm::kCostUnit)));
     const int gi = c / S;
-    t0 = gi < NGe ? static_cast<long long>(gi) * W / NGe : 0;
-    t1 = gi < NGe ? static_cast<long long>(gi + 1) * W / NGe : 0;
-    const long long excl = base + v - local;
-    if (local > 0 && t0 < t1 && t0 >= excl && t0 < excl + local) {
-      long long acc = excl;
+    t0 = gi < NGe ? static_cast<long long>(gi) * Wc / NGe : 0;
+    t1 = gi < NGe ? static_cast<long long>(gi + 1) * Wc / NGe : 0;
+    const long long excl = base + v - local;  // packed sums of the windows before s0
+    const long long ec = cost_of(excl), lc = cost_of(local);
+    if (gi < NGe && t1 == Wc && threadIdx.x == 0) tpos[1] = Wpk >> tcm::kPackShift;
+    // the tile whose span holds position `pos` of this thread's windows: window, tile of the
+    // window, global tile index, and the cost end of its unit
+    for (int e = 0; e < 2; ++e) {
+      const long long pos = e == 0 ? t0 : t1;
+      if (gi >= NGe || pos >= Wc || pos < ec || pos >= ec + lc) continue;
+      long long acc = ec, acct = excl >> tcm::kPackShift;
       for (int ww = s0; ww < s1; ++ww) {
-        const long long tb = static_cast<long long>(tcm::window_tiles<kWin>(p, ww)) * upb;
-        if (t0 < acc + tb) {
-          start[0] = ww;
-          start[1] = static_cast<int>(t0 - acc);
+        const int tw = tcm::window_tiles<kWin>(p, ww);
+        const long long uc = tcm::kCostUnit + static_cast<long long>(tcm::kCostTile) * tw;
+        const long long cw = tw > 0 ? uc * upb : 0;
+        if (pos < acc + cw) {
+          const int k = static_cast<int>((pos - acc) / uc);
+          const long long within = pos - acc - k * uc;
+          const int x = within < tcm::kCostUnit + tcm::kCostTile
+                            ? 0 : static_cast<int>((within - tcm::kCostUnit) / tcm::kCostTile);
+          if (e == 0) {
+            start[0] = ww;
+            start[1] = k * tw + x;
+            tpos[0] = acct + static_cast<long long>(k) * tw + x;
+          } else {
+            tpos[1] = acct + static_cast<long long>(k) * tw + x;
+            tpos[2] = acc + (k + 1) * uc;
+          }
           break;
         }
-        acc += tb;
+        acc += cw;
+        acct += static_cast<long long>(tw) * upb;
       }
     }
     __syncthreads();
+    n = gi < NGe ? static_cast<int>(tpos[1] - tpos[0]) : 0;
   }
-  const int n = static_cast<int>(t1 - t0);
   if (n <= 0) {  // uniform: no tiles for this CTA
     if (threadIdx.x == 0) p.tc_desc[c] = make_int4(-1, 0, 0, 0);
     grid_launch_dependents();
@@ -871,8 +909,10 @@ decode_tcm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap
           // started here, so this CTA holds its first piece
           int4 dsc = make_int4(-1, 0, 0, 0);
           if (w.x != w.tiles - 1 && (j > 0 || first_x == 0)) {
-            const long long E = t1 + (w.tiles - 1 - w.x);  // end tile (exclusive) of the unit
-            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((E * NGe - 1) / W) * S + li, w.w, w.k);
+            // the unit ends at cost position UE past t1: the last group whose t0 is below it
+            // holds its last tile
+            const long long UE = tpos[2];
+            dsc = make_int4(j == 0 ? 2 * c : 2 * c + 1, static_cast<int>((UE * NGe - 1) / Wc) * S + li, w.w, w.k);
           }
           p.tc_desc[c] = dsc;
         }
