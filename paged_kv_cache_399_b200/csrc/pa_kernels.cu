@@ -1511,27 +1511,48 @@ __global__ void __launch_bounds__(32 * kMergeMaxWarps) merge_kernel(const Decode
     return (k < nsh ? static_cast<size_t>(b) * p.share_splits + k
                     : own_region + static_cast<size_t>(b) * p.num_splits + (k - nsh)) * RQ + rq;
   };
-  // this warp's maximum: its splits' (m, l) are spread over the lanes
-  float Mw = -INFINITY;
-  for (int s = warp + MW * lane; s < ns; s += 32 * MW) Mw = fmaxf(Mw, p.ws_ml[rec_of(s)].x);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) Mw = fmaxf(Mw, __shfl_xor_sync(kFull, Mw, off));
-  float Lw = 0.f, acc[DPL];
+  // this warp's splits s = warp, warp + MW, ...: four at a time, their (m, l) and this lane's
+  // slices of their o loaded together, folded in against the warp's running maximum
+  float Mw = -INFINITY, Lw = 0.f, acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-  for (int s = warp; s < ns; s += MW) {
-    const size_t rec = rec_of(s);
-    const float2 ml = p.ws_ml[rec];
-    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - Mw);
-    Lw += w * ml.y;
-    const float* src = p.ws_o + rec * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(src);
-      acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-    } else {
-      const float2 x = *reinterpret_cast<const float2*>(src);
-      acc[0] += w * x.x; acc[1] += w * x.y;
+  for (int s0 = warp; s0 < ns; s0 += 4 * MW) {
+    float2 ml[4];
+    float x[4][DPL];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + u * MW;
+      ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) x[u][e] = 0.f;
+      if (s < ns) {
+        const size_t rec = rec_of(s);
+        ml[u] = p.ws_ml[rec];
+        const float* src = p.ws_o + rec * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          x[u][0] = v.x; x[u][1] = v.y;
+        }
+      }
+    }
+    float Mn = Mw;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) Mn = fmaxf(Mn, ml[u].x);
+    if (Mn == -INFINITY) continue;  // uniform over the warp: no key in these splits yet
+    const float rs = Mw == -INFINITY ? 0.f : fast_exp2(Mw - Mn);  // what is folded in so far
+    Lw *= rs;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] *= rs;
+    Mw = Mn;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = (ml[u].x == -INFINITY) ? 0.f : fast_exp2(ml[u].x - Mw);
+      Lw += w * ml[u].y;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] += w * x[u][e];
     }
   }
   if (lane == 0) s_ml[warp] = make_float2(Mw, Lw);

@@ -961,42 +961,54 @@ __global__ void __launch_bounds__(tcm::kMergeThreads) tcm_merge_kernel(const Dec
     auto rec_of = [=](int k) {
       return recs + static_cast<size_t>(k == 0 ? slot0 : 2 * (c + k * S)) * rs;
     };
-    // one row per warp: lanes take the pieces for the maximum and the weights, then each
-    // lane accumulates 4 of the D columns over the pieces in order, 4 pieces' loads at a time
+    // one row per warp, 32 pieces at a time: lane k takes piece k's (m, l), and the output
+    // slices of the first four pieces are loaded with them (nothing waits for the maximum);
+    // each lane accumulates 4 of the D columns over the pieces in order, 4 pieces' loads at
+    // a time, against a running maximum
     for (int r = warp; r < nrows; r += tcm::kMergeThreads / 32) {
-      float M = -INFINITY;
-      for (int k = lane; k < pieces; k += 32) M = fmaxf(M, reinterpret_cast<const float2*>(rec_of(k) + N * D)[r].x);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+      float M = -INFINITY, l = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float l = 0.f;
-      if (M != -INFINITY) {
-        for (int k0 = 0; k0 < pieces; k0 += 32) {
-          float wk = 0.f, lk = 0.f;
-          if (k0 + lane < pieces) {
-            const float2 ml = reinterpret_cast<const float2*>(rec_of(k0 + lane) + N * D)[r];
-            wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
-            lk = ml.y * wk;
-          }
+      for (int k0 = 0; k0 < pieces; k0 += 32) {
+        const int kn = min(32, pieces - k0);
+        const float2 ml = lane < kn ? reinterpret_cast<const float2*>(rec_of(k0 + lane) + N * D)[r]
+                                    : make_float2(-INFINITY, 0.f);
+        float4 o4[4];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
-          l += lk;
-          const int kn = min(32, pieces - k0);
-          for (int kk = 0; kk < kn; kk += 4) {
-            float4 o4[4];
+        for (int u = 0; u < 4; ++u)
+          o4[u] = u < kn ? reinterpret_cast<const float4*>(rec_of(k0 + u) + r * D)[lane]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        float Mb = ml.x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(kFull, Mb, o));
+        const float Mn = fmaxf(M, Mb);
+        if (Mn == -INFINITY) continue;  // uniform: no key in these pieces yet
+        const float rs = M == -INFINITY ? 0.f : fast_exp2(M - Mn);  // what is folded in so far
+        acc.x *= rs;
+        acc.y *= rs;
+        acc.z *= rs;
+        acc.w *= rs;
+        l *= rs;
+        M = Mn;
+        const float wk = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - M);
+        float lk = ml.y * wk;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
+        l += lk;
+        for (int kk = 0; kk < kn; kk += 4) {
+          if (kk > 0) {
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               o4[u] = kk + u < kn ? reinterpret_cast<const float4*>(rec_of(k0 + kk + u) + r * D)[lane]
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float wb = __shfl_sync(kFull, wk, (kk + u) & 31);
-              if (kk + u < kn) {
-                acc.x = fmaf(o4[u].x, wb, acc.x);
-                acc.y = fmaf(o4[u].y, wb, acc.y);
-                acc.z = fmaf(o4[u].z, wb, acc.z);
-                acc.w = fmaf(o4[u].w, wb, acc.w);
-              }
+          for (int u = 0; u < 4; ++u) {
+            const float wb = __shfl_sync(kFull, wk, (kk + u) & 31);
+            if (kk + u < kn) {
+              acc.x = fmaf(o4[u].x, wb, acc.x);
+              acc.y = fmaf(o4[u].y, wb, acc.y);
+              acc.z = fmaf(o4[u].z, wb, acc.z);
+              acc.w = fmaf(o4[u].w, wb, acc.w);
             }
           }
         }
