@@ -8,29 +8,27 @@
 //
 // This is a contraction with hundreds of query rows per kv head, so the query rows go on the
 // MMA's M dimension (the decode kernels put the keys there):
-//   S[128 rows][128 keys] = Q[128 rows][D] . K^T[D][128 keys]    K-major A (Q) and B (K)
-//   softmax per row over the tile's 128 keys, split between two warpgroups: thread r of
-//   warpgroup h owns row r (TMEM lane r) and keys 64h .. 64h+63, so the two threads of a row
-//   exchange only their partial maxima (shared memory, one named barrier per tile); the
-//   running reference maximum moves only when a tile's maximum exceeds it by more than 2^8
-//   (numerator and denominator share the reference, so the result is exact either way);
-//   each warpgroup keeps its own part of the row sum, joined at the end;
-//   O[128 rows][D] += P[128 rows][128 keys] . V[128 keys][D]     K-major A (P, from shared
+//   S[128 rows][64 keys] = Q[128 rows][D] . K^T[D][64 keys]      K-major A (Q) and B (K)
+//   softmax per row over the tile's 64 keys: thread r owns row r (TMEM lane r) and the
+//   whole tile row, so no thread waits for another's maximum; the running reference
+//   maximum moves only when a tile's maximum exceeds it by more than 2^8 (numerator and
+//   denominator share the reference, so the result is exact either way);
+//   O[128 rows][D] += P[128 rows][64 keys] . V[64 keys][D]       K-major A (P, from shared
 //                                                                memory), MN-major B (V)
-// Two warps per SM sub-partition share the softmax, so one's latencies hide behind the
-// other's work; warpgroup h also rescales and writes columns 64h .. 64h+63 of O.
+// Two CTAs share an SM (112 KB of shared memory and 256 TMEM columns each), so the softmax
+// of one runs while the other's MMAs do, and each SM sub-partition holds a softmax warp of
+// both.
 // A CTA owns 128 rows = 128 / G consecutive chunk tokens x the G query heads of one kv head
-// (GQA: every row of a CTA reads the same K/V), and walks the key tiles of 8 blocks from
+// (GQA: every row of a CTA reads the same K/V), and walks the key tiles of 4 blocks from
 // the sequence's first block to the block of its last row's position.
 //
-// Roles: warps 0-7 load Q, run the softmax and the epilogue (two warpgroups); warp 8 issues
-// the K boxes and warp 9 the V boxes (16 TMA boxes of 2 KB per tile each); warp 10 holds the
-// TMEM allocation and one of its threads issues the MMAs (S of a tile as soon as its K has
-// landed and an S buffer is free; PV of a tile as soon as its P and V are in shared memory).
-// A K stage is released when its S completes, a V stage when its PV completes.
-// TMEM: S double buffer in columns [0, 256), O in [256, 384).
-// Shared memory: Q (32 KB), P (32 KB), 2 K stages and 2 V stages of 32 KB, the softmax's
-// exchange area, barriers.
+// Roles: warps 0-3 load Q, run the softmax and the epilogue; warp 4 issues the K boxes and
+// warp 5 the V boxes (8 TMA boxes of 2 KB per tile each); warp 6 holds the TMEM allocation
+// and one of its threads issues the MMAs (S of a tile as soon as its K has landed and an S
+// buffer is free; PV of a tile as soon as its P and V are in shared memory). A K stage is
+// released when its S completes, a V stage when its PV completes.
+// TMEM: S double buffer in columns [0, 128), O in [128, 256).
+// Shared memory: Q (32 KB), P (16 KB), 2 K stages and 2 V stages of 16 KB, barriers.
 
 namespace pa {
 
@@ -38,30 +36,30 @@ namespace pfl {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                        // query rows of a CTA: the MMA's M
-constexpr int kTileBlocks = 8;
-constexpr int kKeys = kTileBlocks * kBlockSize;   // 128 keys per tile
+constexpr int kTileBlocks = 4;
+constexpr int kKeys = kTileBlocks * kBlockSize;   // 64 keys per tile
 constexpr int kStages = 2;
-constexpr int kThreads = 352;                     // 11 warps
-constexpr int kSoftmaxWarps = 8;                  // two warpgroups, each owning half of the keys
-constexpr int kKWarp = 8, kVWarp = 9, kMmaWarp = 10;
-constexpr int kHalfBytes = kKeys * 128;           // one 64-column half of a K or V tile: 16 KB
-constexpr int kTileBytes = 2 * kHalfBytes;        // 32 KB
-constexpr int kRowsHalfBytes = kRows * 128;       // one 64-column half of Q or P: 16 KB
+constexpr int kThreads = 224;                     // 7 warps
+constexpr int kCtasPerSm = 2;
+constexpr int kSoftmaxWarps = 4;                  // one warpgroup: thread r owns row r
+constexpr int kKWarp = 4, kVWarp = 5, kMmaWarp = 6;
+constexpr int kHalfBytes = kKeys * 128;           // one 64-column half of a K or V tile: 8 KB
+constexpr int kTileBytes = 2 * kHalfBytes;        // 16 KB
+constexpr int kRowsHalfBytes = kRows * 128;       // one 64-column half of Q, or P: 16 KB
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kTmemCols = 512;               // S double buffer + O, rounded to a power of 2
+constexpr uint32_t kTmemCols = 256;               // S double buffer + O (a power of 2)
 constexpr uint32_t kTmemO = 2 * kKeys;            // column of O
 
 struct Smem {
   static constexpr int offQ = 0;
   static constexpr int offP = offQ + 2 * kRowsHalfBytes;
-  static constexpr int offK = offP + 2 * kRowsHalfBytes;
+  static constexpr int offK = offP + kRowsHalfBytes;
   static constexpr int offV = offK + kStages * kTileBytes;
-  // per tile parity and warpgroup: each row's partial maximum; then the partial row sums
-  static constexpr int offX = offV + kStages * kTileBytes;
-  static constexpr int offBars = offX + (2 * 2 + 2) * kRows * 4;
+  static constexpr int offBars = offV + kStages * kTileBytes;
   static constexpr int kBytes = offBars + 256;
   static_assert(offK % 1024 == 0 && offV % 1024 == 0 && offP % 1024 == 0, "swizzled operands");
-  static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
+  // two CTAs per SM: 228 KB of shared memory less 1 KB reserved per CTA
+  static_assert(kCtasPerSm * (kBytes + 1024) <= 228 * 1024, "shared memory of two CTAs");
 };
 
 struct Bars {
@@ -75,12 +73,10 @@ __device__ __forceinline__ uint32_t row_chunk_offset(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * kRowsHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// Named barrier of the two softmax warpgroups (id 1, 256 threads).
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 }  // namespace pfl
 
-__global__ void __launch_bounds__(pfl::kThreads, 1)
+__global__ void __launch_bounds__(pfl::kThreads, pfl::kCtasPerSm)
 prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v) {
   using L = pfl::Smem;
@@ -145,7 +141,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
 
   if (warp == pfl::kKWarp || warp == pfl::kVWarp) {
     // ------------------------------------------------------------ TMA producers
-    // lanes 0..15 issue the tile's 16 boxes (half = lane / 8, block = lane % 8); lanes 0..7
+    // lanes 0..7 issue the tile's 8 boxes (half = lane / 4, block = lane % 4); lanes 0..3
     // read the next tile's block ids while this one is issued
     const bool is_k = warp == pfl::kKWarp;
     const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
@@ -169,7 +165,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       if (!ok) break;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], pfl::kTileBytes);
       __syncwarp();
-      const int hf = lane >> 3, jj = lane & (kTileBlocks - 1);
+      const int hf = lane / kTileBlocks, jj = lane & (kTileBlocks - 1);
       if (lane < 2 * kTileBlocks)
         tma_load_3d(smem + stage_off + s * pfl::kTileBytes + hf * pfl::kHalfBytes + jj * kHalfTileBytes, tmap,
                     &full[s], hf * 64, kvh, ph * kBlockSize);
@@ -279,22 +275,18 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     __syncwarp();
   } else {
     // ------------------------------------------------------------ Q, softmax, epilogue
-    const int hk = warp >> 2;                  // warpgroup: keys 64hk .. 64hk+63 of a tile
-    const int r = threadIdx.x & 127;           // row = TMEM lane
+    const int r = threadIdx.x;                 // row = TMEM lane
     const int tt = r / p.group;                // chunk token of the row (within the CTA)
     const int h = kvh * p.group + (r - tt * p.group);
     const bool valid = tt < ntok;
     const int pos = valid ? pos0 + tt : -1;    // the row's position: keys 0 .. pos visible
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t o_col = tmem + lane_off + pfl::kTmemO + hk * (D / 2);
-    float* xmax = reinterpret_cast<float*>(smem + L::offX);             // [2 parities][2 groups][128]
-    float* xsum = xmax + 4 * pfl::kRows;                                 // [2 groups][128]
+    const uint32_t o_col = tmem + lane_off + pfl::kTmemO;
     const size_t row_off = (static_cast<size_t>(qs + tok0 + tt) * p.num_q_heads + h) * D;
-    {  // this warpgroup's half of the Q row -> shared memory, 128-byte swizzled K-major;
-       // zeros for rows past the chunk
+    {  // the Q row -> shared memory, 128-byte swizzled K-major; zeros for rows past the chunk
       const uint4* src = reinterpret_cast<const uint4*>(p.query + row_off);
 #pragma unroll
-      for (int c = hk * 8; c < hk * 8 + 8; ++c) {
+      for (int c = 0; c < 16; ++c) {
         const uint4 v = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(smem + L::offQ + pfl::row_chunk_offset(r, c)) = v;
       }
@@ -311,9 +303,9 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     for (int j = 0; j < nk; ++j) {
       wait(&bars.s_full[j & 1], (j >> 1) & 1);
       tc_fence_after_sync();
-      uint32_t sv[64];
-      tmem_ld32(tmem + lane_off + (j & 1) * kKeys + hk * 64, *reinterpret_cast<uint32_t(*)[32]>(sv));
-      tmem_ld32(tmem + lane_off + (j & 1) * kKeys + hk * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      uint32_t sv[kKeys];
+      tmem_ld32(tmem + lane_off + (j & 1) * kKeys, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tmem + lane_off + (j & 1) * kKeys + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
       tc_wait_ld();
       tc_fence_before_sync();
       __syncwarp();
@@ -322,38 +314,55 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       // position are past the context or belong to later chunk tokens): only tiles that reach
       // past the row's position take the mask. The maximum is taken over the raw scores
       // (the scale is >= 0) and the scale is applied once, in the exponent's FMA.
-      const int k0 = j * kKeys + hk * 64;
-      const bool edge = k0 + 63 > pos;
-      float pmx = -INFINITY;
+      const int k0 = j * kKeys;
+      const bool edge = k0 + kKeys - 1 > pos;
+      const int nvis = edge ? min(kKeys, max(0, pos - k0 + 1)) : kKeys;  // keys k < nvis are visible
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (edge) {
-        const int nvis = min(64, max(0, pos - k0 + 1));  // keys k < nvis are visible
 #pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (k < nvis) pmx = fmaxf(pmx, __uint_as_float(sv[k]));
+        for (int k = 0; k < kKeys; ++k)
+          if (k < nvis) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[k]));
       } else {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) pmx = fmaxf(pmx, __uint_as_float(sv[k]));
+        for (int k = 0; k < kKeys; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[k]));
       }
-      // the row's maximum over both halves of the tile, in log2 units
-      xmax[((j & 1) * 2 + hk) * pfl::kRows + r] = pmx;
-      pfl::softmax_sync();
-      const float rmx = fmaxf(pmx, xmax[((j & 1) * 2 + (hk ^ 1)) * pfl::kRows + r]);
-      const float mx = rmx == -INFINITY ? -INFINITY : rmx * cs;
-      // move the reference when the tile's maximum exceeds it by more than 2^8; this
-      // warpgroup's half of O (TMEM) is rescaled by the whole warp whenever one of its rows
-      // moved (tcgen05.ld/st are warp-collective), the other rows by 1
+      const float rmx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mx = rmx == -INFINITY ? -INFINITY : rmx * cs;   // the tile's row maximum, log2 units
+      // move the reference when the tile's maximum exceeds it by more than 2^8; O (TMEM) is
+      // rescaled by the whole warp whenever one of its rows moved (tcgen05.ld/st are
+      // warp-collective), the other rows by 1
       const bool need = mx > mref + pfl::kRescaleLog2 || (mref == -INFINITY && mx != -INFINITY);
       float alpha = 1.f;
       if (need) {
         alpha = mref == -INFINITY ? 0.f : fast_exp2(mref - mx);
         l *= alpha;
       }
-      if (__any_sync(kFull, need && j > 0 && mref != -INFINITY)) {
-        // O holds the earlier tiles once the PV of tile j-1 has completed
-        wait(&bars.pv_done, (j - 1) & 1);
+      const bool rescale = __any_sync(kFull, need && j > 0 && mref != -INFINITY);
+      if (need) mref = mx;
+      const float mu = mref == -INFINITY ? 0.f : mref;
+      // p = 2^(s * scale - reference): one FMA and one exponential per key
+      uint32_t pk[kKeys / 2];
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < kKeys; k += 2) {
+        float p0 = fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu));
+        float p1 = fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu));
+        if (edge) {
+          p0 = k < nvis ? p0 : 0.f;
+          p1 = k + 1 < nvis ? p1 : 0.f;
+        }
+        l0 += p0;
+        l1 += p1;
+        pk[k / 2] = pack_bf16x2(p0, p1);
+      }
+      l += l0 + l1;
+      // the P buffer was read by the PV of tile j-1, and O holds the earlier tiles once that
+      // PV has completed: the rescale of O comes before this tile's PV is released
+      if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
+      if (rescale) {
         tc_fence_after_sync();
 #pragma unroll
-        for (int q4 = 0; q4 < 2; ++q4) {
+        for (int q4 = 0; q4 < D / 32; ++q4) {
           uint32_t ov[32];
           tmem_ld32(o_col + q4 * 32, ov);
           tc_wait_ld();
@@ -363,53 +372,22 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         }
         tc_wait_st();
       }
-      if (need) mref = mx;
-      const float mu = mref == -INFINITY ? 0.f : mref;
-      // p = 2^(s * scale - reference): one FMA and one exponential per key
-      uint32_t pk[32];
-      float l0 = 0.f, l1 = 0.f;
-      if (edge) {
-        const int nvis = min(64, max(0, pos - k0 + 1));
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float p0 = k < nvis ? fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu)) : 0.f;
-          const float p1 = k + 1 < nvis ? fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu)) : 0.f;
-          l0 += p0;
-          l1 += p1;
-          pk[k / 2] = pack_bf16x2(p0, p1);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu));
-          l0 += p0;
-          l1 += p1;
-          pk[k / 2] = pack_bf16x2(p0, p1);
-        }
-      }
-      l += l0 + l1;
-      // the P buffer was read by the PV of tile j-1
-      if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, hk * 8 + c)) =
+      for (int c = 0; c < kKeys / 8; ++c)
+        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, c)) =
             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full);
     }
-    // ---- epilogue: O / l once the last PV has completed; l = the two warpgroups' parts
-    xsum[hk * pfl::kRows + r] = l;
-    pfl::softmax_sync();
-    l += xsum[(hk ^ 1) * pfl::kRows + r];
+    // ---- epilogue: O / l once the last PV has completed
     wait(&bars.pv_done, (nk - 1) & 1);
     tc_fence_after_sync();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint4* dst = reinterpret_cast<uint4*>(p.out + row_off) + hk * 8;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + row_off);
 #pragma unroll
-    for (int q4 = 0; q4 < 2; ++q4) {
+    for (int q4 = 0; q4 < D / 32; ++q4) {
       uint32_t ov[32];
       tmem_ld32(o_col + q4 * 32, ov);
       tc_wait_ld();
