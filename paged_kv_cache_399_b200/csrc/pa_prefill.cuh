@@ -13,9 +13,10 @@
 //   whole tile row, so no thread waits for another's maximum; the running reference
 //   maximum moves only when a tile's maximum exceeds it by more than 2^8 (numerator and
 //   denominator share the reference, so the result is exact either way);
-//   O[128 rows][D] += P[128 rows][64 keys] . V[64 keys][D]       K-major A (P, from shared
-//                                                                memory), MN-major B (V)
-// Two CTAs share an SM (112 KB of shared memory and 256 TMEM columns each), so the softmax
+//   O[128 rows][D] += P[128 rows][64 keys] . V[64 keys][D]       A = P from TMEM (written
+//                                                                over the tile's scores),
+//                                                                MN-major B (V)
+// Two CTAs share an SM (80 KB of shared memory and 256 TMEM columns each), so the softmax
 // of one runs while the other's MMAs do, and each SM sub-partition holds a softmax warp of
 // both.
 // A CTA owns 128 rows = 128 / G consecutive chunk tokens x the G query heads of one kv head
@@ -25,10 +26,12 @@
 // Roles: warps 0-3 load Q, run the softmax and the epilogue; warp 4 issues the K boxes and
 // warp 5 the V boxes (8 TMA boxes of 2 KB per tile each); warp 6 holds the TMEM allocation
 // and one of its threads issues the MMAs (S of a tile as soon as its K has landed and an S
-// buffer is free; PV of a tile as soon as its P and V are in shared memory). A K stage is
-// released when its S completes, a V stage when its PV completes.
-// TMEM: S double buffer in columns [0, 128), O in [128, 256).
-// Shared memory: Q (32 KB), P (16 KB), 2 K stages and 2 V stages of 16 KB, barriers.
+// buffer is free, i.e. the PV of the tile two before has read its P; PV of a tile as soon as
+// its P is in TMEM and its V in shared memory). A K stage is released when its S completes,
+// a V stage when its PV completes.
+// TMEM: S double buffer in columns [0, 128) (a tile's P, bf16 pairs, over the first 32
+// columns of its S), O in [128, 256).
+// Shared memory: Q (32 KB), 2 K stages and 2 V stages of 16 KB, barriers.
 
 namespace pa {
 
@@ -52,19 +55,18 @@ constexpr uint32_t kTmemO = 2 * kKeys;            // column of O
 
 struct Smem {
   static constexpr int offQ = 0;
-  static constexpr int offP = offQ + 2 * kRowsHalfBytes;
-  static constexpr int offK = offP + kRowsHalfBytes;
+  static constexpr int offK = offQ + 2 * kRowsHalfBytes;
   static constexpr int offV = offK + kStages * kTileBytes;
   static constexpr int offBars = offV + kStages * kTileBytes;
   static constexpr int kBytes = offBars + 256;
-  static_assert(offK % 1024 == 0 && offV % 1024 == 0 && offP % 1024 == 0, "swizzled operands");
+  static_assert(offK % 1024 == 0 && offV % 1024 == 0, "swizzled operands");
   // two CTAs per SM: 228 KB of shared memory less 1 KB reserved per CTA
   static_assert(kCtasPerSm * (kBytes + 1024) <= 228 * 1024, "shared memory of two CTAs");
 };
 
 struct Bars {
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full, pv_done, q_full, drain;
+  uint64_t s_full[2], p_full[2], pv_done[2], q_full, drain;
 };
 
 // Byte offset of 16-byte chunk c (0..15) of row r in a 128-row operand of two 64-column
@@ -101,8 +103,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
   if (threadIdx.x == 0) {
     uint64_t* all = reinterpret_cast<uint64_t*>(&bars);
     for (int i = 0; i < static_cast<int>(sizeof(pfl::Bars) / 8); ++i) mbar_init(all + i, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&bars.s_free[i], pfl::kSoftmaxWarps);  // one arrival per softmax warp
-    mbar_init(&bars.p_full, pfl::kSoftmaxWarps);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars.p_full[i], pfl::kSoftmaxWarps);  // one arrival per softmax warp
     mbar_init(&bars.q_full, pfl::kSoftmaxWarps);
     fence_barrier_init();
     tma_prefetch_desc(&tmap_k);
@@ -192,7 +193,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       bool progressed = false;
       bool pv_ready = false;
       if (lane == 0)
-        pv_ready = gp < gs && mbar_test_wait(&bars.p_full, gp & 1) &&
+        pv_ready = gp < gs && mbar_test_wait(&bars.p_full[gp & 1], (gp >> 1) & 1) &&
                    mbar_test_wait(&bars.v_full[gp % kStages], (gp / kStages) & 1);
       if (__shfl_sync(kFull, pv_ready, 0)) {
         const int jj = last_blk - gp * kTileBlocks;
@@ -212,16 +213,16 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         if (lane == 0) {
           tc_fence_after_sync();
           const uint32_t vst = sm + L::offV + (gp % kStages) * pfl::kTileBytes;
-          const uint32_t pst = sm + L::offP;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
-            // A = P: keys 16kk .. 16kk+15 of each row (K-major, 128-byte swizzle, two halves)
-            const uint64_t ad = smem_desc_sw128(pst + (kk >> 2) * pfl::kRowsHalfBytes + (kk & 3) * 32, 16, 1024);
+            // A = P in TMEM: keys 16kk .. 16kk+15 of each row = columns 8kk .. 8kk+7 of the S
+            // buffer the tile's scores came from
+            const uint32_t ta = tmem + (gp & 1) * kKeys + kk * 8;
             // B = V: keys 16kk .. 16kk+15 (rows of the tile) x all D columns (MN-major)
             const uint64_t bd = smem_desc_sw128(vst + kk * 2048, pfl::kHalfBytes, 1024);
-            tc_mma_bf16(tmem + pfl::kTmemO, ad, bd, idesc_o, (gp == 0 && kk == 0) ? 0u : 1u);
+            tc_mma_bf16_ta(tmem + pfl::kTmemO, ta, bd, idesc_o, (gp == 0 && kk == 0) ? 0u : 1u);
           }
-          tc_commit(&bars.pv_done);
+          tc_commit(&bars.pv_done[gp & 1]);
           tc_commit(&bars.v_empty[gp % kStages]);
         }
         __syncwarp();
@@ -234,7 +235,7 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         if (lane == 0)
           s_ready = (gs > 0 || mbar_test_wait(&bars.q_full, 0)) &&
                     mbar_test_wait(&bars.k_full[s], (gs / kStages) & 1) &&
-                    (gs < 2 || mbar_test_wait(&bars.s_free[gs & 1], ((gs >> 1) - 1) & 1));
+                    (gs < 2 || mbar_test_wait(&bars.pv_done[gs & 1], ((gs >> 1) - 1) & 1));
         if (__shfl_sync(kFull, s_ready, 0)) {
           if (lane == 0) {
             tc_fence_after_sync();
@@ -307,9 +308,6 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       tmem_ld32(tmem + lane_off + (j & 1) * kKeys, *reinterpret_cast<uint32_t(*)[32]>(sv));
       tmem_ld32(tmem + lane_off + (j & 1) * kKeys + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
       tc_wait_ld();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
       // keys past the row's position are masked (the chunk is causal; keys past every row's
       // position are past the context or belong to later chunk tokens): only tiles that reach
       // past the row's position take the mask. The maximum is taken over the raw scores
@@ -356,10 +354,10 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         pk[k / 2] = pack_bf16x2(p0, p1);
       }
       l += l0 + l1;
-      // the P buffer was read by the PV of tile j-1, and O holds the earlier tiles once that
-      // PV has completed: the rescale of O comes before this tile's PV is released
-      if (j > 0) wait(&bars.pv_done, (j - 1) & 1);
+      // O holds the earlier tiles once the PV of tile j-1 has completed: the rescale of O
+      // comes before this tile's PV is released
       if (rescale) {
+        wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1);
         tc_fence_after_sync();
 #pragma unroll
         for (int q4 = 0; q4 < D / 32; ++q4) {
@@ -372,17 +370,16 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         }
         tc_wait_st();
       }
-#pragma unroll
-      for (int c = 0; c < kKeys / 8; ++c)
-        *reinterpret_cast<uint4*>(smem + L::offP + pfl::row_chunk_offset(r, c)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+      // P over the tile's scores in TMEM (the S buffer is taken again only by S of tile j+2,
+      // which waits for this tile's PV)
+      tmem_st32(tmem + lane_off + (j & 1) * kKeys, pk);
+      tc_wait_st();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
+      if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
     }
     // ---- epilogue: O / l once the last PV has completed
-    wait(&bars.pv_done, (nk - 1) & 1);
+    wait(&bars.pv_done[(nk - 1) & 1], ((nk - 1) >> 1) & 1);
     tc_fence_after_sync();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     uint4* dst = reinterpret_cast<uint4*>(p.out + row_off);
