@@ -37,6 +37,29 @@ namespace pa {
 
 namespace pfl {
 
+// Three-input maximum and paired f32 arithmetic (sm_100): half the instructions of the
+// softmax's maximum, scaling and row sums.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// (a.x * b + c, a.y * b + c) and (a.x + b.x, a.y + b.y) as single paired instructions
+__device__ __forceinline__ float2 fma2(float2 a, float b, float c) {
+  unsigned long long r;
+  const float2 bb = make_float2(b, b), cc = make_float2(c, c);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r)
+      : "l"(*reinterpret_cast<const unsigned long long*>(&a)), "l"(*reinterpret_cast<const unsigned long long*>(&bb)),
+        "l"(*reinterpret_cast<const unsigned long long*>(&cc)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r)
+      : "l"(*reinterpret_cast<const unsigned long long*>(&a)), "l"(*reinterpret_cast<const unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+
 constexpr int kD = 128;
 constexpr int kRows = 128;                        // query rows of a CTA: the MMA's M
 constexpr int kTileBlocks = 4;
@@ -322,7 +345,8 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
           if (k < nvis) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[k]));
       } else {
 #pragma unroll
-        for (int k = 0; k < kKeys; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sv[k]));
+        for (int k = 0; k < kKeys; k += 2)
+          m4[(k >> 1) & 3] = pfl::max3(m4[(k >> 1) & 3], __uint_as_float(sv[k]), __uint_as_float(sv[k + 1]));
       }
       const float rmx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mx = rmx == -INFINITY ? -INFINITY : rmx * cs;   // the tile's row maximum, log2 units
@@ -340,20 +364,20 @@ prefill_tcm_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
       const float mu = mref == -INFINITY ? 0.f : mref;
       // p = 2^(s * scale - reference): one FMA and one exponential per key
       uint32_t pk[kKeys / 2];
-      float l0 = 0.f, l1 = 0.f;
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
 #pragma unroll
       for (int k = 0; k < kKeys; k += 2) {
-        float p0 = fast_exp2(fmaf(__uint_as_float(sv[k]), cs, -mu));
-        float p1 = fast_exp2(fmaf(__uint_as_float(sv[k + 1]), cs, -mu));
+        const float2 x = pfl::fma2(make_float2(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), cs, -mu);
+        float p0 = fast_exp2(x.x);
+        float p1 = fast_exp2(x.y);
         if (edge) {
           p0 = k < nvis ? p0 : 0.f;
           p1 = k + 1 < nvis ? p1 : 0.f;
         }
-        l0 += p0;
-        l1 += p1;
+        if (k & 2) lb = pfl::add2(lb, make_float2(p0, p1)); else la = pfl::add2(la, make_float2(p0, p1));
         pk[k / 2] = pack_bf16x2(p0, p1);
       }
-      l += l0 + l1;
+      l += (la.x + la.y) + (lb.x + lb.y);
       // O holds the earlier tiles once the PV of tile j-1 has completed: the rescale of O
       // comes before this tile's PV is released
       if (rescale) {
