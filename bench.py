@@ -37,12 +37,12 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call (mean
     # of three calls), from one ncu capture per workload (commands in profiles/); valid only for
     # the kernel sources they were taken on
-    "llama8b": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 654_440_000},
-    "llama70b_long": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 1_352_130_000},
-    "spec_verify": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 414_870_000},
-    "prefix_sharing": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 210_040_000},
-    "sliding_window": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 273_460_000},
-    "llama8b_fp8": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 280_740_000},
+    "llama8b": {"source_hash": "4695251692d1e707", "bytes_per_launch": 654_430_000},
+    "llama70b_long": {"source_hash": "4695251692d1e707", "bytes_per_launch": 1_352_380_000},
+    "spec_verify": {"source_hash": "4695251692d1e707", "bytes_per_launch": 414_770_000},
+    "prefix_sharing": {"source_hash": "4695251692d1e707", "bytes_per_launch": 210_140_000},
+    "sliding_window": {"source_hash": "4695251692d1e707", "bytes_per_launch": 273_290_000},
+    "llama8b_fp8": {"source_hash": "4695251692d1e707", "bytes_per_launch": 281_130_000},
 }
 
 # the same for one pa_copy_blocks launch of a copy workload (keyed by COPY_SOURCES' hash;
@@ -333,8 +333,10 @@ def _ncu_traffic(name):
 def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
     """CUDA-event times of `calls` pa_decode calls (each after the step's cache write, events
     on the launching stream around the decode only): their mean and median in ms; the median
-    of the same calls made cold, with `flush` (a buffer twice the L2 size) written before each
-    step outside the events (None without `flush`); the calls without host overhead: one CUDA graph of 20
+    of the same calls made cold, with `flush` (a buffer twice the L2 size) read before each
+    step outside the events (None without `flush`): a read leaves L2 holding clean lines of
+    the buffer, where a write would leave dirty lines whose write-back the decode would pay
+    for; the calls without host overhead: one CUDA graph of 20
     back-to-back calls, replayed (µs per call, None when capture is unavailable); and the mean
     event time of the step's cache writes (ms), timed apart from the decode."""
     import torch
@@ -355,8 +357,9 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
     cold_ms = None
     if flush is not None:
         pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+        sink = torch.empty((), dtype=flush.dtype, device=flush.device)
         for a, b in pairs:
-            flush.zero_()
+            torch.amax(flush, dim=0, out=sink)
             write()
             a.record(stream)
             decode()
@@ -408,7 +411,7 @@ def measure_config(name, args, dev, stream, peaks):
         decode()
     barrier()
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(dev.index)
     with sampler:
         decode_ms, median_ms, cold_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream,
@@ -422,7 +425,7 @@ def measure_config(name, args, dev, stream, peaks):
         "calls": args.config_calls,
         "decode_us_per_call": round(decode_ms * 1e3, 3),
         "decode_us_per_call_median": round(median_ms * 1e3, 3),
-        # L2 written over (a buffer twice its size) before every step, outside the events
+        # L2 filled with another buffer (one twice its size read) before every step, outside the events
         "decode_us_per_call_cold": round(cold_ms * 1e3, 3),
         "frac_cold": round(dec_bytes / (cold_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "decode_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
@@ -447,7 +450,7 @@ def measure_config(name, args, dev, stream, peaks):
 NCU_PREFILL_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one pa_prefill launch (mean of three),
     # valid only for the kernel sources it was taken on
-    "chunked_prefill": {"source_hash": "8b47d6df4d2f0606", "bytes_per_launch": 199_280_000},
+    "chunked_prefill": {"source_hash": "4695251692d1e707", "bytes_per_launch": 141_810_000},
 }
 
 
