@@ -16,7 +16,7 @@
 //   O[128 rows][D] += P[128 rows][64 keys] . V[64 keys][D]       A = P from TMEM (written
 //                                                                over the tile's scores),
 //                                                                MN-major B (V)
-// Two CTAs share an SM (80 KB of shared memory and 256 TMEM columns each), so the softmax
+// Two CTAs share an SM (96 KB of shared memory and 256 TMEM columns each), so the softmax
 // of one runs while the other's MMAs do, and each SM sub-partition holds a softmax warp of
 // both.
 // A CTA owns 128 rows = 128 / G consecutive chunk tokens x the G query heads of one kv head
