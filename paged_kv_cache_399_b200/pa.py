@@ -162,20 +162,48 @@ def _check(status: int, where: str) -> None:
         raise PAError(status, where)
 
 
+# The per-step calls below (cache write, decode) check dtypes and layouts with as few calls
+# into torch as they can: their host time sits between a step's kernels.
+_BF16, _U8, _INT32, _INT64 = torch.bfloat16, torch.uint8, torch.int32, torch.int64
+
+
+def _require(ok: bool, what: str) -> None:
+    if not ok:
+        raise ValueError(what)
+
+
+def _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, q_per_seq, cache_dtype, where):
+    """The C arguments of pa_decode(_fp8) up to num_blocks, after the layout checks."""
+    if not (out.dtype is _BF16 and query.dtype is _BF16 and key_cache.dtype is cache_dtype and
+            value_cache.dtype is cache_dtype and block_tables.dtype is _INT32 and context_lens.dtype is _INT32):
+        raise TypeError(f"{where}: out/query bf16, caches {cache_dtype}, block_tables/context_lens int32")
+    _require(out.is_contiguous() and query.is_contiguous() and key_cache.is_contiguous() and
+             value_cache.is_contiguous() and block_tables.is_contiguous() and context_lens.is_contiguous(),
+             f"{where}: every tensor must be contiguous")
+    B, QS, HQ, D = query.shape
+    _require(QS == q_per_seq and out.shape == query.shape, f"{where}: out/query [B, q_per_seq, H_q, D]")
+    NB, BS, HKV = key_cache.shape[:3]
+    return (out.data_ptr(), query.data_ptr(), key_cache.data_ptr(), value_cache.data_ptr(),
+            block_tables.data_ptr(), context_lens.data_ptr(), B, QS, HQ, HKV, D, BS, block_tables.shape[1], NB)
+
+
 def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
                          value_cache: torch.Tensor, slot_mapping: torch.Tensor,
                          stream=None) -> None:
     """key/value [T, H_kv, D] bf16 (token stride may exceed H_kv*D); caches
     [NB, 16, H_kv, D] bf16; slot_mapping [T] int64."""
-    assert key.dtype == value.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
-    assert slot_mapping.dtype == torch.int64 and slot_mapping.is_contiguous()
+    if not (key.dtype is _BF16 and value.dtype is _BF16 and key_cache.dtype is _BF16 and
+            value_cache.dtype is _BF16 and slot_mapping.dtype is _INT64):
+        raise TypeError("pa_reshape_and_cache: key/value/caches bf16, slot_mapping int64")
     T, H, D = key.shape
-    assert key.stride(2) == 1 and key.stride(1) == D and value.stride(2) == 1 and value.stride(1) == D
-    assert key_cache.is_contiguous() and value_cache.is_contiguous()
-    NB, BS = key_cache.shape[0], key_cache.shape[1]
-    st = _lib.pa_reshape_and_cache(_ptr(key), _ptr(value), key.stride(0), value.stride(0),
-                                   _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping), T, H, D,
-                                   NB, BS, _stream(stream))
+    ks, vs = key.stride(), value.stride()
+    _require(ks[2] == 1 and ks[1] == D and vs[2] == 1 and vs[1] == D and value.shape == key.shape and
+             slot_mapping.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous(),
+             "pa_reshape_and_cache: rows of key/value contiguous, caches and slot_mapping contiguous")
+    NB, BS = key_cache.shape[:2]
+    st = _lib.pa_reshape_and_cache(key.data_ptr(), value.data_ptr(), ks[0], vs[0], key_cache.data_ptr(),
+                                   value_cache.data_ptr(), slot_mapping.data_ptr(), T, H, D, NB, BS,
+                                   _stream(stream))
     _check(st, "pa_reshape_and_cache")
 
 
@@ -202,16 +230,18 @@ def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: 
                              v_scale: float, stream=None) -> None:
     """FP8 cache write. key/value [T, H_kv, D] bf16 (token stride may exceed H_kv*D);
     caches [NB, 16, H_kv, D] uint8 (E4M3 codes); slot_mapping [T] int64; one scale per pool."""
-    assert key.dtype == value.dtype == torch.bfloat16
-    assert key_cache.dtype == value_cache.dtype == torch.uint8
-    assert slot_mapping.dtype == torch.int64 and slot_mapping.is_contiguous()
+    if not (key.dtype is _BF16 and value.dtype is _BF16 and key_cache.dtype is _U8 and
+            value_cache.dtype is _U8 and slot_mapping.dtype is _INT64):
+        raise TypeError("pa_reshape_and_cache_fp8: key/value bf16, caches uint8, slot_mapping int64")
     T, H, D = key.shape
-    assert key.stride(2) == 1 and key.stride(1) == D and value.stride(2) == 1 and value.stride(1) == D
-    assert key_cache.is_contiguous() and value_cache.is_contiguous()
-    NB, BS = key_cache.shape[0], key_cache.shape[1]
-    st = _lib.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(key_cache),
-                                       _ptr(value_cache), _ptr(slot_mapping), T, H, D, NB, BS, float(k_scale),
-                                       float(v_scale), _stream(stream))
+    ks, vs = key.stride(), value.stride()
+    _require(ks[2] == 1 and ks[1] == D and vs[2] == 1 and vs[1] == D and value.shape == key.shape and
+             slot_mapping.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous(),
+             "pa_reshape_and_cache_fp8: rows of key/value contiguous, caches and slot_mapping contiguous")
+    NB, BS = key_cache.shape[:2]
+    st = _lib.pa_reshape_and_cache_fp8(key.data_ptr(), value.data_ptr(), ks[0], vs[0], key_cache.data_ptr(),
+                                       value_cache.data_ptr(), slot_mapping.data_ptr(), T, H, D, NB, BS,
+                                       float(k_scale), float(v_scale), _stream(stream))
     _check(st, "pa_reshape_and_cache_fp8")
 
 
@@ -248,19 +278,11 @@ def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
     """out/query [B, q, H_q, D] bf16; caches [NB, 16, H_kv, D] bf16; block_tables
     [B, max_blocks] int32; context_lens [B] int32. workspace: any contiguous CUDA
     tensor of at least pa_decode_workspace_size(plan, ...) bytes (None when 0)."""
-    assert out.dtype == query.dtype == key_cache.dtype == value_cache.dtype == torch.bfloat16
-    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
-    for t in (out, query, key_cache, value_cache, block_tables, context_lens):
-        assert t.is_contiguous()
-    B, QS, HQ, D = query.shape
-    assert QS == q_per_seq and tuple(out.shape) == tuple(query.shape)
-    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = _lib.pa_decode(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-                        _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
-                        block_tables.shape[1], NB, float(scale),
-                        None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
-                        _stream(stream))
+    args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, q_per_seq, _BF16,
+                        "pa_decode")
+    st = _lib.pa_decode(*args, float(scale), None if plan is None else ctypes.byref(plan),
+                        None if workspace is None else workspace.data_ptr(),
+                        0 if workspace is None else workspace.nbytes, _stream(stream))
     _check(st, "pa_decode")
 
 
@@ -271,21 +293,76 @@ def pa_decode_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tenso
     """pa_decode over FP8 pools: caches [NB, 16, H_kv, D] uint8 (E4M3 codes, values code *
     k_scale / code * v_scale); everything else as pa_decode. plan: None or one made with
     kv_cache_dtype=PA_KV_FP8_E4M3."""
-    assert out.dtype == query.dtype == torch.bfloat16
-    assert key_cache.dtype == value_cache.dtype == torch.uint8
-    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
-    for t in (out, query, key_cache, value_cache, block_tables, context_lens):
-        assert t.is_contiguous()
-    B, QS, HQ, D = query.shape
-    assert QS == q_per_seq and tuple(out.shape) == tuple(query.shape)
-    NB, BS, HKV = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = _lib.pa_decode_fp8(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-                            _ptr(block_tables), _ptr(context_lens), B, QS, HQ, HKV, D, BS,
-                            block_tables.shape[1], NB, float(scale), float(k_scale), float(v_scale),
-                            None if plan is None else ctypes.byref(plan), _ptr(workspace), ws_bytes,
-                            _stream(stream))
+    args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, q_per_seq, _U8,
+                        "pa_decode_fp8")
+    st = _lib.pa_decode_fp8(*args, float(scale), float(k_scale), float(v_scale),
+                            None if plan is None else ctypes.byref(plan),
+                            None if workspace is None else workspace.data_ptr(),
+                            0 if workspace is None else workspace.nbytes, _stream(stream))
     _check(st, "pa_decode_fp8")
+
+
+class PreparedDecode:
+    """pa_decode (bf16 pools) or pa_decode_fp8 (uint8 pools: give k_scale and v_scale) with its
+    tensors checked and its C arguments built once; each call launches the decode on the same
+    buffers and stream. For a step loop that reuses its buffers: a call then costs the C entry
+    point alone, not the per-call checks of the tensors. The tensors must keep their storage,
+    shapes and layout while the object is used (it holds references to them)."""
+
+    def __init__(self, out, query, key_cache, value_cache, block_tables, context_lens, q_per_seq, scale,
+                 plan: pa_plan_t | None = None, workspace: torch.Tensor | None = None, stream=None,
+                 k_scale: float | None = None, v_scale: float | None = None):
+        fp8 = key_cache.dtype is _U8
+        if fp8 != (k_scale is not None and v_scale is not None):
+            raise ValueError("PreparedDecode: k_scale and v_scale go with uint8 (E4M3) pools, and only with them")
+        where = "pa_decode_fp8" if fp8 else "pa_decode"
+        args = _decode_args(out, query, key_cache, value_cache, block_tables, context_lens, q_per_seq,
+                            _U8 if fp8 else _BF16, where)
+        scales = (float(scale), float(k_scale), float(v_scale)) if fp8 else (float(scale),)
+        self._keep = (out, query, key_cache, value_cache, block_tables, context_lens, plan, workspace)
+        self._fn = _lib.pa_decode_fp8 if fp8 else _lib.pa_decode
+        self._where = where
+        self._args = args + scales + (None if plan is None else ctypes.byref(plan),
+                                      None if workspace is None else workspace.data_ptr(),
+                                      0 if workspace is None else workspace.nbytes, _stream(stream))
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != PA_OK:
+            raise PAError(st, self._where)
+
+
+class PreparedCacheWrite:
+    """pa_reshape_and_cache (bf16 pools) or pa_reshape_and_cache_fp8 (uint8 pools: give k_scale
+    and v_scale) prepared like PreparedDecode."""
+
+    def __init__(self, key, value, key_cache, value_cache, slot_mapping, stream=None,
+                 k_scale: float | None = None, v_scale: float | None = None):
+        fp8 = key_cache.dtype is _U8
+        if fp8 != (k_scale is not None and v_scale is not None):
+            raise ValueError("PreparedCacheWrite: k_scale and v_scale go with uint8 (E4M3) pools, and only with them")
+        where = "pa_reshape_and_cache_fp8" if fp8 else "pa_reshape_and_cache"
+        cdt = _U8 if fp8 else _BF16
+        if not (key.dtype is _BF16 and value.dtype is _BF16 and key_cache.dtype is cdt and
+                value_cache.dtype is cdt and slot_mapping.dtype is _INT64):
+            raise TypeError(f"{where}: key/value bf16, caches {cdt}, slot_mapping int64")
+        T, H, D = key.shape
+        ks, vs = key.stride(), value.stride()
+        _require(ks[2] == 1 and ks[1] == D and vs[2] == 1 and vs[1] == D and value.shape == key.shape and
+                 slot_mapping.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous(),
+                 f"{where}: rows of key/value contiguous, caches and slot_mapping contiguous")
+        NB, BS = key_cache.shape[:2]
+        self._keep = (key, value, key_cache, value_cache, slot_mapping)
+        self._fn = _lib.pa_reshape_and_cache_fp8 if fp8 else _lib.pa_reshape_and_cache
+        self._where = where
+        self._args = ((key.data_ptr(), value.data_ptr(), ks[0], vs[0], key_cache.data_ptr(), value_cache.data_ptr(),
+                       slot_mapping.data_ptr(), T, H, D, NB, BS) +
+                      ((float(k_scale), float(v_scale)) if fp8 else ()) + (_stream(stream),))
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != PA_OK:
+            raise PAError(st, self._where)
 
 
 def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor, value_cache: torch.Tensor,

@@ -404,3 +404,37 @@ def test_partial_decode_and_merge_reject_bad_arguments_before_launch(pa):
     assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 128, 1024) >= 1
     assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 96, 1024) == 0
     assert pa.pa_decode_partial_pieces(4, 1, 64, 8, 128, -1) == 0
+
+
+def test_prepared_calls_check_their_tensors_once_on_the_host(pa):
+    """PreparedDecode / PreparedCacheWrite build their C arguments at construction (host only,
+    stream given as a handle): wrong dtypes, layouts or scale arguments are refused there."""
+    import torch
+    B, q, HQ, HKV, D, NB, MB = 2, 1, 8, 2, 128, 8, 4
+    out = torch.zeros(B, q, HQ, D, dtype=torch.bfloat16)
+    query = torch.zeros(B, q, HQ, D, dtype=torch.bfloat16)
+    kc = torch.zeros(NB, 16, HKV, D, dtype=torch.bfloat16)
+    vc = torch.zeros_like(kc)
+    tables = torch.zeros(B, MB, dtype=torch.int32)
+    ctx = torch.ones(B, dtype=torch.int32)
+    call = pa.PreparedDecode(out, query, kc, vc, tables, ctx, q, 0.1, stream=0)
+    assert call._args[6:14] == (B, q, HQ, HKV, D, 16, MB, NB)
+    with pytest.raises(TypeError):
+        pa.PreparedDecode(out, query, kc, vc, tables.long(), ctx, q, 0.1, stream=0)
+    with pytest.raises(ValueError):
+        pa.PreparedDecode(out, query, kc, vc, tables.t().contiguous().t(), ctx, q, 0.1, stream=0)
+    with pytest.raises(ValueError):   # scales belong to E4M3 pools
+        pa.PreparedDecode(out, query, kc, vc, tables, ctx, q, 0.1, stream=0, k_scale=1.0, v_scale=1.0)
+    with pytest.raises(ValueError):   # q_per_seq disagrees with the query
+        pa.PreparedDecode(out, query, kc, vc, tables, ctx, 2, 0.1, stream=0)
+    k8 = torch.zeros(NB, 16, HKV, D, dtype=torch.uint8)
+    with pytest.raises(ValueError):   # E4M3 pools need both scales
+        pa.PreparedDecode(out, query, k8, k8.clone(), tables, ctx, q, 0.1, stream=0)
+    pa.PreparedDecode(out, query, k8, k8.clone(), tables, ctx, q, 0.1, stream=0, k_scale=0.5, v_scale=0.5)
+    key = torch.zeros(3, HKV, D, dtype=torch.bfloat16)
+    slots = torch.zeros(3, dtype=torch.int64)
+    pa.PreparedCacheWrite(key, key.clone(), kc, vc, slots, stream=0)
+    with pytest.raises(TypeError):
+        pa.PreparedCacheWrite(key, key.clone(), kc, vc, slots.int(), stream=0)
+    with pytest.raises(ValueError):
+        pa.PreparedCacheWrite(key, key.clone(), k8, k8.clone(), slots, stream=0)
