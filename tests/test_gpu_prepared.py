@@ -90,3 +90,34 @@ def test_prepared_decode_reports_the_entry_points_errors():
                              plan=plan, workspace=small)
     with pytest.raises(pa.PAError):
         call()
+
+
+@pytest.mark.parametrize("case", CASES[:2], ids=[c[0] for c in CASES[:2]])
+def test_prepared_decode_in_a_cuda_graph(case):
+    """A prepared decode made on the capture stream is captured like the per-call one; the
+    replays read the buffers' current contents."""
+    name, ctxs, q, hq, hkv, d = case
+    w = workloads.build_workload(name, 7400, ctxs, q, hq, hkv, d, scale=1.0 / math.sqrt(d))
+    dw = DeviceWorkload(w)
+    pa.pa_reshape_and_cache(dw.key, dw.value, dw.key_cache, dw.value_cache, dw.slots)
+    plan = pa.pa_decode_plan(w.num_seqs, q, hq, hkv, d, w.max_blocks_per_seq)
+    ws = _ws(plan, w)
+    ref = torch.empty_like(dw.out)
+    pa.pa_decode(ref, dw.query, dw.key_cache, dw.value_cache, dw.tables, dw.ctx, q, w.scale, plan=plan, workspace=ws)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call = pa.PreparedDecode(dw.out, dw.query, dw.key_cache, dw.value_cache, dw.tables, dw.ctx, q, w.scale,
+                                 plan=plan, workspace=ws)
+        call()
+    dw.out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error(reset=True) == 0
+    assert torch.equal(dw.out, ref)
+    dw.query.mul_(-1.0)   # new contents, same buffer
+    graph.replay()
+    pa.pa_decode(ref, dw.query, dw.key_cache, dw.value_cache, dw.tables, dw.ctx, q, w.scale, plan=plan, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(dw.out, ref)
+    del graph
