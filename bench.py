@@ -37,12 +37,12 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum over the kernels of one pa_decode call (mean
     # of three calls), from one ncu capture per workload (commands in profiles/); valid only for
     # the kernel sources they were taken on
-    "llama8b": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 654_430_000},
-    "llama70b_long": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 1_352_380_000},
-    "spec_verify": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 414_770_000},
-    "prefix_sharing": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 210_140_000},
-    "sliding_window": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 273_290_000},
-    "llama8b_fp8": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 281_130_000},
+    "llama8b": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 654_760_000},
+    "llama70b_long": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 1_352_130_000},
+    "spec_verify": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 414_730_000},
+    "prefix_sharing": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 210_150_000},
+    "sliding_window": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 273_290_000},
+    "llama8b_fp8": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 280_710_000},
 }
 
 # the same for one pa_copy_blocks launch of a copy workload (keyed by COPY_SOURCES' hash;
@@ -451,7 +451,7 @@ def measure_config(name, args, dev, stream, peaks):
 NCU_PREFILL_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one pa_prefill launch (mean of three),
     # valid only for the kernel sources it was taken on
-    "chunked_prefill": {"source_hash": "106d2a8f5aa63d78", "bytes_per_launch": 141_810_000},
+    "chunked_prefill": {"source_hash": "14d5107606101b9d", "bytes_per_launch": 142_000_000},
 }
 
 

@@ -52,7 +52,9 @@
  *     Query head h reads kv head h / (num_q_heads / num_kv_heads).
  *   - Supported: block_size 16, head_dim 64 or 128, num_q_heads % num_kv_heads == 0,
  *     1 <= q_per_seq <= 16. Anything else returns PA_ERR_UNSUPPORTED before any
- *     launch. There is no CPU fallback.
+ *     launch. A tcgen05 plan also needs num_seqs * num_kv_heads * row chunks below 2^28,
+ *     and that times (max_blocks_per_seq / 8 + 1) below 2^35 (its in-kernel range scan).
+ *     There is no CPU fallback.
  *   - Errors: host-side argument checks run before any launch and return a status
  *     with nothing enqueued. Device-resident values (slots, block ids, context
  *     lengths) are preconditions: 0 <= slot < num_blocks*block_size or slot < 0,

@@ -501,6 +501,14 @@ pa_status_t decode_impl(void* out, const void* query, const void* key_cache, con
     plan = &local;
   }
   if (st != PA_OK) return st;
+  if (plan->path == PA_PATH_TCGEN05) {
+    // the tcgen05 kernel's range scan adds (tiles, units with tiles) packed in one 64-bit word:
+    // the units must stay below 2^28 and the tiles below 2^35 (bounds over every kv head)
+    const int64_t rows = static_cast<int64_t>(num_q_heads / num_kv_heads) * q_per_seq;
+    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads * ceil_div(rows, plan->rows_per_cta);
+    const int64_t tiles = units * (max_blocks_per_seq / 8 + 1);
+    if (units >= (int64_t{1} << 28) || tiles >= (int64_t{1} << 35)) return PA_ERR_UNSUPPORTED;
+  }
   const size_t need =
       part ? 0 : workspace_bytes_for(*plan, num_seqs, q_per_seq, num_q_heads, num_kv_heads, head_dim);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;

@@ -438,3 +438,16 @@ def test_prepared_calls_check_their_tensors_once_on_the_host(pa):
         pa.PreparedCacheWrite(key, key.clone(), kc, vc, slots.int(), stream=0)
     with pytest.raises(ValueError):
         pa.PreparedCacheWrite(key, key.clone(), k8, k8.clone(), slots, stream=0)
+
+
+def test_tcgen05_decode_refuses_shapes_past_its_scan_range(pa):
+    """The tcgen05 kernel's range scan packs (tiles, units) sums in 64 bits: a decode whose
+    units (sequence x kv head x row chunk) reach 2^28, or whose tiles reach 2^35, is refused
+    on the host (PA_ERR_UNSUPPORTED) before the workspace check and before any launch."""
+    fake = 1 << 12   # aligned non-null pointers: nothing is read before the refusal
+    for B, hq, hkv, mb in [(65535, 8192, 8192, 4), (65535, 64, 64, 65536)]:
+        plan = pa.pa_decode_plan(B, 1, hq, hkv, 128, mb, path=3)
+        assert plan.path == 3
+        st = pa._lib.pa_decode(fake, fake, fake, fake, fake, fake, B, 1, hq, hkv, 128, 16, mb, 1000, 0.1,
+                               ctypes.byref(plan), None, 0, None)
+        assert st == pa.PA_ERR_UNSUPPORTED, (B, hq, hkv, mb, st)
