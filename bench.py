@@ -333,7 +333,11 @@ def _ncu_traffic(name):
 
 def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
     """CUDA-event times of `calls` pa_decode calls (each after the step's cache write, events
-    on the launching stream around the decode only): their mean and median in ms; the median
+    on the launching stream around the decode only), queued behind a sleep kernel so that the
+    host's own time per call (the binding, the C entry point) never leaves the GPU idle inside
+    an interval: their mean and median in ms, the device time of a call; the mean of the same
+    calls made one after another with nothing queued (host-paced: an interval then also holds
+    whatever the GPU waits for the host's next launch); the median
     of the same calls made cold, with `flush` (a buffer twice the L2 size) read before each
     step outside the events (None without `flush`): a read leaves L2 holding clean lines of
     the buffer, where a write would leave dirty lines whose write-back the decode would pay
@@ -343,18 +347,23 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
     import torch
     write, decode = _hot_path(pa, w, v, plan, ws, stream)
     barrier()
-    # one event between the write and the decode ends the one and starts the other
-    triples = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(calls)]
-    for c, a, b in triples:
-        c.record(stream)
-        write()
-        a.record(stream)
-        decode()
-        b.record(stream)
-    barrier()
-    times = [a.elapsed_time(b) for _, a, b in triples]
+    def per_call(queued):
+        # one event between the write and the decode ends the one and starts the other
+        triples = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(calls)]
+        if queued:   # about 5 ms of GPU time: the host enqueues every call before the GPU reaches them
+            torch.cuda._sleep(10_000_000)
+        for c, a, b in triples:
+            c.record(stream)
+            write()
+            a.record(stream)
+            decode()
+            b.record(stream)
+        barrier()
+        return [a.elapsed_time(b) for _, a, b in triples], [c.elapsed_time(a) for c, a, _ in triples]
+    times, writes = per_call(True)
     decode_ms, median_ms = statistics.mean(times), statistics.median(times)
-    write_ms = statistics.mean(c.elapsed_time(a) for c, a, _ in triples)
+    write_ms = statistics.mean(writes)
+    paced_ms = statistics.mean(per_call(False)[0])
     cold_ms = None
     if flush is not None:
         pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
@@ -387,7 +396,7 @@ def _time_calls(pa, w, v, plan, ws, stream, calls, barrier, flush=None):
         del graph
     except Exception as exc:  # capture is a measurement aid: report why it is missing
         print(f"graph timing unavailable: {exc}", file=sys.stderr)
-    return decode_ms, median_ms, cold_ms, graph_us, write_ms
+    return decode_ms, median_ms, cold_ms, graph_us, write_ms, paced_ms
 
 
 def measure_config(name, args, dev, stream, peaks):
@@ -415,8 +424,8 @@ def measure_config(name, args, dev, stream, peaks):
     flush = torch.zeros(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(dev.index)
     with sampler:
-        decode_ms, median_ms, cold_ms, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream,
-                                                                        args.config_calls, barrier, flush)
+        decode_ms, median_ms, cold_ms, graph_us, write_ms, paced_ms = _time_calls(
+            pa, w, v, plan, ws, stream, args.config_calls, barrier, flush)
     assert pa.pa_get_device_error(reset=True, stream=stream) == 0
     del flush
     dec_bytes = decode_bytes(w)
@@ -426,6 +435,8 @@ def measure_config(name, args, dev, stream, peaks):
         "calls": args.config_calls,
         "decode_us_per_call": round(decode_ms * 1e3, 3),
         "decode_us_per_call_median": round(median_ms * 1e3, 3),
+        # the same calls made one after another with nothing queued ahead of them
+        "decode_us_per_call_host_paced": round(paced_ms * 1e3, 3),
         # L2 filled with another buffer (one twice its size read) before every step, outside the events
         "decode_us_per_call_cold": round(cold_ms * 1e3, 3),
         "frac_cold": round(dec_bytes / (cold_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -753,8 +764,10 @@ def run_gpu(args):
         # (2) per-kernel: events around each pa_decode launch of another K steps, and the
         # same calls graph-replayed (for the small configs the events mostly time the
         # Python call)
-        decode_ms, _, _, graph_us, write_ms = _time_calls(pa, w, v, plan, ws, stream, args.steps, barrier)
+        decode_ms, _, _, graph_us, write_ms, paced_ms = _time_calls(pa, w, v, plan, ws, stream, args.steps,
+                                                                   barrier)
         decode_ms = max_over_ranks(decode_ms)
+        paced_ms = max_over_ranks(paced_ms)
         if graph_us is not None:
             graph_us = max_over_ranks(graph_us)
 
@@ -849,6 +862,7 @@ def run_gpu(args):
                 "decode_alg_bytes": dec_bytes,
                 "decode_logical_bytes": decode_bytes(w, unique=False),
                 "decode_us_per_call": round(decode_ms * 1e3, 3),
+                "decode_us_per_call_host_paced": round(paced_ms * 1e3, 3),
                 "decode_us_per_call_graph": None if graph_us is None else round(graph_us, 3),
                 "cache_write_us_per_call": round(write_ms * 1e3, 3),
                 "decode_gbs": round(achieved, 2),
